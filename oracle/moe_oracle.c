@@ -1,0 +1,412 @@
+/*
+ * moe_oracle.c -- plain, slow, fp64 CPU oracle of the forward pass of a
+ * top-k routed Mixture-of-Experts SwiGLU FFN layer.
+ *
+ * TEST INFRASTRUCTURE. Only the test suite, the package smoke check and the
+ * benchmark's CPU-baseline leg load this library. The product (the CUDA
+ * library and its Python binding) never calls it, shares no code, header,
+ * table or helper with it, and must fail loudly rather than fall back here.
+ *
+ * What it follows (web pages that define the layer):
+ *  [MIX] "MoE Model Architectures" (architectures.md), section "Mixtral 8x7B",
+ *        subsections "Sparse MoE Block" (gate -> softmax over all experts ->
+ *        top-k -> divide by the top-k sum -> per-expert FFN on the routed rows
+ *        -> scale by the routing weight -> index_add into token order) and
+ *        "Expert FFN" (w2(silu(w1 x) * w3 x), no biases).
+ *  [DSK] same page, section "DeepSeek-V3": "DeepSeekMoE Architecture" (shared
+ *        experts always run and are added unweighted) and "Auxiliary-Loss-Free
+ *        Load Balancing" (F.linear(x, W, b): a per-expert bias on the logits).
+ *  [SWT] same page, section "Switch Transformers", "Top-1 Routing" (an expert
+ *        capacity beyond which routed tokens are dropped; the printed mask is
+ *        garbled: it compares per-expert totals, not per-token ranks).
+ *  [CUR] "Current Bug: CuTeDSLMoERunner produces wrong output", sections "How
+ *        the pipeline works" / "How the runner currently works": token counts
+ *        [4,4,0] give expert offsets [4,8,8], or [0,4,8,8] with a leading 0.
+ *  [MGA] "Faster writing: run only the chosen experts; uncap the large profile"
+ *        (a capacity factor of 0 means uncapped).
+ *
+ * Readings taken where the pages are silent or garbled (also listed in the
+ * design notes of the repository):
+ *  R1  top-k is chosen on the fp32 logits. Softmax is strictly increasing in
+ *      the logit, so this is the top-k of [MIX]'s probabilities wherever those
+ *      are not rounded to equal values. Ties go to the lowest expert index;
+ *      -0.0 and +0.0 compare equal. Output order is selection order.
+ *  R2  the weights are [MIX]'s softmax over all E, restricted to the top-k
+ *      and divided by their sum (computed literally, in fp64).
+ *  R3  capacity C: an assignment (t, j) is kept iff fewer than C assignments
+ *      to the same expert come before it in row-major (token, slot) order;
+ *      C <= 0 is uncapped ([MGA]). Kept weights are not renormalised; a
+ *      dropped assignment contributes nothing.
+ *  R4  expert offsets have E+1 entries with a leading 0 ([CUR]'s GPU form);
+ *      an expert's kept rows are laid out in ascending token order.
+ *  R5  the bias enters both the selection and the weights ([DSK]'s
+ *      F.linear(x, W, b) feeds the softmax); a shared expert is added with
+ *      weight 1.
+ *  R6  the SwiGLU product h is optionally rounded to bf16 (round to nearest,
+ *      ties to even) before w2, modelling the one rounding a bf16 tensor-core
+ *      path must make; with h_bf16 = 0 the whole layer is pure fp64.
+ *
+ * Inputs are bf16 bit patterns (uint16) and are widened exactly to double.
+ * Error codes: 0 ok, 1 invalid argument, 5 non-finite logit, 6 bad expert id.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define ORC_OK 0
+#define ORC_EINVAL 1
+#define ORC_ENONFINITE 5
+#define ORC_EBADEXPERT 6
+
+/* bf16 is the upper half of an IEEE binary32; widening is exact. */
+static double bf16_to_double(uint16_t b)
+{
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/* Round a double to the nearest bf16 value (8 significant bits, binary32
+ * exponent range), ties to even, returned as a double. */
+double oracle_round_bf16(double v)
+{
+    if (!isfinite(v) || v == 0.0)
+        return v;
+    int e;
+    (void)frexp(v, &e);           /* v = m * 2^e, 0.5 <= |m| < 1 */
+    int q = e - 8;                /* weight of the last kept bit */
+    if (q < -133)                 /* bf16 subnormals: spacing 2^-133 */
+        q = -133;
+    double r = nearbyint(ldexp(v, -q));   /* default mode: ties to even */
+    double out = ldexp(r, q);
+    if (fabs(out) > 3.3895313892515355e38)  /* past the largest finite bf16 */
+        out = copysign(INFINITY, v);
+    return out;
+}
+
+/* Widen a bf16 array to double (helper for callers that want the values). */
+void oracle_bf16_to_f64(int64_t n, const uint16_t *src, double *dst)
+{
+    for (int64_t i = 0; i < n; ++i)
+        dst[i] = bf16_to_double(src[i]);
+}
+
+/* [MIX] "Sparse MoE Block": router_logits = gate(x), gate = Linear(d, E)
+ * stored [E, d]; [DSK] adds the bias b[E]. Exact products, fp64 sums.
+ * L64 [T,E] (may be NULL) receives the fp64 logits, L32 [T,E] (may be NULL)
+ * the same values rounded once to fp32. */
+int oracle_router_logits(int T, int d, int E, const uint16_t *x,
+                         const uint16_t *wg, const float *bias,
+                         double *L64, float *L32)
+{
+    if (T < 0 || d < 1 || E < 1 || !x || !wg)
+        return ORC_EINVAL;
+#pragma omp parallel for schedule(static)
+    for (int t = 0; t < T; ++t) {
+        for (int e = 0; e < E; ++e) {
+            double s = 0.0;
+            for (int i = 0; i < d; ++i)
+                s += bf16_to_double(x[(int64_t)t * d + i]) *
+                     bf16_to_double(wg[(int64_t)e * d + i]);
+            if (bias)
+                s += (double)bias[e];
+            if (L64)
+                L64[(int64_t)t * E + e] = s;
+            if (L32)
+                L32[(int64_t)t * E + e] = (float)s;
+        }
+    }
+    return ORC_OK;
+}
+
+/* [MIX] "Sparse MoE Block": softmax over all E, top-k, divide by the top-k
+ * sum; readings R1 and R2. L [T,E] fp32 -> idx [T,k] (selection order),
+ * w [T,k] fp64. A row holding a NaN, or whose maximum is not finite,
+ * returns ORC_ENONFINITE. */
+int oracle_route(int T, int E, int k, const float *L, int32_t *idx, double *w)
+{
+    if (T < 0 || E < 1 || k < 1 || k > E || !L || !idx || !w)
+        return ORC_EINVAL;
+    int rc = ORC_OK;
+    double *p = (double *)malloc(sizeof(double) * (size_t)E);
+    char *chosen = (char *)malloc((size_t)E);
+    if (!p || !chosen) {
+        free(p);
+        free(chosen);
+        return ORC_EINVAL;
+    }
+    for (int t = 0; t < T && rc == ORC_OK; ++t) {
+        const float *l = L + (int64_t)t * E;
+        /* softmax over all E, in fp64 */
+        double M = -INFINITY;
+        for (int e = 0; e < E; ++e) {
+            if (isnan(l[e]))
+                rc = ORC_ENONFINITE;
+            if ((double)l[e] > M)
+                M = (double)l[e];
+        }
+        if (rc != ORC_OK || !isfinite(M)) {
+            rc = ORC_ENONFINITE;
+            break;
+        }
+        double S = 0.0;
+        for (int e = 0; e < E; ++e) {
+            p[e] = exp((double)l[e] - M);
+            S += p[e];
+        }
+        for (int e = 0; e < E; ++e)
+            p[e] /= S;
+        /* top-k: k rounds of "largest logit not yet taken", lowest index on ties */
+        memset(chosen, 0, (size_t)E);
+        for (int j = 0; j < k; ++j) {
+            int best = -1;
+            for (int e = 0; e < E; ++e) {
+                if (chosen[e])
+                    continue;
+                if (best < 0 || l[e] > l[best])
+                    best = e;
+            }
+            chosen[best] = 1;
+            idx[(int64_t)t * k + j] = best;
+        }
+        /* renormalise over the chosen k */
+        double s = 0.0;
+        for (int j = 0; j < k; ++j)
+            s += p[idx[(int64_t)t * k + j]];
+        for (int j = 0; j < k; ++j)
+            w[(int64_t)t * k + j] = p[idx[(int64_t)t * k + j]] / s;
+    }
+    free(p);
+    free(chosen);
+    return rc;
+}
+
+/* Expert histogram, capacity, offsets and permutation: [CUR]'s counts and
+ * offsets, [MIX]'s torch.where(selected_experts == e) row-major order, and
+ * readings R3/R4.
+ *   counts[E]       routed assignments per expert (before capacity)
+ *   offsets[E+1]    exclusive scan of the kept counts min(counts, C)
+ *   slot_pos[T*k]   permuted row of (t, j), or -1 if dropped
+ *   perm_token[T*k] token of each permuted row; rows >= n_kept are -1
+ *   n_kept[1]       offsets[E]
+ * Ids must lie in [0, E) and be distinct within a token (ORC_EBADEXPERT). */
+int oracle_dispatch(int T, int E, int k, int C, const int32_t *idx,
+                    int32_t *counts, int32_t *offsets, int32_t *slot_pos,
+                    int32_t *perm_token, int32_t *n_kept)
+{
+    if (T < 0 || E < 1 || k < 1 || k > E || !idx || !counts || !offsets ||
+        !slot_pos || !perm_token || !n_kept)
+        return ORC_EINVAL;
+    const int64_t N = (int64_t)T * k;
+    int32_t *rank = (int32_t *)malloc(sizeof(int32_t) * (size_t)(N > 0 ? N : 1));
+    if (!rank)
+        return ORC_EINVAL;
+    for (int e = 0; e < E; ++e)
+        counts[e] = 0;
+    /* pass 1: each assignment's rank among earlier assignments to its expert */
+    for (int t = 0; t < T; ++t) {
+        for (int j = 0; j < k; ++j) {
+            int32_t e = idx[(int64_t)t * k + j];
+            if (e < 0 || e >= E) {
+                free(rank);
+                return ORC_EBADEXPERT;
+            }
+            for (int jj = 0; jj < j; ++jj)
+                if (idx[(int64_t)t * k + jj] == e) {
+                    free(rank);
+                    return ORC_EBADEXPERT;
+                }
+            rank[(int64_t)t * k + j] = counts[e];
+            counts[e] += 1;
+        }
+    }
+    /* offsets: exclusive scan of kept counts */
+    offsets[0] = 0;
+    for (int e = 0; e < E; ++e) {
+        int32_t kept = counts[e];
+        if (C > 0 && kept > C)
+            kept = C;
+        offsets[e + 1] = offsets[e] + kept;
+    }
+    *n_kept = offsets[E];
+    /* pass 2: positions and the inverse map */
+    for (int64_t r = 0; r < N; ++r)
+        perm_token[r] = -1;
+    for (int t = 0; t < T; ++t) {
+        for (int j = 0; j < k; ++j) {
+            int64_t a = (int64_t)t * k + j;
+            int32_t e = idx[a];
+            int keep = (C <= 0) || (rank[a] < C);
+            if (keep) {
+                slot_pos[a] = offsets[e] + rank[a];
+                perm_token[slot_pos[a]] = t;
+            } else {
+                slot_pos[a] = -1;
+            }
+        }
+    }
+    free(rank);
+    return ORC_OK;
+}
+
+/* [MIX] "Expert FFN": y = w2(silu(w1 x) * w3 x); w1, w3 are [d_ff, d],
+ * w2 is [d, d_ff] (nn.Linear [out, in]); reading R6 for h. */
+static void swiglu_ffn(int d, int d_ff, const double *xv, const uint16_t *w1,
+                       const uint16_t *w3, const uint16_t *w2, int h_bf16,
+                       double *h, double *y)
+{
+    for (int c = 0; c < d_ff; ++c) {
+        double g = 0.0, u = 0.0;
+        const uint16_t *r1 = w1 + (int64_t)c * d;
+        const uint16_t *r3 = w3 + (int64_t)c * d;
+        for (int i = 0; i < d; ++i) {
+            g += bf16_to_double(r1[i]) * xv[i];
+            u += bf16_to_double(r3[i]) * xv[i];
+        }
+        double hv = g / (1.0 + exp(-g)) * u;   /* silu(g) = g * sigmoid(g) */
+        h[c] = h_bf16 ? oracle_round_bf16(hv) : hv;
+    }
+    for (int r = 0; r < d; ++r) {
+        double s = 0.0;
+        const uint16_t *r2 = w2 + (int64_t)r * d_ff;
+        for (int c = 0; c < d_ff; ++c)
+            s += bf16_to_double(r2[c]) * h[c];
+        y[r] = s;
+    }
+}
+
+/* The layer output for a list of tokens, given the routing:
+ * out[s, :] = sum over kept (t, j), in ascending expert order as [MIX]'s
+ * expert loop visits them, of w[t, j] * FFN_{idx[t, j]}(x_t), plus the
+ * shared expert FFN_s(x_t) ([DSK], reading R5) when d_ff_s > 0.
+ * x [T,d]; W1, W3 [E,d_ff,d]; W2 [E,d,d_ff]; W1s, W3s [d_ff_s,d];
+ * W2s [d,d_ff_s]; idx, slot_pos [T,k]; w [T,k] fp64;
+ * tokens [n_tok] (each in [0,T)); out [n_tok, d] fp64. */
+int oracle_moe_tokens(int T, int d, int d_ff, int E, int k, int d_ff_s,
+                      const uint16_t *x, const uint16_t *W1, const uint16_t *W3,
+                      const uint16_t *W2, const uint16_t *W1s,
+                      const uint16_t *W3s, const uint16_t *W2s,
+                      const int32_t *idx, const double *w,
+                      const int32_t *slot_pos, int h_bf16, int n_tok,
+                      const int32_t *tokens, double *out)
+{
+    if (T < 0 || d < 1 || d_ff < 1 || E < 1 || k < 1 || k > E || d_ff_s < 0 ||
+        n_tok < 0 || !x || !W1 || !W3 || !W2 || !idx || !w || !slot_pos ||
+        (n_tok > 0 && (!tokens || !out)))
+        return ORC_EINVAL;
+    if (d_ff_s > 0 && (!W1s || !W3s || !W2s))
+        return ORC_EINVAL;
+    for (int s = 0; s < n_tok; ++s)
+        if (tokens[s] < 0 || tokens[s] >= T)
+            return ORC_EINVAL;
+    for (int s = 0; s < n_tok; ++s)
+        for (int j = 0; j < k; ++j) {
+            int32_t e = idx[(int64_t)tokens[s] * k + j];
+            if (e < 0 || e >= E)
+                return ORC_EBADEXPERT;
+        }
+    const int hmax = d_ff > d_ff_s ? d_ff : d_ff_s;
+    int rc = ORC_OK;
+#pragma omp parallel
+    {
+        double *xv = (double *)malloc(sizeof(double) * (size_t)d);
+        double *h = (double *)malloc(sizeof(double) * (size_t)hmax);
+        double *y = (double *)malloc(sizeof(double) * (size_t)d);
+        if (!xv || !h || !y) {
+#pragma omp atomic write
+            rc = ORC_EINVAL;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (int s = 0; s < n_tok; ++s) {
+                const int t = tokens[s];
+                double *o = out + (int64_t)s * d;
+                for (int i = 0; i < d; ++i) {
+                    xv[i] = bf16_to_double(x[(int64_t)t * d + i]);
+                    o[i] = 0.0;
+                }
+                /* routed experts, visited in ascending expert index */
+                for (int e = 0; e < E; ++e) {
+                    for (int j = 0; j < k; ++j) {
+                        int64_t a = (int64_t)t * k + j;
+                        if (idx[a] != e || slot_pos[a] < 0)
+                            continue;
+                        swiglu_ffn(d, d_ff, xv, W1 + (int64_t)e * d_ff * d,
+                                   W3 + (int64_t)e * d_ff * d,
+                                   W2 + (int64_t)e * d * d_ff, h_bf16, h, y);
+                        for (int i = 0; i < d; ++i)
+                            o[i] += w[a] * y[i];
+                    }
+                }
+                /* shared expert, weight 1: shared_output + routed_output */
+                if (d_ff_s > 0) {
+                    swiglu_ffn(d, d_ff_s, xv, W1s, W3s, W2s, h_bf16, h, y);
+                    for (int i = 0; i < d; ++i)
+                        o[i] = y[i] + o[i];
+                }
+            }
+        }
+        free(xv);
+        free(h);
+        free(y);
+    }
+    return rc;
+}
+
+/* The expert FFN alone for a list of (token, expert) pairs, unweighted:
+ * y[s, :] = FFN_{experts[s]}(x_{tokens[s]}). Used to check per-row expert
+ * outputs (the permuted y of the unfused path). */
+int oracle_expert_rows(int T, int d, int d_ff, int E, const uint16_t *x,
+                       const uint16_t *W1, const uint16_t *W3,
+                       const uint16_t *W2, int h_bf16, int n,
+                       const int32_t *tokens, const int32_t *experts,
+                       double *y_out)
+{
+    if (T < 0 || d < 1 || d_ff < 1 || E < 1 || n < 0 || !x || !W1 || !W3 ||
+        !W2 || (n > 0 && (!tokens || !experts || !y_out)))
+        return ORC_EINVAL;
+    for (int s = 0; s < n; ++s) {
+        if (tokens[s] < 0 || tokens[s] >= T)
+            return ORC_EINVAL;
+        if (experts[s] < 0 || experts[s] >= E)
+            return ORC_EBADEXPERT;
+    }
+    int rc = ORC_OK;
+#pragma omp parallel
+    {
+        double *xv = (double *)malloc(sizeof(double) * (size_t)d);
+        double *h = (double *)malloc(sizeof(double) * (size_t)d_ff);
+        if (!xv || !h) {
+#pragma omp atomic write
+            rc = ORC_EINVAL;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (int s = 0; s < n; ++s) {
+                const int t = tokens[s], e = experts[s];
+                for (int i = 0; i < d; ++i)
+                    xv[i] = bf16_to_double(x[(int64_t)t * d + i]);
+                swiglu_ffn(d, d_ff, xv, W1 + (int64_t)e * d_ff * d,
+                           W3 + (int64_t)e * d_ff * d,
+                           W2 + (int64_t)e * d * d_ff, h_bf16, h,
+                           y_out + (int64_t)s * d);
+            }
+        }
+        free(xv);
+        free(h);
+    }
+    return rc;
+}
+
+/* Number of OpenMP threads a parallel region of this library uses. */
+int oracle_num_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}

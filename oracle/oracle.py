@@ -1,0 +1,181 @@
+"""Python face of the fp64 CPU oracle (``moe_oracle.c``).
+
+TEST INFRASTRUCTURE. Only ``tests/``, the package smoke check and the
+benchmark's CPU-baseline leg may import this module. It marshals numpy arrays
+into the C oracle and back; it holds no arithmetic of the layer itself.
+
+bf16 tensors are passed as their uint16 bit patterns.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "moe_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+OK, EINVAL, ENONFINITE, EBADEXPERT = 0, 1, 5, 6
+
+
+class OracleError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        super().__init__(f"oracle {fn} returned {code}")
+        self.code = code
+
+
+def build(force: bool = False) -> str:
+    """Compile liboracle.so next to its source (plain gcc, OpenMP, IEEE math)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-fopenmp", "-shared", "-fPIC", "-Wall",
+                               "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        build()
+        L = ctypes.CDLL(_LIB)
+        P = ctypes.c_void_p
+        i = ctypes.c_int
+        L.oracle_round_bf16.argtypes = [ctypes.c_double]
+        L.oracle_round_bf16.restype = ctypes.c_double
+        L.oracle_router_logits.argtypes = [i, i, i, P, P, P, P, P]
+        L.oracle_route.argtypes = [i, i, i, P, P, P]
+        L.oracle_dispatch.argtypes = [i, i, i, i, P, P, P, P, P, P]
+        L.oracle_moe_tokens.argtypes = [i, i, i, i, i, i, P, P, P, P, P, P, P, P, P, P,
+                                        i, i, P, P]
+        L.oracle_expert_rows.argtypes = [i, i, i, i, P, P, P, P, i, i, P, P, P]
+        L.oracle_num_threads.argtypes = []
+        for f in (L.oracle_router_logits, L.oracle_route, L.oracle_dispatch,
+                  L.oracle_moe_tokens, L.oracle_expert_rows, L.oracle_num_threads):
+            f.restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def _p(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _u16(a):
+    a = np.ascontiguousarray(a)
+    assert a.dtype == np.uint16, a.dtype
+    return a
+
+
+def _check(fn, rc):
+    if rc != OK:
+        raise OracleError(fn, rc)
+
+
+def num_threads() -> int:
+    return lib().oracle_num_threads()
+
+
+def round_bf16(v: float) -> float:
+    return lib().oracle_round_bf16(float(v))
+
+
+def router_logits(x, wg, bias=None):
+    """x [T,d] u16, wg [E,d] u16, bias [E] f32|None -> (L64 [T,E] f64, L32 [T,E] f32)."""
+    x, wg = _u16(x), _u16(wg)
+    T, d = x.shape
+    E = wg.shape[0]
+    L64 = np.empty((T, E), np.float64)
+    L32 = np.empty((T, E), np.float32)
+    b = None if bias is None else np.ascontiguousarray(bias, np.float32)
+    _check("router_logits", lib().oracle_router_logits(T, d, E, _p(x), _p(wg), _p(b), _p(L64), _p(L32)))
+    return L64, L32
+
+
+def route(L32, k):
+    """L32 [T,E] f32 -> (idx [T,k] i32, w [T,k] f64)."""
+    L = np.ascontiguousarray(L32, np.float32)
+    T, E = L.shape
+    idx = np.empty((T, k), np.int32)
+    w = np.empty((T, k), np.float64)
+    _check("route", lib().oracle_route(T, E, k, _p(L), _p(idx), _p(w)))
+    return idx, w
+
+
+def dispatch(idx, E, C=0):
+    """idx [T,k] -> dict(counts [E], offsets [E+1], slot_pos [T,k], perm_token [T*k], n_kept)."""
+    idx = np.ascontiguousarray(idx, np.int32)
+    T, k = idx.shape
+    counts = np.empty(E, np.int32)
+    offsets = np.empty(E + 1, np.int32)
+    slot_pos = np.empty((T, k), np.int32)
+    perm_token = np.empty(max(T * k, 1), np.int32)
+    n_kept = np.zeros(1, np.int32)
+    _check("dispatch", lib().oracle_dispatch(T, E, k, int(C), _p(idx), _p(counts), _p(offsets),
+                                             _p(slot_pos), _p(perm_token), _p(n_kept)))
+    return dict(counts=counts, offsets=offsets, slot_pos=slot_pos,
+                perm_token=perm_token[: T * k], n_kept=int(n_kept[0]))
+
+
+def moe_tokens(x, W1, W3, W2, idx, w, slot_pos, tokens, h_bf16=True, W1s=None, W3s=None, W2s=None):
+    """Layer output rows (fp64) for the listed tokens, given the routing."""
+    x, W1, W3, W2 = _u16(x), _u16(W1), _u16(W3), _u16(W2)
+    T, d = x.shape
+    E, d_ff, _ = W1.shape
+    k = idx.shape[1]
+    d_ff_s = 0
+    if W1s is not None:
+        W1s, W3s, W2s = _u16(W1s), _u16(W3s), _u16(W2s)
+        d_ff_s = W1s.shape[0]
+    idx = np.ascontiguousarray(idx, np.int32)
+    w = np.ascontiguousarray(w, np.float64)
+    slot_pos = np.ascontiguousarray(slot_pos, np.int32)
+    tokens = np.ascontiguousarray(tokens, np.int32)
+    out = np.empty((len(tokens), d), np.float64)
+    _check("moe_tokens", lib().oracle_moe_tokens(
+        T, d, d_ff, E, k, d_ff_s, _p(x), _p(W1), _p(W3), _p(W2), _p(W1s), _p(W3s), _p(W2s),
+        _p(idx), _p(w), _p(slot_pos), int(bool(h_bf16)), len(tokens), _p(tokens), _p(out)))
+    return out
+
+
+def expert_rows(x, W1, W3, W2, tokens, experts, h_bf16=True):
+    """Unweighted expert outputs y[s] = FFN_{experts[s]}(x[tokens[s]]) in fp64."""
+    x, W1, W3, W2 = _u16(x), _u16(W1), _u16(W3), _u16(W2)
+    T, d = x.shape
+    E, d_ff, _ = W1.shape
+    tokens = np.ascontiguousarray(tokens, np.int32)
+    experts = np.ascontiguousarray(experts, np.int32)
+    y = np.empty((len(tokens), d), np.float64)
+    _check("expert_rows", lib().oracle_expert_rows(T, d, d_ff, E, _p(x), _p(W1), _p(W3), _p(W2),
+                                                   int(bool(h_bf16)), len(tokens), _p(tokens),
+                                                   _p(experts), _p(y)))
+    return y
+
+
+def forward(inp: dict, tokens=None, logits=None, h_bf16=True):
+    """Whole layer: logits (or the given fp32 logits), routing over all T tokens,
+    dispatch with the capacity, then outputs for ``tokens`` (default: all).
+
+    ``inp`` holds numpy arrays: x, wg, bias (or None), W1, W3, W2, optional
+    W1s/W3s/W2s, and ints k, capacity.
+    """
+    T = inp["x"].shape[0]
+    E = inp["wg"].shape[0]
+    L64 = None
+    if logits is None:
+        L64, L32 = router_logits(inp["x"], inp["wg"], inp.get("bias"))
+    else:
+        L32 = np.ascontiguousarray(logits, np.float32)
+    idx, w = route(L32, inp["k"])
+    disp = dispatch(idx, E, inp.get("capacity", 0))
+    if tokens is None:
+        tokens = np.arange(T, dtype=np.int32)
+    out = moe_tokens(inp["x"], inp["W1"], inp["W3"], inp["W2"], idx, w, disp["slot_pos"], tokens,
+                     h_bf16=h_bf16, W1s=inp.get("W1s"), W3s=inp.get("W3s"), W2s=inp.get("W2s"))
+    return dict(L64=L64, L32=L32, idx=idx, w=w, out=out, tokens=np.asarray(tokens, np.int32), **disp)
