@@ -1,0 +1,400 @@
+#!/usr/bin/env python
+"""Benchmark of the MoE-layer forward (top-k routed SwiGLU experts) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload prefill|...]
+    python bench.py --impl reference ...     # the fp64 CPU oracle, timed on host cores
+
+One step = one full forward of the layer (router GEMM -> softmax/top-k ->
+histogram/offsets -> permutation -> grouped w1/w3 GEMM + SwiGLU -> grouped w2
+GEMM + weighted combine) on one batch of seeded synthetic input already
+resident in HBM. Rank 0 prints ONE JSON line. With N > 1 (torchrun), every
+rank runs an independent replica of the same workload on its own GPU (the
+layer has no cross-GPU exchange in this configuration): value = tokens of all
+ranks / max-over-ranks device time ("weak" scaling).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+import torch.distributed as dist
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from sparse_mixture_experts_17_b200 import inputs as I  # noqa: E402
+
+METRIC = "MoE-layer tokens/s + active TFLOP/s (prefill), HBM GB/s (decode) vs roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ---------------------------------------------------------------- distributed plumbing
+
+def dist_setup(use_cuda: bool):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend="nccl" if use_cuda else "gloo",
+                                timeout=datetime.timedelta(seconds=180))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x: float, world: int, device) -> float:
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons while running."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.p = None
+
+    def __enter__(self):
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                                       "-lms", "200", "-i", str(self.gpu)],
+                                      stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.p = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        self.rows = []
+        if self.p is None:
+            return False
+        time.sleep(0.3)
+        self.p.terminate()
+        try:
+            out, _ = self.p.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.p.kill()
+            out, _ = self.p.communicate()
+        for line in out.splitlines():
+            f = [c.strip() for c in line.split(",")]
+            if len(f) >= 9:
+                self.rows.append(f)
+        return False
+
+    def summary(self):
+        rows = getattr(self, "rows", [])
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+
+        def num(v):
+            try:
+                return float(v)
+            except ValueError:
+                return None
+        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+        mx = [num(r[2]) for r in rows if num(r[2]) is not None]
+        pw = [num(r[3]) for r in rows if num(r[3]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        loaded = [s for s, p in zip(sm, pw) if p is not None and p > 200] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "power_w_max": max(pw) if pw else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---------------------------------------------------------------- work accounting
+
+def routed_kept(idx: torch.Tensor, E: int, capacity: int) -> int:
+    counts = torch.bincount(idx.flatten().long(), minlength=E)
+    if capacity > 0:
+        counts = counts.clamp(max=capacity)
+    return int(counts.sum().item())
+
+
+def prefill_flops(w, n_kept):
+    ffn = 2.0 * n_kept * 3 * w.d * w.d_ff
+    router = 2.0 * w.T * w.d * w.E
+    shared = 2.0 * w.T * 3 * w.d * w.d_ff_shared
+    return ffn + router + shared, 2.0 * n_kept * w.d * 2 * w.d_ff, 2.0 * n_kept * w.d * w.d_ff
+
+
+def decode_bytes(w, T, idx):
+    U = int(torch.unique(idx.flatten()).numel())
+    expert = U * 3 * w.d * w.d_ff * 2
+    w13 = U * 2 * w.d * w.d_ff * 2
+    other = w.E * w.d * 2 + T * w.d * 2 + T * w.d * 4 + 3 * w.d * w.d_ff_shared * 2
+    return U, expert + other, w13, expert
+
+
+# ---------------------------------------------------------------- CPU baseline (the oracle)
+
+def cpu_oracle_timing(w, budget_s=15.0, steps=1, warmup=0):
+    """The fp64 oracle, as it stands, on a bounded token sample of workload `w`:
+    router logits, top-k, histogram/offsets/capacity and the expert FFN with the
+    combine, for n sample tokens. Returns (tokens/s, cores, sample text)."""
+    from oracle import oracle as O
+    threads = O.num_threads()
+    gen_dev = "cuda" if torch.cuda.is_available() else "cpu"
+    inp = I.make_inputs(w, gen_dev, seed=0)
+    oi = I.oracle_arrays(inp)
+    del inp
+
+    def run(n):
+        sub = dict(oi)
+        sub["x"] = oi["x"][:n]
+        t0 = time.perf_counter()
+        O.forward(sub)
+        return time.perf_counter() - t0
+
+    n = max(1, min(w.T, threads))
+    t = run(n)
+    while t < budget_s / 4 and n < w.T:
+        n = min(w.T, int(n * max(2.0, budget_s / max(t, 1e-3) / 2)))
+        t = run(n)
+    times = [t]
+    for _ in range(max(0, steps - 1)):
+        times.append(run(n))
+    rate = n / statistics.median(times)
+    sample = (f"first {n} of {w.T} tokens; router, top-k, offsets (capacity over the sample) and "
+              f"expert FFN + combine in fp64 on {threads} OpenMP threads; median of {len(times)}")
+    return rate, threads, sample, n
+
+
+# ---------------------------------------------------------------- our arm
+
+def time_loop(fn, steps, stream):
+    s = torch.cuda.Event(enable_timing=True)
+    e = torch.cuda.Event(enable_timing=True)
+    s.record(stream)
+    for _ in range(steps):
+        fn()
+    e.record(stream)
+    e.synchronize()
+    return s.elapsed_time(e) / steps
+
+
+def run_ours(a, world, rank, local):
+    from sparse_mixture_experts_17_b200 import build as B
+    from sparse_mixture_experts_17_b200 import moe as M
+    if rank == 0 or not os.path.exists(M.LIB_PATH):
+        B.build()
+    barrier(world)
+    M.lib()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    peaks, peak_src = load_peaks()
+    w = I.WORKLOADS[a.workload]
+    inp = I.make_inputs(w, dev, seed=0)
+    layer = M.MoeLayer(inp)
+    x = inp["x"]
+    out = torch.empty(w.T, w.d, dtype=torch.float32, device=dev)
+    idx = torch.empty(w.T, w.k, dtype=torch.int32, device=dev)
+
+    for _ in range(a.warmup):
+        layer.forward(x, out=out, topk_idx_out=idx)
+    torch.cuda.synchronize()
+    if int(layer.status.item()) != 0:
+        raise RuntimeError(f"device status {int(layer.status.item())} after warm-up")
+    n_kept = routed_kept(idx, w.E, w.capacity)
+
+    launches0 = M.moe_kernel_launches()
+    M.moe_profile_enable(True)
+    with ClockSampler(local) as clk:
+        barrier(world)
+        torch.cuda.synchronize()
+        step_ms = time_loop(lambda: layer.forward(x, out=out), a.steps, stream)
+        torch.cuda.synchronize()
+        barrier(world)
+    M.moe_profile_enable(False)
+    stages = M.moe_profile_read()
+    launches = M.moe_kernel_launches() - launches0
+    step_ms_max = max_over_ranks(step_ms, world, dev)
+    tokens_all = sum_over_ranks(float(w.T), world, dev)
+    value = tokens_all / (step_ms_max / 1e3)
+
+    flops, w13_flops, w2_flops = prefill_flops(w, n_kept)
+    w13_ms = stages["w13"][0] / stages["w13"][1]
+    w2_ms = stages["w2"][0] / stages["w2"][1]
+    peak_t = peaks["bf16_tflops_sustained"]
+    ach = w13_flops / (w13_ms / 1e3) / 1e12
+    roofline = {"bound": "tensor", "kernel": "k_gemm_tc<256,SWIGLU> (grouped w1/w3 GEMM + SwiGLU)",
+                "achieved": round(ach, 1), "peak": peak_t, "unit": "TFLOP/s",
+                "frac": round(ach / peak_t, 4), "traffic": None,
+                "peak_source": f"{peak_src} bf16_tflops_sustained",
+                "frac_of_burst_peak": round(ach / peaks["bf16_tflops"], 4),
+                "frac_of_nominal_2250": round(ach / 2250.0, 4),
+                "algorithmic_flops_per_launch": w13_flops, "avg_launch_ms": round(w13_ms, 4)}
+    stage_ms = {k: round(v[0] / v[1], 4) for k, v in stages.items()}
+    w2_tflops = w2_flops / (w2_ms / 1e3) / 1e12
+
+    # ---- end to end through the C ABI with host buffers (H2D + D2H inside)
+    shape_h = M.shape_of(w, M.MOE_FLAG_HOST_IO)
+    ws_h = M.alloc_workspace(shape_h, dev)
+    x_h = x.cpu().pin_memory()
+    out_h = torch.empty(w.T, w.d, dtype=torch.float32).pin_memory()
+
+    def e2e_step():
+        M.moe_forward_host(shape_h, x_h, layer.Wg, layer.bias, layer.W13, layer.W2, layer.W13s,
+                           layer.W2s, out_h, layer.status, ws_h)
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = time_loop(e2e_step, max(3, a.steps // 2), stream)
+    e2e_ms = max_over_ranks(e2e_ms, world, dev)
+    e2e = {"value": round(tokens_all / (e2e_ms / 1e3), 1), "unit": "tokens/s",
+           "h2d_bytes_per_step": x_h.numel() * 2, "d2h_bytes_per_step": out_h.numel() * 4,
+           "ms_per_step": round(e2e_ms, 4), "api": "moe_forward_host (pinned host x and out)"}
+    del ws_h
+
+    # ---- decode (T = 1, 2, 4, 8 on the same Mixtral-shape weights)
+    decode = None
+    if a.workload == "prefill" and not a.no_extra:
+        decode = {}
+        for T in I.DECODE_TS:
+            xt = x[:T].contiguous()
+            it = torch.empty(T, w.k, dtype=torch.int32, device=dev)
+            ot = torch.empty(T, w.d, dtype=torch.float32, device=dev)
+            for _ in range(5):
+                layer.forward(xt, out=ot, topk_idx_out=it)
+            torch.cuda.synchronize()
+            U, nbytes, w13_bytes, expert_bytes = decode_bytes(w, T, it)
+            M.moe_profile_enable(True)
+            ms = time_loop(lambda: layer.forward(xt, out=ot), 50, stream)
+            M.moe_profile_enable(False)
+            st = M.moe_profile_read()
+            ms = max_over_ranks(ms, world, dev)
+            k13 = st["dec_w13"][0] / st["dec_w13"][1]
+            k2 = st["dec_w2"][0] / st["dec_w2"][1]
+            decode[f"T{T}"] = {
+                "tokens_per_s": round(T * world / (ms / 1e3), 1), "ms_per_step": round(ms, 4),
+                "unique_experts": U, "bytes_per_step": nbytes,
+                "GB_s": round(nbytes / (ms / 1e3) / 1e9, 1),
+                "frac_hbm_measured": round(nbytes / (ms / 1e3) / 1e9 / peaks["hbm_gbs"], 4),
+                "frac_hbm_nominal_8000": round(nbytes / (ms / 1e3) / 1e9 / 8000.0, 4),
+                "chosen_expert_GB_s_kernels": round(expert_bytes / ((k13 + k2) / 1e3) / 1e9, 1),
+                "dec_w13_GB_s": round(w13_bytes / (k13 / 1e3) / 1e9, 1),
+                "stages_ms": {k: round(v[0] / v[1], 4) for k, v in st.items()}}
+
+    # ---- CPU baseline: the oracle on host cores (rank 0, N = 1 only)
+    cpu = None
+    if world == 1 and not a.no_cpu_baseline:
+        rate, cores, sample, _ = cpu_oracle_timing(w, budget_s=a.cpu_budget)
+        cpu = {"value": round(rate, 3), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+               "sample": sample}
+
+    res = {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+        "steps": a.steps, "warmup": a.warmup, "ms_per_step": round(step_ms_max, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded, N(0,1) x, N(0,0.02) bf16 weights)",
+        "config": {"workload": w.name, "T": w.T, "d_model": w.d, "d_ff": w.d_ff, "E": w.E,
+                   "k": w.k, "capacity": w.capacity, "d_ff_shared": w.d_ff_shared,
+                   "zipf_s": w.zipf_s, "seed": 0, "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2 (expert weights and activations exceed 126 MB)",
+                   "output": "fp32 [T, d]"},
+        "active_tflops": round(flops / (step_ms_max / 1e3) / 1e12, 1),
+        "active_tflops_frac_measured_sustained": round(flops / (step_ms_max / 1e3) / 1e12 / peak_t, 4),
+        "n_kept": n_kept,
+        "w2_tflops": round(w2_tflops, 1),
+        "stages_ms": stage_ms,
+        "roofline": roofline,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": int(launches),
+        "clocks": clk.summary(),
+    }
+    if decode is not None:
+        res["decode"] = decode
+    return res
+
+
+def run_reference(a, world, rank):
+    """The oracle as the reference arm: same metric/unit/config, host cores."""
+    w = I.WORKLOADS[a.workload]
+    from oracle import oracle as O
+    O.build()
+    rate, cores, sample, n = cpu_oracle_timing(w, budget_s=a.cpu_budget, steps=max(1, a.steps // 10))
+    ms = n / rate * 1e3
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(rate, 3), "unit": "tokens/s",
+        "n_gpus": world, "steps": a.steps, "warmup": a.warmup, "ms_per_step": round(ms, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded, N(0,1) x, N(0,0.02) bf16 weights)",
+        "config": {"workload": w.name, "T": w.T, "d_model": w.d, "d_ff": w.d_ff, "E": w.E,
+                   "k": w.k, "capacity": w.capacity, "d_ff_shared": w.d_ff_shared,
+                   "zipf_s": w.zipf_s, "seed": 0, "parallelism": "host cores"},
+        "cpu_baseline": {"value": round(rate, 3), "unit": "tokens/s", "cores": cores,
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(rate, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(I.WORKLOADS), default="prefill")
+    ap.add_argument("--no-extra", action="store_true", help="skip the decode measurements")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds per oracle sample")
+    a = ap.parse_args(argv)
+    if a.warmup < 3 and a.impl == "ours":
+        a.warmup = 3
+    if a.impl == "reference":
+        world, rank, _ = dist_setup(False)
+        if rank != 0:
+            return 0
+        print(json.dumps(run_reference(a, world, rank)), flush=True)
+        return 0
+    world, rank, local = dist_setup(True)
+    res = run_ours(a, world, rank, local)
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,242 @@
+/*
+ * moe.h -- C ABI of libmoe.so: the forward pass of a top-k routed
+ * Mixture-of-Experts SwiGLU FFN layer on NVIDIA B200 (sm_100a).
+ *
+ * The layer (defined on "MoE Model Architectures", architectures.md, section
+ * "Mixtral 8x7B", subsections "Sparse MoE Block" and "Expert FFN"; the bias
+ * and the shared expert from section "DeepSeek-V3"):
+ *   logits = x W_g^T + b                          router GEMM, fp32
+ *   idx, w = top-k of softmax(logits), w / sum(w)  lowest index wins ties
+ *   counts, offsets, permutation                   grouped by expert
+ *   h      = silu(x W1_e^T) * (x W3_e^T)           per chosen expert, bf16
+ *   out[t] = sum_j w[t,j] * (h W2_e^T) [+ shared]  fp32
+ *
+ * Conventions for every call
+ *  - Tensor arguments are DEVICE pointers owned by the caller, contiguous and
+ *    row-major, at least 16-byte aligned (256-byte alignment recommended).
+ *    The library never allocates device memory, never frees the caller's
+ *    memory and never synchronises the stream.
+ *  - Scratch space comes from a caller-provided workspace `ws` of `ws_bytes`
+ *    bytes (at least moe_workspace_size()), 256-byte aligned. Calls that
+ *    share one workspace must be ordered on the GPU (same stream).
+ *  - Every call is asynchronous on `stream` and performs no host<->device
+ *    synchronisation, so a sequence of calls can be captured in a CUDA graph.
+ *  - The return value is a host-detected status (MOE_OK or an MOE_ERR_* code).
+ *    On any non-zero return nothing was launched. A launch failure reported
+ *    by the CUDA runtime returns MOE_ERR_CUDA.
+ *  - Errors found on the device are OR-ed into `*status` (a device uint32,
+ *    which may be NULL to ignore them) as the bit (1u << MOE_ERR_*). The
+ *    caller clears it and reads it whenever it chooses. When a device error
+ *    is flagged, the outputs of that call are unspecified.
+ *  - T = 0 is a valid no-op for every call.
+ *
+ * Types: bf16 is the 16-bit bfloat16 bit pattern (uint16_t here); fp32 is
+ * float; ids and positions are int32_t.
+ */
+#ifndef MOE_H_
+#define MOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t moe_bf16_t;
+typedef struct CUstream_st *moe_stream_t; /* same object as cudaStream_t; NULL = legacy default stream */
+
+/* Status codes (host return values, and bit positions of the device word). */
+enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1, /* null pointer, bad shape (see moe_shape_t), misaligned pointer */
+    MOE_ERR_UNSUPPORTED = 2, /* valid request that this build does not implement */
+    MOE_ERR_WORKSPACE = 3,   /* ws too small or misaligned */
+    MOE_ERR_CUDA = 4,        /* the CUDA runtime refused a launch or query */
+    MOE_ERR_NONFINITE = 5,   /* device: a logit row holds NaN, or its maximum is +-inf */
+    MOE_ERR_BAD_EXPERT = 6,  /* device: an expert id outside [0,E) or repeated within a token */
+    MOE_ERR_TIMEOUT = 7      /* device: a pipeline wait gave up (the kernel returned, no hang) */
+};
+
+/* Flags (moe_shape_t.flags). */
+enum {
+    MOE_FLAG_DETERMINISTIC = 1 << 0, /* combine in a fixed order (y_perm + moe_combine) instead
+                                        of fused fp32 atomics in the w2 epilogue */
+    MOE_FLAG_FORCE_PREFILL = 1 << 1, /* moe_forward: never take the small-T decode kernels */
+    MOE_FLAG_FORCE_DECODE = 1 << 2,  /* moe_forward: take the decode kernels whenever
+                                        T <= MOE_DECODE_MAX_T (else MOE_ERR_UNSUPPORTED) */
+    MOE_FLAG_SIMT_FFN = 1 << 3,      /* expert GEMMs on CUDA cores (slow debugging path that
+                                        cross-checks the tensor-core kernels) */
+    MOE_FLAG_HOST_IO = 1 << 4        /* workspace also holds device staging for x and out,
+                                        as moe_forward_host needs */
+};
+
+#define MOE_MAX_E 256
+#define MOE_MAX_K 16
+#define MOE_DECODE_MAX_T 16
+#define MOE_DECODE_DEFAULT_T 16
+
+/* Layer shape. Requirements (else MOE_ERR_INVALID_ARG):
+ *   0 <= T <= 2^24; 1 <= E <= MOE_MAX_E; 1 <= k <= min(E, MOE_MAX_K);
+ *   d and d_ff multiples of 128 in [128, 32768]; d_ff_shared 0 or a multiple
+ *   of 128 in [128, 32768]; capacity <= 0 means uncapped.
+ * capacity (reading of "Switch Transformers" / "Top-1 Routing" on the
+ * architectures page, whose mask is garbled, and of "Faster writing: run only
+ * the chosen experts", where a capacity factor of 0 means uncapped): an
+ * assignment (t, j) is kept iff fewer than `capacity` assignments to the same
+ * expert precede it in row-major (token, slot) order. Dropped assignments
+ * contribute nothing and the kept weights are not renormalised. */
+typedef struct moe_shape {
+    int32_t T, d, d_ff, E, k;
+    int32_t capacity;
+    int32_t d_ff_shared;
+    int32_t flags;
+} moe_shape_t;
+
+/* Short text for a status code (static storage). */
+MOE_API const char *moe_status_string(int code);
+
+/* Bytes of workspace that every call below needs for this shape and flags. */
+MOE_API int moe_workspace_size(const moe_shape_t *shape, size_t *bytes);
+
+/* Pack the expert gate and up projections for the tensor-core GEMM.
+ *   W1, W3  [E, d_ff, d] bf16 (nn.Linear [out, in], "Expert FFN": w1, w3)
+ *   W13     [E, 2*d_ff, d] bf16 output: for each block b of 128 columns,
+ *           rows 256b..256b+127 are W1 rows 128b.., rows 256b+128..256b+255
+ *           are W3 rows 128b.. (gate and up of a column side by side).
+ * With E = 1 it packs a shared expert (d_ff = d_ff_shared). */
+MOE_API int moe_pack_w13(const moe_shape_t *shape, const moe_bf16_t *W1, const moe_bf16_t *W3,
+                 moe_bf16_t *W13, moe_stream_t stream);
+
+/* Router and top-k ("Sparse MoE Block": gate -> softmax -> topk -> divide by
+ * the sum; bias from "Auxiliary-Loss-Free Load Balancing").
+ *   x       [T, d] bf16, or NULL: then `logits` is an INPUT [T, E] fp32
+ *   Wg      [E, d] bf16 (ignored when x is NULL)
+ *   bias    [E] fp32 or NULL (ignored when x is NULL)
+ *   logits  [T, E] fp32, output (x != NULL) or input (x == NULL)
+ *   topk_idx [T, k] int32 out: experts in selection order (largest logit
+ *            first; equal logits -> lower index first; -0.0 == +0.0)
+ *   topk_w  [T, k] fp32 out: exp(l_j - max) / sum over the chosen k, which
+ *           equals the softmax over all E renormalised over the top-k
+ * Device errors: MOE_ERR_NONFINITE. */
+MOE_API int moe_route(const moe_shape_t *shape, const moe_bf16_t *x, const moe_bf16_t *Wg,
+              const float *bias, float *logits, int32_t *topk_idx, float *topk_w,
+              uint32_t *status, void *ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Expert histogram, offsets, capacity and token permutation ("Current Bug:
+ * CuTeDSLMoERunner produces wrong output", "How the pipeline works": counts
+ * [4,4,0] -> offsets [0,4,8,8]; "Sparse MoE Block": torch.where order).
+ *   topk_idx       [T, k] int32 in: distinct ids in [0, E) per token
+ *   x              [T, d] bf16 in (may be NULL: then x_perm is not written)
+ *   expert_counts  [E] int32 out: routed assignments per expert (before capacity)
+ *   expert_offsets [E+1] int32 out: exclusive scan of min(count, capacity)
+ *   slot_pos       [T, k] int32 out: permuted row of (t, j), -1 if dropped
+ *   perm_token     [T*k] int32 out: token of each permuted row; rows within an
+ *                  expert are in ascending token order; rows >= n_kept untouched
+ *   x_perm         [T*k, d] bf16 out: x_perm[slot_pos[t,j]] = x[t]
+ *   n_kept         [1] int32 out: expert_offsets[E]
+ * Bit-exact: the result is a function of topk_idx alone.
+ * Device errors: MOE_ERR_BAD_EXPERT. */
+MOE_API int moe_permute(const moe_shape_t *shape, const int32_t *topk_idx, const moe_bf16_t *x,
+                int32_t *expert_counts, int32_t *expert_offsets, int32_t *slot_pos,
+                int32_t *perm_token, moe_bf16_t *x_perm, int32_t *n_kept, uint32_t *status,
+                void *ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Grouped expert FFN over the chosen experts only ("Expert FFN", run on the
+ * rows [offsets[e], offsets[e+1]) of each expert as "Sparse MoE Block" does).
+ *   x_perm   [T*k, d] bf16 in; expert_offsets [E+1] int32 in
+ *   W13      [E, 2*d_ff, d] bf16 (moe_pack_w13); W2 [E, d, d_ff] bf16
+ *   perm_token [T*k], slot_pos [T, k] int32, topk_w [T, k] fp32 (used only
+ *            by the fused combine)
+ *   y_perm   [T*k, d] fp32 or NULL. Non-NULL: writes the UNWEIGHTED expert
+ *            output of each kept row (for moe_combine); `out` is ignored.
+ *            NULL: fused combine, out[perm_token[r]] += w * y[r] with fp32
+ *            atomics; `out` [T, d] fp32 must hold zeros or a partial sum
+ *            (e.g. the shared expert's output).
+ * H, the bf16 SwiGLU product [T*k, d_ff], lives in the workspace. */
+MOE_API int moe_expert_ffn(const moe_shape_t *shape, const moe_bf16_t *x_perm,
+                   const int32_t *expert_offsets, const moe_bf16_t *W13, const moe_bf16_t *W2,
+                   const int32_t *perm_token, const int32_t *slot_pos, const float *topk_w,
+                   float *y_perm, float *out, uint32_t *status, void *ws, size_t ws_bytes,
+                   moe_stream_t stream);
+
+/* Routing-weighted combine in a fixed order ("Sparse MoE Block": scale by
+ * the routing weight, index_add into token order; "DeepSeekMoE Architecture":
+ * shared_output + routed_output):
+ *   out[t] = shared_out[t] + sum_{j = 0..k-1, slot_pos[t,j] >= 0} w[t,j] * y_perm[slot_pos[t,j]]
+ *   y_perm [T*k, d] fp32; slot_pos [T, k]; topk_w [T, k]; shared_out [T, d]
+ *   fp32 or NULL; out [T, d] fp32 (may alias shared_out). Deterministic. */
+MOE_API int moe_combine(const moe_shape_t *shape, const float *y_perm, const int32_t *slot_pos,
+                const float *topk_w, const float *shared_out, float *out, moe_stream_t stream);
+
+/* The whole layer forward, one stream, no host synchronisation.
+ *   x [T, d] bf16; Wg [E, d] bf16; bias [E] fp32 or NULL;
+ *   W13 [E, 2*d_ff, d] bf16 packed; W2 [E, d, d_ff] bf16;
+ *   W13_shared [2*d_ff_shared, d] bf16 packed and W2_shared [d, d_ff_shared]
+ *   bf16 when d_ff_shared > 0 (else NULL);
+ *   out [T, d] fp32 (fully written);
+ *   logits_out [T, E] fp32, topk_idx_out [T, k] int32: optional copies.
+ * T <= MOE_DECODE_DEFAULT_T takes the decode kernels, which stream only the
+ * chosen experts' weights once ("Faster writing: run only the chosen
+ * experts"; "perf(moe): route granite-4.0-h single-token MoE through the fused
+ * kernel"); larger T takes router -> top-k -> histogram -> permute -> grouped
+ * tensor-core GEMMs with the SwiGLU and the weighted combine in their
+ * epilogues. Device errors: NONFINITE, BAD_EXPERT, TIMEOUT. */
+MOE_API int moe_forward(const moe_shape_t *shape, const moe_bf16_t *x, const moe_bf16_t *Wg,
+                const float *bias, const moe_bf16_t *W13, const moe_bf16_t *W2,
+                const moe_bf16_t *W13_shared, const moe_bf16_t *W2_shared, float *out,
+                float *logits_out, int32_t *topk_idx_out, uint32_t *status, void *ws,
+                size_t ws_bytes, moe_stream_t stream);
+
+/* moe_forward from and to HOST memory: copies x_host [T, d] bf16 into the
+ * workspace, runs the layer, copies out [T, d] fp32 back into out_host, all
+ * asynchronously on `stream` (cudaMemcpyAsync; use pinned host buffers for
+ * true asynchrony). The caller synchronises the stream before reading
+ * out_host. Weights and bias are device pointers as in moe_forward. The
+ * workspace must be sized with MOE_FLAG_HOST_IO set in shape->flags. */
+MOE_API int moe_forward_host(const moe_shape_t *shape, const moe_bf16_t *x_host, const moe_bf16_t *Wg,
+                     const float *bias, const moe_bf16_t *W13, const moe_bf16_t *W2,
+                     const moe_bf16_t *W13_shared, const moe_bf16_t *W2_shared, float *out_host,
+                     uint32_t *status, void *ws, size_t ws_bytes, moe_stream_t stream);
+
+/* ---- Instrumentation (computes nothing; for measurement and tests). ---- */
+
+/* Stages of moe_forward timed by the profiler below. */
+enum {
+    MOE_STAGE_ROUTER = 0,   /* router logits */
+    MOE_STAGE_TOPK = 1,     /* softmax / top-k / weights */
+    MOE_STAGE_HIST = 2,     /* histogram, offsets, tile list */
+    MOE_STAGE_PERMUTE = 3,  /* permutation and gather of x */
+    MOE_STAGE_SHARED = 4,   /* shared expert (both GEMMs) */
+    MOE_STAGE_W13 = 5,      /* grouped w1/w3 GEMM + SwiGLU */
+    MOE_STAGE_W2 = 6,       /* grouped w2 GEMM + weighted combine */
+    MOE_STAGE_COMBINE = 7,  /* fixed-order combine (deterministic mode) */
+    MOE_STAGE_DEC_W13 = 8,  /* decode: chosen experts' w1/w3 + SwiGLU */
+    MOE_STAGE_DEC_W2 = 9,   /* decode: chosen experts' w2 + combine */
+    MOE_NUM_STAGES = 10
+};
+
+/* Number of kernels this library has launched in this process. */
+MOE_API uint64_t moe_kernel_launches(void);
+
+/* on != 0: from now on moe_forward records a CUDA event before and after each
+ * stage, on the caller's stream (events are created here, once); on == 0:
+ * stop recording. Not for concurrent use from several host threads. */
+MOE_API int moe_profile_enable(int on);
+
+/* Wait for the recorded events, then write per-stage total milliseconds and
+ * call counts since the last read (arrays of n <= MOE_NUM_STAGES entries;
+ * either may be NULL) and forget the records. */
+MOE_API int moe_profile_read(double *ms, int64_t *calls, int n);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_H_ */

@@ -1,0 +1,581 @@
+// dispatch.cu -- router (CUDA-core path), softmax/top-k, expert histogram and
+// offsets, token permutation, fixed-order combine and W1/W3 packing.
+//
+// Layer definition: "MoE Model Architectures" (architectures.md), section
+// "Mixtral 8x7B", "Sparse MoE Block"; offsets as in "Current Bug:
+// CuTeDSLMoERunner produces wrong output", "How the pipeline works".
+#include <climits>
+#include <cmath>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+
+// ---------------------------------------------------------------- router (CUDA cores)
+// logits[t, e] = sum_i x[t, i] * Wg[e, i] + bias[e]. A CTA computes a tile of
+// 64 tokens x EC experts; each thread owns TPT tokens x 4 experts; K is staged
+// through shared memory 32 at a time. Used for decode-sized T, for the
+// CUDA-core debugging path, and as the router when tensor cores are not used.
+template <int EC>
+__global__ void __launch_bounds__(256) k_router_simt(const uint16_t *__restrict__ x,
+                                                     const uint16_t *__restrict__ Wg,
+                                                     const float *__restrict__ bias, int T, int d,
+                                                     int E, float *__restrict__ logits)
+{
+    constexpr int EG = EC / 4;      // expert groups of 4
+    constexpr int TG = 256 / EG;    // token groups
+    constexpr int TPT = 64 / TG;    // tokens per thread
+    __shared__ float xs[32][64 + 1];
+    __shared__ float ws[32][EC + 1];
+    const int tid = threadIdx.x;
+    const int t0 = blockIdx.x * 64, e0 = blockIdx.y * EC;
+    const int eg = tid % EG, tg = tid / EG;
+    float acc[TPT][4];
+#pragma unroll
+    for (int i = 0; i < TPT; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            acc[i][j] = 0.f;
+
+    for (int k0 = 0; k0 < d; k0 += 32) {
+        {   // x tile: 64 tokens x 32 k, one 16-B load per thread
+            const int tt = tid / 4, kk = (tid % 4) * 8;
+            uint4 v = make_uint4(0, 0, 0, 0);
+            if (t0 + tt < T)
+                v = *reinterpret_cast<const uint4 *>(x + (size_t)(t0 + tt) * d + k0 + kk);
+            const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                xs[kk + 2 * q][tt] = bf16lo(u[q]);
+                xs[kk + 2 * q + 1][tt] = bf16hi(u[q]);
+            }
+        }
+        if (tid < EC * 4) {   // Wg tile: EC experts x 32 k
+            const int ee = tid / 4, kk = (tid % 4) * 8;
+            uint4 v = make_uint4(0, 0, 0, 0);
+            if (e0 + ee < E)
+                v = *reinterpret_cast<const uint4 *>(Wg + (size_t)(e0 + ee) * d + k0 + kk);
+            const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                ws[kk + 2 * q][ee] = bf16lo(u[q]);
+                ws[kk + 2 * q + 1][ee] = bf16hi(u[q]);
+            }
+        }
+        __syncthreads();
+#pragma unroll 8
+        for (int kk = 0; kk < 32; ++kk) {
+            float a[TPT], b[4];
+#pragma unroll
+            for (int i = 0; i < TPT; ++i)
+                a[i] = xs[kk][tg + i * TG];
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                b[j] = ws[kk][eg + j * EG];
+#pragma unroll
+            for (int i = 0; i < TPT; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+        }
+        __syncthreads();
+    }
+#pragma unroll
+    for (int i = 0; i < TPT; ++i) {
+        const int t = t0 + tg + i * TG;
+        if (t >= T)
+            continue;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int e = e0 + eg + j * EG;
+            if (e < E)
+                logits[(size_t)t * E + e] = acc[i][j] + (bias ? bias[e] : 0.f);
+        }
+    }
+}
+
+int launch_router_simt(const moe_shape_t &s, const uint16_t *x, const uint16_t *Wg,
+                       const float *bias, float *logits, cudaStream_t st)
+{
+    if (s.T == 0)
+        return MOE_OK;
+    const dim3 block(256);
+    if (s.E <= 16) {
+        k_router_simt<16><<<dim3((s.T + 63) / 64, 1), block, 0, st>>>(x, Wg, bias, s.T, s.d, s.E,
+                                                                        logits);
+    } else {
+        k_router_simt<64><<<dim3((s.T + 63) / 64, (s.E + 63) / 64), block, 0, st>>>(
+            x, Wg, bias, s.T, s.d, s.E, logits);
+    }
+    return launched();
+}
+
+// ---------------------------------------------------------------- softmax + top-k
+// One warp per token. Lane l holds logits l, l+32, ... (VPL per lane). k
+// rounds of a butterfly arg-max with the key (larger value, then smaller
+// index) pick the experts in selection order; the weights are
+// exp(l_j - l_max) / sum over the chosen k, which is the softmax over all E
+// renormalised over the top-k (the full-E denominator cancels).
+template <int VPL>
+__global__ void __launch_bounds__(256) k_topk(const float *__restrict__ logits, int T, int E,
+                                              int k, int32_t *__restrict__ idx,
+                                              float *__restrict__ w, int32_t *counter_to_zero,
+                                              uint32_t *status)
+{
+    if (counter_to_zero && blockIdx.x == 0 && threadIdx.x == 0)
+        *counter_to_zero = 0;
+    const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (t >= T)
+        return;
+    const float *l = logits + (size_t)t * E;
+    float v[VPL];
+    uint32_t avail = 0;
+    bool bad = false;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+        const int e = lane + 32 * i;
+        v[i] = -INFINITY;
+        if (e < E) {
+            v[i] = l[e];
+            avail |= 1u << i;
+            bad |= isnan(v[i]);
+        }
+    }
+    float my_v = 0.f;
+    int my_i = 0;
+    for (int j = 0; j < k; ++j) {
+        float bv = -INFINITY;
+        int bi = INT_MAX;
+#pragma unroll
+        for (int i = 0; i < VPL; ++i) {
+            const int e = lane + 32 * i;
+            if (((avail >> i) & 1u) && (v[i] > bv || (v[i] == bv && e < bi))) {
+                bv = v[i];
+                bi = e;
+            }
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            const float ov = __shfl_xor_sync(kFullMask, bv, off);
+            const int oi = __shfl_xor_sync(kFullMask, bi, off);
+            if (ov > bv || (ov == bv && oi < bi)) {
+                bv = ov;
+                bi = oi;
+            }
+        }
+        if (bi != INT_MAX && (bi & 31) == lane)
+            avail &= ~(1u << (bi >> 5));
+        if (lane == j) {
+            my_v = bv;
+            my_i = bi;
+        }
+    }
+    const float M = __shfl_sync(kFullMask, my_v, 0);
+    bad |= !isfinite(M);
+    if (__any_sync(kFullMask, bad)) {
+        if (lane == 0)
+            flag_status(status, MOE_ERR_NONFINITE);
+    }
+    float ex = (lane < k) ? expf(my_v - M) : 0.f;
+    float sum = ex;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1)
+        sum += __shfl_xor_sync(kFullMask, sum, off);
+    if (lane < k) {
+        idx[(size_t)t * k + lane] = my_i;
+        w[(size_t)t * k + lane] = ex / sum;
+    }
+}
+
+int launch_topk(const moe_shape_t &s, const float *logits, int32_t *idx, float *w,
+                int32_t *counter_to_zero, uint32_t *status, cudaStream_t st)
+{
+    if (s.T == 0)
+        return MOE_OK;
+    const int blocks = (s.T + 7) / 8;
+    const int vpl = (s.E + 31) / 32;
+#define MOE_TOPK_CASE(V)                                                                         \
+    case V:                                                                                      \
+        k_topk<V><<<blocks, 256, 0, st>>>(logits, s.T, s.E, s.k, idx, w, counter_to_zero,       \
+                                          status);                                               \
+        break;
+    switch (vpl) {
+        MOE_TOPK_CASE(1)
+        MOE_TOPK_CASE(2)
+        MOE_TOPK_CASE(4)
+        MOE_TOPK_CASE(8)
+    case 3:
+        k_topk<4><<<blocks, 256, 0, st>>>(logits, s.T, s.E, s.k, idx, w, counter_to_zero, status);
+        break;
+    default:
+        k_topk<8><<<blocks, 256, 0, st>>>(logits, s.T, s.E, s.k, idx, w, counter_to_zero, status);
+        break;
+    }
+#undef MOE_TOPK_CASE
+    return launched();
+}
+
+// ---------------------------------------------------------------- block scan helper
+// Exclusive scan of one int per thread over a 256-thread block.
+__device__ __forceinline__ int block_excl_scan_256(int v, int *s_warp, int *total)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int inc = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int o = __shfl_up_sync(kFullMask, inc, off);
+        if (lane >= off)
+            inc += o;
+    }
+    if (lane == 31)
+        s_warp[warp] = inc;
+    __syncthreads();
+    if (warp == 0) {
+        int wv = (lane < 8) ? s_warp[lane] : 0;
+        int winc = wv;
+#pragma unroll
+        for (int off = 1; off < 8; off <<= 1) {
+            const int o = __shfl_up_sync(kFullMask, winc, off);
+            if (lane >= off)
+                winc += o;
+        }
+        if (lane < 8)
+            s_warp[8 + lane] = winc - wv;
+        if (lane == 7)
+            s_warp[16] = winc;
+    }
+    __syncthreads();
+    const int r = s_warp[8 + warp] + inc - v;
+    *total = s_warp[16];
+    __syncthreads();
+    return r;
+}
+
+// Writes the grouped-GEMM m-tile list for kept counts in s_kept[E]:
+// expert e contributes ceil(kept/128) tiles starting at rows offsets[e] + 128 i.
+__device__ void build_tiles(const int *s_kept, const int32_t *offsets_smem_or_global, int E,
+                            int32_t *mt_row0, int32_t *mt_group, int32_t *num_mt, int *s_warp)
+{
+    const int tid = threadIdx.x;
+    const int e = tid;
+    const int nt = (e < E) ? (s_kept[e] + kBlockM - 1) / kBlockM : 0;
+    int total;
+    const int start = block_excl_scan_256(nt, s_warp, &total);
+    if (e < E) {
+        const int base = offsets_smem_or_global[e];
+        for (int i = 0; i < nt; ++i) {
+            mt_row0[start + i] = base + i * kBlockM;
+            mt_group[start + i] = e;
+        }
+    }
+    if (tid == 0)
+        *num_mt = total;
+}
+
+// ---------------------------------------------------------------- histogram + scan
+// One CTA per chunk of 256 tokens (thread = token). For each slot j the warp
+// groups equal expert ids with __match_any_sync; the group leader ORs the
+// group's lane mask into mask[warp][e] (no atomics: leaders are unique per
+// round, rounds are ordered by __syncwarp). A token's rank within the chunk
+// is the popcount of earlier warps' masks plus the lower lanes of its own.
+// The last CTA to finish (ticket counter) scans the per-chunk counts in chunk
+// order, applies the capacity, writes offsets and the GEMM tile list, and
+// re-arms the counter. The result depends only on idx: bit-exact.
+__global__ void __launch_bounds__(256) k_hist_scan(
+    const int32_t *__restrict__ idx, int T, int E, int k, int C, int32_t *chunk_counts,
+    int32_t *__restrict__ rank_local, int32_t *counter, int32_t *__restrict__ counts,
+    int32_t *__restrict__ offsets, int32_t *__restrict__ n_kept, int32_t *mt_row0,
+    int32_t *mt_group, int32_t *num_mt, uint32_t *status)
+{
+    __shared__ uint32_t mask[8][MOE_MAX_E];
+    __shared__ int32_t wpre[8][MOE_MAX_E];
+    __shared__ int s_last;
+    __shared__ int s_warp[17];
+    __shared__ int s_kept[MOE_MAX_E];
+    __shared__ int s_off[MOE_MAX_E + 1];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int t = blockIdx.x * kChunkTokens + tid;
+    const bool live = t < T;
+    for (int i = tid; i < 8 * MOE_MAX_E; i += 256)
+        (&mask[0][0])[i] = 0u;
+    __syncthreads();
+
+    bool flagged = false;
+    for (int j = 0; j < k; ++j) {
+        int e = live ? idx[(size_t)t * k + j] : -1;
+        if (live && (e < 0 || e >= E)) {
+            flagged = true;
+            e = -1;
+        }
+        if (e >= 0) {
+            for (int jj = 0; jj < j; ++jj)
+                if (idx[(size_t)t * k + jj] == e) {
+                    flagged = true;
+                    e = -1;
+                    break;
+                }
+        }
+        const uint32_t g = __match_any_sync(kFullMask, e);
+        if (e >= 0 && lane == __ffs(g) - 1)
+            mask[warp][e] |= g;
+        __syncwarp();
+    }
+    if (flagged)
+        flag_status(status, MOE_ERR_BAD_EXPERT);
+    __syncthreads();
+    for (int e = tid; e < E; e += 256) {
+        int run = 0;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) {
+            wpre[w][e] = run;
+            run += __popc(mask[w][e]);
+        }
+        chunk_counts[(size_t)blockIdx.x * E + e] = run;
+    }
+    __syncthreads();
+    if (live) {
+        for (int j = 0; j < k; ++j) {
+            int e = idx[(size_t)t * k + j];
+            int r = -1;
+            if (e >= 0 && e < E) {
+                bool dup = false;
+                for (int jj = 0; jj < j; ++jj)
+                    dup |= (idx[(size_t)t * k + jj] == e);
+                if (!dup)
+                    r = wpre[warp][e] + __popc(mask[warp][e] & lanemask_lt());
+            }
+            rank_local[(size_t)t * k + j] = r;
+        }
+    }
+
+    // ---- the last CTA scans all chunks
+    __threadfence();
+    __syncthreads();
+    if (tid == 0)
+        s_last = (atomicAdd(counter, 1) == (int)gridDim.x - 1);
+    __syncthreads();
+    if (!s_last)
+        return;
+    __threadfence();
+    const int nchunks = gridDim.x;
+    for (int e = tid; e < MOE_MAX_E; e += 256) {
+        int kept = 0;
+        if (e < E) {
+            int run = 0;
+            for (int c = 0; c < nchunks; ++c) {
+                const int v = __ldcg(&chunk_counts[(size_t)c * E + e]);
+                __stcg(&chunk_counts[(size_t)c * E + e], run);
+                run += v;
+            }
+            counts[e] = run;
+            kept = (C > 0 && run > C) ? C : run;
+        }
+        s_kept[e] = kept;
+    }
+    __syncthreads();
+    int total;
+    const int ex = block_excl_scan_256(tid < E ? s_kept[tid] : 0, s_warp, &total);
+    if (tid < E) {
+        offsets[tid] = ex;
+        s_off[tid] = ex;
+    }
+    if (tid == 0) {
+        offsets[E] = total;
+        *n_kept = total;
+    }
+    __syncthreads();
+    build_tiles(s_kept, s_off, E, mt_row0, mt_group, num_mt, s_warp);
+    if (tid == 0)
+        *counter = 0;
+}
+
+int launch_hist_scan(const moe_shape_t &s, const int32_t *idx, int32_t *chunk_counts,
+                     int32_t *rank_local, int32_t *counter, int32_t *counts, int32_t *offsets,
+                     int32_t *n_kept, int32_t *mt_row0, int32_t *mt_group, int32_t *num_mt,
+                     uint32_t *status, cudaStream_t st)
+{
+    const int nchunks = (s.T + kChunkTokens - 1) / kChunkTokens;
+    if (nchunks == 0)
+        return MOE_OK;
+    k_hist_scan<<<nchunks, 256, 0, st>>>(idx, s.T, s.E, s.k, s.capacity, chunk_counts,
+                                         rank_local, counter, counts, offsets, n_kept, mt_row0,
+                                         mt_group, num_mt, status);
+    return launched();
+}
+
+// ---------------------------------------------------------------- permutation
+// One warp per token: lane j < k resolves slot j's permuted row
+// (offsets[e] + chunk base + rank within the chunk, -1 past the capacity);
+// then the warp copies x[t] once into every kept row with 16-B loads/stores
+// and, when asked, zeroes out[t] (the fused combine accumulates into it).
+__global__ void __launch_bounds__(256) k_permute(
+    const int32_t *__restrict__ idx, int T, int E, int k, int C, int d,
+    const int32_t *__restrict__ chunk_base, const int32_t *__restrict__ rank_local,
+    const int32_t *__restrict__ offsets, const uint4 *__restrict__ x, int32_t *__restrict__ slot_pos,
+    int32_t *__restrict__ perm_token, uint4 *__restrict__ x_perm, float4 *__restrict__ out_zero)
+{
+    const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (t >= T)
+        return;
+    int pos = -1;
+    if (lane < k) {
+        const int e = idx[(size_t)t * k + lane];
+        const int rl = rank_local[(size_t)t * k + lane];
+        if (e >= 0 && e < E && rl >= 0) {
+            const int r = chunk_base[(size_t)(t / kChunkTokens) * E + e] + rl;
+            if (C <= 0 || r < C)
+                pos = offsets[e] + r;
+        }
+        slot_pos[(size_t)t * k + lane] = pos;
+        if (pos >= 0)
+            perm_token[pos] = t;
+    }
+    if (x_perm) {
+        int pj[MOE_MAX_K];
+#pragma unroll
+        for (int j = 0; j < MOE_MAX_K; ++j)
+            pj[j] = __shfl_sync(kFullMask, pos, j);
+        const int nv = d / 8;
+        const uint4 *src = x + (size_t)t * nv;
+        for (int c = lane; c < nv; c += 32) {
+            const uint4 v = src[c];
+#pragma unroll
+            for (int j = 0; j < MOE_MAX_K; ++j)
+                if (j < k && pj[j] >= 0)
+                    x_perm[(size_t)pj[j] * nv + c] = v;
+        }
+    }
+    if (out_zero) {
+        const int nv = d / 4;
+        for (int c = lane; c < nv; c += 32)
+            out_zero[(size_t)t * nv + c] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+}
+
+int launch_permute(const moe_shape_t &s, const int32_t *idx, const int32_t *chunk_base,
+                   const int32_t *rank_local, const int32_t *offsets, const uint16_t *x,
+                   int32_t *slot_pos, int32_t *perm_token, uint16_t *x_perm, float *out_zero,
+                   cudaStream_t st)
+{
+    if (s.T == 0)
+        return MOE_OK;
+    k_permute<<<(s.T + 7) / 8, 256, 0, st>>>(
+        idx, s.T, s.E, s.k, s.capacity, s.d, chunk_base, rank_local, offsets,
+        reinterpret_cast<const uint4 *>(x), slot_pos, perm_token, reinterpret_cast<uint4 *>(x_perm),
+        reinterpret_cast<float4 *>(out_zero));
+    return launched();
+}
+
+// ---------------------------------------------------------------- tile list from offsets
+__global__ void __launch_bounds__(256) k_tiles_from_offsets(const int32_t *__restrict__ offsets,
+                                                            int E, int32_t *mt_row0,
+                                                            int32_t *mt_group, int32_t *num_mt)
+{
+    __shared__ int s_kept[MOE_MAX_E];
+    __shared__ int s_off[MOE_MAX_E];
+    __shared__ int s_warp[17];
+    const int e = threadIdx.x;
+    s_kept[e] = (e < E) ? max(0, offsets[e + 1] - offsets[e]) : 0;
+    s_off[e] = (e < E) ? offsets[e] : 0;
+    __syncthreads();
+    build_tiles(s_kept, s_off, E, mt_row0, mt_group, num_mt, s_warp);
+}
+
+int launch_tiles_from_offsets(const moe_shape_t &s, const int32_t *offsets, int32_t *mt_row0,
+                              int32_t *mt_group, int32_t *num_mt, cudaStream_t st)
+{
+    k_tiles_from_offsets<<<1, 256, 0, st>>>(offsets, s.E, mt_row0, mt_group, num_mt);
+    return launched();
+}
+
+// ---------------------------------------------------------------- combine (fixed order)
+__global__ void __launch_bounds__(256) k_combine(const float4 *__restrict__ y,
+                                                 const int32_t *__restrict__ slot_pos,
+                                                 const float *__restrict__ w, int T, int k, int d,
+                                                 const float4 *shared_out, float4 *out)
+{
+    const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (t >= T)
+        return;
+    int pj = -1;
+    float wj = 0.f;
+    if (lane < k) {
+        pj = slot_pos[(size_t)t * k + lane];
+        wj = w[(size_t)t * k + lane];
+    }
+    int ps[MOE_MAX_K];
+    float ws[MOE_MAX_K];
+#pragma unroll
+    for (int j = 0; j < MOE_MAX_K; ++j) {
+        ps[j] = __shfl_sync(kFullMask, pj, j);
+        ws[j] = __shfl_sync(kFullMask, wj, j);
+    }
+    const int nv = d / 4;
+    for (int c = lane; c < nv; c += 32) {
+        float4 acc = shared_out ? shared_out[(size_t)t * nv + c] : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int j = 0; j < MOE_MAX_K; ++j) {
+            const int p = ps[j];
+            const float ww = ws[j];
+            if (j >= k || p < 0)
+                continue;
+            const float4 v = y[(size_t)p * nv + c];
+            acc.x = fmaf(ww, v.x, acc.x);
+            acc.y = fmaf(ww, v.y, acc.y);
+            acc.z = fmaf(ww, v.z, acc.z);
+            acc.w = fmaf(ww, v.w, acc.w);
+        }
+        out[(size_t)t * nv + c] = acc;
+    }
+}
+
+int launch_combine(const moe_shape_t &s, const float *y_perm, const int32_t *slot_pos,
+                   const float *topk_w, const float *shared_out, float *out, cudaStream_t st)
+{
+    if (s.T == 0)
+        return MOE_OK;
+    k_combine<<<(s.T + 7) / 8, 256, 0, st>>>(reinterpret_cast<const float4 *>(y_perm), slot_pos,
+                                             topk_w, s.T, s.k, s.d,
+                                             reinterpret_cast<const float4 *>(shared_out),
+                                             reinterpret_cast<float4 *>(out));
+    return launched();
+}
+
+// ---------------------------------------------------------------- W1/W3 packing
+// W13[e, 256 b + r] = r < 128 ? W1[e, 128 b + r] : W3[e, 128 b + r - 128].
+__global__ void k_pack_w13(const uint4 *__restrict__ W1, const uint4 *__restrict__ W3,
+                           uint4 *__restrict__ W13, int E, int d_ff, int d)
+{
+    const int nv = d / 8;
+    const long long rows = (long long)E * 2 * d_ff;
+    const long long total = rows * nv;
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
+         i += (long long)gridDim.x * blockDim.x) {
+        const long long row = i / nv;
+        const int c = (int)(i - row * nv);
+        const int e = (int)(row / (2 * d_ff));
+        const int r = (int)(row - (long long)e * 2 * d_ff);
+        const int b = r / 256, within = r % 256;
+        const long long src_row = (long long)e * d_ff + b * 128 + (within & 127);
+        W13[i] = (within < 128 ? W1 : W3)[src_row * nv + c];
+    }
+}
+
+int launch_pack_w13(int E, int d_ff, int d, const uint16_t *W1, const uint16_t *W3,
+                    uint16_t *W13, cudaStream_t st)
+{
+    const long long total = (long long)E * 2 * d_ff * (d / 8);
+    if (total == 0)
+        return MOE_OK;
+    const int blocks = (int)std::min<long long>((total + 255) / 256, 148LL * 16);
+    k_pack_w13<<<blocks, 256, 0, st>>>(reinterpret_cast<const uint4 *>(W1),
+                                       reinterpret_cast<const uint4 *>(W3),
+                                       reinterpret_cast<uint4 *>(W13), E, d_ff, d);
+    return launched();
+}
+
+} // namespace moe

@@ -1,0 +1,409 @@
+// gemm_tc.cu -- persistent grouped GEMM on the 5th-generation tensor cores.
+//
+// C[rows of one expert, :] = A[rows, K] * B_e[:, K]^T with A, B bf16 K-major,
+// fp32 accumulation in tensor memory (TMEM), and one of four fused
+// epilogues (EpiMode): the SwiGLU of the w1/w3 GEMM ("Expert FFN" on
+// "MoE Model Architectures"), the routing-weighted scatter-add of the w2 GEMM
+// ("Sparse MoE Block": scale by the routing weight and index_add into token
+// order), a plain fp32 store, and the router logits with bias.
+//
+// Structure (one CTA per SM, 192 threads):
+//   warp 0     TMA producer: 128 x 64 A tile + BN x 64 B tile per stage,
+//              128-byte swizzle, STAGES-deep ring of shared-memory buffers
+//   warp 1     allocates 2*BN TMEM columns; one thread issues
+//              tcgen05.mma (M=128, N=BN, K=16) x4 per stage, commits the
+//              stage back to the producer and the finished accumulator to
+//              the epilogue
+//   warps 2-5  epilogue: tcgen05.ld of the accumulator (each warp owns the
+//              32 TMEM lanes = tile rows of its lane quarter), fused math,
+//              global stores / fp32 vector atomics
+// Two TMEM accumulators alternate so the epilogue of tile i overlaps the
+// main loop of tile i+1. Tiles never mix experts: the m-tile list (built on
+// the device from the expert offsets) gives each 128-row tile one expert; rows
+// past the expert's end are computed and discarded by the epilogue.
+// Every CTA fetches its own tiles; no copy is shared across CTAs.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+
+struct TcArgs {
+    int kblocks;
+    int n_tiles;
+    int group_m;
+    int b_rows_per_group;
+    const int32_t *mt_row0;
+    const int32_t *mt_group;
+    const int32_t *num_mt_dev;
+    int num_mt_host;
+    const int32_t *seg_offsets;
+    long long rows_valid;
+    void *out;
+    long long ldo;
+    const int32_t *perm_token;
+    const int32_t *slot_pos;
+    const float *topk_w;
+    int k;
+    const float *bias;
+    int n_valid;
+    uint32_t *status;
+};
+
+template <int BN>
+struct TcCfg {
+    static constexpr int BM = 128, BK = 64;
+    static constexpr int A_BYTES = BM * BK * 2;
+    static constexpr int B_BYTES = BN * BK * 2;
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+    static constexpr int STAGES = (BN == 256) ? 4 : (BN == 128 ? 6 : 8);
+    static constexpr int TMEM_COLS = 2 * BN;
+    static constexpr int BAR_BYTES = 256;
+    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES;
+};
+
+__device__ __forceinline__ void tile_coords(long long tile, int num_mt, int n_tiles, int group_m,
+                                            int &m_idx, int &n_idx)
+{
+    const long long band_size = (long long)group_m * n_tiles;
+    const int band = (int)(tile / band_size);
+    const int first_m = band * group_m;
+    const int rows = min(group_m, num_mt - first_m);
+    const int r = (int)(tile - (long long)band * band_size);
+    m_idx = first_m + r % rows;
+    n_idx = r / rows;
+}
+
+template <int BN, int MODE>
+__global__ void __launch_bounds__(192, 1)
+    k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+              const TcArgs p)
+{
+    using C = TcCfg<BN>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint8_t *sA = smem;
+    uint8_t *sB = smem + C::STAGES * C::A_BYTES;
+    uint64_t *full = reinterpret_cast<uint64_t *>(sB + C::STAGES * C::B_BYTES);
+    uint64_t *empty = full + C::STAGES;
+    uint64_t *tfull = empty + C::STAGES;
+    uint64_t *tempty = tfull + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tempty + 2);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&tfull[b], 1);
+            mbar_init(&tempty[b], 4);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    const int num_mt = p.num_mt_dev ? *p.num_mt_dev : p.num_mt_host;
+    const long long total = (long long)num_mt * p.n_tiles;
+
+    if (warp == 0) {
+        if (lane == 0) {   // ---------------- TMA producer
+            uint32_t it = 0;
+            for (long long tile = blockIdx.x; tile < total; tile += gridDim.x) {
+                int m_idx, n_idx;
+                tile_coords(tile, num_mt, p.n_tiles, p.group_m, m_idx, n_idx);
+                const int row0 = p.mt_row0 ? p.mt_row0[m_idx] : m_idx * C::BM;
+                const int grp = p.mt_group ? p.mt_group[m_idx] : 0;
+                const int brow = grp * p.b_rows_per_group + n_idx * BN;
+                bool ok = true;
+                for (int kb = 0; kb < p.kblocks; ++kb, ++it) {
+                    const int s = it % C::STAGES;
+                    const uint32_t ph = (it / C::STAGES) & 1u;
+                    if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag, p.status)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&full[s], C::STAGE_BYTES);
+                    tma_load_2d(sA + s * C::A_BYTES, &tmA, kb * C::BK, row0, &full[s]);
+                    tma_load_2d(sB + s * C::B_BYTES, &tmB, kb * C::BK, brow, &full[s]);
+                }
+                if (!ok)
+                    break;
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {   // ---------------- MMA issuer
+            constexpr uint32_t IDESC = idesc_bf16_f32(128, BN);
+            uint32_t it = 0, local = 0;
+            for (long long tile = blockIdx.x; tile < total; tile += gridDim.x, ++local) {
+                const uint32_t b = local & 1u, aph = (local >> 1) & 1u;
+                if (!mbar_wait(&tempty[b], aph ^ 1u, abort_flag, p.status))
+                    break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + b * BN;
+                bool ok = true;
+                for (int kb = 0; kb < p.kblocks; ++kb, ++it) {
+                    const int s = it % C::STAGES;
+                    const uint32_t ph = (it / C::STAGES) & 1u;
+                    if (!mbar_wait(&full[s], ph, abort_flag, p.status)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a0 = smem_u32(sA + s * C::A_BYTES);
+                    const uint32_t b0 = smem_u32(sB + s * C::B_BYTES);
+#pragma unroll
+                    for (int kk = 0; kk < C::BK / 16; ++kk)
+                        tc_mma_bf16(d_tmem, smem_desc_k128(a0 + kk * 32),
+                                    smem_desc_k128(b0 + kk * 32), IDESC, (kb | kk) != 0);
+                    tc_commit(&empty[s]);
+                }
+                if (!ok)
+                    break;
+                tc_commit(&tfull[b]);
+            }
+        }
+    } else {   // ---------------- epilogue warps 2..5
+        const int q = warp & 3;   // TMEM lane quarter this warp may access
+        uint32_t local = 0;
+        for (long long tile = blockIdx.x; tile < total; tile += gridDim.x, ++local) {
+            int m_idx, n_idx;
+            tile_coords(tile, num_mt, p.n_tiles, p.group_m, m_idx, n_idx);
+            const long long row0 = p.mt_row0 ? p.mt_row0[m_idx] : (long long)m_idx * C::BM;
+            const int grp = p.mt_group ? p.mt_group[m_idx] : 0;
+            const long long row_end = p.seg_offsets ? p.seg_offsets[grp + 1] : p.rows_valid;
+            const uint32_t b = local & 1u, aph = (local >> 1) & 1u;
+            if (!mbar_wait(&tfull[b], aph, abort_flag, p.status))
+                break;
+            tc_fence_after();
+            const long long row = row0 + q * 32 + lane;
+            const bool valid = row < row_end;
+            const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + b * BN;
+
+            if (MODE == EPI_SWIGLU) {
+                // accumulator columns [0,128) = gate, [128,256) = up of H columns n_idx*128..
+                uint16_t *H = static_cast<uint16_t *>(p.out) + row * p.ldo + n_idx * 128;
+#pragma unroll 1
+                for (int c = 0; c < 4; ++c) {
+                    float g[32], u[32];
+                    tmem_ld32(tb + c * 32, g);
+                    tmem_ld32(tb + 128 + c * 32, u);
+                    tmem_ld_wait();
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        pk[i] = pack_bf16x2(silu_mul(g[2 * i], u[2 * i]),
+                                            silu_mul(g[2 * i + 1], u[2 * i + 1]));
+                    if (valid) {
+                        uint4 *dst = reinterpret_cast<uint4 *>(H + c * 32);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+                    }
+                }
+            } else if (MODE == EPI_COMBINE) {
+                int t = 0;
+                float wgt = 0.f;
+                if (valid) {
+                    t = p.perm_token[row];
+                    for (int j = 0; j < p.k; ++j)
+                        if (p.slot_pos[(long long)t * p.k + j] == row)
+                            wgt = p.topk_w[(long long)t * p.k + j];
+                }
+                float *o = static_cast<float *>(p.out) + (long long)t * p.ldo + n_idx * BN;
+#pragma unroll 1
+                for (int c = 0; c < BN / 32; ++c) {
+                    float v[32];
+                    tmem_ld32(tb + c * 32, v);
+                    tmem_ld_wait();
+                    if (valid) {
+                        float4 *dst = reinterpret_cast<float4 *>(o + c * 32);
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            atomicAdd(dst + i, make_float4(wgt * v[4 * i], wgt * v[4 * i + 1],
+                                                           wgt * v[4 * i + 2], wgt * v[4 * i + 3]));
+                    }
+                }
+            } else if (MODE == EPI_STORE_F32) {
+                float *o = static_cast<float *>(p.out) + row * p.ldo + n_idx * BN;
+#pragma unroll 1
+                for (int c = 0; c < BN / 32; ++c) {
+                    float v[32];
+                    tmem_ld32(tb + c * 32, v);
+                    tmem_ld_wait();
+                    if (valid) {
+                        float4 *dst = reinterpret_cast<float4 *>(o + c * 32);
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+                    }
+                }
+            } else {   // EPI_ROUTER
+                float *o = static_cast<float *>(p.out) + row * p.ldo;
+#pragma unroll 1
+                for (int c = 0; c < BN / 32; ++c) {
+                    float v[32];
+                    tmem_ld32(tb + c * 32, v);
+                    tmem_ld_wait();
+                    if (valid) {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) {
+                            const int n = n_idx * BN + c * 32 + i;
+                            if (n < p.n_valid)
+                                o[n] = v[i] + (p.bias ? p.bias[n] : 0.f);
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(&tempty[b]);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, C::TMEM_COLS);
+    }
+}
+
+// ---------------------------------------------------------------- host side
+
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    });
+    return fn;
+}
+
+// Row-major bf16 matrix [rows, cols] as a 2-D TMA tensor; box = 64 x box_rows
+// elements (128 B inner extent), 128-byte swizzle, zero fill out of bounds.
+static int make_tmap(CUtensorMap *m, const void *base, long long cols, long long rows,
+                     int box_rows)
+{
+    auto fn = encode_fn();
+    if (!fn)
+        return MOE_ERR_CUDA;
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+    cuuint32_t box[2] = {64u, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1u, 1u};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
+}
+
+int num_sms()
+{
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess)
+        return 148;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+        return 148;
+    return n;
+}
+
+template <int BN, int MODE>
+static int launch_tc_impl(const GemmArgs &g, cudaStream_t st)
+{
+    using C = TcCfg<BN>;
+    CUtensorMap tA, tB;
+    int rc = make_tmap(&tA, g.A, g.K, g.a_rows, 128);
+    if (rc)
+        return rc;
+    rc = make_tmap(&tB, g.B, g.K, g.b_rows_total, BN);
+    if (rc)
+        return rc;
+    TcArgs p;
+    p.kblocks = g.K / 64;
+    p.n_tiles = (MODE == EPI_SWIGLU) ? g.N / 256 : (g.N + BN - 1) / BN;
+    p.group_m = (MODE == EPI_SWIGLU) ? 8 : 16;
+    p.b_rows_per_group = g.b_rows_per_group;
+    p.mt_row0 = g.mt_row0;
+    p.mt_group = g.mt_group;
+    p.num_mt_dev = g.num_mt_dev;
+    p.num_mt_host = g.num_mt_host;
+    p.seg_offsets = g.seg_offsets;
+    p.rows_valid = g.rows_valid;
+    p.out = g.out;
+    p.ldo = g.ldo;
+    p.perm_token = g.perm_token;
+    p.slot_pos = g.slot_pos;
+    p.topk_w = g.topk_w;
+    p.k = g.k;
+    p.bias = g.bias;
+    p.n_valid = g.n_valid;
+    p.status = g.status;
+
+    static int attr_done[64] = {0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < 64 && !attr_done[dev]) {
+        if (cudaFuncSetAttribute(k_gemm_tc<BN, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 C::SMEM_BYTES) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        attr_done[dev] = 1;
+    }
+    const int max_mt = g.num_mt_dev ? g.max_mt : g.num_mt_host;
+    const long long tiles = (long long)max_mt * p.n_tiles;
+    if (tiles <= 0)
+        return MOE_OK;
+    const int grid = (int)std::min<long long>(tiles, num_sms());
+    k_gemm_tc<BN, MODE><<<grid, 192, C::SMEM_BYTES, st>>>(tA, tB, p);
+    return launched();
+}
+
+int launch_gemm_tc(const GemmArgs &g, cudaStream_t st)
+{
+    switch (g.mode) {
+    case EPI_SWIGLU:
+        return launch_tc_impl<256, EPI_SWIGLU>(g, st);
+    case EPI_COMBINE:
+        return (g.N % 256 == 0) ? launch_tc_impl<256, EPI_COMBINE>(g, st)
+                                : launch_tc_impl<128, EPI_COMBINE>(g, st);
+    case EPI_STORE_F32:
+        return (g.N % 256 == 0) ? launch_tc_impl<256, EPI_STORE_F32>(g, st)
+                                : launch_tc_impl<128, EPI_STORE_F32>(g, st);
+    case EPI_ROUTER:
+        if (g.N <= 64)
+            return launch_tc_impl<64, EPI_ROUTER>(g, st);
+        if (g.N <= 128)
+            return launch_tc_impl<128, EPI_ROUTER>(g, st);
+        return launch_tc_impl<256, EPI_ROUTER>(g, st);
+    default:
+        return MOE_ERR_INVALID_ARG;
+    }
+}
+
+} // namespace moe

@@ -1,0 +1,113 @@
+// internal.h -- host-side interface between the C-ABI layer and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "moe.h"
+
+namespace moe {
+
+// Counts every kernel launch of this library (moe_kernel_launches).
+void note_launch();
+
+// Call right after one kernel launch: counts it and maps the launch result.
+inline int launched()
+{
+    note_launch();
+    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+constexpr int kBlockM = 128;      // rows of one grouped-GEMM m-tile
+constexpr int kChunkTokens = 256; // tokens per histogram chunk (one CTA)
+
+// Scratch layout inside the caller's workspace (byte offsets, 256-B aligned).
+struct WsLayout {
+    size_t logits, topk_idx, topk_w;
+    size_t counts, offsets, n_kept, counter, num_mt;
+    size_t chunk_counts, rank_local;
+    size_t slot_pos, perm_token;
+    size_t mt_row0, mt_group;
+    size_t x_perm, H, H_shared, Y;
+    size_t dec_H;
+    size_t x_stage, out_stage;
+    size_t total;
+    int nchunks, max_mt;
+};
+
+WsLayout ws_layout(const moe_shape_t &s);
+
+// ---- routing / dispatch (dispatch.cu)
+int launch_router_simt(const moe_shape_t &s, const uint16_t *x, const uint16_t *Wg,
+                       const float *bias, float *logits, cudaStream_t st);
+int launch_topk(const moe_shape_t &s, const float *logits, int32_t *idx, float *w,
+                int32_t *counter_to_zero, uint32_t *status, cudaStream_t st);
+int launch_hist_scan(const moe_shape_t &s, const int32_t *idx, int32_t *chunk_counts,
+                     int32_t *rank_local, int32_t *counter, int32_t *counts, int32_t *offsets,
+                     int32_t *n_kept, int32_t *mt_row0, int32_t *mt_group, int32_t *num_mt,
+                     uint32_t *status, cudaStream_t st);
+int launch_permute(const moe_shape_t &s, const int32_t *idx, const int32_t *chunk_base,
+                   const int32_t *rank_local, const int32_t *offsets, const uint16_t *x,
+                   int32_t *slot_pos, int32_t *perm_token, uint16_t *x_perm, float *out_zero,
+                   cudaStream_t st);
+int launch_tiles_from_offsets(const moe_shape_t &s, const int32_t *offsets, int32_t *mt_row0,
+                              int32_t *mt_group, int32_t *num_mt, cudaStream_t st);
+int launch_combine(const moe_shape_t &s, const float *y_perm, const int32_t *slot_pos,
+                   const float *topk_w, const float *shared_out, float *out, cudaStream_t st);
+int launch_pack_w13(int E, int d_ff, int d, const uint16_t *W1, const uint16_t *W3,
+                    uint16_t *W13, cudaStream_t st);
+
+// ---- grouped GEMMs (gemm_tc.cu: tcgen05 + TMA; gemm_simt.cu: CUDA cores)
+enum EpiMode {
+    EPI_SWIGLU = 0,     // H[row, n*128 + c] = bf16(silu(acc[c]) * acc[128 + c])
+    EPI_COMBINE = 1,    // out[perm_token[row], :] += w(row) * acc  (fp32 atomics)
+    EPI_STORE_F32 = 2,  // out[row, :] = acc  (fp32)
+    EPI_ROUTER = 3      // out[row, n] = acc[n] + bias[n] for n < n_valid
+};
+
+struct GemmArgs {
+    int mode;
+    // A [a_rows, K] bf16 row-major; B [groups * b_rows_per_group, K] bf16 row-major
+    const uint16_t *A;
+    long long a_rows;
+    const uint16_t *B;
+    long long b_rows_total;
+    int K;
+    int N;                    // output columns of one group (2*d_ff for SWIGLU)
+    int b_rows_per_group;
+    // m-tiles: routed (list on device) or identity (row0 = 128 * i)
+    const int32_t *mt_row0;   // NULL: identity tiles
+    const int32_t *mt_group;
+    const int32_t *num_mt_dev; // NULL: use num_mt_host
+    int num_mt_host;
+    int max_mt;               // upper bound of the m-tile count (grid sizing)
+    const int32_t *seg_offsets; // group g rows end at seg_offsets[g+1]; NULL: rows_valid
+    long long rows_valid;
+    // epilogue
+    void *out;
+    long long ldo;
+    const int32_t *perm_token;
+    const int32_t *slot_pos;
+    const float *topk_w;
+    int k;
+    const float *bias;
+    int n_valid;
+    uint32_t *status;
+};
+
+int launch_gemm_tc(const GemmArgs &g, cudaStream_t st);
+int launch_gemm_simt(const GemmArgs &g, cudaStream_t st);
+int num_sms();
+
+// ---- decode (decode.cu): small T, only the chosen experts' weights are read
+int launch_dec_router(const moe_shape_t &s, const uint16_t *x, const uint16_t *Wg,
+                      const float *bias, float *logits, cudaStream_t st);
+int launch_dec_w13(const moe_shape_t &s, const uint16_t *x, const int32_t *topk_idx,
+                   const uint16_t *W13, const uint16_t *W13s, uint16_t *Hdec, uint32_t *status,
+                   cudaStream_t st);
+int launch_dec_w2(const moe_shape_t &s, const int32_t *topk_idx, const float *topk_w,
+                  const uint16_t *W2, const uint16_t *W2s, const uint16_t *Hdec, float *out,
+                  uint32_t *status, cudaStream_t st);
+
+} // namespace moe

@@ -1,0 +1,605 @@
+// moe_api.cu -- the extern "C" entry points of libmoe.so (declared in moe.h):
+// argument validation, workspace carving, and the launch sequences.
+#include <atomic>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "internal.h"
+
+namespace moe {
+
+// ---------------------------------------------------------------- instrumentation
+static std::atomic<uint64_t> g_launches{0};
+void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+namespace {
+struct StageRecord {
+    int stage;
+    cudaEvent_t a, b;
+};
+struct Profiler {
+    std::mutex mu;
+    bool on = false;
+    std::vector<cudaEvent_t> pool;   // created once, reused
+    size_t next = 0;
+    std::vector<StageRecord> recs;
+};
+Profiler &prof()
+{
+    static Profiler p;
+    return p;
+}
+cudaEvent_t take_event(Profiler &P)
+{
+    if (P.next == P.pool.size()) {
+        cudaEvent_t e;
+        if (cudaEventCreate(&e) != cudaSuccess)
+            return nullptr;
+        P.pool.push_back(e);
+    }
+    return P.pool[P.next++];
+}
+} // namespace
+
+// Brackets one stage of moe_forward with two events when profiling is on.
+struct StageMark {
+    int stage;
+    cudaStream_t st;
+    cudaEvent_t a = nullptr;
+    StageMark(int stage_, cudaStream_t st_) : stage(stage_), st(st_)
+    {
+        Profiler &P = prof();
+        std::lock_guard<std::mutex> g(P.mu);
+        if (P.on && (a = take_event(P)))
+            cudaEventRecord(a, st);
+    }
+    ~StageMark()
+    {
+        if (!a)
+            return;
+        Profiler &P = prof();
+        std::lock_guard<std::mutex> g(P.mu);
+        cudaEvent_t b = take_event(P);
+        if (b && cudaEventRecord(b, st) == cudaSuccess)
+            P.recs.push_back({stage, a, b});
+    }
+};
+int launch_dec_router(const moe_shape_t &s, const uint16_t *x, const uint16_t *Wg,
+                      const float *bias, float *logits, cudaStream_t st);
+
+static bool dim_ok(int v) { return v >= 128 && v <= 32768 && v % 128 == 0; }
+
+static int check_shape(const moe_shape_t *s)
+{
+    if (!s)
+        return MOE_ERR_INVALID_ARG;
+    if (s->T < 0 || s->T > (1 << 24))
+        return MOE_ERR_INVALID_ARG;
+    if (s->E < 1 || s->E > MOE_MAX_E)
+        return MOE_ERR_INVALID_ARG;
+    if (s->k < 1 || s->k > s->E || s->k > MOE_MAX_K)
+        return MOE_ERR_INVALID_ARG;
+    if (!dim_ok(s->d) || !dim_ok(s->d_ff))
+        return MOE_ERR_INVALID_ARG;
+    if (s->d_ff_shared != 0 && !dim_ok(s->d_ff_shared))
+        return MOE_ERR_INVALID_ARG;
+    return MOE_OK;
+}
+
+static bool al16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+WsLayout ws_layout(const moe_shape_t &s)
+{
+    WsLayout L;
+    std::memset(&L, 0, sizeof L);
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t o = off;
+        off += (bytes + 255) & ~static_cast<size_t>(255);
+        return o;
+    };
+    const size_t T = s.T, k = s.k, E = s.E, N = T * k;
+    L.nchunks = (int)((T + kChunkTokens - 1) / kChunkTokens);
+    L.max_mt = (int)((N + kBlockM - 1) / kBlockM + E);
+    L.logits = take(T * E * 4);
+    L.topk_idx = take(N * 4);
+    L.topk_w = take(N * 4);
+    L.counts = take(E * 4);
+    L.offsets = take((E + 1) * 4);
+    L.n_kept = take(4);
+    L.counter = take(4);
+    L.num_mt = take(4);
+    L.chunk_counts = take((size_t)L.nchunks * E * 4);
+    L.rank_local = take(N * 4);
+    L.slot_pos = take(N * 4);
+    L.perm_token = take(N * 4);
+    L.mt_row0 = take((size_t)L.max_mt * 4);
+    L.mt_group = take((size_t)L.max_mt * 4);
+    L.x_perm = take(N * s.d * 2);
+    L.H = take(N * s.d_ff * 2);
+    L.H_shared = take(s.d_ff_shared ? T * s.d_ff_shared * 2 : 0);
+    L.Y = take((s.flags & MOE_FLAG_DETERMINISTIC) ? N * s.d * 4 : 0);
+    const size_t Td = T < (size_t)MOE_DECODE_MAX_T ? T : (size_t)MOE_DECODE_MAX_T;
+    L.dec_H = take((Td * k * s.d_ff + Td * s.d_ff_shared) * 2);
+    L.x_stage = take((s.flags & MOE_FLAG_HOST_IO) ? T * s.d * 2 : 0);
+    L.out_stage = take((s.flags & MOE_FLAG_HOST_IO) ? T * s.d * 4 : 0);
+    L.total = off;
+    return L;
+}
+
+template <class P>
+static P *at(void *ws, size_t off)
+{
+    return reinterpret_cast<P *>(static_cast<char *>(ws) + off);
+}
+
+static int check_ws(const moe_shape_t &s, void *ws, size_t ws_bytes, WsLayout &L)
+{
+    L = ws_layout(s);
+    if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0 || ws_bytes < L.total)
+        return MOE_ERR_WORKSPACE;
+    return MOE_OK;
+}
+
+static int run_gemm(const moe_shape_t &s, const GemmArgs &g, cudaStream_t st)
+{
+    return (s.flags & MOE_FLAG_SIMT_FFN) ? launch_gemm_simt(g, st) : launch_gemm_tc(g, st);
+}
+
+static GemmArgs gemm_base()
+{
+    GemmArgs g;
+    std::memset(&g, 0, sizeof g);
+    return g;
+}
+
+// Routed grouped GEMMs: SwiGLU into H, then w2 with the chosen epilogue.
+static int expert_ffn_core(const moe_shape_t &s, const WsLayout &L, void *ws,
+                           const uint16_t *x_perm, const int32_t *offsets, const uint16_t *W13,
+                           const uint16_t *W2, const int32_t *perm_token, const int32_t *slot_pos,
+                           const float *topk_w, float *y_perm, float *out, uint32_t *status,
+                           cudaStream_t st)
+{
+    const long long N = (long long)s.T * s.k;
+    uint16_t *H = at<uint16_t>(ws, L.H);
+    GemmArgs g = gemm_base();
+    g.mode = EPI_SWIGLU;
+    g.A = x_perm;
+    g.a_rows = N;
+    g.B = W13;
+    g.b_rows_total = (long long)s.E * 2 * s.d_ff;
+    g.K = s.d;
+    g.N = 2 * s.d_ff;
+    g.b_rows_per_group = 2 * s.d_ff;
+    g.mt_row0 = at<int32_t>(ws, L.mt_row0);
+    g.mt_group = at<int32_t>(ws, L.mt_group);
+    g.num_mt_dev = at<int32_t>(ws, L.num_mt);
+    g.max_mt = L.max_mt;
+    g.seg_offsets = offsets;
+    g.out = H;
+    g.ldo = s.d_ff;
+    g.status = status;
+    int rc;
+    {
+        StageMark m(MOE_STAGE_W13, st);
+        rc = run_gemm(s, g, st);
+    }
+    if (rc)
+        return rc;
+    g.A = H;
+    g.B = W2;
+    g.b_rows_total = (long long)s.E * s.d;
+    g.K = s.d_ff;
+    g.N = s.d;
+    g.b_rows_per_group = s.d;
+    g.ldo = s.d;
+    if (y_perm) {
+        g.mode = EPI_STORE_F32;
+        g.out = y_perm;
+    } else {
+        g.mode = EPI_COMBINE;
+        g.out = out;
+        g.perm_token = perm_token;
+        g.slot_pos = slot_pos;
+        g.topk_w = topk_w;
+        g.k = s.k;
+    }
+    StageMark m(MOE_STAGE_W2, st);
+    return run_gemm(s, g, st);
+}
+
+// Shared expert on all T tokens: out = W2s (silu(W1s x) * W3s x), plain store.
+static int shared_expert(const moe_shape_t &s, const WsLayout &L, void *ws, const uint16_t *x,
+                         const uint16_t *W13s, const uint16_t *W2s, float *out, uint32_t *status,
+                         cudaStream_t st)
+{
+    uint16_t *Hs = at<uint16_t>(ws, L.H_shared);
+    const int mt = (s.T + kBlockM - 1) / kBlockM;
+    GemmArgs g = gemm_base();
+    g.mode = EPI_SWIGLU;
+    g.A = x;
+    g.a_rows = s.T;
+    g.B = W13s;
+    g.b_rows_total = 2LL * s.d_ff_shared;
+    g.K = s.d;
+    g.N = 2 * s.d_ff_shared;
+    g.b_rows_per_group = 2 * s.d_ff_shared;
+    g.num_mt_host = mt;
+    g.max_mt = mt;
+    g.rows_valid = s.T;
+    g.out = Hs;
+    g.ldo = s.d_ff_shared;
+    g.status = status;
+    int rc = run_gemm(s, g, st);
+    if (rc)
+        return rc;
+    g.mode = EPI_STORE_F32;
+    g.A = Hs;
+    g.B = W2s;
+    g.b_rows_total = s.d;
+    g.K = s.d_ff_shared;
+    g.N = s.d;
+    g.b_rows_per_group = s.d;
+    g.out = out;
+    g.ldo = s.d;
+    return run_gemm(s, g, st);
+}
+
+static int router(const moe_shape_t &s, const uint16_t *x, const uint16_t *Wg, const float *bias,
+                  float *logits, uint32_t *status, cudaStream_t st)
+{
+    if (s.T <= MOE_DECODE_MAX_T)
+        return launch_dec_router(s, x, Wg, bias, logits, st);
+    if (s.flags & MOE_FLAG_SIMT_FFN)
+        return launch_router_simt(s, x, Wg, bias, logits, st);
+    GemmArgs g = gemm_base();
+    g.mode = EPI_ROUTER;
+    g.A = x;
+    g.a_rows = s.T;
+    g.B = Wg;
+    g.b_rows_total = s.E;
+    g.K = s.d;
+    g.N = s.E;
+    g.b_rows_per_group = 0;
+    g.num_mt_host = (s.T + kBlockM - 1) / kBlockM;
+    g.max_mt = g.num_mt_host;
+    g.rows_valid = s.T;
+    g.out = logits;
+    g.ldo = s.E;
+    g.bias = bias;
+    g.n_valid = s.E;
+    g.status = status;
+    return launch_gemm_tc(g, st);
+}
+
+static int forward_impl(const moe_shape_t &s, const WsLayout &L, void *ws, const uint16_t *x,
+                        const uint16_t *Wg, const float *bias, const uint16_t *W13,
+                        const uint16_t *W2, const uint16_t *W13s, const uint16_t *W2s,
+                        float *out, float *logits_out, int32_t *idx_out, uint32_t *status,
+                        cudaStream_t st)
+{
+    float *logits = logits_out ? logits_out : at<float>(ws, L.logits);
+    int32_t *idx = idx_out ? idx_out : at<int32_t>(ws, L.topk_idx);
+    float *w = at<float>(ws, L.topk_w);
+    const bool force_dec = (s.flags & MOE_FLAG_FORCE_DECODE) != 0;
+    const bool force_pre = (s.flags & MOE_FLAG_FORCE_PREFILL) != 0;
+    if (force_dec && s.T > MOE_DECODE_MAX_T)
+        return MOE_ERR_UNSUPPORTED;
+    const bool decode = force_dec || (!force_pre && s.T <= MOE_DECODE_DEFAULT_T);
+    int rc;
+    {
+        StageMark m(MOE_STAGE_ROUTER, st);
+        rc = router(s, x, Wg, bias, logits, status, st);
+    }
+    if (rc)
+        return rc;
+    int32_t *counter = at<int32_t>(ws, L.counter);
+    {
+        StageMark m(MOE_STAGE_TOPK, st);
+        rc = launch_topk(s, logits, idx, w, counter, status, st);
+    }
+    if (rc)
+        return rc;
+    if (decode) {
+        uint16_t *Hdec = at<uint16_t>(ws, L.dec_H);
+        {
+            StageMark m(MOE_STAGE_DEC_W13, st);
+            rc = launch_dec_w13(s, x, idx, W13, W13s, Hdec, status, st);
+        }
+        if (rc)
+            return rc;
+        StageMark m(MOE_STAGE_DEC_W2, st);
+        return launch_dec_w2(s, idx, w, W2, W2s, Hdec, out, status, st);
+    }
+
+    const bool det = (s.flags & MOE_FLAG_DETERMINISTIC) != 0;
+    const bool shared = s.d_ff_shared > 0;
+    int32_t *counts = at<int32_t>(ws, L.counts);
+    int32_t *offsets = at<int32_t>(ws, L.offsets);
+    int32_t *chunk = at<int32_t>(ws, L.chunk_counts);
+    int32_t *rank = at<int32_t>(ws, L.rank_local);
+    int32_t *slot_pos = at<int32_t>(ws, L.slot_pos);
+    int32_t *perm_token = at<int32_t>(ws, L.perm_token);
+    uint16_t *x_perm = at<uint16_t>(ws, L.x_perm);
+    {
+        StageMark m(MOE_STAGE_HIST, st);
+        rc = launch_hist_scan(s, idx, chunk, rank, counter, counts, offsets,
+                              at<int32_t>(ws, L.n_kept), at<int32_t>(ws, L.mt_row0),
+                              at<int32_t>(ws, L.mt_group), at<int32_t>(ws, L.num_mt), status, st);
+    }
+    if (rc)
+        return rc;
+    {
+        StageMark m(MOE_STAGE_PERMUTE, st);
+        rc = launch_permute(s, idx, chunk, rank, offsets, x, slot_pos, perm_token, x_perm,
+                            (!shared && !det) ? out : nullptr, st);
+    }
+    if (rc)
+        return rc;
+    if (shared) {
+        StageMark m(MOE_STAGE_SHARED, st);
+        rc = shared_expert(s, L, ws, x, W13s, W2s, out, status, st);
+        if (rc)
+            return rc;
+    }
+    float *Y = det ? at<float>(ws, L.Y) : nullptr;
+    rc = expert_ffn_core(s, L, ws, x_perm, offsets, W13, W2, perm_token, slot_pos, w, Y, out,
+                         status, st);
+    if (rc)
+        return rc;
+    if (det) {
+        StageMark m(MOE_STAGE_COMBINE, st);
+        rc = launch_combine(s, Y, slot_pos, w, shared ? out : nullptr, out, st);
+    }
+    return rc;
+}
+
+} // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+const char *moe_status_string(int code)
+{
+    switch (code) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "unsupported";
+    case MOE_ERR_WORKSPACE: return "workspace too small or misaligned";
+    case MOE_ERR_CUDA: return "CUDA runtime error";
+    case MOE_ERR_NONFINITE: return "non-finite router logit";
+    case MOE_ERR_BAD_EXPERT: return "expert id out of range or repeated";
+    case MOE_ERR_TIMEOUT: return "device pipeline wait timed out";
+    default: return "unknown status";
+    }
+}
+
+uint64_t moe_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
+
+int moe_profile_enable(int on)
+{
+    Profiler &P = prof();
+    std::lock_guard<std::mutex> g(P.mu);
+    P.on = on != 0;
+    return MOE_OK;
+}
+
+int moe_profile_read(double *ms, int64_t *calls, int n)
+{
+    if (n < 0 || n > MOE_NUM_STAGES)
+        return MOE_ERR_INVALID_ARG;
+    Profiler &P = prof();
+    std::lock_guard<std::mutex> g(P.mu);
+    for (int i = 0; i < n; ++i) {
+        if (ms)
+            ms[i] = 0.0;
+        if (calls)
+            calls[i] = 0;
+    }
+    int rc = MOE_OK;
+    for (const StageRecord &r : P.recs) {
+        float t = 0.f;
+        if (cudaEventSynchronize(r.b) != cudaSuccess || cudaEventElapsedTime(&t, r.a, r.b) != cudaSuccess) {
+            rc = MOE_ERR_CUDA;
+            continue;
+        }
+        if (r.stage < n) {
+            if (ms)
+                ms[r.stage] += t;
+            if (calls)
+                calls[r.stage] += 1;
+        }
+    }
+    P.recs.clear();
+    P.next = 0;
+    return rc;
+}
+
+int moe_workspace_size(const moe_shape_t *shape, size_t *bytes)
+{
+    int rc = check_shape(shape);
+    if (rc)
+        return rc;
+    if (!bytes)
+        return MOE_ERR_INVALID_ARG;
+    *bytes = ws_layout(*shape).total;
+    return MOE_OK;
+}
+
+int moe_pack_w13(const moe_shape_t *shape, const moe_bf16_t *W1, const moe_bf16_t *W3,
+                 moe_bf16_t *W13, moe_stream_t stream)
+{
+    int rc = check_shape(shape);
+    if (rc)
+        return rc;
+    if (!W1 || !W3 || !W13 || !al16(W1) || !al16(W3) || !al16(W13))
+        return MOE_ERR_INVALID_ARG;
+    return launch_pack_w13(shape->E, shape->d_ff, shape->d, W1, W3, W13,
+                           reinterpret_cast<cudaStream_t>(stream));
+}
+
+int moe_route(const moe_shape_t *shape, const moe_bf16_t *x, const moe_bf16_t *Wg,
+              const float *bias, float *logits, int32_t *topk_idx, float *topk_w,
+              uint32_t *status, void *ws, size_t ws_bytes, moe_stream_t stream)
+{
+    int rc = check_shape(shape);
+    if (rc)
+        return rc;
+    const moe_shape_t &s = *shape;
+    if (!logits || !topk_idx || !topk_w || (x && !Wg) || (x && (!al16(x) || !al16(Wg))))
+        return MOE_ERR_INVALID_ARG;
+    WsLayout L;
+    if ((rc = check_ws(s, ws, ws_bytes, L)))
+        return rc;
+    if (s.T == 0)
+        return MOE_OK;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (x && (rc = router(s, x, Wg, bias, logits, status, st)))
+        return rc;
+    return launch_topk(s, logits, topk_idx, topk_w, nullptr, status, st);
+}
+
+int moe_permute(const moe_shape_t *shape, const int32_t *topk_idx, const moe_bf16_t *x,
+                int32_t *expert_counts, int32_t *expert_offsets, int32_t *slot_pos,
+                int32_t *perm_token, moe_bf16_t *x_perm, int32_t *n_kept, uint32_t *status,
+                void *ws, size_t ws_bytes, moe_stream_t stream)
+{
+    int rc = check_shape(shape);
+    if (rc)
+        return rc;
+    const moe_shape_t &s = *shape;
+    if (!topk_idx || !expert_counts || !expert_offsets || !slot_pos || !perm_token ||
+        (x && !x_perm) || (x && (!al16(x) || !al16(x_perm))))
+        return MOE_ERR_INVALID_ARG;
+    WsLayout L;
+    if ((rc = check_ws(s, ws, ws_bytes, L)))
+        return rc;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (s.T == 0) {
+        // offsets of an empty batch: all zero (a no-op kernel-free answer)
+        if (cudaMemsetAsync(expert_counts, 0, sizeof(int32_t) * s.E, st) != cudaSuccess ||
+            cudaMemsetAsync(expert_offsets, 0, sizeof(int32_t) * (s.E + 1), st) != cudaSuccess ||
+            (n_kept && cudaMemsetAsync(n_kept, 0, sizeof(int32_t), st) != cudaSuccess))
+            return MOE_ERR_CUDA;
+        return MOE_OK;
+    }
+    int32_t *counter = at<int32_t>(ws, L.counter);
+    if (cudaMemsetAsync(counter, 0, sizeof(int32_t), st) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    int32_t *chunk = at<int32_t>(ws, L.chunk_counts);
+    int32_t *rank = at<int32_t>(ws, L.rank_local);
+    rc = launch_hist_scan(s, topk_idx, chunk, rank, counter, expert_counts, expert_offsets,
+                          n_kept ? n_kept : at<int32_t>(ws, L.n_kept), at<int32_t>(ws, L.mt_row0),
+                          at<int32_t>(ws, L.mt_group), at<int32_t>(ws, L.num_mt), status, st);
+    if (rc)
+        return rc;
+    return launch_permute(s, topk_idx, chunk, rank, expert_offsets, x, slot_pos, perm_token,
+                          x ? x_perm : nullptr, nullptr, st);
+}
+
+int moe_expert_ffn(const moe_shape_t *shape, const moe_bf16_t *x_perm,
+                   const int32_t *expert_offsets, const moe_bf16_t *W13, const moe_bf16_t *W2,
+                   const int32_t *perm_token, const int32_t *slot_pos, const float *topk_w,
+                   float *y_perm, float *out, uint32_t *status, void *ws, size_t ws_bytes,
+                   moe_stream_t stream)
+{
+    int rc = check_shape(shape);
+    if (rc)
+        return rc;
+    const moe_shape_t &s = *shape;
+    if (!x_perm || !expert_offsets || !W13 || !W2 || !al16(x_perm) || !al16(W13) || !al16(W2))
+        return MOE_ERR_INVALID_ARG;
+    if (y_perm ? !al16(y_perm) : (!out || !perm_token || !slot_pos || !topk_w || !al16(out)))
+        return MOE_ERR_INVALID_ARG;
+    WsLayout L;
+    if ((rc = check_ws(s, ws, ws_bytes, L)))
+        return rc;
+    if (s.T == 0)
+        return MOE_OK;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    rc = launch_tiles_from_offsets(s, expert_offsets, at<int32_t>(ws, L.mt_row0),
+                                   at<int32_t>(ws, L.mt_group), at<int32_t>(ws, L.num_mt), st);
+    if (rc)
+        return rc;
+    return expert_ffn_core(s, L, ws, x_perm, expert_offsets, W13, W2, perm_token, slot_pos, topk_w,
+                           y_perm, out, status, st);
+}
+
+int moe_combine(const moe_shape_t *shape, const float *y_perm, const int32_t *slot_pos,
+                const float *topk_w, const float *shared_out, float *out, moe_stream_t stream)
+{
+    int rc = check_shape(shape);
+    if (rc)
+        return rc;
+    if (!y_perm || !slot_pos || !topk_w || !out || !al16(y_perm) || !al16(out) ||
+        (shared_out && !al16(shared_out)))
+        return MOE_ERR_INVALID_ARG;
+    return launch_combine(*shape, y_perm, slot_pos, topk_w, shared_out, out,
+                          reinterpret_cast<cudaStream_t>(stream));
+}
+
+int moe_forward(const moe_shape_t *shape, const moe_bf16_t *x, const moe_bf16_t *Wg,
+                const float *bias, const moe_bf16_t *W13, const moe_bf16_t *W2,
+                const moe_bf16_t *W13_shared, const moe_bf16_t *W2_shared, float *out,
+                float *logits_out, int32_t *topk_idx_out, uint32_t *status, void *ws,
+                size_t ws_bytes, moe_stream_t stream)
+{
+    int rc = check_shape(shape);
+    if (rc)
+        return rc;
+    const moe_shape_t &s = *shape;
+    if (!x || !Wg || !W13 || !W2 || !out || !al16(x) || !al16(Wg) || !al16(W13) || !al16(W2) ||
+        !al16(out))
+        return MOE_ERR_INVALID_ARG;
+    if (s.d_ff_shared > 0 &&
+        (!W13_shared || !W2_shared || !al16(W13_shared) || !al16(W2_shared)))
+        return MOE_ERR_INVALID_ARG;
+    WsLayout L;
+    if ((rc = check_ws(s, ws, ws_bytes, L)))
+        return rc;
+    if (s.T == 0)
+        return MOE_OK;
+    return forward_impl(s, L, ws, x, Wg, bias, W13, W2, W13_shared, W2_shared, out, logits_out,
+                        topk_idx_out, status, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int moe_forward_host(const moe_shape_t *shape, const moe_bf16_t *x_host, const moe_bf16_t *Wg,
+                     const float *bias, const moe_bf16_t *W13, const moe_bf16_t *W2,
+                     const moe_bf16_t *W13_shared, const moe_bf16_t *W2_shared, float *out_host,
+                     uint32_t *status, void *ws, size_t ws_bytes, moe_stream_t stream)
+{
+    int rc = check_shape(shape);
+    if (rc)
+        return rc;
+    const moe_shape_t &s = *shape;
+    if (!(s.flags & MOE_FLAG_HOST_IO))
+        return MOE_ERR_INVALID_ARG;
+    if (!x_host || !out_host || !Wg || !W13 || !W2 || !al16(Wg) || !al16(W13) || !al16(W2))
+        return MOE_ERR_INVALID_ARG;
+    if (s.d_ff_shared > 0 &&
+        (!W13_shared || !W2_shared || !al16(W13_shared) || !al16(W2_shared)))
+        return MOE_ERR_INVALID_ARG;
+    WsLayout L;
+    if ((rc = check_ws(s, ws, ws_bytes, L)))
+        return rc;
+    if (s.T == 0)
+        return MOE_OK;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    uint16_t *xd = at<uint16_t>(ws, L.x_stage);
+    float *od = at<float>(ws, L.out_stage);
+    const size_t xb = (size_t)s.T * s.d * 2, ob = (size_t)s.T * s.d * 4;
+    if (cudaMemcpyAsync(xd, x_host, xb, cudaMemcpyHostToDevice, st) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    rc = forward_impl(s, L, ws, xd, Wg, bias, W13, W2, W13_shared, W2_shared, od, nullptr, nullptr,
+                      status, st);
+    if (rc)
+        return rc;
+    if (cudaMemcpyAsync(out_host, od, ob, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    return MOE_OK;
+}
+
+} // extern "C"

@@ -1,0 +1,284 @@
+"""Thin Python binding of libmoe.so (the C ABI declared in include/moe.h).
+
+Argument marshalling only: every function here checks tensor dtypes and
+devices, turns torch tensors into raw device pointers and the current torch
+stream into a cudaStream_t, and calls the entry point of the same name. All
+arithmetic runs in the library's CUDA kernels. There is no fallback: if the
+library is missing or a call fails, an exception is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoe.so")
+HEADER = os.path.join(os.path.dirname(_HERE), "include", "moe.h")
+
+MOE_OK = 0
+MOE_ERR_INVALID_ARG = 1
+MOE_ERR_UNSUPPORTED = 2
+MOE_ERR_WORKSPACE = 3
+MOE_ERR_CUDA = 4
+MOE_ERR_NONFINITE = 5
+MOE_ERR_BAD_EXPERT = 6
+MOE_ERR_TIMEOUT = 7
+
+MOE_FLAG_DETERMINISTIC = 1 << 0
+MOE_FLAG_FORCE_PREFILL = 1 << 1
+MOE_FLAG_FORCE_DECODE = 1 << 2
+MOE_FLAG_SIMT_FFN = 1 << 3
+MOE_FLAG_HOST_IO = 1 << 4
+
+MOE_MAX_E = 256
+MOE_MAX_K = 16
+MOE_DECODE_MAX_T = 16
+
+
+class MoeError(RuntimeError):
+    def __init__(self, fn: str, code: int, msg: str):
+        super().__init__(f"{fn} failed: {code} ({msg})")
+        self.code = code
+
+
+class moe_shape_t(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int32), ("d", ctypes.c_int32), ("d_ff", ctypes.c_int32),
+                ("E", ctypes.c_int32), ("k", ctypes.c_int32), ("capacity", ctypes.c_int32),
+                ("d_ff_shared", ctypes.c_int32), ("flags", ctypes.c_int32)]
+
+    def __repr__(self):
+        return "moe_shape_t(" + ", ".join(f"{n}={getattr(self, n)}" for n, _ in self._fields_) + ")"
+
+
+def make_shape(T, d, d_ff, E, k, capacity=0, d_ff_shared=0, flags=0) -> moe_shape_t:
+    return moe_shape_t(T, d, d_ff, E, k, capacity, d_ff_shared, flags)
+
+
+def shape_of(workload, flags=0, T=None) -> moe_shape_t:
+    w = workload
+    return make_shape(w.T if T is None else T, w.d, w.d_ff, w.E, w.k, w.capacity, w.d_ff_shared,
+                      flags)
+
+
+_lib = None
+_P = ctypes.c_void_p
+_SZ = ctypes.c_size_t
+_SHP = ctypes.POINTER(moe_shape_t)
+
+_SIGS = {
+    "moe_status_string": ([ctypes.c_int], ctypes.c_char_p),
+    "moe_workspace_size": ([_SHP, ctypes.POINTER(_SZ)], ctypes.c_int),
+    "moe_pack_w13": ([_SHP, _P, _P, _P, _P], ctypes.c_int),
+    "moe_route": ([_SHP, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P], ctypes.c_int),
+    "moe_permute": ([_SHP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P], ctypes.c_int),
+    "moe_expert_ffn": ([_SHP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P], ctypes.c_int),
+    "moe_combine": ([_SHP, _P, _P, _P, _P, _P, _P], ctypes.c_int),
+    "moe_forward": ([_SHP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P], ctypes.c_int),
+    "moe_forward_host": ([_SHP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P], ctypes.c_int),
+    "moe_kernel_launches": ([], ctypes.c_uint64),
+    "moe_profile_enable": ([ctypes.c_int], ctypes.c_int),
+    "moe_profile_read": ([_P, _P, ctypes.c_int], ctypes.c_int),
+}
+
+STAGES = ["router", "topk", "hist", "permute", "shared", "w13", "w2", "combine", "dec_w13",
+          "dec_w2"]
+
+
+def header_entry_points() -> list[str]:
+    """Names of the entry points that include/moe.h declares."""
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"MOE_API\s+[\w\s\*]*?\b(moe_\w+)\s*\(", text)))
+
+
+def lib() -> ctypes.CDLL:
+    """Load libmoe.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libmoe.so not found at {LIB_PATH}: build it with "
+                               "`python -m sparse_mixture_experts_17_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (args, res) in _SIGS.items():
+            f = getattr(L, name)
+            f.argtypes = args
+            f.restype = res
+        _lib = L
+    return _lib
+
+
+def status_string(code: int) -> str:
+    return lib().moe_status_string(code).decode()
+
+
+def _check(fn, rc):
+    if rc != MOE_OK:
+        raise MoeError(fn, rc, status_string(rc))
+
+
+def _ptr(t, dtype=None, name="tensor"):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name}: expected a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name}: must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+    return t.data_ptr()
+
+
+def _host_ptr(t, dtype, name):
+    if t.is_cuda or not t.is_contiguous() or t.dtype != dtype:
+        raise ValueError(f"{name}: must be a contiguous host tensor of {dtype}")
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+BF16, F32, I32, U32 = torch.bfloat16, torch.float32, torch.int32, torch.int32
+
+
+# ---------------------------------------------------------------- entry points
+
+def moe_workspace_size(shape: moe_shape_t) -> int:
+    n = _SZ(0)
+    _check("moe_workspace_size", lib().moe_workspace_size(ctypes.byref(shape), ctypes.byref(n)))
+    return n.value
+
+
+def alloc_workspace(shape: moe_shape_t, device="cuda") -> torch.Tensor:
+    """A workspace of the right size (torch allocates; the library never does)."""
+    return torch.empty(max(moe_workspace_size(shape), 256), dtype=torch.uint8, device=device)
+
+
+def moe_pack_w13(shape, W1, W3, W13=None, stream=None):
+    if W13 is None:
+        W13 = torch.empty(shape.E, 2 * shape.d_ff, shape.d, dtype=BF16, device=W1.device)
+    _check("moe_pack_w13", lib().moe_pack_w13(ctypes.byref(shape), _ptr(W1, BF16, "W1"),
+                                              _ptr(W3, BF16, "W3"), _ptr(W13, BF16, "W13"),
+                                              _stream(stream)))
+    return W13
+
+
+def moe_route(shape, x, Wg, bias, logits, topk_idx, topk_w, status, ws, stream=None):
+    _check("moe_route", lib().moe_route(
+        ctypes.byref(shape), _ptr(x, BF16, "x"), _ptr(Wg, BF16, "Wg"), _ptr(bias, F32, "bias"),
+        _ptr(logits, F32, "logits"), _ptr(topk_idx, I32, "topk_idx"), _ptr(topk_w, F32, "topk_w"),
+        _ptr(status, U32, "status"), _ptr(ws, name="ws"), ws.numel() if ws is not None else 0,
+        _stream(stream)))
+
+
+def moe_permute(shape, topk_idx, x, expert_counts, expert_offsets, slot_pos, perm_token, x_perm,
+                n_kept, status, ws, stream=None):
+    _check("moe_permute", lib().moe_permute(
+        ctypes.byref(shape), _ptr(topk_idx, I32, "topk_idx"), _ptr(x, BF16, "x"),
+        _ptr(expert_counts, I32, "expert_counts"), _ptr(expert_offsets, I32, "expert_offsets"),
+        _ptr(slot_pos, I32, "slot_pos"), _ptr(perm_token, I32, "perm_token"),
+        _ptr(x_perm, BF16, "x_perm"), _ptr(n_kept, I32, "n_kept"), _ptr(status, U32, "status"),
+        _ptr(ws, name="ws"), ws.numel(), _stream(stream)))
+
+
+def moe_expert_ffn(shape, x_perm, expert_offsets, W13, W2, perm_token, slot_pos, topk_w, y_perm,
+                   out, status, ws, stream=None):
+    _check("moe_expert_ffn", lib().moe_expert_ffn(
+        ctypes.byref(shape), _ptr(x_perm, BF16, "x_perm"),
+        _ptr(expert_offsets, I32, "expert_offsets"), _ptr(W13, BF16, "W13"), _ptr(W2, BF16, "W2"),
+        _ptr(perm_token, I32, "perm_token"), _ptr(slot_pos, I32, "slot_pos"),
+        _ptr(topk_w, F32, "topk_w"), _ptr(y_perm, F32, "y_perm"), _ptr(out, F32, "out"),
+        _ptr(status, U32, "status"), _ptr(ws, name="ws"), ws.numel(), _stream(stream)))
+
+
+def moe_combine(shape, y_perm, slot_pos, topk_w, shared_out, out, stream=None):
+    _check("moe_combine", lib().moe_combine(
+        ctypes.byref(shape), _ptr(y_perm, F32, "y_perm"), _ptr(slot_pos, I32, "slot_pos"),
+        _ptr(topk_w, F32, "topk_w"), _ptr(shared_out, F32, "shared_out"), _ptr(out, F32, "out"),
+        _stream(stream)))
+
+
+def moe_forward(shape, x, Wg, bias, W13, W2, W13_shared, W2_shared, out, logits_out=None,
+                topk_idx_out=None, status=None, ws=None, stream=None):
+    _check("moe_forward", lib().moe_forward(
+        ctypes.byref(shape), _ptr(x, BF16, "x"), _ptr(Wg, BF16, "Wg"), _ptr(bias, F32, "bias"),
+        _ptr(W13, BF16, "W13"), _ptr(W2, BF16, "W2"), _ptr(W13_shared, BF16, "W13_shared"),
+        _ptr(W2_shared, BF16, "W2_shared"), _ptr(out, F32, "out"),
+        _ptr(logits_out, F32, "logits_out"), _ptr(topk_idx_out, I32, "topk_idx_out"),
+        _ptr(status, U32, "status"), _ptr(ws, name="ws"), ws.numel() if ws is not None else 0,
+        _stream(stream)))
+
+
+def moe_forward_host(shape, x_host, Wg, bias, W13, W2, W13_shared, W2_shared, out_host, status,
+                     ws, stream=None):
+    _check("moe_forward_host", lib().moe_forward_host(
+        ctypes.byref(shape), _host_ptr(x_host, BF16, "x_host"), _ptr(Wg, BF16, "Wg"),
+        _ptr(bias, F32, "bias"), _ptr(W13, BF16, "W13"), _ptr(W2, BF16, "W2"),
+        _ptr(W13_shared, BF16, "W13_shared"), _ptr(W2_shared, BF16, "W2_shared"),
+        _host_ptr(out_host, F32, "out_host"), _ptr(status, U32, "status"), _ptr(ws, name="ws"),
+        ws.numel(), _stream(stream)))
+
+
+# ---------------------------------------------------------------- convenience
+
+class MoeLayer:
+    """Device-resident weights (packed once) plus a workspace; forward() runs
+    the whole layer through moe_forward on the current stream."""
+
+    def __init__(self, inp: dict, flags: int = 0, T_max: int | None = None):
+        w = inp["workload"]
+        self.workload = w
+        self.flags = flags
+        dev = inp["x"].device
+        self.Wg = inp["wg"].contiguous()
+        self.bias = None if inp.get("bias") is None else inp["bias"].to(dev, torch.float32).contiguous()
+        s = shape_of(w, flags)
+        self.W13 = moe_pack_w13(s, inp["W1"].contiguous(), inp["W3"].contiguous())
+        self.W2 = inp["W2"].contiguous()
+        self.W13s = self.W2s = None
+        if w.d_ff_shared:
+            ss = make_shape(w.T, w.d, w.d_ff_shared, 1, 1)
+            self.W13s = moe_pack_w13(ss, inp["W1s"].contiguous()[None], inp["W3s"].contiguous()[None])[0]
+            self.W2s = inp["W2s"].contiguous()
+        self.T_max = T_max or w.T
+        self.ws = alloc_workspace(shape_of(w, flags, T=self.T_max), dev)
+        self.status = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def shape(self, T, flags=None):
+        return shape_of(self.workload, self.flags if flags is None else flags, T=T)
+
+    def forward(self, x, out=None, logits_out=None, topk_idx_out=None, flags=None, stream=None):
+        T = x.shape[0]
+        if T > self.T_max:
+            raise ValueError("T exceeds the workspace's T_max")
+        if out is None:
+            out = torch.empty(T, self.workload.d, dtype=torch.float32, device=x.device)
+        moe_forward(self.shape(T, flags), x, self.Wg, self.bias, self.W13, self.W2, self.W13s,
+                    self.W2s, out, logits_out, topk_idx_out, self.status, self.ws, stream)
+        return out
+
+
+# ---------------------------------------------------------------- instrumentation
+
+def moe_kernel_launches() -> int:
+    return int(lib().moe_kernel_launches())
+
+
+def moe_profile_enable(on: bool = True):
+    _check("moe_profile_enable", lib().moe_profile_enable(int(bool(on))))
+
+
+def moe_profile_read() -> dict:
+    """{stage: (total ms, calls)} since the last read (waits for the events)."""
+    import numpy as np
+    n = len(STAGES)
+    ms = np.zeros(n, np.float64)
+    calls = np.zeros(n, np.int64)
+    _check("moe_profile_read", lib().moe_profile_read(ms.ctypes.data, calls.ctypes.data, n))
+    return {STAGES[i]: (float(ms[i]), int(calls[i])) for i in range(n) if calls[i]}
