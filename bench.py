@@ -221,6 +221,8 @@ def run_ours(a, world, rank, local):
     stream = torch.cuda.current_stream()
     peaks, peak_src = load_peaks()
     w = I.WORKLOADS[a.workload]
+    if a.tokens:
+        w = w.with_T(a.tokens)
     inp = I.make_inputs(w, dev, seed=0)
     layer = M.MoeLayer(inp)
     x = inp["x"]
@@ -250,68 +252,51 @@ def run_ours(a, world, rank, local):
     value = tokens_all / (step_ms_max / 1e3)
 
     flops, w13_flops, w2_flops = prefill_flops(w, n_kept)
-    w13_ms = stages["w13"][0] / stages["w13"][1]
-    w2_ms = stages["w2"][0] / stages["w2"][1]
     peak_t = peaks["bf16_tflops_sustained"]
-    ach = w13_flops / (w13_ms / 1e3) / 1e12
-    roofline = {"bound": "tensor", "kernel": "k_gemm_tc<256,SWIGLU> (grouped w1/w3 GEMM + SwiGLU)",
-                "achieved": round(ach, 1), "peak": peak_t, "unit": "TFLOP/s",
-                "frac": round(ach / peak_t, 4), "traffic": None,
-                "peak_source": f"{peak_src} bf16_tflops_sustained",
-                "frac_of_burst_peak": round(ach / peaks["bf16_tflops"], 4),
-                "frac_of_nominal_2250": round(ach / 2250.0, 4),
-                "algorithmic_flops_per_launch": w13_flops, "avg_launch_ms": round(w13_ms, 4)}
     stage_ms = {k: round(v[0] / v[1], 4) for k, v in stages.items()}
-    w2_tflops = w2_flops / (w2_ms / 1e3) / 1e12
+    decode_path = "dec_w13" in stages
+    extra = {}
+    if not decode_path:
+        w13_ms = stages["w13"][0] / stages["w13"][1]
+        w2_ms = stages["w2"][0] / stages["w2"][1]
+        ach = w13_flops / (w13_ms / 1e3) / 1e12
+        roofline = {"bound": "tensor", "kernel": "k_gemm_tc<256,EPI_SWIGLU> (grouped w1/w3 GEMM + SwiGLU)",
+                    "achieved": round(ach, 1), "peak": peak_t, "unit": "TFLOP/s",
+                    "frac": round(ach / peak_t, 4), "traffic": None,
+                    "peak_source": f"{peak_src} bf16_tflops_sustained",
+                    "frac_of_burst_peak": round(ach / peaks["bf16_tflops"], 4),
+                    "frac_of_nominal_2250": round(ach / 2250.0, 4),
+                    "algorithmic_flops_per_launch": w13_flops, "avg_launch_ms": round(w13_ms, 4)}
+        extra["w2_tflops"] = round(w2_flops / (w2_ms / 1e3) / 1e12, 1)
+        extra["active_tflops"] = round(flops / (step_ms_max / 1e3) / 1e12, 1)
+        extra["active_tflops_frac_measured_sustained"] = round(
+            flops / (step_ms_max / 1e3) / 1e12 / peak_t, 4)
+        extra["n_kept"] = n_kept
+    else:
+        idx_now = torch.empty(w.T, w.k, dtype=torch.int32, device=dev)
+        layer.forward(x, out=out, topk_idx_out=idx_now)
+        U, nbytes, w13_bytes, expert_bytes = decode_bytes(w, w.T, idx_now)
+        k13 = stages["dec_w13"][0] / stages["dec_w13"][1]
+        ach = w13_bytes / (k13 / 1e3) / 1e9
+        roofline = {"bound": "hbm", "kernel": "k_dec_w13 (chosen experts' w1/w3 rows + SwiGLU)",
+                    "achieved": round(ach, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                    "frac": round(ach / peaks["hbm_gbs"], 4), "traffic": None,
+                    "peak_source": f"{peak_src} hbm_gbs",
+                    "frac_of_nominal_8000": round(ach / 8000.0, 4),
+                    "algorithmic_bytes_per_launch": w13_bytes, "avg_launch_ms": round(k13, 4)}
+        extra["unique_experts"] = U
+        extra["hbm_GB_s_step"] = round(nbytes / (step_ms_max / 1e3) / 1e9, 1)
+        extra["hbm_frac_step_measured"] = round(nbytes / (step_ms_max / 1e3) / 1e9 / peaks["hbm_gbs"], 4)
 
     # ---- end to end through the C ABI with host buffers (H2D + D2H inside)
-    shape_h = M.shape_of(w, M.MOE_FLAG_HOST_IO)
-    ws_h = M.alloc_workspace(shape_h, dev)
-    x_h = x.cpu().pin_memory()
-    out_h = torch.empty(w.T, w.d, dtype=torch.float32).pin_memory()
-
-    def e2e_step():
-        M.moe_forward_host(shape_h, x_h, layer.Wg, layer.bias, layer.W13, layer.W2, layer.W13s,
-                           layer.W2s, out_h, layer.status, ws_h)
-    for _ in range(2):
-        e2e_step()
-    torch.cuda.synchronize()
-    barrier(world)
-    e2e_ms = time_loop(e2e_step, max(3, a.steps // 2), stream)
-    e2e_ms = max_over_ranks(e2e_ms, world, dev)
-    e2e = {"value": round(tokens_all / (e2e_ms / 1e3), 1), "unit": "tokens/s",
-           "h2d_bytes_per_step": x_h.numel() * 2, "d2h_bytes_per_step": out_h.numel() * 4,
-           "ms_per_step": round(e2e_ms, 4), "api": "moe_forward_host (pinned host x and out)"}
-    del ws_h
+    e2e = None
+    if not a.no_e2e:
+        e2e = run_e2e(M, w, layer, x, dev, stream, world, tokens_all, a)
 
     # ---- decode (T = 1, 2, 4, 8 on the same Mixtral-shape weights)
     decode = None
     if a.workload == "prefill" and not a.no_extra:
-        decode = {}
-        for T in I.DECODE_TS:
-            xt = x[:T].contiguous()
-            it = torch.empty(T, w.k, dtype=torch.int32, device=dev)
-            ot = torch.empty(T, w.d, dtype=torch.float32, device=dev)
-            for _ in range(5):
-                layer.forward(xt, out=ot, topk_idx_out=it)
-            torch.cuda.synchronize()
-            U, nbytes, w13_bytes, expert_bytes = decode_bytes(w, T, it)
-            M.moe_profile_enable(True)
-            ms = time_loop(lambda: layer.forward(xt, out=ot), 50, stream)
-            M.moe_profile_enable(False)
-            st = M.moe_profile_read()
-            ms = max_over_ranks(ms, world, dev)
-            k13 = st["dec_w13"][0] / st["dec_w13"][1]
-            k2 = st["dec_w2"][0] / st["dec_w2"][1]
-            decode[f"T{T}"] = {
-                "tokens_per_s": round(T * world / (ms / 1e3), 1), "ms_per_step": round(ms, 4),
-                "unique_experts": U, "bytes_per_step": nbytes,
-                "GB_s": round(nbytes / (ms / 1e3) / 1e9, 1),
-                "frac_hbm_measured": round(nbytes / (ms / 1e3) / 1e9 / peaks["hbm_gbs"], 4),
-                "frac_hbm_nominal_8000": round(nbytes / (ms / 1e3) / 1e9 / 8000.0, 4),
-                "chosen_expert_GB_s_kernels": round(expert_bytes / ((k13 + k2) / 1e3) / 1e9, 1),
-                "dec_w13_GB_s": round(w13_bytes / (k13 / 1e3) / 1e9, 1),
-                "stages_ms": {k: round(v[0] / v[1], 4) for k, v in st.items()}}
+        decode = run_decode_set(M, w, layer, x, dev, stream, world, peaks)
 
     # ---- CPU baseline: the oracle on host cores (rank 0, N = 1 only)
     cpu = None
@@ -330,10 +315,7 @@ def run_ours(a, world, rank, local):
                    "zipf_s": w.zipf_s, "seed": 0, "parallelism": f"replicas x{world}",
                    "l2": "inputs larger than L2 (expert weights and activations exceed 126 MB)",
                    "output": "fp32 [T, d]"},
-        "active_tflops": round(flops / (step_ms_max / 1e3) / 1e12, 1),
-        "active_tflops_frac_measured_sustained": round(flops / (step_ms_max / 1e3) / 1e12 / peak_t, 4),
-        "n_kept": n_kept,
-        "w2_tflops": round(w2_tflops, 1),
+        **extra,
         "stages_ms": stage_ms,
         "roofline": roofline,
         "cpu_baseline": cpu,
@@ -344,6 +326,58 @@ def run_ours(a, world, rank, local):
     if decode is not None:
         res["decode"] = decode
     return res
+
+
+def run_e2e(M, w, layer, x, dev, stream, world, tokens_all, a):
+    shape_h = M.shape_of(w, M.MOE_FLAG_HOST_IO)
+    ws_h = M.alloc_workspace(shape_h, dev)
+    x_h = x.cpu().pin_memory()
+    out_h = torch.empty(w.T, w.d, dtype=torch.float32).pin_memory()
+
+    def e2e_step():
+        M.moe_forward_host(shape_h, x_h, layer.Wg, layer.bias, layer.W13, layer.W2, layer.W13s,
+                           layer.W2s, out_h, layer.status, ws_h)
+    ws_h = M.alloc_workspace(shape_h, dev)
+    x_h = x.cpu().pin_memory()
+    out_h = torch.empty(w.T, w.d, dtype=torch.float32).pin_memory()
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = time_loop(e2e_step, max(3, a.steps // 2), stream)
+    e2e_ms = max_over_ranks(e2e_ms, world, dev)
+    return {"value": round(tokens_all / (e2e_ms / 1e3), 1), "unit": "tokens/s",
+            "h2d_bytes_per_step": x_h.numel() * 2, "d2h_bytes_per_step": out_h.numel() * 4,
+            "ms_per_step": round(e2e_ms, 4), "api": "moe_forward_host (pinned host x and out)"}
+
+
+def run_decode_set(M, w, layer, x, dev, stream, world, peaks):
+    decode = {}
+    for T in I.DECODE_TS:
+        xt = x[:T].contiguous()
+        it = torch.empty(T, w.k, dtype=torch.int32, device=dev)
+        ot = torch.empty(T, w.d, dtype=torch.float32, device=dev)
+        for _ in range(5):
+            layer.forward(xt, out=ot, topk_idx_out=it)
+        torch.cuda.synchronize()
+        U, nbytes, w13_bytes, expert_bytes = decode_bytes(w, T, it)
+        M.moe_profile_enable(True)
+        ms = time_loop(lambda: layer.forward(xt, out=ot), 50, stream)
+        M.moe_profile_enable(False)
+        st = M.moe_profile_read()
+        ms = max_over_ranks(ms, world, dev)
+        k13 = st["dec_w13"][0] / st["dec_w13"][1]
+        k2 = st["dec_w2"][0] / st["dec_w2"][1]
+        decode[f"T{T}"] = {
+            "tokens_per_s": round(T * world / (ms / 1e3), 1), "ms_per_step": round(ms, 4),
+            "unique_experts": U, "bytes_per_step": nbytes,
+            "GB_s": round(nbytes / (ms / 1e3) / 1e9, 1),
+            "frac_hbm_measured": round(nbytes / (ms / 1e3) / 1e9 / peaks["hbm_gbs"], 4),
+            "frac_hbm_nominal_8000": round(nbytes / (ms / 1e3) / 1e9 / 8000.0, 4),
+            "chosen_expert_GB_s_kernels": round(expert_bytes / ((k13 + k2) / 1e3) / 1e9, 1),
+            "dec_w13_GB_s": round(w13_bytes / (k13 / 1e3) / 1e9, 1),
+            "stages_ms": {k: round(v[0] / v[1], 4) for k, v in st.items()}}
+    return decode
 
 
 def run_reference(a, world, rank):
@@ -378,6 +412,8 @@ def main(argv=None):
     ap.add_argument("--no-extra", action="store_true", help="skip the decode measurements")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds per oracle sample")
+    ap.add_argument("--tokens", type=int, default=0, help="override T (profiling runs)")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end run")
     a = ap.parse_args(argv)
     if a.warmup < 3 and a.impl == "ours":
         a.warmup = 3

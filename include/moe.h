@@ -28,7 +28,8 @@
  *    which may be NULL to ignore them) as the bit (1u << MOE_ERR_*). The
  *    caller clears it and reads it whenever it chooses. When a device error
  *    is flagged, the outputs of that call are unspecified.
- *  - T = 0 is a valid no-op for every call.
+ *  - T = 0 is a valid no-op for every call (pointers may then be NULL);
+ *    moe_permute then only zeroes the counts, offsets and n_kept it is given.
  *
  * Types: bf16 is the 16-bit bfloat16 bit pattern (uint16_t here); fp32 is
  * float; ids and positions are int32_t.

@@ -435,6 +435,8 @@ int moe_pack_w13(const moe_shape_t *shape, const moe_bf16_t *W1, const moe_bf16_
     int rc = check_shape(shape);
     if (rc)
         return rc;
+    if (shape->T == 0)
+        return MOE_OK;   // empty batch: nothing to read or write
     if (!W1 || !W3 || !W13 || !al16(W1) || !al16(W3) || !al16(W13))
         return MOE_ERR_INVALID_ARG;
     return launch_pack_w13(shape->E, shape->d_ff, shape->d, W1, W3, W13,
@@ -448,6 +450,8 @@ int moe_route(const moe_shape_t *shape, const moe_bf16_t *x, const moe_bf16_t *W
     int rc = check_shape(shape);
     if (rc)
         return rc;
+    if (shape->T == 0)
+        return MOE_OK;   // empty batch: nothing to read or write
     const moe_shape_t &s = *shape;
     if (!logits || !topk_idx || !topk_w || (x && !Wg) || (x && (!al16(x) || !al16(Wg))))
         return MOE_ERR_INVALID_ARG;
@@ -471,21 +475,21 @@ int moe_permute(const moe_shape_t *shape, const int32_t *topk_idx, const moe_bf1
     if (rc)
         return rc;
     const moe_shape_t &s = *shape;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (s.T == 0) {
+        // empty batch: every expert has 0 rows (async memsets, no kernel)
+        if ((expert_counts && cudaMemsetAsync(expert_counts, 0, sizeof(int32_t) * s.E, st) != cudaSuccess) ||
+            (expert_offsets && cudaMemsetAsync(expert_offsets, 0, sizeof(int32_t) * (s.E + 1), st) != cudaSuccess) ||
+            (n_kept && cudaMemsetAsync(n_kept, 0, sizeof(int32_t), st) != cudaSuccess))
+            return MOE_ERR_CUDA;
+        return MOE_OK;
+    }
     if (!topk_idx || !expert_counts || !expert_offsets || !slot_pos || !perm_token ||
         (x && !x_perm) || (x && (!al16(x) || !al16(x_perm))))
         return MOE_ERR_INVALID_ARG;
     WsLayout L;
     if ((rc = check_ws(s, ws, ws_bytes, L)))
         return rc;
-    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    if (s.T == 0) {
-        // offsets of an empty batch: all zero (a no-op kernel-free answer)
-        if (cudaMemsetAsync(expert_counts, 0, sizeof(int32_t) * s.E, st) != cudaSuccess ||
-            cudaMemsetAsync(expert_offsets, 0, sizeof(int32_t) * (s.E + 1), st) != cudaSuccess ||
-            (n_kept && cudaMemsetAsync(n_kept, 0, sizeof(int32_t), st) != cudaSuccess))
-            return MOE_ERR_CUDA;
-        return MOE_OK;
-    }
     int32_t *counter = at<int32_t>(ws, L.counter);
     if (cudaMemsetAsync(counter, 0, sizeof(int32_t), st) != cudaSuccess)
         return MOE_ERR_CUDA;
@@ -509,6 +513,8 @@ int moe_expert_ffn(const moe_shape_t *shape, const moe_bf16_t *x_perm,
     int rc = check_shape(shape);
     if (rc)
         return rc;
+    if (shape->T == 0)
+        return MOE_OK;   // empty batch: nothing to read or write
     const moe_shape_t &s = *shape;
     if (!x_perm || !expert_offsets || !W13 || !W2 || !al16(x_perm) || !al16(W13) || !al16(W2))
         return MOE_ERR_INVALID_ARG;
@@ -534,6 +540,8 @@ int moe_combine(const moe_shape_t *shape, const float *y_perm, const int32_t *sl
     int rc = check_shape(shape);
     if (rc)
         return rc;
+    if (shape->T == 0)
+        return MOE_OK;   // empty batch: nothing to read or write
     if (!y_perm || !slot_pos || !topk_w || !out || !al16(y_perm) || !al16(out) ||
         (shared_out && !al16(shared_out)))
         return MOE_ERR_INVALID_ARG;
@@ -550,6 +558,8 @@ int moe_forward(const moe_shape_t *shape, const moe_bf16_t *x, const moe_bf16_t 
     int rc = check_shape(shape);
     if (rc)
         return rc;
+    if (shape->T == 0)
+        return MOE_OK;   // empty batch: nothing to read or write
     const moe_shape_t &s = *shape;
     if (!x || !Wg || !W13 || !W2 || !out || !al16(x) || !al16(Wg) || !al16(W13) || !al16(W2) ||
         !al16(out))
@@ -574,6 +584,8 @@ int moe_forward_host(const moe_shape_t *shape, const moe_bf16_t *x_host, const m
     int rc = check_shape(shape);
     if (rc)
         return rc;
+    if (shape->T == 0)
+        return MOE_OK;   // empty batch: nothing to read or write
     const moe_shape_t &s = *shape;
     if (!(s.flags & MOE_FLAG_HOST_IO))
         return MOE_ERR_INVALID_ARG;
