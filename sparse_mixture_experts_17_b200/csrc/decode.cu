@@ -7,8 +7,11 @@
 // the fused kernel" (mlxcel) routes one-token decode to a fused kernel fed by
 // the router's top-k indices and renormalised scores. Here the chosen experts
 // are known only on the device, so every CTA rebuilds the (tiny) plan in
-// shared memory from topk_idx and the weight stream is spread over all SMs.
+// shared memory from topk_idx, and the weight stream is spread over all SMs.
 //
+// Routing (k_dec_route): one CTA computes the T x E logits (warps over
+// experts, lanes over d) and then the top-k (one warp per token), when W_g is
+// small; otherwise k_dec_router (one warp per expert) feeds k_topk.
 // Phase 1 (k_dec_w13): work unit = one SwiGLU column c of one chosen expert:
 //   h[a, c] = bf16(silu(W1_e[c] . x_t) * (W3_e[c] . x_t)) for every
 //   assignment a = (t, j) routed to e. Each unit streams the gate row and the
@@ -17,8 +20,12 @@
 //   out[t, r] = sum over the chosen experts e (ascending), then the shared
 //   expert, of w[a] * (W2_e[r] . h[a]). Each unit streams W2_e[r] once per
 //   chosen expert; h is L1/L2 resident. Fixed order: deterministic.
+// The kernels are instantiated for MAXT in {1, 2, 4, 8, 16} >= T, the most
+// assignments one expert can have (a token picks an expert at most once), so
+// the per-token accumulators stay in registers and the code stays small.
 #include "common.cuh"
 #include "internal.h"
+#include "topk.cuh"
 
 namespace moe {
 
@@ -41,7 +48,6 @@ __device__ void build_plan(DecPlanSmem &P, const int32_t *__restrict__ idx, int 
     for (int e = threadIdx.x; e < MOE_MAX_E; e += blockDim.x)
         P.cnt[e] = 0;
     __syncthreads();
-    // rank of each assignment among earlier ones of the same expert
     for (int a = threadIdx.x; a < A; a += blockDim.x) {
         const int e = idx[a];
         if (e < 0 || e >= E) {
@@ -67,6 +73,7 @@ __device__ void build_plan(DecPlanSmem &P, const int32_t *__restrict__ idx, int 
         P.U = u;
     }
     __syncthreads();
+    // rank of each assignment among earlier ones of the same expert (token order)
     for (int a = threadIdx.x; a < A; a += blockDim.x) {
         const int e = idx[a];
         if (e < 0 || e >= E)
@@ -100,8 +107,10 @@ __device__ __forceinline__ float warp_sum(float v)
     return v;
 }
 
-// ---------------------------------------------------------------- router for small T
+// ---------------------------------------------------------------- routing for small T
+
 // One warp per expert: logits[t, e] = Wg[e] . x[t] + bias[e] for all t < T.
+template <int MAXT>
 __global__ void __launch_bounds__(256) k_dec_router(const uint16_t *__restrict__ x,
                                                     const uint16_t *__restrict__ Wg,
                                                     const float *__restrict__ bias, int T, int d,
@@ -111,20 +120,20 @@ __global__ void __launch_bounds__(256) k_dec_router(const uint16_t *__restrict__
     const int nwarps = gridDim.x * (blockDim.x >> 5);
     const int nv = d / 8;
     for (int e = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; e < E; e += nwarps) {
-        float acc[MOE_DECODE_MAX_T];
+        float acc[MAXT];
 #pragma unroll
-        for (int t = 0; t < MOE_DECODE_MAX_T; ++t)
+        for (int t = 0; t < MAXT; ++t)
             acc[t] = 0.f;
         const uint4 *wr = reinterpret_cast<const uint4 *>(Wg + (size_t)e * d);
         for (int c = lane; c < nv; c += 32) {
             const uint4 wv = ld_stream_v4(wr + c);
 #pragma unroll
-            for (int t = 0; t < MOE_DECODE_MAX_T; ++t)
+            for (int t = 0; t < MAXT; ++t)
                 if (t < T)
-                    acc[t] = dot8(wv, reinterpret_cast<const uint4 *>(x + (size_t)t * d)[c], acc[t]);
+                    acc[t] = dot8(wv, __ldg(reinterpret_cast<const uint4 *>(x + (size_t)t * d) + c), acc[t]);
         }
 #pragma unroll
-        for (int t = 0; t < MOE_DECODE_MAX_T; ++t) {
+        for (int t = 0; t < MAXT; ++t) {
             if (t < T) {
                 const float s = warp_sum(acc[t]);
                 if (lane == 0)
@@ -134,16 +143,61 @@ __global__ void __launch_bounds__(256) k_dec_router(const uint16_t *__restrict__
     }
 }
 
+// Router and top-k in one CTA of 512 threads, for W_g up to kFusedRouteBytes:
+// warps stride over experts (lanes over d) into shared memory, then warp t
+// selects token t's experts.
+constexpr size_t kFusedRouteBytes = 256 * 1024;
+
+template <int MAXT, int VPL>
+__global__ void __launch_bounds__(512) k_dec_route(const uint16_t *__restrict__ x,
+                                                   const uint16_t *__restrict__ Wg,
+                                                   const float *__restrict__ bias, int T, int d,
+                                                   int E, int k, float *__restrict__ logits,
+                                                   int32_t *__restrict__ idx,
+                                                   float *__restrict__ w, uint32_t *status)
+{
+    __shared__ float sl[MAXT * MOE_MAX_E];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int nv = d / 8;
+    for (int e = warp; e < E; e += 16) {
+        float acc[MAXT];
+#pragma unroll
+        for (int t = 0; t < MAXT; ++t)
+            acc[t] = 0.f;
+        const uint4 *wr = reinterpret_cast<const uint4 *>(Wg + (size_t)e * d);
+        for (int c = lane; c < nv; c += 32) {
+            const uint4 wv = ld_stream_v4(wr + c);
+#pragma unroll
+            for (int t = 0; t < MAXT; ++t)
+                if (t < T)
+                    acc[t] = dot8(wv, __ldg(reinterpret_cast<const uint4 *>(x + (size_t)t * d) + c), acc[t]);
+        }
+#pragma unroll
+        for (int t = 0; t < MAXT; ++t) {
+            if (t < T) {
+                const float s = warp_sum(acc[t]) + (bias ? bias[e] : 0.f);
+                if (lane == 0) {
+                    sl[t * E + e] = s;
+                    logits[(size_t)t * E + e] = s;
+                }
+            }
+        }
+    }
+    __syncthreads();
+    if (warp < T)
+        warp_topk_row<VPL>(sl + warp * E, E, k, idx + (size_t)warp * k, w + (size_t)warp * k,
+                           status);
+}
+
 // ---------------------------------------------------------------- phase 1: W1/W3 + SwiGLU
 constexpr int kDecUnroll = 4;
 
-__global__ void __launch_bounds__(256) k_dec_w13(const uint16_t *__restrict__ x,
-                                                 const int32_t *__restrict__ idx, int T, int d,
-                                                 int d_ff, int E, int k,
-                                                 const uint16_t *__restrict__ W13, int d_ff_s,
-                                                 const uint16_t *__restrict__ W13s,
-                                                 uint16_t *__restrict__ Hdec,
-                                                 uint16_t *__restrict__ Hs, uint32_t *status)
+template <int MAXT>
+__global__ void __launch_bounds__(256, (MAXT <= 2) ? 4 : 2)
+    k_dec_w13(const uint16_t *__restrict__ x, const int32_t *__restrict__ idx, int T, int d,
+              int d_ff, int E, int k, const uint16_t *__restrict__ W13, int d_ff_s,
+              const uint16_t *__restrict__ W13s, uint16_t *__restrict__ Hdec,
+              uint16_t *__restrict__ Hs, uint32_t *status)
 {
     __shared__ DecPlanSmem P;
     build_plan(P, idx, T, E, k, status);
@@ -179,13 +233,14 @@ __global__ void __launch_bounds__(256) k_dec_w13(const uint16_t *__restrict__ x,
             hout = Hs;
             ldh = d_ff_s;
         }
-        int tok[MOE_DECODE_MAX_T];
+        const uint4 *xr[MAXT];
 #pragma unroll
-        for (int s = 0; s < MOE_DECODE_MAX_T; ++s)
-            tok[s] = (s < na) ? (shared ? s : P.list[a0 + s] / k) : 0;
-        float ag[MOE_DECODE_MAX_T], au[MOE_DECODE_MAX_T];
+        for (int s = 0; s < MAXT; ++s)
+            xr[s] = reinterpret_cast<const uint4 *>(
+                x + (size_t)((s < na) ? (shared ? s : P.list[a0 + s] / k) : 0) * d);
+        float ag[MAXT], au[MAXT];
 #pragma unroll
-        for (int s = 0; s < MOE_DECODE_MAX_T; ++s)
+        for (int s = 0; s < MAXT; ++s)
             ag[s] = au[s] = 0.f;
         for (int cb = 0; cb < nv; cb += 32 * kDecUnroll) {
             uint4 wg[kDecUnroll], wu[kDecUnroll];
@@ -203,9 +258,9 @@ __global__ void __launch_bounds__(256) k_dec_w13(const uint16_t *__restrict__ x,
                 if (ci >= nv)
                     continue;
 #pragma unroll
-                for (int s = 0; s < MOE_DECODE_MAX_T; ++s) {
+                for (int s = 0; s < MAXT; ++s) {
                     if (s < na) {
-                        const uint4 xv = reinterpret_cast<const uint4 *>(x + (size_t)tok[s] * d)[ci];
+                        const uint4 xv = __ldg(xr[s] + ci);
                         ag[s] = dot8(wg[i], xv, ag[s]);
                         au[s] = dot8(wu[i], xv, au[s]);
                     }
@@ -213,7 +268,7 @@ __global__ void __launch_bounds__(256) k_dec_w13(const uint16_t *__restrict__ x,
             }
         }
 #pragma unroll
-        for (int s = 0; s < MOE_DECODE_MAX_T; ++s) {
+        for (int s = 0; s < MAXT; ++s) {
             if (s < na) {
                 const float g = warp_sum(ag[s]);
                 const float uu = warp_sum(au[s]);
@@ -228,14 +283,12 @@ __global__ void __launch_bounds__(256) k_dec_w13(const uint16_t *__restrict__ x,
 }
 
 // ---------------------------------------------------------------- phase 2: W2 + combine
-__global__ void __launch_bounds__(256) k_dec_w2(const int32_t *__restrict__ idx,
-                                                const float *__restrict__ topk_w, int T, int d,
-                                                int d_ff, int E, int k,
-                                                const uint16_t *__restrict__ W2, int d_ff_s,
-                                                const uint16_t *__restrict__ W2s,
-                                                const uint16_t *__restrict__ Hdec,
-                                                const uint16_t *__restrict__ Hs,
-                                                float *__restrict__ out, uint32_t *status)
+template <int MAXT>
+__global__ void __launch_bounds__(256, (MAXT <= 2) ? 4 : 2)
+    k_dec_w2(const int32_t *__restrict__ idx, const float *__restrict__ topk_w, int T, int d,
+             int d_ff, int E, int k, const uint16_t *__restrict__ W2, int d_ff_s,
+             const uint16_t *__restrict__ W2s, const uint16_t *__restrict__ Hdec,
+             const uint16_t *__restrict__ Hs, float *__restrict__ out, uint32_t *status)
 {
     __shared__ DecPlanSmem P;
     build_plan(P, idx, T, E, k, status);
@@ -243,9 +296,9 @@ __global__ void __launch_bounds__(256) k_dec_w2(const int32_t *__restrict__ idx,
     const int nwarps = gridDim.x * (blockDim.x >> 5);
     const int n_src = P.U + (W2s ? 1 : 0);
     for (int r = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; r < d; r += nwarps) {
-        float acc[MOE_DECODE_MAX_T];
+        float acc[MAXT];
 #pragma unroll
-        for (int t = 0; t < MOE_DECODE_MAX_T; ++t)
+        for (int t = 0; t < MAXT; ++t)
             acc[t] = 0.f;
         for (int u = 0; u < n_src; ++u) {
             const bool shared = (u == P.U);
@@ -254,15 +307,21 @@ __global__ void __launch_bounds__(256) k_dec_w2(const int32_t *__restrict__ idx,
                 shared ? W2s + (size_t)r * d_ff_s : W2 + ((size_t)P.uniq[u] * d + r) * d_ff);
             const int a0 = shared ? 0 : P.ustart[u];
             const int na = shared ? T : P.ustart[u + 1] - a0;
-            int arow[MOE_DECODE_MAX_T];
-#pragma unroll
-            for (int s = 0; s < MOE_DECODE_MAX_T; ++s)
-                arow[s] = (s < na) ? (shared ? s : P.list[a0 + s]) : 0;
             const uint16_t *hb = shared ? Hs : Hdec;
-            const int nv = ff / 8;
-            float pa[MOE_DECODE_MAX_T];
+            const uint4 *hr[MAXT];
+            int tk[MAXT];
+            float wt[MAXT];
 #pragma unroll
-            for (int s = 0; s < MOE_DECODE_MAX_T; ++s)
+            for (int s = 0; s < MAXT; ++s) {
+                const int a = (s < na) ? (shared ? s : P.list[a0 + s]) : 0;
+                hr[s] = reinterpret_cast<const uint4 *>(hb + (size_t)a * ff);
+                tk[s] = shared ? s : a / k;
+                wt[s] = (s < na) ? (shared ? 1.f : topk_w[a]) : 0.f;
+            }
+            const int nv = ff / 8;
+            float pa[MAXT];
+#pragma unroll
+            for (int s = 0; s < MAXT; ++s)
                 pa[s] = 0.f;
             for (int cb = 0; cb < nv; cb += 32 * kDecUnroll) {
                 uint4 wv[kDecUnroll];
@@ -278,28 +337,24 @@ __global__ void __launch_bounds__(256) k_dec_w2(const int32_t *__restrict__ idx,
                     if (ci >= nv)
                         continue;
 #pragma unroll
-                    for (int s = 0; s < MOE_DECODE_MAX_T; ++s)
+                    for (int s = 0; s < MAXT; ++s)
                         if (s < na)
-                            pa[s] = dot8(wv[i],
-                                         reinterpret_cast<const uint4 *>(hb + (size_t)arow[s] * ff)[ci],
-                                         pa[s]);
+                            pa[s] = dot8(wv[i], __ldg(hr[s] + ci), pa[s]);
                 }
             }
             // fold the lane partials into the tokens' accumulators, weighted
 #pragma unroll
-            for (int s = 0; s < MOE_DECODE_MAX_T; ++s) {
+            for (int s = 0; s < MAXT; ++s) {
                 if (s < na) {
-                    const int t = shared ? s : arow[s] / k;
-                    const float wgt = shared ? 1.f : topk_w[arow[s]];
 #pragma unroll
-                    for (int tt = 0; tt < MOE_DECODE_MAX_T; ++tt)
-                        if (tt == t)
-                            acc[tt] = fmaf(wgt, pa[s], acc[tt]);
+                    for (int tt = 0; tt < MAXT; ++tt)
+                        if (tt == tk[s])
+                            acc[tt] = fmaf(wt[s], pa[s], acc[tt]);
                 }
             }
         }
 #pragma unroll
-        for (int t = 0; t < MOE_DECODE_MAX_T; ++t) {
+        for (int t = 0; t < MAXT; ++t) {
             if (t < T) {
                 const float s = warp_sum(acc[t]);
                 if (lane == 0)
@@ -309,15 +364,84 @@ __global__ void __launch_bounds__(256) k_dec_w2(const int32_t *__restrict__ idx,
     }
 }
 
+// ---------------------------------------------------------------- host side
+
+static int maxt_for(int T) { return T <= 1 ? 1 : T <= 2 ? 2 : T <= 4 ? 4 : T <= 8 ? 8 : 16; }
+
+int launch_dec_router(const moe_shape_t &s, const uint16_t *x, const uint16_t *Wg,
+                      const float *bias, float *logits, cudaStream_t st)
+{
+    if (s.T == 0)
+        return MOE_OK;
+    const int blocks = (s.E + 7) / 8;
+    switch (maxt_for(s.T)) {
+    case 1: k_dec_router<1><<<blocks, 256, 0, st>>>(x, Wg, bias, s.T, s.d, s.E, logits); break;
+    case 2: k_dec_router<2><<<blocks, 256, 0, st>>>(x, Wg, bias, s.T, s.d, s.E, logits); break;
+    case 4: k_dec_router<4><<<blocks, 256, 0, st>>>(x, Wg, bias, s.T, s.d, s.E, logits); break;
+    case 8: k_dec_router<8><<<blocks, 256, 0, st>>>(x, Wg, bias, s.T, s.d, s.E, logits); break;
+    default: k_dec_router<16><<<blocks, 256, 0, st>>>(x, Wg, bias, s.T, s.d, s.E, logits); break;
+    }
+    return launched();
+}
+
+bool dec_route_fusable(const moe_shape_t &s)
+{
+    return s.T <= MOE_DECODE_MAX_T && (size_t)s.E * s.d * 2 <= kFusedRouteBytes;
+}
+
+template <int MAXT>
+static void launch_dec_route_t(const moe_shape_t &s, const uint16_t *x, const uint16_t *Wg,
+                               const float *bias, float *logits, int32_t *idx, float *w,
+                               uint32_t *status, cudaStream_t st)
+{
+    const int vpl = (s.E + 31) / 32;
+    if (vpl <= 1)
+        k_dec_route<MAXT, 1><<<1, 512, 0, st>>>(x, Wg, bias, s.T, s.d, s.E, s.k, logits, idx, w, status);
+    else if (vpl <= 2)
+        k_dec_route<MAXT, 2><<<1, 512, 0, st>>>(x, Wg, bias, s.T, s.d, s.E, s.k, logits, idx, w, status);
+    else if (vpl <= 4)
+        k_dec_route<MAXT, 4><<<1, 512, 0, st>>>(x, Wg, bias, s.T, s.d, s.E, s.k, logits, idx, w, status);
+    else
+        k_dec_route<MAXT, 8><<<1, 512, 0, st>>>(x, Wg, bias, s.T, s.d, s.E, s.k, logits, idx, w, status);
+}
+
+int launch_dec_route(const moe_shape_t &s, const uint16_t *x, const uint16_t *Wg,
+                     const float *bias, float *logits, int32_t *idx, float *w, uint32_t *status,
+                     cudaStream_t st)
+{
+    if (s.T == 0)
+        return MOE_OK;
+    switch (maxt_for(s.T)) {
+    case 1: launch_dec_route_t<1>(s, x, Wg, bias, logits, idx, w, status, st); break;
+    case 2: launch_dec_route_t<2>(s, x, Wg, bias, logits, idx, w, status, st); break;
+    case 4: launch_dec_route_t<4>(s, x, Wg, bias, logits, idx, w, status, st); break;
+    case 8: launch_dec_route_t<8>(s, x, Wg, bias, logits, idx, w, status, st); break;
+    default: launch_dec_route_t<16>(s, x, Wg, bias, logits, idx, w, status, st); break;
+    }
+    return launched();
+}
+
 int launch_dec_w13(const moe_shape_t &s, const uint16_t *x, const int32_t *topk_idx,
                    const uint16_t *W13, const uint16_t *W13s, uint16_t *Hdec, uint32_t *status,
                    cudaStream_t st)
 {
     if (s.T == 0)
         return MOE_OK;
-    k_dec_w13<<<num_sms() * 4, 256, 0, st>>>(x, topk_idx, s.T, s.d, s.d_ff, s.E, s.k, W13,
-                                            s.d_ff_shared, s.d_ff_shared ? W13s : nullptr, Hdec,
-                                            Hdec + (size_t)s.T * s.k * s.d_ff, status);
+    const int mt = maxt_for(s.T);
+    const int blocks = num_sms() * ((mt <= 2) ? 4 : 2);
+    uint16_t *Hs = Hdec + (size_t)s.T * s.k * s.d_ff;
+    const uint16_t *ws = s.d_ff_shared ? W13s : nullptr;
+#define MOE_DEC13(M)                                                                            \
+    k_dec_w13<M><<<blocks, 256, 0, st>>>(x, topk_idx, s.T, s.d, s.d_ff, s.E, s.k, W13,         \
+                                         s.d_ff_shared, ws, Hdec, Hs, status)
+    switch (mt) {
+    case 1: MOE_DEC13(1); break;
+    case 2: MOE_DEC13(2); break;
+    case 4: MOE_DEC13(4); break;
+    case 8: MOE_DEC13(8); break;
+    default: MOE_DEC13(16); break;
+    }
+#undef MOE_DEC13
     return launched();
 }
 
@@ -327,19 +451,21 @@ int launch_dec_w2(const moe_shape_t &s, const int32_t *topk_idx, const float *to
 {
     if (s.T == 0)
         return MOE_OK;
-    k_dec_w2<<<num_sms() * 4, 256, 0, st>>>(topk_idx, topk_w, s.T, s.d, s.d_ff, s.E, s.k, W2,
-                                           s.d_ff_shared, s.d_ff_shared ? W2s : nullptr, Hdec,
-                                           Hdec + (size_t)s.T * s.k * s.d_ff, out, status);
-    return launched();
-}
-
-int launch_dec_router(const moe_shape_t &s, const uint16_t *x, const uint16_t *Wg,
-                      const float *bias, float *logits, cudaStream_t st)
-{
-    if (s.T == 0)
-        return MOE_OK;
-    const int blocks = (s.E + 7) / 8;
-    k_dec_router<<<blocks, 256, 0, st>>>(x, Wg, bias, s.T, s.d, s.E, logits);
+    const int mt = maxt_for(s.T);
+    const int blocks = num_sms() * ((mt <= 2) ? 4 : 2);
+    const uint16_t *Hs = Hdec + (size_t)s.T * s.k * s.d_ff;
+    const uint16_t *ws = s.d_ff_shared ? W2s : nullptr;
+#define MOE_DEC2(M)                                                                             \
+    k_dec_w2<M><<<blocks, 256, 0, st>>>(topk_idx, topk_w, s.T, s.d, s.d_ff, s.E, s.k, W2,      \
+                                        s.d_ff_shared, ws, Hdec, Hs, out, status)
+    switch (mt) {
+    case 1: MOE_DEC2(1); break;
+    case 2: MOE_DEC2(2); break;
+    case 4: MOE_DEC2(4); break;
+    case 8: MOE_DEC2(8); break;
+    default: MOE_DEC2(16); break;
+    }
+#undef MOE_DEC2
     return launched();
 }
 

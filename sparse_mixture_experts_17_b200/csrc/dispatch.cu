@@ -9,6 +9,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "topk.cuh"
 
 namespace moe {
 
@@ -112,11 +113,6 @@ int launch_router_simt(const moe_shape_t &s, const uint16_t *x, const uint16_t *
 }
 
 // ---------------------------------------------------------------- softmax + top-k
-// One warp per token. Lane l holds logits l, l+32, ... (VPL per lane). k
-// rounds of a butterfly arg-max with the key (larger value, then smaller
-// index) pick the experts in selection order; the weights are
-// exp(l_j - l_max) / sum over the chosen k, which is the softmax over all E
-// renormalised over the top-k (the full-E denominator cancels).
 template <int VPL>
 __global__ void __launch_bounds__(256) k_topk(const float *__restrict__ logits, int T, int E,
                                               int k, int32_t *__restrict__ idx,
@@ -126,67 +122,10 @@ __global__ void __launch_bounds__(256) k_topk(const float *__restrict__ logits, 
     if (counter_to_zero && blockIdx.x == 0 && threadIdx.x == 0)
         *counter_to_zero = 0;
     const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    const int lane = threadIdx.x & 31;
     if (t >= T)
         return;
-    const float *l = logits + (size_t)t * E;
-    float v[VPL];
-    uint32_t avail = 0;
-    bool bad = false;
-#pragma unroll
-    for (int i = 0; i < VPL; ++i) {
-        const int e = lane + 32 * i;
-        v[i] = -INFINITY;
-        if (e < E) {
-            v[i] = l[e];
-            avail |= 1u << i;
-            bad |= isnan(v[i]);
-        }
-    }
-    float my_v = 0.f;
-    int my_i = 0;
-    for (int j = 0; j < k; ++j) {
-        float bv = -INFINITY;
-        int bi = INT_MAX;
-#pragma unroll
-        for (int i = 0; i < VPL; ++i) {
-            const int e = lane + 32 * i;
-            if (((avail >> i) & 1u) && (v[i] > bv || (v[i] == bv && e < bi))) {
-                bv = v[i];
-                bi = e;
-            }
-        }
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-            const float ov = __shfl_xor_sync(kFullMask, bv, off);
-            const int oi = __shfl_xor_sync(kFullMask, bi, off);
-            if (ov > bv || (ov == bv && oi < bi)) {
-                bv = ov;
-                bi = oi;
-            }
-        }
-        if (bi != INT_MAX && (bi & 31) == lane)
-            avail &= ~(1u << (bi >> 5));
-        if (lane == j) {
-            my_v = bv;
-            my_i = bi;
-        }
-    }
-    const float M = __shfl_sync(kFullMask, my_v, 0);
-    bad |= !isfinite(M);
-    if (__any_sync(kFullMask, bad)) {
-        if (lane == 0)
-            flag_status(status, MOE_ERR_NONFINITE);
-    }
-    float ex = (lane < k) ? expf(my_v - M) : 0.f;
-    float sum = ex;
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1)
-        sum += __shfl_xor_sync(kFullMask, sum, off);
-    if (lane < k) {
-        idx[(size_t)t * k + lane] = my_i;
-        w[(size_t)t * k + lane] = ex / sum;
-    }
+    warp_topk_row<VPL>(logits + (size_t)t * E, E, k, idx + (size_t)t * k, w + (size_t)t * k,
+                       status);
 }
 
 int launch_topk(const moe_shape_t &s, const float *logits, int32_t *idx, float *w,

@@ -289,14 +289,17 @@ static int forward_impl(const moe_shape_t &s, const WsLayout &L, void *ws, const
         return MOE_ERR_UNSUPPORTED;
     const bool decode = force_dec || (!force_pre && s.T <= MOE_DECODE_DEFAULT_T);
     int rc;
-    {
-        StageMark m(MOE_STAGE_ROUTER, st);
-        rc = router(s, x, Wg, bias, logits, status, st);
-    }
-    if (rc)
-        return rc;
     int32_t *counter = at<int32_t>(ws, L.counter);
-    {
+    if (decode && dec_route_fusable(s)) {
+        StageMark m(MOE_STAGE_ROUTER, st);   // router and top-k in one launch
+        rc = launch_dec_route(s, x, Wg, bias, logits, idx, w, status, st);
+    } else {
+        {
+            StageMark m(MOE_STAGE_ROUTER, st);
+            rc = router(s, x, Wg, bias, logits, status, st);
+        }
+        if (rc)
+            return rc;
         StageMark m(MOE_STAGE_TOPK, st);
         rc = launch_topk(s, logits, idx, w, counter, status, st);
     }
@@ -461,6 +464,8 @@ int moe_route(const moe_shape_t *shape, const moe_bf16_t *x, const moe_bf16_t *W
     if (s.T == 0)
         return MOE_OK;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (x && dec_route_fusable(s))
+        return launch_dec_route(s, x, Wg, bias, logits, topk_idx, topk_w, status, st);
     if (x && (rc = router(s, x, Wg, bias, logits, status, st)))
         return rc;
     return launch_topk(s, logits, topk_idx, topk_w, nullptr, status, st);

@@ -74,13 +74,26 @@ def pipeline_from_logits(inp, logits, flags=0, fused=True):
     M.moe_permute(s, b.idx, inp["x"], b.counts, b.offsets, b.slot_pos, b.perm_token, b.x_perm,
                   b.n_kept, b.status, b.ws)
     W13 = M.moe_pack_w13(s, inp["W1"], inp["W3"])
+    shared = None
+    if w.d_ff_shared:
+        # the shared expert through the same calls: one group of all T rows, unweighted
+        ss = M.make_shape(w.T, w.d, w.d_ff_shared, 1, 1)
+        W13s = M.moe_pack_w13(ss, inp["W1s"][None].contiguous(), inp["W3s"][None].contiguous())
+        offs = torch.tensor([0, w.T], dtype=torch.int32, device=inp["x"].device)
+        shared = torch.empty(w.T, w.d, dtype=torch.float32, device=inp["x"].device)
+        M.moe_expert_ffn(ss, inp["x"], offs, W13s, inp["W2s"][None].contiguous(), None, None, None,
+                         shared, None, b.status, M.alloc_workspace(ss, inp["x"].device))
     if fused:
+        if shared is not None:
+            b.out.copy_(shared)
+        else:
+            b.out.zero_()
         M.moe_expert_ffn(s, b.x_perm, b.offsets, W13, inp["W2"], b.perm_token, b.slot_pos, b.w,
                          None, b.out, b.status, b.ws)
     else:
         M.moe_expert_ffn(s, b.x_perm, b.offsets, W13, inp["W2"], None, None, None, b.y_perm, None,
                          b.status, b.ws)
-        M.moe_combine(s, b.y_perm, b.slot_pos, b.w, None, b.out)
+        M.moe_combine(s, b.y_perm, b.slot_pos, b.w, shared, b.out)
     torch.cuda.synchronize()
     return b
 
