@@ -23,7 +23,7 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libmoe.so")
 SOURCES = ["dispatch.cu", "gemm_simt.cu", "gemm_tc.cu", "decode.cu", "moe_api.cu"]
-HEADERS = ["common.cuh", "internal.h"]
+HEADERS = ["common.cuh", "internal.h", "topk.cuh"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC",
