@@ -206,6 +206,28 @@ MOE_API int moe_forward_host(const moe_shape_t *shape, const moe_bf16_t *x_host,
                      const moe_bf16_t *W13_shared, const moe_bf16_t *W2_shared, float *out_host,
                      uint32_t *status, void *ws, size_t ws_bytes, moe_stream_t stream);
 
+/* moe_permute without a workspace, for callers that cannot allocate device
+ * memory: code running while a stream is captured in global capture mode
+ * (where cudaMalloc is refused), engines that reserve all device memory for
+ * their own pool, and paths that cannot pay for cudaMalloc/cudaFree (cudaFree
+ * synchronises the device). The pages have no counterpart of this call.
+ *   Arguments, outputs and results are those of moe_permute (bit-identical),
+ *   minus ws/ws_bytes: the scratch is one fixed 4 MiB array inside the
+ *   library's device image, held on every GPU that loads the library until
+ *   the process exits. Shapes whose scratch does not fit return
+ *   MOE_ERR_UNSUPPORTED and launch nothing; every shape with T*k <= 262144
+ *   and T <= 262144 fits.
+ *   The call allocates nothing. Its first call on a device looks up the
+ *   array's device address (cudaGetSymbolAddress, with that device current);
+ *   make that first call before any stream capture.
+ *   All calls share the one array and each call clears what must start at
+ *   zero, so calls that overlap on the GPU (other streams, other host threads)
+ *   race and corrupt each other's results: order them on one stream. */
+MOE_API int moe_permute_static(const moe_shape_t *shape, const int32_t *topk_idx,
+                               const moe_bf16_t *x, int32_t *expert_counts, int32_t *expert_offsets,
+                               int32_t *slot_pos, int32_t *perm_token, moe_bf16_t *x_perm,
+                               int32_t *n_kept, uint32_t *status, moe_stream_t stream);
+
 /* ---- Instrumentation (computes nothing; for measurement and tests). ---- */
 
 /* Stages of moe_forward timed by the profiler below. */

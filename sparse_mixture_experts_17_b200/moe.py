@@ -78,6 +78,7 @@ _SIGS = {
     "moe_combine": ([_SHP, _P, _P, _P, _P, _P, _P], ctypes.c_int),
     "moe_forward": ([_SHP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P], ctypes.c_int),
     "moe_forward_host": ([_SHP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P], ctypes.c_int),
+    "moe_permute_static": ([_SHP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P], ctypes.c_int),
     "moe_kernel_launches": ([], ctypes.c_uint64),
     "moe_profile_enable": ([ctypes.c_int], ctypes.c_int),
     "moe_profile_read": ([_P, _P, ctypes.c_int], ctypes.c_int),
@@ -185,6 +186,17 @@ def moe_permute(shape, topk_idx, x, expert_counts, expert_offsets, slot_pos, per
         _ptr(slot_pos, I32, "slot_pos"), _ptr(perm_token, I32, "perm_token"),
         _ptr(x_perm, BF16, "x_perm"), _ptr(n_kept, I32, "n_kept"), _ptr(status, U32, "status"),
         _ptr(ws, name="ws"), ws.numel(), _stream(stream)))
+
+
+def moe_permute_static(shape, topk_idx, x, expert_counts, expert_offsets, slot_pos, perm_token,
+                       x_perm, n_kept, status, stream=None):
+    """moe_permute with the library's own fixed scratch: allocates nothing."""
+    _check("moe_permute_static", lib().moe_permute_static(
+        ctypes.byref(shape), _ptr(topk_idx, I32, "topk_idx"), _ptr(x, BF16, "x"),
+        _ptr(expert_counts, I32, "expert_counts"), _ptr(expert_offsets, I32, "expert_offsets"),
+        _ptr(slot_pos, I32, "slot_pos"), _ptr(perm_token, I32, "perm_token"),
+        _ptr(x_perm, BF16, "x_perm"), _ptr(n_kept, I32, "n_kept"), _ptr(status, U32, "status"),
+        _stream(stream)))
 
 
 def moe_expert_ffn(shape, x_perm, expert_offsets, W13, W2, perm_token, slot_pos, topk_w, y_perm,
