@@ -23,6 +23,7 @@ import statistics
 import subprocess
 import sys
 import time
+from dataclasses import replace
 
 import torch
 import torch.distributed as dist
@@ -223,6 +224,9 @@ def run_ours(a, world, rank, local):
     w = I.WORKLOADS[a.workload]
     if a.tokens:
         w = w.with_T(a.tokens)
+    if a.experts:
+        w = replace(w, E=a.experts, name=f"{w.name}@E{a.experts}",
+                    capacity=I.capacity_for(w.T, w.k, a.experts) if w.capacity else 0)
     inp = I.make_inputs(w, dev, seed=0)
     layer = M.MoeLayer(inp)
     x = inp["x"]
@@ -413,6 +417,7 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds per oracle sample")
     ap.add_argument("--tokens", type=int, default=0, help="override T (profiling runs)")
+    ap.add_argument("--experts", type=int, default=0, help="override E (profiling runs)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end run")
     a = ap.parse_args(argv)
     if a.warmup < 3 and a.impl == "ours":

@@ -74,14 +74,19 @@ enum {
                                         T <= MOE_DECODE_MAX_T (else MOE_ERR_UNSUPPORTED) */
     MOE_FLAG_SIMT_FFN = 1 << 3,      /* expert GEMMs on CUDA cores (slow debugging path that
                                         cross-checks the tensor-core kernels) */
-    MOE_FLAG_HOST_IO = 1 << 4        /* workspace also holds device staging for x and out,
+    MOE_FLAG_HOST_IO = 1 << 4,       /* workspace also holds device staging for x and out,
                                         as moe_forward_host needs */
+    MOE_FLAG_GEMM_1SM = 1 << 5,      /* tensor-core GEMMs: always the single-SM kernel */
+    MOE_FLAG_GEMM_2SM = 1 << 6       /* tensor-core GEMMs: the 2-SM pair kernel (256 x 256
+                                        tiles, cta_group::2) wherever the output width is a
+                                        multiple of 256 (default: the single-SM kernel) */
 };
 
 #define MOE_MAX_E 256
 #define MOE_MAX_K 16
-#define MOE_DECODE_MAX_T 16
-#define MOE_DECODE_DEFAULT_T 16
+#define MOE_DECODE_MAX_T 16     /* largest T the decode kernels accept */
+#define MOE_DECODE_DEFAULT_T 2  /* moe_forward takes them for T <= this (measured crossover
+                                   with the tensor-core chain on the Mixtral shape) */
 
 /* Layer shape. Requirements (else MOE_ERR_INVALID_ARG):
  *   0 <= T <= 2^24; 1 <= E <= MOE_MAX_E; 1 <= k <= min(E, MOE_MAX_K);
@@ -188,7 +193,8 @@ MOE_API int moe_combine(const moe_shape_t *shape, const float *y_perm, const int
  * experts"; "perf(moe): route granite-4.0-h single-token MoE through the fused
  * kernel"); larger T takes router -> top-k -> histogram -> permute -> grouped
  * tensor-core GEMMs with the SwiGLU and the weighted combine in their
- * epilogues. Device errors: NONFINITE, BAD_EXPERT, TIMEOUT. */
+ * epilogues, which also read only the chosen experts (tiles exist only for
+ * experts with rows). Device errors: NONFINITE, BAD_EXPERT, TIMEOUT. */
 MOE_API int moe_forward(const moe_shape_t *shape, const moe_bf16_t *x, const moe_bf16_t *Wg,
                 const float *bias, const moe_bf16_t *W13, const moe_bf16_t *W2,
                 const moe_bf16_t *W13_shared, const moe_bf16_t *W2_shared, float *out,

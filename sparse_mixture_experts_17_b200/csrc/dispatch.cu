@@ -192,20 +192,21 @@ __device__ __forceinline__ int block_excl_scan_256(int v, int *s_warp, int *tota
     return r;
 }
 
-// Writes the grouped-GEMM m-tile list for kept counts in s_kept[E]:
-// expert e contributes ceil(kept/128) tiles starting at rows offsets[e] + 128 i.
+// Writes the grouped-GEMM m-tile list for kept counts in s_kept[E]: expert e
+// contributes ceil(kept/tile_m) tiles starting at rows offsets[e] + tile_m i.
 __device__ void build_tiles(const int *s_kept, const int32_t *offsets_smem_or_global, int E,
-                            int32_t *mt_row0, int32_t *mt_group, int32_t *num_mt, int *s_warp)
+                            int tile_m, int32_t *mt_row0, int32_t *mt_group, int32_t *num_mt,
+                            int *s_warp)
 {
     const int tid = threadIdx.x;
     const int e = tid;
-    const int nt = (e < E) ? (s_kept[e] + kBlockM - 1) / kBlockM : 0;
+    const int nt = (e < E) ? (s_kept[e] + tile_m - 1) / tile_m : 0;
     int total;
     const int start = block_excl_scan_256(nt, s_warp, &total);
     if (e < E) {
         const int base = offsets_smem_or_global[e];
         for (int i = 0; i < nt; ++i) {
-            mt_row0[start + i] = base + i * kBlockM;
+            mt_row0[start + i] = base + i * tile_m;
             mt_group[start + i] = e;
         }
     }
@@ -226,7 +227,8 @@ __global__ void __launch_bounds__(256) k_hist_scan(
     const int32_t *__restrict__ idx, int T, int E, int k, int C, int32_t *chunk_counts,
     int32_t *__restrict__ rank_local, int32_t *counter, int32_t *__restrict__ counts,
     int32_t *__restrict__ offsets, int32_t *__restrict__ n_kept, int32_t *mt_row0,
-    int32_t *mt_group, int32_t *num_mt, uint32_t *status)
+    int32_t *mt_group, int32_t *num_mt, int32_t *mt2_row0, int32_t *mt2_group, int32_t *num_mt2,
+    uint32_t *status)
 {
     __shared__ uint32_t mask[8][MOE_MAX_E];
     __shared__ int32_t wpre[8][MOE_MAX_E];
@@ -325,7 +327,9 @@ __global__ void __launch_bounds__(256) k_hist_scan(
         *n_kept = total;
     }
     __syncthreads();
-    build_tiles(s_kept, s_off, E, mt_row0, mt_group, num_mt, s_warp);
+    build_tiles(s_kept, s_off, E, kBlockM, mt_row0, mt_group, num_mt, s_warp);
+    if (mt2_row0)
+        build_tiles(s_kept, s_off, E, 2 * kBlockM, mt2_row0, mt2_group, num_mt2, s_warp);
     if (tid == 0)
         *counter = 0;
 }
@@ -333,14 +337,15 @@ __global__ void __launch_bounds__(256) k_hist_scan(
 int launch_hist_scan(const moe_shape_t &s, const int32_t *idx, int32_t *chunk_counts,
                      int32_t *rank_local, int32_t *counter, int32_t *counts, int32_t *offsets,
                      int32_t *n_kept, int32_t *mt_row0, int32_t *mt_group, int32_t *num_mt,
-                     uint32_t *status, cudaStream_t st)
+                     int32_t *mt2_row0, int32_t *mt2_group, int32_t *num_mt2, uint32_t *status,
+                     cudaStream_t st)
 {
     const int nchunks = (s.T + kChunkTokens - 1) / kChunkTokens;
     if (nchunks == 0)
         return MOE_OK;
     k_hist_scan<<<nchunks, 256, 0, st>>>(idx, s.T, s.E, s.k, s.capacity, chunk_counts,
                                          rank_local, counter, counts, offsets, n_kept, mt_row0,
-                                         mt_group, num_mt, status);
+                                         mt_group, num_mt, mt2_row0, mt2_group, num_mt2, status);
     return launched();
 }
 
@@ -411,7 +416,9 @@ int launch_permute(const moe_shape_t &s, const int32_t *idx, const int32_t *chun
 // ---------------------------------------------------------------- tile list from offsets
 __global__ void __launch_bounds__(256) k_tiles_from_offsets(const int32_t *__restrict__ offsets,
                                                             int E, int32_t *mt_row0,
-                                                            int32_t *mt_group, int32_t *num_mt)
+                                                            int32_t *mt_group, int32_t *num_mt,
+                                                            int32_t *mt2_row0, int32_t *mt2_group,
+                                                            int32_t *num_mt2)
 {
     __shared__ int s_kept[MOE_MAX_E];
     __shared__ int s_off[MOE_MAX_E];
@@ -420,13 +427,17 @@ __global__ void __launch_bounds__(256) k_tiles_from_offsets(const int32_t *__res
     s_kept[e] = (e < E) ? max(0, offsets[e + 1] - offsets[e]) : 0;
     s_off[e] = (e < E) ? offsets[e] : 0;
     __syncthreads();
-    build_tiles(s_kept, s_off, E, mt_row0, mt_group, num_mt, s_warp);
+    build_tiles(s_kept, s_off, E, kBlockM, mt_row0, mt_group, num_mt, s_warp);
+    if (mt2_row0)
+        build_tiles(s_kept, s_off, E, 2 * kBlockM, mt2_row0, mt2_group, num_mt2, s_warp);
 }
 
 int launch_tiles_from_offsets(const moe_shape_t &s, const int32_t *offsets, int32_t *mt_row0,
-                              int32_t *mt_group, int32_t *num_mt, cudaStream_t st)
+                              int32_t *mt_group, int32_t *num_mt, int32_t *mt2_row0,
+                              int32_t *mt2_group, int32_t *num_mt2, cudaStream_t st)
 {
-    k_tiles_from_offsets<<<1, 256, 0, st>>>(offsets, s.E, mt_row0, mt_group, num_mt);
+    k_tiles_from_offsets<<<1, 256, 0, st>>>(offsets, s.E, mt_row0, mt_group, num_mt, mt2_row0,
+                                            mt2_group, num_mt2);
     return launched();
 }
 

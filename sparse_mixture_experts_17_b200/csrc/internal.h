@@ -29,11 +29,12 @@ struct WsLayout {
     size_t chunk_counts, rank_local;
     size_t slot_pos, perm_token;
     size_t mt_row0, mt_group;
+    size_t mt2_row0, mt2_group, num_mt2;   // 256-row tiles of the 2-SM GEMM
     size_t x_perm, H, H_shared, Y;
     size_t dec_H;
     size_t x_stage, out_stage;
     size_t total;
-    int nchunks, max_mt;
+    int nchunks, max_mt, max_mt2;
 };
 
 WsLayout ws_layout(const moe_shape_t &s);
@@ -43,16 +44,19 @@ int launch_router_simt(const moe_shape_t &s, const uint16_t *x, const uint16_t *
                        const float *bias, float *logits, cudaStream_t st);
 int launch_topk(const moe_shape_t &s, const float *logits, int32_t *idx, float *w,
                 int32_t *counter_to_zero, uint32_t *status, cudaStream_t st);
+// Also writes the 256-row m-tile list of the 2-SM GEMM when mt2_row0 is non-NULL.
 int launch_hist_scan(const moe_shape_t &s, const int32_t *idx, int32_t *chunk_counts,
                      int32_t *rank_local, int32_t *counter, int32_t *counts, int32_t *offsets,
                      int32_t *n_kept, int32_t *mt_row0, int32_t *mt_group, int32_t *num_mt,
-                     uint32_t *status, cudaStream_t st);
+                     int32_t *mt2_row0, int32_t *mt2_group, int32_t *num_mt2, uint32_t *status,
+                     cudaStream_t st);
 int launch_permute(const moe_shape_t &s, const int32_t *idx, const int32_t *chunk_base,
                    const int32_t *rank_local, const int32_t *offsets, const uint16_t *x,
                    int32_t *slot_pos, int32_t *perm_token, uint16_t *x_perm, float *out_zero,
                    cudaStream_t st);
 int launch_tiles_from_offsets(const moe_shape_t &s, const int32_t *offsets, int32_t *mt_row0,
-                              int32_t *mt_group, int32_t *num_mt, cudaStream_t st);
+                              int32_t *mt_group, int32_t *num_mt, int32_t *mt2_row0,
+                              int32_t *mt2_group, int32_t *num_mt2, cudaStream_t st);
 int launch_combine(const moe_shape_t &s, const float *y_perm, const int32_t *slot_pos,
                    const float *topk_w, const float *shared_out, float *out, cudaStream_t st);
 int launch_pack_w13(int E, int d_ff, int d, const uint16_t *W1, const uint16_t *W3,
@@ -94,6 +98,8 @@ struct GemmArgs {
     const float *bias;
     int n_valid;
     uint32_t *status;
+    // 1: 2-SM pair kernel (256 x 256 tiles; the m-tile list must hold 256-row tiles)
+    int pair;
 };
 
 int launch_gemm_tc(const GemmArgs &g, cudaStream_t st);

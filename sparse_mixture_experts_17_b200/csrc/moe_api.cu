@@ -103,6 +103,7 @@ WsLayout ws_layout(const moe_shape_t &s)
     const size_t T = s.T, k = s.k, E = s.E, N = T * k;
     L.nchunks = (int)((T + kChunkTokens - 1) / kChunkTokens);
     L.max_mt = (int)((N + kBlockM - 1) / kBlockM + E);
+    L.max_mt2 = (int)((N + 2 * kBlockM - 1) / (2 * kBlockM) + E);
     L.logits = take(T * E * 4);
     L.topk_idx = take(N * 4);
     L.topk_w = take(N * 4);
@@ -117,6 +118,9 @@ WsLayout ws_layout(const moe_shape_t &s)
     L.perm_token = take(N * 4);
     L.mt_row0 = take((size_t)L.max_mt * 4);
     L.mt_group = take((size_t)L.max_mt * 4);
+    L.mt2_row0 = take((size_t)L.max_mt2 * 4);
+    L.mt2_group = take((size_t)L.max_mt2 * 4);
+    L.num_mt2 = take(4);
     L.x_perm = take(N * s.d * 2);
     L.H = take(N * s.d_ff * 2);
     L.H_shared = take(s.d_ff_shared ? T * s.d_ff_shared * 2 : 0);
@@ -145,7 +149,32 @@ static int check_ws(const moe_shape_t &s, void *ws, size_t ws_bytes, WsLayout &L
 
 static int run_gemm(const moe_shape_t &s, const GemmArgs &g, cudaStream_t st)
 {
-    return (s.flags & MOE_FLAG_SIMT_FFN) ? launch_gemm_simt(g, st) : launch_gemm_tc(g, st);
+    if (s.flags & MOE_FLAG_SIMT_FFN) {
+        GemmArgs g1 = g;
+        g1.pair = 0;
+        return launch_gemm_simt(g1, st);
+    }
+    return launch_gemm_tc(g, st);
+}
+
+// The 2-SM pair kernel (256-row tiles) is taken only on request: it moves a
+// third less operand data per FLOP, but measured on the power-capped B200 the
+// single-SM kernel finishes sooner. Output widths must be multiples of 256.
+static bool use_pair(const moe_shape_t &s, long long avg_rows, int n_out)
+{
+    if ((s.flags & (MOE_FLAG_SIMT_FFN | MOE_FLAG_GEMM_1SM)) || n_out % 256 != 0)
+        return false;
+    return (s.flags & MOE_FLAG_GEMM_2SM) != 0;
+}
+
+// Point a routed GEMM at the m-tile list of its engine.
+static void set_tiles(GemmArgs &g, const WsLayout &L, void *ws, bool pair)
+{
+    g.pair = pair ? 1 : 0;
+    g.mt_row0 = reinterpret_cast<int32_t *>(static_cast<char *>(ws) + (pair ? L.mt2_row0 : L.mt_row0));
+    g.mt_group = reinterpret_cast<int32_t *>(static_cast<char *>(ws) + (pair ? L.mt2_group : L.mt_group));
+    g.num_mt_dev = reinterpret_cast<int32_t *>(static_cast<char *>(ws) + (pair ? L.num_mt2 : L.num_mt));
+    g.max_mt = pair ? L.max_mt2 : L.max_mt;
 }
 
 static GemmArgs gemm_base()
@@ -173,10 +202,8 @@ static int expert_ffn_core(const moe_shape_t &s, const WsLayout &L, void *ws,
     g.K = s.d;
     g.N = 2 * s.d_ff;
     g.b_rows_per_group = 2 * s.d_ff;
-    g.mt_row0 = at<int32_t>(ws, L.mt_row0);
-    g.mt_group = at<int32_t>(ws, L.mt_group);
-    g.num_mt_dev = at<int32_t>(ws, L.num_mt);
-    g.max_mt = L.max_mt;
+    const long long avg_rows = N / s.E;
+    set_tiles(g, L, ws, use_pair(s, avg_rows, g.N));
     g.seg_offsets = offsets;
     g.out = H;
     g.ldo = s.d_ff;
@@ -195,6 +222,7 @@ static int expert_ffn_core(const moe_shape_t &s, const WsLayout &L, void *ws,
     g.N = s.d;
     g.b_rows_per_group = s.d;
     g.ldo = s.d;
+    set_tiles(g, L, ws, use_pair(s, avg_rows, g.N));
     if (y_perm) {
         g.mode = EPI_STORE_F32;
         g.out = y_perm;
@@ -216,8 +244,10 @@ static int shared_expert(const moe_shape_t &s, const WsLayout &L, void *ws, cons
                          cudaStream_t st)
 {
     uint16_t *Hs = at<uint16_t>(ws, L.H_shared);
-    const int mt = (s.T + kBlockM - 1) / kBlockM;
+    const bool pair1 = use_pair(s, s.T, 2 * s.d_ff_shared);
+    const int mt = (s.T + (pair1 ? 256 : kBlockM) - 1) / (pair1 ? 256 : kBlockM);
     GemmArgs g = gemm_base();
+    g.pair = pair1 ? 1 : 0;
     g.mode = EPI_SWIGLU;
     g.A = x;
     g.a_rows = s.T;
@@ -244,6 +274,9 @@ static int shared_expert(const moe_shape_t &s, const WsLayout &L, void *ws, cons
     g.b_rows_per_group = s.d;
     g.out = out;
     g.ldo = s.d;
+    const bool pair2 = use_pair(s, s.T, s.d);
+    g.pair = pair2 ? 1 : 0;
+    g.num_mt_host = g.max_mt = (s.T + (pair2 ? 256 : kBlockM) - 1) / (pair2 ? 256 : kBlockM);
     return run_gemm(s, g, st);
 }
 
@@ -330,7 +363,9 @@ static int forward_impl(const moe_shape_t &s, const WsLayout &L, void *ws, const
         StageMark m(MOE_STAGE_HIST, st);
         rc = launch_hist_scan(s, idx, chunk, rank, counter, counts, offsets,
                               at<int32_t>(ws, L.n_kept), at<int32_t>(ws, L.mt_row0),
-                              at<int32_t>(ws, L.mt_group), at<int32_t>(ws, L.num_mt), status, st);
+                              at<int32_t>(ws, L.mt_group), at<int32_t>(ws, L.num_mt),
+                              at<int32_t>(ws, L.mt2_row0), at<int32_t>(ws, L.mt2_group),
+                              at<int32_t>(ws, L.num_mt2), status, st);
     }
     if (rc)
         return rc;
@@ -502,7 +537,9 @@ int moe_permute(const moe_shape_t *shape, const int32_t *topk_idx, const moe_bf1
     int32_t *rank = at<int32_t>(ws, L.rank_local);
     rc = launch_hist_scan(s, topk_idx, chunk, rank, counter, expert_counts, expert_offsets,
                           n_kept ? n_kept : at<int32_t>(ws, L.n_kept), at<int32_t>(ws, L.mt_row0),
-                          at<int32_t>(ws, L.mt_group), at<int32_t>(ws, L.num_mt), status, st);
+                          at<int32_t>(ws, L.mt_group), at<int32_t>(ws, L.num_mt),
+                          at<int32_t>(ws, L.mt2_row0), at<int32_t>(ws, L.mt2_group),
+                          at<int32_t>(ws, L.num_mt2), status, st);
     if (rc)
         return rc;
     return launch_permute(s, topk_idx, chunk, rank, expert_offsets, x, slot_pos, perm_token,
@@ -532,7 +569,9 @@ int moe_expert_ffn(const moe_shape_t *shape, const moe_bf16_t *x_perm,
         return MOE_OK;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     rc = launch_tiles_from_offsets(s, expert_offsets, at<int32_t>(ws, L.mt_row0),
-                                   at<int32_t>(ws, L.mt_group), at<int32_t>(ws, L.num_mt), st);
+                                   at<int32_t>(ws, L.mt_group), at<int32_t>(ws, L.num_mt),
+                                   at<int32_t>(ws, L.mt2_row0), at<int32_t>(ws, L.mt2_group),
+                                   at<int32_t>(ws, L.num_mt2), st);
     if (rc)
         return rc;
     return expert_ffn_core(s, L, ws, x_perm, expert_offsets, W13, W2, perm_token, slot_pos, topk_w,

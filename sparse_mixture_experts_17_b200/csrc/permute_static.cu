@@ -123,7 +123,8 @@ extern "C" int moe_permute_static(const moe_shape_t *shape, const int32_t *topk_
                           n_kept ? n_kept : reinterpret_cast<int32_t *>(base + L.n_kept),
                           reinterpret_cast<int32_t *>(base + L.mt_row0),
                           reinterpret_cast<int32_t *>(base + L.mt_group),
-                          reinterpret_cast<int32_t *>(base + L.num_mt), status, st);
+                          reinterpret_cast<int32_t *>(base + L.num_mt), nullptr, nullptr,
+                          nullptr, status, st);
     if (rc)
         return rc;
     return launch_permute(s, topk_idx, chunk, rank, expert_offsets, x, slot_pos, perm_token,

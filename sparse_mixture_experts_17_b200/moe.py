@@ -32,6 +32,8 @@ MOE_FLAG_FORCE_PREFILL = 1 << 1
 MOE_FLAG_FORCE_DECODE = 1 << 2
 MOE_FLAG_SIMT_FFN = 1 << 3
 MOE_FLAG_HOST_IO = 1 << 4
+MOE_FLAG_GEMM_1SM = 1 << 5
+MOE_FLAG_GEMM_2SM = 1 << 6
 
 MOE_MAX_E = 256
 MOE_MAX_K = 16

@@ -148,6 +148,8 @@ def test_p3_worked_example_on_gpu():
 FFN_CASES = [
     # name, T, d, d_ff, E, k, capacity, zipf
     ("ragged8", 700, 256, 384, 8, 2, 0, 0.0),
+    ("long_groups", 2600, 512, 512, 4, 2, 0, 0.0),      # > 1024 rows per expert, ragged tails
+    ("peer_tail", 1100, 256, 256, 8, 1, 0, 0.0),         # segments just past 128 rows
     ("cap16", 1500, 1024, 512, 16, 4, 400, 1.0),
     ("d128", 300, 128, 256, 8, 2, 0, 0.0),
     ("many_tiles", 3000, 512, 640, 32, 4, 0, 0.8),
@@ -155,7 +157,8 @@ FFN_CASES = [
 
 
 @pytest.mark.parametrize("case", FFN_CASES, ids=lambda c: c[0])
-@pytest.mark.parametrize("flags", [0, M.MOE_FLAG_SIMT_FFN], ids=["tc", "simt"])
+@pytest.mark.parametrize("flags", [M.MOE_FLAG_GEMM_1SM, M.MOE_FLAG_GEMM_2SM, M.MOE_FLAG_SIMT_FFN],
+                         ids=["tc1", "tc2", "simt"])
 @pytest.mark.parametrize("fused", [True, False], ids=["fused", "yperm"])
 def test_expert_ffn_parity(case, flags, fused):
     name, T, d, d_ff, E, k, C, zipf = case
@@ -202,8 +205,9 @@ def _gap_ok(L64, k, margin):
 
 @pytest.mark.parametrize("case", FWD_CASES, ids=lambda c: c[0])
 @pytest.mark.parametrize("flags", [0, M.MOE_FLAG_DETERMINISTIC, M.MOE_FLAG_SIMT_FFN,
-                                   M.MOE_FLAG_FORCE_PREFILL],
-                         ids=["default", "det", "simt", "prefill"])
+                                   M.MOE_FLAG_FORCE_PREFILL, M.MOE_FLAG_GEMM_2SM,
+                                   M.MOE_FLAG_GEMM_2SM | M.MOE_FLAG_DETERMINISTIC],
+                         ids=["default", "det", "simt", "prefill", "tc2", "tc2det"])
 def test_forward_parity(case, flags):
     name, w = case
     inp = I.make_inputs(w, "cuda", seed=0)
@@ -244,18 +248,25 @@ def test_decode_mixtral_shape(T):
     layer = M.MoeLayer(inp)
     idx = torch.empty(T, w.k, dtype=torch.int32, device="cuda")
     logits = torch.empty(T, w.E, dtype=torch.float32, device="cuda")
-    out = layer.forward(inp["x"], logits_out=logits, topk_idx_out=idx)
+    # the decode kernels (streaming only the chosen experts' rows)
+    out = layer.forward(inp["x"], logits_out=logits, topk_idx_out=idx,
+                        flags=M.MOE_FLAG_FORCE_DECODE)
     torch.cuda.synchronize()
     assert int(layer.status.item()) == 0
     ref = O.forward(oi, logits=logits.cpu().numpy())   # routing: identical fp32 logits
     L64, _ = O.router_logits(oi["x"], oi["wg"], None)
     assert np.abs(logits.double().cpu().numpy() - L64).max() <= LOGIT_ABS
     assert (idx.cpu().numpy() == ref["idx"]).all()
-    assert_layer_close(out, ref["out"], f"decode T={T}")
-    # the tensor-core prefill chain on the same input agrees
+    assert_layer_close(out, ref["out"], f"decode kernels T={T}")
+    # the tensor-core chain (taken by default from T = 3 on) on the same input
     out_p = layer.forward(inp["x"], flags=M.MOE_FLAG_FORCE_PREFILL)
     torch.cuda.synchronize()
-    assert_layer_close(out_p, ref["out"], f"prefill chain T={T}")
+    assert_layer_close(out_p, ref["out"], f"tensor-core chain T={T}")
+    # the default choice is one of them, bit for bit (k = 2: the fp32 atomic
+    # combine adds two terms onto zero, which is order-independent)
+    out_def = layer.forward(inp["x"])
+    torch.cuda.synchronize()
+    assert torch.equal(out_def, out if T <= 2 else out_p)
 
 
 def test_decode_shared_many_experts():
@@ -311,7 +322,7 @@ def test_empty_batch_is_noop():
 
 # ---------------------------------------------------------------- graphs and host I/O
 
-@pytest.mark.parametrize("T", [4, 500])
+@pytest.mark.parametrize("T", [2, 4, 500])
 def test_cuda_graph_capture_replay(T):
     w = small_workload("graph", T, 256, 256, 16, 4, d_ff_shared=128, zipf_s=1.0)
     inp = I.make_inputs(w, "cuda", seed=5)
