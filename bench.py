@@ -370,16 +370,19 @@ def run_decode_set(M, w, layer, x, dev, stream, world, peaks):
         M.moe_profile_enable(False)
         st = M.moe_profile_read()
         ms = max_over_ranks(ms, world, dev)
-        k13 = st["dec_w13"][0] / st["dec_w13"][1]
-        k2 = st["dec_w2"][0] / st["dec_w2"][1]
+        dec = "dec_w13" in st
+        s13, s2 = (st["dec_w13"], st["dec_w2"]) if dec else (st["w13"], st["w2"])
+        k13 = s13[0] / s13[1]
+        k2 = s2[0] / s2[1]
         decode[f"T{T}"] = {
+            "path": "decode kernels" if dec else "tensor-core chain",
             "tokens_per_s": round(T * world / (ms / 1e3), 1), "ms_per_step": round(ms, 4),
             "unique_experts": U, "bytes_per_step": nbytes,
             "GB_s": round(nbytes / (ms / 1e3) / 1e9, 1),
             "frac_hbm_measured": round(nbytes / (ms / 1e3) / 1e9 / peaks["hbm_gbs"], 4),
             "frac_hbm_nominal_8000": round(nbytes / (ms / 1e3) / 1e9 / 8000.0, 4),
             "chosen_expert_GB_s_kernels": round(expert_bytes / ((k13 + k2) / 1e3) / 1e9, 1),
-            "dec_w13_GB_s": round(w13_bytes / (k13 / 1e3) / 1e9, 1),
+            "w13_kernel_GB_s": round(w13_bytes / (k13 / 1e3) / 1e9, 1),
             "stages_ms": {k: round(v[0] / v[1], 4) for k, v in st.items()}}
     return decode
 

@@ -143,8 +143,10 @@ __global__ void __launch_bounds__(256) k_dec_router(const uint16_t *__restrict__
     }
 }
 
-// Router and top-k in one CTA of 512 threads, for W_g up to kFusedRouteBytes:
-// warps stride over experts (lanes over d) into shared memory, then warp t
+// Router and top-k in one CTA of 512 threads, for W_g up to kFusedRouteBytes.
+// Work item = (expert e, slice of d): with E < 16 each expert's row is split
+// into 16/E slices so all 16 warps stream W_g; each lane keeps four 16-byte
+// loads in flight. Partial dot products meet in shared memory, then warp t
 // selects token t's experts.
 constexpr size_t kFusedRouteBytes = 256 * 1024;
 
@@ -156,32 +158,56 @@ __global__ void __launch_bounds__(512) k_dec_route(const uint16_t *__restrict__ 
                                                    int32_t *__restrict__ idx,
                                                    float *__restrict__ w, uint32_t *status)
 {
+    __shared__ float part[MAXT * 256];   // [t][e * S + slice], E * S <= 256
     __shared__ float sl[MAXT * MOE_MAX_E];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int nv = d / 8;
-    for (int e = warp; e < E; e += 16) {
+    const int S = E < 16 ? 16 / E : 1;
+    const int slice = (nv + S - 1) / S;
+    for (int item = warp; item < E * S; item += 16) {
+        const int e = item / S, sidx = item - e * S;
+        const int c0 = sidx * slice, c1 = min(nv, c0 + slice);
         float acc[MAXT];
 #pragma unroll
         for (int t = 0; t < MAXT; ++t)
             acc[t] = 0.f;
         const uint4 *wr = reinterpret_cast<const uint4 *>(Wg + (size_t)e * d);
-        for (int c = lane; c < nv; c += 32) {
-            const uint4 wv = ld_stream_v4(wr + c);
+        for (int cb = c0; cb < c1; cb += 128) {
+            uint4 wv[4];
 #pragma unroll
-            for (int t = 0; t < MAXT; ++t)
-                if (t < T)
-                    acc[t] = dot8(wv, __ldg(reinterpret_cast<const uint4 *>(x + (size_t)t * d) + c), acc[t]);
+            for (int i = 0; i < 4; ++i) {
+                const int c = cb + lane + 32 * i;
+                if (c < c1)
+                    wv[i] = ld_stream_v4(wr + c);
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int c = cb + lane + 32 * i;
+                if (c >= c1)
+                    continue;
+#pragma unroll
+                for (int t = 0; t < MAXT; ++t)
+                    if (t < T)
+                        acc[t] = dot8(wv[i], __ldg(reinterpret_cast<const uint4 *>(x + (size_t)t * d) + c), acc[t]);
+            }
         }
 #pragma unroll
         for (int t = 0; t < MAXT; ++t) {
             if (t < T) {
-                const float s = warp_sum(acc[t]) + (bias ? bias[e] : 0.f);
-                if (lane == 0) {
-                    sl[t * E + e] = s;
-                    logits[(size_t)t * E + e] = s;
-                }
+                const float v = warp_sum(acc[t]);
+                if (lane == 0)
+                    part[t * 256 + item] = v;
             }
         }
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < T * E; i += blockDim.x) {
+        const int t = i / E, e = i - t * E;
+        float v = bias ? bias[e] : 0.f;
+        for (int q = 0; q < S; ++q)
+            v += part[t * 256 + e * S + q];
+        sl[t * E + e] = v;
+        logits[(size_t)t * E + e] = v;
     }
     __syncthreads();
     if (warp < T)
@@ -319,20 +345,21 @@ __global__ void __launch_bounds__(256, (MAXT <= 2) ? 4 : 2)
                 wt[s] = (s < na) ? (shared ? 1.f : topk_w[a]) : 0.f;
             }
             const int nv = ff / 8;
+            constexpr int UNR = (MAXT <= 2) ? 8 : kDecUnroll;   // loads in flight per lane
             float pa[MAXT];
 #pragma unroll
             for (int s = 0; s < MAXT; ++s)
                 pa[s] = 0.f;
-            for (int cb = 0; cb < nv; cb += 32 * kDecUnroll) {
-                uint4 wv[kDecUnroll];
+            for (int cb = 0; cb < nv; cb += 32 * UNR) {
+                uint4 wv[UNR];
 #pragma unroll
-                for (int i = 0; i < kDecUnroll; ++i) {
+                for (int i = 0; i < UNR; ++i) {
                     const int ci = cb + lane + 32 * i;
                     if (ci < nv)
                         wv[i] = ld_stream_v4(wrow + ci);
                 }
 #pragma unroll
-                for (int i = 0; i < kDecUnroll; ++i) {
+                for (int i = 0; i < UNR; ++i) {
                     const int ci = cb + lane + 32 * i;
                     if (ci >= nv)
                         continue;

@@ -205,9 +205,12 @@ __device__ void build_tiles(const int *s_kept, const int32_t *offsets_smem_or_gl
     const int start = block_excl_scan_256(nt, s_warp, &total);
     if (e < E) {
         const int base = offsets_smem_or_global[e];
+        // a last tile of <= 64 rows is marked for the M = 64 MMA (128-row lists only)
+        const int rem = s_kept[e] - (nt - 1) * tile_m;
         for (int i = 0; i < nt; ++i) {
             mt_row0[start + i] = base + i * tile_m;
-            mt_group[start + i] = e;
+            const bool half = (tile_m == kBlockM) && (i == nt - 1) && rem <= 64;
+            mt_group[start + i] = e | (half ? kHalfTileBit : 0);
         }
     }
     if (tid == 0)

@@ -20,7 +20,7 @@ __global__ void __launch_bounds__(256) k_gemm_simt(const GemmArgs g)
     if (m_idx >= num_mt)
         return;
     const long long row0 = g.mt_row0 ? g.mt_row0[m_idx] : (long long)m_idx * BM;
-    const int grp = g.mt_group ? g.mt_group[m_idx] : 0;
+    const int grp = g.mt_group ? (g.mt_group[m_idx] & ~kHalfTileBit) : 0;
     const long long row_end = g.seg_offsets ? g.seg_offsets[grp + 1] : g.rows_valid;
     const int n0 = blockIdx.y * BN;   // output column (H column for SWIGLU)
     const long long bgrp = (long long)grp * g.b_rows_per_group;

@@ -217,7 +217,7 @@ __global__ void __launch_bounds__(192, 1)
                 int m_idx, n_idx;
                 tile_coords(tile, num_mt, p.n_tiles, p.group_m, m_idx, n_idx);
                 const int row0 = p.mt_row0 ? p.mt_row0[m_idx] : m_idx * C::BM;
-                const int grp = p.mt_group ? p.mt_group[m_idx] : 0;
+                const int grp = p.mt_group ? (p.mt_group[m_idx] & ~kHalfTileBit) : 0;
                 const int brow = grp * p.b_rows_per_group + n_idx * BN;
                 bool ok = true;
                 for (int kb = 0; kb < p.kblocks; ++kb, ++it) {
@@ -237,10 +237,15 @@ __global__ void __launch_bounds__(192, 1)
         }
     } else if (warp == 1) {
         if (lane == 0) {   // ---------------- MMA issuer
-            constexpr uint32_t IDESC = idesc_bf16_f32(128, BN);
+            constexpr uint32_t IDESC128 = idesc_bf16_f32(128, BN);
+            constexpr uint32_t IDESC64 = idesc_bf16_f32(64, BN);
             uint32_t it = 0, local = 0;
             for (long long tile = blockIdx.x; tile < total; tile += gridDim.x, ++local) {
                 const uint32_t b = local & 1u, aph = (local >> 1) & 1u;
+                int m_idx, n_idx;
+                tile_coords(tile, num_mt, p.n_tiles, p.group_m, m_idx, n_idx);
+                const bool half = p.mt_group && (p.mt_group[m_idx] & kHalfTileBit);
+                const uint32_t IDESC = half ? IDESC64 : IDESC128;
                 if (!mbar_wait(&tempty[b], aph ^ 1u, abort_flag, p.status))
                     break;
                 tc_fence_after();
@@ -274,14 +279,18 @@ __global__ void __launch_bounds__(192, 1)
             int m_idx, n_idx;
             tile_coords(tile, num_mt, p.n_tiles, p.group_m, m_idx, n_idx);
             const long long row0 = p.mt_row0 ? p.mt_row0[m_idx] : (long long)m_idx * C::BM;
-            const int grp = p.mt_group ? p.mt_group[m_idx] : 0;
+            const int gword = p.mt_group ? p.mt_group[m_idx] : 0;
+            const int grp = gword & ~kHalfTileBit;
+            const bool half = (gword & kHalfTileBit) != 0;
             const long long row_end = p.seg_offsets ? p.seg_offsets[grp + 1] : p.rows_valid;
             const uint32_t b = local & 1u, aph = (local >> 1) & 1u;
             if (!mbar_wait(&tfull[b], aph, abort_flag, p.status))
                 break;
             tc_fence_after();
-            const long long row = row0 + q * 32 + lane;
-            const bool valid = row < row_end;
+            // M = 128: tile row q*32 + lane sits in lane q*32 + lane. M = 64: tile
+            // row 16 q + l sits in lane 32 q + l (l < 16); lanes 16..31 hold nothing.
+            const long long row = row0 + (half ? q * 16 + lane : q * 32 + lane);
+            const bool valid = (!half || lane < 16) && row < row_end;
             const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + b * BN;
 
             epilogue_tile<BN, MODE>(p, tb, row, valid, n_idx);
@@ -378,7 +387,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
                 int m_idx, n_idx;
                 tile_coords(tile, num_mt, p.n_tiles, p.group_m, m_idx, n_idx);
                 const int row0 = (p.mt_row0 ? p.mt_row0[m_idx] : m_idx * 256) + 128 * (int)rank;
-                const int grp = p.mt_group ? p.mt_group[m_idx] : 0;
+                const int grp = p.mt_group ? (p.mt_group[m_idx] & ~kHalfTileBit) : 0;
                 const int brow = grp * p.b_rows_per_group + n_idx * BN + 128 * (int)rank;
                 bool ok = true;
                 for (int kb = 0; kb < p.kblocks; ++kb, ++it) {
@@ -437,7 +446,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
             int m_idx, n_idx;
             tile_coords(tile, num_mt, p.n_tiles, p.group_m, m_idx, n_idx);
             const long long row0 = (p.mt_row0 ? p.mt_row0[m_idx] : (long long)m_idx * 256) + 128 * rank;
-            const int grp = p.mt_group ? p.mt_group[m_idx] : 0;
+            const int grp = p.mt_group ? (p.mt_group[m_idx] & ~kHalfTileBit) : 0;
             const long long row_end = p.seg_offsets ? p.seg_offsets[grp + 1] : p.rows_valid;
             const uint32_t b = local & 1u, aph = (local >> 1) & 1u;
             if (!mbar_wait(&tfull[b], aph, abort_flag, p.status))

@@ -20,6 +20,9 @@ inline int launched()
 }
 
 constexpr int kBlockM = 128;      // rows of one grouped-GEMM m-tile
+// Bit of an m-tile's group entry marking a tail tile of at most 64 rows: the
+// single-SM tensor-core GEMM runs it with M = 64 MMAs (half the tensor time).
+constexpr int32_t kHalfTileBit = 1 << 30;
 constexpr int kChunkTokens = 256; // tokens per histogram chunk (one CTA)
 
 // Scratch layout inside the caller's workspace (byte offsets, 256-B aligned).
