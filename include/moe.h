@@ -79,7 +79,8 @@ enum {
     MOE_FLAG_GEMM_1SM = 1 << 5,      /* tensor-core GEMMs: always the single-SM kernel */
     MOE_FLAG_GEMM_2SM = 1 << 6       /* tensor-core GEMMs: the 2-SM pair kernel (256 x 256
                                         tiles, cta_group::2) wherever the output width is a
-                                        multiple of 256 (default: the single-SM kernel) */
+                                        multiple of 256 (default: the pair kernel for w2 when
+                                        experts average >= 1024 rows, else single-SM) */
 };
 
 #define MOE_MAX_E 256

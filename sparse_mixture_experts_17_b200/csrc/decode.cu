@@ -156,9 +156,12 @@ __global__ void __launch_bounds__(512) k_dec_route(const uint16_t *__restrict__ 
                                                    const float *__restrict__ bias, int T, int d,
                                                    int E, int k, float *__restrict__ logits,
                                                    int32_t *__restrict__ idx,
-                                                   float *__restrict__ w, uint32_t *status)
+                                                   float *__restrict__ w, int32_t *counter_to_zero,
+                                                   uint32_t *status)
 {
     __shared__ float part[MAXT * 256];   // [t][e * S + slice], E * S <= 256
+    if (counter_to_zero && threadIdx.x == 0)
+        *counter_to_zero = 0;   // re-arms the histogram's ticket for a following permute
     __shared__ float sl[MAXT * MOE_MAX_E];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int nv = d / 8;
@@ -419,31 +422,32 @@ bool dec_route_fusable(const moe_shape_t &s)
 template <int MAXT>
 static void launch_dec_route_t(const moe_shape_t &s, const uint16_t *x, const uint16_t *Wg,
                                const float *bias, float *logits, int32_t *idx, float *w,
-                               uint32_t *status, cudaStream_t st)
+                               int32_t *ctr, uint32_t *status, cudaStream_t st)
 {
     const int vpl = (s.E + 31) / 32;
     if (vpl <= 1)
-        k_dec_route<MAXT, 1><<<1, 512, 0, st>>>(x, Wg, bias, s.T, s.d, s.E, s.k, logits, idx, w, status);
+        k_dec_route<MAXT, 1><<<1, 512, 0, st>>>(x, Wg, bias, s.T, s.d, s.E, s.k, logits, idx, w, ctr, status);
     else if (vpl <= 2)
-        k_dec_route<MAXT, 2><<<1, 512, 0, st>>>(x, Wg, bias, s.T, s.d, s.E, s.k, logits, idx, w, status);
+        k_dec_route<MAXT, 2><<<1, 512, 0, st>>>(x, Wg, bias, s.T, s.d, s.E, s.k, logits, idx, w, ctr, status);
     else if (vpl <= 4)
-        k_dec_route<MAXT, 4><<<1, 512, 0, st>>>(x, Wg, bias, s.T, s.d, s.E, s.k, logits, idx, w, status);
+        k_dec_route<MAXT, 4><<<1, 512, 0, st>>>(x, Wg, bias, s.T, s.d, s.E, s.k, logits, idx, w, ctr, status);
     else
-        k_dec_route<MAXT, 8><<<1, 512, 0, st>>>(x, Wg, bias, s.T, s.d, s.E, s.k, logits, idx, w, status);
+        k_dec_route<MAXT, 8><<<1, 512, 0, st>>>(x, Wg, bias, s.T, s.d, s.E, s.k, logits, idx, w, ctr, status);
 }
 
 int launch_dec_route(const moe_shape_t &s, const uint16_t *x, const uint16_t *Wg,
-                     const float *bias, float *logits, int32_t *idx, float *w, uint32_t *status,
-                     cudaStream_t st)
+                     const float *bias, float *logits, int32_t *idx, float *w,
+                     int32_t *counter_to_zero, uint32_t *status, cudaStream_t st)
 {
     if (s.T == 0)
         return MOE_OK;
+    int32_t *c = counter_to_zero;
     switch (maxt_for(s.T)) {
-    case 1: launch_dec_route_t<1>(s, x, Wg, bias, logits, idx, w, status, st); break;
-    case 2: launch_dec_route_t<2>(s, x, Wg, bias, logits, idx, w, status, st); break;
-    case 4: launch_dec_route_t<4>(s, x, Wg, bias, logits, idx, w, status, st); break;
-    case 8: launch_dec_route_t<8>(s, x, Wg, bias, logits, idx, w, status, st); break;
-    default: launch_dec_route_t<16>(s, x, Wg, bias, logits, idx, w, status, st); break;
+    case 1: launch_dec_route_t<1>(s, x, Wg, bias, logits, idx, w, c, status, st); break;
+    case 2: launch_dec_route_t<2>(s, x, Wg, bias, logits, idx, w, c, status, st); break;
+    case 4: launch_dec_route_t<4>(s, x, Wg, bias, logits, idx, w, c, status, st); break;
+    case 8: launch_dec_route_t<8>(s, x, Wg, bias, logits, idx, w, c, status, st); break;
+    default: launch_dec_route_t<16>(s, x, Wg, bias, logits, idx, w, c, status, st); break;
     }
     return launched();
 }

@@ -115,8 +115,8 @@ int launch_dec_router(const moe_shape_t &s, const uint16_t *x, const uint16_t *W
 // Router + top-k in one single-CTA launch (small T and small W_g only).
 bool dec_route_fusable(const moe_shape_t &s);
 int launch_dec_route(const moe_shape_t &s, const uint16_t *x, const uint16_t *Wg,
-                     const float *bias, float *logits, int32_t *idx, float *w, uint32_t *status,
-                     cudaStream_t st);
+                     const float *bias, float *logits, int32_t *idx, float *w,
+                     int32_t *counter_to_zero, uint32_t *status, cudaStream_t st);
 int launch_dec_w13(const moe_shape_t &s, const uint16_t *x, const int32_t *topk_idx,
                    const uint16_t *W13, const uint16_t *W13s, uint16_t *Hdec, uint32_t *status,
                    cudaStream_t st);

@@ -157,14 +157,18 @@ static int run_gemm(const moe_shape_t &s, const GemmArgs &g, cudaStream_t st)
     return launch_gemm_tc(g, st);
 }
 
-// The 2-SM pair kernel (256-row tiles) is taken only on request: it moves a
-// third less operand data per FLOP, but measured on the power-capped B200 the
-// single-SM kernel finishes sooner. Output widths must be multiples of 256.
-static bool use_pair(const moe_shape_t &s, long long avg_rows, int n_out)
+// Engine choice. The 2-SM pair kernel (256-row tiles) moves a third less
+// operand data per FLOP. In interleaved measurements on the power-capped B200
+// it is 3-5% faster on the long-K w2 GEMM when experts hold >= 1024 rows, and
+// no faster on w1/w3, so by default only w2 takes it. Short groups would pad
+// up to 255 rows per tile. Output widths must be multiples of 256.
+static bool use_pair(const moe_shape_t &s, long long avg_rows, int n_out, bool is_w2)
 {
     if ((s.flags & (MOE_FLAG_SIMT_FFN | MOE_FLAG_GEMM_1SM)) || n_out % 256 != 0)
         return false;
-    return (s.flags & MOE_FLAG_GEMM_2SM) != 0;
+    if (s.flags & MOE_FLAG_GEMM_2SM)
+        return true;
+    return is_w2 && avg_rows >= 1024;
 }
 
 // Point a routed GEMM at the m-tile list of its engine.
@@ -203,7 +207,7 @@ static int expert_ffn_core(const moe_shape_t &s, const WsLayout &L, void *ws,
     g.N = 2 * s.d_ff;
     g.b_rows_per_group = 2 * s.d_ff;
     const long long avg_rows = N / s.E;
-    set_tiles(g, L, ws, use_pair(s, avg_rows, g.N));
+    set_tiles(g, L, ws, use_pair(s, avg_rows, g.N, false));
     g.seg_offsets = offsets;
     g.out = H;
     g.ldo = s.d_ff;
@@ -222,7 +226,7 @@ static int expert_ffn_core(const moe_shape_t &s, const WsLayout &L, void *ws,
     g.N = s.d;
     g.b_rows_per_group = s.d;
     g.ldo = s.d;
-    set_tiles(g, L, ws, use_pair(s, avg_rows, g.N));
+    set_tiles(g, L, ws, use_pair(s, avg_rows, g.N, true));
     if (y_perm) {
         g.mode = EPI_STORE_F32;
         g.out = y_perm;
@@ -244,7 +248,7 @@ static int shared_expert(const moe_shape_t &s, const WsLayout &L, void *ws, cons
                          cudaStream_t st)
 {
     uint16_t *Hs = at<uint16_t>(ws, L.H_shared);
-    const bool pair1 = use_pair(s, s.T, 2 * s.d_ff_shared);
+    const bool pair1 = use_pair(s, s.T, 2 * s.d_ff_shared, false);
     const int mt = (s.T + (pair1 ? 256 : kBlockM) - 1) / (pair1 ? 256 : kBlockM);
     GemmArgs g = gemm_base();
     g.pair = pair1 ? 1 : 0;
@@ -274,7 +278,7 @@ static int shared_expert(const moe_shape_t &s, const WsLayout &L, void *ws, cons
     g.b_rows_per_group = s.d;
     g.out = out;
     g.ldo = s.d;
-    const bool pair2 = use_pair(s, s.T, s.d);
+    const bool pair2 = use_pair(s, s.T, s.d, true);
     g.pair = pair2 ? 1 : 0;
     g.num_mt_host = g.max_mt = (s.T + (pair2 ? 256 : kBlockM) - 1) / (pair2 ? 256 : kBlockM);
     return run_gemm(s, g, st);
@@ -323,9 +327,9 @@ static int forward_impl(const moe_shape_t &s, const WsLayout &L, void *ws, const
     const bool decode = force_dec || (!force_pre && s.T <= MOE_DECODE_DEFAULT_T);
     int rc;
     int32_t *counter = at<int32_t>(ws, L.counter);
-    if (decode && dec_route_fusable(s)) {
+    if (dec_route_fusable(s)) {
         StageMark m(MOE_STAGE_ROUTER, st);   // router and top-k in one launch
-        rc = launch_dec_route(s, x, Wg, bias, logits, idx, w, status, st);
+        rc = launch_dec_route(s, x, Wg, bias, logits, idx, w, counter, status, st);
     } else {
         {
             StageMark m(MOE_STAGE_ROUTER, st);
@@ -500,7 +504,7 @@ int moe_route(const moe_shape_t *shape, const moe_bf16_t *x, const moe_bf16_t *W
         return MOE_OK;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (x && dec_route_fusable(s))
-        return launch_dec_route(s, x, Wg, bias, logits, topk_idx, topk_w, status, st);
+        return launch_dec_route(s, x, Wg, bias, logits, topk_idx, topk_w, nullptr, status, st);
     if (x && (rc = router(s, x, Wg, bias, logits, status, st)))
         return rc;
     return launch_topk(s, logits, topk_idx, topk_w, nullptr, status, st);
