@@ -250,6 +250,14 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N)
            | ((uint32_t)(M >> 4) << 24);  // M / 16
 }
 
+// ------------------------------------------------------------------ programmatic dependent launch
+// A kernel launched with programmatic stream serialization may start while
+// its predecessor in the stream is still running; it must call pdl_wait()
+// before touching anything the predecessor writes. pdl_trigger() lets the
+// successor's CTAs be scheduled early. Both are no-ops without the attribute.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ------------------------------------------------------------------ CTA pairs (cta_group::2)
 // A cluster of two CTAs on one TPC shares one MMA: the leader (rank 0) issues
 // it, each CTA holds half of A (its 128 rows) and half of B in its own shared

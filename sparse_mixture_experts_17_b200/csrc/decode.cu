@@ -23,6 +23,8 @@
 // The kernels are instantiated for MAXT in {1, 2, 4, 8, 16} >= T, the most
 // assignments one expert can have (a token picks an expert at most once), so
 // the per-token accumulators stay in registers and the code stays small.
+#include <cstring>
+
 #include "common.cuh"
 #include "internal.h"
 #include "topk.cuh"
@@ -160,6 +162,7 @@ __global__ void __launch_bounds__(512) k_dec_route(const uint16_t *__restrict__ 
                                                    uint32_t *status)
 {
     __shared__ float part[MAXT * 256];   // [t][e * S + slice], E * S <= 256
+    pdl_trigger();   // the weight-streaming kernel may be scheduled on the other SMs
     if (counter_to_zero && threadIdx.x == 0)
         *counter_to_zero = 0;   // re-arms the histogram's ticket for a following permute
     __shared__ float sl[MAXT * MOE_MAX_E];
@@ -229,6 +232,8 @@ __global__ void __launch_bounds__(256, (MAXT <= 2) ? 4 : 2)
               uint16_t *__restrict__ Hs, uint32_t *status)
 {
     __shared__ DecPlanSmem P;
+    pdl_wait();      // topk_idx comes from the routing kernel
+    pdl_trigger();
     build_plan(P, idx, T, E, k, status);
     const int lane = threadIdx.x & 31;
     const int nwarps = gridDim.x * (blockDim.x >> 5);
@@ -312,6 +317,10 @@ __global__ void __launch_bounds__(256, (MAXT <= 2) ? 4 : 2)
 }
 
 // ---------------------------------------------------------------- phase 2: W2 + combine
+// At MAXT = 1 the weight stream is software-pipelined (two 16-byte loads per
+// lane in flight while two are consumed); at MAXT >= 2 a batch of eight (four
+// above MAXT = 2) loads is issued and then consumed. Both measured best for
+// their token counts on the Mixtral shape.
 template <int MAXT>
 __global__ void __launch_bounds__(256, (MAXT <= 2) ? 4 : 2)
     k_dec_w2(const int32_t *__restrict__ idx, const float *__restrict__ topk_w, int T, int d,
@@ -320,6 +329,7 @@ __global__ void __launch_bounds__(256, (MAXT <= 2) ? 4 : 2)
              const uint16_t *__restrict__ Hs, float *__restrict__ out, uint32_t *status)
 {
     __shared__ DecPlanSmem P;
+    pdl_wait();      // h comes from the w1/w3 kernel
     build_plan(P, idx, T, E, k, status);
     const int lane = threadIdx.x & 31;
     const int nwarps = gridDim.x * (blockDim.x >> 5);
@@ -348,28 +358,57 @@ __global__ void __launch_bounds__(256, (MAXT <= 2) ? 4 : 2)
                 wt[s] = (s < na) ? (shared ? 1.f : topk_w[a]) : 0.f;
             }
             const int nv = ff / 8;
-            constexpr int UNR = (MAXT <= 2) ? 8 : kDecUnroll;   // loads in flight per lane
             float pa[MAXT];
 #pragma unroll
             for (int s = 0; s < MAXT; ++s)
                 pa[s] = 0.f;
-            for (int cb = 0; cb < nv; cb += 32 * UNR) {
-                uint4 wv[UNR];
+            if constexpr (MAXT == 1) {
+                constexpr int UNR = 2;
+                uint4 cur[UNR], nxt[UNR];
 #pragma unroll
                 for (int i = 0; i < UNR; ++i) {
-                    const int ci = cb + lane + 32 * i;
+                    const int ci = lane + 32 * i;
                     if (ci < nv)
-                        wv[i] = ld_stream_v4(wrow + ci);
+                        cur[i] = ld_stream_v4(wrow + ci);
                 }
+                for (int cb = 0; cb < nv; cb += 32 * UNR) {
+                    const int nb = cb + 32 * UNR;
 #pragma unroll
-                for (int i = 0; i < UNR; ++i) {
-                    const int ci = cb + lane + 32 * i;
-                    if (ci >= nv)
-                        continue;
+                    for (int i = 0; i < UNR; ++i) {
+                        const int ci = nb + lane + 32 * i;
+                        if (ci < nv)
+                            nxt[i] = ld_stream_v4(wrow + ci);
+                    }
 #pragma unroll
-                    for (int s = 0; s < MAXT; ++s)
-                        if (s < na)
-                            pa[s] = dot8(wv[i], __ldg(hr[s] + ci), pa[s]);
+                    for (int i = 0; i < UNR; ++i) {
+                        const int ci = cb + lane + 32 * i;
+                        if (ci < nv && na > 0)
+                            pa[0] = dot8(cur[i], __ldg(hr[0] + ci), pa[0]);
+                    }
+#pragma unroll
+                    for (int i = 0; i < UNR; ++i)
+                        cur[i] = nxt[i];
+                }
+            } else {
+                constexpr int UNR = (MAXT <= 2) ? 8 : kDecUnroll;
+                for (int cb = 0; cb < nv; cb += 32 * UNR) {
+                    uint4 wv[UNR];
+#pragma unroll
+                    for (int i = 0; i < UNR; ++i) {
+                        const int ci = cb + lane + 32 * i;
+                        if (ci < nv)
+                            wv[i] = ld_stream_v4(wrow + ci);
+                    }
+#pragma unroll
+                    for (int i = 0; i < UNR; ++i) {
+                        const int ci = cb + lane + 32 * i;
+                        if (ci >= nv)
+                            continue;
+#pragma unroll
+                        for (int s = 0; s < MAXT; ++s)
+                            if (s < na)
+                                pa[s] = dot8(wv[i], __ldg(hr[s] + ci), pa[s]);
+                    }
                 }
             }
             // fold the lane partials into the tokens' accumulators, weighted
@@ -395,6 +434,26 @@ __global__ void __launch_bounds__(256, (MAXT <= 2) ? 4 : 2)
 }
 
 // ---------------------------------------------------------------- host side
+
+// Launch with programmatic stream serialization (the kernel calls pdl_wait()
+// before reading its predecessor's output), hiding the launch gap.
+template <typename... KArgs, typename... Args>
+static void launch_pdl(void (*kernel)(KArgs...), int grid, int block, cudaStream_t st,
+                       Args... args)
+{
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof cfg);
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(block);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaLaunchKernelEx(&cfg, kernel, args...);
+}
 
 static int maxt_for(int T) { return T <= 1 ? 1 : T <= 2 ? 2 : T <= 4 ? 4 : T <= 8 ? 8 : 16; }
 
@@ -463,8 +522,8 @@ int launch_dec_w13(const moe_shape_t &s, const uint16_t *x, const int32_t *topk_
     uint16_t *Hs = Hdec + (size_t)s.T * s.k * s.d_ff;
     const uint16_t *ws = s.d_ff_shared ? W13s : nullptr;
 #define MOE_DEC13(M)                                                                            \
-    k_dec_w13<M><<<blocks, 256, 0, st>>>(x, topk_idx, s.T, s.d, s.d_ff, s.E, s.k, W13,         \
-                                         s.d_ff_shared, ws, Hdec, Hs, status)
+    launch_pdl(k_dec_w13<M>, blocks, 256, st, x, topk_idx, s.T, s.d, s.d_ff, s.E, s.k, W13,    \
+               s.d_ff_shared, ws, Hdec, Hs, status)
     switch (mt) {
     case 1: MOE_DEC13(1); break;
     case 2: MOE_DEC13(2); break;
@@ -487,8 +546,8 @@ int launch_dec_w2(const moe_shape_t &s, const int32_t *topk_idx, const float *to
     const uint16_t *Hs = Hdec + (size_t)s.T * s.k * s.d_ff;
     const uint16_t *ws = s.d_ff_shared ? W2s : nullptr;
 #define MOE_DEC2(M)                                                                             \
-    k_dec_w2<M><<<blocks, 256, 0, st>>>(topk_idx, topk_w, s.T, s.d, s.d_ff, s.E, s.k, W2,      \
-                                        s.d_ff_shared, ws, Hdec, Hs, out, status)
+    launch_pdl(k_dec_w2<M>, blocks, 256, st, topk_idx, topk_w, s.T, s.d, s.d_ff, s.E, s.k, W2, \
+               s.d_ff_shared, ws, Hdec, Hs, out, status)
     switch (mt) {
     case 1: MOE_DEC2(1); break;
     case 2: MOE_DEC2(2); break;
