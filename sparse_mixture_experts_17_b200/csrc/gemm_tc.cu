@@ -33,6 +33,20 @@
 
 namespace moe {
 
+// Rasterisation bands (m-tiles per band) of the grouped GEMMs.
+#ifndef MOE_GM_1SM_W13
+#define MOE_GM_1SM_W13 32
+#endif
+#ifndef MOE_GM_1SM_W2
+#define MOE_GM_1SM_W2 16
+#endif
+#ifndef MOE_GM_2SM_W13
+#define MOE_GM_2SM_W13 16
+#endif
+#ifndef MOE_GM_2SM_W2
+#define MOE_GM_2SM_W2 8
+#endif
+
 struct TcArgs {
     int kblocks;
     int n_tiles;
@@ -534,7 +548,7 @@ static int launch_tc_impl(const GemmArgs &g, cudaStream_t st)
     // all n-tiles, so a band's B tiles are fetched from HBM about once while
     // its A rows stay in L2. Measured on the Mixtral-shape prefill: bands of 32
     // cut w1/w3 DRAM reads by ~15% and time by ~5% against 8; w2 is flat.
-    p.group_m = (MODE == EPI_SWIGLU) ? 32 : 16;
+    p.group_m = (MODE == EPI_SWIGLU) ? MOE_GM_1SM_W13 : MOE_GM_1SM_W2;
     p.b_rows_per_group = g.b_rows_per_group;
     p.mt_row0 = g.mt_row0;
     p.mt_group = g.mt_group;
@@ -585,7 +599,7 @@ static int launch_tc2_impl(const GemmArgs &g, cudaStream_t st)
     std::memset(&p, 0, sizeof p);
     p.kblocks = g.K / 64;
     p.n_tiles = g.N / 256;
-    p.group_m = (MODE == EPI_SWIGLU) ? 16 : 8;
+    p.group_m = (MODE == EPI_SWIGLU) ? MOE_GM_2SM_W13 : MOE_GM_2SM_W2;
     p.b_rows_per_group = g.b_rows_per_group;
     p.mt_row0 = g.mt_row0;
     p.mt_group = g.mt_group;
