@@ -385,14 +385,29 @@ __global__ void __launch_bounds__(256) k_permute(
 #pragma unroll
         for (int j = 0; j < MOE_MAX_K; ++j)
             pj[j] = __shfl_sync(kFullMask, pos, j);
-        const int nv = d / 8;
+        const int nv = d / 8;   // a multiple of 16 (d % 128 == 0)
         const uint4 *src = x + (size_t)t * nv;
-        for (int c = lane; c < nv; c += 32) {
-            const uint4 v = src[c];
+        // four 16-byte loads in flight per lane, each copied to every kept row
+        for (int c0 = 0; c0 < nv; c0 += 128) {
+            uint4 v[4];
 #pragma unroll
-            for (int j = 0; j < MOE_MAX_K; ++j)
-                if (j < k && pj[j] >= 0)
-                    x_perm[(size_t)pj[j] * nv + c] = v;
+            for (int i = 0; i < 4; ++i) {
+                const int c = c0 + lane + 32 * i;
+                if (c < nv)
+                    v[i] = src[c];
+            }
+#pragma unroll
+            for (int j = 0; j < MOE_MAX_K; ++j) {
+                if (j < k && pj[j] >= 0) {
+                    uint4 *dst = x_perm + (size_t)pj[j] * nv;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int c = c0 + lane + 32 * i;
+                        if (c < nv)
+                            dst[c] = v[i];
+                    }
+                }
+            }
         }
     }
     if (out_zero) {
