@@ -302,8 +302,10 @@ def run_ours(a, world, rank, local):
 
     # ---- decode (T = 1, 2, 4, 8 on the same Mixtral-shape weights)
     decode = None
+    graphs = None
     if a.workload == "prefill" and not a.no_extra:
         decode = run_decode_set(M, w, layer, x, dev, stream, world, peaks)
+        graphs = run_graph_set(M, layer, x, dev)
 
     # ---- CPU baseline: the oracle on host cores (rank 0, N = 1 only)
     cpu = None
@@ -333,6 +335,8 @@ def run_ours(a, world, rank, local):
     }
     if decode is not None:
         res["decode"] = decode
+    if graphs is not None:
+        res["launch_overhead"] = graphs
     return res
 
 
@@ -357,6 +361,32 @@ def run_e2e(M, w, layer, x, dev, stream, world, tokens_all, a):
     return {"value": round(tokens_all / (e2e_ms / 1e3), 1), "unit": "tokens/s",
             "h2d_bytes_per_step": x_h.numel() * 2, "d2h_bytes_per_step": out_h.numel() * 4,
             "ms_per_step": round(e2e_ms, 4), "api": "moe_forward_host (pinned host x and out)"}
+
+
+def run_graph_set(M, layer, x, dev):
+    """Launch overhead: the tiny workload and one-token decode, eager vs replay
+    of a captured CUDA graph of the same moe_forward call."""
+    res = {}
+    tiny = I.make_inputs(I.TINY, dev, seed=0)
+    cases = {"tiny_T64": (M.MoeLayer(tiny), tiny["x"]), "decode_T1": (layer, x[:1].contiguous())}
+    for name, (lay, xin) in cases.items():
+        o = torch.empty(xin.shape[0], lay.workload.d, dtype=torch.float32, device=dev)
+        side = torch.cuda.Stream(device=dev)
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            for _ in range(3):
+                lay.forward(xin, out=o)
+        torch.cuda.current_stream().wait_stream(side)
+        eager = time_loop(lambda: lay.forward(xin, out=o), 200, torch.cuda.current_stream())
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            lay.forward(xin, out=o)
+        g.replay()
+        torch.cuda.synchronize()
+        replay = time_loop(g.replay, 200, torch.cuda.current_stream())
+        res[name] = {"eager_us": round(eager * 1e3, 2), "graph_replay_us": round(replay * 1e3, 2)}
+        del g
+    return res
 
 
 def run_decode_set(M, w, layer, x, dev, stream, world, peaks):

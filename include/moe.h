@@ -207,7 +207,15 @@ MOE_API int moe_forward(const moe_shape_t *shape, const moe_bf16_t *x, const moe
  * asynchronously on `stream` (cudaMemcpyAsync; use pinned host buffers for
  * true asynchrony). The caller synchronises the stream before reading
  * out_host. Weights and bias are device pointers as in moe_forward. The
- * workspace must be sized with MOE_FLAG_HOST_IO set in shape->flags. */
+ * workspace must be sized with MOE_FLAG_HOST_IO set in shape->flags.
+ * An uncapped batch of at least 4096 tokens (each token's output depends on
+ * its own row only) is processed in up to 4 chunks: the library forks two
+ * copy streams of its own (created once per device) from `stream`, so each
+ * chunk's upload and download overlap the other chunks' compute, and joins
+ * them back into `stream` before returning. Results equal the unchunked ones
+ * (bit for bit with MOE_FLAG_DETERMINISTIC or k <= 2; otherwise up to the order
+ * of the fp32 atomic additions of the combine).
+ * Not for concurrent calls from several host threads on one device. */
 MOE_API int moe_forward_host(const moe_shape_t *shape, const moe_bf16_t *x_host, const moe_bf16_t *Wg,
                      const float *bias, const moe_bf16_t *W13, const moe_bf16_t *W2,
                      const moe_bf16_t *W13_shared, const moe_bf16_t *W2_shared, float *out_host,

@@ -1,5 +1,6 @@
 // moe_api.cu -- the extern "C" entry points of libmoe.so (declared in moe.h):
 // argument validation, workspace carving, and the launch sequences.
+#include <algorithm>
 #include <atomic>
 #include <cstdint>
 #include <cstring>
@@ -398,6 +399,96 @@ static int forward_impl(const moe_shape_t &s, const WsLayout &L, void *ws, const
     return rc;
 }
 
+// ---------------------------------------------------------------- host I/O pipeline
+// moe_forward_host splits a token-separable batch (uncapped: every token's
+// output depends only on its own row) into chunks, so chunk c+1's upload and
+// chunk c-1's download run on the copy engines while chunk c computes. The two
+// copy streams and the events are created once per device and kept.
+namespace {
+constexpr int kHostIoMaxChunks = 4;
+constexpr int kHostIoMinChunkRows = 2048;
+
+struct HostIo {
+    std::mutex mu;
+    bool ready = false;
+    cudaStream_t in = nullptr, out = nullptr;
+    cudaEvent_t fork = nullptr, join = nullptr;
+    cudaEvent_t in_done[kHostIoMaxChunks] = {};
+    cudaEvent_t compute_done[kHostIoMaxChunks] = {};
+};
+
+HostIo *host_io_for_current_device()
+{
+    static HostIo per_dev[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+        return nullptr;
+    HostIo &h = per_dev[dev];
+    std::lock_guard<std::mutex> g(h.mu);
+    if (!h.ready) {
+        bool ok = cudaStreamCreateWithFlags(&h.in, cudaStreamNonBlocking) == cudaSuccess &&
+                  cudaStreamCreateWithFlags(&h.out, cudaStreamNonBlocking) == cudaSuccess &&
+                  cudaEventCreateWithFlags(&h.fork, cudaEventDisableTiming) == cudaSuccess &&
+                  cudaEventCreateWithFlags(&h.join, cudaEventDisableTiming) == cudaSuccess;
+        for (int c = 0; ok && c < kHostIoMaxChunks; ++c)
+            ok = cudaEventCreateWithFlags(&h.in_done[c], cudaEventDisableTiming) == cudaSuccess &&
+                 cudaEventCreateWithFlags(&h.compute_done[c], cudaEventDisableTiming) == cudaSuccess;
+        if (!ok)
+            return nullptr;
+        h.ready = true;
+    }
+    return &h;
+}
+} // namespace
+
+static int forward_host_pipelined(const moe_shape_t &s, const WsLayout &L, void *ws,
+                                  const uint16_t *x_host, const uint16_t *Wg, const float *bias,
+                                  const uint16_t *W13, const uint16_t *W2, const uint16_t *W13s,
+                                  const uint16_t *W2s, float *out_host, uint32_t *status,
+                                  cudaStream_t st, int nchunks)
+{
+    HostIo *h = host_io_for_current_device();
+    if (!h)
+        return MOE_ERR_CUDA;
+    std::lock_guard<std::mutex> g(h->mu);
+    uint16_t *xd = at<uint16_t>(ws, L.x_stage);
+    float *od = at<float>(ws, L.out_stage);
+    // fork: the copy streams start after everything already queued on `st`
+    if (cudaEventRecord(h->fork, st) != cudaSuccess ||
+        cudaStreamWaitEvent(h->in, h->fork, 0) != cudaSuccess ||
+        cudaStreamWaitEvent(h->out, h->fork, 0) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    const int rows = (s.T + nchunks - 1) / nchunks;
+    for (int c = 0; c < nchunks; ++c) {
+        const int r0 = c * rows, n = std::min(rows, s.T - r0);
+        if (cudaMemcpyAsync(xd + (size_t)r0 * s.d, x_host + (size_t)r0 * s.d, (size_t)n * s.d * 2,
+                            cudaMemcpyHostToDevice, h->in) != cudaSuccess ||
+            cudaEventRecord(h->in_done[c], h->in) != cudaSuccess)
+            return MOE_ERR_CUDA;
+    }
+    for (int c = 0; c < nchunks; ++c) {
+        const int r0 = c * rows, n = std::min(rows, s.T - r0);
+        moe_shape_t sc = s;
+        sc.T = n;
+        if (cudaStreamWaitEvent(st, h->in_done[c], 0) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        int rc = forward_impl(sc, L, ws, xd + (size_t)r0 * s.d, Wg, bias, W13, W2, W13s, W2s,
+                              od + (size_t)r0 * s.d, nullptr, nullptr, status, st);
+        if (rc)
+            return rc;
+        if (cudaEventRecord(h->compute_done[c], st) != cudaSuccess ||
+            cudaStreamWaitEvent(h->out, h->compute_done[c], 0) != cudaSuccess ||
+            cudaMemcpyAsync(out_host + (size_t)r0 * s.d, od + (size_t)r0 * s.d,
+                            (size_t)n * s.d * 4, cudaMemcpyDeviceToHost, h->out) != cudaSuccess)
+            return MOE_ERR_CUDA;
+    }
+    // join: `st` completes only after the last download
+    if (cudaEventRecord(h->join, h->out) != cudaSuccess ||
+        cudaStreamWaitEvent(st, h->join, 0) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    return MOE_OK;
+}
+
 } // namespace moe
 
 using namespace moe;
@@ -648,6 +739,11 @@ int moe_forward_host(const moe_shape_t *shape, const moe_bf16_t *x_host, const m
     if (s.T == 0)
         return MOE_OK;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    // token-separable batches large enough to split: overlap copies with compute
+    const int nchunks = std::min(kHostIoMaxChunks, s.T / kHostIoMinChunkRows);
+    if (s.capacity <= 0 && nchunks >= 2)
+        return forward_host_pipelined(s, L, ws, x_host, Wg, bias, W13, W2, W13_shared, W2_shared,
+                                      out_host, status, st, nchunks);
     uint16_t *xd = at<uint16_t>(ws, L.x_stage);
     float *od = at<float>(ws, L.out_stage);
     const size_t xb = (size_t)s.T * s.d * 2, ob = (size_t)s.T * s.d * 4;

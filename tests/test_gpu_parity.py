@@ -348,10 +348,13 @@ def test_cuda_graph_capture_replay(T):
     assert torch.equal(out, layer.forward(x).clone())
 
 
-def test_forward_host_matches_device():
-    w = small_workload("hostio", 300, 256, 256, 8, 2)
+@pytest.mark.parametrize("T,k,flags", [(300, 2, 0), (5000, 2, 0), (9000, 4, M.MOE_FLAG_DETERMINISTIC)],
+                         ids=["single", "chunked2", "chunked4_det"])
+def test_forward_host_matches_device(T, k, flags):
+    """Host-buffer forward; from 4096 tokens on it runs in overlapped chunks."""
+    w = small_workload("hostio", T, 256, 256, 8, k)
     inp = I.make_inputs(w, "cuda", seed=8)
-    layer = M.MoeLayer(inp, flags=M.MOE_FLAG_HOST_IO)
+    layer = M.MoeLayer(inp, flags=M.MOE_FLAG_HOST_IO | flags)
     ref = layer.forward(inp["x"]).clone()
     x_h = inp["x"].cpu().pin_memory()
     out_h = torch.empty(w.T, w.d, dtype=torch.float32).pin_memory()
