@@ -401,6 +401,80 @@ int oracle_expert_rows(int T, int d, int d_ff, int E, const uint16_t *x,
     return rc;
 }
 
+/* [MIX] "Sparse MoE Block": the softmax over all E of one token's logits,
+ * in fp64. S [T,E] receives the probabilities. */
+int oracle_softmax_rows(int T, int E, const float *L, double *S)
+{
+    if (T < 0 || E < 1 || !L || !S)
+        return ORC_EINVAL;
+    for (int t = 0; t < T; ++t) {
+        const float *l = L + (int64_t)t * E;
+        double M = -INFINITY;
+        for (int e = 0; e < E; ++e) {
+            if (isnan(l[e]))
+                return ORC_ENONFINITE;
+            if ((double)l[e] > M)
+                M = (double)l[e];
+        }
+        if (!isfinite(M))
+            return ORC_ENONFINITE;
+        double Z = 0.0;
+        for (int e = 0; e < E; ++e)
+            Z += exp((double)l[e] - M);
+        for (int e = 0; e < E; ++e)
+            S[(int64_t)t * E + e] = exp((double)l[e] - M) / Z;
+    }
+    return ORC_OK;
+}
+
+/* Expert-choice routing: "MoE Model Architectures", "Design Patterns",
+ * "Pattern 3: Expert Choice Routing" (each expert selects its top tokens from
+ * all tokens). Readings: the score of (t, e) is the softmax over experts
+ * S[t, e] (given here in fp32, as both sides use it); expert e takes the
+ * Ceff = min(C, T) tokens with the largest S[:, e], equal scores going to the
+ * lower token index; its selected tokens are listed in ascending token order
+ * with weight S[t, e]. tokens, w: [E, Ceff]; *ceff receives Ceff. */
+int oracle_expert_choice(int T, int E, int C, const float *S, int32_t *tokens, double *w,
+                         int32_t *ceff)
+{
+    if (T < 0 || E < 1 || C < 1 || !S || !tokens || !w || !ceff)
+        return ORC_EINVAL;
+    const int K = C < T ? C : T;
+    *ceff = K;
+    char *taken = (char *)malloc((size_t)(T > 0 ? T : 1));
+    if (!taken)
+        return ORC_EINVAL;
+    for (int e = 0; e < E; ++e) {
+        memset(taken, 0, (size_t)(T > 0 ? T : 1));
+        /* K rounds of "largest score not yet taken", lowest token on ties */
+        for (int i = 0; i < K; ++i) {
+            int best = -1;
+            for (int t = 0; t < T; ++t) {
+                if (taken[t])
+                    continue;
+                const float v = S[(int64_t)t * E + e];
+                if (isnan(v)) {
+                    free(taken);
+                    return ORC_ENONFINITE;
+                }
+                if (best < 0 || v > S[(int64_t)best * E + e])
+                    best = t;
+            }
+            taken[best] = 1;
+        }
+        /* ascending token order */
+        int n = 0;
+        for (int t = 0; t < T; ++t)
+            if (taken[t]) {
+                tokens[(int64_t)e * K + n] = t;
+                w[(int64_t)e * K + n] = (double)S[(int64_t)t * E + e];
+                ++n;
+            }
+    }
+    free(taken);
+    return ORC_OK;
+}
+
 /* Number of OpenMP threads a parallel region of this library uses. */
 int oracle_num_threads(void)
 {

@@ -56,6 +56,10 @@ def lib():
                                         i, i, P, P]
         L.oracle_expert_rows.argtypes = [i, i, i, i, P, P, P, P, i, i, P, P, P]
         L.oracle_num_threads.argtypes = []
+        L.oracle_softmax_rows.argtypes = [i, i, P, P]
+        L.oracle_expert_choice.argtypes = [i, i, i, P, P, P, P]
+        L.oracle_softmax_rows.restype = ctypes.c_int
+        L.oracle_expert_choice.restype = ctypes.c_int
         for f in (L.oracle_router_logits, L.oracle_route, L.oracle_dispatch,
                   L.oracle_moe_tokens, L.oracle_expert_rows, L.oracle_num_threads):
             f.restype = ctypes.c_int
@@ -179,3 +183,45 @@ def forward(inp: dict, tokens=None, logits=None, h_bf16=True):
     out = moe_tokens(inp["x"], inp["W1"], inp["W3"], inp["W2"], idx, w, disp["slot_pos"], tokens,
                      h_bf16=h_bf16, W1s=inp.get("W1s"), W3s=inp.get("W3s"), W2s=inp.get("W2s"))
     return dict(L64=L64, L32=L32, idx=idx, w=w, out=out, tokens=np.asarray(tokens, np.int32), **disp)
+
+
+def softmax_rows(L32):
+    """fp64 softmax over experts of fp32 logits [T,E]."""
+    L = np.ascontiguousarray(L32, np.float32)
+    T, E = L.shape
+    S = np.empty((T, E), np.float64)
+    _check("softmax_rows", lib().oracle_softmax_rows(T, E, _p(L), _p(S)))
+    return S
+
+
+def expert_choice(S32, C):
+    """Expert-choice selection on fp32 scores [T,E] -> (tokens [E,Ceff], w [E,Ceff])."""
+    S = np.ascontiguousarray(S32, np.float32)
+    T, E = S.shape
+    K = min(C, T)
+    tokens = np.empty((E, K), np.int32)
+    w = np.empty((E, K), np.float64)
+    ceff = np.zeros(1, np.int32)
+    _check("expert_choice", lib().oracle_expert_choice(T, E, int(C), _p(S), _p(tokens), _p(w),
+                                                       _p(ceff)))
+    return tokens, w
+
+
+def expert_choice_layer(inp, S32, C, tokens=None, h_bf16=True):
+    """Layer output under expert-choice routing, for `tokens` (default all):
+    out[t] = sum over the experts that selected t of S[t,e] * FFN_e(x_t)
+    (+ the shared expert), via the per-token evaluation with E slots where
+    slot e is kept iff expert e selected the token."""
+    T, E = S32.shape
+    sel_tok, sel_w = expert_choice(S32, C)
+    idx = np.tile(np.arange(E, dtype=np.int32), (T, 1))
+    w = np.zeros((T, E), np.float64)
+    slot = np.full((T, E), -1, np.int32)
+    for e in range(E):
+        w[sel_tok[e], e] = sel_w[e]
+        slot[sel_tok[e], e] = 0
+    if tokens is None:
+        tokens = np.arange(T, dtype=np.int32)
+    out = moe_tokens(inp["x"], inp["W1"], inp["W3"], inp["W2"], idx, w, slot, tokens,
+                     h_bf16=h_bf16, W1s=inp.get("W1s"), W3s=inp.get("W3s"), W2s=inp.get("W2s"))
+    return dict(out=out, tokens=sel_tok, w=sel_w, tokens_eval=np.asarray(tokens, np.int32))
