@@ -303,9 +303,12 @@ def run_ours(a, world, rank, local):
     # ---- decode (T = 1, 2, 4, 8 on the same Mixtral-shape weights)
     decode = None
     graphs = None
+    expert_choice = None
     if a.workload == "prefill" and not a.no_extra:
         decode = run_decode_set(M, w, layer, x, dev, stream, world, peaks)
         graphs = run_graph_set(M, layer, x, dev)
+        expert_choice = run_expert_choice_set(M, w, layer, x, dev, stream, world, peaks,
+                                              max(3, a.steps // 2))
 
     # ---- CPU baseline: the oracle on host cores (rank 0, N = 1 only)
     cpu = None
@@ -337,6 +340,8 @@ def run_ours(a, world, rank, local):
         res["decode"] = decode
     if graphs is not None:
         res["launch_overhead"] = graphs
+    if expert_choice is not None:
+        res["expert_choice"] = expert_choice
     return res
 
 
@@ -420,6 +425,38 @@ def run_decode_set(M, w, layer, x, dev, stream, world, peaks):
             "w13_kernel_GB_s": round(w13_bytes / (k13 / 1e3) / 1e9, 1),
             "stages_ms": {k: round(v[0] / v[1], 4) for k, v in st.items()}}
     return decode
+
+
+def run_expert_choice_set(M, w, layer, x, dev, stream, world, peaks, steps):
+    """Expert-choice routing on the same weights and tokens: each expert takes
+    C = T k / E tokens, so the GEMMs process as many rows as top-k routing."""
+    C = w.T * w.k // w.E
+    s = M.make_shape(w.T, w.d, w.d_ff, w.E, 1, C, w.d_ff_shared, M.MOE_FLAG_EXPERT_CHOICE)
+    ws = M.alloc_workspace(s, dev)
+    out = torch.empty(w.T, w.d, dtype=torch.float32, device=dev)
+
+    def step():
+        M.moe_forward_expert_choice(s, x, layer.Wg, layer.bias, layer.W13, layer.W2, layer.W13s,
+                                    layer.W2s, out, layer.status, ws)
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    if int(layer.status.item()) != 0:
+        raise RuntimeError(f"device status {int(layer.status.item())} (expert choice)")
+    ms = max_over_ranks(time_loop(step, steps, stream), world, dev)
+    M.moe_profile_enable(True)
+    time_loop(step, steps, stream)
+    M.moe_profile_enable(False)
+    st = M.moe_profile_read()
+    rows = w.E * min(C, w.T)
+    w13_flops = 2.0 * rows * w.d * 2 * w.d_ff
+    k13 = st["w13"][0] / st["w13"][1]
+    return {"capacity_per_expert": C, "rows": rows, "tokens_per_s": round(w.T * world / (ms / 1e3), 1),
+            "ms_per_step": round(ms, 4),
+            "w13_tflops": round(w13_flops / (k13 / 1e3) / 1e12, 1),
+            "w13_frac_measured_sustained": round(w13_flops / (k13 / 1e3) / 1e12
+                                                 / peaks["bf16_tflops_sustained"], 4),
+            "stages_ms": {k: round(v[0] / v[1], 4) for k, v in st.items()}}
 
 
 def run_reference(a, world, rank):

@@ -77,10 +77,12 @@ enum {
     MOE_FLAG_HOST_IO = 1 << 4,       /* workspace also holds device staging for x and out,
                                         as moe_forward_host needs */
     MOE_FLAG_GEMM_1SM = 1 << 5,      /* tensor-core GEMMs: always the single-SM kernel */
-    MOE_FLAG_GEMM_2SM = 1 << 6       /* tensor-core GEMMs: the 2-SM pair kernel (256 x 256
+    MOE_FLAG_GEMM_2SM = 1 << 6,      /* tensor-core GEMMs: the 2-SM pair kernel (256 x 256
                                         tiles, cta_group::2) wherever the output width is a
                                         multiple of 256 (default: the pair kernel for w2 when
                                         experts average >= 1024 rows, else single-SM) */
+    MOE_FLAG_EXPERT_CHOICE = 1 << 7  /* workspace sized for the expert-choice calls
+                                        (moe_route_expert_choice, moe_forward_expert_choice) */
 };
 
 #define MOE_MAX_E 256
@@ -220,6 +222,44 @@ MOE_API int moe_forward_host(const moe_shape_t *shape, const moe_bf16_t *x_host,
                      const float *bias, const moe_bf16_t *W13, const moe_bf16_t *W2,
                      const moe_bf16_t *W13_shared, const moe_bf16_t *W2_shared, float *out_host,
                      uint32_t *status, void *ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Expert-choice routing ("MoE Model Architectures", "Design Patterns",
+ * "Pattern 3: Expert Choice Routing": experts choose tokens instead of tokens
+ * choosing experts). Requires MOE_FLAG_EXPERT_CHOICE in shape->flags (also
+ * for moe_workspace_size) and shape->capacity = C >= 1; shape->k is not used
+ * (any valid value, e.g. 1). MOE_FLAG_DETERMINISTIC and MOE_FLAG_HOST_IO are
+ * rejected with MOE_ERR_INVALID_ARG: the combine adds each expert's weighted
+ * rows into out with atomics, so the last bits of out may differ between runs.
+ *   score S[t, e] = softmax over experts of token t's logits (fp32);
+ *   expert e takes the K = min(C, T) tokens with the largest S[:, e], equal
+ *   scores going to the lower token index;
+ *   out[t] = sum over the experts that took t of S[t, e] * FFN_e(x_t)
+ *            (+ the shared expert), not renormalised; a token no expert takes
+ *            gets only the shared expert (or zero).
+ * moe_route_expert_choice:
+ *   x [T, d] bf16 or NULL: with x, logits [T, E] (out, or NULL to keep them in
+ *   the workspace) and scores [T, E] (out) are computed; with x == NULL,
+ *   scores [T, E] fp32 is the INPUT (identical scores give bit-identical
+ *   selections).
+ *   expert_tokens [E, K] int32 out: each expert's tokens, ascending;
+ *   expert_w [E, K] fp32 out: their scores S[t, e].
+ *   Device errors: MOE_ERR_NONFINITE (NaN logit or score). */
+MOE_API int moe_route_expert_choice(const moe_shape_t *shape, const moe_bf16_t *x,
+                                    const moe_bf16_t *Wg, const float *bias, float *logits,
+                                    float *scores, int32_t *expert_tokens, float *expert_w,
+                                    uint32_t *status, void *ws, size_t ws_bytes,
+                                    moe_stream_t stream);
+
+/* The whole layer under expert-choice routing: router, softmax, per-expert
+ * top-K, gather, grouped w1/w3 GEMM + SwiGLU, grouped w2 GEMM with the
+ * score-weighted combine into out [T, d] fp32 (fully written). Arguments as
+ * in moe_forward. */
+MOE_API int moe_forward_expert_choice(const moe_shape_t *shape, const moe_bf16_t *x,
+                                      const moe_bf16_t *Wg, const float *bias,
+                                      const moe_bf16_t *W13, const moe_bf16_t *W2,
+                                      const moe_bf16_t *W13_shared, const moe_bf16_t *W2_shared,
+                                      float *out, uint32_t *status, void *ws, size_t ws_bytes,
+                                      moe_stream_t stream);
 
 /* moe_permute without a workspace, for callers that cannot allocate device
  * memory: code running while a stream is captured in global capture mode

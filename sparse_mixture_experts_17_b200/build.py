@@ -22,8 +22,8 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libmoe.so")
-SOURCES = ["dispatch.cu", "gemm_simt.cu", "gemm_tc.cu", "decode.cu", "moe_api.cu",
-           "permute_static.cu"]
+SOURCES = ["dispatch.cu", "gemm_simt.cu", "gemm_tc.cu", "decode.cu", "expert_choice.cu",
+           "moe_api.cu", "permute_static.cu"]
 HEADERS = ["common.cuh", "internal.h", "topk.cuh"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

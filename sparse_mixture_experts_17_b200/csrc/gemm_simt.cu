@@ -101,9 +101,13 @@ __global__ void __launch_bounds__(256) k_gemm_simt(const GemmArgs g)
         } else if (MODE == EPI_COMBINE) {
             const int t = g.perm_token[row];
             float wgt = 0.f;
-            for (int j = 0; j < g.k; ++j)
-                if (g.slot_pos[(size_t)t * g.k + j] == row)
-                    wgt = g.topk_w[(size_t)t * g.k + j];
+            if (g.perm_w) {
+                wgt = g.perm_w[row];
+            } else {
+                for (int j = 0; j < g.k; ++j)
+                    if (g.slot_pos[(size_t)t * g.k + j] == row)
+                        wgt = g.topk_w[(size_t)t * g.k + j];
+            }
             float *o = static_cast<float *>(g.out) + (long long)t * g.ldo;
 #pragma unroll
             for (int j = 0; j < 4; ++j)

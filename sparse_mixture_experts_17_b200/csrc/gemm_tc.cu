@@ -64,6 +64,7 @@ struct TcArgs {
     const int32_t *slot_pos;
     const float *topk_w;
     int k;
+    const float *perm_w;
     const float *bias;
     int n_valid;
     uint32_t *status;
@@ -126,9 +127,13 @@ __device__ __forceinline__ void epilogue_tile(const TcArgs &p, uint32_t tb, long
         float wgt = 0.f;
         if (valid) {
             t = p.perm_token[row];
-            for (int j = 0; j < p.k; ++j)
-                if (p.slot_pos[(long long)t * p.k + j] == row)
-                    wgt = p.topk_w[(long long)t * p.k + j];
+            if (p.perm_w) {
+                wgt = p.perm_w[row];
+            } else {
+                for (int j = 0; j < p.k; ++j)
+                    if (p.slot_pos[(long long)t * p.k + j] == row)
+                        wgt = p.topk_w[(long long)t * p.k + j];
+            }
         }
         float *o = static_cast<float *>(p.out) + (long long)t * p.ldo + n_idx * BN;
 #pragma unroll 1
@@ -562,6 +567,7 @@ static int launch_tc_impl(const GemmArgs &g, cudaStream_t st)
     p.slot_pos = g.slot_pos;
     p.topk_w = g.topk_w;
     p.k = g.k;
+    p.perm_w = g.perm_w;
     p.bias = g.bias;
     p.n_valid = g.n_valid;
     p.status = g.status;
@@ -613,6 +619,7 @@ static int launch_tc2_impl(const GemmArgs &g, cudaStream_t st)
     p.slot_pos = g.slot_pos;
     p.topk_w = g.topk_w;
     p.k = g.k;
+    p.perm_w = g.perm_w;
     p.bias = g.bias;
     p.n_valid = g.n_valid;
     p.status = g.status;

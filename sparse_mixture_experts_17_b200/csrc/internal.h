@@ -36,6 +36,7 @@ struct WsLayout {
     size_t x_perm, H, H_shared, Y;
     size_t dec_H;
     size_t x_stage, out_stage;
+    size_t scores, ec_w;   // expert-choice routing
     size_t total;
     int nchunks, max_mt, max_mt2;
 };
@@ -98,6 +99,7 @@ struct GemmArgs {
     const int32_t *slot_pos;
     const float *topk_w;
     int k;
+    const float *perm_w;      // EPI_COMBINE: weight of each row (else found via slot_pos)
     const float *bias;
     int n_valid;
     uint32_t *status;
@@ -123,5 +125,14 @@ int launch_dec_w13(const moe_shape_t &s, const uint16_t *x, const int32_t *topk_
 int launch_dec_w2(const moe_shape_t &s, const int32_t *topk_idx, const float *topk_w,
                   const uint16_t *W2, const uint16_t *W2s, const uint16_t *Hdec, float *out,
                   uint32_t *status, cudaStream_t st);
+
+// ---- expert-choice routing (expert_choice.cu)
+int launch_softmax_rows(const moe_shape_t &s, const float *logits, float *scores,
+                        uint32_t *status, cudaStream_t st);
+int launch_ec_select(const moe_shape_t &s, int K, const float *scores, int32_t *tokens,
+                     float *weights, int32_t *offsets, int32_t *mt_row0, int32_t *mt_group,
+                     int32_t *num_mt, uint32_t *status, cudaStream_t st);
+int launch_ec_gather(const moe_shape_t &s, int rows, const uint16_t *x, const int32_t *tokens,
+                     uint16_t *x_perm, float *out_zero, cudaStream_t st);
 
 } // namespace moe

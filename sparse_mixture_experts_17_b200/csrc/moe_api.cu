@@ -101,7 +101,9 @@ WsLayout ws_layout(const moe_shape_t &s)
         off += (bytes + 255) & ~static_cast<size_t>(255);
         return o;
     };
-    const size_t T = s.T, k = s.k, E = s.E, N = T * k;
+    const bool ec = (s.flags & MOE_FLAG_EXPERT_CHOICE) != 0;
+    const size_t Kec = ec ? (size_t)std::min(std::max(s.capacity, 0), s.T) : 0;
+    const size_t T = s.T, k = s.k, E = s.E, N = std::max(T * k, E * Kec);
     L.nchunks = (int)((T + kChunkTokens - 1) / kChunkTokens);
     L.max_mt = (int)((N + kBlockM - 1) / kBlockM + E);
     L.max_mt2 = (int)((N + 2 * kBlockM - 1) / (2 * kBlockM) + E);
@@ -128,6 +130,8 @@ WsLayout ws_layout(const moe_shape_t &s)
     L.Y = take((s.flags & MOE_FLAG_DETERMINISTIC) ? N * s.d * 4 : 0);
     const size_t Td = T < (size_t)MOE_DECODE_MAX_T ? T : (size_t)MOE_DECODE_MAX_T;
     L.dec_H = take((Td * k * s.d_ff + Td * s.d_ff_shared) * 2);
+    L.scores = take(ec ? T * E * 4 : 0);
+    L.ec_w = take(ec ? N * 4 : 0);
     L.x_stage = take((s.flags & MOE_FLAG_HOST_IO) ? T * s.d * 2 : 0);
     L.out_stage = take((s.flags & MOE_FLAG_HOST_IO) ? T * s.d * 4 : 0);
     L.total = off;
@@ -194,9 +198,10 @@ static int expert_ffn_core(const moe_shape_t &s, const WsLayout &L, void *ws,
                            const uint16_t *x_perm, const int32_t *offsets, const uint16_t *W13,
                            const uint16_t *W2, const int32_t *perm_token, const int32_t *slot_pos,
                            const float *topk_w, float *y_perm, float *out, uint32_t *status,
-                           cudaStream_t st)
+                           cudaStream_t st, long long n_rows = -1, const float *perm_w = nullptr,
+                           bool allow_pair = true)
 {
-    const long long N = (long long)s.T * s.k;
+    const long long N = n_rows >= 0 ? n_rows : (long long)s.T * s.k;
     uint16_t *H = at<uint16_t>(ws, L.H);
     GemmArgs g = gemm_base();
     g.mode = EPI_SWIGLU;
@@ -208,7 +213,7 @@ static int expert_ffn_core(const moe_shape_t &s, const WsLayout &L, void *ws,
     g.N = 2 * s.d_ff;
     g.b_rows_per_group = 2 * s.d_ff;
     const long long avg_rows = N / s.E;
-    set_tiles(g, L, ws, use_pair(s, avg_rows, g.N, false));
+    set_tiles(g, L, ws, allow_pair && use_pair(s, avg_rows, g.N, false));
     g.seg_offsets = offsets;
     g.out = H;
     g.ldo = s.d_ff;
@@ -227,7 +232,7 @@ static int expert_ffn_core(const moe_shape_t &s, const WsLayout &L, void *ws,
     g.N = s.d;
     g.b_rows_per_group = s.d;
     g.ldo = s.d;
-    set_tiles(g, L, ws, use_pair(s, avg_rows, g.N, true));
+    set_tiles(g, L, ws, allow_pair && use_pair(s, avg_rows, g.N, true));
     if (y_perm) {
         g.mode = EPI_STORE_F32;
         g.out = y_perm;
@@ -238,6 +243,7 @@ static int expert_ffn_core(const moe_shape_t &s, const WsLayout &L, void *ws,
         g.slot_pos = slot_pos;
         g.topk_w = topk_w;
         g.k = s.k;
+        g.perm_w = perm_w;
     }
     StageMark m(MOE_STAGE_W2, st);
     return run_gemm(s, g, st);
@@ -397,6 +403,43 @@ static int forward_impl(const moe_shape_t &s, const WsLayout &L, void *ws, const
         rc = launch_combine(s, Y, slot_pos, w, shared ? out : nullptr, out, st);
     }
     return rc;
+}
+
+// ---------------------------------------------------------------- expert-choice routing
+// Expert choice needs its flag (workspace sizing) and a capacity. Its combine
+// is the w2 epilogue's atomic add (a token may be taken by any number of
+// experts), so the bitwise-repeatable mode is not offered for it.
+static int ec_check(const moe_shape_t &s)
+{
+    if (!(s.flags & MOE_FLAG_EXPERT_CHOICE) || s.capacity <= 0 ||
+        (s.flags & (MOE_FLAG_DETERMINISTIC | MOE_FLAG_HOST_IO)))
+        return MOE_ERR_INVALID_ARG;
+    return MOE_OK;
+}
+
+// Router + softmax (when x is given) and the per-expert selection; writes the
+// selected tokens / weights, the expert offsets and the GEMM m-tile list.
+static int ec_route(const moe_shape_t &s, const WsLayout &L, void *ws, const uint16_t *x,
+                    const uint16_t *Wg, const float *bias, float *logits, float *scores,
+                    int32_t *tokens, float *weights, uint32_t *status, cudaStream_t st)
+{
+    const int K = std::min(s.capacity, s.T);
+    int rc;
+    if (x) {
+        {
+            StageMark m(MOE_STAGE_ROUTER, st);
+            rc = router(s, x, Wg, bias, logits, status, st);
+        }
+        if (rc)
+            return rc;
+        StageMark m(MOE_STAGE_TOPK, st);
+        if ((rc = launch_softmax_rows(s, logits, scores, status, st)))
+            return rc;
+    }
+    StageMark m(MOE_STAGE_HIST, st);
+    return launch_ec_select(s, K, scores, tokens, weights, at<int32_t>(ws, L.offsets),
+                            at<int32_t>(ws, L.mt_row0), at<int32_t>(ws, L.mt_group),
+                            at<int32_t>(ws, L.num_mt), status, st);
 }
 
 // ---------------------------------------------------------------- host I/O pipeline
@@ -756,6 +799,75 @@ int moe_forward_host(const moe_shape_t *shape, const moe_bf16_t *x_host, const m
     if (cudaMemcpyAsync(out_host, od, ob, cudaMemcpyDeviceToHost, st) != cudaSuccess)
         return MOE_ERR_CUDA;
     return MOE_OK;
+}
+
+int moe_route_expert_choice(const moe_shape_t *shape, const moe_bf16_t *x, const moe_bf16_t *Wg,
+                            const float *bias, float *logits, float *scores,
+                            int32_t *expert_tokens, float *expert_w, uint32_t *status, void *ws,
+                            size_t ws_bytes, moe_stream_t stream)
+{
+    int rc = check_shape(shape);
+    if (rc)
+        return rc;
+    if ((rc = ec_check(*shape)))
+        return rc;
+    if (shape->T == 0)
+        return MOE_OK;
+    const moe_shape_t &s = *shape;
+    if (!scores || !expert_tokens || !expert_w || (x && (!Wg || !al16(x) || !al16(Wg))))
+        return MOE_ERR_INVALID_ARG;
+    WsLayout L;
+    if ((rc = check_ws(s, ws, ws_bytes, L)))
+        return rc;
+    return ec_route(s, L, ws, x, Wg, bias, logits ? logits : at<float>(ws, L.logits), scores,
+                    expert_tokens, expert_w, status, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int moe_forward_expert_choice(const moe_shape_t *shape, const moe_bf16_t *x, const moe_bf16_t *Wg,
+                              const float *bias, const moe_bf16_t *W13, const moe_bf16_t *W2,
+                              const moe_bf16_t *W13_shared, const moe_bf16_t *W2_shared,
+                              float *out, uint32_t *status, void *ws, size_t ws_bytes,
+                              moe_stream_t stream)
+{
+    int rc = check_shape(shape);
+    if (rc)
+        return rc;
+    if ((rc = ec_check(*shape)))
+        return rc;
+    if (shape->T == 0)
+        return MOE_OK;
+    const moe_shape_t &s = *shape;
+    if (!x || !Wg || !W13 || !W2 || !out || !al16(x) || !al16(Wg) || !al16(W13) || !al16(W2) ||
+        !al16(out))
+        return MOE_ERR_INVALID_ARG;
+    if (s.d_ff_shared > 0 &&
+        (!W13_shared || !W2_shared || !al16(W13_shared) || !al16(W2_shared)))
+        return MOE_ERR_INVALID_ARG;
+    WsLayout L;
+    if ((rc = check_ws(s, ws, ws_bytes, L)))
+        return rc;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const int K = std::min(s.capacity, s.T);
+    const long long rows = (long long)s.E * K;
+    int32_t *tokens = at<int32_t>(ws, L.perm_token);
+    float *wts = at<float>(ws, L.ec_w);
+    if ((rc = ec_route(s, L, ws, x, Wg, bias, at<float>(ws, L.logits), at<float>(ws, L.scores),
+                       tokens, wts, status, st)))
+        return rc;
+    const bool shared = s.d_ff_shared > 0;
+    uint16_t *x_perm = at<uint16_t>(ws, L.x_perm);
+    {
+        StageMark m(MOE_STAGE_PERMUTE, st);
+        if ((rc = launch_ec_gather(s, (int)rows, x, tokens, x_perm, shared ? nullptr : out, st)))
+            return rc;
+    }
+    if (shared) {
+        StageMark m(MOE_STAGE_SHARED, st);
+        if ((rc = shared_expert(s, L, ws, x, W13_shared, W2_shared, out, status, st)))
+            return rc;
+    }
+    return expert_ffn_core(s, L, ws, x_perm, at<int32_t>(ws, L.offsets), W13, W2, tokens, nullptr,
+                           nullptr, nullptr, out, status, st, rows, wts, false);
 }
 
 } // extern "C"

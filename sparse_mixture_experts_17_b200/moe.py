@@ -34,6 +34,7 @@ MOE_FLAG_SIMT_FFN = 1 << 3
 MOE_FLAG_HOST_IO = 1 << 4
 MOE_FLAG_GEMM_1SM = 1 << 5
 MOE_FLAG_GEMM_2SM = 1 << 6
+MOE_FLAG_EXPERT_CHOICE = 1 << 7
 
 MOE_MAX_E = 256
 MOE_MAX_K = 16
@@ -81,6 +82,9 @@ _SIGS = {
     "moe_forward": ([_SHP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P], ctypes.c_int),
     "moe_forward_host": ([_SHP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P], ctypes.c_int),
     "moe_permute_static": ([_SHP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P], ctypes.c_int),
+    "moe_route_expert_choice": ([_SHP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P], ctypes.c_int),
+    "moe_forward_expert_choice": ([_SHP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P],
+                                  ctypes.c_int),
     "moe_kernel_launches": ([], ctypes.c_uint64),
     "moe_profile_enable": ([ctypes.c_int], ctypes.c_int),
     "moe_profile_read": ([_P, _P, ctypes.c_int], ctypes.c_int),
@@ -199,6 +203,24 @@ def moe_permute_static(shape, topk_idx, x, expert_counts, expert_offsets, slot_p
         _ptr(slot_pos, I32, "slot_pos"), _ptr(perm_token, I32, "perm_token"),
         _ptr(x_perm, BF16, "x_perm"), _ptr(n_kept, I32, "n_kept"), _ptr(status, U32, "status"),
         _stream(stream)))
+
+
+def moe_route_expert_choice(shape, x, Wg, bias, logits, scores, expert_tokens, expert_w, status,
+                            ws, stream=None):
+    _check("moe_route_expert_choice", lib().moe_route_expert_choice(
+        ctypes.byref(shape), _ptr(x, BF16, "x"), _ptr(Wg, BF16, "Wg"), _ptr(bias, F32, "bias"),
+        _ptr(logits, F32, "logits"), _ptr(scores, F32, "scores"),
+        _ptr(expert_tokens, I32, "expert_tokens"), _ptr(expert_w, F32, "expert_w"),
+        _ptr(status, U32, "status"), _ptr(ws, name="ws"), ws.numel(), _stream(stream)))
+
+
+def moe_forward_expert_choice(shape, x, Wg, bias, W13, W2, W13_shared, W2_shared, out, status, ws,
+                              stream=None):
+    _check("moe_forward_expert_choice", lib().moe_forward_expert_choice(
+        ctypes.byref(shape), _ptr(x, BF16, "x"), _ptr(Wg, BF16, "Wg"), _ptr(bias, F32, "bias"),
+        _ptr(W13, BF16, "W13"), _ptr(W2, BF16, "W2"), _ptr(W13_shared, BF16, "W13_shared"),
+        _ptr(W2_shared, BF16, "W2_shared"), _ptr(out, F32, "out"), _ptr(status, U32, "status"),
+        _ptr(ws, name="ws"), ws.numel(), _stream(stream)))
 
 
 def moe_expert_ffn(shape, x_perm, expert_offsets, W13, W2, perm_token, slot_pos, topk_w, y_perm,
