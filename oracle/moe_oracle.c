@@ -37,8 +37,14 @@
  *      to the same expert come before it in row-major (token, slot) order;
  *      C <= 0 is uncapped ([MGA]). Kept weights are not renormalised; a
  *      dropped assignment contributes nothing.
+ *      Slot-priority variant (R3b): the same rule with the assignments in
+ *      slot-major (slot, token) order, so every token's first choice is
+ *      placed before any token's second choice (the priority GShard/GLaM-style
+ *      top-2 dispatch gives the first expert; the page's comparison table
+ *      names GLaM's capacity-factor tuning, and its Switch mask is garbled).
  *  R4  expert offsets have E+1 entries with a leading 0 ([CUR]'s GPU form);
- *      an expert's kept rows are laid out in ascending token order.
+ *      an expert's kept rows are laid out in rank order: ascending token (R3),
+ *      or by slot, then ascending token (R3b).
  *  R5  the bias enters both the selection and the weights ([DSK]'s
  *      F.linear(x, W, b) feeds the softmax); a shared expert is added with
  *      weight 1.
@@ -188,42 +194,45 @@ int oracle_route(int T, int E, int k, const float *L, int32_t *idx, double *w)
 
 /* Expert histogram, capacity, offsets and permutation: [CUR]'s counts and
  * offsets, [MIX]'s torch.where(selected_experts == e) row-major order, and
- * readings R3/R4.
+ * readings R3/R4 (R3b with slot_major = 1).
  *   counts[E]       routed assignments per expert (before capacity)
  *   offsets[E+1]    exclusive scan of the kept counts min(counts, C)
  *   slot_pos[T*k]   permuted row of (t, j), or -1 if dropped
  *   perm_token[T*k] token of each permuted row; rows >= n_kept are -1
  *   n_kept[1]       offsets[E]
  * Ids must lie in [0, E) and be distinct within a token (ORC_EBADEXPERT). */
-int oracle_dispatch(int T, int E, int k, int C, const int32_t *idx,
+int oracle_dispatch(int T, int E, int k, int C, int slot_major, const int32_t *idx,
                     int32_t *counts, int32_t *offsets, int32_t *slot_pos,
                     int32_t *perm_token, int32_t *n_kept)
 {
     if (T < 0 || E < 1 || k < 1 || k > E || !idx || !counts || !offsets ||
         !slot_pos || !perm_token || !n_kept)
         return ORC_EINVAL;
+    for (int t = 0; t < T; ++t) {
+        for (int j = 0; j < k; ++j) {
+            int32_t e = idx[(int64_t)t * k + j];
+            if (e < 0 || e >= E)
+                return ORC_EBADEXPERT;
+            for (int jj = 0; jj < j; ++jj)
+                if (idx[(int64_t)t * k + jj] == e)
+                    return ORC_EBADEXPERT;
+        }
+    }
     const int64_t N = (int64_t)T * k;
     int32_t *rank = (int32_t *)malloc(sizeof(int32_t) * (size_t)(N > 0 ? N : 1));
     if (!rank)
         return ORC_EINVAL;
     for (int e = 0; e < E; ++e)
         counts[e] = 0;
-    /* pass 1: each assignment's rank among earlier assignments to its expert */
-    for (int t = 0; t < T; ++t) {
-        for (int j = 0; j < k; ++j) {
-            int32_t e = idx[(int64_t)t * k + j];
-            if (e < 0 || e >= E) {
-                free(rank);
-                return ORC_EBADEXPERT;
-            }
-            for (int jj = 0; jj < j; ++jj)
-                if (idx[(int64_t)t * k + jj] == e) {
-                    free(rank);
-                    return ORC_EBADEXPERT;
-                }
-            rank[(int64_t)t * k + j] = counts[e];
-            counts[e] += 1;
-        }
+    /* pass 1: each assignment's rank among the assignments to its expert that
+     * come before it in the priority order */
+    for (int64_t i = 0; i < N; ++i) {
+        const int t = slot_major ? (int)(i % (T > 0 ? T : 1)) : (int)(i / k);
+        const int j = slot_major ? (int)(i / (T > 0 ? T : 1)) : (int)(i % k);
+        const int64_t a = (int64_t)t * k + j;
+        const int32_t e = idx[a];
+        rank[a] = counts[e];
+        counts[e] += 1;
     }
     /* offsets: exclusive scan of kept counts */
     offsets[0] = 0;

@@ -51,7 +51,7 @@ def lib():
         L.oracle_round_bf16.restype = ctypes.c_double
         L.oracle_router_logits.argtypes = [i, i, i, P, P, P, P, P]
         L.oracle_route.argtypes = [i, i, i, P, P, P]
-        L.oracle_dispatch.argtypes = [i, i, i, i, P, P, P, P, P, P]
+        L.oracle_dispatch.argtypes = [i, i, i, i, i, P, P, P, P, P, P]
         L.oracle_moe_tokens.argtypes = [i, i, i, i, i, i, P, P, P, P, P, P, P, P, P, P,
                                         i, i, P, P]
         L.oracle_expert_rows.argtypes = [i, i, i, i, P, P, P, P, i, i, P, P, P]
@@ -112,8 +112,9 @@ def route(L32, k):
     return idx, w
 
 
-def dispatch(idx, E, C=0):
-    """idx [T,k] -> dict(counts [E], offsets [E+1], slot_pos [T,k], perm_token [T*k], n_kept)."""
+def dispatch(idx, E, C=0, slot_priority=False):
+    """idx [T,k] -> dict(counts [E], offsets [E+1], slot_pos [T,k], perm_token [T*k], n_kept).
+    slot_priority: capacity ranks (and segment order) in slot-major order."""
     idx = np.ascontiguousarray(idx, np.int32)
     T, k = idx.shape
     counts = np.empty(E, np.int32)
@@ -121,7 +122,8 @@ def dispatch(idx, E, C=0):
     slot_pos = np.empty((T, k), np.int32)
     perm_token = np.empty(max(T * k, 1), np.int32)
     n_kept = np.zeros(1, np.int32)
-    _check("dispatch", lib().oracle_dispatch(T, E, k, int(C), _p(idx), _p(counts), _p(offsets),
+    _check("dispatch", lib().oracle_dispatch(T, E, k, int(C), int(bool(slot_priority)), _p(idx),
+                                             _p(counts), _p(offsets),
                                              _p(slot_pos), _p(perm_token), _p(n_kept)))
     return dict(counts=counts, offsets=offsets, slot_pos=slot_pos,
                 perm_token=perm_token[: T * k], n_kept=int(n_kept[0]))
@@ -167,7 +169,7 @@ def forward(inp: dict, tokens=None, logits=None, h_bf16=True):
     dispatch with the capacity, then outputs for ``tokens`` (default: all).
 
     ``inp`` holds numpy arrays: x, wg, bias (or None), W1, W3, W2, optional
-    W1s/W3s/W2s, and ints k, capacity.
+    W1s/W3s/W2s, ints k, capacity, and an optional bool slot_priority.
     """
     T = inp["x"].shape[0]
     E = inp["wg"].shape[0]
@@ -177,7 +179,7 @@ def forward(inp: dict, tokens=None, logits=None, h_bf16=True):
     else:
         L32 = np.ascontiguousarray(logits, np.float32)
     idx, w = route(L32, inp["k"])
-    disp = dispatch(idx, E, inp.get("capacity", 0))
+    disp = dispatch(idx, E, inp.get("capacity", 0), inp.get("slot_priority", False))
     if tokens is None:
         tokens = np.arange(T, dtype=np.int32)
     out = moe_tokens(inp["x"], inp["W1"], inp["W3"], inp["W2"], idx, w, disp["slot_pos"], tokens,

@@ -202,6 +202,55 @@ def test_dispatch_invariants_and_brute_rank(orc, T, E, k, C):
             assert seg.max() < dropped.min()
 
 
+@pytest.mark.parametrize("T,E,k,C", [(37, 5, 2, 5), (200, 16, 4, 30), (300, 12, 3, 40),
+                                     (64, 8, 2, 1), (50, 4, 1, 7), (80, 6, 3, 0)])
+def test_dispatch_slot_priority_brute_force(orc, T, E, k, C):
+    """Slot-priority capacity: per expert, its assignments sorted by (slot, token)
+    with a plain Python sort; the first C are kept, in that order."""
+    rng = np.random.default_rng(T * 3 + E + k + C)
+    idx = _random_idx(rng, T, E, k, skew=1.2)
+    d = orc.dispatch(idx, E, C, slot_priority=True)
+    off = [0]
+    order = {}
+    for e in range(E):
+        a_e = sorted(((j, t) for t in range(T) for j in range(k) if idx[t, j] == e))
+        keep = a_e if C <= 0 else a_e[:C]
+        order[e] = keep
+        off.append(off[-1] + len(keep))
+    assert d["offsets"].tolist() == off
+    assert (d["counts"] == np.bincount(idx.reshape(-1), minlength=E)).all()
+    sp = np.full((T, k), -1)
+    for e in range(E):
+        for r, (j, t) in enumerate(order[e]):
+            sp[t, j] = off[e] + r
+            assert d["perm_token"][off[e] + r] == t
+    assert (d["slot_pos"] == sp).all()
+
+
+def test_dispatch_slot_priority_special_cases(orc):
+    rng = np.random.default_rng(9)
+    # k = 1: slot-major and row-major orders coincide
+    idx1 = _random_idx(rng, 120, 6, 1, skew=1.0)
+    a, b = orc.dispatch(idx1, 6, 9), orc.dispatch(idx1, 6, 9, slot_priority=True)
+    for key in ("counts", "offsets", "slot_pos", "perm_token"):
+        assert (a[key] == b[key]).all()
+    # uncapped: the same rows per expert (only their order differs)
+    idx = _random_idx(rng, 90, 8, 3, skew=0.5)
+    a, b = orc.dispatch(idx, 8, 0), orc.dispatch(idx, 8, 0, slot_priority=True)
+    assert (a["offsets"] == b["offsets"]).all()
+    for e in range(8):
+        sa = a["perm_token"][a["offsets"][e]:a["offsets"][e + 1]]
+        sb = b["perm_token"][b["offsets"][e]:b["offsets"][e + 1]]
+        assert sorted(sa.tolist()) == sorted(sb.tolist())
+    # every first choice survives whenever C covers the first choices
+    idx = _random_idx(rng, 100, 5, 2, skew=0.0)
+    C = int(np.bincount(idx[:, 0], minlength=5).max())
+    b = orc.dispatch(idx, 5, C, slot_priority=True)
+    assert (b["slot_pos"][:, 0] >= 0).all()
+    a = orc.dispatch(idx, 5, C)
+    assert a["n_kept"] == b["n_kept"]          # same kept count per expert: min(count, C)
+
+
 def test_dispatch_rejects_bad_ids(orc):
     with pytest.raises(orc.OracleError) as ei:
         orc.dispatch(np.array([[0, 3]], np.int32), 3, 0)
