@@ -81,8 +81,9 @@ enum {
                                         tiles, cta_group::2) wherever the output width is a
                                         multiple of 256 (default: the pair kernel for w2 when
                                         experts average >= 1024 rows, else single-SM) */
-    MOE_FLAG_EXPERT_CHOICE = 1 << 7  /* workspace sized for the expert-choice calls
+    MOE_FLAG_EXPERT_CHOICE = 1 << 7, /* workspace sized for the expert-choice calls
                                         (moe_route_expert_choice, moe_forward_expert_choice) */
+    MOE_FLAG_SLOT_PRIORITY = 1 << 8  /* capacity ranks in slot-major order (see moe_shape_t) */
 };
 
 #define MOE_MAX_E 256
@@ -100,7 +101,12 @@ enum {
  * the chosen experts", where a capacity factor of 0 means uncapped): an
  * assignment (t, j) is kept iff fewer than `capacity` assignments to the same
  * expert precede it in row-major (token, slot) order. Dropped assignments
- * contribute nothing and the kept weights are not renormalised. */
+ * contribute nothing and the kept weights are not renormalised.
+ * With MOE_FLAG_SLOT_PRIORITY the order is slot-major (slot, token) instead:
+ * every token's first choice ranks before any token's second choice (the
+ * first-expert priority of top-2 dispatch with a capacity factor, the
+ * "Capacity factor tuning" of the page's GLaM row), and an expert's kept
+ * rows are laid out in that order (by slot, then ascending token). */
 typedef struct moe_shape {
     int32_t T, d, d_ff, E, k;
     int32_t capacity;
@@ -147,7 +153,8 @@ MOE_API int moe_route(const moe_shape_t *shape, const moe_bf16_t *x, const moe_b
  *   expert_offsets [E+1] int32 out: exclusive scan of min(count, capacity)
  *   slot_pos       [T, k] int32 out: permuted row of (t, j), -1 if dropped
  *   perm_token     [T*k] int32 out: token of each permuted row; rows within an
- *                  expert are in ascending token order; rows >= n_kept untouched
+ *                  expert are in ascending token order (MOE_FLAG_SLOT_PRIORITY:
+ *                  by slot, then token); rows >= n_kept untouched
  *   x_perm         [T*k, d] bf16 out: x_perm[slot_pos[t,j]] = x[t]
  *   n_kept         [1] int32 out: expert_offsets[E]
  * Bit-exact: the result is a function of topk_idx alone.

@@ -12,6 +12,8 @@
 // Routing (k_dec_route): one CTA computes the T x E logits (warps over
 // experts, lanes over d) and then the top-k (one warp per token), when W_g is
 // small; otherwise k_dec_router (one warp per expert) feeds k_topk.
+// The plan applies the capacity (in the same rank order as the histogram
+// kernel), so a dropped assignment reads no weights and adds nothing.
 // Phase 1 (k_dec_w13): work unit = one SwiGLU column c of one chosen expert:
 //   h[a, c] = bf16(silu(W1_e[c] . x_t) * (W3_e[c] . x_t)) for every
 //   assignment a = (t, j) routed to e. Each unit streams the gate row and the
@@ -42,9 +44,31 @@ struct DecPlanSmem {
     int start[MOE_MAX_E];
 };
 
-// Every thread of the CTA participates; ends with __syncthreads().
+// Rank of assignment a among the assignments to the same expert that come
+// before it in the capacity order: row-major (t, j), or slot-major (j, t).
+__device__ __forceinline__ int plan_rank(const int32_t *__restrict__ idx, int A, int k, int a,
+                                         int slot_major)
+{
+    const int e = idx[a];
+    int r = 0;
+    if (!slot_major) {
+        for (int b = 0; b < a; ++b)
+            r += (idx[b] == e);
+    } else {
+        const int ja = a % k;
+        for (int b = 0; b < A; ++b) {
+            const int jb = b % k;
+            r += (idx[b] == e) && (jb < ja || (jb == ja && b < a));
+        }
+    }
+    return r;
+}
+
+// Every thread of the CTA participates; ends with __syncthreads(). An
+// assignment whose rank reaches the capacity C (> 0) is dropped: it is in no
+// expert's list, so it gets no h row and adds nothing to out.
 __device__ void build_plan(DecPlanSmem &P, const int32_t *__restrict__ idx, int T, int E, int k,
-                           uint32_t *status)
+                           int C, int slot_major, uint32_t *status)
 {
     const int A = T * k;
     for (int e = threadIdx.x; e < MOE_MAX_E; e += blockDim.x)
@@ -57,6 +81,8 @@ __device__ void build_plan(DecPlanSmem &P, const int32_t *__restrict__ idx, int 
                 flag_status(status, MOE_ERR_BAD_EXPERT);
             continue;
         }
+        if (C > 0 && plan_rank(idx, A, k, a, slot_major) >= C)
+            continue;
         atomicAdd(&P.cnt[e], 1);
     }
     __syncthreads();
@@ -75,14 +101,14 @@ __device__ void build_plan(DecPlanSmem &P, const int32_t *__restrict__ idx, int 
         P.U = u;
     }
     __syncthreads();
-    // rank of each assignment among earlier ones of the same expert (token order)
+    // each kept assignment at its rank within its expert's list
     for (int a = threadIdx.x; a < A; a += blockDim.x) {
         const int e = idx[a];
         if (e < 0 || e >= E)
             continue;
-        int r = 0;
-        for (int b = 0; b < a; ++b)
-            r += (idx[b] == e);
+        const int r = plan_rank(idx, A, k, a, slot_major);
+        if (C > 0 && r >= C)
+            continue;
         P.list[P.start[e] + r] = a;
     }
     __syncthreads();
@@ -227,14 +253,15 @@ constexpr int kDecUnroll = 4;
 template <int MAXT>
 __global__ void __launch_bounds__(256, (MAXT <= 2) ? 4 : 2)
     k_dec_w13(const uint16_t *__restrict__ x, const int32_t *__restrict__ idx, int T, int d,
-              int d_ff, int E, int k, const uint16_t *__restrict__ W13, int d_ff_s,
+              int d_ff, int E, int k, int C, int slot_major, const uint16_t *__restrict__ W13,
+              int d_ff_s,
               const uint16_t *__restrict__ W13s, uint16_t *__restrict__ Hdec,
               uint16_t *__restrict__ Hs, uint32_t *status)
 {
     __shared__ DecPlanSmem P;
     pdl_wait();      // topk_idx comes from the routing kernel
     pdl_trigger();
-    build_plan(P, idx, T, E, k, status);
+    build_plan(P, idx, T, E, k, C, slot_major, status);
     const int lane = threadIdx.x & 31;
     const int nwarps = gridDim.x * (blockDim.x >> 5);
     const long long routed_units = (long long)P.U * d_ff;
@@ -324,13 +351,14 @@ __global__ void __launch_bounds__(256, (MAXT <= 2) ? 4 : 2)
 template <int MAXT>
 __global__ void __launch_bounds__(256, (MAXT <= 2) ? 4 : 2)
     k_dec_w2(const int32_t *__restrict__ idx, const float *__restrict__ topk_w, int T, int d,
-             int d_ff, int E, int k, const uint16_t *__restrict__ W2, int d_ff_s,
+             int d_ff, int E, int k, int C, int slot_major, const uint16_t *__restrict__ W2,
+             int d_ff_s,
              const uint16_t *__restrict__ W2s, const uint16_t *__restrict__ Hdec,
              const uint16_t *__restrict__ Hs, float *__restrict__ out, uint32_t *status)
 {
     __shared__ DecPlanSmem P;
     pdl_wait();      // h comes from the w1/w3 kernel
-    build_plan(P, idx, T, E, k, status);
+    build_plan(P, idx, T, E, k, C, slot_major, status);
     const int lane = threadIdx.x & 31;
     const int nwarps = gridDim.x * (blockDim.x >> 5);
     const int n_src = P.U + (W2s ? 1 : 0);
@@ -522,8 +550,8 @@ int launch_dec_w13(const moe_shape_t &s, const uint16_t *x, const int32_t *topk_
     uint16_t *Hs = Hdec + (size_t)s.T * s.k * s.d_ff;
     const uint16_t *ws = s.d_ff_shared ? W13s : nullptr;
 #define MOE_DEC13(M)                                                                            \
-    launch_pdl(k_dec_w13<M>, blocks, 256, st, x, topk_idx, s.T, s.d, s.d_ff, s.E, s.k, W13,    \
-               s.d_ff_shared, ws, Hdec, Hs, status)
+    launch_pdl(k_dec_w13<M>, blocks, 256, st, x, topk_idx, s.T, s.d, s.d_ff, s.E, s.k,        \
+               s.capacity, slot_major(s), W13, s.d_ff_shared, ws, Hdec, Hs, status)
     switch (mt) {
     case 1: MOE_DEC13(1); break;
     case 2: MOE_DEC13(2); break;
@@ -546,8 +574,8 @@ int launch_dec_w2(const moe_shape_t &s, const int32_t *topk_idx, const float *to
     const uint16_t *Hs = Hdec + (size_t)s.T * s.k * s.d_ff;
     const uint16_t *ws = s.d_ff_shared ? W2s : nullptr;
 #define MOE_DEC2(M)                                                                             \
-    launch_pdl(k_dec_w2<M>, blocks, 256, st, topk_idx, topk_w, s.T, s.d, s.d_ff, s.E, s.k, W2, \
-               s.d_ff_shared, ws, Hdec, Hs, out, status)
+    launch_pdl(k_dec_w2<M>, blocks, 256, st, topk_idx, topk_w, s.T, s.d, s.d_ff, s.E, s.k,     \
+               s.capacity, slot_major(s), W2, s.d_ff_shared, ws, Hdec, Hs, out, status)
     switch (mt) {
     case 1: MOE_DEC2(1); break;
     case 2: MOE_DEC2(2); break;

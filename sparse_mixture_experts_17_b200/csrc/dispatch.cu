@@ -226,12 +226,15 @@ __device__ void build_tiles(const int *s_kept, const int32_t *offsets_smem_or_gl
 // The last CTA to finish (ticket counter) scans the per-chunk counts in chunk
 // order, applies the capacity, writes offsets and the GEMM tile list, and
 // re-arms the counter. The result depends only on idx: bit-exact.
+// Slot-major priority: the same per slot, with counts per (chunk, slot), and
+// the scan runs over slots, then chunks, so that every first choice ranks
+// before any second choice.
 __global__ void __launch_bounds__(256) k_hist_scan(
-    const int32_t *__restrict__ idx, int T, int E, int k, int C, int32_t *chunk_counts,
-    int32_t *__restrict__ rank_local, int32_t *counter, int32_t *__restrict__ counts,
-    int32_t *__restrict__ offsets, int32_t *__restrict__ n_kept, int32_t *mt_row0,
-    int32_t *mt_group, int32_t *num_mt, int32_t *mt2_row0, int32_t *mt2_group, int32_t *num_mt2,
-    uint32_t *status)
+    const int32_t *__restrict__ idx, int T, int E, int k, int C, int slot_major,
+    int32_t *chunk_counts, int32_t *__restrict__ rank_local, int32_t *counter,
+    int32_t *__restrict__ counts, int32_t *__restrict__ offsets, int32_t *__restrict__ n_kept,
+    int32_t *mt_row0, int32_t *mt_group, int32_t *num_mt, int32_t *mt2_row0, int32_t *mt2_group,
+    int32_t *num_mt2, uint32_t *status)
 {
     __shared__ uint32_t mask[8][MOE_MAX_E];
     __shared__ int32_t wpre[8][MOE_MAX_E];
@@ -242,57 +245,73 @@ __global__ void __launch_bounds__(256) k_hist_scan(
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int t = blockIdx.x * kChunkTokens + tid;
     const bool live = t < T;
-    for (int i = tid; i < 8 * MOE_MAX_E; i += 256)
-        (&mask[0][0])[i] = 0u;
-    __syncthreads();
 
+    // expert of slot j of this thread's token, -1 if absent, out of range or a
+    // repeat of an earlier slot (those two are flagged)
     bool flagged = false;
-    for (int j = 0; j < k; ++j) {
+    auto slot_expert = [&](int j) {
         int e = live ? idx[(size_t)t * k + j] : -1;
         if (live && (e < 0 || e >= E)) {
             flagged = true;
-            e = -1;
+            return -1;
         }
-        if (e >= 0) {
+        if (e >= 0)
             for (int jj = 0; jj < j; ++jj)
                 if (idx[(size_t)t * k + jj] == e) {
                     flagged = true;
-                    e = -1;
-                    break;
+                    return -1;
                 }
+        return e;
+    };
+    // one group of slots [j0, j1): per-warp lane masks, then per-expert warp
+    // prefixes and the chunk's count (written at chunk_counts[row])
+    auto count_slots = [&](int j0, int j1, size_t row) {
+        for (int i = tid; i < 8 * MOE_MAX_E; i += 256)
+            (&mask[0][0])[i] = 0u;
+        __syncthreads();
+        for (int j = j0; j < j1; ++j) {
+            const int e = slot_expert(j);
+            const uint32_t g = __match_any_sync(kFullMask, e);
+            if (e >= 0 && lane == __ffs(g) - 1)
+                mask[warp][e] |= g;
+            __syncwarp();
         }
-        const uint32_t g = __match_any_sync(kFullMask, e);
-        if (e >= 0 && lane == __ffs(g) - 1)
-            mask[warp][e] |= g;
-        __syncwarp();
+        __syncthreads();
+        for (int e = tid; e < E; e += 256) {
+            int run = 0;
+#pragma unroll
+            for (int w = 0; w < 8; ++w) {
+                wpre[w][e] = run;
+                run += __popc(mask[w][e]);
+            }
+            chunk_counts[row * E + e] = run;
+        }
+        __syncthreads();
+        if (live) {
+            for (int j = j0; j < j1; ++j) {
+                const int e = idx[(size_t)t * k + j];
+                int r = -1;
+                if (e >= 0 && e < E) {
+                    bool dup = false;
+                    for (int jj = 0; jj < j; ++jj)
+                        dup |= (idx[(size_t)t * k + jj] == e);
+                    if (!dup)
+                        r = wpre[warp][e] + __popc(mask[warp][e] & lanemask_lt());
+                }
+                rank_local[(size_t)t * k + j] = r;
+            }
+        }
+        __syncthreads();
+    };
+    if (slot_major) {
+        // chunk_counts[(chunk k + j) E + e]: slot j's assignments only
+        for (int j = 0; j < k; ++j)
+            count_slots(j, j + 1, (size_t)blockIdx.x * k + j);
+    } else {
+        count_slots(0, k, blockIdx.x);
     }
     if (flagged)
         flag_status(status, MOE_ERR_BAD_EXPERT);
-    __syncthreads();
-    for (int e = tid; e < E; e += 256) {
-        int run = 0;
-#pragma unroll
-        for (int w = 0; w < 8; ++w) {
-            wpre[w][e] = run;
-            run += __popc(mask[w][e]);
-        }
-        chunk_counts[(size_t)blockIdx.x * E + e] = run;
-    }
-    __syncthreads();
-    if (live) {
-        for (int j = 0; j < k; ++j) {
-            int e = idx[(size_t)t * k + j];
-            int r = -1;
-            if (e >= 0 && e < E) {
-                bool dup = false;
-                for (int jj = 0; jj < j; ++jj)
-                    dup |= (idx[(size_t)t * k + jj] == e);
-                if (!dup)
-                    r = wpre[warp][e] + __popc(mask[warp][e] & lanemask_lt());
-            }
-            rank_local[(size_t)t * k + j] = r;
-        }
-    }
 
     // ---- the last CTA scans all chunks
     __threadfence();
@@ -307,12 +326,17 @@ __global__ void __launch_bounds__(256) k_hist_scan(
     for (int e = tid; e < MOE_MAX_E; e += 256) {
         int kept = 0;
         if (e < E) {
+            // exclusive prefix in rank order: chunks (row-major), or slots then
+            // chunks (slot-major)
             int run = 0;
-            for (int c = 0; c < nchunks; ++c) {
-                const int v = __ldcg(&chunk_counts[(size_t)c * E + e]);
-                __stcg(&chunk_counts[(size_t)c * E + e], run);
-                run += v;
-            }
+            const int nj = slot_major ? k : 1;
+            for (int j = 0; j < nj; ++j)
+                for (int c = 0; c < nchunks; ++c) {
+                    const size_t i = ((size_t)c * nj + j) * E + e;
+                    const int v = __ldcg(&chunk_counts[i]);
+                    __stcg(&chunk_counts[i], run);
+                    run += v;
+                }
             counts[e] = run;
             kept = (C > 0 && run > C) ? C : run;
         }
@@ -346,19 +370,21 @@ int launch_hist_scan(const moe_shape_t &s, const int32_t *idx, int32_t *chunk_co
     const int nchunks = (s.T + kChunkTokens - 1) / kChunkTokens;
     if (nchunks == 0)
         return MOE_OK;
-    k_hist_scan<<<nchunks, 256, 0, st>>>(idx, s.T, s.E, s.k, s.capacity, chunk_counts,
-                                         rank_local, counter, counts, offsets, n_kept, mt_row0,
-                                         mt_group, num_mt, mt2_row0, mt2_group, num_mt2, status);
+    k_hist_scan<<<nchunks, 256, 0, st>>>(idx, s.T, s.E, s.k, s.capacity, slot_major(s),
+                                         chunk_counts, rank_local, counter, counts, offsets,
+                                         n_kept, mt_row0, mt_group, num_mt, mt2_row0, mt2_group,
+                                         num_mt2, status);
     return launched();
 }
 
 // ---------------------------------------------------------------- permutation
 // One warp per token: lane j < k resolves slot j's permuted row
-// (offsets[e] + chunk base + rank within the chunk, -1 past the capacity);
+// (offsets[e] + chunk base + rank within the chunk, -1 past the capacity;
+// with slot-major priority the base is per (chunk, slot));
 // then the warp copies x[t] once into every kept row with 16-B loads/stores
 // and, when asked, zeroes out[t] (the fused combine accumulates into it).
 __global__ void __launch_bounds__(256) k_permute(
-    const int32_t *__restrict__ idx, int T, int E, int k, int C, int d,
+    const int32_t *__restrict__ idx, int T, int E, int k, int C, int slot_major, int d,
     const int32_t *__restrict__ chunk_base, const int32_t *__restrict__ rank_local,
     const int32_t *__restrict__ offsets, const uint4 *__restrict__ x, int32_t *__restrict__ slot_pos,
     int32_t *__restrict__ perm_token, uint4 *__restrict__ x_perm, float4 *__restrict__ out_zero)
@@ -372,7 +398,9 @@ __global__ void __launch_bounds__(256) k_permute(
         const int e = idx[(size_t)t * k + lane];
         const int rl = rank_local[(size_t)t * k + lane];
         if (e >= 0 && e < E && rl >= 0) {
-            const int r = chunk_base[(size_t)(t / kChunkTokens) * E + e] + rl;
+            const size_t row = slot_major ? (size_t)(t / kChunkTokens) * k + lane
+                                          : (size_t)(t / kChunkTokens);
+            const int r = chunk_base[row * E + e] + rl;
             if (C <= 0 || r < C)
                 pos = offsets[e] + r;
         }
@@ -425,7 +453,7 @@ int launch_permute(const moe_shape_t &s, const int32_t *idx, const int32_t *chun
     if (s.T == 0)
         return MOE_OK;
     k_permute<<<(s.T + 7) / 8, 256, 0, st>>>(
-        idx, s.T, s.E, s.k, s.capacity, s.d, chunk_base, rank_local, offsets,
+        idx, s.T, s.E, s.k, s.capacity, slot_major(s), s.d, chunk_base, rank_local, offsets,
         reinterpret_cast<const uint4 *>(x), slot_pos, perm_token, reinterpret_cast<uint4 *>(x_perm),
         reinterpret_cast<float4 *>(out_zero));
     return launched();

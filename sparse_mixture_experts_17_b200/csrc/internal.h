@@ -25,6 +25,17 @@ constexpr int kBlockM = 128;      // rows of one grouped-GEMM m-tile
 constexpr int32_t kHalfTileBit = 1 << 30;
 constexpr int kChunkTokens = 256; // tokens per histogram chunk (one CTA)
 
+// Capacity ranks in slot-major order (MOE_FLAG_SLOT_PRIORITY with a capacity).
+inline int slot_major(const moe_shape_t &s)
+{
+    return (s.flags & MOE_FLAG_SLOT_PRIORITY) ? 1 : 0;
+}
+// Per-chunk count rows of the histogram: one per chunk, or one per (chunk, slot).
+inline size_t chunk_count_rows(const moe_shape_t &s, size_t nchunks)
+{
+    return nchunks * (slot_major(s) ? (size_t)s.k : 1);
+}
+
 // Scratch layout inside the caller's workspace (byte offsets, 256-B aligned).
 struct WsLayout {
     size_t logits, topk_idx, topk_w;

@@ -115,7 +115,7 @@ WsLayout ws_layout(const moe_shape_t &s)
     L.n_kept = take(4);
     L.counter = take(4);
     L.num_mt = take(4);
-    L.chunk_counts = take((size_t)L.nchunks * E * 4);
+    L.chunk_counts = take(chunk_count_rows(s, L.nchunks) * E * 4);
     L.rank_local = take(N * 4);
     L.slot_pos = take(N * 4);
     L.perm_token = take(N * 4);

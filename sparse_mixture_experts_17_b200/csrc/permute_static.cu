@@ -42,7 +42,7 @@ StaticLayout static_layout(const moe_shape_t &s)
     L.counter = take(4);
     L.n_kept = take(4);
     L.num_mt = take(4);
-    L.chunk_counts = take(nchunks * E * 4);
+    L.chunk_counts = take(chunk_count_rows(s, nchunks) * E * 4);
     L.rank_local = take(N * 4);
     L.mt_row0 = take(max_mt * 4);
     L.mt_group = take(max_mt * 4);

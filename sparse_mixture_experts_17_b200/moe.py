@@ -35,6 +35,7 @@ MOE_FLAG_HOST_IO = 1 << 4
 MOE_FLAG_GEMM_1SM = 1 << 5
 MOE_FLAG_GEMM_2SM = 1 << 6
 MOE_FLAG_EXPERT_CHOICE = 1 << 7
+MOE_FLAG_SLOT_PRIORITY = 1 << 8
 
 MOE_MAX_E = 256
 MOE_MAX_K = 16

@@ -95,12 +95,13 @@ def _random_idx(rng, T, E, k, skew):
     (1000, 16, 4, 200, 1.0), (4096, 128, 8, 320, 1.0), (3000, 256, 8, 0, 1.1),
     (2000, 64, 16, 100, 0.8), (700, 8, 8, 0, 0.0), (513, 3, 1, 50, 2.0),
 ])
-def test_permute_bitexact(T, E, k, C, skew):
+@pytest.mark.parametrize("prio", [False, True], ids=["rowmajor", "slotmajor"])
+def test_permute_bitexact(T, E, k, C, skew, prio):
     rng = np.random.default_rng(T * 3 + E)
     idx = _random_idx(rng, T, E, k, skew)
-    ref = O.dispatch(idx, E, C)
+    ref = O.dispatch(idx, E, C, slot_priority=prio)
     w = small_workload("p", T, 128, 128, E, k, capacity=C)
-    b = Buffers(w)
+    b = Buffers(w, flags=M.MOE_FLAG_SLOT_PRIORITY if prio else 0)
     x = torch.randn(T, 128, device="cuda").to(torch.bfloat16)
     b.idx.copy_(torch.from_numpy(idx))
     M.moe_permute(b.shape, b.idx, x, b.counts, b.offsets, b.slot_pos, b.perm_token, b.x_perm,
@@ -227,6 +228,52 @@ def test_forward_parity(case, flags):
         # a flip anywhere can move later ranks; require none for an exact comparison
         assert same.all()
     assert_layer_close(out[torch.from_numpy(np.nonzero(same)[0]).cuda()], ref["out"][same], name)
+
+
+@pytest.mark.parametrize("flags", [0, M.MOE_FLAG_DETERMINISTIC, M.MOE_FLAG_SIMT_FFN],
+                         ids=["default", "det", "simt"])
+def test_forward_slot_priority(flags):
+    """Capacity with slot-major priority, through moe_forward, on a skewed load
+    where most experts overflow."""
+    w = small_workload("slotprio", 1200, 256, 256, 16, 4, capacity=150, zipf_s=1.2)
+    inp = I.make_inputs(w, "cuda", seed=5)
+    oi = dict(I.oracle_arrays(inp), slot_priority=True)
+    layer = M.MoeLayer(inp, flags=flags | M.MOE_FLAG_SLOT_PRIORITY)
+    logits = torch.empty(w.T, w.E, dtype=torch.float32, device="cuda")
+    idx = torch.empty(w.T, w.k, dtype=torch.int32, device="cuda")
+    out = layer.forward(inp["x"], logits_out=logits, topk_idx_out=idx)
+    torch.cuda.synchronize()
+    assert int(layer.status.item()) == 0
+    ref = O.forward(oi, logits=logits.cpu().numpy())   # identical fp32 logits
+    assert (idx.cpu().numpy() == ref["idx"]).all()
+    drops = (ref["slot_pos"] < 0)
+    assert drops.any() and not drops[:, 0].all()
+    # the row-major order would keep a different set of assignments here
+    kept_rm = O.dispatch(ref["idx"], w.E, w.capacity)["slot_pos"] >= 0
+    assert (kept_rm != (ref["slot_pos"] >= 0)).any()
+    assert_layer_close(out, ref["out"], "slot priority")
+
+
+@pytest.mark.parametrize("T,C", [(2, 1), (8, 2), (16, 3)])
+@pytest.mark.parametrize("prio", [False, True], ids=["rowmajor", "slotmajor"])
+def test_decode_kernels_apply_capacity(T, C, prio):
+    """The decode kernels drop the same assignments as the histogram path."""
+    # a steep load skew (Zipf 3) makes every token pick the same two experts
+    w = small_workload("deccap", T, 512, 256, 4, 2, capacity=C, d_ff_shared=128, zipf_s=3.0)
+    inp = I.make_inputs(w, "cuda", seed=T + C)
+    fl = M.MOE_FLAG_SLOT_PRIORITY if prio else 0
+    oi = dict(I.oracle_arrays(inp), slot_priority=prio)
+    layer = M.MoeLayer(inp, flags=fl)
+    logits = torch.empty(T, w.E, dtype=torch.float32, device="cuda")
+    out_d = layer.forward(inp["x"], logits_out=logits, flags=fl | M.MOE_FLAG_FORCE_DECODE)
+    torch.cuda.synchronize()
+    assert int(layer.status.item()) == 0
+    ref = O.forward(oi, logits=logits.cpu().numpy())
+    assert (ref["slot_pos"] < 0).any()
+    assert_layer_close(out_d, ref["out"], f"decode kernels with capacity T={T}")
+    out_p = layer.forward(inp["x"], flags=fl | M.MOE_FLAG_FORCE_PREFILL)
+    torch.cuda.synchronize()
+    assert_layer_close(out_p, ref["out"], f"tensor-core chain with capacity T={T}")
 
 
 def test_deterministic_flag_is_bitwise_repeatable():
