@@ -51,6 +51,9 @@
  *  R6  the SwiGLU product h is optionally rounded to bf16 (round to nearest,
  *      ties to even) before w2, modelling the one rounding a bf16 tensor-core
  *      path must make; with h_bf16 = 0 the whole layer is pure fp64.
+ *  R7  block-scaled 8-bit experts (precision mode 2): MXFP8 as defined at
+ *      oracle_e4m3_decode, applied to x, to every expert weight row and to h
+ *      along the contraction dimension; the router stays on bf16 weights.
  *
  * Inputs are bf16 bit patterns (uint16) and are widened exactly to double.
  * Error codes: 0 ok, 1 invalid argument, 5 non-finite logit, 6 bad expert id.
@@ -100,6 +103,104 @@ void oracle_bf16_to_f64(int64_t n, const uint16_t *src, double *dst)
 {
     for (int64_t i = 0; i < n; ++i)
         dst[i] = bf16_to_double(src[i]);
+}
+
+/* ---- MXFP8: OCP "Microscaling (MX) Formats" v1.0, element type E4M3 with
+ * one shared E8M0 (power-of-two) scale per block of 32 consecutive elements
+ * along the contraction dimension. The pages name block-scaled 4- and 8-bit
+ * expert weights and activations ("Current Bug: CuTeDSLMoERunner produces
+ * wrong output": per-expert activation and weight scale factors) without
+ * fixing the encoding; reading R7 takes MXFP8 for weights and activations:
+ *  - E4M3: sign, 4 exponent bits (bias 7), 3 mantissa bits, subnormals
+ *    m/8 * 2^-6, largest finite 448, no infinities, S.1111.111 = NaN;
+ *  - the scale of a block is 2^X with X the smallest integer in [-127, 127]
+ *    such that max|v| <= 448 * 2^X (so no element saturates); E8M0 code
+ *    X + 127;
+ *  - each element is v * 2^-X rounded to the nearest E4M3 value, ties to
+ *    even (the sign of a zero result is the sign of v). */
+double oracle_e4m3_decode(int code)
+{
+    const int s = (code >> 7) & 1, e = (code >> 3) & 15, m = code & 7;
+    if (e == 15 && m == 7)
+        return NAN;
+    const double v = (e == 0) ? ldexp((double)m, -9)          /* m/8 * 2^-6 */
+                              : ldexp(8.0 + m, e - 10);       /* (1 + m/8) * 2^(e-7) */
+    return s ? -v : v;
+}
+
+/* Nearest E4M3 value of |v| (ties to even), as in oracle_round_bf16: keep 3
+ * fractional bits in the binade of |v|, or a spacing of 2^-9 below 2^-6;
+ * saturate at 448. Returns the code. */
+int oracle_e4m3_encode(double v)
+{
+    const double a = fabs(v);
+    double r;
+    if (a < ldexp(1.0, -6)) {
+        r = ldexp(nearbyint(ldexp(a, 9)), -9);
+    } else {
+        int e;
+        (void)frexp(a, &e);               /* a = f * 2^e, 0.5 <= f < 1 */
+        const int q = e - 1 - 3;          /* weight of the last mantissa bit */
+        r = ldexp(nearbyint(ldexp(a, -q)), q);
+    }
+    if (r > 448.0)
+        r = 448.0;
+    int code;
+    if (r < ldexp(1.0, -6)) {
+        code = (int)ldexp(r, 9);          /* subnormal (or zero): m = r / 2^-9 */
+    } else {
+        int e;
+        const double f = frexp(r, &e);    /* r = f * 2^e = (1 + m/8) 2^(e-1) */
+        const int m = (int)((2.0 * f - 1.0) * 8.0);
+        code = ((e - 1 + 7) << 3) | m;
+    }
+    return code | (signbit(v) ? 0x80 : 0);
+}
+
+/* Shared exponent X of a block with maximum magnitude amax. */
+int oracle_mx_scale_exp(double amax)
+{
+    int X = -127;
+    while (X < 127 && amax > ldexp(448.0, X))
+        ++X;
+    return X;
+}
+
+/* Quantize rows x K (K a multiple of 32) of doubles to MXFP8:
+ * codes [rows, K] (E4M3), scales [rows, K / 32] (E8M0). */
+int oracle_mx_quantize(int64_t rows, int K, const double *in, uint8_t *codes, uint8_t *scales)
+{
+    if (rows < 0 || K < 32 || K % 32 != 0 || !in || !codes || !scales)
+        return ORC_EINVAL;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int b = 0; b < K / 32; ++b) {
+            const double *v = in + r * K + b * 32;
+            double amax = 0.0;
+            for (int i = 0; i < 32; ++i)
+                if (fabs(v[i]) > amax)
+                    amax = fabs(v[i]);
+            const int X = oracle_mx_scale_exp(amax);
+            scales[r * (K / 32) + b] = (uint8_t)(X + 127);
+            for (int i = 0; i < 32; ++i)
+                codes[r * K + b * 32 + i] = (uint8_t)oracle_e4m3_encode(ldexp(v[i], -X));
+        }
+    return ORC_OK;
+}
+
+/* A row through MXFP8 and back: dst = dequantize(quantize(src)), in place
+ * allowed. */
+static void mx_qdq_row(int K, const double *src, double *dst)
+{
+    for (int b = 0; b < K / 32; ++b) {
+        double amax = 0.0;
+        for (int i = 0; i < 32; ++i)
+            if (fabs(src[b * 32 + i]) > amax)
+                amax = fabs(src[b * 32 + i]);
+        const int X = oracle_mx_scale_exp(amax);
+        for (int i = 0; i < 32; ++i)
+            dst[b * 32 + i] = ldexp(oracle_e4m3_decode(oracle_e4m3_encode(
+                                        ldexp(src[b * 32 + i], -X))), X);
+    }
 }
 
 /* [MIX] "Sparse MoE Block": router_logits = gate(x), gate = Linear(d, E)
@@ -263,30 +364,59 @@ int oracle_dispatch(int T, int E, int k, int C, int slot_major, const int32_t *i
     return ORC_OK;
 }
 
+/* Precision modes of the expert FFN (argument `h_bf16` of the entry points):
+ *   0  pure fp64;
+ *   1  h rounded once to bf16 (reading R6);
+ *   2  MXFP8 (reading R7): x (by the caller), every weight row and h pass
+ *      through MXFP8 along their contraction dimension; products and sums
+ *      of the dequantized values in fp64. */
+#define ORC_MODE_MXFP8 2
+
+/* A weight row widened from bf16, through MXFP8 in mode 2. */
+static void weight_row(int K, const uint16_t *src, int mode, double *dst)
+{
+    for (int i = 0; i < K; ++i)
+        dst[i] = bf16_to_double(src[i]);
+    if (mode == ORC_MODE_MXFP8)
+        mx_qdq_row(K, dst, dst);
+}
+
 /* [MIX] "Expert FFN": y = w2(silu(w1 x) * w3 x); w1, w3 are [d_ff, d],
- * w2 is [d, d_ff] (nn.Linear [out, in]); reading R6 for h. */
+ * w2 is [d, d_ff] (nn.Linear [out, in]); readings R6/R7 for h. `wrow` is
+ * scratch of max(d, d_ff) doubles. */
 static void swiglu_ffn(int d, int d_ff, const double *xv, const uint16_t *w1,
-                       const uint16_t *w3, const uint16_t *w2, int h_bf16,
-                       double *h, double *y)
+                       const uint16_t *w3, const uint16_t *w2, int mode,
+                       double *h, double *y, double *wrow)
 {
     for (int c = 0; c < d_ff; ++c) {
         double g = 0.0, u = 0.0;
-        const uint16_t *r1 = w1 + (int64_t)c * d;
-        const uint16_t *r3 = w3 + (int64_t)c * d;
-        for (int i = 0; i < d; ++i) {
-            g += bf16_to_double(r1[i]) * xv[i];
-            u += bf16_to_double(r3[i]) * xv[i];
-        }
+        weight_row(d, w1 + (int64_t)c * d, mode, wrow);
+        for (int i = 0; i < d; ++i)
+            g += wrow[i] * xv[i];
+        weight_row(d, w3 + (int64_t)c * d, mode, wrow);
+        for (int i = 0; i < d; ++i)
+            u += wrow[i] * xv[i];
         double hv = g / (1.0 + exp(-g)) * u;   /* silu(g) = g * sigmoid(g) */
-        h[c] = h_bf16 ? oracle_round_bf16(hv) : hv;
+        h[c] = (mode == 1) ? oracle_round_bf16(hv) : hv;
     }
+    if (mode == ORC_MODE_MXFP8)
+        mx_qdq_row(d_ff, h, h);
     for (int r = 0; r < d; ++r) {
         double s = 0.0;
-        const uint16_t *r2 = w2 + (int64_t)r * d_ff;
+        weight_row(d_ff, w2 + (int64_t)r * d_ff, mode, wrow);
         for (int c = 0; c < d_ff; ++c)
-            s += bf16_to_double(r2[c]) * h[c];
+            s += wrow[c] * h[c];
         y[r] = s;
     }
+}
+
+/* A token's input row, through MXFP8 in mode 2. */
+static void input_row(int d, const uint16_t *x, int mode, double *xv)
+{
+    for (int i = 0; i < d; ++i)
+        xv[i] = bf16_to_double(x[i]);
+    if (mode == ORC_MODE_MXFP8)
+        mx_qdq_row(d, xv, xv);
 }
 
 /* The layer output for a list of tokens, given the routing:
@@ -319,14 +449,18 @@ int oracle_moe_tokens(int T, int d, int d_ff, int E, int k, int d_ff_s,
             if (e < 0 || e >= E)
                 return ORC_EBADEXPERT;
         }
+    if (h_bf16 == ORC_MODE_MXFP8 && (d % 32 || d_ff % 32 || d_ff_s % 32))
+        return ORC_EINVAL;
     const int hmax = d_ff > d_ff_s ? d_ff : d_ff_s;
+    const int wmax = hmax > d ? hmax : d;
     int rc = ORC_OK;
 #pragma omp parallel
     {
         double *xv = (double *)malloc(sizeof(double) * (size_t)d);
         double *h = (double *)malloc(sizeof(double) * (size_t)hmax);
         double *y = (double *)malloc(sizeof(double) * (size_t)d);
-        if (!xv || !h || !y) {
+        double *wrow = (double *)malloc(sizeof(double) * (size_t)wmax);
+        if (!xv || !h || !y || !wrow) {
 #pragma omp atomic write
             rc = ORC_EINVAL;
         } else {
@@ -334,10 +468,9 @@ int oracle_moe_tokens(int T, int d, int d_ff, int E, int k, int d_ff_s,
             for (int s = 0; s < n_tok; ++s) {
                 const int t = tokens[s];
                 double *o = out + (int64_t)s * d;
-                for (int i = 0; i < d; ++i) {
-                    xv[i] = bf16_to_double(x[(int64_t)t * d + i]);
+                input_row(d, x + (int64_t)t * d, h_bf16, xv);
+                for (int i = 0; i < d; ++i)
                     o[i] = 0.0;
-                }
                 /* routed experts, visited in ascending expert index */
                 for (int e = 0; e < E; ++e) {
                     for (int j = 0; j < k; ++j) {
@@ -346,14 +479,14 @@ int oracle_moe_tokens(int T, int d, int d_ff, int E, int k, int d_ff_s,
                             continue;
                         swiglu_ffn(d, d_ff, xv, W1 + (int64_t)e * d_ff * d,
                                    W3 + (int64_t)e * d_ff * d,
-                                   W2 + (int64_t)e * d * d_ff, h_bf16, h, y);
+                                   W2 + (int64_t)e * d * d_ff, h_bf16, h, y, wrow);
                         for (int i = 0; i < d; ++i)
                             o[i] += w[a] * y[i];
                     }
                 }
                 /* shared expert, weight 1: shared_output + routed_output */
                 if (d_ff_s > 0) {
-                    swiglu_ffn(d, d_ff_s, xv, W1s, W3s, W2s, h_bf16, h, y);
+                    swiglu_ffn(d, d_ff_s, xv, W1s, W3s, W2s, h_bf16, h, y, wrow);
                     for (int i = 0; i < d; ++i)
                         o[i] = y[i] + o[i];
                 }
@@ -362,6 +495,7 @@ int oracle_moe_tokens(int T, int d, int d_ff, int E, int k, int d_ff_s,
         free(xv);
         free(h);
         free(y);
+        free(wrow);
     }
     return rc;
 }
@@ -384,28 +518,31 @@ int oracle_expert_rows(int T, int d, int d_ff, int E, const uint16_t *x,
         if (experts[s] < 0 || experts[s] >= E)
             return ORC_EBADEXPERT;
     }
+    if (h_bf16 == ORC_MODE_MXFP8 && (d % 32 || d_ff % 32))
+        return ORC_EINVAL;
     int rc = ORC_OK;
 #pragma omp parallel
     {
         double *xv = (double *)malloc(sizeof(double) * (size_t)d);
         double *h = (double *)malloc(sizeof(double) * (size_t)d_ff);
-        if (!xv || !h) {
+        double *wrow = (double *)malloc(sizeof(double) * (size_t)(d > d_ff ? d : d_ff));
+        if (!xv || !h || !wrow) {
 #pragma omp atomic write
             rc = ORC_EINVAL;
         } else {
 #pragma omp for schedule(dynamic, 1)
             for (int s = 0; s < n; ++s) {
                 const int t = tokens[s], e = experts[s];
-                for (int i = 0; i < d; ++i)
-                    xv[i] = bf16_to_double(x[(int64_t)t * d + i]);
+                input_row(d, x + (int64_t)t * d, h_bf16, xv);
                 swiglu_ffn(d, d_ff, xv, W1 + (int64_t)e * d_ff * d,
                            W3 + (int64_t)e * d_ff * d,
                            W2 + (int64_t)e * d * d_ff, h_bf16, h,
-                           y_out + (int64_t)s * d);
+                           y_out + (int64_t)s * d, wrow);
             }
         }
         free(xv);
         free(h);
+        free(wrow);
     }
     return rc;
 }

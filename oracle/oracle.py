@@ -58,6 +58,14 @@ def lib():
         L.oracle_num_threads.argtypes = []
         L.oracle_softmax_rows.argtypes = [i, i, P, P]
         L.oracle_expert_choice.argtypes = [i, i, i, P, P, P, P]
+        L.oracle_e4m3_decode.argtypes = [i]
+        L.oracle_e4m3_decode.restype = ctypes.c_double
+        L.oracle_e4m3_encode.argtypes = [ctypes.c_double]
+        L.oracle_e4m3_encode.restype = ctypes.c_int
+        L.oracle_mx_scale_exp.argtypes = [ctypes.c_double]
+        L.oracle_mx_scale_exp.restype = ctypes.c_int
+        L.oracle_mx_quantize.argtypes = [ctypes.c_int64, i, P, P, P]
+        L.oracle_mx_quantize.restype = ctypes.c_int
         L.oracle_softmax_rows.restype = ctypes.c_int
         L.oracle_expert_choice.restype = ctypes.c_int
         for f in (L.oracle_router_logits, L.oracle_route, L.oracle_dispatch,
@@ -129,8 +137,15 @@ def dispatch(idx, E, C=0, slot_priority=False):
                 perm_token=perm_token[: T * k], n_kept=int(n_kept[0]))
 
 
-def moe_tokens(x, W1, W3, W2, idx, w, slot_pos, tokens, h_bf16=True, W1s=None, W3s=None, W2s=None):
-    """Layer output rows (fp64) for the listed tokens, given the routing."""
+def _mode(h_bf16, mx):
+    """Precision mode of the oracle's expert FFN: 0 fp64, 1 bf16 h, 2 MXFP8."""
+    return 2 if mx else int(bool(h_bf16))
+
+
+def moe_tokens(x, W1, W3, W2, idx, w, slot_pos, tokens, h_bf16=True, W1s=None, W3s=None, W2s=None,
+               mx=False):
+    """Layer output rows (fp64) for the listed tokens, given the routing.
+    mx: MXFP8 experts (x, weights and h through MXFP8)."""
     x, W1, W3, W2 = _u16(x), _u16(W1), _u16(W3), _u16(W2)
     T, d = x.shape
     E, d_ff, _ = W1.shape
@@ -146,11 +161,11 @@ def moe_tokens(x, W1, W3, W2, idx, w, slot_pos, tokens, h_bf16=True, W1s=None, W
     out = np.empty((len(tokens), d), np.float64)
     _check("moe_tokens", lib().oracle_moe_tokens(
         T, d, d_ff, E, k, d_ff_s, _p(x), _p(W1), _p(W3), _p(W2), _p(W1s), _p(W3s), _p(W2s),
-        _p(idx), _p(w), _p(slot_pos), int(bool(h_bf16)), len(tokens), _p(tokens), _p(out)))
+        _p(idx), _p(w), _p(slot_pos), _mode(h_bf16, mx), len(tokens), _p(tokens), _p(out)))
     return out
 
 
-def expert_rows(x, W1, W3, W2, tokens, experts, h_bf16=True):
+def expert_rows(x, W1, W3, W2, tokens, experts, h_bf16=True, mx=False):
     """Unweighted expert outputs y[s] = FFN_{experts[s]}(x[tokens[s]]) in fp64."""
     x, W1, W3, W2 = _u16(x), _u16(W1), _u16(W3), _u16(W2)
     T, d = x.shape
@@ -159,12 +174,12 @@ def expert_rows(x, W1, W3, W2, tokens, experts, h_bf16=True):
     experts = np.ascontiguousarray(experts, np.int32)
     y = np.empty((len(tokens), d), np.float64)
     _check("expert_rows", lib().oracle_expert_rows(T, d, d_ff, E, _p(x), _p(W1), _p(W3), _p(W2),
-                                                   int(bool(h_bf16)), len(tokens), _p(tokens),
+                                                   _mode(h_bf16, mx), len(tokens), _p(tokens),
                                                    _p(experts), _p(y)))
     return y
 
 
-def forward(inp: dict, tokens=None, logits=None, h_bf16=True):
+def forward(inp: dict, tokens=None, logits=None, h_bf16=True, mx=False):
     """Whole layer: logits (or the given fp32 logits), routing over all T tokens,
     dispatch with the capacity, then outputs for ``tokens`` (default: all).
 
@@ -183,7 +198,8 @@ def forward(inp: dict, tokens=None, logits=None, h_bf16=True):
     if tokens is None:
         tokens = np.arange(T, dtype=np.int32)
     out = moe_tokens(inp["x"], inp["W1"], inp["W3"], inp["W2"], idx, w, disp["slot_pos"], tokens,
-                     h_bf16=h_bf16, W1s=inp.get("W1s"), W3s=inp.get("W3s"), W2s=inp.get("W2s"))
+                     h_bf16=h_bf16, W1s=inp.get("W1s"), W3s=inp.get("W3s"), W2s=inp.get("W2s"),
+                     mx=mx)
     return dict(L64=L64, L32=L32, idx=idx, w=w, out=out, tokens=np.asarray(tokens, np.int32), **disp)
 
 
@@ -227,3 +243,36 @@ def expert_choice_layer(inp, S32, C, tokens=None, h_bf16=True):
     out = moe_tokens(inp["x"], inp["W1"], inp["W3"], inp["W2"], idx, w, slot, tokens,
                      h_bf16=h_bf16, W1s=inp.get("W1s"), W3s=inp.get("W3s"), W2s=inp.get("W2s"))
     return dict(out=out, tokens=sel_tok, w=sel_w, tokens_eval=np.asarray(tokens, np.int32))
+
+
+# ---------------------------------------------------------------- MXFP8
+
+def e4m3_decode(codes):
+    """E4M3 codes (uint8 array) -> float64 values."""
+    table = np.array([lib().oracle_e4m3_decode(c) for c in range(256)], np.float64)
+    return table[np.asarray(codes, np.uint8)]
+
+
+def e4m3_encode(v: float) -> int:
+    return lib().oracle_e4m3_encode(float(v))
+
+
+def mx_scale_exp(amax: float) -> int:
+    return lib().oracle_mx_scale_exp(float(amax))
+
+
+def mx_quantize(a):
+    """Rows of a [rows, K] (K % 32 == 0) -> (codes u8 [rows, K], scales u8 [rows, K/32])."""
+    a = np.ascontiguousarray(a, np.float64)
+    rows, K = a.shape
+    codes = np.empty((rows, K), np.uint8)
+    scales = np.empty((rows, K // 32), np.uint8)
+    _check("mx_quantize", lib().oracle_mx_quantize(rows, K, _p(a), _p(codes), _p(scales)))
+    return codes, scales
+
+
+def mx_dequantize(codes, scales):
+    """Inverse map of mx_quantize's output back to float64 values."""
+    v = e4m3_decode(codes)
+    X = scales.astype(np.int64) - 127
+    return v * np.repeat(np.exp2(X.astype(np.float64)), 32, axis=1)
