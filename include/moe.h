@@ -83,7 +83,9 @@ enum {
                                         experts average >= 1024 rows, else single-SM) */
     MOE_FLAG_EXPERT_CHOICE = 1 << 7, /* workspace sized for the expert-choice calls
                                         (moe_route_expert_choice, moe_forward_expert_choice) */
-    MOE_FLAG_SLOT_PRIORITY = 1 << 8  /* capacity ranks in slot-major order (see moe_shape_t) */
+    MOE_FLAG_SLOT_PRIORITY = 1 << 8, /* capacity ranks in slot-major order (see moe_shape_t) */
+    MOE_FLAG_MXFP8 = 1 << 9          /* workspace for moe_forward_mxfp8 (MXFP8 experts); the
+                                        bf16 layer calls reject it */
 };
 
 #define MOE_MAX_E 256
@@ -267,6 +269,53 @@ MOE_API int moe_forward_expert_choice(const moe_shape_t *shape, const moe_bf16_t
                                       const moe_bf16_t *W13_shared, const moe_bf16_t *W2_shared,
                                       float *out, uint32_t *status, void *ws, size_t ws_bytes,
                                       moe_stream_t stream);
+
+/* ---- MXFP8 experts: block-scaled 8-bit weights and activations
+ * (the low-precision expert pipeline of "Current Bug: CuTeDSLMoERunner
+ * produces wrong output": per-expert weight and activation scale factors
+ * feeding a block-scaled grouped GEMM; the encoding is OCP "Microscaling (MX)
+ * Formats" v1.0 MXFP8, which the page does not fix):
+ *   - a block is 32 consecutive elements along the contraction dimension
+ *     (d for x and w1/w3, d_ff for h and w2);
+ *   - its scale is 2^X, X the smallest integer in [-127, 127] with
+ *     max|v| <= 448 * 2^X (no element saturates), stored as the E8M0 byte
+ *     X + 127;
+ *   - its elements are E4M3 codes of v * 2^-X, rounded to nearest even.
+ * The router, top-k and dispatch are those of moe_forward (bf16 W_g, fp32
+ * logits); x and h are quantized on the fly; the GEMMs accumulate in fp32;
+ * out is fp32.
+ *
+ * moe_quantize_experts_mxfp8: one-time conversion of bf16 experts.
+ *   W1, W3  [E, d_ff, d] bf16 in; W2 [E, d, d_ff] bf16 in
+ *   W13q    [E, 2*d_ff, d] E4M3 out, packed: for each block b of 64 h
+ *           columns, rows 128b..128b+63 are W1 rows 64b.., rows 128b+64..
+ *           128b+127 are W3 rows 64b.. (gate and up side by side in one
+ *           128-column tile)
+ *   W13sf   [E, 2*d_ff, d/32] E8M0 out (same row order)
+ *   W2q     [E, d, d_ff] E4M3 out; W2sf [E, d, d_ff/32] E8M0 out
+ * With E = 1 and d_ff = d_ff_shared it converts a shared expert. Code
+ * arrays 16-byte aligned, scale arrays 4-byte aligned. */
+MOE_API int moe_quantize_experts_mxfp8(const moe_shape_t *shape, const moe_bf16_t *W1,
+                                       const moe_bf16_t *W3, const moe_bf16_t *W2,
+                                       uint8_t *W13q, uint8_t *W13sf, uint8_t *W2q,
+                                       uint8_t *W2sf, moe_stream_t stream);
+
+/* The layer with MXFP8 experts. Requires MOE_FLAG_MXFP8 in shape->flags
+ * (also when sizing the workspace); MOE_FLAG_HOST_IO is rejected
+ * (MOE_ERR_INVALID_ARG). Arguments as in moe_forward, with the experts (and
+ * the shared expert, when d_ff_shared > 0) as moe_quantize_experts_mxfp8
+ * writes them. MOE_FLAG_DETERMINISTIC, capacity, MOE_FLAG_SLOT_PRIORITY and
+ * the decode / prefill choice (MOE_FLAG_FORCE_*) act as in moe_forward: small
+ * T streams only the chosen experts' codes and scales (8.25 bits a weight);
+ * larger T runs the block-scaled tensor-core GEMMs.
+ * Device errors: MOE_ERR_NONFINITE, MOE_ERR_BAD_EXPERT, MOE_ERR_TIMEOUT. */
+MOE_API int moe_forward_mxfp8(const moe_shape_t *shape, const moe_bf16_t *x, const moe_bf16_t *Wg,
+                              const float *bias, const uint8_t *W13q, const uint8_t *W13sf,
+                              const uint8_t *W2q, const uint8_t *W2sf, const uint8_t *W13s_q,
+                              const uint8_t *W13s_sf, const uint8_t *W2s_q,
+                              const uint8_t *W2s_sf, float *out, float *logits_out,
+                              int32_t *topk_idx_out, uint32_t *status, void *ws, size_t ws_bytes,
+                              moe_stream_t stream);
 
 /* moe_permute without a workspace, for callers that cannot allocate device
  * memory: code running while a stream is captured in global capture mode

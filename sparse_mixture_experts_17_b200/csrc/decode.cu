@@ -29,6 +29,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "mxfp8.cuh"
 #include "topk.cuh"
 
 namespace moe {
@@ -461,6 +462,220 @@ __global__ void __launch_bounds__(256, (MAXT <= 2) ? 4 : 2)
     }
 }
 
+// ---------------------------------------------------------------- MXFP8 experts
+// The same two phases on MXFP8 weights: a lane's 16-byte load carries 16 E4M3
+// codes (twice the elements of a bf16 load) and each 32-element block adds one
+// E8M0 byte, so a chosen expert streams 8.25 bits per weight instead of 16.
+// The activations arrive already through MXFP8 and back (exact in bf16): x
+// before phase 1, h between the phases. Phase 1 writes h in fp32.
+
+// sum over 16 elements of E4M3 code value * bf16 value (fp32)
+__device__ __forceinline__ float dot16_mx(uint4 w, uint4 xa, uint4 xb, float acc)
+{
+    const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+    const uint32_t xx[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 lo = mx_decode2((uint16_t)(ww[i] & 0xffffu));
+        const float2 hi = mx_decode2((uint16_t)(ww[i] >> 16));
+        acc = fmaf(lo.x, bf16lo(xx[2 * i]), acc);
+        acc = fmaf(lo.y, bf16hi(xx[2 * i]), acc);
+        acc = fmaf(hi.x, bf16lo(xx[2 * i + 1]), acc);
+        acc = fmaf(hi.y, bf16hi(xx[2 * i + 1]), acc);
+    }
+    return acc;
+}
+
+template <int MAXT>
+__global__ void __launch_bounds__(256, (MAXT <= 2) ? 4 : 2)
+    k_dec_w13_mx(const uint16_t *__restrict__ xdq, const int32_t *__restrict__ idx, int T, int d,
+                 int d_ff, int E, int k, int C, int slot_major, const uint8_t *__restrict__ W13q,
+                 const uint8_t *__restrict__ W13sf, int d_ff_s, const uint8_t *__restrict__ W13s_q,
+                 const uint8_t *__restrict__ W13s_sf, float *__restrict__ H32,
+                 float *__restrict__ Hs32, uint32_t *status)
+{
+    __shared__ DecPlanSmem P;
+    pdl_wait();
+    pdl_trigger();
+    build_plan(P, idx, T, E, k, C, slot_major, status);
+    const int lane = threadIdx.x & 31;
+    const int nwarps = gridDim.x * (blockDim.x >> 5);
+    const long long routed_units = (long long)P.U * d_ff;
+    const long long units = routed_units + (W13s_q ? d_ff_s : 0);
+    const int nv = d / 16, ldsf = d / kMxBlock;
+    for (long long unit = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; unit < units;
+         unit += nwarps) {
+        const uint8_t *qb, *sb;
+        int a0, na, c, ldh;
+        float *hout;
+        const bool shared = unit >= routed_units;
+        size_t prow;
+        if (!shared) {
+            const int u = (int)(unit / d_ff);
+            c = (int)(unit - (long long)u * d_ff);
+            // packed gate row of h column c; the up row is 64 rows further
+            prow = (size_t)P.uniq[u] * 2 * d_ff + (size_t)(c / 64) * 128 + (c % 64);
+            qb = W13q;
+            sb = W13sf;
+            a0 = P.ustart[u];
+            na = P.ustart[u + 1] - a0;
+            hout = H32;
+            ldh = d_ff;
+        } else {
+            c = (int)(unit - routed_units);
+            prow = (size_t)(c / 64) * 128 + (c % 64);
+            qb = W13s_q;
+            sb = W13s_sf;
+            a0 = 0;
+            na = T;
+            hout = Hs32;
+            ldh = d_ff_s;
+        }
+        const uint4 *gate = reinterpret_cast<const uint4 *>(qb + prow * d);
+        const uint4 *up = reinterpret_cast<const uint4 *>(qb + (prow + 64) * d);
+        const uint8_t *gsf = sb + prow * ldsf;
+        const uint8_t *usf = sb + (prow + 64) * ldsf;
+        const uint4 *xr[MAXT];
+#pragma unroll
+        for (int s = 0; s < MAXT; ++s)
+            xr[s] = reinterpret_cast<const uint4 *>(
+                xdq + (size_t)((s < na) ? (shared ? s : P.list[a0 + s] / k) : 0) * d);
+        float ag[MAXT], au[MAXT];
+#pragma unroll
+        for (int s = 0; s < MAXT; ++s)
+            ag[s] = au[s] = 0.f;
+        for (int cb = 0; cb < nv; cb += 32 * kDecUnroll) {
+            uint4 wg[kDecUnroll], wu[kDecUnroll];
+            uint8_t sg[kDecUnroll], su[kDecUnroll];
+#pragma unroll
+            for (int i = 0; i < kDecUnroll; ++i) {
+                const int ci = cb + lane + 32 * i;
+                if (ci < nv) {
+                    wg[i] = ld_stream_v4(gate + ci);
+                    wu[i] = ld_stream_v4(up + ci);
+                    sg[i] = __ldg(gsf + (ci >> 1));
+                    su[i] = __ldg(usf + (ci >> 1));
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < kDecUnroll; ++i) {
+                const int ci = cb + lane + 32 * i;
+                if (ci >= nv)
+                    continue;
+                const float fg = mx_scale_value(sg[i]), fu = mx_scale_value(su[i]);
+#pragma unroll
+                for (int s = 0; s < MAXT; ++s) {
+                    if (s < na) {
+                        const uint4 xa = __ldg(xr[s] + 2 * ci), xb = __ldg(xr[s] + 2 * ci + 1);
+                        ag[s] = fmaf(fg, dot16_mx(wg[i], xa, xb, 0.f), ag[s]);
+                        au[s] = fmaf(fu, dot16_mx(wu[i], xa, xb, 0.f), au[s]);
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int s = 0; s < MAXT; ++s) {
+            if (s < na) {
+                const float g = warp_sum(ag[s]);
+                const float uu = warp_sum(au[s]);
+                if (lane == 0) {
+                    const int row = shared ? s : P.list[a0 + s];
+                    hout[(size_t)row * ldh + c] = silu_mul(g, uu);
+                }
+            }
+        }
+    }
+}
+
+template <int MAXT>
+__global__ void __launch_bounds__(256, (MAXT <= 2) ? 4 : 2)
+    k_dec_w2_mx(const int32_t *__restrict__ idx, const float *__restrict__ topk_w, int T, int d,
+                int d_ff, int E, int k, int C, int slot_major, const uint8_t *__restrict__ W2q,
+                const uint8_t *__restrict__ W2sf, int d_ff_s, const uint8_t *__restrict__ W2s_q,
+                const uint8_t *__restrict__ W2s_sf, const uint16_t *__restrict__ Hdq,
+                const uint16_t *__restrict__ Hsdq, float *__restrict__ out, uint32_t *status)
+{
+    __shared__ DecPlanSmem P;
+    pdl_wait();      // h comes from the quantization between the phases
+    build_plan(P, idx, T, E, k, C, slot_major, status);
+    const int lane = threadIdx.x & 31;
+    const int nwarps = gridDim.x * (blockDim.x >> 5);
+    const int n_src = P.U + (W2s_q ? 1 : 0);
+    for (int r = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; r < d; r += nwarps) {
+        float acc[MAXT];
+#pragma unroll
+        for (int t = 0; t < MAXT; ++t)
+            acc[t] = 0.f;
+        for (int u = 0; u < n_src; ++u) {
+            const bool shared = (u == P.U);
+            const int ff = shared ? d_ff_s : d_ff;
+            const size_t wr = shared ? (size_t)r : (size_t)P.uniq[u] * d + r;
+            const uint4 *wrow = reinterpret_cast<const uint4 *>((shared ? W2s_q : W2q) + wr * ff);
+            const uint8_t *wsf = (shared ? W2s_sf : W2sf) + wr * (ff / kMxBlock);
+            const int a0 = shared ? 0 : P.ustart[u];
+            const int na = shared ? T : P.ustart[u + 1] - a0;
+            const uint16_t *hb = shared ? Hsdq : Hdq;
+            const uint4 *hr[MAXT];
+            int tk[MAXT];
+            float wt[MAXT];
+#pragma unroll
+            for (int s = 0; s < MAXT; ++s) {
+                const int a = (s < na) ? (shared ? s : P.list[a0 + s]) : 0;
+                hr[s] = reinterpret_cast<const uint4 *>(hb + (size_t)a * ff);
+                tk[s] = shared ? s : a / k;
+                wt[s] = (s < na) ? (shared ? 1.f : topk_w[a]) : 0.f;
+            }
+            const int nv = ff / 16;
+            float pa[MAXT];
+#pragma unroll
+            for (int s = 0; s < MAXT; ++s)
+                pa[s] = 0.f;
+            for (int cb = 0; cb < nv; cb += 32 * kDecUnroll) {
+                uint4 wv[kDecUnroll];
+                uint8_t sc[kDecUnroll];
+#pragma unroll
+                for (int i = 0; i < kDecUnroll; ++i) {
+                    const int ci = cb + lane + 32 * i;
+                    if (ci < nv) {
+                        wv[i] = ld_stream_v4(wrow + ci);
+                        sc[i] = __ldg(wsf + (ci >> 1));
+                    }
+                }
+#pragma unroll
+                for (int i = 0; i < kDecUnroll; ++i) {
+                    const int ci = cb + lane + 32 * i;
+                    if (ci >= nv)
+                        continue;
+                    const float f = mx_scale_value(sc[i]);
+#pragma unroll
+                    for (int s = 0; s < MAXT; ++s)
+                        if (s < na)
+                            pa[s] = fmaf(f, dot16_mx(wv[i], __ldg(hr[s] + 2 * ci),
+                                                     __ldg(hr[s] + 2 * ci + 1), 0.f),
+                                         pa[s]);
+                }
+            }
+#pragma unroll
+            for (int s = 0; s < MAXT; ++s) {
+                if (s < na) {
+#pragma unroll
+                    for (int tt = 0; tt < MAXT; ++tt)
+                        if (tt == tk[s])
+                            acc[tt] = fmaf(wt[s], pa[s], acc[tt]);
+                }
+            }
+        }
+#pragma unroll
+        for (int t = 0; t < MAXT; ++t) {
+            if (t < T) {
+                const float s = warp_sum(acc[t]);
+                if (lane == 0)
+                    out[(size_t)t * d + r] = s;
+            }
+        }
+    }
+}
+
 // ---------------------------------------------------------------- host side
 
 // Launch with programmatic stream serialization (the kernel calls pdl_wait()
@@ -584,6 +799,57 @@ int launch_dec_w2(const moe_shape_t &s, const int32_t *topk_idx, const float *to
     default: MOE_DEC2(16); break;
     }
 #undef MOE_DEC2
+    return launched();
+}
+
+int launch_dec_w13_mx(const moe_shape_t &s, const uint16_t *xdq, const int32_t *topk_idx,
+                      const uint8_t *W13q, const uint8_t *W13sf, const uint8_t *W13s_q,
+                      const uint8_t *W13s_sf, float *H32, uint32_t *status, cudaStream_t st)
+{
+    if (s.T == 0)
+        return MOE_OK;
+    const int mt = maxt_for(s.T);
+    const int blocks = num_sms() * ((mt <= 2) ? 4 : 2);
+    float *Hs = H32 + (size_t)s.T * s.k * s.d_ff;
+    const uint8_t *wq = s.d_ff_shared ? W13s_q : nullptr;
+#define MOE_DEC13MX(M)                                                                          \
+    launch_pdl(k_dec_w13_mx<M>, blocks, 256, st, xdq, topk_idx, s.T, s.d, s.d_ff, s.E, s.k,    \
+               s.capacity, slot_major(s), W13q, W13sf, s.d_ff_shared, wq, W13s_sf, H32, Hs,     \
+               status)
+    switch (mt) {
+    case 1: MOE_DEC13MX(1); break;
+    case 2: MOE_DEC13MX(2); break;
+    case 4: MOE_DEC13MX(4); break;
+    case 8: MOE_DEC13MX(8); break;
+    default: MOE_DEC13MX(16); break;
+    }
+#undef MOE_DEC13MX
+    return launched();
+}
+
+int launch_dec_w2_mx(const moe_shape_t &s, const int32_t *topk_idx, const float *topk_w,
+                     const uint8_t *W2q, const uint8_t *W2sf, const uint8_t *W2s_q,
+                     const uint8_t *W2s_sf, const uint16_t *Hdq, float *out, uint32_t *status,
+                     cudaStream_t st)
+{
+    if (s.T == 0)
+        return MOE_OK;
+    const int mt = maxt_for(s.T);
+    const int blocks = num_sms() * ((mt <= 2) ? 4 : 2);
+    const uint16_t *Hs = Hdq + (size_t)s.T * s.k * s.d_ff;
+    const uint8_t *wq = s.d_ff_shared ? W2s_q : nullptr;
+#define MOE_DEC2MX(M)                                                                           \
+    launch_pdl(k_dec_w2_mx<M>, blocks, 256, st, topk_idx, topk_w, s.T, s.d, s.d_ff, s.E, s.k,  \
+               s.capacity, slot_major(s), W2q, W2sf, s.d_ff_shared, wq, W2s_sf, Hdq, Hs, out,   \
+               status)
+    switch (mt) {
+    case 1: MOE_DEC2MX(1); break;
+    case 2: MOE_DEC2MX(2); break;
+    case 4: MOE_DEC2MX(4); break;
+    case 8: MOE_DEC2MX(8); break;
+    default: MOE_DEC2MX(16); break;
+    }
+#undef MOE_DEC2MX
     return launched();
 }
 

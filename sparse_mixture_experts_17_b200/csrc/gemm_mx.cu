@@ -1,0 +1,490 @@
+// gemm_mx.cu -- persistent grouped GEMM on MXFP8 operands with the
+// block-scaled 5th-generation tensor-core MMA (tcgen05.mma kind::mxf8f6f4
+// .block_scale): C[rows of one expert, :] = A[rows, K] * B_e[:, K]^T where A
+// and B hold E4M3 codes (K-major) and every 32 consecutive K elements of a
+// row share one E8M0 scale. The tensor core applies the scales; C is fp32 in
+// tensor memory (TMEM).
+//
+// The pages' low-precision expert pipeline ("Current Bug: CuTeDSLMoERunner
+// produces wrong output") broke on the layout of the per-expert activation
+// scales: padded 128-row scale blocks per expert did not match the
+// contiguous expert offsets the GEMM indexes by. Here the scales stay plain
+// row-major arrays ([rows, K/32] bytes, indexed exactly like the codes), and
+// the producer warp rearranges each stage's 128 x 4 scale bytes into the
+// tensor core's 32 x 16-byte atom in shared memory. A tile may therefore start
+// at any row, like the bf16 kernel's tiles, and no padding exists.
+//
+// Structure (one CTA per SM, 192 threads), as in gemm_tc.cu:
+//   warp 0     producer: TMA of the 128 x 128-byte A and B code tiles
+//              (128-byte swizzle) and, by all 32 lanes, the stage's A and B
+//              scale bytes into shared memory; STAGES-deep ring
+//   warp 1     allocates TMEM (two 128-column accumulators + the scale
+//              columns); one thread copies the stage's scales into TMEM
+//              (tcgen05.cp 32x128b.warpx4) and issues four M=128 N=128 K=32
+//              block-scaled MMAs, selecting the scale byte of each K step in
+//              the instruction descriptor
+//   warps 2-5  epilogue: SwiGLU followed by MXFP8 quantization of h (each
+//              thread holds one 32-column block of its row, so the block
+//              maximum needs no exchange), or the routing-weighted scatter-add,
+//              or a plain fp32 store
+// Tensor-core copies and MMAs issued by one thread execute in order, so one
+// TMEM scale region serves every stage: the copy for stage s+1 is issued after
+// the MMAs of stage s.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <cstring>
+#include <mutex>
+
+#include "common.cuh"
+#include "internal.h"
+#include "mxfp8.cuh"
+
+namespace moe {
+
+#ifndef MOE_GM_MX_W13
+#define MOE_GM_MX_W13 32
+#endif
+#ifndef MOE_GM_MX_W2
+#define MOE_GM_MX_W2 16
+#endif
+
+struct MxArgs {
+    int kblocks;            // K / 128
+    int sf_ld;              // K / 32: bytes per row of a scale array
+    int n_tiles;
+    int group_m;
+    int b_rows_per_group;
+    const int32_t *mt_row0;
+    const int32_t *mt_group;
+    const int32_t *num_mt_dev;
+    int num_mt_host;
+    const int32_t *seg_offsets;
+    long long rows_valid;
+    long long a_rows, b_rows;
+    const uint8_t *A_sf;
+    const uint8_t *B_sf;
+    void *out;
+    long long ldo;
+    uint8_t *out_sf;
+    long long ldo_sf;
+    const int32_t *perm_token;
+    const int32_t *slot_pos;
+    const float *topk_w;
+    int k;
+    const float *perm_w;
+    uint32_t *status;
+};
+
+struct MxCfg {
+    static constexpr int BM = 128, BN = 128, BK = 128;   // BK in elements = bytes
+    static constexpr int A_BYTES = BM * BK;
+    static constexpr int B_BYTES = BN * BK;
+    static constexpr int SF_BYTES = 512;                  // 128 rows x 4 scale bytes
+    static constexpr int STAGES = 6;
+    static constexpr int TMEM_COLS = 512;
+    static constexpr int SF_COL = 2 * BN;                 // scale columns after the accumulators
+    static constexpr int SMEM_BYTES =
+        1024 + STAGES * (A_BYTES + B_BYTES) + STAGES * 2 * SF_BYTES + 256;
+};
+
+__device__ __forceinline__ void mx_tile_coords(long long tile, int num_mt, int n_tiles,
+                                               int group_m, int &m_idx, int &n_idx)
+{
+    const long long band_size = (long long)group_m * n_tiles;
+    const int band = (int)(tile / band_size);
+    const int first_m = band * group_m;
+    const int rows = min(group_m, num_mt - first_m);
+    const int r = (int)(tile - (long long)band * band_size);
+    m_idx = first_m + r % rows;
+    n_idx = r / rows;
+}
+
+// Shared-memory descriptor of one 32-row x 16-byte scale atom (no swizzle:
+// 8-row core matrices of 16-byte rows, 128 bytes apart).
+__device__ __forceinline__ uint64_t smem_desc_sf(uint32_t smem_addr)
+{
+    uint64_t d = 0;
+    d |= (uint64_t)((smem_addr & 0x3FFFFu) >> 4);
+    d |= (uint64_t)(16u >> 4) << 16;    // leading byte offset (a single 16-byte column)
+    d |= (uint64_t)(128u >> 4) << 32;   // stride byte offset: next 8 rows
+    d |= (uint64_t)1 << 46;             // descriptor version
+    return d;                           // layout type 0: no swizzle
+}
+
+// Instruction descriptor, kind::mxf8f6f4 block-scaled: E4M3 A and B
+// (format 0), K-major, E8M0 scales, fp32 D, M = 128, N = 128; `sf_id` picks
+// the scale byte (K block) of each 32-bit TMEM scale word for A and B.
+__device__ __forceinline__ uint32_t idesc_mx(uint32_t sf_id)
+{
+    return (sf_id << 4)                      // B scale factor id
+           | (1u << 23)                      // scale format: E8M0
+           | ((uint32_t)(MxCfg::BN >> 3) << 17)
+           | ((uint32_t)(MxCfg::BM >> 4) << 24)
+           | (sf_id << 29);                  // A scale factor id
+}
+
+__device__ __forceinline__ void tc_cp_sf(uint32_t taddr, uint64_t desc)
+{
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(desc)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tc_mma_mx(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t sfa, uint32_t sfb,
+                                          uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+        : "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem()
+{
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Four scale words (K blocks 4kb..4kb+3) of rows r0 + 32 i, i = 0..3; rows at
+// or past `rows` read as zero.
+__device__ __forceinline__ uint4 load_sf4(const uint8_t *sf, long long r0, long long rows,
+                                          int sf_ld, int kb)
+{
+    uint32_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const long long r = r0 + 32 * i;
+        w[i] = (r < rows) ? __ldg(reinterpret_cast<const uint32_t *>(sf + r * sf_ld + 4 * kb)) : 0u;
+    }
+    return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+template <int MODE>
+__device__ __forceinline__ void mx_epilogue(const MxArgs &p, uint32_t tb, long long row,
+                                            bool valid, int n_idx)
+{
+    constexpr int BN = MxCfg::BN;
+    if (MODE == EPI_SWIGLU_MX) {
+        // columns [0,64) = gate, [64,128) = up of h columns n_idx*64 ..
+        uint8_t *hq = static_cast<uint8_t *>(p.out) + row * p.ldo + n_idx * 64;
+        uint8_t *hs = p.out_sf + row * p.ldo_sf + n_idx * 2;
+#pragma unroll 1
+        for (int c = 0; c < 2; ++c) {
+            float g[32], u[32];
+            tmem_ld32(tb + c * 32, g);
+            tmem_ld32(tb + 64 + c * 32, u);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+                g[i] = silu_mul(g[i], u[i]);
+            uint32_t q[8];
+            const uint8_t sc = mx_quantize32(g, q);
+            if (valid) {
+                uint4 *dst = reinterpret_cast<uint4 *>(hq + c * 32);
+                dst[0] = make_uint4(q[0], q[1], q[2], q[3]);
+                dst[1] = make_uint4(q[4], q[5], q[6], q[7]);
+                hs[c] = sc;
+            }
+        }
+    } else if (MODE == EPI_COMBINE) {
+        int t = 0;
+        float wgt = 0.f;
+        if (valid) {
+            t = p.perm_token[row];
+            if (p.perm_w) {
+                wgt = p.perm_w[row];
+            } else {
+                for (int j = 0; j < p.k; ++j)
+                    if (p.slot_pos[(long long)t * p.k + j] == row)
+                        wgt = p.topk_w[(long long)t * p.k + j];
+            }
+        }
+        float *o = static_cast<float *>(p.out) + (long long)t * p.ldo + n_idx * BN;
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+            float v[32];
+            tmem_ld32(tb + c * 32, v);
+            tmem_ld_wait();
+            if (valid) {
+                float4 *dst = reinterpret_cast<float4 *>(o + c * 32);
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    atomicAdd(dst + i, make_float4(wgt * v[4 * i], wgt * v[4 * i + 1],
+                                                   wgt * v[4 * i + 2], wgt * v[4 * i + 3]));
+            }
+        }
+    } else {   // EPI_STORE_F32
+        float *o = static_cast<float *>(p.out) + row * p.ldo + n_idx * BN;
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+            float v[32];
+            tmem_ld32(tb + c * 32, v);
+            tmem_ld_wait();
+            if (valid) {
+                float4 *dst = reinterpret_cast<float4 *>(o + c * 32);
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+            }
+        }
+    }
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(192, 1)
+    k_gemm_mx(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+              const MxArgs p)
+{
+    using C = MxCfg;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint8_t *sA = smem;
+    uint8_t *sB = sA + C::STAGES * C::A_BYTES;
+    uint8_t *sSF = sB + C::STAGES * C::B_BYTES;   // per stage: 512 B of A scales, 512 B of B
+    uint64_t *full = reinterpret_cast<uint64_t *>(sSF + C::STAGES * 2 * C::SF_BYTES);
+    uint64_t *empty = full + C::STAGES;
+    uint64_t *tfull = empty + C::STAGES;
+    uint64_t *tempty = tfull + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tempty + 2);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::STAGES; ++s) {
+            mbar_init(&full[s], 32);   // every producer lane arrives (lane 0 with the bytes)
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&tfull[b], 1);
+            mbar_init(&tempty[b], 4);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    const int num_mt = p.num_mt_dev ? *p.num_mt_dev : p.num_mt_host;
+    const long long total = (long long)num_mt * p.n_tiles;
+
+    if (warp == 0) {   // ---------------- producer (whole warp)
+        uint32_t it = 0;
+        bool ok = true;
+        for (long long tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+            int m_idx, n_idx;
+            mx_tile_coords(tile, num_mt, p.n_tiles, p.group_m, m_idx, n_idx);
+            const long long row0 = p.mt_row0 ? p.mt_row0[m_idx] : (long long)m_idx * C::BM;
+            const int grp = p.mt_group ? (p.mt_group[m_idx] & ~kHalfTileBit) : 0;
+            const long long brow = (long long)grp * p.b_rows_per_group + (long long)n_idx * C::BN;
+            for (int kb = 0; kb < p.kblocks; ++kb, ++it) {
+                const int s = it % C::STAGES;
+                const uint32_t ph = (it / C::STAGES) & 1u;
+                // the scale words do not depend on the ring: load before waiting
+                const uint4 fa = load_sf4(p.A_sf, row0 + lane, p.a_rows, p.sf_ld, kb);
+                const uint4 fb = load_sf4(p.B_sf, brow + lane, p.b_rows, p.sf_ld, kb);
+                int got = 1;
+                if (lane == 0)
+                    got = mbar_wait(&empty[s], ph ^ 1u, abort_flag, p.status) ? 1 : 0;
+                if (!__shfl_sync(kFullMask, got, 0)) {
+                    ok = false;
+                    break;
+                }
+                // atom layout: byte (m % 32) * 16 + (m / 32) * 4 + k-block
+                uint8_t *sf = sSF + s * 2 * C::SF_BYTES;
+                reinterpret_cast<uint4 *>(sf)[lane] = fa;
+                reinterpret_cast<uint4 *>(sf + C::SF_BYTES)[lane] = fb;
+                fence_proxy_async_smem();
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(&full[s], C::A_BYTES + C::B_BYTES);
+                    tma_load_2d(sA + s * C::A_BYTES, &tmA, kb * C::BK, (int)row0, &full[s]);
+                    tma_load_2d(sB + s * C::B_BYTES, &tmB, kb * C::BK, (int)brow, &full[s]);
+                } else {
+                    mbar_arrive(&full[s]);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {   // ---------------- MMA issuer
+            const uint32_t sf_a = tmem_base + C::SF_COL;
+            const uint32_t sf_b = tmem_base + C::SF_COL + 4;
+            uint32_t it = 0, local = 0;
+            for (long long tile = blockIdx.x; tile < total; tile += gridDim.x, ++local) {
+                const uint32_t b = local & 1u, aph = (local >> 1) & 1u;
+                if (!mbar_wait(&tempty[b], aph ^ 1u, abort_flag, p.status))
+                    break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + b * C::BN;
+                bool ok = true;
+                for (int kb = 0; kb < p.kblocks; ++kb, ++it) {
+                    const int s = it % C::STAGES;
+                    const uint32_t ph = (it / C::STAGES) & 1u;
+                    if (!mbar_wait(&full[s], ph, abort_flag, p.status)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t sf0 = smem_u32(sSF + s * 2 * C::SF_BYTES);
+                    tc_cp_sf(sf_a, smem_desc_sf(sf0));
+                    tc_cp_sf(sf_b, smem_desc_sf(sf0 + C::SF_BYTES));
+                    const uint32_t a0 = smem_u32(sA + s * C::A_BYTES);
+                    const uint32_t b0 = smem_u32(sB + s * C::B_BYTES);
+#pragma unroll
+                    for (int kk = 0; kk < C::BK / 32; ++kk)
+                        tc_mma_mx(d_tmem, smem_desc_k128(a0 + kk * 32), smem_desc_k128(b0 + kk * 32),
+                                  idesc_mx(kk), sf_a, sf_b, (kb | kk) != 0);
+                    tc_commit(&empty[s]);
+                }
+                if (!ok)
+                    break;
+                tc_commit(&tfull[b]);
+            }
+        }
+    } else {   // ---------------- epilogue warps 2..5
+        const int q = warp & 3;
+        uint32_t local = 0;
+        for (long long tile = blockIdx.x; tile < total; tile += gridDim.x, ++local) {
+            int m_idx, n_idx;
+            mx_tile_coords(tile, num_mt, p.n_tiles, p.group_m, m_idx, n_idx);
+            const long long row0 = p.mt_row0 ? p.mt_row0[m_idx] : (long long)m_idx * C::BM;
+            const int grp = p.mt_group ? (p.mt_group[m_idx] & ~kHalfTileBit) : 0;
+            const long long row_end = p.seg_offsets ? p.seg_offsets[grp + 1] : p.rows_valid;
+            const uint32_t b = local & 1u, aph = (local >> 1) & 1u;
+            if (!mbar_wait(&tfull[b], aph, abort_flag, p.status))
+                break;
+            tc_fence_after();
+            const long long row = row0 + q * 32 + lane;
+            const bool valid = row < row_end;
+            const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + b * C::BN;
+            mx_epilogue<MODE>(p, tb, row, valid, n_idx);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(&tempty[b]);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, C::TMEM_COLS);
+    }
+}
+
+// ---------------------------------------------------------------- host side
+
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn_mx()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    });
+    return fn;
+}
+
+// Row-major byte matrix [rows, cols] as a 2-D TMA tensor; box 128 x 128 bytes,
+// 128-byte swizzle, zero fill out of bounds.
+static int make_tmap_u8(CUtensorMap *m, const void *base, long long cols, long long rows)
+{
+    auto fn = encode_fn_mx();
+    if (!fn)
+        return MOE_ERR_CUDA;
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)cols};
+    cuuint32_t box[2] = {128u, 128u};
+    cuuint32_t estr[2] = {1u, 1u};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
+}
+
+template <int MODE>
+static int launch_mx_impl(const GemmArgs &g, cudaStream_t st)
+{
+    using C = MxCfg;
+    if (g.K % 128 != 0 || g.N % 128 != 0)
+        return MOE_ERR_INVALID_ARG;
+    CUtensorMap tA, tB;
+    int rc = make_tmap_u8(&tA, g.Aq, g.K, g.a_rows);
+    if (rc)
+        return rc;
+    rc = make_tmap_u8(&tB, g.Bq, g.K, g.b_rows_total);
+    if (rc)
+        return rc;
+    MxArgs p;
+    std::memset(&p, 0, sizeof p);
+    p.kblocks = g.K / C::BK;
+    p.sf_ld = g.K / kMxBlock;
+    p.n_tiles = g.N / C::BN;
+    p.group_m = (MODE == EPI_SWIGLU_MX) ? MOE_GM_MX_W13 : MOE_GM_MX_W2;
+    p.b_rows_per_group = g.b_rows_per_group;
+    p.mt_row0 = g.mt_row0;
+    p.mt_group = g.mt_group;
+    p.num_mt_dev = g.num_mt_dev;
+    p.num_mt_host = g.num_mt_host;
+    p.seg_offsets = g.seg_offsets;
+    p.rows_valid = g.rows_valid;
+    p.a_rows = g.a_rows;
+    p.b_rows = g.b_rows_total;
+    p.A_sf = g.A_sf;
+    p.B_sf = g.B_sf;
+    p.out = g.out;
+    p.ldo = g.ldo;
+    p.out_sf = g.out_sf;
+    p.ldo_sf = g.ldo_sf;
+    p.perm_token = g.perm_token;
+    p.slot_pos = g.slot_pos;
+    p.topk_w = g.topk_w;
+    p.k = g.k;
+    p.perm_w = g.perm_w;
+    p.status = g.status;
+
+    static int attr_done[64] = {0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < 64 && !attr_done[dev]) {
+        if (cudaFuncSetAttribute(k_gemm_mx<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 C::SMEM_BYTES) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        attr_done[dev] = 1;
+    }
+    const int max_mt = g.num_mt_dev ? g.max_mt : g.num_mt_host;
+    const long long tiles = (long long)max_mt * p.n_tiles;
+    if (tiles <= 0)
+        return MOE_OK;
+    const int grid = (int)std::min<long long>(tiles, num_sms());
+    k_gemm_mx<MODE><<<grid, 192, C::SMEM_BYTES, st>>>(tA, tB, p);
+    return launched();
+}
+
+int launch_gemm_mx(const GemmArgs &g, cudaStream_t st)
+{
+    switch (g.mode) {
+    case EPI_SWIGLU_MX: return launch_mx_impl<EPI_SWIGLU_MX>(g, st);
+    case EPI_COMBINE: return launch_mx_impl<EPI_COMBINE>(g, st);
+    case EPI_STORE_F32: return launch_mx_impl<EPI_STORE_F32>(g, st);
+    default: return MOE_ERR_INVALID_ARG;
+    }
+}
+
+} // namespace moe

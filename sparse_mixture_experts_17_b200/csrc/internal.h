@@ -48,6 +48,8 @@ struct WsLayout {
     size_t dec_H;
     size_t x_stage, out_stage;
     size_t scores, ec_w;   // expert-choice routing
+    size_t xq, xsf, Hq, Hsf, xq_s, xsf_s, Hsq, Hssf;   // MXFP8 operands
+    size_t dec_xdq, dec_H32;                             // MXFP8 decode
     size_t total;
     int nchunks, max_mt, max_mt2;
 };
@@ -82,7 +84,9 @@ enum EpiMode {
     EPI_SWIGLU = 0,     // H[row, n*128 + c] = bf16(silu(acc[c]) * acc[128 + c])
     EPI_COMBINE = 1,    // out[perm_token[row], :] += w(row) * acc  (fp32 atomics)
     EPI_STORE_F32 = 2,  // out[row, :] = acc  (fp32)
-    EPI_ROUTER = 3      // out[row, n] = acc[n] + bias[n] for n < n_valid
+    EPI_ROUTER = 3,     // out[row, n] = acc[n] + bias[n] for n < n_valid
+    EPI_SWIGLU_MX = 4   // MXFP8 GEMM: h = silu(gate) * up, quantized to MXFP8 codes (out)
+                        // and block scales (out_sf)
 };
 
 struct GemmArgs {
@@ -116,9 +120,14 @@ struct GemmArgs {
     uint32_t *status;
     // 1: 2-SM pair kernel (256 x 256 tiles; the m-tile list must hold 256-row tiles)
     int pair;
+    // MXFP8 GEMM (launch_gemm_mx): E4M3 codes and E8M0 scales [rows, K/32] of A and B
+    const uint8_t *Aq, *A_sf, *Bq, *B_sf;
+    uint8_t *out_sf;          // EPI_SWIGLU_MX: scales of h [rows, ldo_sf]
+    long long ldo_sf;
 };
 
 int launch_gemm_tc(const GemmArgs &g, cudaStream_t st);
+int launch_gemm_mx(const GemmArgs &g, cudaStream_t st);
 int launch_gemm_simt(const GemmArgs &g, cudaStream_t st);
 int num_sms();
 
@@ -136,6 +145,26 @@ int launch_dec_w13(const moe_shape_t &s, const uint16_t *x, const int32_t *topk_
 int launch_dec_w2(const moe_shape_t &s, const int32_t *topk_idx, const float *topk_w,
                   const uint16_t *W2, const uint16_t *W2s, const uint16_t *Hdec, float *out,
                   uint32_t *status, cudaStream_t st);
+
+// ---- MXFP8 quantization (mx_quant.cu)
+int launch_mx_quantize_rows(const uint16_t *src, long long rows, int K, uint8_t *codes,
+                            uint8_t *scales, cudaStream_t st);
+int launch_mx_pack_w13(const moe_shape_t &s, const uint16_t *W1, const uint16_t *W3,
+                       uint8_t *codes, uint8_t *scales, cudaStream_t st);
+int launch_mx_gather(const moe_shape_t &s, const uint16_t *x, const int32_t *slot_pos,
+                     uint8_t *xq, uint8_t *xsf, cudaStream_t st);
+// n values (a multiple of 32) through MXFP8 and back, as bf16 (PDL launch)
+int launch_mx_qdq_bf16(const uint16_t *src, long long n, uint16_t *dst, cudaStream_t st);
+int launch_mx_qdq_f32(const float *src, long long n, uint16_t *dst, cudaStream_t st);
+// decode phases on MXFP8 experts (decode.cu); xdq and Hdq are bf16 values
+// already through MXFP8; H32 receives h in fp32 (routed rows, then shared)
+int launch_dec_w13_mx(const moe_shape_t &s, const uint16_t *xdq, const int32_t *topk_idx,
+                      const uint8_t *W13q, const uint8_t *W13sf, const uint8_t *W13s_q,
+                      const uint8_t *W13s_sf, float *H32, uint32_t *status, cudaStream_t st);
+int launch_dec_w2_mx(const moe_shape_t &s, const int32_t *topk_idx, const float *topk_w,
+                     const uint8_t *W2q, const uint8_t *W2sf, const uint8_t *W2s_q,
+                     const uint8_t *W2s_sf, const uint16_t *Hdq, float *out, uint32_t *status,
+                     cudaStream_t st);
 
 // ---- expert-choice routing (expert_choice.cu)
 int launch_softmax_rows(const moe_shape_t &s, const float *logits, float *scores,

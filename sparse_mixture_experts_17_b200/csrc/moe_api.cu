@@ -124,12 +124,24 @@ WsLayout ws_layout(const moe_shape_t &s)
     L.mt2_row0 = take((size_t)L.max_mt2 * 4);
     L.mt2_group = take((size_t)L.max_mt2 * 4);
     L.num_mt2 = take(4);
-    L.x_perm = take(N * s.d * 2);
-    L.H = take(N * s.d_ff * 2);
-    L.H_shared = take(s.d_ff_shared ? T * s.d_ff_shared * 2 : 0);
+    const bool mx = (s.flags & MOE_FLAG_MXFP8) != 0;
+    const size_t dfs = s.d_ff_shared;
+    L.x_perm = take(mx ? 0 : N * s.d * 2);
+    L.H = take(mx ? 0 : N * s.d_ff * 2);
+    L.H_shared = take(!mx && dfs ? T * dfs * 2 : 0);
     L.Y = take((s.flags & MOE_FLAG_DETERMINISTIC) ? N * s.d * 4 : 0);
     const size_t Td = T < (size_t)MOE_DECODE_MAX_T ? T : (size_t)MOE_DECODE_MAX_T;
-    L.dec_H = take((Td * k * s.d_ff + Td * s.d_ff_shared) * 2);
+    L.dec_H = take((Td * k * s.d_ff + Td * dfs) * 2);
+    L.dec_xdq = take(mx ? Td * s.d * 2 : 0);
+    L.dec_H32 = take(mx ? (Td * k * s.d_ff + Td * dfs) * 4 : 0);
+    L.xq = take(mx ? N * s.d : 0);
+    L.xsf = take(mx ? N * s.d / 32 : 0);
+    L.Hq = take(mx ? N * s.d_ff : 0);
+    L.Hsf = take(mx ? N * s.d_ff / 32 : 0);
+    L.xq_s = take(mx && dfs ? T * s.d : 0);
+    L.xsf_s = take(mx && dfs ? T * s.d / 32 : 0);
+    L.Hsq = take(mx && dfs ? T * dfs : 0);
+    L.Hssf = take(mx && dfs ? T * dfs / 32 : 0);
     L.scores = take(ec ? T * E * 4 : 0);
     L.ec_w = take(ec ? N * 4 : 0);
     L.x_stage = take((s.flags & MOE_FLAG_HOST_IO) ? T * s.d * 2 : 0);
@@ -403,6 +415,207 @@ static int forward_impl(const moe_shape_t &s, const WsLayout &L, void *ws, const
         rc = launch_combine(s, Y, slot_pos, w, shared ? out : nullptr, out, st);
     }
     return rc;
+}
+
+// ---------------------------------------------------------------- MXFP8 experts
+// Grouped MXFP8 GEMMs over the routed rows: w1/w3 with the SwiGLU + MXFP8
+// epilogue into Hq/Hsf, then w2 with the chosen epilogue.
+static int expert_ffn_mx(const moe_shape_t &s, const WsLayout &L, void *ws, const uint8_t *W13q,
+                         const uint8_t *W13sf, const uint8_t *W2q, const uint8_t *W2sf,
+                         const int32_t *offsets, const int32_t *perm_token,
+                         const int32_t *slot_pos, const float *topk_w, float *y_perm, float *out,
+                         uint32_t *status, cudaStream_t st)
+{
+    const long long N = (long long)s.T * s.k;
+    GemmArgs g = gemm_base();
+    g.mode = EPI_SWIGLU_MX;
+    g.Aq = at<uint8_t>(ws, L.xq);
+    g.A_sf = at<uint8_t>(ws, L.xsf);
+    g.a_rows = N;
+    g.Bq = W13q;
+    g.B_sf = W13sf;
+    g.b_rows_total = (long long)s.E * 2 * s.d_ff;
+    g.K = s.d;
+    g.N = 2 * s.d_ff;
+    g.b_rows_per_group = 2 * s.d_ff;
+    set_tiles(g, L, ws, false);
+    g.seg_offsets = offsets;
+    g.out = at<uint8_t>(ws, L.Hq);
+    g.ldo = s.d_ff;
+    g.out_sf = at<uint8_t>(ws, L.Hsf);
+    g.ldo_sf = s.d_ff / 32;
+    g.status = status;
+    int rc;
+    {
+        StageMark m(MOE_STAGE_W13, st);
+        rc = launch_gemm_mx(g, st);
+    }
+    if (rc)
+        return rc;
+    g.Aq = at<uint8_t>(ws, L.Hq);
+    g.A_sf = at<uint8_t>(ws, L.Hsf);
+    g.Bq = W2q;
+    g.B_sf = W2sf;
+    g.b_rows_total = (long long)s.E * s.d;
+    g.K = s.d_ff;
+    g.N = s.d;
+    g.b_rows_per_group = s.d;
+    g.ldo = s.d;
+    g.out_sf = nullptr;
+    if (y_perm) {
+        g.mode = EPI_STORE_F32;
+        g.out = y_perm;
+    } else {
+        g.mode = EPI_COMBINE;
+        g.out = out;
+        g.perm_token = perm_token;
+        g.slot_pos = slot_pos;
+        g.topk_w = topk_w;
+        g.k = s.k;
+    }
+    StageMark m(MOE_STAGE_W2, st);
+    return launch_gemm_mx(g, st);
+}
+
+// Shared expert on all T tokens in MXFP8: quantize x, w1/w3 + SwiGLU + MXFP8,
+// w2 with a plain store into out.
+static int shared_expert_mx(const moe_shape_t &s, const WsLayout &L, void *ws, const uint16_t *x,
+                            const uint8_t *W13q, const uint8_t *W13sf, const uint8_t *W2q,
+                            const uint8_t *W2sf, float *out, uint32_t *status, cudaStream_t st)
+{
+    const int dfs = s.d_ff_shared;
+    int rc = launch_mx_quantize_rows(x, s.T, s.d, at<uint8_t>(ws, L.xq_s), at<uint8_t>(ws, L.xsf_s),
+                                     st);
+    if (rc)
+        return rc;
+    const int mt = (s.T + kBlockM - 1) / kBlockM;
+    GemmArgs g = gemm_base();
+    g.mode = EPI_SWIGLU_MX;
+    g.Aq = at<uint8_t>(ws, L.xq_s);
+    g.A_sf = at<uint8_t>(ws, L.xsf_s);
+    g.a_rows = s.T;
+    g.Bq = W13q;
+    g.B_sf = W13sf;
+    g.b_rows_total = 2LL * dfs;
+    g.K = s.d;
+    g.N = 2 * dfs;
+    g.b_rows_per_group = 2 * dfs;
+    g.num_mt_host = mt;
+    g.max_mt = mt;
+    g.rows_valid = s.T;
+    g.out = at<uint8_t>(ws, L.Hsq);
+    g.ldo = dfs;
+    g.out_sf = at<uint8_t>(ws, L.Hssf);
+    g.ldo_sf = dfs / 32;
+    g.status = status;
+    if ((rc = launch_gemm_mx(g, st)))
+        return rc;
+    g.mode = EPI_STORE_F32;
+    g.Aq = at<uint8_t>(ws, L.Hsq);
+    g.A_sf = at<uint8_t>(ws, L.Hssf);
+    g.Bq = W2q;
+    g.B_sf = W2sf;
+    g.b_rows_total = s.d;
+    g.K = dfs;
+    g.N = s.d;
+    g.b_rows_per_group = s.d;
+    g.out = out;
+    g.ldo = s.d;
+    g.out_sf = nullptr;
+    return launch_gemm_mx(g, st);
+}
+
+static int forward_mx_impl(const moe_shape_t &s, const WsLayout &L, void *ws, const uint16_t *x,
+                           const uint16_t *Wg, const float *bias, const uint8_t *W13q,
+                           const uint8_t *W13sf, const uint8_t *W2q, const uint8_t *W2sf,
+                           const uint8_t *W13s_q, const uint8_t *W13s_sf, const uint8_t *W2s_q,
+                           const uint8_t *W2s_sf, float *out, float *logits_out,
+                           int32_t *idx_out, uint32_t *status, cudaStream_t st)
+{
+    float *logits = logits_out ? logits_out : at<float>(ws, L.logits);
+    int32_t *idx = idx_out ? idx_out : at<int32_t>(ws, L.topk_idx);
+    float *w = at<float>(ws, L.topk_w);
+    int32_t *counter = at<int32_t>(ws, L.counter);
+    const bool force_dec = (s.flags & MOE_FLAG_FORCE_DECODE) != 0;
+    const bool force_pre = (s.flags & MOE_FLAG_FORCE_PREFILL) != 0;
+    if (force_dec && s.T > MOE_DECODE_MAX_T)
+        return MOE_ERR_UNSUPPORTED;
+    const bool decode = force_dec || (!force_pre && s.T <= MOE_DECODE_DEFAULT_T);
+    int rc;
+    if (dec_route_fusable(s)) {
+        StageMark m(MOE_STAGE_ROUTER, st);
+        rc = launch_dec_route(s, x, Wg, bias, logits, idx, w, counter, status, st);
+    } else {
+        {
+            StageMark m(MOE_STAGE_ROUTER, st);
+            rc = router(s, x, Wg, bias, logits, status, st);
+        }
+        if (rc)
+            return rc;
+        StageMark m(MOE_STAGE_TOPK, st);
+        rc = launch_topk(s, logits, idx, w, counter, status, st);
+    }
+    if (rc)
+        return rc;
+    if (decode) {
+        // only the chosen experts' codes and scales are read, each once
+        uint16_t *xdq = at<uint16_t>(ws, L.dec_xdq);
+        float *H32 = at<float>(ws, L.dec_H32);
+        uint16_t *Hdq = at<uint16_t>(ws, L.dec_H);
+        const long long nh = (long long)s.T * s.k * s.d_ff + (long long)s.T * s.d_ff_shared;
+        {
+            StageMark m(MOE_STAGE_DEC_W13, st);
+            rc = launch_mx_qdq_bf16(x, (long long)s.T * s.d, xdq, st);
+            if (!rc)
+                rc = launch_dec_w13_mx(s, xdq, idx, W13q, W13sf, W13s_q, W13s_sf, H32, status, st);
+        }
+        if (rc)
+            return rc;
+        StageMark m(MOE_STAGE_DEC_W2, st);
+        rc = launch_mx_qdq_f32(H32, nh, Hdq, st);
+        if (!rc)
+            rc = launch_dec_w2_mx(s, idx, w, W2q, W2sf, W2s_q, W2s_sf, Hdq, out, status, st);
+        return rc;
+    }
+    const bool det = (s.flags & MOE_FLAG_DETERMINISTIC) != 0;
+    const bool shared = s.d_ff_shared > 0;
+    int32_t *offsets = at<int32_t>(ws, L.offsets);
+    int32_t *chunk = at<int32_t>(ws, L.chunk_counts);
+    int32_t *rank = at<int32_t>(ws, L.rank_local);
+    int32_t *slot_pos = at<int32_t>(ws, L.slot_pos);
+    int32_t *perm_token = at<int32_t>(ws, L.perm_token);
+    {
+        StageMark m(MOE_STAGE_HIST, st);
+        rc = launch_hist_scan(s, idx, chunk, rank, counter, at<int32_t>(ws, L.counts), offsets,
+                              at<int32_t>(ws, L.n_kept), at<int32_t>(ws, L.mt_row0),
+                              at<int32_t>(ws, L.mt_group), at<int32_t>(ws, L.num_mt), nullptr,
+                              nullptr, nullptr, status, st);
+    }
+    if (rc)
+        return rc;
+    {
+        StageMark m(MOE_STAGE_PERMUTE, st);
+        rc = launch_permute(s, idx, chunk, rank, offsets, nullptr, slot_pos, perm_token, nullptr,
+                            (!shared && !det) ? out : nullptr, st);
+        if (!rc)
+            rc = launch_mx_gather(s, x, slot_pos, at<uint8_t>(ws, L.xq), at<uint8_t>(ws, L.xsf),
+                                  st);
+    }
+    if (rc)
+        return rc;
+    if (shared) {
+        StageMark m(MOE_STAGE_SHARED, st);
+        rc = shared_expert_mx(s, L, ws, x, W13s_q, W13s_sf, W2s_q, W2s_sf, out, status, st);
+        if (rc)
+            return rc;
+    }
+    float *Y = det ? at<float>(ws, L.Y) : nullptr;
+    rc = expert_ffn_mx(s, L, ws, W13q, W13sf, W2q, W2sf, offsets, perm_token, slot_pos, w, Y, out,
+                       status, st);
+    if (rc || !det)
+        return rc;
+    StageMark m(MOE_STAGE_COMBINE, st);
+    return launch_combine(s, Y, slot_pos, w, shared ? out : nullptr, out, st);
 }
 
 // ---------------------------------------------------------------- expert-choice routing
@@ -693,6 +906,8 @@ int moe_expert_ffn(const moe_shape_t *shape, const moe_bf16_t *x_perm,
     int rc = check_shape(shape);
     if (rc)
         return rc;
+    if (shape->flags & MOE_FLAG_MXFP8)
+        return MOE_ERR_INVALID_ARG;   // bf16 experts: the MXFP8 workspace has no bf16 buffers
     if (shape->T == 0)
         return MOE_OK;   // empty batch: nothing to read or write
     const moe_shape_t &s = *shape;
@@ -740,6 +955,8 @@ int moe_forward(const moe_shape_t *shape, const moe_bf16_t *x, const moe_bf16_t 
     int rc = check_shape(shape);
     if (rc)
         return rc;
+    if (shape->flags & MOE_FLAG_MXFP8)
+        return MOE_ERR_INVALID_ARG;   // bf16 experts: the MXFP8 workspace has no bf16 buffers
     if (shape->T == 0)
         return MOE_OK;   // empty batch: nothing to read or write
     const moe_shape_t &s = *shape;
@@ -766,6 +983,8 @@ int moe_forward_host(const moe_shape_t *shape, const moe_bf16_t *x_host, const m
     int rc = check_shape(shape);
     if (rc)
         return rc;
+    if (shape->flags & MOE_FLAG_MXFP8)
+        return MOE_ERR_INVALID_ARG;   // bf16 experts: the MXFP8 workspace has no bf16 buffers
     if (shape->T == 0)
         return MOE_OK;   // empty batch: nothing to read or write
     const moe_shape_t &s = *shape;
@@ -832,6 +1051,8 @@ int moe_forward_expert_choice(const moe_shape_t *shape, const moe_bf16_t *x, con
     int rc = check_shape(shape);
     if (rc)
         return rc;
+    if (shape->flags & MOE_FLAG_MXFP8)
+        return MOE_ERR_INVALID_ARG;   // bf16 experts: the MXFP8 workspace has no bf16 buffers
     if ((rc = ec_check(*shape)))
         return rc;
     if (shape->T == 0)
@@ -868,6 +1089,56 @@ int moe_forward_expert_choice(const moe_shape_t *shape, const moe_bf16_t *x, con
     }
     return expert_ffn_core(s, L, ws, x_perm, at<int32_t>(ws, L.offsets), W13, W2, tokens, nullptr,
                            nullptr, nullptr, out, status, st, rows, wts, false);
+}
+
+int moe_quantize_experts_mxfp8(const moe_shape_t *shape, const moe_bf16_t *W1,
+                               const moe_bf16_t *W3, const moe_bf16_t *W2, uint8_t *W13q,
+                               uint8_t *W13sf, uint8_t *W2q, uint8_t *W2sf, moe_stream_t stream)
+{
+    int rc = check_shape(shape);
+    if (rc)
+        return rc;
+    if (shape->T == 0)
+        return MOE_OK;
+    const moe_shape_t &s = *shape;
+    if (!W1 || !W3 || !W2 || !W13q || !W13sf || !W2q || !W2sf || !al16(W1) || !al16(W3) ||
+        !al16(W2) || !al16(W13q) || !al16(W2q) || (reinterpret_cast<uintptr_t>(W13sf) & 3u) ||
+        (reinterpret_cast<uintptr_t>(W2sf) & 3u))
+        return MOE_ERR_INVALID_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if ((rc = launch_mx_pack_w13(s, W1, W3, W13q, W13sf, st)))
+        return rc;
+    return launch_mx_quantize_rows(W2, (long long)s.E * s.d, s.d_ff, W2q, W2sf, st);
+}
+
+int moe_forward_mxfp8(const moe_shape_t *shape, const moe_bf16_t *x, const moe_bf16_t *Wg,
+                      const float *bias, const uint8_t *W13q, const uint8_t *W13sf,
+                      const uint8_t *W2q, const uint8_t *W2sf, const uint8_t *W13s_q,
+                      const uint8_t *W13s_sf, const uint8_t *W2s_q, const uint8_t *W2s_sf,
+                      float *out, float *logits_out, int32_t *topk_idx_out, uint32_t *status,
+                      void *ws, size_t ws_bytes, moe_stream_t stream)
+{
+    int rc = check_shape(shape);
+    if (rc)
+        return rc;
+    if (shape->T == 0)
+        return MOE_OK;
+    const moe_shape_t &s = *shape;
+    if (!(s.flags & MOE_FLAG_MXFP8) || (s.flags & MOE_FLAG_HOST_IO))
+        return MOE_ERR_INVALID_ARG;
+    auto al4 = [](const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; };
+    if (!x || !Wg || !W13q || !W13sf || !W2q || !W2sf || !out || !al16(x) || !al16(Wg) ||
+        !al16(W13q) || !al16(W2q) || !al4(W13sf) || !al4(W2sf) || !al16(out))
+        return MOE_ERR_INVALID_ARG;
+    if (s.d_ff_shared > 0 && (!W13s_q || !W13s_sf || !W2s_q || !W2s_sf || !al16(W13s_q) ||
+                              !al16(W2s_q) || !al4(W13s_sf) || !al4(W2s_sf)))
+        return MOE_ERR_INVALID_ARG;
+    WsLayout L;
+    if ((rc = check_ws(s, ws, ws_bytes, L)))
+        return rc;
+    return forward_mx_impl(s, L, ws, x, Wg, bias, W13q, W13sf, W2q, W2sf, W13s_q, W13s_sf, W2s_q,
+                           W2s_sf, out, logits_out, topk_idx_out, status,
+                           reinterpret_cast<cudaStream_t>(stream));
 }
 
 } // extern "C"

@@ -36,6 +36,7 @@ MOE_FLAG_GEMM_1SM = 1 << 5
 MOE_FLAG_GEMM_2SM = 1 << 6
 MOE_FLAG_EXPERT_CHOICE = 1 << 7
 MOE_FLAG_SLOT_PRIORITY = 1 << 8
+MOE_FLAG_MXFP8 = 1 << 9
 
 MOE_MAX_E = 256
 MOE_MAX_K = 16
@@ -83,6 +84,8 @@ _SIGS = {
     "moe_forward": ([_SHP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P], ctypes.c_int),
     "moe_forward_host": ([_SHP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P], ctypes.c_int),
     "moe_permute_static": ([_SHP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P], ctypes.c_int),
+    "moe_quantize_experts_mxfp8": ([_SHP, _P, _P, _P, _P, _P, _P, _P, _P], ctypes.c_int),
+    "moe_forward_mxfp8": ([_SHP] + [_P] * 16 + [_SZ, _P], ctypes.c_int),
     "moe_route_expert_choice": ([_SHP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P], ctypes.c_int),
     "moe_forward_expert_choice": ([_SHP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P],
                                   ctypes.c_int),
@@ -152,7 +155,7 @@ def _stream(stream):
     return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
 
 
-BF16, F32, I32, U32 = torch.bfloat16, torch.float32, torch.int32, torch.int32
+BF16, F32, I32, U32, U8 = torch.bfloat16, torch.float32, torch.int32, torch.int32, torch.uint8
 
 
 # ---------------------------------------------------------------- entry points
@@ -222,6 +225,36 @@ def moe_forward_expert_choice(shape, x, Wg, bias, W13, W2, W13_shared, W2_shared
         _ptr(W13, BF16, "W13"), _ptr(W2, BF16, "W2"), _ptr(W13_shared, BF16, "W13_shared"),
         _ptr(W2_shared, BF16, "W2_shared"), _ptr(out, F32, "out"), _ptr(status, U32, "status"),
         _ptr(ws, name="ws"), ws.numel(), _stream(stream)))
+
+
+def moe_quantize_experts_mxfp8(shape, W1, W3, W2, stream=None) -> dict:
+    """MXFP8 experts from bf16 ones: dict(W13q, W13sf, W2q, W2sf) (uint8 tensors)."""
+    E, d_ff, d = shape.E, shape.d_ff, shape.d
+    dev = W1.device
+    q = dict(W13q=torch.empty(E, 2 * d_ff, d, dtype=U8, device=dev),
+             W13sf=torch.empty(E, 2 * d_ff, d // 32, dtype=U8, device=dev),
+             W2q=torch.empty(E, d, d_ff, dtype=U8, device=dev),
+             W2sf=torch.empty(E, d, d_ff // 32, dtype=U8, device=dev))
+    _check("moe_quantize_experts_mxfp8", lib().moe_quantize_experts_mxfp8(
+        ctypes.byref(shape), _ptr(W1, BF16, "W1"), _ptr(W3, BF16, "W3"), _ptr(W2, BF16, "W2"),
+        _ptr(q["W13q"], U8, "W13q"), _ptr(q["W13sf"], U8, "W13sf"), _ptr(q["W2q"], U8, "W2q"),
+        _ptr(q["W2sf"], U8, "W2sf"), _stream(stream)))
+    return q
+
+
+def moe_forward_mxfp8(shape, x, Wg, bias, q, qs, out, logits_out, topk_idx_out, status, ws,
+                      stream=None):
+    """q: routed experts, qs: shared expert (or None), both as moe_quantize_experts_mxfp8 gives."""
+    qs = qs or {}
+    _check("moe_forward_mxfp8", lib().moe_forward_mxfp8(
+        ctypes.byref(shape), _ptr(x, BF16, "x"), _ptr(Wg, BF16, "Wg"), _ptr(bias, F32, "bias"),
+        _ptr(q["W13q"], U8, "W13q"), _ptr(q["W13sf"], U8, "W13sf"), _ptr(q["W2q"], U8, "W2q"),
+        _ptr(q["W2sf"], U8, "W2sf"), _ptr(qs.get("W13q"), U8, "W13s_q"),
+        _ptr(qs.get("W13sf"), U8, "W13s_sf"), _ptr(qs.get("W2q"), U8, "W2s_q"),
+        _ptr(qs.get("W2sf"), U8, "W2s_sf"), _ptr(out, F32, "out"),
+        _ptr(logits_out, F32, "logits_out"), _ptr(topk_idx_out, I32, "topk_idx_out"),
+        _ptr(status, U32, "status"), _ptr(ws, name="ws"), ws.numel(), _stream(stream)))
+    return out
 
 
 def moe_expert_ffn(shape, x_perm, expert_offsets, W13, W2, perm_token, slot_pos, topk_w, y_perm,
@@ -299,6 +332,43 @@ class MoeLayer:
         moe_forward(self.shape(T, flags), x, self.Wg, self.bias, self.W13, self.W2, self.W13s,
                     self.W2s, out, logits_out, topk_idx_out, self.status, self.ws, stream)
         return out
+
+
+class MoeLayerMx:
+    """The layer with MXFP8 experts: quantizes the bf16 experts of `inp` once
+    (moe_quantize_experts_mxfp8) and runs moe_forward_mxfp8."""
+
+    def __init__(self, inp: dict, flags: int = 0, T_max: int | None = None):
+        w = inp["workload"]
+        self.workload = w
+        self.flags = flags | MOE_FLAG_MXFP8
+        dev = inp["x"].device
+        self.Wg = inp["wg"].contiguous()
+        self.bias = None if inp.get("bias") is None else inp["bias"].to(dev, torch.float32).contiguous()
+        s = shape_of(w, self.flags)
+        self.q = moe_quantize_experts_mxfp8(s, inp["W1"].contiguous(), inp["W3"].contiguous(),
+                                            inp["W2"].contiguous())
+        self.qs = None
+        if w.d_ff_shared:
+            ss = make_shape(w.T, w.d, w.d_ff_shared, 1, 1)
+            self.qs = moe_quantize_experts_mxfp8(ss, inp["W1s"].contiguous()[None],
+                                                 inp["W3s"].contiguous()[None],
+                                                 inp["W2s"].contiguous()[None])
+        self.T_max = T_max or w.T
+        self.ws = alloc_workspace(shape_of(w, self.flags, T=self.T_max), dev)
+        self.status = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def shape(self, T, flags=None):
+        return shape_of(self.workload, self.flags if flags is None else flags | MOE_FLAG_MXFP8, T=T)
+
+    def forward(self, x, out=None, logits_out=None, topk_idx_out=None, flags=None, stream=None):
+        T = x.shape[0]
+        if T > self.T_max:
+            raise ValueError("T exceeds the workspace's T_max")
+        if out is None:
+            out = torch.empty(T, self.workload.d, dtype=torch.float32, device=x.device)
+        return moe_forward_mxfp8(self.shape(T, flags), x, self.Wg, self.bias, self.q, self.qs, out,
+                                 logits_out, topk_idx_out, self.status, self.ws, stream)
 
 
 # ---------------------------------------------------------------- instrumentation

@@ -98,7 +98,7 @@ def pipeline_from_logits(inp, logits, flags=0, fused=True):
     return b
 
 
-def oracle_tokens_subset(inp, idx, w, slot_pos, tokens, h_bf16=True):
+def oracle_tokens_subset(inp, idx, w, slot_pos, tokens, h_bf16=True, mx=False):
     """Oracle layer rows for `tokens`, copying to the host only the experts
     those tokens keep (the large configurations do not fit on the host whole)."""
     tokens = np.asarray(tokens, np.int32)
@@ -118,7 +118,7 @@ def oracle_tokens_subset(inp, idx, w, slot_pos, tokens, h_bf16=True):
     # dropped slots keep distinct placeholder ids only if the expert count allows; the
     # oracle skips them (slot_pos < 0) after checking the id range
     return O.moe_tokens(x, W1, W3, W2, idx_r, w_t, sp_t, np.arange(len(tokens)), h_bf16=h_bf16,
-                        **kw)
+                        mx=mx, **kw)
 
 
 def sample_tokens(T, disp, n_random=24, seed=0, extra=()):
