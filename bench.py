@@ -304,11 +304,13 @@ def run_ours(a, world, rank, local):
     decode = None
     graphs = None
     expert_choice = None
+    mxfp8 = None
     if a.workload == "prefill" and not a.no_extra:
         decode = run_decode_set(M, w, layer, x, dev, stream, world, peaks)
         graphs = run_graph_set(M, layer, x, dev)
         expert_choice = run_expert_choice_set(M, w, layer, x, dev, stream, world, peaks,
                                               max(3, a.steps // 2))
+        mxfp8 = run_mxfp8_set(M, w, inp, x, dev, stream, world, peaks, max(3, a.steps // 2))
 
     # ---- CPU baseline: the oracle on host cores (rank 0, N = 1 only)
     cpu = None
@@ -342,6 +344,8 @@ def run_ours(a, world, rank, local):
         res["launch_overhead"] = graphs
     if expert_choice is not None:
         res["expert_choice"] = expert_choice
+    if mxfp8 is not None:
+        res["mxfp8"] = mxfp8
     return res
 
 
@@ -457,6 +461,66 @@ def run_expert_choice_set(M, w, layer, x, dev, stream, world, peaks, steps):
             "w13_frac_measured_sustained": round(w13_flops / (k13 / 1e3) / 1e12
                                                  / peaks["bf16_tflops_sustained"], 4),
             "stages_ms": {k: round(v[0] / v[1], 4) for k, v in st.items()}}
+
+
+def run_mxfp8_set(M, w, inp, x, dev, stream, world, peaks, steps):
+    """MXFP8 experts on the same weights and tokens: the prefill step (the
+    block-scaled w1/w3 GEMM against the fp8 dense peak, taken as twice the
+    measured sustained bf16 peak, the nominal fp8:bf16 ratio) and decode at
+    T = 1, 2, 4, 8 (GB/s over the chosen experts' codes and scales)."""
+    lay = M.MoeLayerMx(inp)
+    out = torch.empty(w.T, w.d, dtype=torch.float32, device=dev)
+    idx = torch.empty(w.T, w.k, dtype=torch.int32, device=dev)
+    for _ in range(3):
+        lay.forward(x, out=out, topk_idx_out=idx)
+    torch.cuda.synchronize()
+    if int(lay.status.item()) != 0:
+        raise RuntimeError(f"device status {int(lay.status.item())} (mxfp8)")
+    n_kept = routed_kept(idx, w.E, w.capacity)
+    ms = max_over_ranks(time_loop(lambda: lay.forward(x, out=out), steps, stream), world, dev)
+    M.moe_profile_enable(True)
+    time_loop(lambda: lay.forward(x, out=out), steps, stream)
+    M.moe_profile_enable(False)
+    st = M.moe_profile_read()
+    flops, w13_flops, w2_flops = prefill_flops(w, n_kept)
+    fp8_peak = 2.0 * peaks["bf16_tflops_sustained"]
+    k13 = st["w13"][0] / st["w13"][1]
+    k2 = st["w2"][0] / st["w2"][1]
+    res = {"format": "MXFP8 (E4M3, E8M0 scale per 32) weights, x and h; bf16 router",
+           "prefill": {"tokens_per_s": round(w.T * world / (ms / 1e3), 1), "ms_per_step": round(ms, 4),
+                       "active_tflops": round(flops / (ms / 1e3) / 1e12, 1),
+                       "w13_tflops": round(w13_flops / (k13 / 1e3) / 1e12, 1),
+                       "w13_frac_fp8_peak": round(w13_flops / (k13 / 1e3) / 1e12 / fp8_peak, 4),
+                       "w2_tflops": round(w2_flops / (k2 / 1e3) / 1e12, 1),
+                       "fp8_peak_tflops": fp8_peak,
+                       "fp8_peak_source": "2 x measured bf16_tflops_sustained (nominal ratio)",
+                       "stages_ms": {k: round(v[0] / v[1], 4) for k, v in st.items()}}}
+    dec = {}
+    per_weight = 1.0 + 1.0 / 32.0        # code byte + its share of the block scale
+    for T in I.DECODE_TS:
+        xt = x[:T].contiguous()
+        it = torch.empty(T, w.k, dtype=torch.int32, device=dev)
+        ot = torch.empty(T, w.d, dtype=torch.float32, device=dev)
+        for _ in range(5):
+            lay.forward(xt, out=ot, topk_idx_out=it)
+        torch.cuda.synchronize()
+        U = int(torch.unique(it).numel())
+        nbytes = int(U * 3 * w.d * w.d_ff * per_weight + w.E * w.d * 2 + T * w.d * 2 + T * w.d * 4)
+        msd = max_over_ranks(time_loop(lambda: lay.forward(xt, out=ot), 50, stream), world, dev)
+        M.moe_profile_enable(True)
+        time_loop(lambda: lay.forward(xt, out=ot), 50, stream)
+        M.moe_profile_enable(False)
+        sd = M.moe_profile_read()
+        path = "decode kernels" if "dec_w13" in sd else "tensor-core chain"
+        dec[f"T{T}"] = {"path": path, "tokens_per_s": round(T * world / (msd / 1e3), 1),
+                        "ms_per_step": round(msd, 4), "unique_experts": U,
+                        "bytes_per_step": nbytes, "GB_s": round(nbytes / (msd / 1e3) / 1e9, 1),
+                        "frac_hbm_measured": round(nbytes / (msd / 1e3) / 1e9 / peaks["hbm_gbs"], 4),
+                        "stages_ms": {k: round(v[0] / v[1], 4) for k, v in sd.items()}}
+    res["decode"] = dec
+    del lay
+    torch.cuda.empty_cache()
+    return res
 
 
 def run_reference(a, world, rank):

@@ -16,8 +16,9 @@
 //
 // Structure (one CTA per SM, 192 threads), as in gemm_tc.cu:
 //   warp 0     producer: TMA of the 128 x 128-byte A and B code tiles
-//              (128-byte swizzle) and, by all 32 lanes, the stage's A and B
-//              scale bytes into shared memory; STAGES-deep ring
+//              (128-byte swizzle) and, by all 32 lanes, 4-byte cp.async copies
+//              of the stage's A and B scale words into shared memory, both
+//              completing on the stage's barrier; STAGES-deep ring
 //   warp 1     allocates TMEM (two 128-column accumulators + the scale
 //              columns); one thread copies the stage's scales into TMEM
 //              (tcgen05.cp 32x128b.warpx4) and issues four M=128 N=128 K=32
@@ -27,9 +28,11 @@
 //              thread holds one 32-column block of its row, so the block
 //              maximum needs no exchange), or the routing-weighted scatter-add,
 //              or a plain fp32 store
-// Tensor-core copies and MMAs issued by one thread execute in order, so one
-// TMEM scale region serves every stage: the copy for stage s+1 is issued after
-// the MMAs of stage s.
+// Tensor-core copies and MMAs issued by one thread execute in order. Each
+// ring stage has its own 8 TMEM scale columns (after the 256 accumulator
+// columns), so a stage's copy never waits for the previous stage's MMAs to
+// finish reading; a stage's columns are rewritten only after its MMAs have
+// committed (the producer refills its buffers only then).
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -84,9 +87,13 @@ struct MxCfg {
     static constexpr int STAGES = 6;
     static constexpr int TMEM_COLS = 512;
     static constexpr int SF_COL = 2 * BN;                 // scale columns after the accumulators
+    static constexpr int SF_COLS_PER_STAGE = 8;           // 4 for A's scales, 4 for B's
     static constexpr int SMEM_BYTES =
         1024 + STAGES * (A_BYTES + B_BYTES) + STAGES * 2 * SF_BYTES + 256;
 };
+
+static_assert(MxCfg::SF_COL + MxCfg::STAGES * MxCfg::SF_COLS_PER_STAGE <= MxCfg::TMEM_COLS,
+              "accumulators and per-stage scale columns must fit the TMEM allocation");
 
 __device__ __forceinline__ void mx_tile_coords(long long tile, int num_mt, int n_tiles,
                                                int group_m, int &m_idx, int &n_idx)
@@ -147,18 +154,30 @@ __device__ __forceinline__ void fence_proxy_async_smem()
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-// Four scale words (K blocks 4kb..4kb+3) of rows r0 + 32 i, i = 0..3; rows at
-// or past `rows` read as zero.
-__device__ __forceinline__ uint4 load_sf4(const uint8_t *sf, long long r0, long long rows,
-                                          int sf_ld, int kb)
+// Asynchronous copy of the four scale words (K blocks 4kb..4kb+3) of rows
+// r0 + 32 i, i = 0..3, to dst[4 i .. 4 i + 3]; rows at or past `rows` are
+// zero-filled (source size 0). Completion is tracked by the stage barrier
+// (cp.async.mbarrier.arrive), so the producer never waits on the loads.
+__device__ __forceinline__ void copy_sf4_async(uint8_t *dst, const uint8_t *sf, long long r0,
+                                               long long rows, int sf_ld, int kb)
 {
-    uint32_t w[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         const long long r = r0 + 32 * i;
-        w[i] = (r < rows) ? __ldg(reinterpret_cast<const uint32_t *>(sf + r * sf_ld + 4 * kb)) : 0u;
+        const bool in = r < rows;
+        const uint8_t *src = sf + (in ? r : 0) * sf_ld + 4 * kb;
+        asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_u32(dst + 4 * i)),
+                     "l"(src), "r"(in ? 4 : 0)
+                     : "memory");
     }
-    return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// One arrival on `bar` once every cp.async this thread issued has landed
+// (counted in the barrier's initial arrival count).
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t *bar)
+{
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
 }
 
 template <int MODE>
@@ -254,7 +273,8 @@ __global__ void __launch_bounds__(192, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::STAGES; ++s) {
-            mbar_init(&full[s], 32);   // every producer lane arrives (lane 0 with the bytes)
+            // 32 producer lanes (when their scale copies land) + lane 0 with the TMA bytes
+            mbar_init(&full[s], 33);
             mbar_init(&empty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
@@ -292,9 +312,6 @@ __global__ void __launch_bounds__(192, 1)
             for (int kb = 0; kb < p.kblocks; ++kb, ++it) {
                 const int s = it % C::STAGES;
                 const uint32_t ph = (it / C::STAGES) & 1u;
-                // the scale words do not depend on the ring: load before waiting
-                const uint4 fa = load_sf4(p.A_sf, row0 + lane, p.a_rows, p.sf_ld, kb);
-                const uint4 fb = load_sf4(p.B_sf, brow + lane, p.b_rows, p.sf_ld, kb);
                 int got = 1;
                 if (lane == 0)
                     got = mbar_wait(&empty[s], ph ^ 1u, abort_flag, p.status) ? 1 : 0;
@@ -302,24 +319,22 @@ __global__ void __launch_bounds__(192, 1)
                     ok = false;
                     break;
                 }
-                // atom layout: byte (m % 32) * 16 + (m / 32) * 4 + k-block
+                // atom layout: byte (m % 32) * 16 + (m / 32) * 4 + k-block, so lane l
+                // fills bytes [16 l, 16 l + 16) with rows l, l + 32, l + 64, l + 96
                 uint8_t *sf = sSF + s * 2 * C::SF_BYTES;
-                reinterpret_cast<uint4 *>(sf)[lane] = fa;
-                reinterpret_cast<uint4 *>(sf + C::SF_BYTES)[lane] = fb;
-                fence_proxy_async_smem();
+                copy_sf4_async(sf + 16 * lane, p.A_sf, row0 + lane, p.a_rows, p.sf_ld, kb);
+                copy_sf4_async(sf + C::SF_BYTES + 16 * lane, p.B_sf, brow + lane, p.b_rows,
+                               p.sf_ld, kb);
+                cp_async_arrive_noinc(&full[s]);
                 if (lane == 0) {
                     mbar_arrive_expect_tx(&full[s], C::A_BYTES + C::B_BYTES);
                     tma_load_2d(sA + s * C::A_BYTES, &tmA, kb * C::BK, (int)row0, &full[s]);
                     tma_load_2d(sB + s * C::B_BYTES, &tmB, kb * C::BK, (int)brow, &full[s]);
-                } else {
-                    mbar_arrive(&full[s]);
                 }
             }
         }
     } else if (warp == 1) {
         if (lane == 0) {   // ---------------- MMA issuer
-            const uint32_t sf_a = tmem_base + C::SF_COL;
-            const uint32_t sf_b = tmem_base + C::SF_COL + 4;
             uint32_t it = 0, local = 0;
             for (long long tile = blockIdx.x; tile < total; tile += gridDim.x, ++local) {
                 const uint32_t b = local & 1u, aph = (local >> 1) & 1u;
@@ -336,7 +351,14 @@ __global__ void __launch_bounds__(192, 1)
                         break;
                     }
                     tc_fence_after();
+                    // the scale bytes were written by cp.async (generic proxy);
+                    // tcgen05.cp reads them through the async proxy
+                    fence_proxy_async_smem();
                     const uint32_t sf0 = smem_u32(sSF + s * 2 * C::SF_BYTES);
+                    // each stage has its own scale columns: the copy for this
+                    // stage never overwrites columns that earlier MMAs still read
+                    const uint32_t sf_a = tmem_base + C::SF_COL + s * C::SF_COLS_PER_STAGE;
+                    const uint32_t sf_b = sf_a + 4;
                     tc_cp_sf(sf_a, smem_desc_sf(sf0));
                     tc_cp_sf(sf_b, smem_desc_sf(sf0 + C::SF_BYTES));
                     const uint32_t a0 = smem_u32(sA + s * C::A_BYTES);
