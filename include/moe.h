@@ -291,10 +291,16 @@ MOE_API int moe_forward_expert_choice(const moe_shape_t *shape, const moe_bf16_t
  *           columns, rows 128b..128b+63 are W1 rows 64b.., rows 128b+64..
  *           128b+127 are W3 rows 64b.. (gate and up side by side in one
  *           128-column tile)
- *   W13sf   [E, 2*d_ff, d/32] E8M0 out (same row order)
- *   W2q     [E, d, d_ff] E4M3 out; W2sf [E, d, d_ff/32] E8M0 out
- * With E = 1 and d_ff = d_ff_shared it converts a shared expert. Code
- * arrays 16-byte aligned, scale arrays 4-byte aligned. */
+ *   W13sf   E*2*d_ff*d/32 E8M0 bytes out, in the scale-atom order the
+ *           block-scaled tensor-core MMA reads: the scales of rows
+ *           128t..128t+127 and K elements 128g..128g+127 form the 512-byte
+ *           atom (t * (K/128) + g), inside which row 128t + m, 32-element
+ *           block 4g + j sits at byte (m % 32) * 16 + (m / 32) * 4 + j
+ *           (K = d; rows in W13q's packed order)
+ *   W2q     [E, d, d_ff] E4M3 out; W2sf E*d*d_ff/32 E8M0 bytes out, atoms as
+ *           above with K = d_ff
+ * With E = 1 and d_ff = d_ff_shared it converts a shared expert. All four
+ * arrays 16-byte aligned. */
 MOE_API int moe_quantize_experts_mxfp8(const moe_shape_t *shape, const moe_bf16_t *W1,
                                        const moe_bf16_t *W3, const moe_bf16_t *W2,
                                        uint8_t *W13q, uint8_t *W13sf, uint8_t *W2q,

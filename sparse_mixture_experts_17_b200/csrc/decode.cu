@@ -502,7 +502,7 @@ __global__ void __launch_bounds__(256, (MAXT <= 2) ? 4 : 2)
     const int nwarps = gridDim.x * (blockDim.x >> 5);
     const long long routed_units = (long long)P.U * d_ff;
     const long long units = routed_units + (W13s_q ? d_ff_s : 0);
-    const int nv = d / 16, ldsf = d / kMxBlock;
+    const int nv = d / 16;
     for (long long unit = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; unit < units;
          unit += nwarps) {
         const uint8_t *qb, *sb;
@@ -533,8 +533,9 @@ __global__ void __launch_bounds__(256, (MAXT <= 2) ? 4 : 2)
         }
         const uint4 *gate = reinterpret_cast<const uint4 *>(qb + prow * d);
         const uint4 *up = reinterpret_cast<const uint4 *>(qb + (prow + 64) * d);
-        const uint8_t *gsf = sb + prow * ldsf;
-        const uint8_t *usf = sb + (prow + 64) * ldsf;
+        // scale atoms of the gate and up rows (tile = row / 128)
+        const long long gt = (long long)(prow >> 7), ut = (long long)((prow + 64) >> 7);
+        const int gm = (int)(prow & 127), um = (int)((prow + 64) & 127);
         const uint4 *xr[MAXT];
 #pragma unroll
         for (int s = 0; s < MAXT; ++s)
@@ -553,8 +554,8 @@ __global__ void __launch_bounds__(256, (MAXT <= 2) ? 4 : 2)
                 if (ci < nv) {
                     wg[i] = ld_stream_v4(gate + ci);
                     wu[i] = ld_stream_v4(up + ci);
-                    sg[i] = __ldg(gsf + (ci >> 1));
-                    su[i] = __ldg(usf + (ci >> 1));
+                    sg[i] = __ldg(sb + sf_atom_offset(gt, gm, ci >> 1, d));
+                    su[i] = __ldg(sb + sf_atom_offset(ut, um, ci >> 1, d));
                 }
             }
 #pragma unroll
@@ -611,7 +612,9 @@ __global__ void __launch_bounds__(256, (MAXT <= 2) ? 4 : 2)
             const int ff = shared ? d_ff_s : d_ff;
             const size_t wr = shared ? (size_t)r : (size_t)P.uniq[u] * d + r;
             const uint4 *wrow = reinterpret_cast<const uint4 *>((shared ? W2s_q : W2q) + wr * ff);
-            const uint8_t *wsf = (shared ? W2s_sf : W2sf) + wr * (ff / kMxBlock);
+            const uint8_t *wsf = shared ? W2s_sf : W2sf;
+            const long long wt_tile = (long long)(wr >> 7);
+            const int wt_m = (int)(wr & 127);
             const int a0 = shared ? 0 : P.ustart[u];
             const int na = shared ? T : P.ustart[u + 1] - a0;
             const uint16_t *hb = shared ? Hsdq : Hdq;
@@ -638,7 +641,7 @@ __global__ void __launch_bounds__(256, (MAXT <= 2) ? 4 : 2)
                     const int ci = cb + lane + 32 * i;
                     if (ci < nv) {
                         wv[i] = ld_stream_v4(wrow + ci);
-                        sc[i] = __ldg(wsf + (ci >> 1));
+                        sc[i] = __ldg(wsf + sf_atom_offset(wt_tile, wt_m, ci >> 1, ff));
                     }
                 }
 #pragma unroll

@@ -194,15 +194,18 @@ __device__ __forceinline__ int block_excl_scan_256(int v, int *s_warp, int *tota
 
 // Writes the grouped-GEMM m-tile list for kept counts in s_kept[E]: expert e
 // contributes ceil(kept/tile_m) tiles starting at rows offsets[e] + tile_m i.
+// tile_start (may be NULL) receives each expert's first tile index.
 __device__ void build_tiles(const int *s_kept, const int32_t *offsets_smem_or_global, int E,
                             int tile_m, int32_t *mt_row0, int32_t *mt_group, int32_t *num_mt,
-                            int *s_warp)
+                            int *s_warp, int32_t *tile_start = nullptr)
 {
     const int tid = threadIdx.x;
     const int e = tid;
     const int nt = (e < E) ? (s_kept[e] + tile_m - 1) / tile_m : 0;
     int total;
     const int start = block_excl_scan_256(nt, s_warp, &total);
+    if (e < E && tile_start)
+        tile_start[e] = start;
     if (e < E) {
         const int base = offsets_smem_or_global[e];
         // a last tile of <= 64 rows is marked for the M = 64 MMA (128-row lists only)
@@ -234,7 +237,7 @@ __global__ void __launch_bounds__(256) k_hist_scan(
     int32_t *chunk_counts, int32_t *__restrict__ rank_local, int32_t *counter,
     int32_t *__restrict__ counts, int32_t *__restrict__ offsets, int32_t *__restrict__ n_kept,
     int32_t *mt_row0, int32_t *mt_group, int32_t *num_mt, int32_t *mt2_row0, int32_t *mt2_group,
-    int32_t *num_mt2, uint32_t *status)
+    int32_t *num_mt2, int32_t *tile_start, uint32_t *status)
 {
     __shared__ uint32_t mask[8][MOE_MAX_E];
     __shared__ int32_t wpre[8][MOE_MAX_E];
@@ -354,7 +357,7 @@ __global__ void __launch_bounds__(256) k_hist_scan(
         *n_kept = total;
     }
     __syncthreads();
-    build_tiles(s_kept, s_off, E, kBlockM, mt_row0, mt_group, num_mt, s_warp);
+    build_tiles(s_kept, s_off, E, kBlockM, mt_row0, mt_group, num_mt, s_warp, tile_start);
     if (mt2_row0)
         build_tiles(s_kept, s_off, E, 2 * kBlockM, mt2_row0, mt2_group, num_mt2, s_warp);
     if (tid == 0)
@@ -365,7 +368,7 @@ int launch_hist_scan(const moe_shape_t &s, const int32_t *idx, int32_t *chunk_co
                      int32_t *rank_local, int32_t *counter, int32_t *counts, int32_t *offsets,
                      int32_t *n_kept, int32_t *mt_row0, int32_t *mt_group, int32_t *num_mt,
                      int32_t *mt2_row0, int32_t *mt2_group, int32_t *num_mt2, uint32_t *status,
-                     cudaStream_t st)
+                     cudaStream_t st, int32_t *tile_start)
 {
     const int nchunks = (s.T + kChunkTokens - 1) / kChunkTokens;
     if (nchunks == 0)
@@ -373,7 +376,7 @@ int launch_hist_scan(const moe_shape_t &s, const int32_t *idx, int32_t *chunk_co
     k_hist_scan<<<nchunks, 256, 0, st>>>(idx, s.T, s.E, s.k, s.capacity, slot_major(s),
                                          chunk_counts, rank_local, counter, counts, offsets,
                                          n_kept, mt_row0, mt_group, num_mt, mt2_row0, mt2_group,
-                                         num_mt2, status);
+                                         num_mt2, tile_start, status);
     return launched();
 }
 

@@ -8,17 +8,18 @@
 // The pages' low-precision expert pipeline ("Current Bug: CuTeDSLMoERunner
 // produces wrong output") broke on the layout of the per-expert activation
 // scales: padded 128-row scale blocks per expert did not match the
-// contiguous expert offsets the GEMM indexes by. Here the scales stay plain
-// row-major arrays ([rows, K/32] bytes, indexed exactly like the codes), and
-// the producer warp rearranges each stage's 128 x 4 scale bytes into the
-// tensor core's 32 x 16-byte atom in shared memory. A tile may therefore start
-// at any row, like the bf16 kernel's tiles, and no padding exists.
+// contiguous expert offsets the GEMM indexes by. Here the scales of each
+// 128-row x 128-element tile are stored as one 512-byte atom in the order the
+// tensor core wants (mxfp8.cuh), keyed for activations by the m-tile's index
+// in the device-built tile list (the kernels that produce x's and h's scales
+// place them there) and for weights by row / 128. Expert segments stay
+// contiguous and unpadded, tiles start at any row, and a stage's scales
+// arrive with one 512-byte bulk copy per operand.
 //
 // Structure (one CTA per SM, 192 threads), as in gemm_tc.cu:
-//   warp 0     producer: TMA of the 128 x 128-byte A and B code tiles
-//              (128-byte swizzle) and, by all 32 lanes, 4-byte cp.async copies
-//              of the stage's A and B scale words into shared memory, both
-//              completing on the stage's barrier; STAGES-deep ring
+//   warp 0     producer (one thread): TMA of the 128 x 128-byte A and B code
+//              tiles (128-byte swizzle) and bulk copies of their two scale
+//              atoms, all completing on the stage's barrier; STAGES-deep ring
 //   warp 1     allocates TMEM (two 128-column accumulators + the scale
 //              columns); one thread copies the stage's scales into TMEM
 //              (tcgen05.cp 32x128b.warpx4) and issues four M=128 N=128 K=32
@@ -53,8 +54,7 @@ namespace moe {
 #endif
 
 struct MxArgs {
-    int kblocks;            // K / 128
-    int sf_ld;              // K / 32: bytes per row of a scale array
+    int kblocks;            // K / 128 (= scale atoms per tile row band)
     int n_tiles;
     int group_m;
     int b_rows_per_group;
@@ -64,13 +64,11 @@ struct MxArgs {
     int num_mt_host;
     const int32_t *seg_offsets;
     long long rows_valid;
-    long long a_rows, b_rows;
     const uint8_t *A_sf;
     const uint8_t *B_sf;
     void *out;
     long long ldo;
     uint8_t *out_sf;
-    long long ldo_sf;
     const int32_t *perm_token;
     const int32_t *slot_pos;
     const float *topk_w;
@@ -149,46 +147,25 @@ __device__ __forceinline__ void tc_mma_mx(uint32_t d_tmem, uint64_t a_desc, uint
         : "memory");
 }
 
-__device__ __forceinline__ void fence_proxy_async_smem()
+// 1-D bulk copy global -> shared (16-byte aligned, size a multiple of 16),
+// completion counted in bytes on `bar`.
+__device__ __forceinline__ void bulk_load(void *smem_dst, const void *src, uint32_t bytes,
+                                          uint64_t *bar)
 {
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
-// Asynchronous copy of the four scale words (K blocks 4kb..4kb+3) of rows
-// r0 + 32 i, i = 0..3, to dst[4 i .. 4 i + 3]; rows at or past `rows` are
-// zero-filled (source size 0). Completion is tracked by the stage barrier
-// (cp.async.mbarrier.arrive), so the producer never waits on the loads.
-__device__ __forceinline__ void copy_sf4_async(uint8_t *dst, const uint8_t *sf, long long r0,
-                                               long long rows, int sf_ld, int kb)
-{
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const long long r = r0 + 32 * i;
-        const bool in = r < rows;
-        const uint8_t *src = sf + (in ? r : 0) * sf_ld + 4 * kb;
-        asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_u32(dst + 4 * i)),
-                     "l"(src), "r"(in ? 4 : 0)
-                     : "memory");
-    }
-}
-
-// One arrival on `bar` once every cp.async this thread issued has landed
-// (counted in the barrier's initial arrival count).
-__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t *bar)
-{
-    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar))
-                 : "memory");
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        ::"r"(smem_u32(smem_dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
 }
 
 template <int MODE>
 __device__ __forceinline__ void mx_epilogue(const MxArgs &p, uint32_t tb, long long row,
-                                            bool valid, int n_idx)
+                                            bool valid, int n_idx, int m_idx, int m)
 {
     constexpr int BN = MxCfg::BN;
     if (MODE == EPI_SWIGLU_MX) {
         // columns [0,64) = gate, [64,128) = up of h columns n_idx*64 ..
         uint8_t *hq = static_cast<uint8_t *>(p.out) + row * p.ldo + n_idx * 64;
-        uint8_t *hs = p.out_sf + row * p.ldo_sf + n_idx * 2;
 #pragma unroll 1
         for (int c = 0; c < 2; ++c) {
             float g[32], u[32];
@@ -204,7 +181,8 @@ __device__ __forceinline__ void mx_epilogue(const MxArgs &p, uint32_t tb, long l
                 uint4 *dst = reinterpret_cast<uint4 *>(hq + c * 32);
                 dst[0] = make_uint4(q[0], q[1], q[2], q[3]);
                 dst[1] = make_uint4(q[4], q[5], q[6], q[7]);
-                hs[c] = sc;
+                // h's scales in the atom layout of this m-tile (K of h = ldo)
+                p.out_sf[sf_atom_offset(m_idx, m, 2 * n_idx + c, (int)p.ldo)] = sc;
             }
         }
     } else if (MODE == EPI_COMBINE) {
@@ -273,8 +251,7 @@ __global__ void __launch_bounds__(192, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::STAGES; ++s) {
-            // 32 producer lanes (when their scale copies land) + lane 0 with the TMA bytes
-            mbar_init(&full[s], 33);
+            mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
@@ -300,36 +277,31 @@ __global__ void __launch_bounds__(192, 1)
     const int num_mt = p.num_mt_dev ? *p.num_mt_dev : p.num_mt_host;
     const long long total = (long long)num_mt * p.n_tiles;
 
-    if (warp == 0) {   // ---------------- producer (whole warp)
-        uint32_t it = 0;
-        bool ok = true;
-        for (long long tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
-            int m_idx, n_idx;
-            mx_tile_coords(tile, num_mt, p.n_tiles, p.group_m, m_idx, n_idx);
-            const long long row0 = p.mt_row0 ? p.mt_row0[m_idx] : (long long)m_idx * C::BM;
-            const int grp = p.mt_group ? (p.mt_group[m_idx] & ~kHalfTileBit) : 0;
-            const long long brow = (long long)grp * p.b_rows_per_group + (long long)n_idx * C::BN;
-            for (int kb = 0; kb < p.kblocks; ++kb, ++it) {
-                const int s = it % C::STAGES;
-                const uint32_t ph = (it / C::STAGES) & 1u;
-                int got = 1;
-                if (lane == 0)
-                    got = mbar_wait(&empty[s], ph ^ 1u, abort_flag, p.status) ? 1 : 0;
-                if (!__shfl_sync(kFullMask, got, 0)) {
-                    ok = false;
-                    break;
-                }
-                // atom layout: byte (m % 32) * 16 + (m / 32) * 4 + k-block, so lane l
-                // fills bytes [16 l, 16 l + 16) with rows l, l + 32, l + 64, l + 96
-                uint8_t *sf = sSF + s * 2 * C::SF_BYTES;
-                copy_sf4_async(sf + 16 * lane, p.A_sf, row0 + lane, p.a_rows, p.sf_ld, kb);
-                copy_sf4_async(sf + C::SF_BYTES + 16 * lane, p.B_sf, brow + lane, p.b_rows,
-                               p.sf_ld, kb);
-                cp_async_arrive_noinc(&full[s]);
-                if (lane == 0) {
-                    mbar_arrive_expect_tx(&full[s], C::A_BYTES + C::B_BYTES);
+    if (warp == 0) {
+        if (lane == 0) {   // ---------------- producer
+            uint32_t it = 0;
+            bool ok = true;
+            for (long long tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+                int m_idx, n_idx;
+                mx_tile_coords(tile, num_mt, p.n_tiles, p.group_m, m_idx, n_idx);
+                const long long row0 = p.mt_row0 ? p.mt_row0[m_idx] : (long long)m_idx * C::BM;
+                const int grp = p.mt_group ? (p.mt_group[m_idx] & ~kHalfTileBit) : 0;
+                const long long brow = (long long)grp * p.b_rows_per_group + (long long)n_idx * C::BN;
+                const uint8_t *sfa = p.A_sf + (long long)m_idx * p.kblocks * kSfAtomBytes;
+                const uint8_t *sfb = p.B_sf + (brow >> 7) * p.kblocks * kSfAtomBytes;
+                for (int kb = 0; kb < p.kblocks; ++kb, ++it) {
+                    const int s = it % C::STAGES;
+                    const uint32_t ph = (it / C::STAGES) & 1u;
+                    if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag, p.status)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t *sf = sSF + s * 2 * C::SF_BYTES;
+                    mbar_arrive_expect_tx(&full[s], C::A_BYTES + C::B_BYTES + 2 * C::SF_BYTES);
                     tma_load_2d(sA + s * C::A_BYTES, &tmA, kb * C::BK, (int)row0, &full[s]);
                     tma_load_2d(sB + s * C::B_BYTES, &tmB, kb * C::BK, (int)brow, &full[s]);
+                    bulk_load(sf, sfa + kb * kSfAtomBytes, C::SF_BYTES, &full[s]);
+                    bulk_load(sf + C::SF_BYTES, sfb + kb * kSfAtomBytes, C::SF_BYTES, &full[s]);
                 }
             }
         }
@@ -351,9 +323,6 @@ __global__ void __launch_bounds__(192, 1)
                         break;
                     }
                     tc_fence_after();
-                    // the scale bytes were written by cp.async (generic proxy);
-                    // tcgen05.cp reads them through the async proxy
-                    fence_proxy_async_smem();
                     const uint32_t sf0 = smem_u32(sSF + s * 2 * C::SF_BYTES);
                     // each stage has its own scale columns: the copy for this
                     // stage never overwrites columns that earlier MMAs still read
@@ -390,7 +359,7 @@ __global__ void __launch_bounds__(192, 1)
             const long long row = row0 + q * 32 + lane;
             const bool valid = row < row_end;
             const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + b * C::BN;
-            mx_epilogue<MODE>(p, tb, row, valid, n_idx);
+            mx_epilogue<MODE>(p, tb, row, valid, n_idx, m_idx, q * 32 + lane);
             tc_fence_before();
             __syncwarp();
             if (lane == 0)
@@ -456,7 +425,6 @@ static int launch_mx_impl(const GemmArgs &g, cudaStream_t st)
     MxArgs p;
     std::memset(&p, 0, sizeof p);
     p.kblocks = g.K / C::BK;
-    p.sf_ld = g.K / kMxBlock;
     p.n_tiles = g.N / C::BN;
     p.group_m = (MODE == EPI_SWIGLU_MX) ? MOE_GM_MX_W13 : MOE_GM_MX_W2;
     p.b_rows_per_group = g.b_rows_per_group;
@@ -466,14 +434,11 @@ static int launch_mx_impl(const GemmArgs &g, cudaStream_t st)
     p.num_mt_host = g.num_mt_host;
     p.seg_offsets = g.seg_offsets;
     p.rows_valid = g.rows_valid;
-    p.a_rows = g.a_rows;
-    p.b_rows = g.b_rows_total;
     p.A_sf = g.A_sf;
     p.B_sf = g.B_sf;
     p.out = g.out;
     p.ldo = g.ldo;
     p.out_sf = g.out_sf;
-    p.ldo_sf = g.ldo_sf;
     p.perm_token = g.perm_token;
     p.slot_pos = g.slot_pos;
     p.topk_w = g.topk_w;

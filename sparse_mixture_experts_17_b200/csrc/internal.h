@@ -50,6 +50,7 @@ struct WsLayout {
     size_t scores, ec_w;   // expert-choice routing
     size_t xq, xsf, Hq, Hsf, xq_s, xsf_s, Hsq, Hssf;   // MXFP8 operands
     size_t dec_xdq, dec_H32;                             // MXFP8 decode
+    size_t tile_start;                                   // first m-tile of each expert
     size_t total;
     int nchunks, max_mt, max_mt2;
 };
@@ -66,7 +67,7 @@ int launch_hist_scan(const moe_shape_t &s, const int32_t *idx, int32_t *chunk_co
                      int32_t *rank_local, int32_t *counter, int32_t *counts, int32_t *offsets,
                      int32_t *n_kept, int32_t *mt_row0, int32_t *mt_group, int32_t *num_mt,
                      int32_t *mt2_row0, int32_t *mt2_group, int32_t *num_mt2, uint32_t *status,
-                     cudaStream_t st);
+                     cudaStream_t st, int32_t *tile_start = nullptr);
 int launch_permute(const moe_shape_t &s, const int32_t *idx, const int32_t *chunk_base,
                    const int32_t *rank_local, const int32_t *offsets, const uint16_t *x,
                    int32_t *slot_pos, int32_t *perm_token, uint16_t *x_perm, float *out_zero,
@@ -120,10 +121,10 @@ struct GemmArgs {
     uint32_t *status;
     // 1: 2-SM pair kernel (256 x 256 tiles; the m-tile list must hold 256-row tiles)
     int pair;
-    // MXFP8 GEMM (launch_gemm_mx): E4M3 codes and E8M0 scales [rows, K/32] of A and B
+    // MXFP8 GEMM (launch_gemm_mx): E4M3 codes of A and B and their E8M0 scales
+    // in the atom layout (mxfp8.cuh): A's keyed by m-tile index, B's by row/128
     const uint8_t *Aq, *A_sf, *Bq, *B_sf;
-    uint8_t *out_sf;          // EPI_SWIGLU_MX: scales of h [rows, ldo_sf]
-    long long ldo_sf;
+    uint8_t *out_sf;          // EPI_SWIGLU_MX: scales of h, atom layout keyed by m-tile
 };
 
 int launch_gemm_tc(const GemmArgs &g, cudaStream_t st);
@@ -151,7 +152,8 @@ int launch_mx_quantize_rows(const uint16_t *src, long long rows, int K, uint8_t 
                             uint8_t *scales, cudaStream_t st);
 int launch_mx_pack_w13(const moe_shape_t &s, const uint16_t *W1, const uint16_t *W3,
                        uint8_t *codes, uint8_t *scales, cudaStream_t st);
-int launch_mx_gather(const moe_shape_t &s, const uint16_t *x, const int32_t *slot_pos,
+int launch_mx_gather(const moe_shape_t &s, const uint16_t *x, const int32_t *idx,
+                     const int32_t *slot_pos, const int32_t *offsets, const int32_t *tile_start,
                      uint8_t *xq, uint8_t *xsf, cudaStream_t st);
 // n values (a multiple of 32) through MXFP8 and back, as bf16 (PDL launch)
 int launch_mx_qdq_bf16(const uint16_t *src, long long n, uint16_t *dst, cudaStream_t st);

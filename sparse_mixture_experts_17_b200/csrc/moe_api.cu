@@ -8,6 +8,7 @@
 #include <vector>
 
 #include "internal.h"
+#include "mxfp8.cuh"
 
 namespace moe {
 
@@ -134,14 +135,18 @@ WsLayout ws_layout(const moe_shape_t &s)
     L.dec_H = take((Td * k * s.d_ff + Td * dfs) * 2);
     L.dec_xdq = take(mx ? Td * s.d * 2 : 0);
     L.dec_H32 = take(mx ? (Td * k * s.d_ff + Td * dfs) * 4 : 0);
+    // scales in the atom layout: routed operands keyed by m-tile (at most
+    // max_mt tiles of 128 rows), shared-expert operands by row / 128
+    const size_t mt_rows = (size_t)L.max_mt * 128;
     L.xq = take(mx ? N * s.d : 0);
-    L.xsf = take(mx ? N * s.d / 32 : 0);
+    L.xsf = take(mx ? (size_t)sf_atom_bytes(mt_rows, s.d) : 0);
     L.Hq = take(mx ? N * s.d_ff : 0);
-    L.Hsf = take(mx ? N * s.d_ff / 32 : 0);
+    L.Hsf = take(mx ? (size_t)sf_atom_bytes(mt_rows, s.d_ff) : 0);
     L.xq_s = take(mx && dfs ? T * s.d : 0);
-    L.xsf_s = take(mx && dfs ? T * s.d / 32 : 0);
+    L.xsf_s = take(mx && dfs ? (size_t)sf_atom_bytes(T, s.d) : 0);
     L.Hsq = take(mx && dfs ? T * dfs : 0);
-    L.Hssf = take(mx && dfs ? T * dfs / 32 : 0);
+    L.Hssf = take(mx && dfs ? (size_t)sf_atom_bytes(T, (int)dfs) : 0);
+    L.tile_start = take(mx ? E * 4 : 0);
     L.scores = take(ec ? T * E * 4 : 0);
     L.ec_w = take(ec ? N * 4 : 0);
     L.x_stage = take((s.flags & MOE_FLAG_HOST_IO) ? T * s.d * 2 : 0);
@@ -443,7 +448,6 @@ static int expert_ffn_mx(const moe_shape_t &s, const WsLayout &L, void *ws, cons
     g.out = at<uint8_t>(ws, L.Hq);
     g.ldo = s.d_ff;
     g.out_sf = at<uint8_t>(ws, L.Hsf);
-    g.ldo_sf = s.d_ff / 32;
     g.status = status;
     int rc;
     {
@@ -506,7 +510,6 @@ static int shared_expert_mx(const moe_shape_t &s, const WsLayout &L, void *ws, c
     g.out = at<uint8_t>(ws, L.Hsq);
     g.ldo = dfs;
     g.out_sf = at<uint8_t>(ws, L.Hssf);
-    g.ldo_sf = dfs / 32;
     g.status = status;
     if ((rc = launch_gemm_mx(g, st)))
         return rc;
@@ -589,7 +592,7 @@ static int forward_mx_impl(const moe_shape_t &s, const WsLayout &L, void *ws, co
         rc = launch_hist_scan(s, idx, chunk, rank, counter, at<int32_t>(ws, L.counts), offsets,
                               at<int32_t>(ws, L.n_kept), at<int32_t>(ws, L.mt_row0),
                               at<int32_t>(ws, L.mt_group), at<int32_t>(ws, L.num_mt), nullptr,
-                              nullptr, nullptr, status, st);
+                              nullptr, nullptr, status, st, at<int32_t>(ws, L.tile_start));
     }
     if (rc)
         return rc;
@@ -598,8 +601,8 @@ static int forward_mx_impl(const moe_shape_t &s, const WsLayout &L, void *ws, co
         rc = launch_permute(s, idx, chunk, rank, offsets, nullptr, slot_pos, perm_token, nullptr,
                             (!shared && !det) ? out : nullptr, st);
         if (!rc)
-            rc = launch_mx_gather(s, x, slot_pos, at<uint8_t>(ws, L.xq), at<uint8_t>(ws, L.xsf),
-                                  st);
+            rc = launch_mx_gather(s, x, idx, slot_pos, offsets, at<int32_t>(ws, L.tile_start),
+                                  at<uint8_t>(ws, L.xq), at<uint8_t>(ws, L.xsf), st);
     }
     if (rc)
         return rc;
@@ -1102,8 +1105,7 @@ int moe_quantize_experts_mxfp8(const moe_shape_t *shape, const moe_bf16_t *W1,
         return MOE_OK;
     const moe_shape_t &s = *shape;
     if (!W1 || !W3 || !W2 || !W13q || !W13sf || !W2q || !W2sf || !al16(W1) || !al16(W3) ||
-        !al16(W2) || !al16(W13q) || !al16(W2q) || (reinterpret_cast<uintptr_t>(W13sf) & 3u) ||
-        (reinterpret_cast<uintptr_t>(W2sf) & 3u))
+        !al16(W2) || !al16(W13q) || !al16(W2q) || !al16(W13sf) || !al16(W2sf))
         return MOE_ERR_INVALID_ARG;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if ((rc = launch_mx_pack_w13(s, W1, W3, W13q, W13sf, st)))
@@ -1126,12 +1128,11 @@ int moe_forward_mxfp8(const moe_shape_t *shape, const moe_bf16_t *x, const moe_b
     const moe_shape_t &s = *shape;
     if (!(s.flags & MOE_FLAG_MXFP8) || (s.flags & MOE_FLAG_HOST_IO))
         return MOE_ERR_INVALID_ARG;
-    auto al4 = [](const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; };
     if (!x || !Wg || !W13q || !W13sf || !W2q || !W2sf || !out || !al16(x) || !al16(Wg) ||
-        !al16(W13q) || !al16(W2q) || !al4(W13sf) || !al4(W2sf) || !al16(out))
+        !al16(W13q) || !al16(W2q) || !al16(W13sf) || !al16(W2sf) || !al16(out))
         return MOE_ERR_INVALID_ARG;
     if (s.d_ff_shared > 0 && (!W13s_q || !W13s_sf || !W2s_q || !W2s_sf || !al16(W13s_q) ||
-                              !al16(W2s_q) || !al4(W13s_sf) || !al4(W2s_sf)))
+                              !al16(W2s_q) || !al16(W13s_sf) || !al16(W2s_sf)))
         return MOE_ERR_INVALID_ARG;
     WsLayout L;
     if ((rc = check_ws(s, ws, ws_bytes, L)))

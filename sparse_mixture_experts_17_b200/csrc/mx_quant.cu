@@ -1,8 +1,9 @@
 // mx_quant.cu -- MXFP8 quantization of expert weights and activations (the
 // encoding is defined in mxfp8.cuh).
 //
-//   k_mx_quantize_rows  a bf16 matrix [rows, K] -> codes [rows, K] + scales
-//                       [rows, K/32]; one thread per 32-element block
+//   k_mx_quantize_rows  a bf16 matrix [rows, K] -> codes [rows, K] + scales in
+//                       the atom layout of mxfp8.cuh (tile = row / 128); one
+//                       thread per 32-element block
 //   k_mx_pack_w13       W1, W3 [E, d_ff, d] -> the packed gate/up operand of
 //                       the MXFP8 w1/w3 GEMM: for each block b of 64 h
 //                       columns, packed rows 128b..128b+63 are W1 rows
@@ -11,7 +12,8 @@
 //                       up columns); quantized along d
 //   k_mx_gather         x [T, d] -> every kept permuted row of token t:
 //                       each token is quantized once and its codes and scales
-//                       copied to the rows slot_pos[t, :] names
+//                       copied to the rows slot_pos[t, :] names (scales in the
+//                       atom layout keyed by the row's m-tile)
 #include <algorithm>
 #include <cstring>
 
@@ -44,17 +46,20 @@ __device__ __forceinline__ void store_codes32(uint8_t *dst, const uint32_t (&q)[
 }
 
 __global__ void __launch_bounds__(256) k_mx_quantize_rows(const uint16_t *__restrict__ src,
-                                                          long long nblocks,
+                                                          long long nblocks, int K,
                                                           uint8_t *__restrict__ codes,
                                                           uint8_t *__restrict__ scales)
 {
     const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= nblocks)
         return;
+    const int bpr = K / kMxBlock;
+    const long long row = i / bpr;
+    const int b = (int)(i - row * bpr);
     float v[32];
     load_bf16x32(src + i * kMxBlock, v);
     uint32_t q[8];
-    scales[i] = mx_quantize32(v, q);
+    scales[sf_atom_offset(row >> 7, (int)(row & 127), b, K)] = mx_quantize32(v, q);
     store_codes32(codes + i * kMxBlock, q);
 }
 
@@ -78,13 +83,18 @@ __global__ void __launch_bounds__(256) k_mx_pack_w13(const uint16_t *__restrict_
     float v[32];
     load_bf16x32(src + b * kMxBlock, v);
     uint32_t q[8];
-    scales[i] = mx_quantize32(v, q);
+    scales[sf_atom_offset(prow >> 7, (int)(prow & 127), b, d)] = mx_quantize32(v, q);
     store_codes32(codes + i * kMxBlock, q);
 }
 
-// One warp per token; lane j < k holds slot j's permuted row.
+// One warp per token; lane j < k holds slot j's permuted row, and the row's
+// m-tile (the expert's first tile + its position in the segment / 128) and
+// row within the tile, which place its scales in the atom layout.
 __global__ void __launch_bounds__(256) k_mx_gather(const uint16_t *__restrict__ x,
-                                                   const int32_t *__restrict__ slot_pos, int T,
+                                                   const int32_t *__restrict__ idx,
+                                                   const int32_t *__restrict__ slot_pos,
+                                                   const int32_t *__restrict__ offsets,
+                                                   const int32_t *__restrict__ tile_start, int T,
                                                    int k, int d, uint8_t *__restrict__ xq,
                                                    uint8_t *__restrict__ xsf)
 {
@@ -92,11 +102,23 @@ __global__ void __launch_bounds__(256) k_mx_gather(const uint16_t *__restrict__ 
     const int lane = threadIdx.x & 31;
     if (t >= T)
         return;
-    const int mine = (lane < k) ? slot_pos[(size_t)t * k + lane] : -1;
-    int pos[MOE_MAX_K];
+    int mine = -1, mtile = 0, mrow = 0;
+    if (lane < k) {
+        mine = slot_pos[(size_t)t * k + lane];
+        if (mine >= 0) {
+            const int e = idx[(size_t)t * k + lane];
+            const int p = mine - offsets[e];
+            mtile = tile_start[e] + (p >> 7);
+            mrow = p & 127;
+        }
+    }
+    int pos[MOE_MAX_K], tl[MOE_MAX_K], rw[MOE_MAX_K];
 #pragma unroll
-    for (int j = 0; j < MOE_MAX_K; ++j)
+    for (int j = 0; j < MOE_MAX_K; ++j) {
         pos[j] = __shfl_sync(kFullMask, mine, j);
+        tl[j] = __shfl_sync(kFullMask, mtile, j);
+        rw[j] = __shfl_sync(kFullMask, mrow, j);
+    }
     const int bpr = d / kMxBlock;
     for (int b = lane; b < bpr; b += 32) {
         float v[32];
@@ -107,7 +129,7 @@ __global__ void __launch_bounds__(256) k_mx_gather(const uint16_t *__restrict__ 
         for (int j = 0; j < MOE_MAX_K; ++j) {
             if (j < k && pos[j] >= 0) {
                 store_codes32(xq + (size_t)pos[j] * d + b * kMxBlock, q);
-                xsf[(size_t)pos[j] * bpr + b] = sc;
+                xsf[sf_atom_offset(tl[j], rw[j], b, d)] = sc;
             }
         }
     }
@@ -163,7 +185,7 @@ int launch_mx_quantize_rows(const uint16_t *src, long long rows, int K, uint8_t 
     const long long nblocks = rows * (K / kMxBlock);
     if (nblocks <= 0)
         return MOE_OK;
-    k_mx_quantize_rows<<<(unsigned)((nblocks + 255) / 256), 256, 0, st>>>(src, nblocks, codes,
+    k_mx_quantize_rows<<<(unsigned)((nblocks + 255) / 256), 256, 0, st>>>(src, nblocks, K, codes,
                                                                           scales);
     return launched();
 }
@@ -179,12 +201,14 @@ int launch_mx_pack_w13(const moe_shape_t &s, const uint16_t *W1, const uint16_t 
     return launched();
 }
 
-int launch_mx_gather(const moe_shape_t &s, const uint16_t *x, const int32_t *slot_pos,
+int launch_mx_gather(const moe_shape_t &s, const uint16_t *x, const int32_t *idx,
+                     const int32_t *slot_pos, const int32_t *offsets, const int32_t *tile_start,
                      uint8_t *xq, uint8_t *xsf, cudaStream_t st)
 {
     if (s.T == 0)
         return MOE_OK;
-    k_mx_gather<<<(s.T + 7) / 8, 256, 0, st>>>(x, slot_pos, s.T, s.k, s.d, xq, xsf);
+    k_mx_gather<<<(s.T + 7) / 8, 256, 0, st>>>(x, idx, slot_pos, offsets, tile_start, s.T, s.k,
+                                               s.d, xq, xsf);
     return launched();
 }
 

@@ -59,6 +59,27 @@ __device__ __forceinline__ uint8_t mx_quantize32(const float (&v)[32], uint32_t 
     return (uint8_t)(X + 127);
 }
 
+// Scale layout for the block-scaled MMA ("scale atoms"): the scales of a
+// 128-row x 128-element tile form one 512-byte atom in which the scale of
+// tile row m and 32-element block kb (0..3) sits at byte
+// (m % 32) * 16 + (m / 32) * 4 + kb, the order tcgen05.cp 32x128b.warpx4
+// expects. Atoms are stored tile by tile, K groups innermost: atom
+// (tile, g) at byte (tile * (K / 128) + g) * 512. For weights the tile is
+// row / 128; for routed activations it is the row's m-tile in the GEMM's tile
+// list, so expert segments need no padding.
+constexpr int kSfAtomBytes = 512;
+
+__host__ __device__ __forceinline__ long long sf_atom_offset(long long tile, int m, int b, int K)
+{
+    return (tile * (K / 128) + (b >> 2)) * kSfAtomBytes + (m & 31) * 16 + (m >> 5) * 4 + (b & 3);
+}
+
+// Scale bytes of a [rows, K] operand in the atom layout (rows padded to 128).
+__host__ __device__ __forceinline__ long long sf_atom_bytes(long long rows, int K)
+{
+    return (rows + 127) / 128 * (K / 128) * kSfAtomBytes;
+}
+
 // Two E4M3 codes (low byte first) -> two floats, exact.
 __device__ __forceinline__ float2 mx_decode2(uint16_t c2)
 {

@@ -228,13 +228,14 @@ def moe_forward_expert_choice(shape, x, Wg, bias, W13, W2, W13_shared, W2_shared
 
 
 def moe_quantize_experts_mxfp8(shape, W1, W3, W2, stream=None) -> dict:
-    """MXFP8 experts from bf16 ones: dict(W13q, W13sf, W2q, W2sf) (uint8 tensors)."""
+    """MXFP8 experts from bf16 ones: dict(W13q, W13sf, W2q, W2sf) (uint8 tensors; the
+    scale arrays are flat, in the scale-atom order moe.h describes)."""
     E, d_ff, d = shape.E, shape.d_ff, shape.d
     dev = W1.device
     q = dict(W13q=torch.empty(E, 2 * d_ff, d, dtype=U8, device=dev),
-             W13sf=torch.empty(E, 2 * d_ff, d // 32, dtype=U8, device=dev),
+             W13sf=torch.empty(E * 2 * d_ff * d // 32, dtype=U8, device=dev),
              W2q=torch.empty(E, d, d_ff, dtype=U8, device=dev),
-             W2sf=torch.empty(E, d, d_ff // 32, dtype=U8, device=dev))
+             W2sf=torch.empty(E * d * d_ff // 32, dtype=U8, device=dev))
     _check("moe_quantize_experts_mxfp8", lib().moe_quantize_experts_mxfp8(
         ctypes.byref(shape), _ptr(W1, BF16, "W1"), _ptr(W3, BF16, "W3"), _ptr(W2, BF16, "W2"),
         _ptr(q["W13q"], U8, "W13q"), _ptr(q["W13sf"], U8, "W13sf"), _ptr(q["W2q"], U8, "W2q"),
@@ -332,6 +333,13 @@ class MoeLayer:
         moe_forward(self.shape(T, flags), x, self.Wg, self.bias, self.W13, self.W2, self.W13s,
                     self.W2s, out, logits_out, topk_idx_out, self.status, self.ws, stream)
         return out
+
+
+def sf_atoms_to_rows(sf, rows: int, K: int):
+    """Scale bytes in the atom order -> [rows, K/32] row-major (numpy or torch)."""
+    a = sf.reshape(rows // 128, K // 128, 32, 4, 4)     # [tile, group, m%32, m/32, block]
+    a = a.permute(0, 3, 2, 1, 4) if isinstance(a, torch.Tensor) else a.transpose(0, 3, 2, 1, 4)
+    return a.reshape(rows, K // 32)
 
 
 class MoeLayerMx:

@@ -62,14 +62,15 @@ def test_quantize_experts_bitexact(E, d_ff, d, kind):
     q = M.moe_quantize_experts_mxfp8(s, W1, W3, W2)
     torch.cuda.synchronize()
     c1, c3 = _unpack_w13(q["W13q"].cpu().numpy(), d_ff)
-    s1, s3 = _unpack_w13(q["W13sf"].cpu().numpy(), d_ff)
+    sf13 = M.sf_atoms_to_rows(q["W13sf"].cpu().numpy(), E * 2 * d_ff, d).reshape(E, 2 * d_ff, -1)
+    s1, s3 = _unpack_w13(sf13, d_ff)
     for W, c, sc in ((W1, c1, s1), (W3, c3, s3)):
         oc, os_ = O.mx_quantize(_f64(W).reshape(-1, d))
         assert (c.reshape(-1, d) == oc).all()
         assert (sc.reshape(-1, d // 32) == os_).all()
     oc, os_ = O.mx_quantize(_f64(W2).reshape(-1, d_ff))
     assert (q["W2q"].cpu().numpy().reshape(-1, d_ff) == oc).all()
-    assert (q["W2sf"].cpu().numpy().reshape(-1, d_ff // 32) == os_).all()
+    assert (M.sf_atoms_to_rows(q["W2sf"].cpu().numpy(), E * d, d_ff) == os_).all()
 
 
 MX_CASES = [
