@@ -60,9 +60,11 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
     return *reinterpret_cast<uint32_t *>(&h);
 }
 
+// silu(g) * u = g / (1 + e^-g) * u. The fast division returns 0 once the
+// denominator passes 2^126 (g < -87), where silu(g) is below 2^-120 anyway.
 __device__ __forceinline__ float silu_mul(float g, float u)
 {
-    return g / (1.0f + __expf(-g)) * u;
+    return __fdividef(g, 1.0f + __expf(-g)) * u;
 }
 
 // ------------------------------------------------------------------ mbarrier
