@@ -228,7 +228,15 @@ def run_ours(a, world, rank, local):
         w = replace(w, E=a.experts, name=f"{w.name}@E{a.experts}",
                     capacity=I.capacity_for(w.T, w.k, a.experts) if w.capacity else 0)
     inp = I.make_inputs(w, dev, seed=0)
-    layer = M.MoeLayer(inp)
+    if a.mxfp8:
+        # quantize once, then free the bf16 experts: only the MXFP8 ones stay resident
+        layer = M.MoeLayerMx(inp)
+        for key in ("W1", "W3", "W2", "W1s", "W3s", "W2s"):
+            inp.pop(key, None)
+        torch.cuda.empty_cache()
+        a.no_extra = a.no_e2e = True
+    else:
+        layer = M.MoeLayer(inp)
     x = inp["x"]
     out = torch.empty(w.T, w.d, dtype=torch.float32, device=dev)
     idx = torch.empty(w.T, w.k, dtype=torch.int32, device=dev)
@@ -259,7 +267,9 @@ def run_ours(a, world, rank, local):
     value = tokens_all / (step_ms_max / 1e3)
 
     flops, w13_flops, w2_flops = prefill_flops(w, n_kept)
-    peak_t = peaks["bf16_tflops_sustained"]
+    # MXFP8: the fp8 dense peak, twice the measured sustained bf16 figure (the
+    # nominal fp8:bf16 ratio; no fp8 peak is measured on this machine)
+    peak_t = peaks["bf16_tflops_sustained"] * (2.0 if a.mxfp8 else 1.0)
     stage_ms = {k: round(v[0] / v[1], 4) for k, v in stages.items()}
     decode_path = "dec_w13" in stages
     extra = {}
@@ -267,13 +277,23 @@ def run_ours(a, world, rank, local):
         w13_ms = stages["w13"][0] / stages["w13"][1]
         w2_ms = stages["w2"][0] / stages["w2"][1]
         ach = w13_flops / (w13_ms / 1e3) / 1e12
-        roofline = {"bound": "tensor", "kernel": "k_gemm_tc<256,EPI_SWIGLU> (grouped w1/w3 GEMM + SwiGLU)",
-                    "achieved": round(ach, 1), "peak": peak_t, "unit": "TFLOP/s",
-                    "frac": round(ach / peak_t, 4), "traffic": None,
-                    "peak_source": f"{peak_src} bf16_tflops_sustained",
-                    "frac_of_burst_peak": round(ach / peaks["bf16_tflops"], 4),
-                    "frac_of_nominal_2250": round(ach / 2250.0, 4),
-                    "algorithmic_flops_per_launch": w13_flops, "avg_launch_ms": round(w13_ms, 4)}
+        if a.mxfp8:
+            roofline = {"bound": "tensor",
+                        "kernel": "k_gemm_mx<EPI_SWIGLU_MX> (block-scaled MXFP8 w1/w3 GEMM + SwiGLU)",
+                        "achieved": round(ach, 1), "peak": peak_t, "unit": "TFLOP/s",
+                        "frac": round(ach / peak_t, 4), "traffic": None,
+                        "peak_source": f"2 x {peak_src} bf16_tflops_sustained (nominal fp8:bf16)",
+                        "frac_of_nominal_4500": round(ach / 4500.0, 4),
+                        "algorithmic_flops_per_launch": w13_flops, "avg_launch_ms": round(w13_ms, 4)}
+        else:
+            roofline = {"bound": "tensor",
+                        "kernel": "k_gemm_tc<256,EPI_SWIGLU> (grouped w1/w3 GEMM + SwiGLU)",
+                        "achieved": round(ach, 1), "peak": peak_t, "unit": "TFLOP/s",
+                        "frac": round(ach / peak_t, 4), "traffic": None,
+                        "peak_source": f"{peak_src} bf16_tflops_sustained",
+                        "frac_of_burst_peak": round(ach / peaks["bf16_tflops"], 4),
+                        "frac_of_nominal_2250": round(ach / 2250.0, 4),
+                        "algorithmic_flops_per_launch": w13_flops, "avg_launch_ms": round(w13_ms, 4)}
         extra["w2_tflops"] = round(w2_flops / (w2_ms / 1e3) / 1e12, 1)
         extra["active_tflops"] = round(flops / (step_ms_max / 1e3) / 1e12, 1)
         extra["active_tflops_frac_measured_sustained"] = round(
@@ -283,6 +303,10 @@ def run_ours(a, world, rank, local):
         idx_now = torch.empty(w.T, w.k, dtype=torch.int32, device=dev)
         layer.forward(x, out=out, topk_idx_out=idx_now)
         U, nbytes, w13_bytes, expert_bytes = decode_bytes(w, w.T, idx_now)
+        if a.mxfp8:   # a code byte and 1/32 of a scale byte per weight instead of 2 bytes
+            mx = (1.0 + 1.0 / 32.0) / 2.0
+            nbytes = int(nbytes - expert_bytes * (1.0 - mx))
+            w13_bytes, expert_bytes = int(w13_bytes * mx), int(expert_bytes * mx)
         k13 = stages["dec_w13"][0] / stages["dec_w13"][1]
         ach = w13_bytes / (k13 / 1e3) / 1e9
         roofline = {"bound": "hbm", "kernel": "k_dec_w13 (chosen experts' w1/w3 rows + SwiGLU)",
@@ -322,13 +346,15 @@ def run_ours(a, world, rank, local):
     res = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
         "steps": a.steps, "warmup": a.warmup, "ms_per_step": round(step_ms_max, 4),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "mxfp8 (e4m3 + e8m0/32)" if a.mxfp8 else "bf16",
         "data": "synthetic (seeded, N(0,1) x, N(0,0.02) bf16 weights)",
         "config": {"workload": w.name, "T": w.T, "d_model": w.d, "d_ff": w.d_ff, "E": w.E,
                    "k": w.k, "capacity": w.capacity, "d_ff_shared": w.d_ff_shared,
                    "zipf_s": w.zipf_s, "seed": 0, "parallelism": f"replicas x{world}",
                    "l2": "inputs larger than L2 (expert weights and activations exceed 126 MB)",
-                   "output": "fp32 [T, d]"},
+                   "output": "fp32 [T, d]",
+                   "experts": "mxfp8 (moe_forward_mxfp8)" if a.mxfp8 else "bf16"},
         **extra,
         "stages_ms": stage_ms,
         "profiled_ms_per_step": round(prof_ms, 4),
@@ -558,6 +584,9 @@ def main(argv=None):
     ap.add_argument("--tokens", type=int, default=0, help="override T (profiling runs)")
     ap.add_argument("--experts", type=int, default=0, help="override E (profiling runs)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end run")
+    ap.add_argument("--mxfp8", action="store_true",
+                    help="time the layer on MXFP8 experts (moe_forward_mxfp8) instead of bf16; "
+                         "no extras, no end-to-end run")
     a = ap.parse_args(argv)
     if a.warmup < 3 and a.impl == "ours":
         a.warmup = 3
