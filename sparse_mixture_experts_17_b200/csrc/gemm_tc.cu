@@ -68,6 +68,9 @@ struct TcArgs {
     const float *bias;
     int n_valid;
     uint32_t *status;
+    int32_t *route_idx;
+    float *route_w;
+    int32_t *counter_zero;
 };
 
 template <int BN>
@@ -163,6 +166,54 @@ __device__ __forceinline__ void epilogue_tile(const TcArgs &p, uint32_t tb, long
                     dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
             }
         }
+    } else if (MODE == EPI_ROUTER_TOPK) {
+        // the whole row (E <= 64 logits) is this thread's: logits + bias, then
+        // "Sparse MoE Block" routing in registers: k rounds of arg-max (larger
+        // logit, then lower index; -0.0 == +0.0) and the weights
+        // exp(l_j - l_max) / sum over the chosen k
+        float v[64];
+        tmem_ld32(tb, *reinterpret_cast<float(*)[32]>(&v[0]));
+        tmem_ld32(tb + 32, *reinterpret_cast<float(*)[32]>(&v[32]));
+        tmem_ld_wait();
+        if (valid) {
+            const int E = p.n_valid;
+            float *o = static_cast<float *>(p.out) + row * p.ldo;
+            bool bad = false;
+#pragma unroll
+            for (int n = 0; n < 64; ++n) {
+                if (n < E) {
+                    v[n] += p.bias ? p.bias[n] : 0.f;
+                    o[n] = v[n];
+                    bad |= isnan(v[n]);
+                }
+            }
+            uint64_t taken = 0;
+            int sel[MOE_MAX_K];
+            float ex[MOE_MAX_K];
+            float M = 0.f, sum = 0.f;
+            for (int j = 0; j < p.k; ++j) {
+                float bv = -INFINITY;
+                int bi = -1;
+#pragma unroll
+                for (int n = 0; n < 64; ++n)
+                    if (n < E && !((taken >> n) & 1ull) && (bi < 0 || v[n] > bv)) {
+                        bv = v[n];
+                        bi = n;
+                    }
+                taken |= 1ull << bi;
+                if (j == 0)
+                    M = bv;
+                sel[j] = bi;
+                ex[j] = expf(bv - M);
+                sum += ex[j];
+            }
+            if (bad || !isfinite(M))
+                flag_status(p.status, MOE_ERR_NONFINITE);
+            for (int j = 0; j < p.k; ++j) {
+                p.route_idx[row * p.k + j] = sel[j];
+                p.route_w[row * p.k + j] = ex[j] / sum;
+            }
+        }
     } else {   // EPI_ROUTER
         float *o = static_cast<float *>(p.out) + row * p.ldo;
 #pragma unroll 1
@@ -216,6 +267,10 @@ __global__ void __launch_bounds__(192, 1)
     if (warp == 0 && lane == 0) {
         tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmB);
+        // the fused router also re-arms the histogram kernel's ticket (which
+        // runs after this kernel in stream order)
+        if (MODE == EPI_ROUTER_TOPK && blockIdx.x == 0 && p.counter_zero)
+            *p.counter_zero = 0;
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, C::TMEM_COLS);
@@ -571,6 +626,9 @@ static int launch_tc_impl(const GemmArgs &g, cudaStream_t st)
     p.bias = g.bias;
     p.n_valid = g.n_valid;
     p.status = g.status;
+    p.route_idx = g.route_idx;
+    p.route_w = g.route_w;
+    p.counter_zero = g.counter_zero;
 
     static int attr_done[64] = {0};
     int dev = 0;
@@ -663,6 +721,10 @@ int launch_gemm_tc(const GemmArgs &g, cudaStream_t st)
     case EPI_ROUTER:
         // 64-column tiles: more CTAs for few 128-token tiles; x re-reads hit L2
         return launch_tc_impl<64, EPI_ROUTER>(g, st);
+    case EPI_ROUTER_TOPK:
+        if (g.N > 64 || g.k < 1 || g.k > MOE_MAX_K)
+            return MOE_ERR_INVALID_ARG;
+        return launch_tc_impl<64, EPI_ROUTER_TOPK>(g, st);
     default:
         return MOE_ERR_INVALID_ARG;
     }

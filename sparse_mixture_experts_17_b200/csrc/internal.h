@@ -86,8 +86,10 @@ enum EpiMode {
     EPI_COMBINE = 1,    // out[perm_token[row], :] += w(row) * acc  (fp32 atomics)
     EPI_STORE_F32 = 2,  // out[row, :] = acc  (fp32)
     EPI_ROUTER = 3,     // out[row, n] = acc[n] + bias[n] for n < n_valid
-    EPI_SWIGLU_MX = 4   // MXFP8 GEMM: h = silu(gate) * up, quantized to MXFP8 codes (out)
+    EPI_SWIGLU_MX = 4,  // MXFP8 GEMM: h = silu(gate) * up, quantized to MXFP8 codes (out)
                         // and block scales (out_sf)
+    EPI_ROUTER_TOPK = 5 // EPI_ROUTER, then (E <= 64, one 64-column tile) the top-k of each
+                        // row and its renormalised weights into route_idx / route_w
 };
 
 struct GemmArgs {
@@ -125,6 +127,10 @@ struct GemmArgs {
     // in the atom layout (mxfp8.cuh): A's keyed by m-tile index, B's by row/128
     const uint8_t *Aq, *A_sf, *Bq, *B_sf;
     uint8_t *out_sf;          // EPI_SWIGLU_MX: scales of h, atom layout keyed by m-tile
+    // EPI_ROUTER_TOPK: top-k outputs [rows, k]; counter_zero (one word) is zeroed
+    int32_t *route_idx;
+    float *route_w;
+    int32_t *counter_zero;
 };
 
 int launch_gemm_tc(const GemmArgs &g, cudaStream_t st);

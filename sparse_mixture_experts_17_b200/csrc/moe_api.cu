@@ -335,6 +335,65 @@ static int router(const moe_shape_t &s, const uint16_t *x, const uint16_t *Wg, c
     return launch_gemm_tc(g, st);
 }
 
+// Router GEMM with the top-k in its epilogue (one launch): the tensor-core
+// router with all E <= 64 logits of a token in one 64-column tile.
+static bool router_topk_fusable(const moe_shape_t &s)
+{
+    return s.T > MOE_DECODE_MAX_T && s.E <= 64 && !(s.flags & MOE_FLAG_SIMT_FFN);
+}
+
+static int router_topk(const moe_shape_t &s, const uint16_t *x, const uint16_t *Wg,
+                       const float *bias, float *logits, int32_t *idx, float *w,
+                       int32_t *counter, uint32_t *status, cudaStream_t st)
+{
+    GemmArgs g = gemm_base();
+    g.mode = EPI_ROUTER_TOPK;
+    g.A = x;
+    g.a_rows = s.T;
+    g.B = Wg;
+    g.b_rows_total = s.E;
+    g.K = s.d;
+    g.N = s.E;
+    g.num_mt_host = (s.T + kBlockM - 1) / kBlockM;
+    g.max_mt = g.num_mt_host;
+    g.rows_valid = s.T;
+    g.out = logits;
+    g.ldo = s.E;
+    g.bias = bias;
+    g.n_valid = s.E;
+    g.k = s.k;
+    g.route_idx = idx;
+    g.route_w = w;
+    g.counter_zero = counter;
+    g.status = status;
+    return launch_gemm_tc(g, st);
+}
+
+// Router, softmax / top-k / renormalisation: one launch when a fused form
+// applies (single-CTA for small T and W_g; the GEMM epilogue for E <= 64).
+static int route_tokens(const moe_shape_t &s, const uint16_t *x, const uint16_t *Wg,
+                        const float *bias, float *logits, int32_t *idx, float *w,
+                        int32_t *counter, uint32_t *status, cudaStream_t st)
+{
+    if (dec_route_fusable(s)) {
+        StageMark m(MOE_STAGE_ROUTER, st);
+        return launch_dec_route(s, x, Wg, bias, logits, idx, w, counter, status, st);
+    }
+    if (router_topk_fusable(s)) {
+        StageMark m(MOE_STAGE_ROUTER, st);
+        return router_topk(s, x, Wg, bias, logits, idx, w, counter, status, st);
+    }
+    int rc;
+    {
+        StageMark m(MOE_STAGE_ROUTER, st);
+        rc = router(s, x, Wg, bias, logits, status, st);
+    }
+    if (rc)
+        return rc;
+    StageMark m(MOE_STAGE_TOPK, st);
+    return launch_topk(s, logits, idx, w, counter, status, st);
+}
+
 static int forward_impl(const moe_shape_t &s, const WsLayout &L, void *ws, const uint16_t *x,
                         const uint16_t *Wg, const float *bias, const uint16_t *W13,
                         const uint16_t *W2, const uint16_t *W13s, const uint16_t *W2s,
@@ -349,21 +408,8 @@ static int forward_impl(const moe_shape_t &s, const WsLayout &L, void *ws, const
     if (force_dec && s.T > MOE_DECODE_MAX_T)
         return MOE_ERR_UNSUPPORTED;
     const bool decode = force_dec || (!force_pre && s.T <= MOE_DECODE_DEFAULT_T);
-    int rc;
     int32_t *counter = at<int32_t>(ws, L.counter);
-    if (dec_route_fusable(s)) {
-        StageMark m(MOE_STAGE_ROUTER, st);   // router and top-k in one launch
-        rc = launch_dec_route(s, x, Wg, bias, logits, idx, w, counter, status, st);
-    } else {
-        {
-            StageMark m(MOE_STAGE_ROUTER, st);
-            rc = router(s, x, Wg, bias, logits, status, st);
-        }
-        if (rc)
-            return rc;
-        StageMark m(MOE_STAGE_TOPK, st);
-        rc = launch_topk(s, logits, idx, w, counter, status, st);
-    }
+    int rc = route_tokens(s, x, Wg, bias, logits, idx, w, counter, status, st);
     if (rc)
         return rc;
     if (decode) {
@@ -544,20 +590,7 @@ static int forward_mx_impl(const moe_shape_t &s, const WsLayout &L, void *ws, co
     if (force_dec && s.T > MOE_DECODE_MAX_T)
         return MOE_ERR_UNSUPPORTED;
     const bool decode = force_dec || (!force_pre && s.T <= MOE_DECODE_DEFAULT_T);
-    int rc;
-    if (dec_route_fusable(s)) {
-        StageMark m(MOE_STAGE_ROUTER, st);
-        rc = launch_dec_route(s, x, Wg, bias, logits, idx, w, counter, status, st);
-    } else {
-        {
-            StageMark m(MOE_STAGE_ROUTER, st);
-            rc = router(s, x, Wg, bias, logits, status, st);
-        }
-        if (rc)
-            return rc;
-        StageMark m(MOE_STAGE_TOPK, st);
-        rc = launch_topk(s, logits, idx, w, counter, status, st);
-    }
+    int rc = route_tokens(s, x, Wg, bias, logits, idx, w, counter, status, st);
     if (rc)
         return rc;
     if (decode) {
@@ -855,6 +888,8 @@ int moe_route(const moe_shape_t *shape, const moe_bf16_t *x, const moe_bf16_t *W
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (x && dec_route_fusable(s))
         return launch_dec_route(s, x, Wg, bias, logits, topk_idx, topk_w, nullptr, status, st);
+    if (x && router_topk_fusable(s))
+        return router_topk(s, x, Wg, bias, logits, topk_idx, topk_w, nullptr, status, st);
     if (x && (rc = router(s, x, Wg, bias, logits, status, st)))
         return rc;
     return launch_topk(s, logits, topk_idx, topk_w, nullptr, status, st);

@@ -82,6 +82,37 @@ def test_router_logits(T, d, E, zipf, flags):
     assert err <= LOGIT_ABS, err
 
 
+# ---------------------------------------------------------------- S1+S2 fused (router GEMM epilogue)
+
+@pytest.mark.parametrize("T,E,k,ties", [(300, 8, 2, False), (1000, 64, 8, False), (257, 40, 3, False),
+                                        (500, 16, 1, False), (300, 8, 2, True), (200, 64, 6, True)])
+def test_router_topk_fused_matches_separate(T, E, k, ties):
+    """moe_route on x (E <= 64: top-k in the router GEMM's epilogue) against the
+    separate top-k kernel on the very logits it produced: indices bit for bit,
+    weights within W_ABS, and the logits against the fp64 oracle."""
+    w = small_workload("rtk", T, 512, 128, E, k)
+    inp = I.make_inputs(w, "cuda", seed=T + E + k)
+    wg, bias = inp["wg"], inp["bias"]
+    if ties:   # logits = bias only, with repeated values: ties decided by expert index
+        wg = torch.zeros_like(wg)
+        bias = torch.tensor([0.5, -1.0, 0.5, 2.0, 2.0, 0.0, -0.0, 0.5] * (E // 8),
+                            dtype=torch.float32, device="cuda")
+    b1 = Buffers(w)
+    M.moe_route(b1.shape, inp["x"], wg, bias, b1.logits, b1.idx, b1.w, b1.status, b1.ws)
+    b2 = Buffers(w)
+    b2.logits.copy_(b1.logits)
+    M.moe_route(b2.shape, None, None, None, b2.logits, b2.idx, b2.w, b2.status, b2.ws)
+    torch.cuda.synchronize()
+    assert int(b1.status.item()) == 0 and int(b2.status.item()) == 0
+    assert torch.equal(b1.idx, b2.idx)
+    assert (b1.w - b2.w).abs().max().item() <= W_ABS
+    idx_o, w_o = O.route(b1.logits.cpu().numpy(), k)
+    assert (b1.idx.cpu().numpy() == idx_o).all()
+    assert np.abs(b1.w.double().cpu().numpy() - w_o).max() <= W_ABS
+    L64, _ = O.router_logits(u16(inp["x"]), u16(wg), None if bias is None else bias.cpu().numpy())
+    assert np.abs(b1.logits.double().cpu().numpy() - L64).max() <= LOGIT_ABS
+
+
 # ---------------------------------------------------------------- S3/S4: histogram, offsets, permutation
 
 def _random_idx(rng, T, E, k, skew):
