@@ -54,6 +54,9 @@
  *  R7  block-scaled 8-bit experts (precision mode 2): MXFP8 as defined at
  *      oracle_e4m3_decode, applied to x, to every expert weight row and to h
  *      along the contraction dimension; the router stays on bf16 weights.
+ *  R8  the backward pass differentiates the fp64 layer with the routing
+ *      decisions (top-k set, drops, slots) held fixed; see
+ *      oracle_moe_backward.
  *
  * Inputs are bf16 bit patterns (uint16) and are widened exactly to double.
  * Error codes: 0 ok, 1 invalid argument, 5 non-finite logit, 6 bad expert id.
@@ -618,6 +621,151 @@ int oracle_expert_choice(int T, int E, int C, const float *S, int32_t *tokens, d
             }
     }
     free(taken);
+    return ORC_OK;
+}
+
+/* ---- Backward pass (reading R8): gradients of the fp64 layer (precision
+ * mode 0) with the top-k selection, the capacity drops and the slot
+ * positions held fixed (they are piecewise constant in the inputs). For a kept
+ * assignment (t, j) to expert e with weight w = w[t, j] ([MIX]: softmax over
+ * all E renormalised over the top-k) and dout row delta:
+ *   g = W1_e x, u = W3_e x, s = silu(g), h = s * u, y = W2_e h
+ *   dW2_e += w delta h^T;   dh = w W2_e^T delta
+ *   du = dh * s;            dg = dh * u * silu'(g),
+ *                           silu'(g) = sig(g) (1 + g (1 - sig(g)))
+ *   dW1_e += dg x^T;  dW3_e += du x^T;  dx += W1_e^T dg + W3_e^T du
+ *   G[t, j] = <delta, y>    (the gradient of the loss w.r.t. w[t, j])
+ * A dropped assignment has G = 0. The shared expert ([DSK]) is the same with
+ * weight 1 and no G. Router: w_j = exp(l_j) / sum_{i in top-k} exp(l_i), so
+ *   dl[t, e_j] = w_j (G_j - sum_i w_i G_i) for the k chosen experts, 0 else;
+ *   dWg += dl^T x;  dbias += sum_t dl;  dx += dl Wg.
+ * Inputs as oracle_moe_tokens (bf16 patterns; wg [E, d]); dout [T, d] fp32.
+ * Outputs (fp64, fully written): dx [T, d], dW1 / dW3 [E, d_ff, d],
+ * dW2 [E, d, d_ff], dW1s / dW3s [d_ff_s, d], dW2s [d, d_ff_s] (when
+ * d_ff_s > 0), dlogits [T, E], dWg [E, d], dbias [E], G [T, k].
+ * Plain serial loops: meant for small shapes. */
+int oracle_moe_backward(int T, int d, int d_ff, int E, int k, int d_ff_s,
+                        const uint16_t *x, const uint16_t *W1, const uint16_t *W3,
+                        const uint16_t *W2, const uint16_t *W1s, const uint16_t *W3s,
+                        const uint16_t *W2s, const uint16_t *wg, const int32_t *idx,
+                        const double *w, const int32_t *slot_pos, const float *dout,
+                        double *dx, double *dW1, double *dW3, double *dW2, double *dW1s,
+                        double *dW3s, double *dW2s, double *dlogits, double *dWg,
+                        double *dbias, double *G)
+{
+    if (T < 0 || d < 1 || d_ff < 1 || E < 1 || k < 1 || k > E || d_ff_s < 0 || !x || !W1 ||
+        !W3 || !W2 || !wg || !idx || !w || !slot_pos || !dout || !dx || !dW1 || !dW3 ||
+        !dW2 || !dlogits || !dWg || !dbias || !G)
+        return ORC_EINVAL;
+    if (d_ff_s > 0 && (!W1s || !W3s || !W2s || !dW1s || !dW3s || !dW2s))
+        return ORC_EINVAL;
+    for (int64_t i = 0; i < (int64_t)T * d; ++i)
+        dx[i] = 0.0;
+    for (int64_t i = 0; i < (int64_t)E * d_ff * d; ++i)
+        dW1[i] = dW3[i] = dW2[i] = 0.0;
+    if (d_ff_s > 0)
+        for (int64_t i = 0; i < (int64_t)d_ff_s * d; ++i)
+            dW1s[i] = dW3s[i] = dW2s[i] = 0.0;
+    for (int64_t i = 0; i < (int64_t)T * E; ++i)
+        dlogits[i] = 0.0;
+    for (int64_t i = 0; i < (int64_t)E * d; ++i)
+        dWg[i] = 0.0;
+    for (int e = 0; e < E; ++e)
+        dbias[e] = 0.0;
+    const int hmax = d_ff > d_ff_s ? d_ff : d_ff_s;
+    double *xv = (double *)malloc(sizeof(double) * (size_t)d);
+    double *dl = (double *)malloc(sizeof(double) * (size_t)d);
+    double *gv = (double *)malloc(sizeof(double) * (size_t)hmax);
+    double *uv = (double *)malloc(sizeof(double) * (size_t)hmax);
+    double *hv = (double *)malloc(sizeof(double) * (size_t)hmax);
+    double *dh = (double *)malloc(sizeof(double) * (size_t)hmax);
+    if (!xv || !dl || !gv || !uv || !hv || !dh) {
+        free(xv); free(dl); free(gv); free(uv); free(hv); free(dh);
+        return ORC_EINVAL;
+    }
+    for (int t = 0; t < T; ++t) {
+        for (int i = 0; i < d; ++i) {
+            xv[i] = bf16_to_double(x[(int64_t)t * d + i]);
+            dl[i] = (double)dout[(int64_t)t * d + i];
+        }
+        /* each kept slot, then the shared expert (src = k) */
+        for (int j = 0; j <= k; ++j) {
+            const int shared = (j == k);
+            if (shared && d_ff_s == 0)
+                break;
+            int64_t a = (int64_t)t * k + j;
+            if (!shared) {
+                G[a] = 0.0;
+                if (slot_pos[a] < 0)
+                    continue;
+            }
+            const int e = shared ? 0 : idx[a];
+            const int ff = shared ? d_ff_s : d_ff;
+            const double wt = shared ? 1.0 : w[a];
+            const uint16_t *w1 = shared ? W1s : W1 + (int64_t)e * d_ff * d;
+            const uint16_t *w3 = shared ? W3s : W3 + (int64_t)e * d_ff * d;
+            const uint16_t *w2 = shared ? W2s : W2 + (int64_t)e * d * d_ff;
+            double *g1 = shared ? dW1s : dW1 + (int64_t)e * d_ff * d;
+            double *g3 = shared ? dW3s : dW3 + (int64_t)e * d_ff * d;
+            double *g2 = shared ? dW2s : dW2 + (int64_t)e * d * d_ff;
+            for (int c = 0; c < ff; ++c) {
+                double g = 0.0, u = 0.0;
+                for (int i = 0; i < d; ++i) {
+                    g += bf16_to_double(w1[(int64_t)c * d + i]) * xv[i];
+                    u += bf16_to_double(w3[(int64_t)c * d + i]) * xv[i];
+                }
+                gv[c] = g;
+                uv[c] = u;
+                hv[c] = g / (1.0 + exp(-g)) * u;
+            }
+            /* y, G, dW2, dh */
+            double Gtj = 0.0;
+            for (int c = 0; c < ff; ++c)
+                dh[c] = 0.0;
+            for (int r = 0; r < d; ++r) {
+                double y = 0.0;
+                for (int c = 0; c < ff; ++c) {
+                    const double w2rc = bf16_to_double(w2[(int64_t)r * ff + c]);
+                    y += w2rc * hv[c];
+                    g2[(int64_t)r * ff + c] += wt * dl[r] * hv[c];
+                    dh[c] += wt * w2rc * dl[r];
+                }
+                Gtj += dl[r] * y;
+            }
+            if (!shared)
+                G[a] = Gtj;
+            /* SwiGLU backward, dW1, dW3, dx */
+            for (int c = 0; c < ff; ++c) {
+                const double sg = 1.0 / (1.0 + exp(-gv[c]));
+                const double silu = gv[c] * sg;
+                const double du = dh[c] * silu;
+                const double dg = dh[c] * uv[c] * sg * (1.0 + gv[c] * (1.0 - sg));
+                for (int i = 0; i < d; ++i) {
+                    g1[(int64_t)c * d + i] += dg * xv[i];
+                    g3[(int64_t)c * d + i] += du * xv[i];
+                    dx[(int64_t)t * d + i] += bf16_to_double(w1[(int64_t)c * d + i]) * dg +
+                                              bf16_to_double(w3[(int64_t)c * d + i]) * du;
+                }
+            }
+        }
+        /* router: renormalised softmax over the k chosen experts */
+        double wG = 0.0;
+        for (int j = 0; j < k; ++j)
+            wG += w[(int64_t)t * k + j] * G[(int64_t)t * k + j];
+        for (int j = 0; j < k; ++j) {
+            const int64_t a = (int64_t)t * k + j;
+            const int e = idx[a];
+            const double g = w[a] * (G[a] - wG);
+            dlogits[(int64_t)t * E + e] = g;
+            dbias[e] += g;
+            for (int i = 0; i < d; ++i) {
+                const double wgi = bf16_to_double(wg[(int64_t)e * d + i]);
+                dWg[(int64_t)e * d + i] += g * xv[i];
+                dx[(int64_t)t * d + i] += g * wgi;
+            }
+        }
+    }
+    free(xv); free(dl); free(gv); free(uv); free(hv); free(dh);
     return ORC_OK;
 }
 

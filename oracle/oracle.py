@@ -66,6 +66,8 @@ def lib():
         L.oracle_mx_scale_exp.restype = ctypes.c_int
         L.oracle_mx_quantize.argtypes = [ctypes.c_int64, i, P, P, P]
         L.oracle_mx_quantize.restype = ctypes.c_int
+        L.oracle_moe_backward.argtypes = [i] * 6 + [P] * 23
+        L.oracle_moe_backward.restype = ctypes.c_int
         L.oracle_softmax_rows.restype = ctypes.c_int
         L.oracle_expert_choice.restype = ctypes.c_int
         for f in (L.oracle_router_logits, L.oracle_route, L.oracle_dispatch,
@@ -276,3 +278,35 @@ def mx_dequantize(codes, scales):
     v = e4m3_decode(codes)
     X = scales.astype(np.int64) - 127
     return v * np.repeat(np.exp2(X.astype(np.float64)), 32, axis=1)
+
+
+# ---------------------------------------------------------------- backward
+
+def moe_backward(inp, idx, w, slot_pos, dout):
+    """Gradients of the fp64 layer with the routing held fixed (see
+    oracle_moe_backward). inp: x, wg, W1, W3, W2 (+ W1s, W3s, W2s) as uint16;
+    idx/w/slot_pos from route/dispatch; dout [T, d] float32. Returns a dict of
+    float64 arrays: dx, dW1, dW3, dW2, (dW1s, dW3s, dW2s), dlogits, dWg, dbias, G."""
+    x, W1, W3, W2, wg = (_u16(inp[kk]) for kk in ("x", "W1", "W3", "W2", "wg"))
+    T, d = x.shape
+    E, d_ff, _ = W1.shape
+    k = idx.shape[1]
+    has_s = inp.get("W1s") is not None
+    W1s = W3s = W2s = None
+    d_ff_s = 0
+    if has_s:
+        W1s, W3s, W2s = _u16(inp["W1s"]), _u16(inp["W3s"]), _u16(inp["W2s"])
+        d_ff_s = W1s.shape[0]
+    out = dict(dx=np.empty((T, d)), dW1=np.empty((E, d_ff, d)), dW3=np.empty((E, d_ff, d)),
+               dW2=np.empty((E, d, d_ff)), dlogits=np.empty((T, E)), dWg=np.empty((E, d)),
+               dbias=np.empty(E), G=np.empty((T, k)))
+    if has_s:
+        out.update(dW1s=np.empty((d_ff_s, d)), dW3s=np.empty((d_ff_s, d)), dW2s=np.empty((d, d_ff_s)))
+    dout = np.ascontiguousarray(dout, np.float32)
+    _check("moe_backward", lib().oracle_moe_backward(
+        T, d, d_ff, E, k, d_ff_s, _p(x), _p(W1), _p(W3), _p(W2), _p(W1s), _p(W3s), _p(W2s),
+        _p(wg), _p(np.ascontiguousarray(idx, np.int32)), _p(np.ascontiguousarray(w, np.float64)),
+        _p(np.ascontiguousarray(slot_pos, np.int32)), _p(dout), _p(out["dx"]), _p(out["dW1"]),
+        _p(out["dW3"]), _p(out["dW2"]), _p(out.get("dW1s")), _p(out.get("dW3s")),
+        _p(out.get("dW2s")), _p(out["dlogits"]), _p(out["dWg"]), _p(out["dbias"]), _p(out["G"])))
+    return out
