@@ -84,8 +84,9 @@ enum {
     MOE_FLAG_EXPERT_CHOICE = 1 << 7, /* workspace sized for the expert-choice calls
                                         (moe_route_expert_choice, moe_forward_expert_choice) */
     MOE_FLAG_SLOT_PRIORITY = 1 << 8, /* capacity ranks in slot-major order (see moe_shape_t) */
-    MOE_FLAG_MXFP8 = 1 << 9          /* workspace for moe_forward_mxfp8 (MXFP8 experts); the
+    MOE_FLAG_MXFP8 = 1 << 9,         /* workspace for moe_forward_mxfp8 (MXFP8 experts); the
                                         bf16 layer calls reject it */
+    MOE_FLAG_BACKWARD = 1 << 10      /* workspace also sized for moe_backward */
 };
 
 #define MOE_MAX_E 256
@@ -322,6 +323,44 @@ MOE_API int moe_forward_mxfp8(const moe_shape_t *shape, const moe_bf16_t *x, con
                               const uint8_t *W2s_sf, float *out, float *logits_out,
                               int32_t *topk_idx_out, uint32_t *status, void *ws, size_t ws_bytes,
                               moe_stream_t stream);
+
+/* ---- Backward pass ("Sparse MoE Block" / "Expert FFN" differentiated with the
+ * routing decisions held fixed: top-k set, capacity drops, slot order).
+ *
+ * moe_pack_backward: the transposed expert weights the backward GEMMs read,
+ * from the forward's packed W13 and W2 (once per weight update):
+ *   W13T [E, d, 2*d_ff] bf16 out: W13T[e][i][p] = W13[e][p][i]
+ *   W2T  [E, d_ff, d]   bf16 out: W2T[e][c][i]  = W2[e][i][c] */
+MOE_API int moe_pack_backward(const moe_shape_t *shape, const moe_bf16_t *W13,
+                              const moe_bf16_t *W2, moe_bf16_t *W13T, moe_bf16_t *W2T,
+                              moe_stream_t stream);
+
+/* Gradients of sum(out * dout) for the layer moe_forward computes (routing
+ * recomputed with the same kernels, so it is identical). Requires
+ * MOE_FLAG_BACKWARD in shape->flags (also for moe_workspace_size); rejects
+ * MOE_FLAG_MXFP8 and MOE_FLAG_SIMT_FFN (MOE_ERR_INVALID_ARG); a shared expert
+ * (d_ff_shared > 0) is not supported by this build (MOE_ERR_UNSUPPORTED).
+ *   x, Wg, bias, W13  as moe_forward; W13T, W2T as moe_pack_backward writes
+ *   dout  [T, d] fp32 in
+ *   dx    [T, d] fp32 out: through the experts and through the router
+ *   dW13  [E, 2*d_ff, d] fp32 out, in the packed W13 order (rows of dW1 and
+ *         dW3 interleaved by 128 as in moe_pack_w13)
+ *   dW2   [E, d, d_ff] fp32 out
+ *   dWg   [E, d] fp32 out; dbias [E] fp32 out (written even if bias is NULL)
+ *   dlogits [T, E] fp32 out, or NULL
+ * For a kept assignment (t, j) to expert e with weight w: dW2_e += w dout_t
+ * h^T, dh = w W2_e^T dout_t, du = dh silu(g), dg = dh u silu'(g),
+ * dW1_e += dg x^T, dW3_e += du x^T, dx_t += W1_e^T dg + W3_e^T du; the
+ * router: dl_j = w_j G_j - w_j sum_i w_i G_i with G_j = <dout_t, y_j> over the
+ * chosen experts, dWg += dl^T x, dbias += sum_t dl, dx += dl Wg. bf16
+ * operands (x, h, w*dout, [dg | du], gate/up), fp32 accumulation. The weight
+ * gradients are plain per-expert GEMMs (bitwise repeatable); dx and dlogits
+ * use fp32 atomic adds. */
+MOE_API int moe_backward(const moe_shape_t *shape, const moe_bf16_t *x, const moe_bf16_t *Wg,
+                         const float *bias, const moe_bf16_t *W13, const moe_bf16_t *W13T,
+                         const moe_bf16_t *W2T, const float *dout, float *dx, float *dW13,
+                         float *dW2, float *dWg, float *dbias, float *dlogits, uint32_t *status,
+                         void *ws, size_t ws_bytes, moe_stream_t stream);
 
 /* moe_permute without a workspace, for callers that cannot allocate device
  * memory: code running while a stream is captured in global capture mode

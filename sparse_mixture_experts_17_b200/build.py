@@ -23,7 +23,7 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libmoe.so")
 SOURCES = ["dispatch.cu", "gemm_simt.cu", "gemm_tc.cu", "gemm_mx.cu", "mx_quant.cu", "decode.cu",
-           "expert_choice.cu", "moe_api.cu", "permute_static.cu"]
+           "expert_choice.cu", "backward.cu", "moe_api.cu", "permute_static.cu"]
 HEADERS = ["common.cuh", "internal.h", "topk.cuh", "mxfp8.cuh"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

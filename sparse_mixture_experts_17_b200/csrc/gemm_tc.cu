@@ -71,6 +71,12 @@ struct TcArgs {
     int32_t *route_idx;
     float *route_w;
     int32_t *counter_zero;
+    void *out2;
+    const uint16_t *gu;
+    float *row_dot;
+    const int32_t *grp_kb0;
+    const int32_t *grp_nkb;
+    long long out_group_stride;
 };
 
 template <int BN>
@@ -102,9 +108,90 @@ __device__ __forceinline__ void tile_coords(long long tile, int num_mt, int n_ti
 // lanes run it; only rows inside the expert's segment (`valid`) are written.
 template <int BN, int MODE>
 __device__ __forceinline__ void epilogue_tile(const TcArgs &p, uint32_t tb, long long row,
-                                              bool valid, int n_idx)
+                                              bool valid, int n_idx, int grp, bool empty_k)
 {
-    if (MODE == EPI_SWIGLU) {
+    if (MODE == EPI_SWIGLU_SAVE) {
+        // as EPI_SWIGLU, and the raw accumulators (gate | up of this 128-column
+        // block, the packed W13 order) as bf16 for the backward pass
+        uint16_t *H = static_cast<uint16_t *>(p.out) + row * p.ldo + n_idx * 128;
+        uint16_t *GU = static_cast<uint16_t *>(p.out2) + row * 2 * p.ldo + n_idx * 256;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+            float g[32], u[32];
+            tmem_ld32(tb + c * 32, g);
+            tmem_ld32(tb + 128 + c * 32, u);
+            tmem_ld_wait();
+            uint32_t ph[16], pg[16], pu[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                ph[i] = pack_bf16x2(silu_mul(g[2 * i], u[2 * i]), silu_mul(g[2 * i + 1], u[2 * i + 1]));
+                pg[i] = pack_bf16x2(g[2 * i], g[2 * i + 1]);
+                pu[i] = pack_bf16x2(u[2 * i], u[2 * i + 1]);
+            }
+            if (valid) {
+                uint4 *dh = reinterpret_cast<uint4 *>(H + c * 32);
+                uint4 *dg = reinterpret_cast<uint4 *>(GU + c * 32);
+                uint4 *du = reinterpret_cast<uint4 *>(GU + 128 + c * 32);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    dh[i] = make_uint4(ph[4 * i], ph[4 * i + 1], ph[4 * i + 2], ph[4 * i + 3]);
+                    dg[i] = make_uint4(pg[4 * i], pg[4 * i + 1], pg[4 * i + 2], pg[4 * i + 3]);
+                    du[i] = make_uint4(pu[4 * i], pu[4 * i + 1], pu[4 * i + 2], pu[4 * i + 3]);
+                }
+            }
+        }
+    } else if (MODE == EPI_SWIGLU_BWD) {
+        // acc columns = dh for h columns n_idx*BN ..; with s = sigmoid(g):
+        //   du = dh * g s,  dg = dh * u * s (1 + g (1 - s)),  row_dot += dh * g s u
+        // written as [dg | du] in the packed W13 order (block of 128 columns)
+        float dot = 0.f;
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+            float v[32];
+            tmem_ld32(tb + c * 32, v);
+            tmem_ld_wait();
+            if (valid) {
+                const int col = n_idx * BN + c * 32;               // h column
+                const long long pk = row * 2 * p.ldo + (long long)(col / 128) * 256 + (col % 128);
+                const uint4 *gsrc = reinterpret_cast<const uint4 *>(p.gu + pk);
+                const uint4 *usrc = reinterpret_cast<const uint4 *>(p.gu + pk + 128);
+                uint32_t og[16], ou[16];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const uint4 gw = gsrc[i], uw = usrc[i];
+                    const uint32_t gg[4] = {gw.x, gw.y, gw.z, gw.w};
+                    const uint32_t uu[4] = {uw.x, uw.y, uw.z, uw.w};
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        float dg2[2], du2[2];
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            const float g = h ? bf16hi(gg[q]) : bf16lo(gg[q]);
+                            const float u = h ? bf16hi(uu[q]) : bf16lo(uu[q]);
+                            const float dh = v[8 * i + 2 * q + h];
+                            const float sg = __fdividef(1.f, 1.f + __expf(-g));
+                            const float silu = g * sg;
+                            du2[h] = dh * silu;
+                            dg2[h] = dh * u * sg * (1.f + g * (1.f - sg));
+                            dot = fmaf(dh, silu * u, dot);
+                        }
+                        og[4 * i + q] = pack_bf16x2(dg2[0], dg2[1]);
+                        ou[4 * i + q] = pack_bf16x2(du2[0], du2[1]);
+                    }
+                }
+                uint16_t *dst = static_cast<uint16_t *>(p.out) + pk;
+                uint4 *dg = reinterpret_cast<uint4 *>(dst);
+                uint4 *du = reinterpret_cast<uint4 *>(dst + 128);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    dg[i] = make_uint4(og[4 * i], og[4 * i + 1], og[4 * i + 2], og[4 * i + 3]);
+                    du[i] = make_uint4(ou[4 * i], ou[4 * i + 1], ou[4 * i + 2], ou[4 * i + 3]);
+                }
+            }
+        }
+        if (valid)
+            atomicAdd(p.row_dot + row, dot);
+    } else if (MODE == EPI_SWIGLU) {
         // accumulator columns [0,128) = gate, [128,256) = up of H columns n_idx*128..
         uint16_t *H = static_cast<uint16_t *>(p.out) + row * p.ldo + n_idx * 128;
 #pragma unroll 1
@@ -132,6 +219,8 @@ __device__ __forceinline__ void epilogue_tile(const TcArgs &p, uint32_t tb, long
             t = p.perm_token[row];
             if (p.perm_w) {
                 wgt = p.perm_w[row];
+            } else if (!p.slot_pos) {
+                wgt = 1.f;   // unweighted scatter-add (the backward pass's dx)
             } else {
                 for (int j = 0; j < p.k; ++j)
                     if (p.slot_pos[(long long)t * p.k + j] == row)
@@ -153,12 +242,18 @@ __device__ __forceinline__ void epilogue_tile(const TcArgs &p, uint32_t tb, long
             }
         }
     } else if (MODE == EPI_STORE_F32) {
-        float *o = static_cast<float *>(p.out) + row * p.ldo + n_idx * BN;
+        float *o = static_cast<float *>(p.out) + (long long)grp * p.out_group_stride +
+                   row * p.ldo + n_idx * BN;
 #pragma unroll 1
         for (int c = 0; c < BN / 32; ++c) {
             float v[32];
             tmem_ld32(tb + c * 32, v);
             tmem_ld_wait();
+            if (empty_k) {   // a group with no k-blocks: its output block is zero
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    v[i] = 0.f;
+            }
             if (valid) {
                 float4 *dst = reinterpret_cast<float4 *>(o + c * 32);
 #pragma unroll
@@ -293,8 +388,11 @@ __global__ void __launch_bounds__(192, 1)
                 const int row0 = p.mt_row0 ? p.mt_row0[m_idx] : m_idx * C::BM;
                 const int grp = p.mt_group ? (p.mt_group[m_idx] & ~kHalfTileBit) : 0;
                 const int brow = grp * p.b_rows_per_group + n_idx * BN;
+                // K-grouped GEMMs contract over their group's own k-block range
+                const int kb0 = p.grp_kb0 ? p.grp_kb0[grp] : 0;
+                const int nkb = p.grp_kb0 ? p.grp_nkb[grp] : p.kblocks;
                 bool ok = true;
-                for (int kb = 0; kb < p.kblocks; ++kb, ++it) {
+                for (int kb = 0; kb < nkb; ++kb, ++it) {
                     const int s = it % C::STAGES;
                     const uint32_t ph = (it / C::STAGES) & 1u;
                     if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag, p.status)) {
@@ -302,8 +400,8 @@ __global__ void __launch_bounds__(192, 1)
                         break;
                     }
                     mbar_arrive_expect_tx(&full[s], C::STAGE_BYTES);
-                    tma_load_2d(sA + s * C::A_BYTES, &tmA, kb * C::BK, row0, &full[s]);
-                    tma_load_2d(sB + s * C::B_BYTES, &tmB, kb * C::BK, brow, &full[s]);
+                    tma_load_2d(sA + s * C::A_BYTES, &tmA, (kb0 + kb) * C::BK, row0, &full[s]);
+                    tma_load_2d(sB + s * C::B_BYTES, &tmB, (kb0 + kb) * C::BK, brow, &full[s]);
                 }
                 if (!ok)
                     break;
@@ -320,12 +418,14 @@ __global__ void __launch_bounds__(192, 1)
                 tile_coords(tile, num_mt, p.n_tiles, p.group_m, m_idx, n_idx);
                 const bool half = p.mt_group && (p.mt_group[m_idx] & kHalfTileBit);
                 const uint32_t IDESC = half ? IDESC64 : IDESC128;
+                const int grp = p.mt_group ? (p.mt_group[m_idx] & ~kHalfTileBit) : 0;
+                const int nkb = p.grp_kb0 ? p.grp_nkb[grp] : p.kblocks;
                 if (!mbar_wait(&tempty[b], aph ^ 1u, abort_flag, p.status))
                     break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + b * BN;
                 bool ok = true;
-                for (int kb = 0; kb < p.kblocks; ++kb, ++it) {
+                for (int kb = 0; kb < nkb; ++kb, ++it) {
                     const int s = it % C::STAGES;
                     const uint32_t ph = (it / C::STAGES) & 1u;
                     if (!mbar_wait(&full[s], ph, abort_flag, p.status)) {
@@ -366,8 +466,9 @@ __global__ void __launch_bounds__(192, 1)
             const long long row = row0 + (half ? q * 16 + lane : q * 32 + lane);
             const bool valid = (!half || lane < 16) && row < row_end;
             const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + b * BN;
+            const bool empty_k = p.grp_kb0 && p.grp_nkb[grp] == 0;
 
-            epilogue_tile<BN, MODE>(p, tb, row, valid, n_idx);
+            epilogue_tile<BN, MODE>(p, tb, row, valid, n_idx, grp, empty_k);
             tc_fence_before();
             __syncwarp();
             if (lane == 0)
@@ -529,7 +630,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
             const long long row = row0 + q * 32 + lane;
             const bool valid = row < row_end;
             const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + b * BN;
-            epilogue_tile<BN, MODE>(p, tb, row, valid, n_idx);
+            epilogue_tile<BN, MODE>(p, tb, row, valid, n_idx, grp, false);
             tc_fence_before();
             __syncwarp();
             if (lane == 0)
@@ -603,7 +704,7 @@ static int launch_tc_impl(const GemmArgs &g, cudaStream_t st)
         return rc;
     TcArgs p;
     p.kblocks = g.K / 64;
-    p.n_tiles = (MODE == EPI_SWIGLU) ? g.N / 256 : (g.N + BN - 1) / BN;
+    p.n_tiles = (MODE == EPI_SWIGLU || MODE == EPI_SWIGLU_SAVE) ? g.N / 256 : (g.N + BN - 1) / BN;
     // Rasterisation: consecutive tiles sweep a band of group_m m-tiles across
     // all n-tiles, so a band's B tiles are fetched from HBM about once while
     // its A rows stay in L2. Measured on the Mixtral-shape prefill: bands of 32
@@ -629,6 +730,12 @@ static int launch_tc_impl(const GemmArgs &g, cudaStream_t st)
     p.route_idx = g.route_idx;
     p.route_w = g.route_w;
     p.counter_zero = g.counter_zero;
+    p.out2 = g.out2;
+    p.gu = g.gu;
+    p.row_dot = g.row_dot;
+    p.grp_kb0 = g.grp_kb0;
+    p.grp_nkb = g.grp_nkb;
+    p.out_group_stride = g.out_group_stride;
 
     static int attr_done[64] = {0};
     int dev = 0;
@@ -721,6 +828,11 @@ int launch_gemm_tc(const GemmArgs &g, cudaStream_t st)
     case EPI_ROUTER:
         // 64-column tiles: more CTAs for few 128-token tiles; x re-reads hit L2
         return launch_tc_impl<64, EPI_ROUTER>(g, st);
+    case EPI_SWIGLU_SAVE:
+        return launch_tc_impl<256, EPI_SWIGLU_SAVE>(g, st);
+    case EPI_SWIGLU_BWD:
+        return (g.N % 256 == 0) ? launch_tc_impl<256, EPI_SWIGLU_BWD>(g, st)
+                                : launch_tc_impl<128, EPI_SWIGLU_BWD>(g, st);
     case EPI_ROUTER_TOPK:
         if (g.N > 64 || g.k < 1 || g.k > MOE_MAX_K)
             return MOE_ERR_INVALID_ARG;

@@ -51,6 +51,10 @@ struct WsLayout {
     size_t xq, xsf, Hq, Hsf, xq_s, xsf_s, Hsq, Hssf;   // MXFP8 operands
     size_t dec_xdq, dec_H32;                             // MXFP8 decode
     size_t tile_start;                                   // first m-tile of each expert
+    // backward pass
+    size_t GU, dYw, dGU, row_dot, pstart, kb0, nkb, mtk1_row0, mtk1_group, mtk2_row0,
+        mtk2_group, dYwT, HT, dGUT, XpT, dl;
+    long long Np;                                        // padded rows of the transposes
     size_t total;
     int nchunks, max_mt, max_mt2;
 };
@@ -88,8 +92,13 @@ enum EpiMode {
     EPI_ROUTER = 3,     // out[row, n] = acc[n] + bias[n] for n < n_valid
     EPI_SWIGLU_MX = 4,  // MXFP8 GEMM: h = silu(gate) * up, quantized to MXFP8 codes (out)
                         // and block scales (out_sf)
-    EPI_ROUTER_TOPK = 5 // EPI_ROUTER, then (E <= 64, one 64-column tile) the top-k of each
+    EPI_ROUTER_TOPK = 5,// EPI_ROUTER, then (E <= 64, one 64-column tile) the top-k of each
                         // row and its renormalised weights into route_idx / route_w
+    EPI_SWIGLU_SAVE = 6,// EPI_SWIGLU, and the raw gate / up accumulators as bf16 in the packed
+                        // W13 order into out2 [rows, 2 N/2] (for the backward pass)
+    EPI_SWIGLU_BWD = 7  // backward through SwiGLU: acc = dh; reads the saved gate / up (gu),
+                        // writes [dg | du] bf16 in the packed order into out and adds
+                        // sum_c dh * h per row into row_dot (fp32)
 };
 
 struct GemmArgs {
@@ -131,6 +140,16 @@ struct GemmArgs {
     int32_t *route_idx;
     float *route_w;
     int32_t *counter_zero;
+    // backward pass
+    void *out2;                  // EPI_SWIGLU_SAVE: gate / up [rows, 2 * ldo]
+    const uint16_t *gu;          // EPI_SWIGLU_BWD: the saved gate / up [rows, 2 * ldo/2]
+    float *row_dot;              // EPI_SWIGLU_BWD: per-row sum of dh * h (atomic adds)
+    // K-grouped GEMM (weight gradients): group g of the m-tile list contracts
+    // over k-blocks [grp_kb0[g], grp_kb0[g] + grp_nkb[g]); its output starts at
+    // out + g * out_group_stride; B rows are shared (b_rows_per_group = 0)
+    const int32_t *grp_kb0;
+    const int32_t *grp_nkb;
+    long long out_group_stride;
 };
 
 int launch_gemm_tc(const GemmArgs &g, cudaStream_t st);
@@ -173,6 +192,22 @@ int launch_dec_w2_mx(const moe_shape_t &s, const int32_t *topk_idx, const float 
                      const uint8_t *W2q, const uint8_t *W2sf, const uint8_t *W2s_q,
                      const uint8_t *W2s_sf, const uint16_t *Hdq, float *out, uint32_t *status,
                      cudaStream_t st);
+
+// ---- backward pass helpers (backward.cu)
+int launch_transpose_batched(const uint16_t *src, int batch, int R, int C, uint16_t *dst,
+                             cudaStream_t st);
+int launch_transpose_grouped(const uint16_t *src, int n, int C, const int32_t *offsets,
+                             const int32_t *pstart, int E, uint16_t *dst, long long ldd,
+                             cudaStream_t st);
+int launch_group_ranges(const int32_t *offsets, int E, int32_t *pstart, int32_t *kb0,
+                        int32_t *nkb, int M1, int32_t *mt1_row0, int32_t *mt1_group, int M2,
+                        int32_t *mt2_row0, int32_t *mt2_group, cudaStream_t st);
+int launch_bwd_dyw(const moe_shape_t &s, const float *dout, const int32_t *slot_pos,
+                   const float *topk_w, uint16_t *dyw, cudaStream_t st);
+int launch_router_bwd(const moe_shape_t &s, const int32_t *idx, const float *topk_w,
+                      const int32_t *slot_pos, const float *row_dot, const uint16_t *x,
+                      const uint16_t *Wg, float *dl, float *dWg, float *dbias, float *dx,
+                      cudaStream_t st);
 
 // ---- expert-choice routing (expert_choice.cu)
 int launch_softmax_rows(const moe_shape_t &s, const float *logits, float *scores,

@@ -147,6 +147,27 @@ WsLayout ws_layout(const moe_shape_t &s)
     L.Hsq = take(mx && dfs ? T * dfs : 0);
     L.Hssf = take(mx && dfs ? (size_t)sf_atom_bytes(T, (int)dfs) : 0);
     L.tile_start = take(mx ? E * 4 : 0);
+    // backward pass: saved gate/up, w * dout, [dg | du], per-row <dh, h>, the
+    // K-grouped GEMMs' ranges and tile lists, and the padded transposes
+    const bool bw = (s.flags & MOE_FLAG_BACKWARD) != 0;
+    const size_t Np = bw ? ((N + 64 * E + 63) / 64) * 64 : 0;
+    L.Np = (long long)Np;
+    L.GU = take(bw ? N * 2 * s.d_ff * 2 : 0);
+    L.dYw = take(bw ? N * s.d * 2 : 0);
+    L.dGU = take(bw ? N * 2 * s.d_ff * 2 : 0);
+    L.row_dot = take(bw ? N * 4 : 0);
+    L.pstart = take(bw ? (E + 1) * 4 : 0);
+    L.kb0 = take(bw ? E * 4 : 0);
+    L.nkb = take(bw ? E * 4 : 0);
+    L.mtk1_row0 = take(bw ? E * (s.d / kBlockM) * 4 : 0);
+    L.mtk1_group = take(bw ? E * (s.d / kBlockM) * 4 : 0);
+    L.mtk2_row0 = take(bw ? E * (2 * s.d_ff / kBlockM) * 4 : 0);
+    L.mtk2_group = take(bw ? E * (2 * s.d_ff / kBlockM) * 4 : 0);
+    L.dYwT = take(bw ? s.d * Np * 2 : 0);
+    L.HT = take(bw ? s.d_ff * Np * 2 : 0);
+    L.dGUT = take(bw ? 2 * s.d_ff * Np * 2 : 0);
+    L.XpT = take(bw ? s.d * Np * 2 : 0);
+    L.dl = take(bw ? T * E * 4 : 0);
     L.scores = take(ec ? T * E * 4 : 0);
     L.ec_w = take(ec ? N * 4 : 0);
     L.x_stage = take((s.flags & MOE_FLAG_HOST_IO) ? T * s.d * 2 : 0);
@@ -652,6 +673,175 @@ static int forward_mx_impl(const moe_shape_t &s, const WsLayout &L, void *ws, co
         return rc;
     StageMark m(MOE_STAGE_COMBINE, st);
     return launch_combine(s, Y, slot_pos, w, shared ? out : nullptr, out, st);
+}
+
+// ---------------------------------------------------------------- backward pass
+static int backward_impl(const moe_shape_t &s, const WsLayout &L, void *ws, const uint16_t *x,
+                         const uint16_t *Wg, const float *bias, const uint16_t *W13,
+                         const uint16_t *W13T, const uint16_t *W2T, const float *dout, float *dx,
+                         float *dW13, float *dW2, float *dWg, float *dbias, float *dlogits,
+                         uint32_t *status, cudaStream_t st)
+{
+    const long long N = (long long)s.T * s.k;
+    float *logits = at<float>(ws, L.logits);
+    int32_t *idx = at<int32_t>(ws, L.topk_idx);
+    float *w = at<float>(ws, L.topk_w);
+    int32_t *counter = at<int32_t>(ws, L.counter);
+    int32_t *offsets = at<int32_t>(ws, L.offsets);
+    int32_t *chunk = at<int32_t>(ws, L.chunk_counts);
+    int32_t *rank = at<int32_t>(ws, L.rank_local);
+    int32_t *slot_pos = at<int32_t>(ws, L.slot_pos);
+    int32_t *perm_token = at<int32_t>(ws, L.perm_token);
+    uint16_t *x_perm = at<uint16_t>(ws, L.x_perm);
+    uint16_t *H = at<uint16_t>(ws, L.H);
+    uint16_t *GU = at<uint16_t>(ws, L.GU);
+    uint16_t *dYw = at<uint16_t>(ws, L.dYw);
+    uint16_t *dGU = at<uint16_t>(ws, L.dGU);
+    float *row_dot = at<float>(ws, L.row_dot);
+    float *dl = dlogits ? dlogits : at<float>(ws, L.dl);
+    int rc;
+    // routing and dispatch: the forward's kernels, so the decisions are identical
+    if ((rc = route_tokens(s, x, Wg, bias, logits, idx, w, counter, status, st)))
+        return rc;
+    {
+        StageMark m(MOE_STAGE_HIST, st);
+        rc = launch_hist_scan(s, idx, chunk, rank, counter, at<int32_t>(ws, L.counts), offsets,
+                              at<int32_t>(ws, L.n_kept), at<int32_t>(ws, L.mt_row0),
+                              at<int32_t>(ws, L.mt_group), at<int32_t>(ws, L.num_mt), nullptr,
+                              nullptr, nullptr, status, st);
+    }
+    if (rc)
+        return rc;
+    {
+        StageMark m(MOE_STAGE_PERMUTE, st);
+        if ((rc = launch_permute(s, idx, chunk, rank, offsets, x, slot_pos, perm_token, x_perm,
+                                 nullptr, st)))
+            return rc;
+        if ((rc = launch_bwd_dyw(s, dout, slot_pos, w, dYw, st)))
+            return rc;
+    }
+    // w1/w3 again, keeping the gate / up accumulators
+    GemmArgs g = gemm_base();
+    g.mode = EPI_SWIGLU_SAVE;
+    g.A = x_perm;
+    g.a_rows = N;
+    g.B = W13;
+    g.b_rows_total = (long long)s.E * 2 * s.d_ff;
+    g.K = s.d;
+    g.N = 2 * s.d_ff;
+    g.b_rows_per_group = 2 * s.d_ff;
+    set_tiles(g, L, ws, false);
+    g.seg_offsets = offsets;
+    g.out = H;
+    g.ldo = s.d_ff;
+    g.out2 = GU;
+    g.status = status;
+    {
+        StageMark m(MOE_STAGE_W13, st);
+        if ((rc = launch_gemm_tc(g, st)))
+            return rc;
+    }
+    // dh = (w dout) W2_e, then through SwiGLU: [dg | du] and row sums <dh, h>
+    if (cudaMemsetAsync(row_dot, 0, sizeof(float) * (size_t)std::max(N, 1LL), st) != cudaSuccess ||
+        cudaMemsetAsync(dx, 0, sizeof(float) * (size_t)s.T * s.d, st) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    g = gemm_base();
+    g.mode = EPI_SWIGLU_BWD;
+    g.A = dYw;
+    g.a_rows = N;
+    g.B = W2T;
+    g.b_rows_total = (long long)s.E * s.d_ff;
+    g.K = s.d;
+    g.N = s.d_ff;
+    g.b_rows_per_group = s.d_ff;
+    set_tiles(g, L, ws, false);
+    g.seg_offsets = offsets;
+    g.out = dGU;
+    g.ldo = s.d_ff;
+    g.gu = GU;
+    g.row_dot = row_dot;
+    g.status = status;
+    {
+        StageMark m(MOE_STAGE_W2, st);
+        if ((rc = launch_gemm_tc(g, st)))
+            return rc;
+    }
+    // dx += [dg | du] [W1; W3]_e, scattered back to the tokens (weight 1)
+    g = gemm_base();
+    g.mode = EPI_COMBINE;
+    g.A = dGU;
+    g.a_rows = N;
+    g.B = W13T;
+    g.b_rows_total = (long long)s.E * s.d;
+    g.K = 2 * s.d_ff;
+    g.N = s.d;
+    g.b_rows_per_group = s.d;
+    set_tiles(g, L, ws, false);
+    g.seg_offsets = offsets;
+    g.out = dx;
+    g.ldo = s.d;
+    g.perm_token = perm_token;
+    g.status = status;
+    if ((rc = launch_gemm_tc(g, st)))
+        return rc;
+    // weight gradients: contractions over each expert's rows
+    int32_t *pstart = at<int32_t>(ws, L.pstart);
+    int32_t *kb0 = at<int32_t>(ws, L.kb0);
+    int32_t *nkb = at<int32_t>(ws, L.nkb);
+    if ((rc = launch_group_ranges(offsets, s.E, pstart, kb0, nkb, s.d, at<int32_t>(ws, L.mtk1_row0),
+                                  at<int32_t>(ws, L.mtk1_group), 2 * s.d_ff,
+                                  at<int32_t>(ws, L.mtk2_row0), at<int32_t>(ws, L.mtk2_group), st)))
+        return rc;
+    const long long Np = L.Np;
+    uint16_t *dYwT = at<uint16_t>(ws, L.dYwT), *HT = at<uint16_t>(ws, L.HT);
+    uint16_t *dGUT = at<uint16_t>(ws, L.dGUT), *XpT = at<uint16_t>(ws, L.XpT);
+    if ((rc = launch_transpose_grouped(dYw, (int)N, s.d, offsets, pstart, s.E, dYwT, Np, st)) ||
+        (rc = launch_transpose_grouped(H, (int)N, s.d_ff, offsets, pstart, s.E, HT, Np, st)) ||
+        (rc = launch_transpose_grouped(dGU, (int)N, 2 * s.d_ff, offsets, pstart, s.E, dGUT, Np, st)) ||
+        (rc = launch_transpose_grouped(x_perm, (int)N, s.d, offsets, pstart, s.E, XpT, Np, st)))
+        return rc;
+    // dW2_e = (w dout)_e^T h_e  [d, d_ff]
+    g = gemm_base();
+    g.mode = EPI_STORE_F32;
+    g.A = dYwT;
+    g.a_rows = s.d;
+    g.B = HT;
+    g.b_rows_total = s.d_ff;
+    g.K = (int)Np;
+    g.N = s.d_ff;
+    g.b_rows_per_group = 0;
+    g.mt_row0 = at<int32_t>(ws, L.mtk1_row0);
+    g.mt_group = at<int32_t>(ws, L.mtk1_group);
+    g.num_mt_host = s.E * (s.d / kBlockM);
+    g.max_mt = g.num_mt_host;
+    g.rows_valid = s.d;
+    g.grp_kb0 = kb0;
+    g.grp_nkb = nkb;
+    g.out = dW2;
+    g.ldo = s.d_ff;
+    g.out_group_stride = (long long)s.d * s.d_ff;
+    g.status = status;
+    if ((rc = launch_gemm_tc(g, st)))
+        return rc;
+    // dW13_e = [dg | du]_e^T x_e  [2 d_ff, d] (the packed W13 order)
+    g.A = dGUT;
+    g.a_rows = 2LL * s.d_ff;
+    g.B = XpT;
+    g.b_rows_total = s.d;
+    g.N = s.d;
+    g.mt_row0 = at<int32_t>(ws, L.mtk2_row0);
+    g.mt_group = at<int32_t>(ws, L.mtk2_group);
+    g.num_mt_host = s.E * (2 * s.d_ff / kBlockM);
+    g.max_mt = g.num_mt_host;
+    g.rows_valid = 2LL * s.d_ff;
+    g.out = dW13;
+    g.ldo = s.d;
+    g.out_group_stride = 2LL * s.d_ff * s.d;
+    if ((rc = launch_gemm_tc(g, st)))
+        return rc;
+    // router: dl, dWg, dbias, and dx += dl Wg
+    StageMark m(MOE_STAGE_COMBINE, st);
+    return launch_router_bwd(s, idx, w, slot_pos, row_dot, x, Wg, dl, dWg, dbias, dx, st);
 }
 
 // ---------------------------------------------------------------- expert-choice routing
@@ -1175,6 +1365,50 @@ int moe_forward_mxfp8(const moe_shape_t *shape, const moe_bf16_t *x, const moe_b
     return forward_mx_impl(s, L, ws, x, Wg, bias, W13q, W13sf, W2q, W2sf, W13s_q, W13s_sf, W2s_q,
                            W2s_sf, out, logits_out, topk_idx_out, status,
                            reinterpret_cast<cudaStream_t>(stream));
+}
+
+int moe_pack_backward(const moe_shape_t *shape, const moe_bf16_t *W13, const moe_bf16_t *W2,
+                      moe_bf16_t *W13T, moe_bf16_t *W2T, moe_stream_t stream)
+{
+    int rc = check_shape(shape);
+    if (rc)
+        return rc;
+    if (shape->T == 0)
+        return MOE_OK;
+    const moe_shape_t &s = *shape;
+    if (!W13 || !W2 || !W13T || !W2T || !al16(W13) || !al16(W2) || !al16(W13T) || !al16(W2T))
+        return MOE_ERR_INVALID_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if ((rc = launch_transpose_batched(W13, s.E, 2 * s.d_ff, s.d, W13T, st)))
+        return rc;
+    return launch_transpose_batched(W2, s.E, s.d, s.d_ff, W2T, st);
+}
+
+int moe_backward(const moe_shape_t *shape, const moe_bf16_t *x, const moe_bf16_t *Wg,
+                 const float *bias, const moe_bf16_t *W13, const moe_bf16_t *W13T,
+                 const moe_bf16_t *W2T, const float *dout, float *dx, float *dW13, float *dW2,
+                 float *dWg, float *dbias, float *dlogits, uint32_t *status, void *ws,
+                 size_t ws_bytes, moe_stream_t stream)
+{
+    int rc = check_shape(shape);
+    if (rc)
+        return rc;
+    if (shape->T == 0)
+        return MOE_OK;
+    const moe_shape_t &s = *shape;
+    if (!(s.flags & MOE_FLAG_BACKWARD) || (s.flags & (MOE_FLAG_MXFP8 | MOE_FLAG_SIMT_FFN)))
+        return MOE_ERR_INVALID_ARG;
+    if (s.d_ff_shared > 0)
+        return MOE_ERR_UNSUPPORTED;
+    if (!x || !Wg || !W13 || !W13T || !W2T || !dout || !dx || !dW13 || !dW2 || !dWg || !dbias ||
+        !al16(x) || !al16(Wg) || !al16(W13) || !al16(W13T) || !al16(W2T) || !al16(dout) ||
+        !al16(dx) || !al16(dW13) || !al16(dW2))
+        return MOE_ERR_INVALID_ARG;
+    WsLayout L;
+    if ((rc = check_ws(s, ws, ws_bytes, L)))
+        return rc;
+    return backward_impl(s, L, ws, x, Wg, bias, W13, W13T, W2T, dout, dx, dW13, dW2, dWg, dbias,
+                         dlogits, status, reinterpret_cast<cudaStream_t>(stream));
 }
 
 } // extern "C"

@@ -37,6 +37,7 @@ MOE_FLAG_GEMM_2SM = 1 << 6
 MOE_FLAG_EXPERT_CHOICE = 1 << 7
 MOE_FLAG_SLOT_PRIORITY = 1 << 8
 MOE_FLAG_MXFP8 = 1 << 9
+MOE_FLAG_BACKWARD = 1 << 10
 
 MOE_MAX_E = 256
 MOE_MAX_K = 16
@@ -86,6 +87,8 @@ _SIGS = {
     "moe_permute_static": ([_SHP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P], ctypes.c_int),
     "moe_quantize_experts_mxfp8": ([_SHP, _P, _P, _P, _P, _P, _P, _P, _P], ctypes.c_int),
     "moe_forward_mxfp8": ([_SHP] + [_P] * 16 + [_SZ, _P], ctypes.c_int),
+    "moe_pack_backward": ([_SHP, _P, _P, _P, _P, _P], ctypes.c_int),
+    "moe_backward": ([_SHP] + [_P] * 15 + [_SZ, _P], ctypes.c_int),
     "moe_route_expert_choice": ([_SHP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P], ctypes.c_int),
     "moe_forward_expert_choice": ([_SHP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P],
                                   ctypes.c_int),
@@ -340,6 +343,39 @@ def sf_atoms_to_rows(sf, rows: int, K: int):
     a = sf.reshape(rows // 128, K // 128, 32, 4, 4)     # [tile, group, m%32, m/32, block]
     a = a.permute(0, 3, 2, 1, 4) if isinstance(a, torch.Tensor) else a.transpose(0, 3, 2, 1, 4)
     return a.reshape(rows, K // 32)
+
+
+def moe_pack_backward(shape, W13, W2, stream=None):
+    """Transposed expert weights for moe_backward: (W13T [E, d, 2 d_ff], W2T [E, d_ff, d])."""
+    E, d_ff, d = shape.E, shape.d_ff, shape.d
+    W13T = torch.empty(E, d, 2 * d_ff, dtype=BF16, device=W13.device)
+    W2T = torch.empty(E, d_ff, d, dtype=BF16, device=W13.device)
+    _check("moe_pack_backward", lib().moe_pack_backward(
+        ctypes.byref(shape), _ptr(W13, BF16, "W13"), _ptr(W2, BF16, "W2"), _ptr(W13T, BF16, "W13T"),
+        _ptr(W2T, BF16, "W2T"), _stream(stream)))
+    return W13T, W2T
+
+
+def moe_backward(shape, x, Wg, bias, W13, W13T, W2T, dout, status, ws, want_dlogits=False,
+                 stream=None) -> dict:
+    """Gradients of sum(out * dout): dict(dx, dW13 (packed order), dW2, dWg, dbias[, dlogits])."""
+    T, d, d_ff, E = shape.T, shape.d, shape.d_ff, shape.E
+    dev = x.device
+    g = dict(dx=torch.empty(T, d, dtype=F32, device=dev),
+             dW13=torch.empty(E, 2 * d_ff, d, dtype=F32, device=dev),
+             dW2=torch.empty(E, d, d_ff, dtype=F32, device=dev),
+             dWg=torch.empty(E, d, dtype=F32, device=dev),
+             dbias=torch.empty(E, dtype=F32, device=dev))
+    if want_dlogits:
+        g["dlogits"] = torch.empty(T, E, dtype=F32, device=dev)
+    _check("moe_backward", lib().moe_backward(
+        ctypes.byref(shape), _ptr(x, BF16, "x"), _ptr(Wg, BF16, "Wg"), _ptr(bias, F32, "bias"),
+        _ptr(W13, BF16, "W13"), _ptr(W13T, BF16, "W13T"), _ptr(W2T, BF16, "W2T"),
+        _ptr(dout, F32, "dout"), _ptr(g["dx"], F32, "dx"), _ptr(g["dW13"], F32, "dW13"),
+        _ptr(g["dW2"], F32, "dW2"), _ptr(g["dWg"], F32, "dWg"), _ptr(g["dbias"], F32, "dbias"),
+        _ptr(g.get("dlogits"), F32, "dlogits"), _ptr(status, U32, "status"), _ptr(ws, name="ws"),
+        ws.numel(), _stream(stream)))
+    return g
 
 
 class MoeLayerMx:
