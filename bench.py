@@ -329,11 +329,14 @@ def run_ours(a, world, rank, local):
     graphs = None
     expert_choice = None
     mxfp8 = None
+    backward = None
     if a.workload == "prefill" and not a.no_extra:
         decode = run_decode_set(M, w, layer, x, dev, stream, world, peaks)
         graphs = run_graph_set(M, layer, x, dev)
         expert_choice = run_expert_choice_set(M, w, layer, x, dev, stream, world, peaks,
                                               max(3, a.steps // 2))
+        backward = run_backward_set(M, w, inp, layer, dev, stream, world, peaks,
+                                    max(3, a.steps // 4))
         mxfp8 = run_mxfp8_set(M, w, inp, x, dev, stream, world, peaks, max(3, a.steps // 2))
 
     # ---- CPU baseline: the oracle on host cores (rank 0, N = 1 only)
@@ -372,6 +375,8 @@ def run_ours(a, world, rank, local):
         res["expert_choice"] = expert_choice
     if mxfp8 is not None:
         res["mxfp8"] = mxfp8
+    if backward is not None:
+        res["backward"] = backward
     return res
 
 
@@ -547,6 +552,48 @@ def run_mxfp8_set(M, w, inp, x, dev, stream, world, peaks, steps):
     del lay
     torch.cuda.empty_cache()
     return res
+
+
+def run_backward_set(M, w, inp, layer, dev, stream, world, peaks, steps):
+    """moe_backward on the same weights and tokens (gradients of sum(out * dout)).
+    GEMM FLOPs per step over the n kept rows: the w1/w3 recompute 4 n d d_ff,
+    dh 2 n d d_ff, dx 4 n d d_ff, dW2 2 n d d_ff, dW1/dW3 4 n d d_ff."""
+    s = M.shape_of(w, M.MOE_FLAG_BACKWARD)
+    ws = M.alloc_workspace(s, dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    W13T, W2T = M.moe_pack_backward(s, layer.W13, layer.W2)
+    g = torch.Generator(dev).manual_seed(1)
+    dout = torch.randn(w.T, w.d, generator=g, device=dev)
+    x = inp["x"]
+    grads = M.moe_backward(s, x, layer.Wg, layer.bias, layer.W13, W13T, W2T, dout, status, ws)
+
+    def step():
+        M.moe_backward(s, x, layer.Wg, layer.bias, layer.W13, W13T, W2T, dout, status, ws)
+    for _ in range(2):
+        step()
+    torch.cuda.synchronize()
+    if int(status.item()) != 0:
+        raise RuntimeError(f"device status {int(status.item())} (backward)")
+    ms = max_over_ranks(time_loop(step, steps, stream), world, dev)
+    M.moe_profile_enable(True)
+    time_loop(step, steps, stream)
+    M.moe_profile_enable(False)
+    st = M.moe_profile_read()
+    n = w.T * w.k if not w.capacity else None
+    if n is None:
+        raise RuntimeError("backward measurement expects an uncapped workload")
+    flops = 16.0 * n * w.d * w.d_ff
+    dw_ms = st["bwd_dw"][0] / st["bwd_dw"][1]
+    dh_ms = st["w2"][0] / st["w2"][1]
+    del grads, W13T, W2T, ws
+    torch.cuda.empty_cache()
+    return {"ms_per_step": round(ms, 4), "tokens_per_s": round(w.T * world / (ms / 1e3), 1),
+            "gemm_tflops": round(flops / (ms / 1e3) / 1e12, 1),
+            "gemm_frac_measured_sustained": round(flops / (ms / 1e3) / 1e12
+                                                  / peaks["bf16_tflops_sustained"], 4),
+            "dh_tflops": round(2.0 * n * w.d * w.d_ff / (dh_ms / 1e3) / 1e12, 1),
+            "weight_grad_stage_tflops": round(6.0 * n * w.d * w.d_ff / (dw_ms / 1e3) / 1e12, 1),
+            "stages_ms": {k: round(v[0] / v[1], 4) for k, v in st.items()}}
 
 
 def run_reference(a, world, rank):

@@ -386,7 +386,8 @@ MOE_API int moe_permute_static(const moe_shape_t *shape, const int32_t *topk_idx
 
 /* ---- Instrumentation (computes nothing; for measurement and tests). ---- */
 
-/* Stages of moe_forward timed by the profiler below. */
+/* Stages of moe_forward (and moe_backward) timed by the profiler below; in
+ * moe_backward, W13 is the w1/w3 recompute and W2 the dh GEMM. */
 enum {
     MOE_STAGE_ROUTER = 0,   /* router logits */
     MOE_STAGE_TOPK = 1,     /* softmax / top-k / weights */
@@ -398,7 +399,10 @@ enum {
     MOE_STAGE_COMBINE = 7,  /* fixed-order combine (deterministic mode) */
     MOE_STAGE_DEC_W13 = 8,  /* decode: chosen experts' w1/w3 + SwiGLU */
     MOE_STAGE_DEC_W2 = 9,   /* decode: chosen experts' w2 + combine */
-    MOE_NUM_STAGES = 10
+    MOE_STAGE_BWD_DX = 10,  /* backward: dx through the experts */
+    MOE_STAGE_BWD_DW = 11,  /* backward: transposes + per-expert weight-gradient GEMMs */
+    MOE_STAGE_BWD_ROUTER = 12, /* backward: router gradient (dlogits, dWg, dbias, dx) */
+    MOE_NUM_STAGES = 13
 };
 
 /* Number of kernels this library has launched in this process. */

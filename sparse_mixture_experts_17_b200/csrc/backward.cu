@@ -202,21 +202,40 @@ __global__ void __launch_bounds__(256) k_router_bwd_dl(const int32_t *__restrict
         dl[(size_t)t * E + e] = gw - wj * sum;
 }
 
-// dWg[e, i] = sum_t dl[t, e] x[t, i] (fixed order over t: deterministic);
-// thread (e, i), consecutive i across a warp.
-__global__ void __launch_bounds__(256) k_router_bwd_dwg(const float *__restrict__ dl,
-                                                        const uint16_t *__restrict__ x, int T,
-                                                        int E, int d, float *__restrict__ dWg)
+// dWg[e, i] = sum_t dl[t, e] x[t, i] in two fixed-order passes (deterministic):
+// chunk c of kDwgChunk tokens -> part[c][e][i], then the chunks summed in order.
+// Thread (e, i) with consecutive i across a warp.
+constexpr int kDwgChunk = 1024;
+
+__global__ void __launch_bounds__(256) k_router_bwd_dwg_part(const float *__restrict__ dl,
+                                                             const uint16_t *__restrict__ x,
+                                                             int T, int E, int d,
+                                                             float *__restrict__ part)
+{
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    const int e = blockIdx.y, c = blockIdx.z;
+    if (i >= d)
+        return;
+    const int t1 = min(T, (c + 1) * kDwgChunk);
+    float acc = 0.f;
+    for (int t = c * kDwgChunk; t < t1; ++t) {
+        const uint16_t xb = x[(size_t)t * d + i];
+        acc = fmaf(dl[(size_t)t * E + e], __uint_as_float((uint32_t)xb << 16), acc);
+    }
+    part[((size_t)c * E + e) * d + i] = acc;
+}
+
+__global__ void __launch_bounds__(256) k_router_bwd_dwg_sum(const float *__restrict__ part,
+                                                            int nchunks, int E, int d,
+                                                            float *__restrict__ dWg)
 {
     const int i = blockIdx.x * blockDim.x + threadIdx.x;
     const int e = blockIdx.y;
     if (i >= d)
         return;
     float acc = 0.f;
-    for (int t = 0; t < T; ++t) {
-        const uint16_t xb = x[(size_t)t * d + i];
-        acc = fmaf(dl[(size_t)t * E + e], __uint_as_float((uint32_t)xb << 16), acc);
-    }
+    for (int c = 0; c < nchunks; ++c)
+        acc += part[((size_t)c * E + e) * d + i];
     dWg[(size_t)e * d + i] = acc;
 }
 
@@ -301,10 +320,15 @@ int launch_bwd_dyw(const moe_shape_t &s, const float *dout, const int32_t *slot_
     return launched();
 }
 
+size_t router_bwd_part_bytes(const moe_shape_t &s)
+{
+    return (size_t)((s.T + kDwgChunk - 1) / kDwgChunk) * s.E * s.d * 4;
+}
+
 int launch_router_bwd(const moe_shape_t &s, const int32_t *idx, const float *topk_w,
                       const int32_t *slot_pos, const float *row_dot, const uint16_t *x,
-                      const uint16_t *Wg, float *dl, float *dWg, float *dbias, float *dx,
-                      cudaStream_t st)
+                      const uint16_t *Wg, float *dl, float *part, float *dWg, float *dbias,
+                      float *dx, cudaStream_t st)
 {
     if (s.T == 0)
         return MOE_OK;
@@ -313,7 +337,13 @@ int launch_router_bwd(const moe_shape_t &s, const int32_t *idx, const float *top
     int rc = launched();
     if (rc)
         return rc;
-    k_router_bwd_dwg<<<dim3((s.d + 255) / 256, s.E), 256, 0, st>>>(dl, x, s.T, s.E, s.d, dWg);
+    const int nchunks = (s.T + kDwgChunk - 1) / kDwgChunk;
+    k_router_bwd_dwg_part<<<dim3((s.d + 255) / 256, s.E, nchunks), 256, 0, st>>>(dl, x, s.T, s.E,
+                                                                                  s.d, part);
+    if ((rc = launched()))
+        return rc;
+    k_router_bwd_dwg_sum<<<dim3((s.d + 255) / 256, s.E), 256, 0, st>>>(part, nchunks, s.E, s.d,
+                                                                      dWg);
     if ((rc = launched()))
         return rc;
     k_router_bwd_dbias<<<s.E, 256, 0, st>>>(dl, s.T, s.E, dbias);

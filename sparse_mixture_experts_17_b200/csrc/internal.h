@@ -53,7 +53,7 @@ struct WsLayout {
     size_t tile_start;                                   // first m-tile of each expert
     // backward pass
     size_t GU, dYw, dGU, row_dot, pstart, kb0, nkb, mtk1_row0, mtk1_group, mtk2_row0,
-        mtk2_group, dYwT, HT, dGUT, XpT, dl;
+        mtk2_group, dYwT, HT, dGUT, XpT, dl, dwg_part;
     long long Np;                                        // padded rows of the transposes
     size_t total;
     int nchunks, max_mt, max_mt2;
@@ -204,10 +204,11 @@ int launch_group_ranges(const int32_t *offsets, int E, int32_t *pstart, int32_t 
                         int32_t *mt2_row0, int32_t *mt2_group, cudaStream_t st);
 int launch_bwd_dyw(const moe_shape_t &s, const float *dout, const int32_t *slot_pos,
                    const float *topk_w, uint16_t *dyw, cudaStream_t st);
+size_t router_bwd_part_bytes(const moe_shape_t &s);
 int launch_router_bwd(const moe_shape_t &s, const int32_t *idx, const float *topk_w,
                       const int32_t *slot_pos, const float *row_dot, const uint16_t *x,
-                      const uint16_t *Wg, float *dl, float *dWg, float *dbias, float *dx,
-                      cudaStream_t st);
+                      const uint16_t *Wg, float *dl, float *part, float *dWg, float *dbias,
+                      float *dx, cudaStream_t st);
 
 // ---- expert-choice routing (expert_choice.cu)
 int launch_softmax_rows(const moe_shape_t &s, const float *logits, float *scores,

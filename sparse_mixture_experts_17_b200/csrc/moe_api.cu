@@ -57,7 +57,8 @@ struct StageMark {
         if (P.on && (a = take_event(P)))
             cudaEventRecord(a, st);
     }
-    ~StageMark()
+    // Close the stage here (the destructor then does nothing).
+    void end()
     {
         if (!a)
             return;
@@ -66,7 +67,9 @@ struct StageMark {
         cudaEvent_t b = take_event(P);
         if (b && cudaEventRecord(b, st) == cudaSuccess)
             P.recs.push_back({stage, a, b});
+        a = nullptr;
     }
+    ~StageMark() { end(); }
 };
 int launch_dec_router(const moe_shape_t &s, const uint16_t *x, const uint16_t *Wg,
                       const float *bias, float *logits, cudaStream_t st);
@@ -168,6 +171,7 @@ WsLayout ws_layout(const moe_shape_t &s)
     L.dGUT = take(bw ? 2 * s.d_ff * Np * 2 : 0);
     L.XpT = take(bw ? s.d * Np * 2 : 0);
     L.dl = take(bw ? T * E * 4 : 0);
+    L.dwg_part = take(bw ? router_bwd_part_bytes(s) : 0);
     L.scores = take(ec ? T * E * 4 : 0);
     L.ec_w = take(ec ? N * 4 : 0);
     L.x_stage = take((s.flags & MOE_FLAG_HOST_IO) ? T * s.d * 2 : 0);
@@ -782,9 +786,13 @@ static int backward_impl(const moe_shape_t &s, const WsLayout &L, void *ws, cons
     g.ldo = s.d;
     g.perm_token = perm_token;
     g.status = status;
-    if ((rc = launch_gemm_tc(g, st)))
-        return rc;
+    {
+        StageMark m(MOE_STAGE_BWD_DX, st);
+        if ((rc = launch_gemm_tc(g, st)))
+            return rc;
+    }
     // weight gradients: contractions over each expert's rows
+    StageMark mdw(MOE_STAGE_BWD_DW, st);
     int32_t *pstart = at<int32_t>(ws, L.pstart);
     int32_t *kb0 = at<int32_t>(ws, L.kb0);
     int32_t *nkb = at<int32_t>(ws, L.nkb);
@@ -839,9 +847,11 @@ static int backward_impl(const moe_shape_t &s, const WsLayout &L, void *ws, cons
     g.out_group_stride = 2LL * s.d_ff * s.d;
     if ((rc = launch_gemm_tc(g, st)))
         return rc;
+    mdw.end();
     // router: dl, dWg, dbias, and dx += dl Wg
-    StageMark m(MOE_STAGE_COMBINE, st);
-    return launch_router_bwd(s, idx, w, slot_pos, row_dot, x, Wg, dl, dWg, dbias, dx, st);
+    StageMark m(MOE_STAGE_BWD_ROUTER, st);
+    return launch_router_bwd(s, idx, w, slot_pos, row_dot, x, Wg, dl, at<float>(ws, L.dwg_part),
+                             dWg, dbias, dx, st);
 }
 
 // ---------------------------------------------------------------- expert-choice routing

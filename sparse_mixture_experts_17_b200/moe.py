@@ -98,7 +98,7 @@ _SIGS = {
 }
 
 STAGES = ["router", "topk", "hist", "permute", "shared", "w13", "w2", "combine", "dec_w13",
-          "dec_w2"]
+          "dec_w2", "bwd_dx", "bwd_dw", "bwd_router"]
 
 
 def header_entry_points() -> list[str]:
