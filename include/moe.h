@@ -338,14 +338,18 @@ MOE_API int moe_pack_backward(const moe_shape_t *shape, const moe_bf16_t *W13,
 /* Gradients of sum(out * dout) for the layer moe_forward computes (routing
  * recomputed with the same kernels, so it is identical). Requires
  * MOE_FLAG_BACKWARD in shape->flags (also for moe_workspace_size); rejects
- * MOE_FLAG_MXFP8 and MOE_FLAG_SIMT_FFN (MOE_ERR_INVALID_ARG); a shared expert
- * (d_ff_shared > 0) is not supported by this build (MOE_ERR_UNSUPPORTED).
+ * MOE_FLAG_MXFP8 and MOE_FLAG_SIMT_FFN (MOE_ERR_INVALID_ARG).
  *   x, Wg, bias, W13  as moe_forward; W13T, W2T as moe_pack_backward writes
+ *   W13_shared, W13T_shared, W2T_shared: with d_ff_shared > 0, the shared
+ *         expert's packed W13 [2*d_ff_shared, d] and its transposes (from
+ *         moe_pack_backward with E = 1, d_ff = d_ff_shared); else NULL
  *   dout  [T, d] fp32 in
  *   dx    [T, d] fp32 out: through the experts and through the router
  *   dW13  [E, 2*d_ff, d] fp32 out, in the packed W13 order (rows of dW1 and
  *         dW3 interleaved by 128 as in moe_pack_w13)
  *   dW2   [E, d, d_ff] fp32 out
+ *   dW13_shared [2*d_ff_shared, d], dW2_shared [d, d_ff_shared] fp32 out
+ *         (with d_ff_shared > 0; else NULL)
  *   dWg   [E, d] fp32 out; dbias [E] fp32 out (written even if bias is NULL)
  *   dlogits [T, E] fp32 out, or NULL
  * For a kept assignment (t, j) to expert e with weight w: dW2_e += w dout_t
@@ -358,9 +362,12 @@ MOE_API int moe_pack_backward(const moe_shape_t *shape, const moe_bf16_t *W13,
  * use fp32 atomic adds. */
 MOE_API int moe_backward(const moe_shape_t *shape, const moe_bf16_t *x, const moe_bf16_t *Wg,
                          const float *bias, const moe_bf16_t *W13, const moe_bf16_t *W13T,
-                         const moe_bf16_t *W2T, const float *dout, float *dx, float *dW13,
-                         float *dW2, float *dWg, float *dbias, float *dlogits, uint32_t *status,
-                         void *ws, size_t ws_bytes, moe_stream_t stream);
+                         const moe_bf16_t *W2T, const moe_bf16_t *W13_shared,
+                         const moe_bf16_t *W13T_shared, const moe_bf16_t *W2T_shared,
+                         const float *dout, float *dx, float *dW13, float *dW2,
+                         float *dW13_shared, float *dW2_shared, float *dWg, float *dbias,
+                         float *dlogits, uint32_t *status, void *ws, size_t ws_bytes,
+                         moe_stream_t stream);
 
 /* moe_permute without a workspace, for callers that cannot allocate device
  * memory: code running while a stream is captured in global capture mode

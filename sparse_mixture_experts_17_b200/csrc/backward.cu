@@ -277,7 +277,35 @@ __global__ void __launch_bounds__(256) k_router_bwd_dx(const float *__restrict__
     dx[(size_t)t * d + i] += acc;
 }
 
+// bf16 copy of dout (the shared expert's w * dout with w = 1), and the
+// single-group offsets {0, T} its weight gradients contract over.
+__global__ void __launch_bounds__(256) k_bwd_shared_prep(const float *__restrict__ dout,
+                                                         long long n4, int T,
+                                                         uint16_t *__restrict__ dout_bf,
+                                                         int32_t *__restrict__ offs)
+{
+    const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i == 0) {
+        offs[0] = 0;
+        offs[1] = T;
+    }
+    if (i >= n4)
+        return;
+    const float4 v = reinterpret_cast<const float4 *>(dout)[i];
+    reinterpret_cast<uint2 *>(dout_bf)[i] =
+        make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
+}
+
 // ---------------------------------------------------------------- host side
+int launch_bwd_shared_prep(const float *dout, int T, int d, uint16_t *dout_bf, int32_t *offs,
+                           cudaStream_t st)
+{
+    const long long n4 = (long long)T * d / 4;
+    k_bwd_shared_prep<<<(unsigned)((std::max(n4, 1LL) + 255) / 256), 256, 0, st>>>(dout, n4, T,
+                                                                                dout_bf, offs);
+    return launched();
+}
+
 int launch_transpose_batched(const uint16_t *src, int batch, int R, int C, uint16_t *dst,
                              cudaStream_t st)
 {

@@ -216,7 +216,7 @@ __device__ __forceinline__ void epilogue_tile(const TcArgs &p, uint32_t tb, long
         int t = 0;
         float wgt = 0.f;
         if (valid) {
-            t = p.perm_token[row];
+            t = p.perm_token ? p.perm_token[row] : (int)row;   // NULL: rows are tokens
             if (p.perm_w) {
                 wgt = p.perm_w[row];
             } else if (!p.slot_pos) {

@@ -54,6 +54,10 @@ struct WsLayout {
     // backward pass
     size_t GU, dYw, dGU, row_dot, pstart, kb0, nkb, mtk1_row0, mtk1_group, mtk2_row0,
         mtk2_group, dYwT, HT, dGUT, XpT, dl, dwg_part;
+    // backward of the shared expert
+    size_t s_GU, s_dout, s_dGU, s_rowdot, s_offs, s_pstart, s_kb0, s_nkb, s_mt1_row0,
+        s_mt1_group, s_mt2_row0, s_mt2_group, s_doutT, s_HT, s_dGUT, s_xT;
+    long long Tp;
     long long Np;                                        // padded rows of the transposes
     size_t total;
     int nchunks, max_mt, max_mt2;
@@ -205,6 +209,8 @@ int launch_group_ranges(const int32_t *offsets, int E, int32_t *pstart, int32_t 
 int launch_bwd_dyw(const moe_shape_t &s, const float *dout, const int32_t *slot_pos,
                    const float *topk_w, uint16_t *dyw, cudaStream_t st);
 size_t router_bwd_part_bytes(const moe_shape_t &s);
+int launch_bwd_shared_prep(const float *dout, int T, int d, uint16_t *dout_bf, int32_t *offs,
+                           cudaStream_t st);
 int launch_router_bwd(const moe_shape_t &s, const int32_t *idx, const float *topk_w,
                       const int32_t *slot_pos, const float *row_dot, const uint16_t *x,
                       const uint16_t *Wg, float *dl, float *part, float *dWg, float *dbias,

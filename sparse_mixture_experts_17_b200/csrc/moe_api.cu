@@ -172,6 +172,26 @@ WsLayout ws_layout(const moe_shape_t &s)
     L.XpT = take(bw ? s.d * Np * 2 : 0);
     L.dl = take(bw ? T * E * 4 : 0);
     L.dwg_part = take(bw ? router_bwd_part_bytes(s) : 0);
+    // shared expert: one group of all T rows
+    const bool bws = bw && dfs > 0;
+    const size_t Tp = bws ? ((T + 63) / 64) * 64 : 0;
+    L.Tp = (long long)Tp;
+    L.s_GU = take(bws ? T * 2 * dfs * 2 : 0);
+    L.s_dout = take(bws ? T * s.d * 2 : 0);
+    L.s_dGU = take(bws ? T * 2 * dfs * 2 : 0);
+    L.s_rowdot = take(bws ? T * 4 : 0);
+    L.s_offs = take(bws ? 2 * 4 : 0);
+    L.s_pstart = take(bws ? 2 * 4 : 0);
+    L.s_kb0 = take(bws ? 4 : 0);
+    L.s_nkb = take(bws ? 4 : 0);
+    L.s_mt1_row0 = take(bws ? (s.d / kBlockM) * 4 : 0);
+    L.s_mt1_group = take(bws ? (s.d / kBlockM) * 4 : 0);
+    L.s_mt2_row0 = take(bws ? (2 * dfs / kBlockM) * 4 : 0);
+    L.s_mt2_group = take(bws ? (2 * dfs / kBlockM) * 4 : 0);
+    L.s_doutT = take(bws ? s.d * Tp * 2 : 0);
+    L.s_HT = take(bws ? dfs * Tp * 2 : 0);
+    L.s_dGUT = take(bws ? 2 * dfs * Tp * 2 : 0);
+    L.s_xT = take(bws ? s.d * Tp * 2 : 0);
     L.scores = take(ec ? T * E * 4 : 0);
     L.ec_w = take(ec ? N * 4 : 0);
     L.x_stage = take((s.flags & MOE_FLAG_HOST_IO) ? T * s.d * 2 : 0);
@@ -680,11 +700,133 @@ static int forward_mx_impl(const moe_shape_t &s, const WsLayout &L, void *ws, co
 }
 
 // ---------------------------------------------------------------- backward pass
+// Backward of the shared expert ([DSK]: added with weight 1 on every token):
+// the routed path's kernels with identity tiles and one K-group of all T rows.
+static int backward_shared(const moe_shape_t &s, const WsLayout &L, void *ws, const uint16_t *x,
+                           const uint16_t *W13s, const uint16_t *W13sT, const uint16_t *W2sT,
+                           const float *dout, float *dx, float *dW13s, float *dW2s,
+                           uint32_t *status, cudaStream_t st)
+{
+    const int dfs = s.d_ff_shared;
+    const int mt = (s.T + kBlockM - 1) / kBlockM;
+    uint16_t *Hs = at<uint16_t>(ws, L.H_shared), *GUs = at<uint16_t>(ws, L.s_GU);
+    uint16_t *dout_bf = at<uint16_t>(ws, L.s_dout), *dGUs = at<uint16_t>(ws, L.s_dGU);
+    float *srow = at<float>(ws, L.s_rowdot);
+    int32_t *soffs = at<int32_t>(ws, L.s_offs);
+    int rc;
+    StageMark mark(MOE_STAGE_SHARED, st);
+    // recompute w1s/w3s keeping gate / up
+    GemmArgs g = gemm_base();
+    g.mode = EPI_SWIGLU_SAVE;
+    g.A = x;
+    g.a_rows = s.T;
+    g.B = W13s;
+    g.b_rows_total = 2LL * dfs;
+    g.K = s.d;
+    g.N = 2 * dfs;
+    g.b_rows_per_group = 2 * dfs;
+    g.num_mt_host = g.max_mt = mt;
+    g.rows_valid = s.T;
+    g.out = Hs;
+    g.ldo = dfs;
+    g.out2 = GUs;
+    g.status = status;
+    if ((rc = launch_gemm_tc(g, st)) || (rc = launch_bwd_shared_prep(dout, s.T, s.d, dout_bf, soffs, st)))
+        return rc;
+    if (cudaMemsetAsync(srow, 0, sizeof(float) * (size_t)s.T, st) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    // dh = dout W2s, through SwiGLU
+    g = gemm_base();
+    g.mode = EPI_SWIGLU_BWD;
+    g.A = dout_bf;
+    g.a_rows = s.T;
+    g.B = W2sT;
+    g.b_rows_total = dfs;
+    g.K = s.d;
+    g.N = dfs;
+    g.b_rows_per_group = dfs;
+    g.num_mt_host = g.max_mt = mt;
+    g.rows_valid = s.T;
+    g.out = dGUs;
+    g.ldo = dfs;
+    g.gu = GUs;
+    g.row_dot = srow;
+    g.status = status;
+    if ((rc = launch_gemm_tc(g, st)))
+        return rc;
+    // dx += [dg | du] W13s (rows are tokens)
+    g = gemm_base();
+    g.mode = EPI_COMBINE;
+    g.A = dGUs;
+    g.a_rows = s.T;
+    g.B = W13sT;
+    g.b_rows_total = s.d;
+    g.K = 2 * dfs;
+    g.N = s.d;
+    g.b_rows_per_group = s.d;
+    g.num_mt_host = g.max_mt = mt;
+    g.rows_valid = s.T;
+    g.out = dx;
+    g.ldo = s.d;
+    g.status = status;
+    if ((rc = launch_gemm_tc(g, st)))
+        return rc;
+    // dW2s = dout^T h_s, dW13s = [dg | du]^T x: one group of all T rows
+    int32_t *pst = at<int32_t>(ws, L.s_pstart), *kb0 = at<int32_t>(ws, L.s_kb0);
+    int32_t *nkb = at<int32_t>(ws, L.s_nkb);
+    if ((rc = launch_group_ranges(soffs, 1, pst, kb0, nkb, s.d, at<int32_t>(ws, L.s_mt1_row0),
+                                  at<int32_t>(ws, L.s_mt1_group), 2 * dfs,
+                                  at<int32_t>(ws, L.s_mt2_row0), at<int32_t>(ws, L.s_mt2_group),
+                                  st)))
+        return rc;
+    const long long Tp = L.Tp;
+    uint16_t *doutT = at<uint16_t>(ws, L.s_doutT), *HT = at<uint16_t>(ws, L.s_HT);
+    uint16_t *dGUT = at<uint16_t>(ws, L.s_dGUT), *xT = at<uint16_t>(ws, L.s_xT);
+    if ((rc = launch_transpose_grouped(dout_bf, s.T, s.d, soffs, pst, 1, doutT, Tp, st)) ||
+        (rc = launch_transpose_grouped(Hs, s.T, dfs, soffs, pst, 1, HT, Tp, st)) ||
+        (rc = launch_transpose_grouped(dGUs, s.T, 2 * dfs, soffs, pst, 1, dGUT, Tp, st)) ||
+        (rc = launch_transpose_grouped(x, s.T, s.d, soffs, pst, 1, xT, Tp, st)))
+        return rc;
+    g = gemm_base();
+    g.mode = EPI_STORE_F32;
+    g.A = doutT;
+    g.a_rows = s.d;
+    g.B = HT;
+    g.b_rows_total = dfs;
+    g.K = (int)Tp;
+    g.N = dfs;
+    g.b_rows_per_group = 0;
+    g.mt_row0 = at<int32_t>(ws, L.s_mt1_row0);
+    g.mt_group = at<int32_t>(ws, L.s_mt1_group);
+    g.num_mt_host = g.max_mt = s.d / kBlockM;
+    g.rows_valid = s.d;
+    g.grp_kb0 = kb0;
+    g.grp_nkb = nkb;
+    g.out = dW2s;
+    g.ldo = dfs;
+    g.status = status;
+    if ((rc = launch_gemm_tc(g, st)))
+        return rc;
+    g.A = dGUT;
+    g.a_rows = 2LL * dfs;
+    g.B = xT;
+    g.b_rows_total = s.d;
+    g.N = s.d;
+    g.mt_row0 = at<int32_t>(ws, L.s_mt2_row0);
+    g.mt_group = at<int32_t>(ws, L.s_mt2_group);
+    g.num_mt_host = g.max_mt = 2 * dfs / kBlockM;
+    g.rows_valid = 2LL * dfs;
+    g.out = dW13s;
+    g.ldo = s.d;
+    return launch_gemm_tc(g, st);
+}
+
 static int backward_impl(const moe_shape_t &s, const WsLayout &L, void *ws, const uint16_t *x,
                          const uint16_t *Wg, const float *bias, const uint16_t *W13,
-                         const uint16_t *W13T, const uint16_t *W2T, const float *dout, float *dx,
-                         float *dW13, float *dW2, float *dWg, float *dbias, float *dlogits,
-                         uint32_t *status, cudaStream_t st)
+                         const uint16_t *W13T, const uint16_t *W2T, const uint16_t *W13s,
+                         const uint16_t *W13sT, const uint16_t *W2sT, const float *dout, float *dx,
+                         float *dW13, float *dW2, float *dW13s, float *dW2s, float *dWg,
+                         float *dbias, float *dlogits, uint32_t *status, cudaStream_t st)
 {
     const long long N = (long long)s.T * s.k;
     float *logits = at<float>(ws, L.logits);
@@ -848,7 +990,10 @@ static int backward_impl(const moe_shape_t &s, const WsLayout &L, void *ws, cons
     if ((rc = launch_gemm_tc(g, st)))
         return rc;
     mdw.end();
-    // router: dl, dWg, dbias, and dx += dl Wg
+    if (s.d_ff_shared > 0 &&
+        (rc = backward_shared(s, L, ws, x, W13s, W13sT, W2sT, dout, dx, dW13s, dW2s, status, st)))
+        return rc;
+    // router: dl, dWg, dbias, and dx += dl Wg (after every scatter-add into dx)
     StageMark m(MOE_STAGE_BWD_ROUTER, st);
     return launch_router_bwd(s, idx, w, slot_pos, row_dot, x, Wg, dl, at<float>(ws, L.dwg_part),
                              dWg, dbias, dx, st);
@@ -1396,7 +1541,9 @@ int moe_pack_backward(const moe_shape_t *shape, const moe_bf16_t *W13, const moe
 
 int moe_backward(const moe_shape_t *shape, const moe_bf16_t *x, const moe_bf16_t *Wg,
                  const float *bias, const moe_bf16_t *W13, const moe_bf16_t *W13T,
-                 const moe_bf16_t *W2T, const float *dout, float *dx, float *dW13, float *dW2,
+                 const moe_bf16_t *W2T, const moe_bf16_t *W13_shared,
+                 const moe_bf16_t *W13T_shared, const moe_bf16_t *W2T_shared, const float *dout,
+                 float *dx, float *dW13, float *dW2, float *dW13_shared, float *dW2_shared,
                  float *dWg, float *dbias, float *dlogits, uint32_t *status, void *ws,
                  size_t ws_bytes, moe_stream_t stream)
 {
@@ -1408,16 +1555,20 @@ int moe_backward(const moe_shape_t *shape, const moe_bf16_t *x, const moe_bf16_t
     const moe_shape_t &s = *shape;
     if (!(s.flags & MOE_FLAG_BACKWARD) || (s.flags & (MOE_FLAG_MXFP8 | MOE_FLAG_SIMT_FFN)))
         return MOE_ERR_INVALID_ARG;
-    if (s.d_ff_shared > 0)
-        return MOE_ERR_UNSUPPORTED;
     if (!x || !Wg || !W13 || !W13T || !W2T || !dout || !dx || !dW13 || !dW2 || !dWg || !dbias ||
         !al16(x) || !al16(Wg) || !al16(W13) || !al16(W13T) || !al16(W2T) || !al16(dout) ||
         !al16(dx) || !al16(dW13) || !al16(dW2))
         return MOE_ERR_INVALID_ARG;
+    if (s.d_ff_shared > 0 &&
+        (!W13_shared || !W13T_shared || !W2T_shared || !dW13_shared || !dW2_shared ||
+         !al16(W13_shared) || !al16(W13T_shared) || !al16(W2T_shared) || !al16(dW13_shared) ||
+         !al16(dW2_shared)))
+        return MOE_ERR_INVALID_ARG;
     WsLayout L;
     if ((rc = check_ws(s, ws, ws_bytes, L)))
         return rc;
-    return backward_impl(s, L, ws, x, Wg, bias, W13, W13T, W2T, dout, dx, dW13, dW2, dWg, dbias,
+    return backward_impl(s, L, ws, x, Wg, bias, W13, W13T, W2T, W13_shared, W13T_shared,
+                         W2T_shared, dout, dx, dW13, dW2, dW13_shared, dW2_shared, dWg, dbias,
                          dlogits, status, reinterpret_cast<cudaStream_t>(stream));
 }
 

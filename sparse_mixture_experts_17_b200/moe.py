@@ -88,7 +88,7 @@ _SIGS = {
     "moe_quantize_experts_mxfp8": ([_SHP, _P, _P, _P, _P, _P, _P, _P, _P], ctypes.c_int),
     "moe_forward_mxfp8": ([_SHP] + [_P] * 16 + [_SZ, _P], ctypes.c_int),
     "moe_pack_backward": ([_SHP, _P, _P, _P, _P, _P], ctypes.c_int),
-    "moe_backward": ([_SHP] + [_P] * 15 + [_SZ, _P], ctypes.c_int),
+    "moe_backward": ([_SHP] + [_P] * 20 + [_SZ, _P], ctypes.c_int),
     "moe_route_expert_choice": ([_SHP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P], ctypes.c_int),
     "moe_forward_expert_choice": ([_SHP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P],
                                   ctypes.c_int),
@@ -357,9 +357,10 @@ def moe_pack_backward(shape, W13, W2, stream=None):
 
 
 def moe_backward(shape, x, Wg, bias, W13, W13T, W2T, dout, status, ws, want_dlogits=False,
-                 stream=None) -> dict:
-    """Gradients of sum(out * dout): dict(dx, dW13 (packed order), dW2, dWg, dbias[, dlogits])."""
-    T, d, d_ff, E = shape.T, shape.d, shape.d_ff, shape.E
+                 shared=None, stream=None) -> dict:
+    """Gradients of sum(out * dout): dict(dx, dW13 (packed order), dW2, dWg, dbias[, dlogits]
+    [, dW13s, dW2s]). shared = (W13s [2 dfs, d], W13sT, W2sT) when d_ff_shared > 0."""
+    T, d, d_ff, E, dfs = shape.T, shape.d, shape.d_ff, shape.E, shape.d_ff_shared
     dev = x.device
     g = dict(dx=torch.empty(T, d, dtype=F32, device=dev),
              dW13=torch.empty(E, 2 * d_ff, d, dtype=F32, device=dev),
@@ -368,13 +369,20 @@ def moe_backward(shape, x, Wg, bias, W13, W13T, W2T, dout, status, ws, want_dlog
              dbias=torch.empty(E, dtype=F32, device=dev))
     if want_dlogits:
         g["dlogits"] = torch.empty(T, E, dtype=F32, device=dev)
+    W13s = W13sT = W2sT = None
+    if dfs:
+        W13s, W13sT, W2sT = shared
+        g["dW13s"] = torch.empty(2 * dfs, d, dtype=F32, device=dev)
+        g["dW2s"] = torch.empty(d, dfs, dtype=F32, device=dev)
     _check("moe_backward", lib().moe_backward(
         ctypes.byref(shape), _ptr(x, BF16, "x"), _ptr(Wg, BF16, "Wg"), _ptr(bias, F32, "bias"),
         _ptr(W13, BF16, "W13"), _ptr(W13T, BF16, "W13T"), _ptr(W2T, BF16, "W2T"),
+        _ptr(W13s, BF16, "W13s"), _ptr(W13sT, BF16, "W13sT"), _ptr(W2sT, BF16, "W2sT"),
         _ptr(dout, F32, "dout"), _ptr(g["dx"], F32, "dx"), _ptr(g["dW13"], F32, "dW13"),
-        _ptr(g["dW2"], F32, "dW2"), _ptr(g["dWg"], F32, "dWg"), _ptr(g["dbias"], F32, "dbias"),
-        _ptr(g.get("dlogits"), F32, "dlogits"), _ptr(status, U32, "status"), _ptr(ws, name="ws"),
-        ws.numel(), _stream(stream)))
+        _ptr(g["dW2"], F32, "dW2"), _ptr(g.get("dW13s"), F32, "dW13s"),
+        _ptr(g.get("dW2s"), F32, "dW2s"), _ptr(g["dWg"], F32, "dWg"),
+        _ptr(g["dbias"], F32, "dbias"), _ptr(g.get("dlogits"), F32, "dlogits"),
+        _ptr(status, U32, "status"), _ptr(ws, name="ws"), ws.numel(), _stream(stream)))
     return g
 
 

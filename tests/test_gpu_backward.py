@@ -111,14 +111,34 @@ def test_backward_weight_grads_repeatable():
         assert torch.equal(a[key], b[key]), key
 
 
-def test_backward_rejects_shared_expert():
-    w = small_workload("sh", 64, 128, 128, 4, 2, d_ff_shared=128)
-    inp = I.make_inputs(w, "cuda", seed=1)
+@pytest.mark.parametrize("T,d,d_ff,E,k,dfs", [(300, 256, 256, 8, 2, 256), (90, 512, 128, 16, 4, 384)])
+def test_backward_shared_expert(T, d, d_ff, E, k, dfs):
+    """With a shared expert ([DSK]: weight 1 on every token): its gradients and
+    its share of dx against the oracle."""
+    w = small_workload("bsh", T, d, d_ff, E, k, d_ff_shared=dfs, zipf_s=1.0)
+    inp = I.make_inputs(w, "cuda", seed=T + dfs)
     s = M.shape_of(w, M.MOE_FLAG_BACKWARD)
     ws = M.alloc_workspace(s)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
     W13 = M.moe_pack_w13(s, inp["W1"], inp["W3"])
     W13T, W2T = M.moe_pack_backward(s, W13, inp["W2"])
-    with pytest.raises(M.MoeError) as ei:
-        M.moe_backward(s, inp["x"], inp["wg"], None, W13, W13T, W2T,
-                       torch.zeros(64, 128, device="cuda"), None, ws)
-    assert ei.value.code == M.MOE_ERR_UNSUPPORTED
+    ss = M.make_shape(T, d, dfs, 1, 1)
+    W13s = M.moe_pack_w13(ss, inp["W1s"][None].contiguous(), inp["W3s"][None].contiguous())
+    W13sT, W2sT = M.moe_pack_backward(ss, W13s, inp["W2s"][None].contiguous())
+    dout = torch.randn(T, d, generator=torch.Generator("cuda").manual_seed(3), device="cuda")
+    grads = M.moe_backward(s, inp["x"], inp["wg"], inp["bias"], W13, W13T, W2T, dout, status, ws,
+                           shared=(W13s[0], W13sT[0], W2sT[0]))
+    b = Buffers(w)
+    M.moe_route(b.shape, inp["x"], inp["wg"], inp["bias"], b.logits, b.idx, b.w, b.status, b.ws)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    idx_o, w_o = O.route(b.logits.cpu().numpy(), k)
+    disp = O.dispatch(idx_o, E, 0)
+    ref = O.moe_backward(I.oracle_arrays(inp), idx_o, w_o, disp["slot_pos"], dout.cpu().numpy())
+    dW1s, dW3s = _unpack13(grads["dW13s"].cpu().numpy()[None], dfs)
+    errs = {"dx": _rel(grads["dx"], ref["dx"]), "dW1s": _rel(dW1s[0], ref["dW1s"]),
+            "dW3s": _rel(dW3s[0], ref["dW3s"]), "dW2s": _rel(grads["dW2s"], ref["dW2s"]),
+            "dW2": _rel(grads["dW2"], ref["dW2"]), "dWg": _rel(grads["dWg"], ref["dWg"])}
+    for key in ("dx", "dW1s", "dW3s", "dW2s", "dW2"):
+        assert errs[key] <= EXPERT_REL, errs
+    assert errs["dWg"] <= ROUTER_REL, errs
