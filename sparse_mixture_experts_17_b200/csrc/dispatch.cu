@@ -9,6 +9,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "tiles.cuh"
 #include "topk.cuh"
 
 namespace moe {
@@ -156,70 +157,6 @@ int launch_topk(const moe_shape_t &s, const float *logits, int32_t *idx, float *
     return launched();
 }
 
-// ---------------------------------------------------------------- block scan helper
-// Exclusive scan of one int per thread over a 256-thread block.
-__device__ __forceinline__ int block_excl_scan_256(int v, int *s_warp, int *total)
-{
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    int inc = v;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-        const int o = __shfl_up_sync(kFullMask, inc, off);
-        if (lane >= off)
-            inc += o;
-    }
-    if (lane == 31)
-        s_warp[warp] = inc;
-    __syncthreads();
-    if (warp == 0) {
-        int wv = (lane < 8) ? s_warp[lane] : 0;
-        int winc = wv;
-#pragma unroll
-        for (int off = 1; off < 8; off <<= 1) {
-            const int o = __shfl_up_sync(kFullMask, winc, off);
-            if (lane >= off)
-                winc += o;
-        }
-        if (lane < 8)
-            s_warp[8 + lane] = winc - wv;
-        if (lane == 7)
-            s_warp[16] = winc;
-    }
-    __syncthreads();
-    const int r = s_warp[8 + warp] + inc - v;
-    *total = s_warp[16];
-    __syncthreads();
-    return r;
-}
-
-// Writes the grouped-GEMM m-tile list for kept counts in s_kept[E]: expert e
-// contributes ceil(kept/tile_m) tiles starting at rows offsets[e] + tile_m i.
-// tile_start (may be NULL) receives each expert's first tile index.
-__device__ void build_tiles(const int *s_kept, const int32_t *offsets_smem_or_global, int E,
-                            int tile_m, int32_t *mt_row0, int32_t *mt_group, int32_t *num_mt,
-                            int *s_warp, int32_t *tile_start = nullptr)
-{
-    const int tid = threadIdx.x;
-    const int e = tid;
-    const int nt = (e < E) ? (s_kept[e] + tile_m - 1) / tile_m : 0;
-    int total;
-    const int start = block_excl_scan_256(nt, s_warp, &total);
-    if (e < E && tile_start)
-        tile_start[e] = start;
-    if (e < E) {
-        const int base = offsets_smem_or_global[e];
-        // a last tile of <= 64 rows is marked for the M = 64 MMA (128-row lists only)
-        const int rem = s_kept[e] - (nt - 1) * tile_m;
-        for (int i = 0; i < nt; ++i) {
-            mt_row0[start + i] = base + i * tile_m;
-            const bool half = (tile_m == kBlockM) && (i == nt - 1) && rem <= 64;
-            mt_group[start + i] = e | (half ? kHalfTileBit : 0);
-        }
-    }
-    if (tid == 0)
-        *num_mt = total;
-}
-
 // ---------------------------------------------------------------- histogram + scan
 // One CTA per chunk of 256 tokens (thread = token). For each slot j the warp
 // groups equal expert ids with __match_any_sync; the group leader ORs the
@@ -325,43 +262,9 @@ __global__ void __launch_bounds__(256) k_hist_scan(
     if (!s_last)
         return;
     __threadfence();
-    const int nchunks = gridDim.x;
-    for (int e = tid; e < MOE_MAX_E; e += 256) {
-        int kept = 0;
-        if (e < E) {
-            // exclusive prefix in rank order: chunks (row-major), or slots then
-            // chunks (slot-major)
-            int run = 0;
-            const int nj = slot_major ? k : 1;
-            for (int j = 0; j < nj; ++j)
-                for (int c = 0; c < nchunks; ++c) {
-                    const size_t i = ((size_t)c * nj + j) * E + e;
-                    const int v = __ldcg(&chunk_counts[i]);
-                    __stcg(&chunk_counts[i], run);
-                    run += v;
-                }
-            counts[e] = run;
-            kept = (C > 0 && run > C) ? C : run;
-        }
-        s_kept[e] = kept;
-    }
-    __syncthreads();
-    int total;
-    const int ex = block_excl_scan_256(tid < E ? s_kept[tid] : 0, s_warp, &total);
-    if (tid < E) {
-        offsets[tid] = ex;
-        s_off[tid] = ex;
-    }
-    if (tid == 0) {
-        offsets[E] = total;
-        *n_kept = total;
-    }
-    __syncthreads();
-    build_tiles(s_kept, s_off, E, kBlockM, mt_row0, mt_group, num_mt, s_warp, tile_start);
-    if (mt2_row0)
-        build_tiles(s_kept, s_off, E, 2 * kBlockM, mt2_row0, mt2_group, num_mt2, s_warp);
-    if (tid == 0)
-        *counter = 0;
+    hist_finish(chunk_counts, gridDim.x, slot_major ? k : 1, E, C, counts, offsets, n_kept,
+                mt_row0, mt_group, num_mt, mt2_row0, mt2_group, num_mt2, tile_start, counter,
+                s_kept, s_off, s_warp);
 }
 
 int launch_hist_scan(const moe_shape_t &s, const int32_t *idx, int32_t *chunk_counts,
@@ -382,13 +285,14 @@ int launch_hist_scan(const moe_shape_t &s, const int32_t *idx, int32_t *chunk_co
 
 // ---------------------------------------------------------------- permutation
 // One warp per token: lane j < k resolves slot j's permuted row
-// (offsets[e] + chunk base + rank within the chunk, -1 past the capacity;
+// (offsets[e] + chunk base + rank within the chunk of chunk_tokens tokens,
+// -1 past the capacity;
 // with slot-major priority the base is per (chunk, slot));
 // then the warp copies x[t] once into every kept row with 16-B loads/stores
 // and, when asked, zeroes out[t] (the fused combine accumulates into it).
 __global__ void __launch_bounds__(256) k_permute(
     const int32_t *__restrict__ idx, int T, int E, int k, int C, int slot_major, int d,
-    const int32_t *__restrict__ chunk_base, const int32_t *__restrict__ rank_local,
+    int chunk_tokens, const int32_t *__restrict__ chunk_base, const int32_t *__restrict__ rank_local,
     const int32_t *__restrict__ offsets, const uint4 *__restrict__ x, int32_t *__restrict__ slot_pos,
     int32_t *__restrict__ perm_token, uint4 *__restrict__ x_perm, float4 *__restrict__ out_zero)
 {
@@ -401,8 +305,8 @@ __global__ void __launch_bounds__(256) k_permute(
         const int e = idx[(size_t)t * k + lane];
         const int rl = rank_local[(size_t)t * k + lane];
         if (e >= 0 && e < E && rl >= 0) {
-            const size_t row = slot_major ? (size_t)(t / kChunkTokens) * k + lane
-                                          : (size_t)(t / kChunkTokens);
+            const size_t row = slot_major ? (size_t)(t / chunk_tokens) * k + lane
+                                          : (size_t)(t / chunk_tokens);
             const int r = chunk_base[row * E + e] + rl;
             if (C <= 0 || r < C)
                 pos = offsets[e] + r;
@@ -451,12 +355,13 @@ __global__ void __launch_bounds__(256) k_permute(
 int launch_permute(const moe_shape_t &s, const int32_t *idx, const int32_t *chunk_base,
                    const int32_t *rank_local, const int32_t *offsets, const uint16_t *x,
                    int32_t *slot_pos, int32_t *perm_token, uint16_t *x_perm, float *out_zero,
-                   cudaStream_t st)
+                   cudaStream_t st, int chunk_tokens)
 {
     if (s.T == 0)
         return MOE_OK;
     k_permute<<<(s.T + 7) / 8, 256, 0, st>>>(
-        idx, s.T, s.E, s.k, s.capacity, slot_major(s), s.d, chunk_base, rank_local, offsets,
+        idx, s.T, s.E, s.k, s.capacity, slot_major(s), s.d, chunk_tokens, chunk_base, rank_local,
+        offsets,
         reinterpret_cast<const uint4 *>(x), slot_pos, perm_token, reinterpret_cast<uint4 *>(x_perm),
         reinterpret_cast<float4 *>(out_zero));
     return launched();

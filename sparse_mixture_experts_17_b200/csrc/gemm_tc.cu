@@ -30,6 +30,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "tiles.cuh"
 
 namespace moe {
 
@@ -77,7 +78,67 @@ struct TcArgs {
     const int32_t *grp_kb0;
     const int32_t *grp_nkb;
     long long out_group_stride;
+    int32_t *hist_chunk, *hist_rank, *hist_counter, *hist_counts, *hist_offsets, *hist_n_kept;
+    int32_t *hist_mt_row0, *hist_mt_group, *hist_num_mt, *hist_mt2_row0, *hist_mt2_group,
+        *hist_num_mt2;
+    int capacity;
 };
+
+// Shared memory of the histogram folded into the router (E <= 64): per-warp
+// lane masks and prefixes of one 128-token tile, then the last CTA's scan.
+struct RouterHistSmem {
+    uint32_t mask[4][64];
+    int wpre[4][64];
+    int kept[MOE_MAX_E];
+    int off[MOE_MAX_E + 1];
+    int warp[17];
+    int last;
+};
+
+__device__ __forceinline__ void epi_barrier()   // the 4 epilogue warps (128 threads)
+{
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+}
+
+// Histogram of one 128-token m-tile (the router's rows), as the histogram
+// kernel computes it for its chunks: lane masks per slot with match_any
+// (leaders are unique per round; rounds ordered by __syncwarp), per-expert
+// prefixes over the 4 warps in tile-row order, the tile's counts, and each
+// kept slot's rank among the earlier tokens of the tile that chose the same
+// expert. All 128 epilogue threads call it once per tile.
+__device__ __forceinline__ void router_hist_tile(const TcArgs &p, RouterHistSmem &H, long long row,
+                                                 bool valid, int q, int lane, int m_idx)
+{
+    const int E = p.n_valid, k = p.k;
+    H.mask[q][lane] = 0u;
+    H.mask[q][lane + 32] = 0u;
+    __syncwarp();
+    for (int j = 0; j < k; ++j) {
+        const int e = valid ? p.route_idx[row * k + j] : -1;
+        const uint32_t g = __match_any_sync(kFullMask, e);
+        if (e >= 0 && lane == __ffs(g) - 1)
+            H.mask[q][e] |= g;
+        __syncwarp();
+    }
+    epi_barrier();
+    const int tix = q * 32 + lane;
+    if (tix < E) {
+        int run = 0;
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+            H.wpre[w][tix] = run;
+            run += __popc(H.mask[w][tix]);
+        }
+        p.hist_chunk[(long long)m_idx * E + tix] = run;
+    }
+    epi_barrier();
+    if (valid)
+        for (int j = 0; j < k; ++j) {
+            const int e = p.route_idx[row * k + j];
+            p.hist_rank[row * k + j] = H.wpre[q][e] + __popc(H.mask[q][e] & lanemask_lt());
+        }
+    epi_barrier();
+}
 
 template <int BN>
 struct TcCfg {
@@ -458,17 +519,27 @@ __global__ void __launch_bounds__(192, 1)
             const bool half = (gword & kHalfTileBit) != 0;
             const long long row_end = p.seg_offsets ? p.seg_offsets[grp + 1] : p.rows_valid;
             const uint32_t b = local & 1u, aph = (local >> 1) & 1u;
-            if (!mbar_wait(&tfull[b], aph, abort_flag, p.status))
+            const bool got = mbar_wait(&tfull[b], aph, abort_flag, p.status);
+            // the folded histogram's named barriers need every epilogue warp on
+            // every tile, so a warp whose wait gave up keeps going without work
+            if (!got && !(MODE == EPI_ROUTER_TOPK && p.hist_chunk))
                 break;
             tc_fence_after();
             // M = 128: tile row q*32 + lane sits in lane q*32 + lane. M = 64: tile
             // row 16 q + l sits in lane 32 q + l (l < 16); lanes 16..31 hold nothing.
             const long long row = row0 + (half ? q * 16 + lane : q * 32 + lane);
-            const bool valid = (!half || lane < 16) && row < row_end;
+            const bool valid = got && (!half || lane < 16) && row < row_end;
             const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + b * BN;
             const bool empty_k = p.grp_kb0 && p.grp_nkb[grp] == 0;
 
-            epilogue_tile<BN, MODE>(p, tb, row, valid, n_idx, grp, empty_k);
+            if (got)
+                epilogue_tile<BN, MODE>(p, tb, row, valid, n_idx, grp, empty_k);
+            if constexpr (MODE == EPI_ROUTER_TOPK) {
+                if (p.hist_chunk)
+                    router_hist_tile(p, *reinterpret_cast<RouterHistSmem *>(
+                                            reinterpret_cast<uint8_t *>(full) + C::BAR_BYTES),
+                                     row, valid, q, lane, m_idx);
+            }
             tc_fence_before();
             __syncwarp();
             if (lane == 0)
@@ -481,6 +552,24 @@ __global__ void __launch_bounds__(192, 1)
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem_base, C::TMEM_COLS);
+    }
+    if constexpr (MODE == EPI_ROUTER_TOPK) {
+        // the folded histogram: the last CTA to finish scans every tile's counts
+        if (p.hist_chunk) {
+            RouterHistSmem &H = *reinterpret_cast<RouterHistSmem *>(
+                reinterpret_cast<uint8_t *>(full) + C::BAR_BYTES);
+            __threadfence();
+            if (threadIdx.x == 0)
+                H.last = (atomicAdd(p.hist_counter, 1) == (int)gridDim.x - 1);
+            __syncthreads();
+            if (H.last) {
+                __threadfence();
+                hist_finish(p.hist_chunk, num_mt, 1, p.n_valid, p.capacity, p.hist_counts,
+                            p.hist_offsets, p.hist_n_kept, p.hist_mt_row0, p.hist_mt_group,
+                            p.hist_num_mt, p.hist_mt2_row0, p.hist_mt2_group, p.hist_num_mt2,
+                            nullptr, p.hist_counter, H.kept, H.off, H.warp);
+            }
+        }
     }
 }
 
@@ -736,13 +825,28 @@ static int launch_tc_impl(const GemmArgs &g, cudaStream_t st)
     p.grp_kb0 = g.grp_kb0;
     p.grp_nkb = g.grp_nkb;
     p.out_group_stride = g.out_group_stride;
+    p.hist_chunk = g.hist_chunk;
+    p.hist_rank = g.hist_rank;
+    p.hist_counter = g.hist_counter;
+    p.hist_counts = g.hist_counts;
+    p.hist_offsets = g.hist_offsets;
+    p.hist_n_kept = g.hist_n_kept;
+    p.hist_mt_row0 = g.hist_mt_row0;
+    p.hist_mt_group = g.hist_mt_group;
+    p.hist_num_mt = g.hist_num_mt;
+    p.hist_mt2_row0 = g.hist_mt2_row0;
+    p.hist_mt2_group = g.hist_mt2_group;
+    p.hist_num_mt2 = g.hist_num_mt2;
+    p.capacity = g.capacity;
 
+    // the router with the folded histogram also needs its tile-histogram area
+    constexpr int SMEM = C::SMEM_BYTES + (MODE == EPI_ROUTER_TOPK ? (int)sizeof(RouterHistSmem) : 0);
     static int attr_done[64] = {0};
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev >= 0 && dev < 64 && !attr_done[dev]) {
         if (cudaFuncSetAttribute(k_gemm_tc<BN, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 C::SMEM_BYTES) != cudaSuccess)
+                                 SMEM) != cudaSuccess)
             return MOE_ERR_CUDA;
         attr_done[dev] = 1;
     }
@@ -751,7 +855,7 @@ static int launch_tc_impl(const GemmArgs &g, cudaStream_t st)
     if (tiles <= 0)
         return MOE_OK;
     const int grid = (int)std::min<long long>(tiles, num_sms());
-    k_gemm_tc<BN, MODE><<<grid, 192, C::SMEM_BYTES, st>>>(tA, tB, p);
+    k_gemm_tc<BN, MODE><<<grid, 192, SMEM, st>>>(tA, tB, p);
     return launched();
 }
 

@@ -79,7 +79,7 @@ int launch_hist_scan(const moe_shape_t &s, const int32_t *idx, int32_t *chunk_co
 int launch_permute(const moe_shape_t &s, const int32_t *idx, const int32_t *chunk_base,
                    const int32_t *rank_local, const int32_t *offsets, const uint16_t *x,
                    int32_t *slot_pos, int32_t *perm_token, uint16_t *x_perm, float *out_zero,
-                   cudaStream_t st);
+                   cudaStream_t st, int chunk_tokens = kChunkTokens);
 int launch_tiles_from_offsets(const moe_shape_t &s, const int32_t *offsets, int32_t *mt_row0,
                               int32_t *mt_group, int32_t *num_mt, int32_t *mt2_row0,
                               int32_t *mt2_group, int32_t *num_mt2, cudaStream_t st);
@@ -154,6 +154,12 @@ struct GemmArgs {
     const int32_t *grp_kb0;
     const int32_t *grp_nkb;
     long long out_group_stride;
+    // EPI_ROUTER_TOPK with the histogram folded in (hist_chunk set): per
+    // 128-token m-tile expert counts and ranks, then the last CTA's scan
+    int32_t *hist_chunk, *hist_rank, *hist_counter, *hist_counts, *hist_offsets, *hist_n_kept;
+    int32_t *hist_mt_row0, *hist_mt_group, *hist_num_mt, *hist_mt2_row0, *hist_mt2_group,
+        *hist_num_mt2;
+    int capacity;
 };
 
 int launch_gemm_tc(const GemmArgs &g, cudaStream_t st);

@@ -119,7 +119,10 @@ WsLayout ws_layout(const moe_shape_t &s)
     L.n_kept = take(4);
     L.counter = take(4);
     L.num_mt = take(4);
-    L.chunk_counts = take(chunk_count_rows(s, L.nchunks) * E * 4);
+    // 256-token chunks of the histogram kernel, or the router's 128-token
+    // m-tiles when it folds the histogram in
+    L.chunk_counts = take(std::max(chunk_count_rows(s, L.nchunks), (size_t)((T + kBlockM - 1) / kBlockM)) *
+                          E * 4);
     L.rank_local = take(N * 4);
     L.slot_pos = take(N * 4);
     L.perm_token = take(N * 4);
@@ -414,6 +417,62 @@ static int router_topk(const moe_shape_t &s, const uint16_t *x, const uint16_t *
     return launch_gemm_tc(g, st);
 }
 
+// The prefill router with the top-k and the expert histogram in its
+// epilogue: per 128-token m-tile counts and ranks, then the last CTA's scan
+// into counts, offsets and the grouped GEMMs' tile lists (token-major
+// priority only; slot-major priority needs every slot's counts first).
+static bool router_hist_fusable(const moe_shape_t &s)
+{
+    return router_topk_fusable(s) && !slot_major(s);
+}
+
+struct HistOut {
+    int32_t *chunk, *rank, *counts, *offsets, *n_kept, *mt_row0, *mt_group, *num_mt, *mt2_row0,
+        *mt2_group, *num_mt2;
+};
+
+static int router_topk_hist(const moe_shape_t &s, const uint16_t *x, const uint16_t *Wg,
+                            const float *bias, float *logits, int32_t *idx, float *w,
+                            int32_t *counter, const HistOut &h, uint32_t *status, cudaStream_t st)
+{
+    GemmArgs g = gemm_base();
+    g.mode = EPI_ROUTER_TOPK;
+    g.A = x;
+    g.a_rows = s.T;
+    g.B = Wg;
+    g.b_rows_total = s.E;
+    g.K = s.d;
+    g.N = s.E;
+    g.num_mt_host = (s.T + kBlockM - 1) / kBlockM;
+    g.max_mt = g.num_mt_host;
+    g.rows_valid = s.T;
+    g.out = logits;
+    g.ldo = s.E;
+    g.bias = bias;
+    g.n_valid = s.E;
+    g.k = s.k;
+    g.route_idx = idx;
+    g.route_w = w;
+    g.status = status;
+    g.hist_chunk = h.chunk;
+    g.hist_rank = h.rank;
+    g.hist_counter = counter;
+    g.hist_counts = h.counts;
+    g.hist_offsets = h.offsets;
+    g.hist_n_kept = h.n_kept;
+    g.hist_mt_row0 = h.mt_row0;
+    g.hist_mt_group = h.mt_group;
+    g.hist_num_mt = h.num_mt;
+    g.hist_mt2_row0 = h.mt2_row0;
+    g.hist_mt2_group = h.mt2_group;
+    g.hist_num_mt2 = h.num_mt2;
+    g.capacity = s.capacity;
+    // the ticket starts at zero whatever an earlier, aborted call left in it
+    if (cudaMemsetAsync(counter, 0, sizeof(int32_t), st) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    return launch_gemm_tc(g, st);
+}
+
 // Router, softmax / top-k / renormalisation: one launch when a fused form
 // applies (single-CTA for small T and W_g; the GEMM epilogue for E <= 64).
 static int route_tokens(const moe_shape_t &s, const uint16_t *x, const uint16_t *Wg,
@@ -454,7 +513,20 @@ static int forward_impl(const moe_shape_t &s, const WsLayout &L, void *ws, const
         return MOE_ERR_UNSUPPORTED;
     const bool decode = force_dec || (!force_pre && s.T <= MOE_DECODE_DEFAULT_T);
     int32_t *counter = at<int32_t>(ws, L.counter);
-    int rc = route_tokens(s, x, Wg, bias, logits, idx, w, counter, status, st);
+    const HistOut hist = {at<int32_t>(ws, L.chunk_counts), at<int32_t>(ws, L.rank_local),
+                          at<int32_t>(ws, L.counts),       at<int32_t>(ws, L.offsets),
+                          at<int32_t>(ws, L.n_kept),       at<int32_t>(ws, L.mt_row0),
+                          at<int32_t>(ws, L.mt_group),     at<int32_t>(ws, L.num_mt),
+                          at<int32_t>(ws, L.mt2_row0),     at<int32_t>(ws, L.mt2_group),
+                          at<int32_t>(ws, L.num_mt2)};
+    const bool hist_fused = !decode && router_hist_fusable(s);
+    int rc;
+    if (hist_fused) {
+        StageMark m(MOE_STAGE_ROUTER, st);
+        rc = router_topk_hist(s, x, Wg, bias, logits, idx, w, counter, hist, status, st);
+    } else {
+        rc = route_tokens(s, x, Wg, bias, logits, idx, w, counter, status, st);
+    }
     if (rc)
         return rc;
     if (decode) {
@@ -478,7 +550,7 @@ static int forward_impl(const moe_shape_t &s, const WsLayout &L, void *ws, const
     int32_t *slot_pos = at<int32_t>(ws, L.slot_pos);
     int32_t *perm_token = at<int32_t>(ws, L.perm_token);
     uint16_t *x_perm = at<uint16_t>(ws, L.x_perm);
-    {
+    if (!hist_fused) {
         StageMark m(MOE_STAGE_HIST, st);
         rc = launch_hist_scan(s, idx, chunk, rank, counter, counts, offsets,
                               at<int32_t>(ws, L.n_kept), at<int32_t>(ws, L.mt_row0),
@@ -491,7 +563,8 @@ static int forward_impl(const moe_shape_t &s, const WsLayout &L, void *ws, const
     {
         StageMark m(MOE_STAGE_PERMUTE, st);
         rc = launch_permute(s, idx, chunk, rank, offsets, x, slot_pos, perm_token, x_perm,
-                            (!shared && !det) ? out : nullptr, st);
+                            (!shared && !det) ? out : nullptr, st,
+                            hist_fused ? kBlockM : kChunkTokens);
     }
     if (rc)
         return rc;

@@ -1,0 +1,128 @@
+// tiles.cuh -- the histogram's last step, shared by the histogram kernel and
+// the router kernel that folds the histogram into its epilogue: per-chunk
+// expert counts become exclusive chunk bases, the capacity is applied, and
+// the offsets and the grouped GEMMs' m-tile lists are written.
+#pragma once
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+
+// Exclusive scan of one int per thread over the block (blockDim.x a multiple
+// of 32, at most 256). s_warp holds 17 ints.
+__device__ __forceinline__ int block_excl_scan(int v, int *s_warp, int *total)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int nw = blockDim.x >> 5;
+    int inc = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int o = __shfl_up_sync(kFullMask, inc, off);
+        if (lane >= off)
+            inc += o;
+    }
+    if (lane == 31)
+        s_warp[warp] = inc;
+    __syncthreads();
+    if (warp == 0) {
+        const int wv = (lane < nw) ? s_warp[lane] : 0;
+        int winc = wv;
+#pragma unroll
+        for (int off = 1; off < 8; off <<= 1) {
+            const int o = __shfl_up_sync(kFullMask, winc, off);
+            if (lane >= off)
+                winc += o;
+        }
+        if (lane < 8)
+            s_warp[8 + lane] = winc - wv;
+        if (lane == 7)
+            s_warp[16] = winc;
+    }
+    __syncthreads();
+    const int r = s_warp[8 + warp] + inc - v;
+    *total = s_warp[16];
+    __syncthreads();
+    return r;
+}
+
+// Writes the grouped-GEMM m-tile list for kept counts in s_kept[E]: expert e
+// contributes ceil(kept/tile_m) tiles starting at rows offsets[e] + tile_m i.
+// tile_start (may be NULL) receives each expert's first tile index. Thread e
+// handles expert e (blockDim.x >= E).
+__device__ inline void build_tiles(const int *s_kept, const int32_t *offsets_smem_or_global, int E,
+                                   int tile_m, int32_t *mt_row0, int32_t *mt_group,
+                                   int32_t *num_mt, int *s_warp, int32_t *tile_start = nullptr)
+{
+    const int tid = threadIdx.x;
+    const int e = tid;
+    const int nt = (e < E) ? (s_kept[e] + tile_m - 1) / tile_m : 0;
+    int total;
+    const int start = block_excl_scan(nt, s_warp, &total);
+    if (e < E && tile_start)
+        tile_start[e] = start;
+    if (e < E) {
+        const int base = offsets_smem_or_global[e];
+        // a last tile of <= 64 rows is marked for the M = 64 MMA (128-row lists only)
+        const int rem = s_kept[e] - (nt - 1) * tile_m;
+        for (int i = 0; i < nt; ++i) {
+            mt_row0[start + i] = base + i * tile_m;
+            const bool half = (tile_m == kBlockM) && (i == nt - 1) && rem <= 64;
+            mt_group[start + i] = e | (half ? kHalfTileBit : 0);
+        }
+    }
+    if (tid == 0)
+        *num_mt = total;
+}
+
+// Run by every thread of the last CTA (after a fence that makes the other
+// CTAs' chunk counts visible). chunk_counts[(c * nj + j) * E + e] holds the
+// count of expert e in chunk c (for slot j when nj = k, slot-major order);
+// it is replaced by the exclusive prefix in rank order (slots, then chunks).
+// Then counts, capacity, offsets (E + 1), n_kept, the 128-row m-tile list
+// (and the 256-row one when mt2_row0 is set), and the ticket is re-armed.
+// s_kept, s_off: MOE_MAX_E (+1) ints of shared memory; s_warp: 17 ints.
+__device__ inline void hist_finish(int32_t *chunk_counts, int nchunks, int nj, int E, int C,
+                                   int32_t *counts, int32_t *offsets, int32_t *n_kept,
+                                   int32_t *mt_row0, int32_t *mt_group, int32_t *num_mt,
+                                   int32_t *mt2_row0, int32_t *mt2_group, int32_t *num_mt2,
+                                   int32_t *tile_start, int32_t *counter, int *s_kept, int *s_off,
+                                   int *s_warp)
+{
+    const int tid = threadIdx.x;
+    for (int e = tid; e < MOE_MAX_E; e += blockDim.x) {
+        int kept = 0;
+        if (e < E) {
+            int run = 0;
+            for (int j = 0; j < nj; ++j)
+                for (int c = 0; c < nchunks; ++c) {
+                    const size_t i = ((size_t)c * nj + j) * E + e;
+                    const int v = __ldcg(&chunk_counts[i]);
+                    __stcg(&chunk_counts[i], run);
+                    run += v;
+                }
+            counts[e] = run;
+            kept = (C > 0 && run > C) ? C : run;
+        }
+        s_kept[e] = kept;
+    }
+    __syncthreads();
+    int total;
+    const int ex = block_excl_scan(tid < E ? s_kept[tid] : 0, s_warp, &total);
+    if (tid < E) {
+        offsets[tid] = ex;
+        s_off[tid] = ex;
+    }
+    if (tid == 0) {
+        offsets[E] = total;
+        *n_kept = total;
+    }
+    __syncthreads();
+    build_tiles(s_kept, s_off, E, kBlockM, mt_row0, mt_group, num_mt, s_warp, tile_start);
+    if (mt2_row0)
+        build_tiles(s_kept, s_off, E, 2 * kBlockM, mt2_row0, mt2_group, num_mt2, s_warp);
+    if (tid == 0)
+        *counter = 0;
+}
+
+} // namespace moe

@@ -261,6 +261,38 @@ def test_forward_parity(case, flags):
     assert_layer_close(out[torch.from_numpy(np.nonzero(same)[0]).cuda()], ref["out"][same], name)
 
 
+@pytest.mark.parametrize("T,E,k,C,zipf", [(300, 8, 2, 0, 0.0), (129, 16, 4, 30, 1.0),
+                                          (1000, 64, 8, 150, 1.0), (20000, 64, 8, 3000, 1.2),
+                                          (19000, 8, 2, 0, 0.5)])
+def test_forward_router_histogram_fused(T, E, k, C, zipf):
+    """Prefill with E <= 64 folds the expert histogram into the router GEMM
+    (per 128-token tile counts and ranks, last-CTA scan). moe_forward against
+    the step-by-step pipeline (separate histogram kernel) on the logits the
+    forward produced: identical top-k, and outputs that agree to fp32
+    rounding of the weights, so every capacity drop and permuted row agrees.
+    20000 tokens are 157 tiles: some CTAs take two."""
+    w = small_workload("rhist", T, 256, 256, E, k, capacity=C, zipf_s=zipf)
+    inp = I.make_inputs(w, "cuda", seed=T + E)
+    layer = M.MoeLayer(inp, flags=M.MOE_FLAG_DETERMINISTIC)
+    logits = torch.empty(T, E, dtype=torch.float32, device="cuda")
+    idx = torch.empty(T, k, dtype=torch.int32, device="cuda")
+    out = layer.forward(inp["x"], logits_out=logits, topk_idx_out=idx)
+    torch.cuda.synchronize()
+    assert int(layer.status.item()) == 0
+    b = pipeline_from_logits(inp, logits, flags=M.MOE_FLAG_DETERMINISTIC, fused=False)
+    assert int(b.status.item()) == 0
+    assert torch.equal(b.idx, idx)
+    if C:
+        assert (b.slot_pos < 0).any()
+    scale = max(b.out.abs().max().item(), 1e-30)
+    assert (out - b.out).abs().max().item() <= 1e-5 * scale
+    # the second call re-uses the ticket the first call's last CTA re-armed
+    out2 = layer.forward(inp["x"])
+    torch.cuda.synchronize()
+    assert int(layer.status.item()) == 0
+    assert torch.equal(out, out2)
+
+
 @pytest.mark.parametrize("flags", [0, M.MOE_FLAG_DETERMINISTIC, M.MOE_FLAG_SIMT_FFN],
                          ids=["default", "det", "simt"])
 def test_forward_slot_priority(flags):
