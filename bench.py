@@ -329,6 +329,7 @@ def run_ours(a, world, rank, local):
     graphs = None
     expert_choice = None
     mxfp8 = None
+    nvfp4 = None
     backward = None
     if a.workload == "prefill" and not a.no_extra:
         decode = run_decode_set(M, w, layer, x, dev, stream, world, peaks)
@@ -337,7 +338,10 @@ def run_ours(a, world, rank, local):
                                               max(3, a.steps // 2))
         backward = run_backward_set(M, w, inp, layer, dev, stream, world, peaks,
                                     max(3, a.steps // 4))
-        mxfp8 = run_mxfp8_set(M, w, inp, x, dev, stream, world, peaks, max(3, a.steps // 2))
+        mxfp8 = run_lowp_set(M, w, inp, x, dev, stream, world, peaks, max(3, a.steps // 2),
+                             "mxfp8")
+        nvfp4 = run_lowp_set(M, w, inp, x, dev, stream, world, peaks, max(3, a.steps // 2),
+                             "nvfp4")
 
     # ---- CPU baseline: the oracle on host cores (rank 0, N = 1 only)
     cpu = None
@@ -375,6 +379,8 @@ def run_ours(a, world, rank, local):
         res["expert_choice"] = expert_choice
     if mxfp8 is not None:
         res["mxfp8"] = mxfp8
+    if nvfp4 is not None:
+        res["nvfp4"] = nvfp4
     if backward is not None:
         res["backward"] = backward
     return res
@@ -494,19 +500,31 @@ def run_expert_choice_set(M, w, layer, x, dev, stream, world, peaks, steps):
             "stages_ms": {k: round(v[0] / v[1], 4) for k, v in st.items()}}
 
 
-def run_mxfp8_set(M, w, inp, x, dev, stream, world, peaks, steps):
-    """MXFP8 experts on the same weights and tokens: the prefill step (the
-    block-scaled w1/w3 GEMM against the fp8 dense peak, taken as twice the
-    measured sustained bf16 peak, the nominal fp8:bf16 ratio) and decode at
-    T = 1, 2, 4, 8 (GB/s over the chosen experts' codes and scales)."""
-    lay = M.MoeLayerMx(inp)
+LOWP = {
+    # layer class, format, bytes per weight (codes + block-scale share),
+    # tensor peak as a multiple of the measured sustained bf16 peak (the nominal ratio)
+    "mxfp8": ("MoeLayerMx", "MXFP8 (E4M3, E8M0 scale per 32) weights, x and h; bf16 router",
+              1.0 + 1.0 / 32.0, 2.0),
+    "nvfp4": ("MoeLayerNv4", "NVFP4 (E2M1, E4M3 scale per 16, fp32 global scale per tensor) "
+              "weights, x and h; bf16 router", 0.5 + 1.0 / 16.0, 4.0),
+}
+
+
+def run_lowp_set(M, w, inp, x, dev, stream, world, peaks, steps, fmt):
+    """Block-scaled experts (MXFP8 or NVFP4) on the same weights and tokens:
+    the prefill step (the w1/w3 GEMM against the format's dense peak, taken as
+    the measured sustained bf16 peak times the nominal ratio: 2 for fp8, 4 for
+    fp4) and decode at T = 1, 2, 4, 8 (GB/s over the chosen experts' codes and
+    scales)."""
+    cls, desc, per_weight, ratio = LOWP[fmt]
+    lay = getattr(M, cls)(inp)
     out = torch.empty(w.T, w.d, dtype=torch.float32, device=dev)
     idx = torch.empty(w.T, w.k, dtype=torch.int32, device=dev)
     for _ in range(3):
         lay.forward(x, out=out, topk_idx_out=idx)
     torch.cuda.synchronize()
     if int(lay.status.item()) != 0:
-        raise RuntimeError(f"device status {int(lay.status.item())} (mxfp8)")
+        raise RuntimeError(f"device status {int(lay.status.item())} ({fmt})")
     n_kept = routed_kept(idx, w.E, w.capacity)
     ms = max_over_ranks(time_loop(lambda: lay.forward(x, out=out), steps, stream), world, dev)
     M.moe_profile_enable(True)
@@ -514,20 +532,20 @@ def run_mxfp8_set(M, w, inp, x, dev, stream, world, peaks, steps):
     M.moe_profile_enable(False)
     st = M.moe_profile_read()
     flops, w13_flops, w2_flops = prefill_flops(w, n_kept)
-    fp8_peak = 2.0 * peaks["bf16_tflops_sustained"]
+    peak = ratio * peaks["bf16_tflops_sustained"]
     k13 = st["w13"][0] / st["w13"][1]
     k2 = st["w2"][0] / st["w2"][1]
-    res = {"format": "MXFP8 (E4M3, E8M0 scale per 32) weights, x and h; bf16 router",
+    res = {"format": desc,
            "prefill": {"tokens_per_s": round(w.T * world / (ms / 1e3), 1), "ms_per_step": round(ms, 4),
                        "active_tflops": round(flops / (ms / 1e3) / 1e12, 1),
                        "w13_tflops": round(w13_flops / (k13 / 1e3) / 1e12, 1),
-                       "w13_frac_fp8_peak": round(w13_flops / (k13 / 1e3) / 1e12 / fp8_peak, 4),
+                       "w13_frac_format_peak": round(w13_flops / (k13 / 1e3) / 1e12 / peak, 4),
                        "w2_tflops": round(w2_flops / (k2 / 1e3) / 1e12, 1),
-                       "fp8_peak_tflops": fp8_peak,
-                       "fp8_peak_source": "2 x measured bf16_tflops_sustained (nominal ratio)",
+                       "format_peak_tflops": peak,
+                       "format_peak_source": f"{ratio:g} x measured bf16_tflops_sustained "
+                                             "(nominal ratio)",
                        "stages_ms": {k: round(v[0] / v[1], 4) for k, v in st.items()}}}
     dec = {}
-    per_weight = 1.0 + 1.0 / 32.0        # code byte + its share of the block scale
     for T in I.DECODE_TS:
         xt = x[:T].contiguous()
         it = torch.empty(T, w.k, dtype=torch.int32, device=dev)

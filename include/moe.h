@@ -86,7 +86,9 @@ enum {
     MOE_FLAG_SLOT_PRIORITY = 1 << 8, /* capacity ranks in slot-major order (see moe_shape_t) */
     MOE_FLAG_MXFP8 = 1 << 9,         /* workspace for moe_forward_mxfp8 (MXFP8 experts); the
                                         bf16 layer calls reject it */
-    MOE_FLAG_BACKWARD = 1 << 10      /* workspace also sized for moe_backward */
+    MOE_FLAG_BACKWARD = 1 << 10,     /* workspace also sized for moe_backward */
+    MOE_FLAG_NVFP4 = 1 << 11         /* workspace for moe_forward_nvfp4 (NVFP4 experts); the
+                                        bf16 layer calls reject it */
 };
 
 #define MOE_MAX_E 256
@@ -324,6 +326,66 @@ MOE_API int moe_forward_mxfp8(const moe_shape_t *shape, const moe_bf16_t *x, con
                               int32_t *topk_idx_out, uint32_t *status, void *ws, size_t ws_bytes,
                               moe_stream_t stream);
 
+/* ---- NVFP4 experts: block-scaled 4-bit weights and activations
+ * (the NVFP4 grouped GEMM of "Current Bug: CuTeDSLMoERunner produces wrong
+ * output", "How the pipeline works": per-expert weight scales and activation
+ * scales feeding a block-scaled grouped GEMM; the page does not spell the
+ * format out, this is NVIDIA's NVFP4):
+ *   - an element is E2M1 (magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6), packed two
+ *     to a byte, element 2i in the low nibble of byte i;
+ *   - a block is 16 consecutive elements along the contraction dimension,
+ *     with one E4M3 scale s;
+ *   - a tensor has one fp32 global encode scale gs: 448 * 6 / max|W| per
+ *     expert for the weights (W1 and W3 of an expert share one, W2 has its
+ *     own; 1 for an all-zero tensor), and the caller's constants x_gs and
+ *     h_gs for x and for the SwiGLU product h;
+ *   - encoding, each step an IEEE fp32 operation: s = E4M3((amax / 6) * gs),
+ *     nearest even, saturating; r = gs / s (0 when s = 0); code = E2M1(v * r),
+ *     nearest even, saturating at 6. A code stands for E2M1 * s / gs.
+ * The router, top-k and dispatch are those of moe_forward; x and h are
+ * quantized on the fly; the GEMMs (tcgen05 kind::mxf4nvf4, 16-element
+ * blocks) accumulate in fp32 and multiply by 1 / (gs_activation * gs_weight);
+ * out is fp32. d, d_ff and d_ff_shared must be multiples of 256
+ * (MOE_ERR_UNSUPPORTED otherwise).
+ *
+ * moe_quantize_experts_nvfp4: one-time conversion of bf16 experts.
+ *   W1, W3  [E, d_ff, d] bf16 in; W2 [E, d, d_ff] bf16 in
+ *   W13q    [E, 2*d_ff, d/2] bytes out: packed E2M1 codes, rows in the
+ *           64-row gate/up interleave of moe_quantize_experts_mxfp8
+ *   W13sf   E*2*d_ff*d/16 E4M3 bytes out, in 512-byte atoms: the scales of
+ *           rows 128t..128t+127 and K elements 64g..64g+63 form atom
+ *           (t * (K/64) + g), inside which row 128t + m, block 4g + j sits at
+ *           byte (m % 32) * 16 + (m / 32) * 4 + j (K = d, packed rows)
+ *   W13_gs  [E] fp32 out: the global encode scale of expert e's W1 and W3
+ *   W2q     [E, d, d_ff/2] bytes out; W2sf E*d*d_ff/16 bytes out, atoms as
+ *           above with K = d_ff; W2_gs [E] fp32 out
+ * With E = 1 and d_ff = d_ff_shared it converts a shared expert. Code and
+ * scale arrays 16-byte aligned, scale vectors 4-byte aligned. */
+MOE_API int moe_quantize_experts_nvfp4(const moe_shape_t *shape, const moe_bf16_t *W1,
+                                       const moe_bf16_t *W3, const moe_bf16_t *W2,
+                                       uint8_t *W13q, uint8_t *W13sf, float *W13_gs,
+                                       uint8_t *W2q, uint8_t *W2sf, float *W2_gs,
+                                       moe_stream_t stream);
+
+/* The layer with NVFP4 experts. Requires MOE_FLAG_NVFP4 in shape->flags (also
+ * when sizing the workspace); MOE_FLAG_HOST_IO and MOE_FLAG_MXFP8 are
+ * rejected (MOE_ERR_INVALID_ARG), as are x_gs or h_gs that are not positive
+ * and finite. Arguments as in moe_forward_mxfp8, with each weight set's
+ * global scales (device pointers, as moe_quantize_experts_nvfp4 writes them).
+ * Every T runs the block-scaled tensor-core GEMMs, which read each chosen
+ * expert's codes and scales once (4.5 bits a weight); MOE_FLAG_FORCE_DECODE
+ * is MOE_ERR_UNSUPPORTED. MOE_FLAG_DETERMINISTIC, capacity and
+ * MOE_FLAG_SLOT_PRIORITY act as in moe_forward.
+ * Device errors: MOE_ERR_NONFINITE, MOE_ERR_BAD_EXPERT, MOE_ERR_TIMEOUT. */
+MOE_API int moe_forward_nvfp4(const moe_shape_t *shape, const moe_bf16_t *x, const moe_bf16_t *Wg,
+                              const float *bias, const uint8_t *W13q, const uint8_t *W13sf,
+                              const float *W13_gs, const uint8_t *W2q, const uint8_t *W2sf,
+                              const float *W2_gs, const uint8_t *W13s_q, const uint8_t *W13s_sf,
+                              const float *W13s_gs, const uint8_t *W2s_q, const uint8_t *W2s_sf,
+                              const float *W2s_gs, float x_gs, float h_gs, float *out,
+                              float *logits_out, int32_t *topk_idx_out, uint32_t *status,
+                              void *ws, size_t ws_bytes, moe_stream_t stream);
+
 /* ---- Backward pass ("Sparse MoE Block" / "Expert FFN" differentiated with the
  * routing decisions held fixed: top-k set, capacity drops, slot order).
  *
@@ -338,7 +400,7 @@ MOE_API int moe_pack_backward(const moe_shape_t *shape, const moe_bf16_t *W13,
 /* Gradients of sum(out * dout) for the layer moe_forward computes (routing
  * recomputed with the same kernels, so it is identical). Requires
  * MOE_FLAG_BACKWARD in shape->flags (also for moe_workspace_size); rejects
- * MOE_FLAG_MXFP8 and MOE_FLAG_SIMT_FFN (MOE_ERR_INVALID_ARG).
+ * MOE_FLAG_MXFP8, MOE_FLAG_NVFP4 and MOE_FLAG_SIMT_FFN (MOE_ERR_INVALID_ARG).
  *   x, Wg, bias, W13  as moe_forward; W13T, W2T as moe_pack_backward writes
  *   W13_shared, W13T_shared, W2T_shared: with d_ff_shared > 0, the shared
  *         expert's packed W13 [2*d_ff_shared, d] and its transposes (from

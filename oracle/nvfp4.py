@@ -53,6 +53,14 @@ def e2m1_encode(v):
     """float32 values -> E2M1 codes: the nearest representable magnitude, ties
     to the even code, |v| > 6 saturating to 6; the sign bit is v's sign."""
     v = np.asarray(v, np.float32)
+    if v.size > (1 << 20):   # in slices, to bound the distance table's memory
+        flat = v.reshape(-1)
+        return np.concatenate([_e2m1_encode(flat[i:i + (1 << 20)])
+                               for i in range(0, flat.size, 1 << 20)]).reshape(v.shape)
+    return _e2m1_encode(v)
+
+
+def _e2m1_encode(v):
     a = np.abs(v.astype(np.float64))
     dist = np.abs(a[..., None] - _E2M1_MAG)               # [..., 8]
     best = dist.min(-1, keepdims=True)

@@ -34,6 +34,14 @@
 // columns), so a stage's copy never waits for the previous stage's MMAs to
 // finish reading; a stage's columns are rewritten only after its MMAs have
 // committed (the producer refills its buffers only then).
+//
+// NVFP4 operands (FMT_NV4, nvfp4.cuh) run on the same engine with
+// tcgen05.mma kind::mxf4nvf4 .block_scale.scale_vec::4X: packed E2M1 codes
+// (a 128-byte K stage holds 256 elements), one E4M3 scale per 16 elements, so
+// a stage brings four 512-byte scale atoms per operand (one 2 KB bulk copy),
+// owns 32 TMEM scale columns, and issues four M=128 N=128 K=64 MMAs, each
+// reading a whole 32-bit scale word per row. The epilogue multiplies the
+// accumulators by 1 / (gs_A * gs_B[expert]) (the two global encode scales).
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -43,6 +51,7 @@
 #include "common.cuh"
 #include "internal.h"
 #include "mxfp8.cuh"
+#include "nvfp4.cuh"
 
 namespace moe {
 
@@ -54,7 +63,7 @@ namespace moe {
 #endif
 
 struct MxArgs {
-    int kblocks;            // K / 128 (= scale atoms per tile row band)
+    int kblocks;            // K stages (K / 128 E4M3 or K / 256 E2M1 elements)
     int n_tiles;
     int group_m;
     int b_rows_per_group;
@@ -75,23 +84,31 @@ struct MxArgs {
     int k;
     const float *perm_w;
     uint32_t *status;
+    const float *b_gs;        // NVFP4: B's global encode scale per group
+    float a_gs, out_gs;       // NVFP4: A's global encode scale; h's (EPI_SWIGLU_MX)
 };
 
+enum { FMT_MX8 = 0, FMT_NV4 = 1 };
+
+template <int FMT>
 struct MxCfg {
-    static constexpr int BM = 128, BN = 128, BK = 128;   // BK in elements = bytes
-    static constexpr int A_BYTES = BM * BK;
-    static constexpr int B_BYTES = BN * BK;
-    static constexpr int SF_BYTES = 512;                  // 128 rows x 4 scale bytes
+    static constexpr int BM = 128, BN = 128;
+    static constexpr int BK_BYTES = 128;                  // one K stage: 128 bytes per row
+    static constexpr int BK = FMT == FMT_NV4 ? 256 : 128; // ... = 256 E2M1 or 128 E4M3 elements
+    static constexpr int A_BYTES = BM * BK_BYTES;
+    static constexpr int B_BYTES = BN * BK_BYTES;
+    static constexpr int SF_ATOMS = FMT == FMT_NV4 ? 4 : 1;   // 512-byte scale atoms per stage
+    static constexpr int SF_BYTES = 512 * SF_ATOMS;       // per operand per stage
     static constexpr int STAGES = 6;
     static constexpr int TMEM_COLS = 512;
     static constexpr int SF_COL = 2 * BN;                 // scale columns after the accumulators
-    static constexpr int SF_COLS_PER_STAGE = 8;           // 4 for A's scales, 4 for B's
+    static constexpr int SF_COLS_PER_STAGE = 8 * SF_ATOMS; // 4 per atom, A's then B's
     static constexpr int SMEM_BYTES =
         1024 + STAGES * (A_BYTES + B_BYTES) + STAGES * 2 * SF_BYTES + 256;
+    static_assert(SF_COL + STAGES * SF_COLS_PER_STAGE <= TMEM_COLS,
+                  "accumulators and per-stage scale columns must fit the TMEM allocation");
+    static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
 };
-
-static_assert(MxCfg::SF_COL + MxCfg::STAGES * MxCfg::SF_COLS_PER_STAGE <= MxCfg::TMEM_COLS,
-              "accumulators and per-stage scale columns must fit the TMEM allocation");
 
 __device__ __forceinline__ void mx_tile_coords(long long tile, int num_mt, int n_tiles,
                                                int group_m, int &m_idx, int &n_idx)
@@ -124,9 +141,20 @@ __device__ __forceinline__ uint32_t idesc_mx(uint32_t sf_id)
 {
     return (sf_id << 4)                      // B scale factor id
            | (1u << 23)                      // scale format: E8M0
-           | ((uint32_t)(MxCfg::BN >> 3) << 17)
-           | ((uint32_t)(MxCfg::BM >> 4) << 24)
+           | ((uint32_t)(128 >> 3) << 17)    // N = 128
+           | ((uint32_t)(128 >> 4) << 24)    // M = 128
            | (sf_id << 29);                  // A scale factor id
+}
+
+// Instruction descriptor, kind::mxf4nvf4 block-scaled with 16-element
+// blocks: E2M1 A and B (format 1), K-major, E4M3 scales (scale format 0),
+// fp32 D, M = 128, N = 128, dense K = 64; each MMA reads a whole 32-bit
+// scale word (four blocks) per row, so the scale ids stay 0.
+__device__ __forceinline__ uint32_t idesc_nv4()
+{
+    return (1u << 7) | (1u << 10)            // A and B: E2M1
+           | ((uint32_t)(128 >> 3) << 17)    // N = 128
+           | ((uint32_t)(128 >> 4) << 24);   // M = 128
 }
 
 __device__ __forceinline__ void tc_cp_sf(uint32_t taddr, uint64_t desc)
@@ -147,6 +175,18 @@ __device__ __forceinline__ void tc_mma_mx(uint32_t d_tmem, uint64_t a_desc, uint
         : "memory");
 }
 
+__device__ __forceinline__ void tc_mma_nv4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                           uint32_t idesc, uint32_t sfa, uint32_t sfb,
+                                           uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+        : "memory");
+}
+
 // 1-D bulk copy global -> shared (16-byte aligned, size a multiple of 16),
 // completion counted in bytes on `bar`.
 __device__ __forceinline__ void bulk_load(void *smem_dst, const void *src, uint32_t bytes,
@@ -158,12 +198,36 @@ __device__ __forceinline__ void bulk_load(void *smem_dst, const void *src, uint3
         : "memory");
 }
 
-template <int MODE>
+template <int MODE, int FMT>
 __device__ __forceinline__ void mx_epilogue(const MxArgs &p, uint32_t tb, long long row,
-                                            bool valid, int n_idx, int m_idx, int m)
+                                            bool valid, int n_idx, int m_idx, int m, float alpha)
 {
-    constexpr int BN = MxCfg::BN;
-    if (MODE == EPI_SWIGLU_MX) {
+    constexpr int BN = 128;
+    if (MODE == EPI_SWIGLU_MX && FMT == FMT_NV4) {
+        // h columns n_idx*64 .. +63: 32 bytes of packed codes per row, two
+        // 16-element blocks (and scales) per 32-column chunk
+        uint8_t *hq = static_cast<uint8_t *>(p.out) + row * (p.ldo / 2) + n_idx * 32;
+#pragma unroll 1
+        for (int c = 0; c < 2; ++c) {
+            float g[32], u[32];
+            tmem_ld32(tb + c * 32, g);
+            tmem_ld32(tb + 64 + c * 32, u);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+                g[i] = silu_mul(g[i] * alpha, u[i] * alpha);
+            uint2 q0, q1;
+            const uint32_t s0 = nv_quantize16(g, p.out_gs, q0);
+            const uint32_t s1 = nv_quantize16(g + 16, p.out_gs, q1);
+            if (valid) {
+                *reinterpret_cast<uint4 *>(hq + c * 16) = make_uint4(q0.x, q0.y, q1.x, q1.y);
+                // blocks 4 n_idx + 2c and + 1: adjacent bytes of one atom word
+                *reinterpret_cast<uint16_t *>(p.out_sf +
+                                              nv_sf_offset(m_idx, m, 4 * n_idx + 2 * c, (int)p.ldo)) =
+                    (uint16_t)(s0 | (s1 << 8));
+            }
+        }
+    } else if (MODE == EPI_SWIGLU_MX) {
         // columns [0,64) = gate, [64,128) = up of h columns n_idx*64 ..
         uint8_t *hq = static_cast<uint8_t *>(p.out) + row * p.ldo + n_idx * 64;
 #pragma unroll 1
@@ -197,6 +261,7 @@ __device__ __forceinline__ void mx_epilogue(const MxArgs &p, uint32_t tb, long l
                     if (p.slot_pos[(long long)t * p.k + j] == row)
                         wgt = p.topk_w[(long long)t * p.k + j];
             }
+            wgt *= alpha;
         }
         float *o = static_cast<float *>(p.out) + (long long)t * p.ldo + n_idx * BN;
 #pragma unroll 1
@@ -223,24 +288,25 @@ __device__ __forceinline__ void mx_epilogue(const MxArgs &p, uint32_t tb, long l
                 float4 *dst = reinterpret_cast<float4 *>(o + c * 32);
 #pragma unroll
                 for (int i = 0; i < 8; ++i)
-                    dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+                    dst[i] = make_float4(alpha * v[4 * i], alpha * v[4 * i + 1],
+                                         alpha * v[4 * i + 2], alpha * v[4 * i + 3]);
             }
         }
     }
 }
 
-template <int MODE>
+template <int MODE, int FMT>
 __global__ void __launch_bounds__(192, 1)
     k_gemm_mx(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
               const MxArgs p)
 {
-    using C = MxCfg;
+    using C = MxCfg<FMT>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     uint8_t *sA = smem;
     uint8_t *sB = sA + C::STAGES * C::A_BYTES;
-    uint8_t *sSF = sB + C::STAGES * C::B_BYTES;   // per stage: 512 B of A scales, 512 B of B
+    uint8_t *sSF = sB + C::STAGES * C::B_BYTES;   // per stage: A's scale atoms, then B's
     uint64_t *full = reinterpret_cast<uint64_t *>(sSF + C::STAGES * 2 * C::SF_BYTES);
     uint64_t *empty = full + C::STAGES;
     uint64_t *tfull = empty + C::STAGES;
@@ -287,8 +353,9 @@ __global__ void __launch_bounds__(192, 1)
                 const long long row0 = p.mt_row0 ? p.mt_row0[m_idx] : (long long)m_idx * C::BM;
                 const int grp = p.mt_group ? (p.mt_group[m_idx] & ~kHalfTileBit) : 0;
                 const long long brow = (long long)grp * p.b_rows_per_group + (long long)n_idx * C::BN;
-                const uint8_t *sfa = p.A_sf + (long long)m_idx * p.kblocks * kSfAtomBytes;
-                const uint8_t *sfb = p.B_sf + (brow >> 7) * p.kblocks * kSfAtomBytes;
+                // a 128-row band's atoms: kblocks stages of SF_BYTES each
+                const uint8_t *sfa = p.A_sf + (long long)m_idx * p.kblocks * C::SF_BYTES;
+                const uint8_t *sfb = p.B_sf + (brow >> 7) * p.kblocks * C::SF_BYTES;
                 for (int kb = 0; kb < p.kblocks; ++kb, ++it) {
                     const int s = it % C::STAGES;
                     const uint32_t ph = (it / C::STAGES) & 1u;
@@ -298,10 +365,11 @@ __global__ void __launch_bounds__(192, 1)
                     }
                     uint8_t *sf = sSF + s * 2 * C::SF_BYTES;
                     mbar_arrive_expect_tx(&full[s], C::A_BYTES + C::B_BYTES + 2 * C::SF_BYTES);
-                    tma_load_2d(sA + s * C::A_BYTES, &tmA, kb * C::BK, (int)row0, &full[s]);
-                    tma_load_2d(sB + s * C::B_BYTES, &tmB, kb * C::BK, (int)brow, &full[s]);
-                    bulk_load(sf, sfa + kb * kSfAtomBytes, C::SF_BYTES, &full[s]);
-                    bulk_load(sf + C::SF_BYTES, sfb + kb * kSfAtomBytes, C::SF_BYTES, &full[s]);
+                    tma_load_2d(sA + s * C::A_BYTES, &tmA, kb * C::BK_BYTES, (int)row0, &full[s]);
+                    tma_load_2d(sB + s * C::B_BYTES, &tmB, kb * C::BK_BYTES, (int)brow, &full[s]);
+                    bulk_load(sf, sfa + (long long)kb * C::SF_BYTES, C::SF_BYTES, &full[s]);
+                    bulk_load(sf + C::SF_BYTES, sfb + (long long)kb * C::SF_BYTES, C::SF_BYTES,
+                              &full[s]);
                 }
             }
         }
@@ -327,15 +395,26 @@ __global__ void __launch_bounds__(192, 1)
                     // each stage has its own scale columns: the copy for this
                     // stage never overwrites columns that earlier MMAs still read
                     const uint32_t sf_a = tmem_base + C::SF_COL + s * C::SF_COLS_PER_STAGE;
-                    const uint32_t sf_b = sf_a + 4;
-                    tc_cp_sf(sf_a, smem_desc_sf(sf0));
-                    tc_cp_sf(sf_b, smem_desc_sf(sf0 + C::SF_BYTES));
+                    const uint32_t sf_b = sf_a + 4 * C::SF_ATOMS;
+#pragma unroll
+                    for (int i = 0; i < C::SF_ATOMS; ++i) {
+                        tc_cp_sf(sf_a + 4 * i, smem_desc_sf(sf0 + 512 * i));
+                        tc_cp_sf(sf_b + 4 * i, smem_desc_sf(sf0 + C::SF_BYTES + 512 * i));
+                    }
                     const uint32_t a0 = smem_u32(sA + s * C::A_BYTES);
                     const uint32_t b0 = smem_u32(sB + s * C::B_BYTES);
+                    // four MMAs of 32 bytes of K each (K = 32 E4M3 or 64 E2M1)
 #pragma unroll
-                    for (int kk = 0; kk < C::BK / 32; ++kk)
-                        tc_mma_mx(d_tmem, smem_desc_k128(a0 + kk * 32), smem_desc_k128(b0 + kk * 32),
-                                  idesc_mx(kk), sf_a, sf_b, (kb | kk) != 0);
+                    for (int kk = 0; kk < 4; ++kk) {
+                        if constexpr (FMT == FMT_NV4)
+                            tc_mma_nv4(d_tmem, smem_desc_k128(a0 + kk * 32),
+                                       smem_desc_k128(b0 + kk * 32), idesc_nv4(), sf_a + 4 * kk,
+                                       sf_b + 4 * kk, (kb | kk) != 0);
+                        else
+                            tc_mma_mx(d_tmem, smem_desc_k128(a0 + kk * 32),
+                                      smem_desc_k128(b0 + kk * 32), idesc_mx(kk), sf_a, sf_b,
+                                      (kb | kk) != 0);
+                    }
                     tc_commit(&empty[s]);
                 }
                 if (!ok)
@@ -359,7 +438,8 @@ __global__ void __launch_bounds__(192, 1)
             const long long row = row0 + q * 32 + lane;
             const bool valid = row < row_end;
             const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + b * C::BN;
-            mx_epilogue<MODE>(p, tb, row, valid, n_idx, m_idx, q * 32 + lane);
+            const float alpha = FMT == FMT_NV4 ? 1.0f / (p.a_gs * p.b_gs[grp]) : 1.0f;
+            mx_epilogue<MODE, FMT>(p, tb, row, valid, n_idx, m_idx, q * 32 + lane, alpha);
             tc_fence_before();
             __syncwarp();
             if (lane == 0)
@@ -409,17 +489,21 @@ static int make_tmap_u8(CUtensorMap *m, const void *base, long long cols, long l
     return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
 }
 
-template <int MODE>
+template <int MODE, int FMT>
 static int launch_mx_impl(const GemmArgs &g, cudaStream_t st)
 {
-    using C = MxCfg;
-    if (g.K % 128 != 0 || g.N % 128 != 0)
+    using C = MxCfg<FMT>;
+    if (g.K % C::BK != 0 || g.N % C::BN != 0)
         return MOE_ERR_INVALID_ARG;
+    if (FMT == FMT_NV4 && !g.b_gs)
+        return MOE_ERR_INVALID_ARG;
+    // code rows are K bytes (E4M3) or K / 2 bytes (packed E2M1)
+    const long long row_bytes = FMT == FMT_NV4 ? g.K / 2 : g.K;
     CUtensorMap tA, tB;
-    int rc = make_tmap_u8(&tA, g.Aq, g.K, g.a_rows);
+    int rc = make_tmap_u8(&tA, g.Aq, row_bytes, g.a_rows);
     if (rc)
         return rc;
-    rc = make_tmap_u8(&tB, g.Bq, g.K, g.b_rows_total);
+    rc = make_tmap_u8(&tB, g.Bq, row_bytes, g.b_rows_total);
     if (rc)
         return rc;
     MxArgs p;
@@ -445,12 +529,15 @@ static int launch_mx_impl(const GemmArgs &g, cudaStream_t st)
     p.k = g.k;
     p.perm_w = g.perm_w;
     p.status = g.status;
+    p.b_gs = g.b_gs;
+    p.a_gs = g.a_gs;
+    p.out_gs = g.out_gs;
 
     static int attr_done[64] = {0};
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev >= 0 && dev < 64 && !attr_done[dev]) {
-        if (cudaFuncSetAttribute(k_gemm_mx<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(k_gemm_mx<MODE, FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  C::SMEM_BYTES) != cudaSuccess)
             return MOE_ERR_CUDA;
         attr_done[dev] = 1;
@@ -460,16 +547,24 @@ static int launch_mx_impl(const GemmArgs &g, cudaStream_t st)
     if (tiles <= 0)
         return MOE_OK;
     const int grid = (int)std::min<long long>(tiles, num_sms());
-    k_gemm_mx<MODE><<<grid, 192, C::SMEM_BYTES, st>>>(tA, tB, p);
+    k_gemm_mx<MODE, FMT><<<grid, 192, C::SMEM_BYTES, st>>>(tA, tB, p);
     return launched();
 }
 
 int launch_gemm_mx(const GemmArgs &g, cudaStream_t st)
 {
+    if (g.fmt == FMT_NV4) {
+        switch (g.mode) {
+        case EPI_SWIGLU_MX: return launch_mx_impl<EPI_SWIGLU_MX, FMT_NV4>(g, st);
+        case EPI_COMBINE: return launch_mx_impl<EPI_COMBINE, FMT_NV4>(g, st);
+        case EPI_STORE_F32: return launch_mx_impl<EPI_STORE_F32, FMT_NV4>(g, st);
+        default: return MOE_ERR_INVALID_ARG;
+        }
+    }
     switch (g.mode) {
-    case EPI_SWIGLU_MX: return launch_mx_impl<EPI_SWIGLU_MX>(g, st);
-    case EPI_COMBINE: return launch_mx_impl<EPI_COMBINE>(g, st);
-    case EPI_STORE_F32: return launch_mx_impl<EPI_STORE_F32>(g, st);
+    case EPI_SWIGLU_MX: return launch_mx_impl<EPI_SWIGLU_MX, FMT_MX8>(g, st);
+    case EPI_COMBINE: return launch_mx_impl<EPI_COMBINE, FMT_MX8>(g, st);
+    case EPI_STORE_F32: return launch_mx_impl<EPI_STORE_F32, FMT_MX8>(g, st);
     default: return MOE_ERR_INVALID_ARG;
     }
 }

@@ -140,6 +140,13 @@ struct GemmArgs {
     // in the atom layout (mxfp8.cuh): A's keyed by m-tile index, B's by row/128
     const uint8_t *Aq, *A_sf, *Bq, *B_sf;
     uint8_t *out_sf;          // EPI_SWIGLU_MX: scales of h, atom layout keyed by m-tile
+    // NVFP4 operands instead (fmt = 1, nvfp4.cuh): packed E2M1 codes, E4M3
+    // scales per 16 in the 64-element atom layout; A's global encode scale
+    // a_gs, B's per group b_gs[g]; the accumulators are multiplied by
+    // 1 / (a_gs * b_gs[g]); EPI_SWIGLU_MX quantizes h with out_gs
+    int fmt;
+    const float *b_gs;
+    float a_gs, out_gs;
     // EPI_ROUTER_TOPK: top-k outputs [rows, k]; counter_zero (one word) is zeroed
     int32_t *route_idx;
     float *route_w;
@@ -190,6 +197,19 @@ int launch_mx_pack_w13(const moe_shape_t &s, const uint16_t *W1, const uint16_t 
 int launch_mx_gather(const moe_shape_t &s, const uint16_t *x, const int32_t *idx,
                      const int32_t *slot_pos, const int32_t *offsets, const int32_t *tile_start,
                      uint8_t *xq, uint8_t *xsf, cudaStream_t st);
+// ---- NVFP4 quantization (nv_quant.cu)
+// per-expert global encode scales of W1 and W3 together (gs13 [E]) and of W2
+int launch_nv_weight_scales(const moe_shape_t &s, const uint16_t *W1, const uint16_t *W3,
+                            const uint16_t *W2, float *gs13, float *gs2, cudaStream_t st);
+// rows of a bf16 matrix; global scale gs_arr[row / rows_per_gs], or gs_const
+int launch_nv_quantize_rows(const uint16_t *src, long long rows, int K, const float *gs_arr,
+                            long long rows_per_gs, float gs_const, uint8_t *codes,
+                            uint8_t *scales, cudaStream_t st);
+int launch_nv_pack_w13(const moe_shape_t &s, const uint16_t *W1, const uint16_t *W3,
+                       const float *gs13, uint8_t *codes, uint8_t *scales, cudaStream_t st);
+int launch_nv_gather(const moe_shape_t &s, const uint16_t *x, const int32_t *idx,
+                     const int32_t *slot_pos, const int32_t *offsets, const int32_t *tile_start,
+                     float gs, uint8_t *xq, uint8_t *xsf, cudaStream_t st);
 // n values (a multiple of 32) through MXFP8 and back, as bf16 (PDL launch)
 int launch_mx_qdq_bf16(const uint16_t *src, long long n, uint16_t *dst, cudaStream_t st);
 int launch_mx_qdq_f32(const float *src, long long n, uint16_t *dst, cudaStream_t st);

@@ -1,6 +1,7 @@
 // moe_api.cu -- the extern "C" entry points of libmoe.so (declared in moe.h):
 // argument validation, workspace carving, and the launch sequences.
 #include <algorithm>
+#include <cmath>
 #include <atomic>
 #include <cstdint>
 #include <cstring>
@@ -9,6 +10,7 @@
 
 #include "internal.h"
 #include "mxfp8.cuh"
+#include "nvfp4.cuh"
 
 namespace moe {
 
@@ -132,27 +134,33 @@ WsLayout ws_layout(const moe_shape_t &s)
     L.mt2_group = take((size_t)L.max_mt2 * 4);
     L.num_mt2 = take(4);
     const bool mx = (s.flags & MOE_FLAG_MXFP8) != 0;
+    const bool nv = (s.flags & MOE_FLAG_NVFP4) != 0;
+    const bool lowp = mx || nv;   // block-scaled experts: codes instead of bf16 copies
     const size_t dfs = s.d_ff_shared;
-    L.x_perm = take(mx ? 0 : N * s.d * 2);
-    L.H = take(mx ? 0 : N * s.d_ff * 2);
-    L.H_shared = take(!mx && dfs ? T * dfs * 2 : 0);
+    L.x_perm = take(lowp ? 0 : N * s.d * 2);
+    L.H = take(lowp ? 0 : N * s.d_ff * 2);
+    L.H_shared = take(!lowp && dfs ? T * dfs * 2 : 0);
     L.Y = take((s.flags & MOE_FLAG_DETERMINISTIC) ? N * s.d * 4 : 0);
     const size_t Td = T < (size_t)MOE_DECODE_MAX_T ? T : (size_t)MOE_DECODE_MAX_T;
     L.dec_H = take((Td * k * s.d_ff + Td * dfs) * 2);
     L.dec_xdq = take(mx ? Td * s.d * 2 : 0);
     L.dec_H32 = take(mx ? (Td * k * s.d_ff + Td * dfs) * 4 : 0);
     // scales in the atom layout: routed operands keyed by m-tile (at most
-    // max_mt tiles of 128 rows), shared-expert operands by row / 128
+    // max_mt tiles of 128 rows), shared-expert operands by row / 128; NVFP4
+    // has twice the scales (16-element blocks) and half the code bytes
     const size_t mt_rows = (size_t)L.max_mt * 128;
-    L.xq = take(mx ? N * s.d : 0);
-    L.xsf = take(mx ? (size_t)sf_atom_bytes(mt_rows, s.d) : 0);
-    L.Hq = take(mx ? N * s.d_ff : 0);
-    L.Hsf = take(mx ? (size_t)sf_atom_bytes(mt_rows, s.d_ff) : 0);
-    L.xq_s = take(mx && dfs ? T * s.d : 0);
-    L.xsf_s = take(mx && dfs ? (size_t)sf_atom_bytes(T, s.d) : 0);
-    L.Hsq = take(mx && dfs ? T * dfs : 0);
-    L.Hssf = take(mx && dfs ? (size_t)sf_atom_bytes(T, (int)dfs) : 0);
-    L.tile_start = take(mx ? E * 4 : 0);
+    auto sf_bytes = [&](size_t rows, size_t K) {
+        return (size_t)(nv ? nv_sf_bytes((long long)rows, (int)K) : sf_atom_bytes((long long)rows, (int)K));
+    };
+    L.xq = take(lowp ? N * s.d : 0);
+    L.xsf = take(lowp ? sf_bytes(mt_rows, s.d) : 0);
+    L.Hq = take(lowp ? N * s.d_ff : 0);
+    L.Hsf = take(lowp ? sf_bytes(mt_rows, s.d_ff) : 0);
+    L.xq_s = take(lowp && dfs ? T * s.d : 0);
+    L.xsf_s = take(lowp && dfs ? sf_bytes(T, s.d) : 0);
+    L.Hsq = take(lowp && dfs ? T * dfs : 0);
+    L.Hssf = take(lowp && dfs ? sf_bytes(T, dfs) : 0);
+    L.tile_start = take(lowp ? E * 4 : 0);
     // backward pass: saved gate/up, w * dout, [dg | du], per-row <dh, h>, the
     // K-grouped GEMMs' ranges and tile lists, and the padded transposes
     const bool bw = (s.flags & MOE_FLAG_BACKWARD) != 0;
@@ -589,8 +597,18 @@ static int forward_impl(const moe_shape_t &s, const WsLayout &L, void *ws, const
 // ---------------------------------------------------------------- MXFP8 experts
 // Grouped MXFP8 GEMMs over the routed rows: w1/w3 with the SwiGLU + MXFP8
 // epilogue into Hq/Hsf, then w2 with the chosen epilogue.
-static int expert_ffn_mx(const moe_shape_t &s, const WsLayout &L, void *ws, const uint8_t *W13q,
-                         const uint8_t *W13sf, const uint8_t *W2q, const uint8_t *W2sf,
+// Block-scaled expert weights: MXFP8 (fmt 0) or NVFP4 (fmt 1, with global
+// encode scales per expert and the activations' constants x_gs, h_gs).
+struct LowpWeights {
+    int fmt;
+    const uint8_t *W13q, *W13sf, *W2q, *W2sf;
+    const float *W13gs, *W2gs;
+    const uint8_t *W13s_q, *W13s_sf, *W2s_q, *W2s_sf;
+    const float *W13s_gs, *W2s_gs;
+    float x_gs, h_gs;
+};
+
+static int expert_ffn_mx(const moe_shape_t &s, const WsLayout &L, void *ws, const LowpWeights &lw,
                          const int32_t *offsets, const int32_t *perm_token,
                          const int32_t *slot_pos, const float *topk_w, float *y_perm, float *out,
                          uint32_t *status, cudaStream_t st)
@@ -598,11 +616,15 @@ static int expert_ffn_mx(const moe_shape_t &s, const WsLayout &L, void *ws, cons
     const long long N = (long long)s.T * s.k;
     GemmArgs g = gemm_base();
     g.mode = EPI_SWIGLU_MX;
+    g.fmt = lw.fmt;
     g.Aq = at<uint8_t>(ws, L.xq);
     g.A_sf = at<uint8_t>(ws, L.xsf);
     g.a_rows = N;
-    g.Bq = W13q;
-    g.B_sf = W13sf;
+    g.Bq = lw.W13q;
+    g.B_sf = lw.W13sf;
+    g.b_gs = lw.W13gs;
+    g.a_gs = lw.x_gs;
+    g.out_gs = lw.h_gs;
     g.b_rows_total = (long long)s.E * 2 * s.d_ff;
     g.K = s.d;
     g.N = 2 * s.d_ff;
@@ -622,8 +644,10 @@ static int expert_ffn_mx(const moe_shape_t &s, const WsLayout &L, void *ws, cons
         return rc;
     g.Aq = at<uint8_t>(ws, L.Hq);
     g.A_sf = at<uint8_t>(ws, L.Hsf);
-    g.Bq = W2q;
-    g.B_sf = W2sf;
+    g.Bq = lw.W2q;
+    g.B_sf = lw.W2sf;
+    g.b_gs = lw.W2gs;
+    g.a_gs = lw.h_gs;
     g.b_rows_total = (long long)s.E * s.d;
     g.K = s.d_ff;
     g.N = s.d;
@@ -648,22 +672,27 @@ static int expert_ffn_mx(const moe_shape_t &s, const WsLayout &L, void *ws, cons
 // Shared expert on all T tokens in MXFP8: quantize x, w1/w3 + SwiGLU + MXFP8,
 // w2 with a plain store into out.
 static int shared_expert_mx(const moe_shape_t &s, const WsLayout &L, void *ws, const uint16_t *x,
-                            const uint8_t *W13q, const uint8_t *W13sf, const uint8_t *W2q,
-                            const uint8_t *W2sf, float *out, uint32_t *status, cudaStream_t st)
+                            const LowpWeights &lw, float *out, uint32_t *status, cudaStream_t st)
 {
     const int dfs = s.d_ff_shared;
-    int rc = launch_mx_quantize_rows(x, s.T, s.d, at<uint8_t>(ws, L.xq_s), at<uint8_t>(ws, L.xsf_s),
-                                     st);
+    int rc = lw.fmt == 1 ? launch_nv_quantize_rows(x, s.T, s.d, nullptr, 0, lw.x_gs,
+                                                   at<uint8_t>(ws, L.xq_s), at<uint8_t>(ws, L.xsf_s), st)
+                         : launch_mx_quantize_rows(x, s.T, s.d, at<uint8_t>(ws, L.xq_s),
+                                                   at<uint8_t>(ws, L.xsf_s), st);
     if (rc)
         return rc;
     const int mt = (s.T + kBlockM - 1) / kBlockM;
     GemmArgs g = gemm_base();
     g.mode = EPI_SWIGLU_MX;
+    g.fmt = lw.fmt;
     g.Aq = at<uint8_t>(ws, L.xq_s);
     g.A_sf = at<uint8_t>(ws, L.xsf_s);
     g.a_rows = s.T;
-    g.Bq = W13q;
-    g.B_sf = W13sf;
+    g.Bq = lw.W13s_q;
+    g.B_sf = lw.W13s_sf;
+    g.b_gs = lw.W13s_gs;
+    g.a_gs = lw.x_gs;
+    g.out_gs = lw.h_gs;
     g.b_rows_total = 2LL * dfs;
     g.K = s.d;
     g.N = 2 * dfs;
@@ -680,8 +709,10 @@ static int shared_expert_mx(const moe_shape_t &s, const WsLayout &L, void *ws, c
     g.mode = EPI_STORE_F32;
     g.Aq = at<uint8_t>(ws, L.Hsq);
     g.A_sf = at<uint8_t>(ws, L.Hssf);
-    g.Bq = W2q;
-    g.B_sf = W2sf;
+    g.Bq = lw.W2s_q;
+    g.B_sf = lw.W2s_sf;
+    g.b_gs = lw.W2s_gs;
+    g.a_gs = lw.h_gs;
     g.b_rows_total = s.d;
     g.K = dfs;
     g.N = s.d;
@@ -693,12 +724,13 @@ static int shared_expert_mx(const moe_shape_t &s, const WsLayout &L, void *ws, c
 }
 
 static int forward_mx_impl(const moe_shape_t &s, const WsLayout &L, void *ws, const uint16_t *x,
-                           const uint16_t *Wg, const float *bias, const uint8_t *W13q,
-                           const uint8_t *W13sf, const uint8_t *W2q, const uint8_t *W2sf,
-                           const uint8_t *W13s_q, const uint8_t *W13s_sf, const uint8_t *W2s_q,
-                           const uint8_t *W2s_sf, float *out, float *logits_out,
-                           int32_t *idx_out, uint32_t *status, cudaStream_t st)
+                           const uint16_t *Wg, const float *bias, const LowpWeights &lw,
+                           float *out, float *logits_out, int32_t *idx_out, uint32_t *status,
+                           cudaStream_t st)
 {
+    const uint8_t *W13q = lw.W13q, *W13sf = lw.W13sf, *W2q = lw.W2q, *W2sf = lw.W2sf;
+    const uint8_t *W13s_q = lw.W13s_q, *W13s_sf = lw.W13s_sf, *W2s_q = lw.W2s_q,
+                  *W2s_sf = lw.W2s_sf;
     float *logits = logits_out ? logits_out : at<float>(ws, L.logits);
     int32_t *idx = idx_out ? idx_out : at<int32_t>(ws, L.topk_idx);
     float *w = at<float>(ws, L.topk_w);
@@ -707,7 +739,12 @@ static int forward_mx_impl(const moe_shape_t &s, const WsLayout &L, void *ws, co
     const bool force_pre = (s.flags & MOE_FLAG_FORCE_PREFILL) != 0;
     if (force_dec && s.T > MOE_DECODE_MAX_T)
         return MOE_ERR_UNSUPPORTED;
-    const bool decode = force_dec || (!force_pre && s.T <= MOE_DECODE_DEFAULT_T);
+    // NVFP4 has no decode kernels of its own: small batches take the
+    // tensor-core chain, which also reads each chosen expert's codes once
+    const bool decode =
+        lw.fmt == 0 && (force_dec || (!force_pre && s.T <= MOE_DECODE_DEFAULT_T));
+    if (force_dec && lw.fmt != 0)
+        return MOE_ERR_UNSUPPORTED;
     int rc = route_tokens(s, x, Wg, bias, logits, idx, w, counter, status, st);
     if (rc)
         return rc;
@@ -752,19 +789,22 @@ static int forward_mx_impl(const moe_shape_t &s, const WsLayout &L, void *ws, co
         rc = launch_permute(s, idx, chunk, rank, offsets, nullptr, slot_pos, perm_token, nullptr,
                             (!shared && !det) ? out : nullptr, st);
         if (!rc)
-            rc = launch_mx_gather(s, x, idx, slot_pos, offsets, at<int32_t>(ws, L.tile_start),
-                                  at<uint8_t>(ws, L.xq), at<uint8_t>(ws, L.xsf), st);
+            rc = lw.fmt == 1
+                     ? launch_nv_gather(s, x, idx, slot_pos, offsets, at<int32_t>(ws, L.tile_start),
+                                        lw.x_gs, at<uint8_t>(ws, L.xq), at<uint8_t>(ws, L.xsf), st)
+                     : launch_mx_gather(s, x, idx, slot_pos, offsets, at<int32_t>(ws, L.tile_start),
+                                        at<uint8_t>(ws, L.xq), at<uint8_t>(ws, L.xsf), st);
     }
     if (rc)
         return rc;
     if (shared) {
         StageMark m(MOE_STAGE_SHARED, st);
-        rc = shared_expert_mx(s, L, ws, x, W13s_q, W13s_sf, W2s_q, W2s_sf, out, status, st);
+        rc = shared_expert_mx(s, L, ws, x, lw, out, status, st);
         if (rc)
             return rc;
     }
     float *Y = det ? at<float>(ws, L.Y) : nullptr;
-    rc = expert_ffn_mx(s, L, ws, W13q, W13sf, W2q, W2sf, offsets, perm_token, slot_pos, w, Y, out,
+    rc = expert_ffn_mx(s, L, ws, lw, offsets, perm_token, slot_pos, w, Y, out,
                        status, st);
     if (rc || !det)
         return rc;
@@ -1362,8 +1402,8 @@ int moe_expert_ffn(const moe_shape_t *shape, const moe_bf16_t *x_perm,
     int rc = check_shape(shape);
     if (rc)
         return rc;
-    if (shape->flags & MOE_FLAG_MXFP8)
-        return MOE_ERR_INVALID_ARG;   // bf16 experts: the MXFP8 workspace has no bf16 buffers
+    if (shape->flags & (MOE_FLAG_MXFP8 | MOE_FLAG_NVFP4))
+        return MOE_ERR_INVALID_ARG;   // bf16 experts: block-scaled workspaces have no bf16 buffers
     if (shape->T == 0)
         return MOE_OK;   // empty batch: nothing to read or write
     const moe_shape_t &s = *shape;
@@ -1411,8 +1451,8 @@ int moe_forward(const moe_shape_t *shape, const moe_bf16_t *x, const moe_bf16_t 
     int rc = check_shape(shape);
     if (rc)
         return rc;
-    if (shape->flags & MOE_FLAG_MXFP8)
-        return MOE_ERR_INVALID_ARG;   // bf16 experts: the MXFP8 workspace has no bf16 buffers
+    if (shape->flags & (MOE_FLAG_MXFP8 | MOE_FLAG_NVFP4))
+        return MOE_ERR_INVALID_ARG;   // bf16 experts: block-scaled workspaces have no bf16 buffers
     if (shape->T == 0)
         return MOE_OK;   // empty batch: nothing to read or write
     const moe_shape_t &s = *shape;
@@ -1439,8 +1479,8 @@ int moe_forward_host(const moe_shape_t *shape, const moe_bf16_t *x_host, const m
     int rc = check_shape(shape);
     if (rc)
         return rc;
-    if (shape->flags & MOE_FLAG_MXFP8)
-        return MOE_ERR_INVALID_ARG;   // bf16 experts: the MXFP8 workspace has no bf16 buffers
+    if (shape->flags & (MOE_FLAG_MXFP8 | MOE_FLAG_NVFP4))
+        return MOE_ERR_INVALID_ARG;   // bf16 experts: block-scaled workspaces have no bf16 buffers
     if (shape->T == 0)
         return MOE_OK;   // empty batch: nothing to read or write
     const moe_shape_t &s = *shape;
@@ -1507,8 +1547,8 @@ int moe_forward_expert_choice(const moe_shape_t *shape, const moe_bf16_t *x, con
     int rc = check_shape(shape);
     if (rc)
         return rc;
-    if (shape->flags & MOE_FLAG_MXFP8)
-        return MOE_ERR_INVALID_ARG;   // bf16 experts: the MXFP8 workspace has no bf16 buffers
+    if (shape->flags & (MOE_FLAG_MXFP8 | MOE_FLAG_NVFP4))
+        return MOE_ERR_INVALID_ARG;   // bf16 experts: block-scaled workspaces have no bf16 buffers
     if ((rc = ec_check(*shape)))
         return rc;
     if (shape->T == 0)
@@ -1590,8 +1630,101 @@ int moe_forward_mxfp8(const moe_shape_t *shape, const moe_bf16_t *x, const moe_b
     WsLayout L;
     if ((rc = check_ws(s, ws, ws_bytes, L)))
         return rc;
-    return forward_mx_impl(s, L, ws, x, Wg, bias, W13q, W13sf, W2q, W2sf, W13s_q, W13s_sf, W2s_q,
-                           W2s_sf, out, logits_out, topk_idx_out, status,
+    LowpWeights lw;
+    std::memset(&lw, 0, sizeof lw);
+    lw.fmt = 0;
+    lw.W13q = W13q;
+    lw.W13sf = W13sf;
+    lw.W2q = W2q;
+    lw.W2sf = W2sf;
+    lw.W13s_q = W13s_q;
+    lw.W13s_sf = W13s_sf;
+    lw.W2s_q = W2s_q;
+    lw.W2s_sf = W2s_sf;
+    return forward_mx_impl(s, L, ws, x, Wg, bias, lw, out, logits_out, topk_idx_out, status,
+                           reinterpret_cast<cudaStream_t>(stream));
+}
+
+// NVFP4 GEMMs take 256-element K stages: every contraction length (d, d_ff,
+// d_ff_shared) must be a multiple of 256.
+static int nv_dims_ok(const moe_shape_t &s)
+{
+    return s.d % 256 == 0 && s.d_ff % 256 == 0 && s.d_ff_shared % 256 == 0;
+}
+
+int moe_quantize_experts_nvfp4(const moe_shape_t *shape, const moe_bf16_t *W1,
+                               const moe_bf16_t *W3, const moe_bf16_t *W2, uint8_t *W13q,
+                               uint8_t *W13sf, float *W13_gs, uint8_t *W2q, uint8_t *W2sf,
+                               float *W2_gs, moe_stream_t stream)
+{
+    int rc = check_shape(shape);
+    if (rc)
+        return rc;
+    const moe_shape_t &s = *shape;
+    if (!nv_dims_ok(s))
+        return MOE_ERR_UNSUPPORTED;
+    if (!W1 || !W3 || !W2 || !W13q || !W13sf || !W13_gs || !W2q || !W2sf || !W2_gs || !al16(W1) ||
+        !al16(W3) || !al16(W2) || !al16(W13q) || !al16(W2q) || !al16(W13sf) || !al16(W2sf) ||
+        (reinterpret_cast<uintptr_t>(W13_gs) & 3u) || (reinterpret_cast<uintptr_t>(W2_gs) & 3u))
+        return MOE_ERR_INVALID_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if ((rc = launch_nv_weight_scales(s, W1, W3, W2, W13_gs, W2_gs, st)))
+        return rc;
+    if ((rc = launch_nv_pack_w13(s, W1, W3, W13_gs, W13q, W13sf, st)))
+        return rc;
+    return launch_nv_quantize_rows(W2, (long long)s.E * s.d, s.d_ff, W2_gs, s.d, 0.f, W2q, W2sf,
+                                   st);
+}
+
+int moe_forward_nvfp4(const moe_shape_t *shape, const moe_bf16_t *x, const moe_bf16_t *Wg,
+                      const float *bias, const uint8_t *W13q, const uint8_t *W13sf,
+                      const float *W13_gs, const uint8_t *W2q, const uint8_t *W2sf,
+                      const float *W2_gs, const uint8_t *W13s_q, const uint8_t *W13s_sf,
+                      const float *W13s_gs, const uint8_t *W2s_q, const uint8_t *W2s_sf,
+                      const float *W2s_gs, float x_gs, float h_gs, float *out,
+                      float *logits_out, int32_t *topk_idx_out, uint32_t *status, void *ws,
+                      size_t ws_bytes, moe_stream_t stream)
+{
+    int rc = check_shape(shape);
+    if (rc)
+        return rc;
+    const moe_shape_t &s = *shape;
+    if (!(s.flags & MOE_FLAG_NVFP4) || (s.flags & (MOE_FLAG_HOST_IO | MOE_FLAG_MXFP8)))
+        return MOE_ERR_INVALID_ARG;
+    if (!nv_dims_ok(s))
+        return MOE_ERR_UNSUPPORTED;
+    if (!(x_gs > 0.f) || !(h_gs > 0.f) || !std::isfinite(x_gs) || !std::isfinite(h_gs))
+        return MOE_ERR_INVALID_ARG;
+    if (s.T == 0)
+        return MOE_OK;
+    if (!x || !Wg || !W13q || !W13sf || !W13_gs || !W2q || !W2sf || !W2_gs || !out || !al16(x) ||
+        !al16(Wg) || !al16(W13q) || !al16(W2q) || !al16(W13sf) || !al16(W2sf) || !al16(out))
+        return MOE_ERR_INVALID_ARG;
+    if (s.d_ff_shared > 0 &&
+        (!W13s_q || !W13s_sf || !W13s_gs || !W2s_q || !W2s_sf || !W2s_gs || !al16(W13s_q) ||
+         !al16(W2s_q) || !al16(W13s_sf) || !al16(W2s_sf)))
+        return MOE_ERR_INVALID_ARG;
+    WsLayout L;
+    if ((rc = check_ws(s, ws, ws_bytes, L)))
+        return rc;
+    LowpWeights lw;
+    std::memset(&lw, 0, sizeof lw);
+    lw.fmt = 1;
+    lw.W13q = W13q;
+    lw.W13sf = W13sf;
+    lw.W13gs = W13_gs;
+    lw.W2q = W2q;
+    lw.W2sf = W2sf;
+    lw.W2gs = W2_gs;
+    lw.W13s_q = W13s_q;
+    lw.W13s_sf = W13s_sf;
+    lw.W13s_gs = W13s_gs;
+    lw.W2s_q = W2s_q;
+    lw.W2s_sf = W2s_sf;
+    lw.W2s_gs = W2s_gs;
+    lw.x_gs = x_gs;
+    lw.h_gs = h_gs;
+    return forward_mx_impl(s, L, ws, x, Wg, bias, lw, out, logits_out, topk_idx_out, status,
                            reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -1626,7 +1759,7 @@ int moe_backward(const moe_shape_t *shape, const moe_bf16_t *x, const moe_bf16_t
     if (shape->T == 0)
         return MOE_OK;
     const moe_shape_t &s = *shape;
-    if (!(s.flags & MOE_FLAG_BACKWARD) || (s.flags & (MOE_FLAG_MXFP8 | MOE_FLAG_SIMT_FFN)))
+    if (!(s.flags & MOE_FLAG_BACKWARD) || (s.flags & (MOE_FLAG_MXFP8 | MOE_FLAG_NVFP4 | MOE_FLAG_SIMT_FFN)))
         return MOE_ERR_INVALID_ARG;
     if (!x || !Wg || !W13 || !W13T || !W2T || !dout || !dx || !dW13 || !dW2 || !dWg || !dbias ||
         !al16(x) || !al16(Wg) || !al16(W13) || !al16(W13T) || !al16(W2T) || !al16(dout) ||

@@ -38,6 +38,7 @@ MOE_FLAG_EXPERT_CHOICE = 1 << 7
 MOE_FLAG_SLOT_PRIORITY = 1 << 8
 MOE_FLAG_MXFP8 = 1 << 9
 MOE_FLAG_BACKWARD = 1 << 10
+MOE_FLAG_NVFP4 = 1 << 11
 
 MOE_MAX_E = 256
 MOE_MAX_K = 16
@@ -87,6 +88,9 @@ _SIGS = {
     "moe_permute_static": ([_SHP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P], ctypes.c_int),
     "moe_quantize_experts_mxfp8": ([_SHP, _P, _P, _P, _P, _P, _P, _P, _P], ctypes.c_int),
     "moe_forward_mxfp8": ([_SHP] + [_P] * 16 + [_SZ, _P], ctypes.c_int),
+    "moe_quantize_experts_nvfp4": ([_SHP] + [_P] * 10, ctypes.c_int),
+    "moe_forward_nvfp4": ([_SHP] + [_P] * 15 + [ctypes.c_float, ctypes.c_float] + [_P] * 5 +
+                          [_SZ, _P], ctypes.c_int),
     "moe_pack_backward": ([_SHP, _P, _P, _P, _P, _P], ctypes.c_int),
     "moe_backward": ([_SHP] + [_P] * 20 + [_SZ, _P], ctypes.c_int),
     "moe_route_expert_choice": ([_SHP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P], ctypes.c_int),
@@ -261,6 +265,43 @@ def moe_forward_mxfp8(shape, x, Wg, bias, q, qs, out, logits_out, topk_idx_out, 
     return out
 
 
+def moe_quantize_experts_nvfp4(shape, W1, W3, W2, stream=None) -> dict:
+    """NVFP4 experts from bf16 ones: dict(W13q, W13sf, W13gs, W2q, W2sf, W2gs): packed
+    E2M1 codes (uint8, two per byte), flat E4M3 scale atoms and fp32 global scales [E]."""
+    E, d_ff, d = shape.E, shape.d_ff, shape.d
+    dev = W1.device
+    q = dict(W13q=torch.empty(E, 2 * d_ff, d // 2, dtype=U8, device=dev),
+             W13sf=torch.empty(E * 2 * d_ff * d // 16, dtype=U8, device=dev),
+             W13gs=torch.empty(E, dtype=F32, device=dev),
+             W2q=torch.empty(E, d, d_ff // 2, dtype=U8, device=dev),
+             W2sf=torch.empty(E * d * d_ff // 16, dtype=U8, device=dev),
+             W2gs=torch.empty(E, dtype=F32, device=dev))
+    _check("moe_quantize_experts_nvfp4", lib().moe_quantize_experts_nvfp4(
+        ctypes.byref(shape), _ptr(W1, BF16, "W1"), _ptr(W3, BF16, "W3"), _ptr(W2, BF16, "W2"),
+        _ptr(q["W13q"], U8, "W13q"), _ptr(q["W13sf"], U8, "W13sf"), _ptr(q["W13gs"], F32, "W13gs"),
+        _ptr(q["W2q"], U8, "W2q"), _ptr(q["W2sf"], U8, "W2sf"), _ptr(q["W2gs"], F32, "W2gs"),
+        _stream(stream)))
+    return q
+
+
+def moe_forward_nvfp4(shape, x, Wg, bias, q, qs, x_gs, h_gs, out, logits_out, topk_idx_out,
+                      status, ws, stream=None):
+    """q: routed experts, qs: shared expert (or None), both as moe_quantize_experts_nvfp4
+    gives; x_gs, h_gs: the activations' global encode scales."""
+    qs = qs or {}
+    _check("moe_forward_nvfp4", lib().moe_forward_nvfp4(
+        ctypes.byref(shape), _ptr(x, BF16, "x"), _ptr(Wg, BF16, "Wg"), _ptr(bias, F32, "bias"),
+        _ptr(q["W13q"], U8, "W13q"), _ptr(q["W13sf"], U8, "W13sf"), _ptr(q["W13gs"], F32, "W13gs"),
+        _ptr(q["W2q"], U8, "W2q"), _ptr(q["W2sf"], U8, "W2sf"), _ptr(q["W2gs"], F32, "W2gs"),
+        _ptr(qs.get("W13q"), U8, "W13s_q"), _ptr(qs.get("W13sf"), U8, "W13s_sf"),
+        _ptr(qs.get("W13gs"), F32, "W13s_gs"), _ptr(qs.get("W2q"), U8, "W2s_q"),
+        _ptr(qs.get("W2sf"), U8, "W2s_sf"), _ptr(qs.get("W2gs"), F32, "W2s_gs"),
+        float(x_gs), float(h_gs), _ptr(out, F32, "out"), _ptr(logits_out, F32, "logits_out"),
+        _ptr(topk_idx_out, I32, "topk_idx_out"), _ptr(status, U32, "status"),
+        _ptr(ws, name="ws"), ws.numel(), _stream(stream)))
+    return out
+
+
 def moe_expert_ffn(shape, x_perm, expert_offsets, W13, W2, perm_token, slot_pos, topk_w, y_perm,
                    out, status, ws, stream=None):
     _check("moe_expert_ffn", lib().moe_expert_ffn(
@@ -421,6 +462,48 @@ class MoeLayerMx:
             out = torch.empty(T, self.workload.d, dtype=torch.float32, device=x.device)
         return moe_forward_mxfp8(self.shape(T, flags), x, self.Wg, self.bias, self.q, self.qs, out,
                                  logits_out, topk_idx_out, self.status, self.ws, stream)
+
+
+class MoeLayerNv4:
+    """The layer with NVFP4 experts: quantizes the bf16 experts of `inp` once
+    (moe_quantize_experts_nvfp4) and runs moe_forward_nvfp4 with the
+    activations' global encode scales x_gs and h_gs (calibration constants;
+    1.0 leaves the E4M3 block scales to cover the values alone)."""
+
+    def __init__(self, inp: dict, flags: int = 0, T_max: int | None = None, x_gs: float = 1.0,
+                 h_gs: float = 1.0):
+        w = inp["workload"]
+        self.workload = w
+        self.flags = flags | MOE_FLAG_NVFP4
+        dev = inp["x"].device
+        self.Wg = inp["wg"].contiguous()
+        self.bias = None if inp.get("bias") is None else inp["bias"].to(dev, torch.float32).contiguous()
+        self.x_gs, self.h_gs = float(x_gs), float(h_gs)
+        s = shape_of(w, self.flags)
+        self.q = moe_quantize_experts_nvfp4(s, inp["W1"].contiguous(), inp["W3"].contiguous(),
+                                            inp["W2"].contiguous())
+        self.qs = None
+        if w.d_ff_shared:
+            ss = make_shape(w.T, w.d, w.d_ff_shared, 1, 1)
+            self.qs = moe_quantize_experts_nvfp4(ss, inp["W1s"].contiguous()[None],
+                                                 inp["W3s"].contiguous()[None],
+                                                 inp["W2s"].contiguous()[None])
+        self.T_max = T_max or w.T
+        self.ws = alloc_workspace(shape_of(w, self.flags, T=self.T_max), dev)
+        self.status = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def shape(self, T, flags=None):
+        return shape_of(self.workload, self.flags if flags is None else flags | MOE_FLAG_NVFP4, T=T)
+
+    def forward(self, x, out=None, logits_out=None, topk_idx_out=None, flags=None, stream=None):
+        T = x.shape[0]
+        if T > self.T_max:
+            raise ValueError("T exceeds the workspace's T_max")
+        if out is None:
+            out = torch.empty(T, self.workload.d, dtype=torch.float32, device=x.device)
+        return moe_forward_nvfp4(self.shape(T, flags), x, self.Wg, self.bias, self.q, self.qs,
+                                 self.x_gs, self.h_gs, out, logits_out, topk_idx_out, self.status,
+                                 self.ws, stream)
 
 
 # ---------------------------------------------------------------- instrumentation

@@ -107,6 +107,29 @@ def test_other_entry_points_validation(lib):
     # moe_forward_host needs the HOST_IO workspace flag
     assert lib.moe_forward_host(ctypes.byref(s), FAKE, FAKE, None, FAKE, FAKE, None, None, FAKE,
                                 None, FAKE, 1 << 40, None) == M.MOE_ERR_INVALID_ARG
+    # NVFP4: dimensions must be multiples of 256; the flag is required; the
+    # activations' global scales must be positive and finite
+    f, P = ctypes.c_float, [FAKE] * 6
+    def nv(shape, xgs=1.0, hgs=1.0):
+        return lib.moe_forward_nvfp4(ctypes.byref(shape), FAKE, FAKE, None, *P, *P, f(xgs), f(hgs),
+                                     FAKE, None, None, FAKE, FAKE, 1 << 40, None)
+    assert nv(M.make_shape(64, 128, 256, 8, 2, flags=M.MOE_FLAG_NVFP4)) == M.MOE_ERR_UNSUPPORTED
+    assert nv(M.make_shape(64, 256, 384, 8, 2, flags=M.MOE_FLAG_NVFP4)) == M.MOE_ERR_UNSUPPORTED
+    s4 = M.make_shape(64, 256, 512, 8, 2, flags=M.MOE_FLAG_NVFP4)
+    assert nv(M.make_shape(64, 256, 512, 8, 2)) == M.MOE_ERR_INVALID_ARG
+    assert nv(s4, xgs=0.0) == M.MOE_ERR_INVALID_ARG
+    assert nv(s4, hgs=float("inf")) == M.MOE_ERR_INVALID_ARG
+    assert nv(M.make_shape(64, 256, 512, 8, 2, flags=M.MOE_FLAG_NVFP4 | M.MOE_FLAG_MXFP8)) == \
+        M.MOE_ERR_INVALID_ARG
+    assert lib.moe_quantize_experts_nvfp4(ctypes.byref(s4), FAKE, FAKE, FAKE, FAKE, FAKE, None,
+                                          FAKE, FAKE, FAKE, None) == M.MOE_ERR_INVALID_ARG
+    assert lib.moe_quantize_experts_nvfp4(ctypes.byref(s), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+                                          FAKE, FAKE, FAKE, None) == M.MOE_ERR_UNSUPPORTED
+    # the NVFP4 workspace is smaller than the bf16 one (no bf16 copies of x and h)
+    sb = M.make_shape(4096, 4096, 14336, 8, 2)
+    assert M.moe_workspace_size(s4) > 0
+    assert M.moe_workspace_size(M.make_shape(4096, 4096, 14336, 8, 2, flags=M.MOE_FLAG_NVFP4)) < \
+        M.moe_workspace_size(sb)
     # FORCE_DECODE above the decode limit is unsupported (checked before launching)
     sd = M.make_shape(64, 128, 256, 8, 2, flags=M.MOE_FLAG_FORCE_DECODE)
     ws = M.moe_workspace_size(sd)
