@@ -228,9 +228,9 @@ def run_ours(a, world, rank, local):
         w = replace(w, E=a.experts, name=f"{w.name}@E{a.experts}",
                     capacity=I.capacity_for(w.T, w.k, a.experts) if w.capacity else 0)
     inp = I.make_inputs(w, dev, seed=0)
-    if a.mxfp8:
-        # quantize once, then free the bf16 experts: only the MXFP8 ones stay resident
-        layer = M.MoeLayerMx(inp)
+    if a.mxfp8 or a.nvfp4:
+        # quantize once, then free the bf16 experts: only the block-scaled ones stay resident
+        layer = M.MoeLayerMx(inp) if a.mxfp8 else M.MoeLayerNv4(inp)
         for key in ("W1", "W3", "W2", "W1s", "W3s", "W2s"):
             inp.pop(key, None)
         torch.cuda.empty_cache()
@@ -269,7 +269,8 @@ def run_ours(a, world, rank, local):
     flops, w13_flops, w2_flops = prefill_flops(w, n_kept)
     # MXFP8: the fp8 dense peak, twice the measured sustained bf16 figure (the
     # nominal fp8:bf16 ratio; no fp8 peak is measured on this machine)
-    peak_t = peaks["bf16_tflops_sustained"] * (2.0 if a.mxfp8 else 1.0)
+    ratio = 2.0 if a.mxfp8 else 4.0 if a.nvfp4 else 1.0   # NVFP4: the fp4:bf16 nominal ratio
+    peak_t = peaks["bf16_tflops_sustained"] * ratio
     stage_ms = {k: round(v[0] / v[1], 4) for k, v in stages.items()}
     decode_path = "dec_w13" in stages
     extra = {}
@@ -277,13 +278,15 @@ def run_ours(a, world, rank, local):
         w13_ms = stages["w13"][0] / stages["w13"][1]
         w2_ms = stages["w2"][0] / stages["w2"][1]
         ach = w13_flops / (w13_ms / 1e3) / 1e12
-        if a.mxfp8:
+        if a.mxfp8 or a.nvfp4:
+            fmt = "MXFP8" if a.mxfp8 else "NVFP4"
+            nominal = 4500.0 if a.mxfp8 else 9000.0
             roofline = {"bound": "tensor",
-                        "kernel": "k_gemm_mx<EPI_SWIGLU_MX> (block-scaled MXFP8 w1/w3 GEMM + SwiGLU)",
+                        "kernel": f"k_gemm_mx<EPI_SWIGLU_MX> (block-scaled {fmt} w1/w3 GEMM + SwiGLU)",
                         "achieved": round(ach, 1), "peak": peak_t, "unit": "TFLOP/s",
                         "frac": round(ach / peak_t, 4), "traffic": None,
-                        "peak_source": f"2 x {peak_src} bf16_tflops_sustained (nominal fp8:bf16)",
-                        "frac_of_nominal_4500": round(ach / 4500.0, 4),
+                        "peak_source": f"{ratio:g} x {peak_src} bf16_tflops_sustained (nominal ratio)",
+                        f"frac_of_nominal_{nominal:.0f}": round(ach / nominal, 4),
                         "algorithmic_flops_per_launch": w13_flops, "avg_launch_ms": round(w13_ms, 4)}
         else:
             roofline = {"bound": "tensor",
@@ -354,14 +357,16 @@ def run_ours(a, world, rank, local):
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
         "steps": a.steps, "warmup": a.warmup, "ms_per_step": round(step_ms_max, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "mxfp8 (e4m3 + e8m0/32)" if a.mxfp8 else "bf16",
+        "dtype": "mxfp8 (e4m3 + e8m0/32)" if a.mxfp8 else
+                 "nvfp4 (e2m1 + e4m3/16 + f32 per tensor)" if a.nvfp4 else "bf16",
         "data": "synthetic (seeded, N(0,1) x, N(0,0.02) bf16 weights)",
         "config": {"workload": w.name, "T": w.T, "d_model": w.d, "d_ff": w.d_ff, "E": w.E,
                    "k": w.k, "capacity": w.capacity, "d_ff_shared": w.d_ff_shared,
                    "zipf_s": w.zipf_s, "seed": 0, "parallelism": f"replicas x{world}",
                    "l2": "inputs larger than L2 (expert weights and activations exceed 126 MB)",
                    "output": "fp32 [T, d]",
-                   "experts": "mxfp8 (moe_forward_mxfp8)" if a.mxfp8 else "bf16"},
+                   "experts": "mxfp8 (moe_forward_mxfp8)" if a.mxfp8 else
+                              "nvfp4 (moe_forward_nvfp4)" if a.nvfp4 else "bf16"},
         **extra,
         "stages_ms": stage_ms,
         "profiled_ms_per_step": round(prof_ms, 4),
@@ -651,6 +656,9 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end run")
     ap.add_argument("--mxfp8", action="store_true",
                     help="time the layer on MXFP8 experts (moe_forward_mxfp8) instead of bf16; "
+                         "no extras, no end-to-end run")
+    ap.add_argument("--nvfp4", action="store_true",
+                    help="time the layer on NVFP4 experts (moe_forward_nvfp4) instead of bf16; "
                          "no extras, no end-to-end run")
     a = ap.parse_args(argv)
     if a.warmup < 3 and a.impl == "ours":
