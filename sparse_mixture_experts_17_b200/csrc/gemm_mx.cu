@@ -88,8 +88,6 @@ struct MxArgs {
     float a_gs, out_gs;       // NVFP4: A's global encode scale; h's (EPI_SWIGLU_MX)
 };
 
-enum { FMT_MX8 = 0, FMT_NV4 = 1 };
-
 template <int FMT>
 struct MxCfg {
     static constexpr int BM = 128, BN = 128;

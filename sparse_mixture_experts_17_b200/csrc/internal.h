@@ -105,6 +105,9 @@ enum EpiMode {
                         // sum_c dh * h per row into row_dot (fp32)
 };
 
+// Block-scaled operand formats of launch_gemm_mx (GemmArgs::fmt).
+enum BlockFormat { FMT_MX8 = 0, FMT_NV4 = 1 };
+
 struct GemmArgs {
     int mode;
     // A [a_rows, K] bf16 row-major; B [groups * b_rows_per_group, K] bf16 row-major
@@ -140,11 +143,11 @@ struct GemmArgs {
     // in the atom layout (mxfp8.cuh): A's keyed by m-tile index, B's by row/128
     const uint8_t *Aq, *A_sf, *Bq, *B_sf;
     uint8_t *out_sf;          // EPI_SWIGLU_MX: scales of h, atom layout keyed by m-tile
-    // NVFP4 operands instead (fmt = 1, nvfp4.cuh): packed E2M1 codes, E4M3
+    // NVFP4 operands instead (fmt = FMT_NV4, nvfp4.cuh): packed E2M1 codes, E4M3
     // scales per 16 in the 64-element atom layout; A's global encode scale
     // a_gs, B's per group b_gs[g]; the accumulators are multiplied by
     // 1 / (a_gs * b_gs[g]); EPI_SWIGLU_MX quantizes h with out_gs
-    int fmt;
+    int fmt;                  // FMT_MX8 or FMT_NV4
     const float *b_gs;
     float a_gs, out_gs;
     // EPI_ROUTER_TOPK: top-k outputs [rows, k]; counter_zero (one word) is zeroed

@@ -597,7 +597,7 @@ static int forward_impl(const moe_shape_t &s, const WsLayout &L, void *ws, const
 // ---------------------------------------------------------------- MXFP8 experts
 // Grouped MXFP8 GEMMs over the routed rows: w1/w3 with the SwiGLU + MXFP8
 // epilogue into Hq/Hsf, then w2 with the chosen epilogue.
-// Block-scaled expert weights: MXFP8 (fmt 0) or NVFP4 (fmt 1, with global
+// Block-scaled expert weights: MXFP8 (FMT_MX8) or NVFP4 (FMT_NV4, with global
 // encode scales per expert and the activations' constants x_gs, h_gs).
 struct LowpWeights {
     int fmt;
@@ -675,7 +675,7 @@ static int shared_expert_mx(const moe_shape_t &s, const WsLayout &L, void *ws, c
                             const LowpWeights &lw, float *out, uint32_t *status, cudaStream_t st)
 {
     const int dfs = s.d_ff_shared;
-    int rc = lw.fmt == 1 ? launch_nv_quantize_rows(x, s.T, s.d, nullptr, 0, lw.x_gs,
+    int rc = lw.fmt == FMT_NV4 ? launch_nv_quantize_rows(x, s.T, s.d, nullptr, 0, lw.x_gs,
                                                    at<uint8_t>(ws, L.xq_s), at<uint8_t>(ws, L.xsf_s), st)
                          : launch_mx_quantize_rows(x, s.T, s.d, at<uint8_t>(ws, L.xq_s),
                                                    at<uint8_t>(ws, L.xsf_s), st);
@@ -742,8 +742,8 @@ static int forward_mx_impl(const moe_shape_t &s, const WsLayout &L, void *ws, co
     // NVFP4 has no decode kernels of its own: small batches take the
     // tensor-core chain, which also reads each chosen expert's codes once
     const bool decode =
-        lw.fmt == 0 && (force_dec || (!force_pre && s.T <= MOE_DECODE_DEFAULT_T));
-    if (force_dec && lw.fmt != 0)
+        lw.fmt == FMT_MX8 && (force_dec || (!force_pre && s.T <= MOE_DECODE_DEFAULT_T));
+    if (force_dec && lw.fmt != FMT_MX8)
         return MOE_ERR_UNSUPPORTED;
     int rc = route_tokens(s, x, Wg, bias, logits, idx, w, counter, status, st);
     if (rc)
@@ -789,7 +789,7 @@ static int forward_mx_impl(const moe_shape_t &s, const WsLayout &L, void *ws, co
         rc = launch_permute(s, idx, chunk, rank, offsets, nullptr, slot_pos, perm_token, nullptr,
                             (!shared && !det) ? out : nullptr, st);
         if (!rc)
-            rc = lw.fmt == 1
+            rc = lw.fmt == FMT_NV4
                      ? launch_nv_gather(s, x, idx, slot_pos, offsets, at<int32_t>(ws, L.tile_start),
                                         lw.x_gs, at<uint8_t>(ws, L.xq), at<uint8_t>(ws, L.xsf), st)
                      : launch_mx_gather(s, x, idx, slot_pos, offsets, at<int32_t>(ws, L.tile_start),
@@ -1632,7 +1632,7 @@ int moe_forward_mxfp8(const moe_shape_t *shape, const moe_bf16_t *x, const moe_b
         return rc;
     LowpWeights lw;
     std::memset(&lw, 0, sizeof lw);
-    lw.fmt = 0;
+    lw.fmt = FMT_MX8;
     lw.W13q = W13q;
     lw.W13sf = W13sf;
     lw.W2q = W2q;
@@ -1709,7 +1709,7 @@ int moe_forward_nvfp4(const moe_shape_t *shape, const moe_bf16_t *x, const moe_b
         return rc;
     LowpWeights lw;
     std::memset(&lw, 0, sizeof lw);
-    lw.fmt = 1;
+    lw.fmt = FMT_NV4;
     lw.W13q = W13q;
     lw.W13sf = W13sf;
     lw.W13gs = W13_gs;
