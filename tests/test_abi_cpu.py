@@ -157,3 +157,57 @@ def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     monkeypatch.setattr(M, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError, match="libmoe.so not found"):
         M.lib()
+
+
+def _header_signatures():
+    """{name: [parameter declarations]} of every MOE_API function in moe.h."""
+    import re
+    text = open(M.HEADER).read()
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)   # drop comments
+    sigs = {}
+    for m in re.finditer(r"MOE_API\s+[\w\s\*]*?\b(moe_\w+)\s*\(([^)]*)\)", text):
+        params = [p.strip() for p in m.group(2).split(",")]
+        sigs[m.group(1)] = [] if params == ["void"] else params
+    return sigs
+
+
+def test_binding_signatures_match_header():
+    """Every ctypes signature in the binding has the header's parameter count,
+    and each parameter's kind matches: pointers (and the stream handle) as
+    pointers, size_t / int / float as themselves. A miscounted argument list
+    would pass garbage on the GPU instead of failing here."""
+    sigs = _header_signatures()
+    assert set(sigs) == set(M._SIGS), set(sigs) ^ set(M._SIGS)
+    for name, params in sigs.items():
+        args = M._SIGS[name][0]
+        assert len(args) == len(params), (name, len(args), len(params))
+        for decl, a in zip(params, args):
+            if "*" in decl or decl.startswith("moe_stream_t"):
+                assert a in (ctypes.c_void_p, ctypes.c_char_p) or \
+                    issubclass(a, ctypes._Pointer), (name, decl, a)
+            elif decl.startswith("size_t"):
+                assert a is ctypes.c_size_t, (name, decl, a)
+            elif decl.startswith("float"):
+                assert a is ctypes.c_float, (name, decl, a)
+            elif decl.startswith("int"):
+                assert a is ctypes.c_int, (name, decl, a)
+            else:
+                raise AssertionError(f"unexpected parameter {decl!r} of {name}")
+
+
+@pytest.mark.parametrize("flags", [0, M.MOE_FLAG_DETERMINISTIC, M.MOE_FLAG_MXFP8, M.MOE_FLAG_NVFP4,
+                                   M.MOE_FLAG_BACKWARD, M.MOE_FLAG_EXPERT_CHOICE,
+                                   M.MOE_FLAG_HOST_IO, M.MOE_FLAG_SLOT_PRIORITY])
+@pytest.mark.parametrize("dims", [(256, 512, 8, 2, 0, 0), (512, 256, 64, 6, 0, 256),
+                                  (256, 256, 16, 4, 100, 0)])
+def test_workspace_never_shrinks_with_T(lib, flags, dims):
+    """A layer sizes its workspace once for T_max and runs smaller batches in
+    it, so the size must be non-decreasing in T for every flag."""
+    d, d_ff, E, k, C, dfs = dims
+    prev = 0
+    for T in [1, 2, 3, 16, 17, 100, 127, 128, 129, 255, 256, 257, 1000, 4096, 4097, 16384]:
+        if flags & M.MOE_FLAG_EXPERT_CHOICE and C <= 0:
+            C = 64
+        n = M.moe_workspace_size(M.make_shape(T, d, d_ff, E, k, C, dfs, flags))
+        assert n >= prev, (T, n, prev)
+        prev = n
