@@ -57,7 +57,7 @@ typedef struct CUstream_st *moe_stream_t; /* same object as cudaStream_t; NULL =
 enum {
     MOE_OK = 0,
     MOE_ERR_INVALID_ARG = 1, /* null pointer, bad shape (see moe_shape_t), misaligned pointer */
-    MOE_ERR_UNSUPPORTED = 2, /* valid request that this build does not implement */
+    MOE_ERR_UNSUPPORTED = 2, /* valid request that the library does not implement */
     MOE_ERR_WORKSPACE = 3,   /* ws too small or misaligned */
     MOE_ERR_CUDA = 4,        /* the CUDA runtime refused a launch or query */
     MOE_ERR_NONFINITE = 5,   /* device: a logit row holds NaN, or its maximum is +-inf */

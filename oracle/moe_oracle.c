@@ -25,8 +25,7 @@
  *  [MGA] "Faster writing: run only the chosen experts; uncap the large profile"
  *        (a capacity factor of 0 means uncapped).
  *
- * Readings taken where the pages are silent or garbled (also listed in the
- * design notes of the repository):
+ * Readings taken where the pages are silent or garbled:
  *  R1  top-k is chosen on the fp32 logits. Softmax is strictly increasing in
  *      the logit, so this is the top-k of [MIX]'s probabilities wherever those
  *      are not rounded to equal values. Ties go to the lowest expert index;

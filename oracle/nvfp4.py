@@ -8,8 +8,7 @@ What it follows. The page "Current Bug: CuTeDSLMoERunner produces wrong
 output" runs the routed experts of the layer ("MoE Model Architectures",
 "Mixtral 8x7B", "Sparse MoE Block" and "Expert FFN") as an NVFP4 grouped GEMM
 with per-expert activation scales ("How the pipeline works"). The pages do not
-spell the format out; this module takes NVFP4 as NVIDIA publishes it
-(reading R9 of the design notes):
+spell the format out; this module takes NVFP4 as NVIDIA publishes it:
 
   * element: E2M1, 1 sign, 2 exponent (bias 1) and 1 mantissa bit; the
     magnitudes are 0, 0.5, 1, 1.5, 2, 3, 4, 6 (codes 0..7, sign in bit 3);
