@@ -16,6 +16,7 @@ from __future__ import annotations
 
 import argparse
 import datetime
+import hashlib
 import json
 import math
 import os
@@ -163,6 +164,34 @@ def decode_bytes(w, T, idx):
     return U, expert + other, w13, expert
 
 
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of
+# the headline kernel, from one ncu capture of the full-size launch; the
+# summary, with the command that made it, is under profiles/. `sources_sha`
+# is the SHA-256 of TRAFFIC_SOURCES when the counters were taken: once any of
+# them changes the figure no longer describes the kernel, and the line
+# reports null instead.
+TRAFFIC_SOURCES = ["sparse_mixture_experts_17_b200/csrc/gemm_tc.cu",
+                   "sparse_mixture_experts_17_b200/csrc/common.cuh",
+                   "sparse_mixture_experts_17_b200/csrc/tiles.cuh",
+                   "sparse_mixture_experts_17_b200/csrc/moe_api.cu"]
+TRAFFIC = {}
+
+
+def sources_sha() -> str:
+    h = hashlib.sha256()
+    for f in TRAFFIC_SOURCES:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def headline_traffic(w):
+    t = TRAFFIC.get(w.name)
+    if not t or t["sources_sha"] != sources_sha():
+        return None
+    return t["bytes"]
+
+
 # ---------------------------------------------------------------- CPU baseline (the oracle)
 
 def cpu_oracle_timing(w, budget_s=15.0, steps=1, warmup=0):
@@ -198,6 +227,64 @@ def cpu_oracle_timing(w, budget_s=15.0, steps=1, warmup=0):
 
 
 # ---------------------------------------------------------------- our arm
+
+L2_SCRUB_BYTES = 256 << 20   # twice the 126 MB L2
+
+
+class L2Scrub:
+    """A 256 MB buffer written between timed iterations, so that no iteration
+    finds the previous one's weights in the 126 MB L2."""
+
+    def __init__(self, dev):
+        self.buf = torch.empty(L2_SCRUB_BYTES // 4, dtype=torch.float32, device=dev)
+
+    def __call__(self):
+        self.buf.fill_(1.0)
+
+
+def time_iters_scrubbed(fn, n, stream, scrub, mean=False):
+    """Median (or mean) of n iterations, each timed alone by CUDA events on
+    `stream`, with the L2 scrubbed before each (outside the events)."""
+    evs = []
+    for _ in range(n):
+        scrub()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        evs.append((a, b))
+    torch.cuda.synchronize()
+    t = [a.elapsed_time(b) for a, b in evs]
+    return statistics.mean(t) if mean else statistics.median(t)
+
+
+def layer_work(w, n_kept, experts_used):
+    """Algorithmic FLOPs and bytes of one forward: the FLOPs of the kept rows'
+    expert FFNs, the router and the shared expert; the bytes of the weights of
+    every expert that has a kept row, the shared expert, W_g, x (bf16) and out
+    (fp32). Intermediates (x_perm, H) are not counted: a layer need not write
+    them."""
+    flops, _, _ = prefill_flops(w, n_kept)
+    nbytes = (experts_used * 3 * w.d * w.d_ff * 2 + 3 * w.d * w.d_ff_shared * 2
+              + w.E * w.d * 2 + w.T * w.d * 2 + w.T * w.d * 4)
+    return flops, nbytes
+
+
+def fits_l2(w) -> bool:
+    """Whether one forward's weights and activations could stay in the 126 MB L2."""
+    return (3 * w.E * w.d * w.d_ff * 2 + 3 * w.d * w.d_ff_shared * 2 + w.T * w.d * 6) < 126e6
+
+
+def config_of(w, world, experts="bf16"):
+    """The workload description both arms print."""
+    l2 = ("L2 scrubbed (256 MB written) before each timed forward" if fits_l2(w) else
+          "inputs larger than L2 (expert weights and activations exceed 126 MB)")
+    return {"workload": w.name, "T": w.T, "d_model": w.d, "d_ff": w.d_ff, "E": w.E,
+            "k": w.k, "capacity": w.capacity, "d_ff_shared": w.d_ff_shared,
+            "zipf_s": w.zipf_s, "seed": 0, "parallelism": f"replicas x{world}",
+            "l2": l2, "output": "fp32 [T, d]", "experts": experts}
+
 
 def time_loop(fn, steps, stream):
     s = torch.cuda.Event(enable_timing=True)
@@ -253,7 +340,13 @@ def run_ours(a, world, rank, local):
         launches0 = M.moe_kernel_launches()
         barrier(world)
         torch.cuda.synchronize()
-        step_ms = time_loop(lambda: layer.forward(x, out=out), a.steps, stream)
+        if fits_l2(w):   # K forwards, each timed alone after an L2 scrub
+            scrub = L2Scrub(dev)
+            step_ms = time_iters_scrubbed(lambda: layer.forward(x, out=out), a.steps, stream,
+                                          scrub, mean=True)
+            del scrub
+        else:
+            step_ms = time_loop(lambda: layer.forward(x, out=out), a.steps, stream)
         torch.cuda.synchronize()
         barrier(world)
         launches = M.moe_kernel_launches() - launches0
@@ -270,7 +363,9 @@ def run_ours(a, world, rank, local):
     # MXFP8: the fp8 dense peak, twice the measured sustained bf16 figure (the
     # nominal fp8:bf16 ratio; no fp8 peak is measured on this machine)
     ratio = 2.0 if a.mxfp8 else 4.0 if a.nvfp4 else 1.0   # NVFP4: the fp4:bf16 nominal ratio
-    peak_t = peaks["bf16_tflops_sustained"] * ratio
+    # the kernel is timed inside a step of a few ms in a run of well under a
+    # second: the burst figure is its peak; the sustained one is reported beside
+    peak_t = peaks["bf16_tflops"] * ratio
     stage_ms = {k: round(v[0] / v[1], 4) for k, v in stages.items()}
     decode_path = "dec_w13" in stages
     extra = {}
@@ -285,22 +380,22 @@ def run_ours(a, world, rank, local):
                         "kernel": f"k_gemm_mx<EPI_SWIGLU_MX> (block-scaled {fmt} w1/w3 GEMM + SwiGLU)",
                         "achieved": round(ach, 1), "peak": peak_t, "unit": "TFLOP/s",
                         "frac": round(ach / peak_t, 4), "traffic": None,
-                        "peak_source": f"{ratio:g} x {peak_src} bf16_tflops_sustained (nominal ratio)",
+                        "peak_source": f"{ratio:g} x {peak_src} bf16_tflops (burst; nominal ratio)",
+                        "frac_of_sustained": round(ach / (peaks["bf16_tflops_sustained"] * ratio), 4),
                         f"frac_of_nominal_{nominal:.0f}": round(ach / nominal, 4),
                         "algorithmic_flops_per_launch": w13_flops, "avg_launch_ms": round(w13_ms, 4)}
         else:
             roofline = {"bound": "tensor",
                         "kernel": "k_gemm_tc<256,EPI_SWIGLU> (grouped w1/w3 GEMM + SwiGLU)",
                         "achieved": round(ach, 1), "peak": peak_t, "unit": "TFLOP/s",
-                        "frac": round(ach / peak_t, 4), "traffic": None,
-                        "peak_source": f"{peak_src} bf16_tflops_sustained",
-                        "frac_of_burst_peak": round(ach / peaks["bf16_tflops"], 4),
+                        "frac": round(ach / peak_t, 4), "traffic": headline_traffic(w),
+                        "peak_source": f"{peak_src} bf16_tflops (burst)",
+                        "frac_of_sustained": round(ach / peaks["bf16_tflops_sustained"], 4),
                         "frac_of_nominal_2250": round(ach / 2250.0, 4),
                         "algorithmic_flops_per_launch": w13_flops, "avg_launch_ms": round(w13_ms, 4)}
         extra["w2_tflops"] = round(w2_flops / (w2_ms / 1e3) / 1e12, 1)
         extra["active_tflops"] = round(flops / (step_ms_max / 1e3) / 1e12, 1)
-        extra["active_tflops_frac_measured_sustained"] = round(
-            flops / (step_ms_max / 1e3) / 1e12 / peak_t, 4)
+        extra["active_tflops_frac_burst"] = round(flops / (step_ms_max / 1e3) / 1e12 / peak_t, 4)
         extra["n_kept"] = n_kept
     else:
         idx_now = torch.empty(w.T, w.k, dtype=torch.int32, device=dev)
@@ -334,6 +429,7 @@ def run_ours(a, world, rank, local):
     mxfp8 = None
     nvfp4 = None
     backward = None
+    configs = None
     if a.workload == "prefill" and not a.no_extra:
         decode = run_decode_set(M, w, layer, x, dev, stream, world, peaks)
         graphs = run_graph_set(M, layer, x, dev)
@@ -345,6 +441,12 @@ def run_ours(a, world, rank, local):
                              "mxfp8")
         nvfp4 = run_lowp_set(M, w, inp, x, dev, stream, world, peaks, max(3, a.steps // 2),
                              "nvfp4")
+        # the other workloads, each on its own inputs (the prefill tensors are
+        # released first: the fine-grained workload holds 22.6 GB of experts)
+        del layer, inp, x, out, idx
+        torch.cuda.empty_cache()
+        configs = {name: run_config_set(M, name, dev, stream, world, peaks, a.steps)
+                   for name in ("tiny", "fine_grained", "capacity")}
 
     # ---- CPU baseline: the oracle on host cores (rank 0, N = 1 only)
     cpu = None
@@ -360,13 +462,8 @@ def run_ours(a, world, rank, local):
         "dtype": "mxfp8 (e4m3 + e8m0/32)" if a.mxfp8 else
                  "nvfp4 (e2m1 + e4m3/16 + f32 per tensor)" if a.nvfp4 else "bf16",
         "data": "synthetic (seeded, N(0,1) x, N(0,0.02) bf16 weights)",
-        "config": {"workload": w.name, "T": w.T, "d_model": w.d, "d_ff": w.d_ff, "E": w.E,
-                   "k": w.k, "capacity": w.capacity, "d_ff_shared": w.d_ff_shared,
-                   "zipf_s": w.zipf_s, "seed": 0, "parallelism": f"replicas x{world}",
-                   "l2": "inputs larger than L2 (expert weights and activations exceed 126 MB)",
-                   "output": "fp32 [T, d]",
-                   "experts": "mxfp8 (moe_forward_mxfp8)" if a.mxfp8 else
-                              "nvfp4 (moe_forward_nvfp4)" if a.nvfp4 else "bf16"},
+        "config": config_of(w, world, "mxfp8 (moe_forward_mxfp8)" if a.mxfp8 else
+                            "nvfp4 (moe_forward_nvfp4)" if a.nvfp4 else "bf16"),
         **extra,
         "stages_ms": stage_ms,
         "profiled_ms_per_step": round(prof_ms, 4),
@@ -376,8 +473,6 @@ def run_ours(a, world, rank, local):
         "gpu_launches": int(launches),
         "clocks": clk.summary(),
     }
-    if decode is not None:
-        res["decode"] = decode
     if graphs is not None:
         res["launch_overhead"] = graphs
     if expert_choice is not None:
@@ -388,6 +483,12 @@ def run_ours(a, world, rank, local):
         res["nvfp4"] = nvfp4
     if backward is not None:
         res["backward"] = backward
+    if configs is not None:
+        res["configs"] = configs
+    if decode is not None:
+        res["decode"] = decode
+    if configs is not None or decode is not None:
+        res["summary"] = summarize(res)
     return res
 
 
@@ -441,7 +542,11 @@ def run_graph_set(M, layer, x, dev):
 
 
 def run_decode_set(M, w, layer, x, dev, stream, world, peaks):
+    """Decode (T = 1, 2, 4, 8) on the prefill workload's weights: the median of
+    30 forwards, each timed alone with the L2 scrubbed before it, in GB/s over
+    the bytes the step must read (the chosen experts' weights, W_g, x, out)."""
     decode = {}
+    scrub = L2Scrub(dev)
     for T in I.DECODE_TS:
         xt = x[:T].contiguous()
         it = torch.empty(T, w.k, dtype=torch.int32, device=dev)
@@ -450,9 +555,12 @@ def run_decode_set(M, w, layer, x, dev, stream, world, peaks):
             layer.forward(xt, out=ot, topk_idx_out=it)
         torch.cuda.synchronize()
         U, nbytes, w13_bytes, expert_bytes = decode_bytes(w, T, it)
-        ms = time_loop(lambda: layer.forward(xt, out=ot), 50, stream)
+        ms = time_iters_scrubbed(lambda: layer.forward(xt, out=ot), 30, stream, scrub)
         M.moe_profile_enable(True)
-        time_loop(lambda: layer.forward(xt, out=ot), 50, stream)
+        for _ in range(30):
+            scrub()
+            layer.forward(xt, out=ot)
+        torch.cuda.synchronize()
         M.moe_profile_enable(False)
         st = M.moe_profile_read()
         ms = max_over_ranks(ms, world, dev)
@@ -469,8 +577,86 @@ def run_decode_set(M, w, layer, x, dev, stream, world, peaks):
             "frac_hbm_nominal_8000": round(nbytes / (ms / 1e3) / 1e9 / 8000.0, 4),
             "chosen_expert_GB_s_kernels": round(expert_bytes / ((k13 + k2) / 1e3) / 1e9, 1),
             "w13_kernel_GB_s": round(w13_bytes / (k13 / 1e3) / 1e9, 1),
+            "timing": "median of 30, L2 scrubbed (256 MB) before each",
             "stages_ms": {k: round(v[0] / v[1], 4) for k, v in st.items()}}
+    del scrub
     return decode
+
+
+def run_config_set(M, name, dev, stream, world, peaks, steps):
+    """One of the other measured workloads (tiny, fine_grained, capacity), on its
+    own seeded inputs: ms per forward, tokens/s, active TFLOP/s, and the
+    fraction of the roof max(FLOPs / burst bf16 peak, bytes / HBM peak) it
+    reaches. Workloads whose bytes fit in L2 are timed one forward at a time
+    with the L2 scrubbed before each; the others in a loop (their weights
+    exceed L2)."""
+    w = I.WORKLOADS[name]
+    inp = I.make_inputs(w, dev, seed=0)
+    layer = M.MoeLayer(inp)
+    x = inp["x"]
+    out = torch.empty(w.T, w.d, dtype=torch.float32, device=dev)
+    idx = torch.empty(w.T, w.k, dtype=torch.int32, device=dev)
+    for _ in range(3):
+        layer.forward(x, out=out, topk_idx_out=idx)
+    torch.cuda.synchronize()
+    if int(layer.status.item()) != 0:
+        raise RuntimeError(f"device status {int(layer.status.item())} ({name})")
+    n_kept = routed_kept(idx, w.E, w.capacity)
+    counts = torch.bincount(idx.flatten().long(), minlength=w.E)
+    used = int((counts > 0).sum().item())
+    flops, nbytes = layer_work(w, n_kept, used)
+    small = fits_l2(w)
+    if small:
+        scrub = L2Scrub(dev)
+        ms = time_iters_scrubbed(lambda: layer.forward(x, out=out), max(20, steps), stream, scrub)
+        del scrub
+    else:
+        ms = time_loop(lambda: layer.forward(x, out=out), max(5, steps), stream)
+    ms = max_over_ranks(ms, world, dev)
+    M.moe_profile_enable(True)
+    time_loop(lambda: layer.forward(x, out=out), max(5, steps // 2), stream)
+    M.moe_profile_enable(False)
+    st = M.moe_profile_read()
+    t_compute = flops / (peaks["bf16_tflops"] * 1e12) * 1e3
+    t_bytes = nbytes / (peaks["hbm_gbs"] * 1e9) * 1e3
+    res = {"T": w.T, "d": w.d, "d_ff": w.d_ff, "E": w.E, "k": w.k, "capacity": w.capacity,
+           "d_ff_shared": w.d_ff_shared, "n_kept": n_kept, "experts_used": used,
+           "ms_per_step": round(ms, 4), "tokens_per_s": round(w.T * world / (ms / 1e3), 1),
+           "active_tflops": round(flops / (ms / 1e3) / 1e12, 1),
+           "GB_s": round(nbytes / (ms / 1e3) / 1e9, 1),
+           "roof_ms": round(max(t_compute, t_bytes), 4),
+           "roof_bound": "tensor" if t_compute >= t_bytes else "hbm",
+           "frac_of_roof": round(max(t_compute, t_bytes) / ms, 4),
+           "algorithmic_flops": flops, "algorithmic_bytes": nbytes,
+           "timing": "median of single forwards, L2 scrubbed before each" if small
+                     else "loop; weights exceed L2",
+           "stages_ms": {k: round(v[0] / v[1], 4) for k, v in st.items()}}
+    if "w13" in st:
+        _, f13, f2 = prefill_flops(w, n_kept)
+        res["w13_tflops"] = round(f13 / (st["w13"][0] / st["w13"][1] / 1e3) / 1e12, 1)
+        res["w2_tflops"] = round(f2 / (st["w2"][0] / st["w2"][1] / 1e3) / 1e12, 1)
+    del layer, inp, x, out, idx
+    torch.cuda.empty_cache()
+    return res
+
+
+def summarize(res):
+    """The headline figures of the five workloads in a few hundred characters,
+    printed last in the line."""
+    out = {"C3_prefill": {"ms": res["ms_per_step"], "tok_s": res["value"],
+                          "w13_frac_burst": res["roofline"]["frac"],
+                          "active_tflops": res.get("active_tflops")}}
+    for key, tag in (("tiny", "C1_tiny"), ("fine_grained", "C4_fine_grained"),
+                     ("capacity", "C5_capacity")):
+        c = res.get("configs", {}).get(key)
+        if c:
+            out[tag] = {"ms": c["ms_per_step"], "tok_s": c["tokens_per_s"],
+                        "frac_of_roof": c["frac_of_roof"], "bound": c["roof_bound"]}
+    dec = res.get("decode")
+    if dec:
+        out["C2_decode"] = {k: {"ms": v["ms_per_step"], "frac_hbm": v["frac_hbm_measured"]}
+                            for k, v in dec.items()}
+    return out
 
 
 def run_expert_choice_set(M, w, layer, x, dev, stream, world, peaks, steps):
@@ -620,21 +806,50 @@ def run_backward_set(M, w, inp, layer, dev, stream, world, peaks, steps):
 
 
 def run_reference(a, world, rank):
-    """The oracle as the reference arm: same metric/unit/config, host cores."""
+    """The oracle as the reference arm, timed as it stands on the host cores:
+    the same metric, unit and config as our arm. Each step is one oracle
+    forward of a fixed token sample (router and routing over the sample, the
+    expert FFNs and the combine), sized so that the K timed steps take about a
+    minute; W warm-up steps run first. value = sample tokens / median step."""
     w = I.WORKLOADS[a.workload]
     from oracle import oracle as O
     O.build()
-    rate, cores, sample, n = cpu_oracle_timing(w, budget_s=a.cpu_budget, steps=max(1, a.steps // 10))
-    ms = n / rate * 1e3
+    threads = O.num_threads()
+    gen_dev = "cuda" if torch.cuda.is_available() else "cpu"
+    inp = I.make_inputs(w, gen_dev, seed=0)
+    oi = I.oracle_arrays(inp)
+    del inp
+
+    def step(n):
+        sub = dict(oi)
+        sub["x"] = oi["x"][:n]
+        t0 = time.perf_counter()
+        O.forward(sub)
+        return time.perf_counter() - t0
+
+    # calibrate the sample: about a.ref_step_s seconds per step
+    n = max(1, min(w.T, threads))
+    t = step(n)
+    while t < a.ref_step_s / 2 and n < w.T:
+        n = min(w.T, max(n + 1, int(n * a.ref_step_s / max(t, 1e-3))))
+        t = step(n)
+    for _ in range(a.warmup):
+        step(n)
+    times = [step(n) for _ in range(a.steps)]
+    med = statistics.median(times)
+    rate = n / med
+    sample = (f"first {n} of {w.T} tokens per step; router, top-k, offsets (capacity over the "
+              f"sample) and expert FFN + combine in fp64 on {threads} OpenMP threads; "
+              f"median of {len(times)} steps after {a.warmup} warm-up")
     return {
         "impl": "reference", "metric": METRIC, "value": round(rate, 3), "unit": "tokens/s",
-        "n_gpus": world, "steps": a.steps, "warmup": a.warmup, "ms_per_step": round(ms, 3),
+        "n_gpus": world, "steps": len(times), "warmup": a.warmup, "ms_per_step": round(med * 1e3, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded, N(0,1) x, N(0,0.02) bf16 weights)",
-        "config": {"workload": w.name, "T": w.T, "d_model": w.d, "d_ff": w.d_ff, "E": w.E,
-                   "k": w.k, "capacity": w.capacity, "d_ff_shared": w.d_ff_shared,
-                   "zipf_s": w.zipf_s, "seed": 0, "parallelism": "host cores"},
-        "cpu_baseline": {"value": round(rate, 3), "unit": "tokens/s", "cores": cores,
+        "config": config_of(w, world),
+        "sample_tokens_per_step": n,
+        "timed_region_s": round(sum(times), 3),
+        "cpu_baseline": {"value": round(rate, 3), "unit": "tokens/s", "cores": threads,
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": round(rate, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
@@ -651,6 +866,8 @@ def main(argv=None):
     ap.add_argument("--no-extra", action="store_true", help="skip the decode measurements")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds per oracle sample")
+    ap.add_argument("--ref-step-s", type=float, default=2.5,
+                    help="--impl reference: seconds of oracle work per step")
     ap.add_argument("--tokens", type=int, default=0, help="override T (profiling runs)")
     ap.add_argument("--experts", type=int, default=0, help="override E (profiling runs)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end run")

@@ -115,11 +115,15 @@ void oracle_bf16_to_f64(int64_t n, const uint16_t *src, double *dst)
  * fixing the encoding; reading R7 takes MXFP8 for weights and activations:
  *  - E4M3: sign, 4 exponent bits (bias 7), 3 mantissa bits, subnormals
  *    m/8 * 2^-6, largest finite 448, no infinities, S.1111.111 = NaN;
- *  - the scale of a block is 2^X with X the smallest integer in [-127, 127]
- *    such that max|v| <= 448 * 2^X (so no element saturates); E8M0 code
- *    X + 127;
+ *  - the shared scale of a block is 2^X with X = floor(log2(max|v|)) - 8,
+ *    8 being the exponent of E4M3's largest normal power of two (the
+ *    standard's conversion of a vector of scalars to an MX block), clamped
+ *    to the E8M0 range [-127, 127]; an all-zero block takes X = -127. E8M0
+ *    code X + 127;
  *  - each element is v * 2^-X rounded to the nearest E4M3 value, ties to
- *    even (the sign of a zero result is the sign of v). */
+ *    even, saturating at 448: the block maximum lands in [256, 512), and
+ *    scaled magnitudes of 464 and above clamp to 448 (the standard's
+ *    saturating conversion). The sign of a zero result is the sign of v. */
 double oracle_e4m3_decode(int code)
 {
     const int s = (code >> 7) & 1, e = (code >> 3) & 15, m = code & 7;
@@ -159,12 +163,19 @@ int oracle_e4m3_encode(double v)
     return code | (signbit(v) ? 0x80 : 0);
 }
 
-/* Shared exponent X of a block with maximum magnitude amax. */
+/* Shared exponent X of a block with maximum magnitude amax:
+ * floor(log2(amax)) - 8, clamped to [-127, 127]; -127 for amax = 0. */
 int oracle_mx_scale_exp(double amax)
 {
-    int X = -127;
-    while (X < 127 && amax > ldexp(448.0, X))
-        ++X;
+    if (!(amax > 0.0))
+        return -127;
+    int e;
+    (void)frexp(amax, &e);   /* amax = f * 2^e with 0.5 <= f < 1: floor(log2 amax) = e - 1 */
+    int X = e - 1 - 8;
+    if (X < -127)
+        X = -127;
+    if (X > 127)
+        X = 127;
     return X;
 }
 

@@ -2,12 +2,14 @@
 // (power-of-two) scale per 32 consecutive elements along the contraction
 // dimension (OCP "Microscaling (MX) Formats" v1.0).
 //
-// The scale of a block is 2^X with X the smallest integer in [-127, 127] such
-// that max|v| <= 448 * 2^X (448 is the largest finite E4M3 value), so no
-// element saturates; its E8M0 code is X + 127. Elements are v * 2^-X rounded
-// to the nearest E4M3 value, ties to even (cvt.rn.satfinite). Multiplying by
-// a power of two is exact here, so the encoding is a function of the fp32
-// inputs alone.
+// The shared scale of a block is 2^X with X = floor(log2(max|v|)) - 8 (8 is
+// the exponent of E4M3's largest normal binade), clamped to [-127, 127]; an
+// all-zero block takes -127. Its E8M0 code is X + 127. Elements are v * 2^-X
+// rounded to the nearest E4M3 value, ties to even, saturating at 448
+// (cvt.rn.satfinite): the block maximum scales into [256, 512), so scaled
+// magnitudes of 464 and above clamp to 448, as the standard's conversion
+// does. Multiplying by a power of two is exact here, so the encoding is a
+// function of the fp32 inputs alone.
 #pragma once
 
 #include <cuda_fp8.h>
@@ -17,15 +19,15 @@ namespace moe {
 
 constexpr int kMxBlock = 32;
 
-// X for a block maximum: with amax = 1.m * 2^E (normal), amax <= 1.75 * 2^(8+X)
-// iff X >= E - 8 + (m > 0.75). Zero and fp32 subnormals (< 2^-126) take -127.
+// X for a block maximum amax = 1.m * 2^E (normal): E - 8, the unbiased
+// exponent field minus 8. Zero and fp32 subnormals (< 2^-126, where E - 8 is
+// below -127 anyway) take -127.
 __device__ __forceinline__ int mx_scale_exp(float amax)
 {
     const uint32_t b = __float_as_uint(amax) & 0x7fffffffu;
     if (b < 0x00800000u)
         return -127;
-    const int E = (int)(b >> 23) - 127;
-    const int X = E - 8 + ((b & 0x007fffffu) > 0x00600000u ? 1 : 0);
+    const int X = (int)(b >> 23) - 127 - 8;
     return max(-127, min(127, X));
 }
 

@@ -51,6 +51,10 @@ def _weights(E, d_ff, d, kind, seed):
         W3[0, 3, :] = 1e-39                              # bf16 subnormals
         W2[0, 1, :32] = 3e38                             # near the bf16 maximum
         W1[-1, 5, :] = torch.linspace(-448, 448, d, device="cuda")  # exact E4M3 grid points
+        # blocks whose maximum scales past 448: elements of 464 and above clamp
+        W1[-1, 6, 0::2] = 500.0
+        W1[-1, 6, 1::2] = 470.0
+        W3[-1, 7, :] = torch.linspace(-511, 511, d, device="cuda")
     return [W.to(torch.bfloat16).contiguous() for W in (W1, W3, W2)]
 
 

@@ -1,8 +1,9 @@
 """Pins of the oracle's MXFP8 arithmetic (OCP "Microscaling (MX) Formats"
 v1.0: E4M3 elements, one E8M0 power-of-two scale per 32 elements) to things
 other than itself: the format's closed-form values, torch's float8_e4m3fn
-conversions, a brute-force nearest-even search over all codes, the scale
-rule's defining inequalities, and a numpy composition of the quantized
+conversions, a brute-force nearest-even search over all codes, the shared
+exponent rule's defining inequalities and hand-worked blocks (saturation
+included), and a numpy composition of the quantized
 expert FFN (CPU only)."""
 import math
 
@@ -69,24 +70,34 @@ def test_e4m3_encode_matches_torch(orc):
 
 
 def test_mx_scale_exponent_rule(orc):
+    """OCP MX v1.0's conversion of a block: the shared exponent is
+    floor(log2(max|v|)) - emax_elem, emax_elem = 8 for E4M3 (its largest
+    normal binade is [256, 512)), clamped to E8M0's [-127, 127]. Pinned by its
+    defining inequality 2^(8+X) <= amax < 2^(9+X) and by hand-worked values."""
     rng = np.random.default_rng(2)
     for amax in np.concatenate([np.exp2(rng.uniform(-60, 60, 500)), [448.0, 448.0 * 2 ** -3,
                                                                         448.0 * 2 ** 5 + 1e-9]]):
         X = orc.mx_scale_exp(amax)
-        assert amax <= 448.0 * 2.0 ** X                 # no element saturates
-        assert amax > 448.0 * 2.0 ** (X - 1)            # the smallest such power of two
+        assert 2.0 ** (8 + X) <= amax < 2.0 ** (9 + X), (amax, X)
+    # hand-worked: the binade [256, 512) is X = 0, whatever saturates in it
+    for amax, X in ((256.0, 0), (448.0, 0), (480.0, 0), (np.nextafter(512.0, 0), 0), (512.0, 1),
+                    (255.0, -1), (1.0, -8), (0.75, -9), (2.0 ** -119, -127), (3e38, 119)):
+        assert orc.mx_scale_exp(amax) == X, (amax, X)
+    # clamped to the E8M0 range; an all-zero block takes the smallest scale
+    assert orc.mx_scale_exp(2.0 ** -120) == -127
     assert orc.mx_scale_exp(0.0) == -127
     assert orc.mx_scale_exp(1e-45) == -127
-    assert orc.mx_scale_exp(448.0) == 0 and orc.mx_scale_exp(np.nextafter(448.0, 1e9)) == 1
 
 
 def test_mx_quantize_error_bound_and_identity(orc):
     rng = np.random.default_rng(3)
     a = rng.normal(0, 1, (16, 256)) * np.exp2(rng.integers(-20, 20, (16, 1)))
     a[3, 32:64] = 0.0                                   # an all-zero block
+    a[5, 64:96] = np.linspace(-505.0, 505.0, 32) * 2.0 ** -7   # saturating block
     codes, scales = orc.mx_quantize(a)
     back = orc.mx_dequantize(codes, scales)
     X = scales.astype(np.int64) - 127
+    n_sat = 0
     for r in range(16):
         for b in range(8):
             blk, q = a[r, 32 * b:32 * b + 32], back[r, 32 * b:32 * b + 32]
@@ -94,16 +105,29 @@ def test_mx_quantize_error_bound_and_identity(orc):
                 assert (q == 0).all()
                 continue
             assert X[r, b] == orc.mx_scale_exp(np.abs(blk).max())
-            # |error| <= half a spacing: 2^-4 relative in a binade (3 mantissa
-            # bits), or half the subnormal step 2^(X-10) near zero
+            top = 448.0 * 2.0 ** X[r, b]
+            sat = np.abs(blk) >= 464.0 * 2.0 ** X[r, b]   # round to nearest past 448: clamp
+            n_sat += int(sat.sum())
+            assert (q[sat] == np.sign(blk[sat]) * top).all()
+            # elsewhere |error| <= half a spacing: 2^-4 relative in a binade (3
+            # mantissa bits), or half the subnormal step 2^(X-10) near zero
             bound = np.maximum(np.abs(blk) * 2.0 ** -4, 2.0 ** (X[r, b] - 10))
-            assert (np.abs(q - blk) <= bound).all()
-    # values already on the grid come back unchanged (a block whose maximum
-    # rounded down may take a smaller scale, with the same values)
+            assert (np.abs(q - blk)[~sat] <= bound[~sat]).all()
+    assert n_sat >= 2                                   # the saturating block did saturate
+    # values already on the grid come back unchanged: their block maximum
+    # stays in the same binade, so the scale and the codes repeat
     assert (orc.mx_dequantize(*orc.mx_quantize(back)) == back).all()
     # a block that reaches 448 * 2^X keeps its scale and codes exactly
     c1, s1 = orc.mx_quantize(back * 0 + np.where(np.arange(256) % 32 == 0, 448.0, 1.0))
     assert (s1 == 127).all() and (c1[:, ::32] == 0x7E).all() and (c1[:, 1::32] == 0x38).all()
+    # hand-worked saturation: a block of maximum 500 takes X = 0, and 500,
+    # 470 and 464 clamp to 448 (code 0x7E) while 463 rounds to 448 and 440 to 448
+    # (spacing 32 in [256, 512)), 430 to 416 (0x7D)
+    blk = np.zeros((1, 32))
+    blk[0, :7] = [500.0, 470.0, 464.0, 463.0, 440.0, 430.0, -500.0]
+    c2, s2 = orc.mx_quantize(blk)
+    assert s2[0, 0] == 127
+    assert c2[0, :7].tolist() == [0x7E, 0x7E, 0x7E, 0x7E, 0x7E, 0x7D, 0xFE]
 
 
 def test_layer_mx_mode_vs_numpy_composition(orc):
