@@ -62,7 +62,9 @@ enum {
     MOE_ERR_CUDA = 4,        /* the CUDA runtime refused a launch or query */
     MOE_ERR_NONFINITE = 5,   /* device: a logit row holds NaN, or its maximum is +-inf */
     MOE_ERR_BAD_EXPERT = 6,  /* device: an expert id outside [0,E) or repeated within a token */
-    MOE_ERR_TIMEOUT = 7      /* device: a pipeline wait gave up (the kernel returned, no hang) */
+    MOE_ERR_TIMEOUT = 7,     /* device: a pipeline wait gave up (the kernel returned, no hang) */
+    MOE_ERR_CHECK = 8        /* device: a dispatch consistency check failed (MOE_FLAG_DEBUG_CHECKS,
+                                moe_check_dispatch) */
 };
 
 /* Flags (moe_shape_t.flags). */
@@ -87,8 +89,20 @@ enum {
     MOE_FLAG_MXFP8 = 1 << 9,         /* workspace for moe_forward_mxfp8 (MXFP8 experts); the
                                         bf16 layer calls reject it */
     MOE_FLAG_BACKWARD = 1 << 10,     /* workspace also sized for moe_backward */
-    MOE_FLAG_NVFP4 = 1 << 11         /* workspace for moe_forward_nvfp4 (NVFP4 experts); the
+    MOE_FLAG_NVFP4 = 1 << 11,        /* workspace for moe_forward_nvfp4 (NVFP4 experts); the
                                         bf16 layer calls reject it */
+    MOE_FLAG_DEBUG_CHECKS = 1 << 12  /* moe_permute and the prefill moe_forward also check the
+                                        dispatch they built (moe_check_dispatch) and flag
+                                        MOE_ERR_CHECK; the workspace holds one int32 per
+                                        assignment more. A build with -DMOE_DEBUG sets it on
+                                        every call */,
+    MOE_FLAG_TEST_TIMEOUT = 1 << 13  /* test only, honoured by moe_expert_ffn alone: its w1/w3
+                                        GEMM runs on the single-SM tensor-core kernel with a
+                                        producer that issues no loads and pipeline waits
+                                        bounded at 50 ms, so every CTA gives up its first wait,
+                                        flags MOE_ERR_TIMEOUT, frees its tensor memory and
+                                        returns with nothing in flight. Exercises the bounded
+                                        waits; the call's results are meaningless */
 };
 
 #define MOE_MAX_E 256
@@ -431,11 +445,31 @@ MOE_API int moe_backward(const moe_shape_t *shape, const moe_bf16_t *x, const mo
                          float *dlogits, uint32_t *status, void *ws, size_t ws_bytes,
                          moe_stream_t stream);
 
+/* Consistency check of a dispatch (the debug bounds checks of the permutation,
+ * which the pages do not describe; they guard the offsets bug class of
+ * "Current Bug: CuTeDSLMoERunner produces wrong output", "Root Cause:
+ * scale_a layout doesn't match expert_offsets"). Reads, never writes, the
+ * dispatch; sets the bit (1u << MOE_ERR_CHECK) of *status when any of these
+ * fails, and (1u << MOE_ERR_BAD_EXPERT) for an id outside [0, E):
+ *   expert_offsets[0] = 0, nondecreasing, expert_offsets[E] = *n_kept <= T*k,
+ *   and with a capacity C > 0 no expert holds more than C rows;
+ *   every kept slot_pos[t, j] lies in [expert_offsets[e], expert_offsets[e+1])
+ *   of its expert e = topk_idx[t, j], and perm_token of that row is t;
+ *   without a capacity no assignment is dropped (slot_pos = -1 only with C > 0;
+ *   any other negative value fails);
+ *   every row in [0, n_kept) is the slot of exactly one assignment.
+ *   Every read is bounds-checked first, so a corrupt dispatch raises the
+ *   status bit and nothing else. The workspace must be sized with
+ *   MOE_FLAG_DEBUG_CHECKS in shape->flags (one int32 per assignment). */
+MOE_API int moe_check_dispatch(const moe_shape_t *shape, const int32_t *topk_idx,
+                               const int32_t *expert_offsets, const int32_t *slot_pos,
+                               const int32_t *perm_token, const int32_t *n_kept, uint32_t *status,
+                               void *ws, size_t ws_bytes, moe_stream_t stream);
+
 /* moe_permute without a workspace, for callers that cannot allocate device
- * memory: code running while a stream is captured in global capture mode
- * (where cudaMalloc is refused), engines that reserve all device memory for
- * their own pool, and paths that cannot pay for cudaMalloc/cudaFree (cudaFree
- * synchronises the device). The pages have no counterpart of this call.
+ * memory: engines that reserve all device memory for their own pool, and
+ * paths that cannot pay for cudaMalloc/cudaFree (cudaFree synchronises the
+ * device). The pages have no counterpart of this call.
  *   Arguments, outputs and results are those of moe_permute (bit-identical),
  *   minus ws/ws_bytes: the scratch is one fixed 4 MiB array inside the
  *   library's device image, held on every GPU that loads the library until
@@ -443,8 +477,10 @@ MOE_API int moe_backward(const moe_shape_t *shape, const moe_bf16_t *x, const mo
  *   MOE_ERR_UNSUPPORTED and launch nothing; every shape with T*k <= 262144
  *   and T <= 262144 fits.
  *   The call allocates nothing. Its first call on a device looks up the
- *   array's device address (cudaGetSymbolAddress, with that device current);
- *   make that first call before any stream capture.
+ *   array's device address (cudaGetSymbolAddress, with that device current)
+ *   and caches it with the device's context; make that first call before any
+ *   stream capture. After a device reset the next call looks the address up
+ *   again.
  *   All calls share the one array and each call clears what must start at
  *   zero, so calls that overlap on the GPU (other streams, other host threads)
  *   race and corrupt each other's results: order them on one stream. */

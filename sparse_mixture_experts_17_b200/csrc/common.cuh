@@ -114,9 +114,9 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
 // Wait for the phase of `bar` with the given parity to complete. Returns false
 // (after flagging MOE_ERR_TIMEOUT and raising *abort) if it does not complete
-// within kWaitLimitNs, or if another role of the CTA has already aborted.
+// within limit_ns, or if another role of the CTA has already aborted.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
-                                          uint32_t *status)
+                                          uint32_t *status, uint64_t limit_ns = kWaitLimitNs)
 {
 #pragma unroll 1
     for (int i = 0; i < 128; ++i)
@@ -129,7 +129,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
             return true;
         if (*abort)
             return false;
-        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        if (globaltimer_ns() - t0 > limit_ns) {
             *abort = 1;
             flag_status(status, MOE_ERR_TIMEOUT);
             return false;

@@ -482,4 +482,92 @@ int launch_pack_w13(int E, int d_ff, int d, const uint16_t *W1, const uint16_t *
     return launched();
 }
 
+
+// ---------------------------------------------------------------- dispatch consistency checks
+// Debug bounds checks of a dispatch (moe_check_dispatch): three passes, each
+// of which bounds-checks every index before it reads with it.
+//   pass 1: zero the per-row counters; one thread checks the offsets
+//   pass 2: one thread per assignment: id range, the row inside its expert's
+//           segment, perm_token of the row, and one count on the row
+//   pass 3: every row below n_kept was counted exactly once
+__global__ void k_dbg_offsets(const int32_t *__restrict__ offsets, const int32_t *__restrict__ n_kept,
+                              int E, long long N, int capacity, int32_t *__restrict__ seen,
+                              uint32_t *status)
+{
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < N;
+         i += (long long)gridDim.x * blockDim.x)
+        seen[i] = 0;
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        bool ok = offsets[0] == 0;
+        for (int e = 0; e < E; ++e) {
+            const int32_t a = offsets[e], b = offsets[e + 1];
+            ok = ok && a <= b && (capacity <= 0 || b - a <= capacity);
+        }
+        const int32_t nk = *n_kept;
+        ok = ok && offsets[E] == nk && nk >= 0 && (long long)nk <= N;
+        if (!ok)
+            flag_status(status, MOE_ERR_CHECK);
+    }
+}
+
+__global__ void k_dbg_assign(const int32_t *__restrict__ idx, const int32_t *__restrict__ slot_pos,
+                             const int32_t *__restrict__ perm_token,
+                             const int32_t *__restrict__ offsets, int T, int k, int E, int capacity,
+                             int32_t *__restrict__ seen, uint32_t *status)
+{
+    const long long N = (long long)T * k;
+    for (long long a = blockIdx.x * (long long)blockDim.x + threadIdx.x; a < N;
+         a += (long long)gridDim.x * blockDim.x) {
+        const int e = idx[a];
+        const int32_t pos = slot_pos[a];
+        const int t = (int)(a / k);
+        if (e < 0 || e >= E) {
+            flag_status(status, MOE_ERR_BAD_EXPERT);
+            continue;
+        }
+        if (pos == -1) {
+            if (capacity <= 0)
+                flag_status(status, MOE_ERR_CHECK);   // nothing is dropped without a capacity
+            continue;
+        }
+        if (pos < 0 || (long long)pos >= N) {
+            flag_status(status, MOE_ERR_CHECK);
+            continue;
+        }
+        if (pos < offsets[e] || pos >= offsets[e + 1] || perm_token[pos] != t)
+            flag_status(status, MOE_ERR_CHECK);
+        atomicAdd(seen + pos, 1);
+    }
+}
+
+__global__ void k_dbg_rows(const int32_t *__restrict__ seen, const int32_t *__restrict__ n_kept,
+                           long long N, uint32_t *status)
+{
+    const long long nk = min((long long)max(*n_kept, 0), N);
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < nk;
+         i += (long long)gridDim.x * blockDim.x)
+        if (seen[i] != 1)
+            flag_status(status, MOE_ERR_CHECK);
+}
+
+int launch_check_dispatch(const moe_shape_t &s, const int32_t *idx, const int32_t *offsets,
+                          const int32_t *slot_pos, const int32_t *perm_token,
+                          const int32_t *n_kept, int32_t *seen, uint32_t *status, cudaStream_t st)
+{
+    const long long N = (long long)s.T * s.k;
+    if (N == 0)
+        return MOE_OK;
+    const int grid = (int)std::min<long long>((N + 255) / 256, 4LL * num_sms());
+    k_dbg_offsets<<<grid, 256, 0, st>>>(offsets, n_kept, s.E, N, s.capacity, seen, status);
+    int rc = launched();
+    if (rc)
+        return rc;
+    k_dbg_assign<<<grid, 256, 0, st>>>(idx, slot_pos, perm_token, offsets, s.T, s.k, s.E,
+                                       s.capacity, seen, status);
+    if ((rc = launched()))
+        return rc;
+    k_dbg_rows<<<grid, 256, 0, st>>>(seen, n_kept, N, status);
+    return launched();
+}
+
 } // namespace moe

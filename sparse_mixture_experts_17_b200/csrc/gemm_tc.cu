@@ -82,6 +82,10 @@ struct TcArgs {
     int32_t *hist_mt_row0, *hist_mt_group, *hist_num_mt, *hist_mt2_row0, *hist_mt2_group,
         *hist_num_mt2;
     int capacity;
+    // bound of every pipeline wait; `starve` (test only): the producer issues
+    // no loads, so the first wait on a full stage runs out and every role unwinds
+    unsigned long long wait_ns;
+    int starve;
 };
 
 // Shared memory of the histogram folded into the router (E <= 64): per-warp
@@ -441,7 +445,7 @@ __global__ void __launch_bounds__(192, 1)
     const long long total = (long long)num_mt * p.n_tiles;
 
     if (warp == 0) {
-        if (lane == 0) {   // ---------------- TMA producer
+        if (lane == 0 && !p.starve) {   // ---------------- TMA producer
             uint32_t it = 0;
             for (long long tile = blockIdx.x; tile < total; tile += gridDim.x) {
                 int m_idx, n_idx;
@@ -456,7 +460,7 @@ __global__ void __launch_bounds__(192, 1)
                 for (int kb = 0; kb < nkb; ++kb, ++it) {
                     const int s = it % C::STAGES;
                     const uint32_t ph = (it / C::STAGES) & 1u;
-                    if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag, p.status)) {
+                    if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag, p.status, p.wait_ns)) {
                         ok = false;
                         break;
                     }
@@ -481,7 +485,7 @@ __global__ void __launch_bounds__(192, 1)
                 const uint32_t IDESC = half ? IDESC64 : IDESC128;
                 const int grp = p.mt_group ? (p.mt_group[m_idx] & ~kHalfTileBit) : 0;
                 const int nkb = p.grp_kb0 ? p.grp_nkb[grp] : p.kblocks;
-                if (!mbar_wait(&tempty[b], aph ^ 1u, abort_flag, p.status))
+                if (!mbar_wait(&tempty[b], aph ^ 1u, abort_flag, p.status, p.wait_ns))
                     break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + b * BN;
@@ -489,7 +493,7 @@ __global__ void __launch_bounds__(192, 1)
                 for (int kb = 0; kb < nkb; ++kb, ++it) {
                     const int s = it % C::STAGES;
                     const uint32_t ph = (it / C::STAGES) & 1u;
-                    if (!mbar_wait(&full[s], ph, abort_flag, p.status)) {
+                    if (!mbar_wait(&full[s], ph, abort_flag, p.status, p.wait_ns)) {
                         ok = false;
                         break;
                     }
@@ -519,7 +523,7 @@ __global__ void __launch_bounds__(192, 1)
             const bool half = (gword & kHalfTileBit) != 0;
             const long long row_end = p.seg_offsets ? p.seg_offsets[grp + 1] : p.rows_valid;
             const uint32_t b = local & 1u, aph = (local >> 1) & 1u;
-            const bool got = mbar_wait(&tfull[b], aph, abort_flag, p.status);
+            const bool got = mbar_wait(&tfull[b], aph, abort_flag, p.status, p.wait_ns);
             // the folded histogram's named barriers need every epilogue warp on
             // every tile, so a warp whose wait gave up keeps going without work
             if (!got && !(MODE == EPI_ROUTER_TOPK && p.hist_chunk))
@@ -737,6 +741,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
 
 // ---------------------------------------------------------------- host side
 
+// Wait bound of the test-only starved launch (GemmArgs::test_starve).
+constexpr unsigned long long kTestWaitLimitNs = 50000000ull;
+
 static PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
 {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -838,6 +845,8 @@ static int launch_tc_impl(const GemmArgs &g, cudaStream_t st)
     p.hist_mt2_group = g.hist_mt2_group;
     p.hist_num_mt2 = g.hist_num_mt2;
     p.capacity = g.capacity;
+    p.starve = g.test_starve;
+    p.wait_ns = g.test_starve ? kTestWaitLimitNs : kWaitLimitNs;
 
     // the router with the folded histogram also needs its tile-histogram area
     constexpr int SMEM = C::SMEM_BYTES + (MODE == EPI_ROUTER_TOPK ? (int)sizeof(RouterHistSmem) : 0);

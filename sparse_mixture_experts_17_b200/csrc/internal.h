@@ -51,6 +51,7 @@ struct WsLayout {
     size_t xq, xsf, Hq, Hsf, xq_s, xsf_s, Hsq, Hssf;   // MXFP8 operands
     size_t dec_xdq, dec_H32;                             // MXFP8 decode
     size_t tile_start;                                   // first m-tile of each expert
+    size_t dbg_seen;                                     // dispatch checks: count per row
     // backward pass
     size_t GU, dYw, dGU, row_dot, pstart, kb0, nkb, mtk1_row0, mtk1_group, mtk2_row0,
         mtk2_group, dYwT, HT, dGUT, XpT, dl, dwg_part;
@@ -64,6 +65,9 @@ struct WsLayout {
 };
 
 WsLayout ws_layout(const moe_shape_t &s);
+
+// The shape rules every entry point applies (MOE_OK or MOE_ERR_INVALID_ARG).
+int check_shape(const moe_shape_t *s);
 
 // ---- routing / dispatch (dispatch.cu)
 int launch_router_simt(const moe_shape_t &s, const uint16_t *x, const uint16_t *Wg,
@@ -87,6 +91,21 @@ int launch_combine(const moe_shape_t &s, const float *y_perm, const int32_t *slo
                    const float *topk_w, const float *shared_out, float *out, cudaStream_t st);
 int launch_pack_w13(int E, int d_ff, int d, const uint16_t *W1, const uint16_t *W3,
                     uint16_t *W13, cudaStream_t st);
+// Debug consistency checks of a dispatch (seen: T*k int32 of scratch).
+int launch_check_dispatch(const moe_shape_t &s, const int32_t *idx, const int32_t *offsets,
+                          const int32_t *slot_pos, const int32_t *perm_token,
+                          const int32_t *n_kept, int32_t *seen, uint32_t *status, cudaStream_t st);
+// Whether the dispatch checks run: MOE_FLAG_DEBUG_CHECKS, or every call in a
+// build compiled with -DMOE_DEBUG.
+inline bool debug_checks(const moe_shape_t &s)
+{
+#ifdef MOE_DEBUG
+    (void)s;
+    return true;
+#else
+    return (s.flags & MOE_FLAG_DEBUG_CHECKS) != 0;
+#endif
+}
 
 // ---- grouped GEMMs (gemm_tc.cu: tcgen05 + TMA; gemm_simt.cu: CUDA cores)
 enum EpiMode {
@@ -170,6 +189,10 @@ struct GemmArgs {
     int32_t *hist_mt_row0, *hist_mt_group, *hist_num_mt, *hist_mt2_row0, *hist_mt2_group,
         *hist_num_mt2;
     int capacity;
+    // test only (single-SM tensor-core kernel): the producer issues no loads and
+    // the pipeline waits give up after 50 ms, so the launch returns with
+    // MOE_ERR_TIMEOUT flagged and nothing in flight
+    int test_starve;
 };
 
 int launch_gemm_tc(const GemmArgs &g, cudaStream_t st);

@@ -78,7 +78,7 @@ int launch_dec_router(const moe_shape_t &s, const uint16_t *x, const uint16_t *W
 
 static bool dim_ok(int v) { return v >= 128 && v <= 32768 && v % 128 == 0; }
 
-static int check_shape(const moe_shape_t *s)
+int check_shape(const moe_shape_t *s)
 {
     if (!s)
         return MOE_ERR_INVALID_ARG;
@@ -205,6 +205,7 @@ WsLayout ws_layout(const moe_shape_t &s)
     L.s_xT = take(bws ? s.d * Tp * 2 : 0);
     L.scores = take(ec ? T * E * 4 : 0);
     L.ec_w = take(ec ? N * 4 : 0);
+    L.dbg_seen = take(debug_checks(s) ? N * 4 : 0);
     L.x_stage = take((s.flags & MOE_FLAG_HOST_IO) ? T * s.d * 2 : 0);
     L.out_stage = take((s.flags & MOE_FLAG_HOST_IO) ? T * s.d * 4 : 0);
     L.total = off;
@@ -272,7 +273,7 @@ static int expert_ffn_core(const moe_shape_t &s, const WsLayout &L, void *ws,
                            const uint16_t *W2, const int32_t *perm_token, const int32_t *slot_pos,
                            const float *topk_w, float *y_perm, float *out, uint32_t *status,
                            cudaStream_t st, long long n_rows = -1, const float *perm_w = nullptr,
-                           bool allow_pair = true)
+                           bool allow_pair = true, bool test_starve = false)
 {
     const long long N = n_rows >= 0 ? n_rows : (long long)s.T * s.k;
     uint16_t *H = at<uint16_t>(ws, L.H);
@@ -291,6 +292,7 @@ static int expert_ffn_core(const moe_shape_t &s, const WsLayout &L, void *ws,
     g.out = H;
     g.ldo = s.d_ff;
     g.status = status;
+    g.test_starve = test_starve ? 1 : 0;
     int rc;
     {
         StageMark m(MOE_STAGE_W13, st);
@@ -298,6 +300,7 @@ static int expert_ffn_core(const moe_shape_t &s, const WsLayout &L, void *ws,
     }
     if (rc)
         return rc;
+    g.test_starve = 0;
     g.A = H;
     g.B = W2;
     g.b_rows_total = (long long)s.E * s.d;
@@ -575,6 +578,11 @@ static int forward_impl(const moe_shape_t &s, const WsLayout &L, void *ws, const
                             hist_fused ? kBlockM : kChunkTokens);
     }
     if (rc)
+        return rc;
+    if (debug_checks(s) &&
+        (rc = launch_check_dispatch(s, idx, offsets, slot_pos, perm_token,
+                                    at<int32_t>(ws, L.n_kept), at<int32_t>(ws, L.dbg_seen),
+                                    status, st)))
         return rc;
     if (shared) {
         StageMark m(MOE_STAGE_SHARED, st);
@@ -1256,6 +1264,7 @@ const char *moe_status_string(int code)
     case MOE_ERR_NONFINITE: return "non-finite router logit";
     case MOE_ERR_BAD_EXPERT: return "expert id out of range or repeated";
     case MOE_ERR_TIMEOUT: return "device pipeline wait timed out";
+    case MOE_ERR_CHECK: return "dispatch consistency check failed";
     default: return "unknown status";
     }
 }
@@ -1382,15 +1391,41 @@ int moe_permute(const moe_shape_t *shape, const int32_t *topk_idx, const moe_bf1
         return MOE_ERR_CUDA;
     int32_t *chunk = at<int32_t>(ws, L.chunk_counts);
     int32_t *rank = at<int32_t>(ws, L.rank_local);
-    rc = launch_hist_scan(s, topk_idx, chunk, rank, counter, expert_counts, expert_offsets,
-                          n_kept ? n_kept : at<int32_t>(ws, L.n_kept), at<int32_t>(ws, L.mt_row0),
-                          at<int32_t>(ws, L.mt_group), at<int32_t>(ws, L.num_mt),
-                          at<int32_t>(ws, L.mt2_row0), at<int32_t>(ws, L.mt2_group),
-                          at<int32_t>(ws, L.num_mt2), status, st);
+    int32_t *nk = n_kept ? n_kept : at<int32_t>(ws, L.n_kept);
+    rc = launch_hist_scan(s, topk_idx, chunk, rank, counter, expert_counts, expert_offsets, nk,
+                          at<int32_t>(ws, L.mt_row0), at<int32_t>(ws, L.mt_group),
+                          at<int32_t>(ws, L.num_mt), at<int32_t>(ws, L.mt2_row0),
+                          at<int32_t>(ws, L.mt2_group), at<int32_t>(ws, L.num_mt2), status, st);
     if (rc)
         return rc;
-    return launch_permute(s, topk_idx, chunk, rank, expert_offsets, x, slot_pos, perm_token,
-                          x ? x_perm : nullptr, nullptr, st);
+    rc = launch_permute(s, topk_idx, chunk, rank, expert_offsets, x, slot_pos, perm_token,
+                        x ? x_perm : nullptr, nullptr, st);
+    if (rc || !debug_checks(s))
+        return rc;
+    return launch_check_dispatch(s, topk_idx, expert_offsets, slot_pos, perm_token, nk,
+                                 at<int32_t>(ws, L.dbg_seen), status, st);
+}
+
+int moe_check_dispatch(const moe_shape_t *shape, const int32_t *topk_idx,
+                       const int32_t *expert_offsets, const int32_t *slot_pos,
+                       const int32_t *perm_token, const int32_t *n_kept, uint32_t *status,
+                       void *ws, size_t ws_bytes, moe_stream_t stream)
+{
+    int rc = check_shape(shape);
+    if (rc)
+        return rc;
+    const moe_shape_t &s = *shape;
+    if (s.T == 0)
+        return MOE_OK;
+    if (!debug_checks(s) || !topk_idx || !expert_offsets || !slot_pos || !perm_token || !n_kept ||
+        !status)
+        return MOE_ERR_INVALID_ARG;
+    WsLayout L;
+    if ((rc = check_ws(s, ws, ws_bytes, L)))
+        return rc;
+    return launch_check_dispatch(s, topk_idx, expert_offsets, slot_pos, perm_token, n_kept,
+                                 at<int32_t>(ws, L.dbg_seen), status,
+                                 reinterpret_cast<cudaStream_t>(stream));
 }
 
 int moe_expert_ffn(const moe_shape_t *shape, const moe_bf16_t *x_perm,
@@ -1411,6 +1446,10 @@ int moe_expert_ffn(const moe_shape_t *shape, const moe_bf16_t *x_perm,
         return MOE_ERR_INVALID_ARG;
     if (y_perm ? !al16(y_perm) : (!out || !perm_token || !slot_pos || !topk_w || !al16(out)))
         return MOE_ERR_INVALID_ARG;
+    // the test-only starved w1/w3 launch: single-SM tensor-core kernel only
+    const bool starve = (s.flags & MOE_FLAG_TEST_TIMEOUT) != 0;
+    if (starve && (s.flags & MOE_FLAG_SIMT_FFN))
+        return MOE_ERR_INVALID_ARG;
     WsLayout L;
     if ((rc = check_ws(s, ws, ws_bytes, L)))
         return rc;
@@ -1424,7 +1463,7 @@ int moe_expert_ffn(const moe_shape_t *shape, const moe_bf16_t *x_perm,
     if (rc)
         return rc;
     return expert_ffn_core(s, L, ws, x_perm, expert_offsets, W13, W2, perm_token, slot_pos, topk_w,
-                           y_perm, out, status, st);
+                           y_perm, out, status, st, -1, nullptr, !starve, starve);
 }
 
 int moe_combine(const moe_shape_t *shape, const float *y_perm, const int32_t *slot_pos,

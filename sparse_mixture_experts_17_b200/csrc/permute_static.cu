@@ -1,13 +1,14 @@
 // permute_static.cu -- moe_permute for callers that cannot allocate.
 //
-// Some callers have no way to hand the library a workspace: code that runs
-// while a stream is being captured in global capture mode (cudaMalloc is
-// refused there), engines that reserve every byte of device memory for their
-// own pool up front, and latency-critical paths that cannot afford
-// cudaMalloc/cudaFree (cudaFree synchronises the whole device). For them,
+// Some callers have no way to hand the library a workspace: engines that
+// reserve every byte of device memory for their own pool up front, and
+// latency-critical paths that cannot afford cudaMalloc/cudaFree (cudaFree
+// synchronises the whole device). For them,
 // moe_permute_static runs the same histogram/offsets/permutation kernels as
 // moe_permute, with their scratch in one fixed array that the library carries
 // in device memory, so the call itself allocates nothing.
+#include <cuda.h>
+
 #include <cstring>
 #include <mutex>
 
@@ -50,33 +51,58 @@ StaticLayout static_layout(const moe_shape_t &s)
     return L;
 }
 
-bool shape_ok(const moe_shape_t *s)
+using CtxGetCurrentFn = CUresult (*)(CUcontext *);
+
+// cuCtxGetCurrent through the runtime's driver entry-point table (the library
+// does not link the driver API directly).
+CtxGetCurrentFn ctx_get_current()
 {
-    auto dim_ok = [](int v) { return v >= 128 && v <= 32768 && v % 128 == 0; };
-    return s && s->T >= 0 && s->T <= (1 << 24) && s->E >= 1 && s->E <= MOE_MAX_E && s->k >= 1 &&
-           s->k <= s->E && s->k <= MOE_MAX_K && dim_ok(s->d) && dim_ok(s->d_ff) &&
-           (s->d_ff_shared == 0 || dim_ok(s->d_ff_shared));
+    static CtxGetCurrentFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<CtxGetCurrentFn>(ptr);
+    });
+    return fn;
 }
 
-// Device address of the scratch array on the current device, resolved once
-// per device (with that device current). Host code must never pass
-// g_permute_scratch itself to a kernel: on the host it names a shadow, not
-// device memory.
+// Device address of the scratch array in the current device's context. It is
+// looked up with cudaGetSymbolAddress, with that device current, the first
+// time a device (or a new context of it, after a reset) is seen, and cached
+// per device together with the context it belongs to. Host code must never
+// pass g_permute_scratch itself to a kernel: on the host it names a shadow,
+// not device memory.
 int scratch_for_current_device(unsigned char **out)
 {
+    struct Entry {
+        CUcontext ctx;
+        unsigned char *ptr;
+    };
     static std::mutex mu;
-    static unsigned char *ptrs[256] = {};
+    static Entry cache[256] = {};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 256)
         return MOE_ERR_CUDA;
+    CtxGetCurrentFn get_ctx = ctx_get_current();
+    if (!get_ctx)
+        return MOE_ERR_CUDA;
     std::lock_guard<std::mutex> g(mu);
-    if (!ptrs[dev]) {
+    CUcontext ctx = nullptr;
+    if (get_ctx(&ctx) != CUDA_SUCCESS)
+        return MOE_ERR_CUDA;
+    if (!cache[dev].ptr || !ctx || cache[dev].ctx != ctx) {
         void *p = nullptr;
         if (cudaGetSymbolAddress(&p, g_permute_scratch) != cudaSuccess || !p)
             return MOE_ERR_CUDA;
-        ptrs[dev] = static_cast<unsigned char *>(p);
+        // the lookup made the device's context current on this thread
+        if (get_ctx(&ctx) != CUDA_SUCCESS || !ctx)
+            return MOE_ERR_CUDA;
+        cache[dev] = Entry{ctx, static_cast<unsigned char *>(p)};
     }
-    *out = ptrs[dev];
+    *out = cache[dev].ptr;
     return MOE_OK;
 }
 
@@ -91,7 +117,7 @@ extern "C" int moe_permute_static(const moe_shape_t *shape, const int32_t *topk_
                                   moe_bf16_t *x_perm, int32_t *n_kept, uint32_t *status,
                                   moe_stream_t stream)
 {
-    if (!shape_ok(shape))
+    if (check_shape(shape) != MOE_OK)
         return MOE_ERR_INVALID_ARG;
     const moe_shape_t &s = *shape;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);

@@ -46,10 +46,41 @@ __device__ __forceinline__ int block_excl_scan(int v, int *s_warp, int *total)
     return r;
 }
 
+// Position of element j of one sorted list (length n) in the merge of two
+// lists of lengths n and m spread evenly over each other: element j carries
+// the key (j + 1/2) / n, the other list's element i the key (i + 1/2) / m,
+// and ties go to `first` (the list whose elements precede on equal keys).
+__device__ __forceinline__ int spread_merge_pos(int j, int n, int m, bool first)
+{
+    if (m == 0)
+        return j;
+    const long long a = (long long)(2 * j + 1) * m;   // key of j, scaled by 2 n m
+    long long before;                                 // elements of the other list before j
+    if (first) {   // other elements i with (2i + 1) n < a
+        const long long num = a - n;
+        before = num <= 0 ? 0 : (num + 2LL * n - 1) / (2LL * n);
+    } else {       // other elements i with (2i + 1) n <= a
+        const long long num = a - n;
+        before = num < 0 ? 0 : num / (2LL * n) + 1;
+    }
+    return j + (int)(before < m ? before : m);
+}
+
 // Writes the grouped-GEMM m-tile list for kept counts in s_kept[E]: expert e
 // contributes ceil(kept/tile_m) tiles starting at rows offsets[e] + tile_m i.
-// tile_start (may be NULL) receives each expert's first tile index. Thread e
-// handles expert e (blockDim.x >= E).
+// Thread e handles expert e (blockDim.x >= E).
+//
+// Order. With tile_start == NULL the list interleaves two kinds of expert:
+// experts of one tile (few rows: their GEMM tiles stream a whole weight
+// block for few rows, so they are bound by DRAM) and experts of several
+// tiles (their tiles share each weight block through L2, so they are bound
+// by the tensor cores). Each list keeps expert order, and the two are spread
+// evenly over each other, so every stretch of the list that the GEMM runs at
+// once holds both kinds and the weight stream of the first overlaps the
+// arithmetic of the second. An expert's tiles stay in order. With tile_start
+// set (block-scaled operands, whose activation scales are keyed by tile
+// index) the list is in plain expert order and tile_start receives each
+// expert's first tile index.
 __device__ inline void build_tiles(const int *s_kept, const int32_t *offsets_smem_or_global, int E,
                                    int tile_m, int32_t *mt_row0, int32_t *mt_group,
                                    int32_t *num_mt, int *s_warp, int32_t *tile_start = nullptr)
@@ -57,8 +88,12 @@ __device__ inline void build_tiles(const int *s_kept, const int32_t *offsets_sme
     const int tid = threadIdx.x;
     const int e = tid;
     const int nt = (e < E) ? (s_kept[e] + tile_m - 1) / tile_m : 0;
-    int total;
+    const bool spread = tile_start == nullptr;
+    const bool multi = nt >= 2;
+    int total, n_multi, n_single;
     const int start = block_excl_scan(nt, s_warp, &total);
+    const int start_m = block_excl_scan(spread && multi ? nt : 0, s_warp, &n_multi);
+    const int start_s = block_excl_scan(spread && !multi ? nt : 0, s_warp, &n_single);
     if (e < E && tile_start)
         tile_start[e] = start;
     if (e < E) {
@@ -66,9 +101,13 @@ __device__ inline void build_tiles(const int *s_kept, const int32_t *offsets_sme
         // a last tile of <= 64 rows is marked for the M = 64 MMA (128-row lists only)
         const int rem = s_kept[e] - (nt - 1) * tile_m;
         for (int i = 0; i < nt; ++i) {
-            mt_row0[start + i] = base + i * tile_m;
+            int pos = start + i;
+            if (spread)
+                pos = multi ? spread_merge_pos(start_m + i, n_multi, n_single, true)
+                            : spread_merge_pos(start_s + i, n_single, n_multi, false);
+            mt_row0[pos] = base + i * tile_m;
             const bool half = (tile_m == kBlockM) && (i == nt - 1) && rem <= 64;
-            mt_group[start + i] = e | (half ? kHalfTileBit : 0);
+            mt_group[pos] = e | (half ? kHalfTileBit : 0);
         }
     }
     if (tid == 0)

@@ -26,6 +26,7 @@ MOE_ERR_CUDA = 4
 MOE_ERR_NONFINITE = 5
 MOE_ERR_BAD_EXPERT = 6
 MOE_ERR_TIMEOUT = 7
+MOE_ERR_CHECK = 8
 
 MOE_FLAG_DETERMINISTIC = 1 << 0
 MOE_FLAG_FORCE_PREFILL = 1 << 1
@@ -39,6 +40,8 @@ MOE_FLAG_SLOT_PRIORITY = 1 << 8
 MOE_FLAG_MXFP8 = 1 << 9
 MOE_FLAG_BACKWARD = 1 << 10
 MOE_FLAG_NVFP4 = 1 << 11
+MOE_FLAG_DEBUG_CHECKS = 1 << 12
+MOE_FLAG_TEST_TIMEOUT = 1 << 13
 
 MOE_MAX_E = 256
 MOE_MAX_K = 16
@@ -86,6 +89,7 @@ _SIGS = {
     "moe_forward": ([_SHP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P], ctypes.c_int),
     "moe_forward_host": ([_SHP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P], ctypes.c_int),
     "moe_permute_static": ([_SHP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P], ctypes.c_int),
+    "moe_check_dispatch": ([_SHP, _P, _P, _P, _P, _P, _P, _P, _SZ, _P], ctypes.c_int),
     "moe_quantize_experts_mxfp8": ([_SHP, _P, _P, _P, _P, _P, _P, _P, _P], ctypes.c_int),
     "moe_forward_mxfp8": ([_SHP] + [_P] * 16 + [_SZ, _P], ctypes.c_int),
     "moe_quantize_experts_nvfp4": ([_SHP] + [_P] * 10, ctypes.c_int),
@@ -203,6 +207,16 @@ def moe_permute(shape, topk_idx, x, expert_counts, expert_offsets, slot_pos, per
         _ptr(slot_pos, I32, "slot_pos"), _ptr(perm_token, I32, "perm_token"),
         _ptr(x_perm, BF16, "x_perm"), _ptr(n_kept, I32, "n_kept"), _ptr(status, U32, "status"),
         _ptr(ws, name="ws"), ws.numel(), _stream(stream)))
+
+
+def moe_check_dispatch(shape, topk_idx, expert_offsets, slot_pos, perm_token, n_kept, status, ws,
+                       stream=None):
+    """Debug consistency checks of a dispatch; failures set bits of `status`."""
+    _check("moe_check_dispatch", lib().moe_check_dispatch(
+        ctypes.byref(shape), _ptr(topk_idx, I32, "topk_idx"),
+        _ptr(expert_offsets, I32, "expert_offsets"), _ptr(slot_pos, I32, "slot_pos"),
+        _ptr(perm_token, I32, "perm_token"), _ptr(n_kept, I32, "n_kept"),
+        _ptr(status, U32, "status"), _ptr(ws, name="ws"), ws.numel(), _stream(stream)))
 
 
 def moe_permute_static(shape, topk_idx, x, expert_counts, expert_offsets, slot_pos, perm_token,
