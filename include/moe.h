@@ -386,10 +386,17 @@ MOE_API int moe_quantize_experts_nvfp4(const moe_shape_t *shape, const moe_bf16_
  * rejected (MOE_ERR_INVALID_ARG), as are x_gs or h_gs that are not positive
  * and finite. Arguments as in moe_forward_mxfp8, with each weight set's
  * global scales (device pointers, as moe_quantize_experts_nvfp4 writes them).
- * Every T runs the block-scaled tensor-core GEMMs, which read each chosen
- * expert's codes and scales once (4.5 bits a weight); MOE_FLAG_FORCE_DECODE
- * is MOE_ERR_UNSUPPORTED. MOE_FLAG_DETERMINISTIC, capacity and
- * MOE_FLAG_SLOT_PRIORITY act as in moe_forward.
+ * T <= MOE_DECODE_DEFAULT_T takes the NVFP4 decode kernels ("perf(moe): route
+ * granite-4.0-h single-token MoE through the fused kernel": a 4-bit
+ * single-token path fed by the top-k indices and weights): x and h are
+ * quantized as the tensor-core chain quantizes them, and each chosen expert's
+ * codes and scales are streamed once through CUDA cores, every 16-element
+ * block dot product exact in f16. Larger T runs the block-scaled tensor-core
+ * GEMMs, which also read each chosen expert's codes and scales once (4.5
+ * bits a weight). MOE_FLAG_FORCE_DECODE takes the decode kernels for T <= 2
+ * and is MOE_ERR_UNSUPPORTED above; MOE_FLAG_FORCE_PREFILL takes the chain.
+ * MOE_FLAG_DETERMINISTIC, capacity and MOE_FLAG_SLOT_PRIORITY act as in
+ * moe_forward.
  * Device errors: MOE_ERR_NONFINITE, MOE_ERR_BAD_EXPERT, MOE_ERR_TIMEOUT. */
 MOE_API int moe_forward_nvfp4(const moe_shape_t *shape, const moe_bf16_t *x, const moe_bf16_t *Wg,
                               const float *bias, const uint8_t *W13q, const uint8_t *W13sf,

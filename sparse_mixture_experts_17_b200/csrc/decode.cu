@@ -30,6 +30,7 @@
 #include "common.cuh"
 #include "internal.h"
 #include "mxfp8.cuh"
+#include "nvfp4.cuh"
 #include "topk.cuh"
 
 namespace moe {
@@ -679,6 +680,259 @@ __global__ void __launch_bounds__(256, (MAXT <= 2) ? 4 : 2)
     }
 }
 
+// ---------------------------------------------------------------- NVFP4 experts (T <= 2)
+// The same two phases on NVFP4 weights (packed E2M1 codes, an E4M3 scale per
+// 16 elements in the atom layout, a global scale per expert), with x and h
+// quantized to NVFP4 as the tensor-core chain quantizes them and handed over
+// as their codes' values in f16 plus each block's scale value in fp32.
+//
+// One 16-element block is a dot product of E2M1 values: every product is a
+// multiple of 1/4 of magnitude <= 36, so each f16 lane of the half2
+// accumulator (8 products) stays a multiple of 1/4 below 288 and is exact in
+// f16; the block sum is then scaled by s_w * s_x (two E4M3 values: exact in
+// fp32) and accumulated in fp32. The global scales divide the row's sum once.
+
+// Exact dot product of one 16-element block: the 8 code bytes (w0, w1; the
+// first element in the low nibble) against 8 f16x2 values.
+__device__ __forceinline__ float nv_block_dot(uint32_t w0, uint32_t w1, const uint4 &xa,
+                                              const uint4 &xb)
+{
+    const uint32_t xv[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+    __half2 acc = __float2half2_rn(0.f);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const uint32_t wb = (j < 4 ? w0 : w1) >> (8 * (j & 3));
+        acc = __hfma2(nv_pair_h2(wb), *reinterpret_cast<const __half2 *>(&xv[j]), acc);
+    }
+    const float2 f = __half22float2(acc);
+    return f.x + f.y;
+}
+
+// One 16-byte chunk of a code row (32 elements = blocks 2ci and 2ci + 1)
+// against one row of values (f16) and block scales (fp32): sum over both
+// blocks of the exact block dot times s_w(block) * s_x(block).
+__device__ __forceinline__ float nv_chunk_dot(const uint4 &w, uint32_t sw2, const uint4 *xh,
+                                              const float2 &xs, int ci)
+{
+    const uint4 x0 = __ldg(xh + 4 * ci), x1 = __ldg(xh + 4 * ci + 1);
+    const uint4 x2 = __ldg(xh + 4 * ci + 2), x3 = __ldg(xh + 4 * ci + 3);
+    const float b0 = nv_block_dot(w.x, w.y, x0, x1);
+    const float b1 = nv_block_dot(w.z, w.w, x2, x3);
+    return fmaf(b1, nv_scale_value(sw2 >> 8) * xs.y, b0 * (nv_scale_value(sw2) * xs.x));
+}
+
+// Phase 1: one work unit = h column c of one chosen expert (its packed gate
+// and up rows, each streamed once), or of the shared expert.
+template <int MAXT>
+__global__ void __launch_bounds__(256, 4)
+    k_dec_w13_nv(const uint16_t *__restrict__ xh, const float *__restrict__ xs, float x_gs,
+                 const int32_t *__restrict__ idx, int T, int d, int d_ff, int E, int k, int C,
+                 int slot_major, const uint8_t *__restrict__ W13q,
+                 const uint8_t *__restrict__ W13sf, const float *__restrict__ gs13, int d_ff_s,
+                 const uint8_t *__restrict__ W13s_q, const uint8_t *__restrict__ W13s_sf,
+                 const float *__restrict__ gs13s, float *__restrict__ H32,
+                 float *__restrict__ Hs32, uint32_t *status)
+{
+    __shared__ DecPlanSmem P;
+    pdl_wait();
+    pdl_trigger();
+    build_plan(P, idx, T, E, k, C, slot_major, status);
+    const int lane = threadIdx.x & 31;
+    const int nwarps = gridDim.x * (blockDim.x >> 5);
+    const long long routed_units = (long long)P.U * d_ff;
+    const long long units = routed_units + (W13s_q ? d_ff_s : 0);
+    const int nv = d / 32;   // 16-byte chunks of a packed row
+    for (long long unit = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; unit < units;
+         unit += nwarps) {
+        const uint8_t *qb, *sb;
+        int a0, na, c, ldh;
+        float *hout;
+        float gsw;
+        const bool shared = unit >= routed_units;
+        size_t prow;
+        if (!shared) {
+            const int u = (int)(unit / d_ff);
+            c = (int)(unit - (long long)u * d_ff);
+            // packed gate row of h column c; the up row is 64 rows further
+            prow = (size_t)P.uniq[u] * 2 * d_ff + (size_t)(c / 64) * 128 + (c % 64);
+            qb = W13q;
+            sb = W13sf;
+            gsw = gs13[P.uniq[u]];
+            a0 = P.ustart[u];
+            na = P.ustart[u + 1] - a0;
+            hout = H32;
+            ldh = d_ff;
+        } else {
+            c = (int)(unit - routed_units);
+            prow = (size_t)(c / 64) * 128 + (c % 64);
+            qb = W13s_q;
+            sb = W13s_sf;
+            gsw = gs13s[0];
+            a0 = 0;
+            na = T;
+            hout = Hs32;
+            ldh = d_ff_s;
+        }
+        const uint4 *gate = reinterpret_cast<const uint4 *>(qb + prow * (d / 2));
+        const uint4 *up = reinterpret_cast<const uint4 *>(qb + (prow + 64) * (d / 2));
+        const long long gt = (long long)(prow >> 7), ut = (long long)((prow + 64) >> 7);
+        const int gm = (int)(prow & 127), um = (int)((prow + 64) & 127);
+        const uint4 *xr[MAXT];
+        const float2 *sr[MAXT];
+#pragma unroll
+        for (int s = 0; s < MAXT; ++s) {
+            const int tok = (s < na) ? (shared ? s : P.list[a0 + s] / k) : 0;
+            xr[s] = reinterpret_cast<const uint4 *>(xh + (size_t)tok * d);
+            sr[s] = reinterpret_cast<const float2 *>(xs + (size_t)tok * (d / 16));
+        }
+        float ag[MAXT], au[MAXT];
+#pragma unroll
+        for (int s = 0; s < MAXT; ++s)
+            ag[s] = au[s] = 0.f;
+        for (int cb = 0; cb < nv; cb += 32 * kDecUnroll) {
+            uint4 wg[kDecUnroll], wu[kDecUnroll];
+            uint32_t sg[kDecUnroll], su[kDecUnroll];
+#pragma unroll
+            for (int i = 0; i < kDecUnroll; ++i) {
+                const int ci = cb + lane + 32 * i;
+                if (ci < nv) {
+                    wg[i] = ld_stream_v4(gate + ci);
+                    wu[i] = ld_stream_v4(up + ci);
+                    // blocks 2ci and 2ci + 1: adjacent bytes of one scale word
+                    sg[i] = __ldg(reinterpret_cast<const uint16_t *>(sb + nv_sf_offset(gt, gm, 2 * ci, d)));
+                    su[i] = __ldg(reinterpret_cast<const uint16_t *>(sb + nv_sf_offset(ut, um, 2 * ci, d)));
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < kDecUnroll; ++i) {
+                const int ci = cb + lane + 32 * i;
+                if (ci >= nv)
+                    continue;
+#pragma unroll
+                for (int s = 0; s < MAXT; ++s) {
+                    if (s < na) {
+                        const float2 xsc = __ldg(sr[s] + ci);
+                        ag[s] += nv_chunk_dot(wg[i], sg[i], xr[s], xsc, ci);
+                        au[s] += nv_chunk_dot(wu[i], su[i], xr[s], xsc, ci);
+                    }
+                }
+            }
+        }
+        const float inv = 1.0f / (x_gs * gsw);
+#pragma unroll
+        for (int s = 0; s < MAXT; ++s) {
+            if (s < na) {
+                const float g = warp_sum(ag[s]) * inv;
+                const float uu = warp_sum(au[s]) * inv;
+                if (lane == 0) {
+                    const int row = shared ? s : P.list[a0 + s];
+                    hout[(size_t)row * ldh + c] = silu_mul(g, uu);
+                }
+            }
+        }
+    }
+}
+
+// Phase 2: one work unit = output row r: for each chosen expert (ascending),
+// then the shared expert, stream W2_e[r] once and dot it with each of the
+// expert's assignments' h rows; fixed order (deterministic).
+template <int MAXT>
+__global__ void __launch_bounds__(256, 4)
+    k_dec_w2_nv(const int32_t *__restrict__ idx, const float *__restrict__ topk_w, int T, int d,
+                int d_ff, int E, int k, int C, int slot_major, const uint8_t *__restrict__ W2q,
+                const uint8_t *__restrict__ W2sf, const float *__restrict__ gs2, int d_ff_s,
+                const uint8_t *__restrict__ W2s_q, const uint8_t *__restrict__ W2s_sf,
+                const float *__restrict__ gs2s, const uint16_t *__restrict__ hh,
+                const float *__restrict__ hsc, float h_gs, float *__restrict__ out,
+                uint32_t *status)
+{
+    __shared__ DecPlanSmem P;
+    pdl_wait();      // h comes from the quantization between the phases
+    build_plan(P, idx, T, E, k, C, slot_major, status);
+    const int lane = threadIdx.x & 31;
+    const int nwarps = gridDim.x * (blockDim.x >> 5);
+    const int n_src = P.U + (W2s_q ? 1 : 0);
+    // shared-expert rows follow the T * k routed rows
+    const uint16_t *hh_s = hh + (size_t)T * k * d_ff;
+    const float *hsc_s = hsc + (size_t)T * k * (d_ff / 16);
+    for (int r = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; r < d; r += nwarps) {
+        float acc[MAXT];
+#pragma unroll
+        for (int t = 0; t < MAXT; ++t)
+            acc[t] = 0.f;
+        for (int u = 0; u < n_src; ++u) {
+            const bool shared = (u == P.U);
+            const int ff = shared ? d_ff_s : d_ff;
+            const size_t wr = shared ? (size_t)r : (size_t)P.uniq[u] * d + r;
+            const uint4 *wrow = reinterpret_cast<const uint4 *>((shared ? W2s_q : W2q) + wr * (ff / 2));
+            const uint8_t *wsf = shared ? W2s_sf : W2sf;
+            const long long wt_tile = (long long)(wr >> 7);
+            const int wt_m = (int)(wr & 127);
+            const int a0 = shared ? 0 : P.ustart[u];
+            const int na = shared ? T : P.ustart[u + 1] - a0;
+            const float inv = 1.0f / (h_gs * (shared ? gs2s[0] : gs2[P.uniq[u]]));
+            const uint4 *hr[MAXT];
+            const float2 *sr[MAXT];
+            int tk[MAXT];
+            float wt[MAXT];
+#pragma unroll
+            for (int s = 0; s < MAXT; ++s) {
+                const int a = (s < na) ? (shared ? s : P.list[a0 + s]) : 0;
+                hr[s] = reinterpret_cast<const uint4 *>((shared ? hh_s : hh) + (size_t)a * ff);
+                sr[s] = reinterpret_cast<const float2 *>((shared ? hsc_s : hsc) + (size_t)a * (ff / 16));
+                tk[s] = shared ? s : a / k;
+                wt[s] = (s < na) ? (shared ? 1.f : topk_w[a]) * inv : 0.f;
+            }
+            const int nv = ff / 32;
+            float pa[MAXT];
+#pragma unroll
+            for (int s = 0; s < MAXT; ++s)
+                pa[s] = 0.f;
+            constexpr int UNR = 8;
+            for (int cb = 0; cb < nv; cb += 32 * UNR) {
+                uint4 wv[UNR];
+                uint32_t sc[UNR];
+#pragma unroll
+                for (int i = 0; i < UNR; ++i) {
+                    const int ci = cb + lane + 32 * i;
+                    if (ci < nv) {
+                        wv[i] = ld_stream_v4(wrow + ci);
+                        sc[i] = __ldg(reinterpret_cast<const uint16_t *>(
+                            wsf + nv_sf_offset(wt_tile, wt_m, 2 * ci, ff)));
+                    }
+                }
+#pragma unroll
+                for (int i = 0; i < UNR; ++i) {
+                    const int ci = cb + lane + 32 * i;
+                    if (ci >= nv)
+                        continue;
+#pragma unroll
+                    for (int s = 0; s < MAXT; ++s)
+                        if (s < na)
+                            pa[s] += nv_chunk_dot(wv[i], sc[i], hr[s], __ldg(sr[s] + ci), ci);
+                }
+            }
+#pragma unroll
+            for (int s = 0; s < MAXT; ++s) {
+                if (s < na) {
+#pragma unroll
+                    for (int tt = 0; tt < MAXT; ++tt)
+                        if (tt == tk[s])
+                            acc[tt] = fmaf(wt[s], pa[s], acc[tt]);
+                }
+            }
+        }
+#pragma unroll
+        for (int t = 0; t < MAXT; ++t) {
+            if (t < T) {
+                const float v = warp_sum(acc[t]);
+                if (lane == 0)
+                    out[(size_t)t * d + r] = v;
+            }
+        }
+    }
+}
+
 // ---------------------------------------------------------------- host side
 
 // Launch with programmatic stream serialization (the kernel calls pdl_wait()
@@ -853,6 +1107,52 @@ int launch_dec_w2_mx(const moe_shape_t &s, const int32_t *topk_idx, const float 
     default: MOE_DEC2MX(16); break;
     }
 #undef MOE_DEC2MX
+    return launched();
+}
+
+int launch_dec_w13_nv(const moe_shape_t &s, const uint16_t *xh, const float *xs, float x_gs,
+                      const int32_t *topk_idx, const uint8_t *W13q, const uint8_t *W13sf,
+                      const float *gs13, const uint8_t *W13s_q, const uint8_t *W13s_sf,
+                      const float *gs13s, float *H32, uint32_t *status, cudaStream_t st)
+{
+    if (s.T == 0)
+        return MOE_OK;
+    if (s.T > 2)
+        return MOE_ERR_UNSUPPORTED;
+    const int blocks = num_sms() * 4;
+    float *Hs = H32 + (size_t)s.T * s.k * s.d_ff;
+    const uint8_t *wq = s.d_ff_shared ? W13s_q : nullptr;
+    if (s.T == 1)
+        launch_pdl(k_dec_w13_nv<1>, blocks, 256, st, xh, xs, x_gs, topk_idx, s.T, s.d, s.d_ff,
+                   s.E, s.k, s.capacity, slot_major(s), W13q, W13sf, gs13, s.d_ff_shared, wq,
+                   W13s_sf, gs13s, H32, Hs, status);
+    else
+        launch_pdl(k_dec_w13_nv<2>, blocks, 256, st, xh, xs, x_gs, topk_idx, s.T, s.d, s.d_ff,
+                   s.E, s.k, s.capacity, slot_major(s), W13q, W13sf, gs13, s.d_ff_shared, wq,
+                   W13s_sf, gs13s, H32, Hs, status);
+    return launched();
+}
+
+int launch_dec_w2_nv(const moe_shape_t &s, const int32_t *topk_idx, const float *topk_w,
+                     const uint8_t *W2q, const uint8_t *W2sf, const float *gs2,
+                     const uint8_t *W2s_q, const uint8_t *W2s_sf, const float *gs2s,
+                     const uint16_t *hh, const float *hs, float h_gs, float *out,
+                     uint32_t *status, cudaStream_t st)
+{
+    if (s.T == 0)
+        return MOE_OK;
+    if (s.T > 2)
+        return MOE_ERR_UNSUPPORTED;
+    const int blocks = num_sms() * 4;
+    const uint8_t *wq = s.d_ff_shared ? W2s_q : nullptr;
+    if (s.T == 1)
+        launch_pdl(k_dec_w2_nv<1>, blocks, 256, st, topk_idx, topk_w, s.T, s.d, s.d_ff, s.E, s.k,
+                   s.capacity, slot_major(s), W2q, W2sf, gs2, s.d_ff_shared, wq, W2s_sf, gs2s,
+                   hh, hs, h_gs, out, status);
+    else
+        launch_pdl(k_dec_w2_nv<2>, blocks, 256, st, topk_idx, topk_w, s.T, s.d, s.d_ff, s.E, s.k,
+                   s.capacity, slot_major(s), W2q, W2sf, gs2, s.d_ff_shared, wq, W2s_sf, gs2s,
+                   hh, hs, h_gs, out, status);
     return launched();
 }
 

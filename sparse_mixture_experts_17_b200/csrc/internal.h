@@ -49,7 +49,8 @@ struct WsLayout {
     size_t x_stage, out_stage;
     size_t scores, ec_w;   // expert-choice routing
     size_t xq, xsf, Hq, Hsf, xq_s, xsf_s, Hsq, Hssf;   // MXFP8 operands
-    size_t dec_xdq, dec_H32;                             // MXFP8 decode
+    size_t dec_xdq, dec_H32;                             // MXFP8 / NVFP4 decode
+    size_t dec_xs, dec_hs;                               // NVFP4 decode: scale values
     size_t tile_start;                                   // first m-tile of each expert
     size_t dbg_seen;                                     // dispatch checks: count per row
     // backward pass
@@ -236,6 +237,23 @@ int launch_nv_pack_w13(const moe_shape_t &s, const uint16_t *W1, const uint16_t 
 int launch_nv_gather(const moe_shape_t &s, const uint16_t *x, const int32_t *idx,
                      const int32_t *slot_pos, const int32_t *offsets, const int32_t *tile_start,
                      float gs, uint8_t *xq, uint8_t *xsf, cudaStream_t st);
+// n values (a multiple of 16) through NVFP4 with global scale gs, as the codes'
+// values in f16 (dst_h, n) and the block scales' values in fp32 (dst_s, n / 16)
+int launch_nv_qrows_f16_bf16(const uint16_t *src, long long n, float gs, uint16_t *dst_h,
+                             float *dst_s, cudaStream_t st);
+int launch_nv_qrows_f16_f32(const float *src, long long n, float gs, uint16_t *dst_h,
+                            float *dst_s, cudaStream_t st);
+// decode phases on NVFP4 experts (decode.cu), T <= 2: x and h as given by
+// launch_nv_qrows_f16_*; H32 receives h in fp32 (routed rows, then shared)
+int launch_dec_w13_nv(const moe_shape_t &s, const uint16_t *xh, const float *xs, float x_gs,
+                      const int32_t *topk_idx, const uint8_t *W13q, const uint8_t *W13sf,
+                      const float *gs13, const uint8_t *W13s_q, const uint8_t *W13s_sf,
+                      const float *gs13s, float *H32, uint32_t *status, cudaStream_t st);
+int launch_dec_w2_nv(const moe_shape_t &s, const int32_t *topk_idx, const float *topk_w,
+                     const uint8_t *W2q, const uint8_t *W2sf, const float *gs2,
+                     const uint8_t *W2s_q, const uint8_t *W2s_sf, const float *gs2s,
+                     const uint16_t *hh, const float *hs, float h_gs, float *out,
+                     uint32_t *status, cudaStream_t st);
 // n values (a multiple of 32) through MXFP8 and back, as bf16 (PDL launch)
 int launch_mx_qdq_bf16(const uint16_t *src, long long n, uint16_t *dst, cudaStream_t st);
 int launch_mx_qdq_f32(const float *src, long long n, uint16_t *dst, cudaStream_t st);

@@ -143,8 +143,10 @@ WsLayout ws_layout(const moe_shape_t &s)
     L.Y = take((s.flags & MOE_FLAG_DETERMINISTIC) ? N * s.d * 4 : 0);
     const size_t Td = T < (size_t)MOE_DECODE_MAX_T ? T : (size_t)MOE_DECODE_MAX_T;
     L.dec_H = take((Td * k * s.d_ff + Td * dfs) * 2);
-    L.dec_xdq = take(mx ? Td * s.d * 2 : 0);
-    L.dec_H32 = take(mx ? (Td * k * s.d_ff + Td * dfs) * 4 : 0);
+    L.dec_xdq = take(lowp ? Td * s.d * 2 : 0);
+    L.dec_H32 = take(lowp ? (Td * k * s.d_ff + Td * dfs) * 4 : 0);
+    L.dec_xs = take(nv ? Td * (s.d / 16) * 4 : 0);
+    L.dec_hs = take(nv ? (Td * k * s.d_ff + Td * dfs) / 16 * 4 : 0);
     // scales in the atom layout: routed operands keyed by m-tile (at most
     // max_mt tiles of 128 rows), shared-expert operands by row / 128; NVFP4
     // has twice the scales (16-element blocks) and half the code bytes
@@ -747,15 +749,38 @@ static int forward_mx_impl(const moe_shape_t &s, const WsLayout &L, void *ws, co
     const bool force_pre = (s.flags & MOE_FLAG_FORCE_PREFILL) != 0;
     if (force_dec && s.T > MOE_DECODE_MAX_T)
         return MOE_ERR_UNSUPPORTED;
-    // NVFP4 has no decode kernels of its own: small batches take the
-    // tensor-core chain, which also reads each chosen expert's codes once
-    const bool decode =
-        lw.fmt == FMT_MX8 && (force_dec || (!force_pre && s.T <= MOE_DECODE_DEFAULT_T));
-    if (force_dec && lw.fmt != FMT_MX8)
+    // the NVFP4 decode kernels take T <= 2 (x and h staged as f16 code values)
+    const bool nv = lw.fmt == FMT_NV4;
+    const bool decode = force_dec || (!force_pre && s.T <= MOE_DECODE_DEFAULT_T);
+    if (nv && decode && s.T > 2)
         return MOE_ERR_UNSUPPORTED;
     int rc = route_tokens(s, x, Wg, bias, logits, idx, w, counter, status, st);
     if (rc)
         return rc;
+    if (decode && nv) {
+        // only the chosen experts' codes and scales are read, each once
+        uint16_t *xh = at<uint16_t>(ws, L.dec_xdq);
+        float *xs = at<float>(ws, L.dec_xs);
+        float *H32 = at<float>(ws, L.dec_H32);
+        uint16_t *hh = at<uint16_t>(ws, L.dec_H);
+        float *hs = at<float>(ws, L.dec_hs);
+        const long long nh = (long long)s.T * s.k * s.d_ff + (long long)s.T * s.d_ff_shared;
+        {
+            StageMark m(MOE_STAGE_DEC_W13, st);
+            rc = launch_nv_qrows_f16_bf16(x, (long long)s.T * s.d, lw.x_gs, xh, xs, st);
+            if (!rc)
+                rc = launch_dec_w13_nv(s, xh, xs, lw.x_gs, idx, W13q, W13sf, lw.W13gs, W13s_q,
+                                       W13s_sf, lw.W13s_gs, H32, status, st);
+        }
+        if (rc)
+            return rc;
+        StageMark m(MOE_STAGE_DEC_W2, st);
+        rc = launch_nv_qrows_f16_f32(H32, nh, lw.h_gs, hh, hs, st);
+        if (!rc)
+            rc = launch_dec_w2_nv(s, idx, w, W2q, W2sf, lw.W2gs, W2s_q, W2s_sf, lw.W2s_gs, hh, hs,
+                                  lw.h_gs, out, status, st);
+        return rc;
+    }
     if (decode) {
         // only the chosen experts' codes and scales are read, each once
         uint16_t *xdq = at<uint16_t>(ws, L.dec_xdq);

@@ -15,7 +15,10 @@
 //   k_nv_gather         x [T, d] -> every kept permuted row of token t,
 //                       quantized once with the activations' global scale;
 //                       scales keyed by the row's m-tile
+//   k_nv_qrows_f16      rows of x or h for the decode kernels: the codes'
+//                       values in f16 and the scales' values in fp32
 #include <algorithm>
+#include <cstring>
 
 #include "common.cuh"
 #include "internal.h"
@@ -119,6 +122,51 @@ __global__ void __launch_bounds__(256) k_nv_pack_w13(const uint16_t *__restrict_
     uint2 q;
     scales[nv_sf_offset(prow >> 7, (int)(prow & 127), b, d)] = nv_quantize16(v, gs13[e], q);
     reinterpret_cast<uint2 *>(codes)[i] = q;
+}
+
+// Rows for the NVFP4 decode kernels: each 16-element block of `src` (bf16 or
+// fp32) quantized with global scale gs by the same rule as every other
+// NVFP4 producer here (nv_quantize16), written as the 16 E2M1 values in f16
+// (exact) and the block's E4M3 scale value in fp32. One thread per block;
+// launched with programmatic stream serialization.
+__device__ __forceinline__ void load16(const uint16_t *src, float (&v)[16]) { load_bf16x16(src, v); }
+__device__ __forceinline__ void load16(const float *src, float (&v)[16])
+{
+    const float4 *s = reinterpret_cast<const float4 *>(src);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float4 f = s[i];
+        v[4 * i] = f.x;
+        v[4 * i + 1] = f.y;
+        v[4 * i + 2] = f.z;
+        v[4 * i + 3] = f.w;
+    }
+}
+
+template <typename InT>
+__global__ void __launch_bounds__(256) k_nv_qrows_f16(const InT *__restrict__ src, long long nblocks,
+                                                      float gs, uint16_t *__restrict__ dst_h,
+                                                      float *__restrict__ dst_s)
+{
+    pdl_wait();
+    pdl_trigger();
+    const long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x;
+    if (i >= nblocks)
+        return;
+    float v[16];
+    load16(src + i * kNvBlock, v);
+    uint2 q;
+    const uint8_t sc = nv_quantize16(v, gs, q);
+    uint32_t o[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const __half2 h = nv_pair_h2((j < 4 ? q.x : q.y) >> (8 * (j & 3)));
+        o[j] = *reinterpret_cast<const uint32_t *>(&h);
+    }
+    uint4 *d4 = reinterpret_cast<uint4 *>(dst_h + i * kNvBlock);
+    d4[0] = make_uint4(o[0], o[1], o[2], o[3]);
+    d4[1] = make_uint4(o[4], o[5], o[6], o[7]);
+    dst_s[i] = nv_scale_value(sc);
 }
 
 // One warp per token (as k_mx_gather): lane j < k holds slot j's permuted
@@ -233,6 +281,39 @@ int launch_nv_gather(const moe_shape_t &s, const uint16_t *x, const int32_t *idx
     k_nv_gather<<<(s.T + 7) / 8, 256, 0, st>>>(x, idx, slot_pos, offsets, tile_start, s.T, s.k,
                                                s.d, gs, xq, xsf);
     return launched();
+}
+
+template <typename InT>
+static int launch_nv_qrows(const InT *src, long long n, float gs, uint16_t *dst_h, float *dst_s,
+                           cudaStream_t st)
+{
+    const long long nblocks = n / kNvBlock;
+    if (nblocks <= 0)
+        return MOE_OK;
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof cfg);
+    cfg.gridDim = dim3((unsigned)((nblocks + 255) / 256));
+    cfg.blockDim = dim3(256);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaLaunchKernelEx(&cfg, k_nv_qrows_f16<InT>, src, nblocks, gs, dst_h, dst_s);
+    return launched();
+}
+
+int launch_nv_qrows_f16_bf16(const uint16_t *src, long long n, float gs, uint16_t *dst_h,
+                             float *dst_s, cudaStream_t st)
+{
+    return launch_nv_qrows(src, n, gs, dst_h, dst_s, st);
+}
+
+int launch_nv_qrows_f16_f32(const float *src, long long n, float gs, uint16_t *dst_h,
+                            float *dst_s, cudaStream_t st)
+{
+    return launch_nv_qrows(src, n, gs, dst_h, dst_s, st);
 }
 
 } // namespace moe

@@ -10,6 +10,7 @@
 // for activations it is a constant the caller supplies.
 #pragma once
 
+#include <cuda_fp16.h>
 #include <cuda_fp4.h>
 #include <cuda_fp8.h>
 #include <stdint.h>
@@ -58,6 +59,21 @@ __device__ __forceinline__ uint8_t nv_quantize16(const float *v, float gs, uint2
     }
     codes = make_uint2(w[0], w[1]);
     return sc;
+}
+
+// Two E2M1 codes (one byte, the first element in the low nibble) -> the two
+// values as f16x2 (exact: every E2M1 value is an f16).
+__device__ __forceinline__ __half2 nv_pair_h2(uint32_t byte)
+{
+    const __half2_raw r = __nv_cvt_fp4x2_to_halfraw2((__nv_fp4x2_storage_t)(byte & 0xffu), __NV_E2M1);
+    return *reinterpret_cast<const __half2 *>(&r);
+}
+
+// The value of an E4M3 scale code (exact in fp32).
+__device__ __forceinline__ float nv_scale_value(uint32_t code)
+{
+    const __half_raw h = __nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)(code & 0xffu), __NV_E4M3);
+    return __half2float(*reinterpret_cast<const __half *>(&h));
 }
 
 // Scale layout for the block-scaled MMA with 16-element blocks: the scales

@@ -129,17 +129,27 @@ __device__ inline void hist_finish(int32_t *chunk_counts, int nchunks, int nj, i
                                    int *s_warp)
 {
     const int tid = threadIdx.x;
+    const int R = nj * nchunks;   // count rows of one expert, in rank order r = j * nchunks + c
+    constexpr int U = 16;         // loads in flight per thread
     for (int e = tid; e < MOE_MAX_E; e += blockDim.x) {
         int kept = 0;
         if (e < E) {
             int run = 0;
-            for (int j = 0; j < nj; ++j)
-                for (int c = 0; c < nchunks; ++c) {
-                    const size_t i = ((size_t)c * nj + j) * E + e;
-                    const int v = __ldcg(&chunk_counts[i]);
-                    __stcg(&chunk_counts[i], run);
-                    run += v;
+            for (int r0 = 0; r0 < R; r0 += U) {
+                int v[U];
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    const int r = r0 + u, j = r / nchunks, c = r - j * nchunks;
+                    v[u] = r < R ? __ldcg(&chunk_counts[((size_t)c * nj + j) * E + e]) : 0;
                 }
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    const int r = r0 + u, j = r / nchunks, c = r - j * nchunks;
+                    if (r < R)
+                        __stcg(&chunk_counts[((size_t)c * nj + j) * E + e], run);
+                    run += v[u];
+                }
+            }
             counts[e] = run;
             kept = (C > 0 && run > C) ? C : run;
         }

@@ -179,8 +179,8 @@ def test_forward_nvfp4_slot_priority_and_repeat():
 
 @pytest.mark.parametrize("T", [1, 2, 8])
 def test_nvfp4_small_batches(T):
-    """Decode-sized batches run the block-scaled tensor-core chain (the
-    chosen experts' codes are read once)."""
+    """Decode-sized batches: T <= 2 takes the NVFP4 decode kernels, T = 8 the
+    block-scaled tensor-core chain; both read each chosen expert's codes once."""
     w = small_workload("nvdec", T, 1024, 2048, 16, 2, d_ff_shared=256)
     inp = I.make_inputs(w, "cuda", seed=T)
     layer = M.MoeLayerNv4(inp, h_gs=2.0)
@@ -190,6 +190,45 @@ def test_nvfp4_small_batches(T):
     assert int(layer.status.item()) == 0
     _, _, ref = _oracle_out(inp, logits.cpu().numpy(), w.k, 0, np.float32(1.0), np.float32(2.0))
     assert_layer_close(out, ref, f"nvfp4 T={T}")
+
+
+@pytest.mark.parametrize("T", [1, 2])
+def test_nvfp4_decode_kernels_and_chain(T):
+    """The NVFP4 decode kernels (codes streamed through CUDA cores, exact
+    16-element block dot products) and the tensor-core chain on the same
+    inputs, both against the oracle, at d = 4096."""
+    w = small_workload("nvdk", T, 4096, 1536, 8, 2, zipf_s=0.5)
+    inp = I.make_inputs(w, "cuda", seed=10 + T)
+    x_gs = float(2688.0 / inp["x"].float().abs().max().item())
+    layer = M.MoeLayerNv4(inp, x_gs=x_gs, h_gs=2.0)
+    logits = torch.empty(T, w.E, dtype=torch.float32, device="cuda")
+    out_d = layer.forward(inp["x"], logits_out=logits, flags=M.MOE_FLAG_FORCE_DECODE).clone()
+    out_p = layer.forward(inp["x"], flags=M.MOE_FLAG_FORCE_PREFILL).clone()
+    out_0 = layer.forward(inp["x"]).clone()
+    torch.cuda.synchronize()
+    assert int(layer.status.item()) == 0
+    _, _, ref = _oracle_out(inp, logits.cpu().numpy(), w.k, 0, np.float32(x_gs), np.float32(2.0))
+    assert_layer_close(out_d, ref, f"nvfp4 decode kernels T={T}")
+    assert_layer_close(out_p, ref, f"nvfp4 tensor-core chain T={T}")
+    # the default path at T <= 2 is the decode kernels (deterministic: fixed order)
+    assert torch.equal(out_0, out_d)
+
+
+@pytest.mark.parametrize("C", [0, 1])
+def test_nvfp4_decode_shared_many_experts(C):
+    """Decode kernels with 64 experts, top-8, a shared expert and (C = 1) a
+    capacity that drops the second token's repeated experts."""
+    w = small_workload("nvdec2", 2, 1024, 512, 64, 8, capacity=C, d_ff_shared=256, zipf_s=3.0)
+    inp = I.make_inputs(w, "cuda", seed=2)
+    layer = M.MoeLayerNv4(inp, h_gs=1.5)
+    logits = torch.empty(w.T, w.E, dtype=torch.float32, device="cuda")
+    out = layer.forward(inp["x"], logits_out=logits)
+    torch.cuda.synchronize()
+    assert int(layer.status.item()) == 0
+    _, disp, ref = _oracle_out(inp, logits.cpu().numpy(), w.k, C, np.float32(1.0), np.float32(1.5))
+    if C:
+        assert (disp["slot_pos"] < 0).any()
+    assert_layer_close(out, ref, f"nvfp4 decode shared C={C}")
 
 
 def test_nvfp4_is_closer_to_bf16_than_its_error_bound():
