@@ -297,6 +297,48 @@ def time_loop(fn, steps, stream):
     return s.elapsed_time(e) / steps
 
 
+def run_route_only(a, world, rank, local):
+    """Profiling aid: moe_route (the router GEMM with its top-k) alone on the
+    workload's x and W_g, K timed calls; no expert weights are allocated.
+    Reports GB/s over the bytes the router must read (x, W_g) and write
+    (logits, indices, weights)."""
+    from sparse_mixture_experts_17_b200 import build as B
+    from sparse_mixture_experts_17_b200 import moe as M
+    if rank == 0 or not os.path.exists(M.LIB_PATH):
+        B.build()
+    barrier(world)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    peaks, peak_src = load_peaks()
+    w = I.WORKLOADS[a.workload]
+    if a.tokens:
+        w = w.with_T(a.tokens)
+    inp = I.make_inputs(w, dev, seed=0, router_only=True)
+    s = M.shape_of(w)
+    ws = M.alloc_workspace(s, dev)
+    logits = torch.empty(w.T, w.E, dtype=torch.float32, device=dev)
+    idx = torch.empty(w.T, w.k, dtype=torch.int32, device=dev)
+    wts = torch.empty(w.T, w.k, dtype=torch.float32, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def step():
+        M.moe_route(s, inp["x"], inp["wg"], inp["bias"], logits, idx, wts, status, ws)
+    for _ in range(a.warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = max_over_ranks(time_loop(step, a.steps, stream), world, dev)
+    nbytes = w.T * w.d * 2 + w.E * w.d * 2 + w.T * w.E * 4 + w.T * w.k * 8
+    gbs = nbytes / (ms / 1e3) / 1e9
+    return {"metric": "moe_route GB/s (router GEMM + top-k)", "value": round(gbs, 1),
+            "unit": "GB/s", "n_gpus": world, "steps": a.steps, "warmup": a.warmup,
+            "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": config_of(w, world), "bytes_per_step": nbytes,
+            "frac_hbm": round(gbs / peaks["hbm_gbs"], 4), "peak_source": f"{peak_src} hbm_gbs"}
+
+
 def run_ours(a, world, rank, local):
     from sparse_mixture_experts_17_b200 import build as B
     from sparse_mixture_experts_17_b200 import moe as M
@@ -874,6 +916,8 @@ def main(argv=None):
     ap.add_argument("--mxfp8", action="store_true",
                     help="time the layer on MXFP8 experts (moe_forward_mxfp8) instead of bf16; "
                          "no extras, no end-to-end run")
+    ap.add_argument("--route-only", action="store_true",
+                    help="profiling aid: time moe_route alone (no expert weights allocated)")
     ap.add_argument("--nvfp4", action="store_true",
                     help="time the layer on NVFP4 experts (moe_forward_nvfp4) instead of bf16; "
                          "no extras, no end-to-end run")
@@ -887,7 +931,7 @@ def main(argv=None):
         print(json.dumps(run_reference(a, world, rank)), flush=True)
         return 0
     world, rank, local = dist_setup(True)
-    res = run_ours(a, world, rank, local)
+    res = run_route_only(a, world, rank, local) if a.route_only else run_ours(a, world, rank, local)
     if rank == 0:
         print(json.dumps(res), flush=True)
     if world > 1:

@@ -47,6 +47,10 @@ namespace moe {
 #ifndef MOE_GM_2SM_W2
 #define MOE_GM_2SM_W2 8
 #endif
+// k-blocks of B the producer asks L2 for ahead of its shared-memory copies.
+#ifndef MOE_B_PREFETCH
+#define MOE_B_PREFETCH 8
+#endif
 
 struct TcArgs {
     int kblocks;
@@ -446,6 +450,12 @@ __global__ void __launch_bounds__(192, 1)
 
     if (warp == 0) {
         if (lane == 0 && !p.starve) {   // ---------------- TMA producer
+            // B rows of an expert whose rows fit one m-tile are read by that
+            // tile alone: they enter L2 as evict-first, so streaming them does
+            // not push out the activation rows and the weights that other
+            // tiles still reuse
+            const uint64_t pol_once = l2_policy_evict_first();
+            const uint64_t pol_reuse = l2_policy_evict_normal();
             uint32_t it = 0;
             for (long long tile = blockIdx.x; tile < total; tile += gridDim.x) {
                 int m_idx, n_idx;
@@ -453,20 +463,29 @@ __global__ void __launch_bounds__(192, 1)
                 const int row0 = p.mt_row0 ? p.mt_row0[m_idx] : m_idx * C::BM;
                 const int grp = p.mt_group ? (p.mt_group[m_idx] & ~kHalfTileBit) : 0;
                 const int brow = grp * p.b_rows_per_group + n_idx * BN;
+                const bool once = p.seg_offsets && p.mt_group && p.b_rows_per_group > 0 &&
+                                  p.seg_offsets[grp + 1] - p.seg_offsets[grp] <= C::BM;
+                const uint64_t pol_b = once ? pol_once : pol_reuse;
                 // K-grouped GEMMs contract over their group's own k-block range
                 const int kb0 = p.grp_kb0 ? p.grp_kb0[grp] : 0;
                 const int nkb = p.grp_kb0 ? p.grp_nkb[grp] : p.kblocks;
                 bool ok = true;
+                if (MOE_B_PREFETCH > 0)
+                    for (int q = 0; q < MOE_B_PREFETCH && q < nkb; ++q)
+                        tma_prefetch_l2_2d(&tmB, (kb0 + q) * C::BK, brow, pol_b);
                 for (int kb = 0; kb < nkb; ++kb, ++it) {
                     const int s = it % C::STAGES;
                     const uint32_t ph = (it / C::STAGES) & 1u;
+                    if (MOE_B_PREFETCH > 0 && kb + MOE_B_PREFETCH < nkb)
+                        tma_prefetch_l2_2d(&tmB, (kb0 + kb + MOE_B_PREFETCH) * C::BK, brow, pol_b);
                     if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag, p.status, p.wait_ns)) {
                         ok = false;
                         break;
                     }
                     mbar_arrive_expect_tx(&full[s], C::STAGE_BYTES);
                     tma_load_2d(sA + s * C::A_BYTES, &tmA, (kb0 + kb) * C::BK, row0, &full[s]);
-                    tma_load_2d(sB + s * C::B_BYTES, &tmB, (kb0 + kb) * C::BK, brow, &full[s]);
+                    tma_load_2d_hint(sB + s * C::B_BYTES, &tmB, (kb0 + kb) * C::BK, brow, &full[s],
+                                     pol_b);
                 }
                 if (!ok)
                     break;

@@ -81,6 +81,12 @@ int launch_hist_scan(const moe_shape_t &s, const int32_t *idx, int32_t *chunk_co
                      int32_t *n_kept, int32_t *mt_row0, int32_t *mt_group, int32_t *num_mt,
                      int32_t *mt2_row0, int32_t *mt2_group, int32_t *num_mt2, uint32_t *status,
                      cudaStream_t st, int32_t *tile_start = nullptr);
+// Top-k of router logits and the histogram in one launch (zeroes the ticket first).
+int launch_topk_hist(const moe_shape_t &s, const float *logits, int32_t *idx, float *w,
+                     int32_t *chunk_counts, int32_t *rank_local, int32_t *counter, int32_t *counts,
+                     int32_t *offsets, int32_t *n_kept, int32_t *mt_row0, int32_t *mt_group,
+                     int32_t *num_mt, int32_t *mt2_row0, int32_t *mt2_group, int32_t *num_mt2,
+                     uint32_t *status, cudaStream_t st, int32_t *tile_start = nullptr);
 int launch_permute(const moe_shape_t &s, const int32_t *idx, const int32_t *chunk_base,
                    const int32_t *rank_local, const int32_t *offsets, const uint16_t *x,
                    int32_t *slot_pos, int32_t *perm_token, uint16_t *x_perm, float *out_zero,

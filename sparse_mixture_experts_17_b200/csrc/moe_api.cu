@@ -533,10 +533,25 @@ static int forward_impl(const moe_shape_t &s, const WsLayout &L, void *ws, const
                           at<int32_t>(ws, L.mt2_row0),     at<int32_t>(ws, L.mt2_group),
                           at<int32_t>(ws, L.num_mt2)};
     const bool hist_fused = !decode && router_hist_fusable(s);
+    // a router GEMM of its own (E > 64): the top-k and the histogram share one launch
+    const bool topk_hist = !decode && !hist_fused && !router_topk_fusable(s) &&
+                           !dec_route_fusable(s);
     int rc;
     if (hist_fused) {
         StageMark m(MOE_STAGE_ROUTER, st);
         rc = router_topk_hist(s, x, Wg, bias, logits, idx, w, counter, hist, status, st);
+    } else if (topk_hist) {
+        {
+            StageMark m(MOE_STAGE_ROUTER, st);
+            rc = router(s, x, Wg, bias, logits, status, st);
+        }
+        if (!rc) {
+            StageMark m(MOE_STAGE_TOPK, st);
+            rc = launch_topk_hist(s, logits, idx, w, hist.chunk, hist.rank, counter, hist.counts,
+                                  hist.offsets, hist.n_kept, hist.mt_row0, hist.mt_group,
+                                  hist.num_mt, hist.mt2_row0, hist.mt2_group, hist.num_mt2, status,
+                                  st);
+        }
     } else {
         rc = route_tokens(s, x, Wg, bias, logits, idx, w, counter, status, st);
     }
@@ -563,7 +578,7 @@ static int forward_impl(const moe_shape_t &s, const WsLayout &L, void *ws, const
     int32_t *slot_pos = at<int32_t>(ws, L.slot_pos);
     int32_t *perm_token = at<int32_t>(ws, L.perm_token);
     uint16_t *x_perm = at<uint16_t>(ws, L.x_perm);
-    if (!hist_fused) {
+    if (!hist_fused && !topk_hist) {
         StageMark m(MOE_STAGE_HIST, st);
         rc = launch_hist_scan(s, idx, chunk, rank, counter, counts, offsets,
                               at<int32_t>(ws, L.n_kept), at<int32_t>(ws, L.mt_row0),

@@ -65,8 +65,11 @@ def zipf_bias(E: int, s: float, seed: int) -> torch.Tensor:
     return (-s * torch.log(r)).to(torch.float32)
 
 
-def make_inputs(w: Workload, device="cpu", seed: int = 0, with_bias: bool | None = None) -> dict:
-    """Draw the workload's tensors on ``device`` (bf16 weights, fp32 bias)."""
+def make_inputs(w: Workload, device="cpu", seed: int = 0, with_bias: bool | None = None,
+                router_only: bool = False) -> dict:
+    """Draw the workload's tensors on ``device`` (bf16 weights, fp32 bias).
+    router_only: stop after x and W_g (the same values as the full draw) and
+    the bias; no expert weights."""
     dev = torch.device(device)
     g = torch.Generator(device=dev).manual_seed(seed)
     bf = torch.bfloat16
@@ -86,6 +89,12 @@ def make_inputs(w: Workload, device="cpu", seed: int = 0, with_bias: bool | None
     inp = dict(workload=w)
     inp["x"] = normal((w.T, w.d), 1.0)
     inp["wg"] = normal((w.E, w.d), 0.02)
+    if router_only:
+        use_bias = (w.zipf_s != 0.0) if with_bias is None else with_bias
+        inp["bias"] = zipf_bias(w.E, w.zipf_s, seed).to(dev) if use_bias else None
+        inp["k"] = w.k
+        inp["capacity"] = w.capacity
+        return inp
     inp["W1"] = stacked(w.E, w.d_ff, w.d)
     inp["W3"] = stacked(w.E, w.d_ff, w.d)
     inp["W2"] = stacked(w.E, w.d, w.d_ff)
