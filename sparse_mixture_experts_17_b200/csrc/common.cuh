@@ -157,45 +157,6 @@ __device__ __forceinline__ void tma_load_2d(void *smem_dst, const void *tmap, in
         : "memory");
 }
 
-// The same copy with an L2 eviction-priority policy (createpolicy) for the
-// lines it brings in.
-__device__ __forceinline__ void tma_load_2d_hint(void *smem_dst, const void *tmap, int c0, int c1,
-                                                 uint64_t *bar, uint64_t policy)
-{
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
-        " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_u32(smem_dst)),
-        "l"(tmap), "r"(c0), "r"(c1), "r"(smem_u32(bar)), "l"(policy)
-        : "memory");
-}
-
-// Bring a 2-D tile into L2 only (no shared memory, no completion to wait
-// for): issued some stages ahead of the copy that will read it, it lets a
-// stream of tiles from DRAM keep more bytes in flight than the shared-memory
-// ring holds.
-__device__ __forceinline__ void tma_prefetch_l2_2d(const void *tmap, int c0, int c1, uint64_t policy)
-{
-    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile.L2::cache_hint [%0, {%1, %2}], %3;"
-                 ::"l"(tmap), "r"(c0), "r"(c1), "l"(policy)
-                 : "memory");
-}
-
-// L2 policies: lines marked evict-first go before any others; evict-normal
-// is the default priority.
-__device__ __forceinline__ uint64_t l2_policy_evict_first()
-{
-    uint64_t p;
-    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
-    return p;
-}
-
-__device__ __forceinline__ uint64_t l2_policy_evict_normal()
-{
-    uint64_t p;
-    asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(p));
-    return p;
-}
-
 // ------------------------------------------------------------------ tcgen05
 
 __device__ __forceinline__ void tmem_alloc(uint32_t *smem_result, uint32_t ncols)

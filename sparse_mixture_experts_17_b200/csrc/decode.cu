@@ -708,23 +708,21 @@ __device__ __forceinline__ float nv_block_dot(uint32_t w0, uint32_t w1, const ui
     return f.x + f.y;
 }
 
-// One 16-byte chunk of a code row (32 elements = blocks 2ci and 2ci + 1)
-// against one row of values (f16) and block scales (fp32): sum over both
-// blocks of the exact block dot times s_w(block) * s_x(block).
-__device__ __forceinline__ float nv_chunk_dot(const uint4 &w, uint32_t sw2, const uint4 *xh,
-                                              const float2 &xs, int ci)
+// One 16-byte chunk of a code row (32 elements = two blocks) against the
+// same 32 values of x or h (f16, x[0..3]) and their two block scales: the sum
+// over both blocks of the exact block dot times s_w(block) * s_x(block).
+__device__ __forceinline__ float nv_chunk_dot(const uint4 &w, float sw0, float sw1, const uint4 (&x)[4],
+                                              const float2 &xs)
 {
-    const uint4 x0 = __ldg(xh + 4 * ci), x1 = __ldg(xh + 4 * ci + 1);
-    const uint4 x2 = __ldg(xh + 4 * ci + 2), x3 = __ldg(xh + 4 * ci + 3);
-    const float b0 = nv_block_dot(w.x, w.y, x0, x1);
-    const float b1 = nv_block_dot(w.z, w.w, x2, x3);
-    return fmaf(b1, nv_scale_value(sw2 >> 8) * xs.y, b0 * (nv_scale_value(sw2) * xs.x));
+    const float b0 = nv_block_dot(w.x, w.y, x[0], x[1]);
+    const float b1 = nv_block_dot(w.z, w.w, x[2], x[3]);
+    return fmaf(b1, sw1 * xs.y, b0 * (sw0 * xs.x));
 }
 
 // Phase 1: one work unit = h column c of one chosen expert (its packed gate
 // and up rows, each streamed once), or of the shared expert.
 template <int MAXT>
-__global__ void __launch_bounds__(256, 4)
+__global__ void __launch_bounds__(256, 2)
     k_dec_w13_nv(const uint16_t *__restrict__ xh, const float *__restrict__ xs, float x_gs,
                  const int32_t *__restrict__ idx, int T, int d, int d_ff, int E, int k, int C,
                  int slot_major, const uint8_t *__restrict__ W13q,
@@ -808,12 +806,17 @@ __global__ void __launch_bounds__(256, 4)
                 const int ci = cb + lane + 32 * i;
                 if (ci >= nv)
                     continue;
+                const float g0 = nv_scale_value(sg[i]), g1 = nv_scale_value(sg[i] >> 8);
+                const float u0 = nv_scale_value(su[i]), u1 = nv_scale_value(su[i] >> 8);
 #pragma unroll
                 for (int s = 0; s < MAXT; ++s) {
                     if (s < na) {
+                        // x's 32 values and two scales, loaded once for the gate and up rows
+                        const uint4 xv[4] = {__ldg(xr[s] + 4 * ci), __ldg(xr[s] + 4 * ci + 1),
+                                             __ldg(xr[s] + 4 * ci + 2), __ldg(xr[s] + 4 * ci + 3)};
                         const float2 xsc = __ldg(sr[s] + ci);
-                        ag[s] += nv_chunk_dot(wg[i], sg[i], xr[s], xsc, ci);
-                        au[s] += nv_chunk_dot(wu[i], su[i], xr[s], xsc, ci);
+                        ag[s] += nv_chunk_dot(wg[i], g0, g1, xv, xsc);
+                        au[s] += nv_chunk_dot(wu[i], u0, u1, xv, xsc);
                     }
                 }
             }
@@ -837,7 +840,7 @@ __global__ void __launch_bounds__(256, 4)
 // then the shared expert, stream W2_e[r] once and dot it with each of the
 // expert's assignments' h rows; fixed order (deterministic).
 template <int MAXT>
-__global__ void __launch_bounds__(256, 4)
+__global__ void __launch_bounds__(256, 2)
     k_dec_w2_nv(const int32_t *__restrict__ idx, const float *__restrict__ topk_w, int T, int d,
                 int d_ff, int E, int k, int C, int slot_major, const uint8_t *__restrict__ W2q,
                 const uint8_t *__restrict__ W2sf, const float *__restrict__ gs2, int d_ff_s,
@@ -906,10 +909,14 @@ __global__ void __launch_bounds__(256, 4)
                     const int ci = cb + lane + 32 * i;
                     if (ci >= nv)
                         continue;
+                    const float f0 = nv_scale_value(sc[i]), f1 = nv_scale_value(sc[i] >> 8);
 #pragma unroll
                     for (int s = 0; s < MAXT; ++s)
-                        if (s < na)
-                            pa[s] += nv_chunk_dot(wv[i], sc[i], hr[s], __ldg(sr[s] + ci), ci);
+                        if (s < na) {
+                            const uint4 hv[4] = {__ldg(hr[s] + 4 * ci), __ldg(hr[s] + 4 * ci + 1),
+                                                 __ldg(hr[s] + 4 * ci + 2), __ldg(hr[s] + 4 * ci + 3)};
+                            pa[s] += nv_chunk_dot(wv[i], f0, f1, hv, __ldg(sr[s] + ci));
+                        }
                 }
             }
 #pragma unroll
@@ -1119,7 +1126,7 @@ int launch_dec_w13_nv(const moe_shape_t &s, const uint16_t *xh, const float *xs,
         return MOE_OK;
     if (s.T > 2)
         return MOE_ERR_UNSUPPORTED;
-    const int blocks = num_sms() * 4;
+    const int blocks = num_sms() * 2;
     float *Hs = H32 + (size_t)s.T * s.k * s.d_ff;
     const uint8_t *wq = s.d_ff_shared ? W13s_q : nullptr;
     if (s.T == 1)
@@ -1143,7 +1150,7 @@ int launch_dec_w2_nv(const moe_shape_t &s, const int32_t *topk_idx, const float 
         return MOE_OK;
     if (s.T > 2)
         return MOE_ERR_UNSUPPORTED;
-    const int blocks = num_sms() * 4;
+    const int blocks = num_sms() * 2;
     const uint8_t *wq = s.d_ff_shared ? W2s_q : nullptr;
     if (s.T == 1)
         launch_pdl(k_dec_w2_nv<1>, blocks, 256, st, topk_idx, topk_w, s.T, s.d, s.d_ff, s.E, s.k,

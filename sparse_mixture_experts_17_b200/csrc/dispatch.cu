@@ -174,7 +174,7 @@ __device__ __forceinline__ void hist_scan_chunk(
     int32_t *chunk_counts, int32_t *__restrict__ rank_local, int32_t *counter,
     int32_t *__restrict__ counts, int32_t *__restrict__ offsets, int32_t *__restrict__ n_kept,
     int32_t *mt_row0, int32_t *mt_group, int32_t *num_mt, int32_t *mt2_row0, int32_t *mt2_group,
-    int32_t *num_mt2, int32_t *tile_start, uint32_t *status)
+    int32_t *num_mt2, int32_t *tile_start, uint32_t *status, int shared_rows)
 {
     __shared__ uint32_t mask[8][MOE_MAX_E];
     __shared__ int32_t wpre[8][MOE_MAX_E];
@@ -264,7 +264,7 @@ __device__ __forceinline__ void hist_scan_chunk(
     __threadfence();
     hist_finish(chunk_counts, gridDim.x, slot_major ? k : 1, E, C, counts, offsets, n_kept,
                 mt_row0, mt_group, num_mt, mt2_row0, mt2_group, num_mt2, tile_start, counter,
-                s_kept, s_off, s_warp);
+                s_kept, s_off, s_warp, shared_rows);
 }
 
 __global__ void __launch_bounds__(256) k_hist_scan(
@@ -272,76 +272,18 @@ __global__ void __launch_bounds__(256) k_hist_scan(
     int32_t *chunk_counts, int32_t *__restrict__ rank_local, int32_t *counter,
     int32_t *__restrict__ counts, int32_t *__restrict__ offsets, int32_t *__restrict__ n_kept,
     int32_t *mt_row0, int32_t *mt_group, int32_t *num_mt, int32_t *mt2_row0, int32_t *mt2_group,
-    int32_t *num_mt2, int32_t *tile_start, uint32_t *status)
+    int32_t *num_mt2, int32_t *tile_start, uint32_t *status, int shared_rows)
 {
     hist_scan_chunk(idx, T, E, k, C, slot_major, chunk_counts, rank_local, counter, counts,
                     offsets, n_kept, mt_row0, mt_group, num_mt, mt2_row0, mt2_group, num_mt2,
-                    tile_start, status);
-}
-
-// Top-k and the histogram in one launch, for logits the router GEMM wrote
-// (E > 64, or any E when the router keeps its own epilogue): each CTA first
-// runs the warp top-k of its chunk's 256 tokens (32 per warp, the routine of
-// k_topk), writes their experts and weights, and then, after a barrier that
-// makes them visible to the block, takes the chunk's histogram exactly as
-// k_hist_scan does; the last CTA scans. The ticket must be zero at launch.
-template <int VPL>
-__global__ void __launch_bounds__(256) k_topk_hist(
-    const float *__restrict__ logits, int32_t *idx, float *__restrict__ w, int T, int E, int k,
-    int C, int slot_major, int32_t *chunk_counts, int32_t *__restrict__ rank_local,
-    int32_t *counter, int32_t *__restrict__ counts, int32_t *__restrict__ offsets,
-    int32_t *__restrict__ n_kept, int32_t *mt_row0, int32_t *mt_group, int32_t *num_mt,
-    int32_t *mt2_row0, int32_t *mt2_group, int32_t *num_mt2, int32_t *tile_start, uint32_t *status)
-{
-    const int warp = threadIdx.x >> 5;
-    for (int tt = warp; tt < kChunkTokens; tt += 8) {
-        const int t = blockIdx.x * kChunkTokens + tt;
-        if (t < T)
-            warp_topk_row<VPL>(logits + (size_t)t * E, E, k, idx + (size_t)t * k,
-                               w + (size_t)t * k, status);
-    }
-    __syncthreads();
-    hist_scan_chunk(idx, T, E, k, C, slot_major, chunk_counts, rank_local, counter, counts,
-                    offsets, n_kept, mt_row0, mt_group, num_mt, mt2_row0, mt2_group, num_mt2,
-                    tile_start, status);
-}
-
-int launch_topk_hist(const moe_shape_t &s, const float *logits, int32_t *idx, float *w,
-                     int32_t *chunk_counts, int32_t *rank_local, int32_t *counter, int32_t *counts,
-                     int32_t *offsets, int32_t *n_kept, int32_t *mt_row0, int32_t *mt_group,
-                     int32_t *num_mt, int32_t *mt2_row0, int32_t *mt2_group, int32_t *num_mt2,
-                     uint32_t *status, cudaStream_t st, int32_t *tile_start)
-{
-    const int nchunks = (s.T + kChunkTokens - 1) / kChunkTokens;
-    if (nchunks == 0)
-        return MOE_OK;
-    // the ticket starts at zero whatever an earlier, aborted call left in it
-    if (cudaMemsetAsync(counter, 0, sizeof(int32_t), st) != cudaSuccess)
-        return MOE_ERR_CUDA;
-    const int vpl = (s.E + 31) / 32;
-#define MOE_TOPK_HIST(V)                                                                         \
-    k_topk_hist<V><<<nchunks, 256, 0, st>>>(logits, idx, w, s.T, s.E, s.k, s.capacity,        \
-                                            slot_major(s), chunk_counts, rank_local, counter,  \
-                                            counts, offsets, n_kept, mt_row0, mt_group,        \
-                                            num_mt, mt2_row0, mt2_group, num_mt2, tile_start,  \
-                                            status)
-    if (vpl <= 1)
-        MOE_TOPK_HIST(1);
-    else if (vpl <= 2)
-        MOE_TOPK_HIST(2);
-    else if (vpl <= 4)
-        MOE_TOPK_HIST(4);
-    else
-        MOE_TOPK_HIST(8);
-#undef MOE_TOPK_HIST
-    return launched();
+                    tile_start, status, shared_rows);
 }
 
 int launch_hist_scan(const moe_shape_t &s, const int32_t *idx, int32_t *chunk_counts,
                      int32_t *rank_local, int32_t *counter, int32_t *counts, int32_t *offsets,
                      int32_t *n_kept, int32_t *mt_row0, int32_t *mt_group, int32_t *num_mt,
                      int32_t *mt2_row0, int32_t *mt2_group, int32_t *num_mt2, uint32_t *status,
-                     cudaStream_t st, int32_t *tile_start)
+                     cudaStream_t st, int32_t *tile_start, int shared_rows)
 {
     const int nchunks = (s.T + kChunkTokens - 1) / kChunkTokens;
     if (nchunks == 0)
@@ -349,7 +291,7 @@ int launch_hist_scan(const moe_shape_t &s, const int32_t *idx, int32_t *chunk_co
     k_hist_scan<<<nchunks, 256, 0, st>>>(idx, s.T, s.E, s.k, s.capacity, slot_major(s),
                                          chunk_counts, rank_local, counter, counts, offsets,
                                          n_kept, mt_row0, mt_group, num_mt, mt2_row0, mt2_group,
-                                         num_mt2, tile_start, status);
+                                         num_mt2, tile_start, status, shared_rows);
     return launched();
 }
 
