@@ -169,12 +169,12 @@ int launch_topk(const moe_shape_t &s, const float *logits, int32_t *idx, float *
 // Slot-major priority: the same per slot, with counts per (chunk, slot), and
 // the scan runs over slots, then chunks, so that every first choice ranks
 // before any second choice.
-__device__ __forceinline__ void hist_scan_chunk(
+__global__ void __launch_bounds__(256) k_hist_scan(
     const int32_t *__restrict__ idx, int T, int E, int k, int C, int slot_major,
     int32_t *chunk_counts, int32_t *__restrict__ rank_local, int32_t *counter,
     int32_t *__restrict__ counts, int32_t *__restrict__ offsets, int32_t *__restrict__ n_kept,
     int32_t *mt_row0, int32_t *mt_group, int32_t *num_mt, int32_t *mt2_row0, int32_t *mt2_group,
-    int32_t *num_mt2, int32_t *tile_start, uint32_t *status, int shared_rows)
+    int32_t *num_mt2, int32_t *tile_start, uint32_t *status)
 {
     __shared__ uint32_t mask[8][MOE_MAX_E];
     __shared__ int32_t wpre[8][MOE_MAX_E];
@@ -264,26 +264,14 @@ __device__ __forceinline__ void hist_scan_chunk(
     __threadfence();
     hist_finish(chunk_counts, gridDim.x, slot_major ? k : 1, E, C, counts, offsets, n_kept,
                 mt_row0, mt_group, num_mt, mt2_row0, mt2_group, num_mt2, tile_start, counter,
-                s_kept, s_off, s_warp, shared_rows);
-}
-
-__global__ void __launch_bounds__(256) k_hist_scan(
-    const int32_t *__restrict__ idx, int T, int E, int k, int C, int slot_major,
-    int32_t *chunk_counts, int32_t *__restrict__ rank_local, int32_t *counter,
-    int32_t *__restrict__ counts, int32_t *__restrict__ offsets, int32_t *__restrict__ n_kept,
-    int32_t *mt_row0, int32_t *mt_group, int32_t *num_mt, int32_t *mt2_row0, int32_t *mt2_group,
-    int32_t *num_mt2, int32_t *tile_start, uint32_t *status, int shared_rows)
-{
-    hist_scan_chunk(idx, T, E, k, C, slot_major, chunk_counts, rank_local, counter, counts,
-                    offsets, n_kept, mt_row0, mt_group, num_mt, mt2_row0, mt2_group, num_mt2,
-                    tile_start, status, shared_rows);
+                s_kept, s_off, s_warp);
 }
 
 int launch_hist_scan(const moe_shape_t &s, const int32_t *idx, int32_t *chunk_counts,
                      int32_t *rank_local, int32_t *counter, int32_t *counts, int32_t *offsets,
                      int32_t *n_kept, int32_t *mt_row0, int32_t *mt_group, int32_t *num_mt,
                      int32_t *mt2_row0, int32_t *mt2_group, int32_t *num_mt2, uint32_t *status,
-                     cudaStream_t st, int32_t *tile_start, int shared_rows)
+                     cudaStream_t st, int32_t *tile_start)
 {
     const int nchunks = (s.T + kChunkTokens - 1) / kChunkTokens;
     if (nchunks == 0)
@@ -291,7 +279,7 @@ int launch_hist_scan(const moe_shape_t &s, const int32_t *idx, int32_t *chunk_co
     k_hist_scan<<<nchunks, 256, 0, st>>>(idx, s.T, s.E, s.k, s.capacity, slot_major(s),
                                          chunk_counts, rank_local, counter, counts, offsets,
                                          n_kept, mt_row0, mt_group, num_mt, mt2_row0, mt2_group,
-                                         num_mt2, tile_start, status, shared_rows);
+                                         num_mt2, tile_start, status);
     return launched();
 }
 

@@ -86,15 +86,6 @@ struct TcArgs {
     // no loads, so the first wait on a full stage runs out and every role unwinds
     unsigned long long wait_ns;
     int starve;
-    // the shared expert run inside a routed grouped GEMM: tiles of group
-    // shared_grp read their A rows from the second A map (the token batch),
-    // their B rows from the second B map (row n_idx * BN), end at rows_shared,
-    // and write out_s (EPI_SWIGLU) or add into out[row] with weight 1
-    // (EPI_COMBINE); -1: no such group
-    int shared_grp;
-    long long rows_shared;
-    void *out_s;
-    int hist_shared_rows;   // the folded histogram's tile list: shared tiles to add
 };
 
 // Shared memory of the histogram folded into the router (E <= 64): per-warp
@@ -182,8 +173,7 @@ __device__ __forceinline__ void tile_coords(long long tile, int num_mt, int n_ti
 // lanes run it; only rows inside the expert's segment (`valid`) are written.
 template <int BN, int MODE>
 __device__ __forceinline__ void epilogue_tile(const TcArgs &p, uint32_t tb, long long row,
-                                              bool valid, int n_idx, int grp, bool empty_k,
-                                              bool sh)
+                                              bool valid, int n_idx, int grp, bool empty_k)
 {
     if (MODE == EPI_SWIGLU_SAVE) {
         // as EPI_SWIGLU, and the raw accumulators (gate | up of this 128-column
@@ -268,7 +258,7 @@ __device__ __forceinline__ void epilogue_tile(const TcArgs &p, uint32_t tb, long
             atomicAdd(p.row_dot + row, dot);
     } else if (MODE == EPI_SWIGLU) {
         // accumulator columns [0,128) = gate, [128,256) = up of H columns n_idx*128..
-        uint16_t *H = static_cast<uint16_t *>(sh ? p.out_s : p.out) + row * p.ldo + n_idx * 128;
+        uint16_t *H = static_cast<uint16_t *>(p.out) + row * p.ldo + n_idx * 128;
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
             float g[32], u[32];
@@ -290,10 +280,7 @@ __device__ __forceinline__ void epilogue_tile(const TcArgs &p, uint32_t tb, long
     } else if (MODE == EPI_COMBINE) {
         int t = 0;
         float wgt = 0.f;
-        if (valid && sh) {   // the shared expert: rows are tokens, weight 1
-            t = (int)row;
-            wgt = 1.f;
-        } else if (valid) {
+        if (valid) {
             t = p.perm_token ? p.perm_token[row] : (int)row;   // NULL: rows are tokens
             if (p.perm_w) {
                 wgt = p.perm_w[row];
@@ -409,7 +396,6 @@ __device__ __forceinline__ void epilogue_tile(const TcArgs &p, uint32_t tb, long
 template <int BN, int MODE>
 __global__ void __launch_bounds__(192, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-              const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
               const TcArgs p)
 {
     using C = TcCfg<BN>;
@@ -441,10 +427,6 @@ __global__ void __launch_bounds__(192, 1)
     if (warp == 0 && lane == 0) {
         tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmB);
-        if (p.shared_grp >= 0) {
-            tma_prefetch_desc(&tmA2);
-            tma_prefetch_desc(&tmB2);
-        }
         // the fused router also re-arms the histogram kernel's ticket (which
         // runs after this kernel in stream order)
         if (MODE == EPI_ROUTER_TOPK && blockIdx.x == 0 && p.counter_zero)
@@ -470,11 +452,7 @@ __global__ void __launch_bounds__(192, 1)
                 tile_coords(tile, num_mt, p.n_tiles, p.group_m, m_idx, n_idx);
                 const int row0 = p.mt_row0 ? p.mt_row0[m_idx] : m_idx * C::BM;
                 const int grp = p.mt_group ? (p.mt_group[m_idx] & ~kHalfTileBit) : 0;
-                const bool sh = grp == p.shared_grp;
-                const void *ta = sh ? static_cast<const void *>(&tmA2) : static_cast<const void *>(&tmA);
-                const void *tb = sh ? static_cast<const void *>(&tmB2) : static_cast<const void *>(&tmB);
-                const int brow = sh ? n_idx * BN : grp * p.b_rows_per_group + n_idx * BN;
-
+                const int brow = grp * p.b_rows_per_group + n_idx * BN;
                 // K-grouped GEMMs contract over their group's own k-block range
                 const int kb0 = p.grp_kb0 ? p.grp_kb0[grp] : 0;
                 const int nkb = p.grp_kb0 ? p.grp_nkb[grp] : p.kblocks;
@@ -487,8 +465,8 @@ __global__ void __launch_bounds__(192, 1)
                         break;
                     }
                     mbar_arrive_expect_tx(&full[s], C::STAGE_BYTES);
-                    tma_load_2d(sA + s * C::A_BYTES, ta, (kb0 + kb) * C::BK, row0, &full[s]);
-                    tma_load_2d(sB + s * C::B_BYTES, tb, (kb0 + kb) * C::BK, brow, &full[s]);
+                    tma_load_2d(sA + s * C::A_BYTES, &tmA, (kb0 + kb) * C::BK, row0, &full[s]);
+                    tma_load_2d(sB + s * C::B_BYTES, &tmB, (kb0 + kb) * C::BK, brow, &full[s]);
                 }
                 if (!ok)
                     break;
@@ -543,9 +521,7 @@ __global__ void __launch_bounds__(192, 1)
             const int gword = p.mt_group ? p.mt_group[m_idx] : 0;
             const int grp = gword & ~kHalfTileBit;
             const bool half = (gword & kHalfTileBit) != 0;
-            const bool sh = grp == p.shared_grp;
-            const long long row_end = sh ? p.rows_shared
-                                         : (p.seg_offsets ? p.seg_offsets[grp + 1] : p.rows_valid);
+            const long long row_end = p.seg_offsets ? p.seg_offsets[grp + 1] : p.rows_valid;
             const uint32_t b = local & 1u, aph = (local >> 1) & 1u;
             const bool got = mbar_wait(&tfull[b], aph, abort_flag, p.status, p.wait_ns);
             // the folded histogram's named barriers need every epilogue warp on
@@ -561,7 +537,7 @@ __global__ void __launch_bounds__(192, 1)
             const bool empty_k = p.grp_kb0 && p.grp_nkb[grp] == 0;
 
             if (got)
-                epilogue_tile<BN, MODE>(p, tb, row, valid, n_idx, grp, empty_k, sh);
+                epilogue_tile<BN, MODE>(p, tb, row, valid, n_idx, grp, empty_k);
             if constexpr (MODE == EPI_ROUTER_TOPK) {
                 if (p.hist_chunk)
                     router_hist_tile(p, *reinterpret_cast<RouterHistSmem *>(
@@ -595,7 +571,7 @@ __global__ void __launch_bounds__(192, 1)
                 hist_finish(p.hist_chunk, num_mt, 1, p.n_valid, p.capacity, p.hist_counts,
                             p.hist_offsets, p.hist_n_kept, p.hist_mt_row0, p.hist_mt_group,
                             p.hist_num_mt, p.hist_mt2_row0, p.hist_mt2_group, p.hist_num_mt2,
-                            nullptr, p.hist_counter, H.kept, H.off, H.warp, p.hist_shared_rows);
+                            nullptr, p.hist_counter, H.kept, H.off, H.warp);
             }
         }
     }
@@ -747,7 +723,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
             const long long row = row0 + q * 32 + lane;
             const bool valid = row < row_end;
             const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + b * BN;
-            epilogue_tile<BN, MODE>(p, tb, row, valid, n_idx, grp, false, false);
+            epilogue_tile<BN, MODE>(p, tb, row, valid, n_idx, grp, false);
             tc_fence_before();
             __syncwarp();
             if (lane == 0)
@@ -822,13 +798,6 @@ static int launch_tc_impl(const GemmArgs &g, cudaStream_t st)
     rc = make_tmap(&tB, g.B, g.K, g.b_rows_total, BN);
     if (rc)
         return rc;
-    CUtensorMap tA2 = tA, tB2 = tB;
-    if (g.shared_grp >= 0) {
-        if ((rc = make_tmap(&tA2, g.A2, g.K, g.a2_rows, 128)))
-            return rc;
-        if ((rc = make_tmap(&tB2, g.B2, g.K, g.b2_rows, BN)))
-            return rc;
-    }
     TcArgs p;
     p.kblocks = g.K / 64;
     p.n_tiles = (MODE == EPI_SWIGLU || MODE == EPI_SWIGLU_SAVE) ? g.N / 256 : (g.N + BN - 1) / BN;
@@ -878,10 +847,6 @@ static int launch_tc_impl(const GemmArgs &g, cudaStream_t st)
     p.capacity = g.capacity;
     p.starve = g.test_starve;
     p.wait_ns = g.test_starve ? kTestWaitLimitNs : kWaitLimitNs;
-    p.shared_grp = g.shared_grp;
-    p.rows_shared = g.rows_shared;
-    p.out_s = g.out_s;
-    p.hist_shared_rows = g.hist_shared_rows;
 
     // the router with the folded histogram also needs its tile-histogram area
     constexpr int SMEM = C::SMEM_BYTES + (MODE == EPI_ROUTER_TOPK ? (int)sizeof(RouterHistSmem) : 0);
@@ -899,7 +864,7 @@ static int launch_tc_impl(const GemmArgs &g, cudaStream_t st)
     if (tiles <= 0)
         return MOE_OK;
     const int grid = (int)std::min<long long>(tiles, num_sms());
-    k_gemm_tc<BN, MODE><<<grid, 192, SMEM, st>>>(tA, tB, tA2, tB2, p);
+    k_gemm_tc<BN, MODE><<<grid, 192, SMEM, st>>>(tA, tB, p);
     return launched();
 }
 

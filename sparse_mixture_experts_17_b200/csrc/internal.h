@@ -75,13 +75,12 @@ int launch_router_simt(const moe_shape_t &s, const uint16_t *x, const uint16_t *
                        const float *bias, float *logits, cudaStream_t st);
 int launch_topk(const moe_shape_t &s, const float *logits, int32_t *idx, float *w,
                 int32_t *counter_to_zero, uint32_t *status, cudaStream_t st);
-// Also writes the 256-row m-tile list of the 2-SM GEMM when mt2_row0 is non-NULL;
-// shared_rows > 0 adds the shared expert's tiles (group E) to the 128-row list.
+// Also writes the 256-row m-tile list of the 2-SM GEMM when mt2_row0 is non-NULL.
 int launch_hist_scan(const moe_shape_t &s, const int32_t *idx, int32_t *chunk_counts,
                      int32_t *rank_local, int32_t *counter, int32_t *counts, int32_t *offsets,
                      int32_t *n_kept, int32_t *mt_row0, int32_t *mt_group, int32_t *num_mt,
                      int32_t *mt2_row0, int32_t *mt2_group, int32_t *num_mt2, uint32_t *status,
-                     cudaStream_t st, int32_t *tile_start = nullptr, int shared_rows = 0);
+                     cudaStream_t st, int32_t *tile_start = nullptr);
 int launch_permute(const moe_shape_t &s, const int32_t *idx, const int32_t *chunk_base,
                    const int32_t *rank_local, const int32_t *offsets, const uint16_t *x,
                    int32_t *slot_pos, int32_t *perm_token, uint16_t *x_perm, float *out_zero,
@@ -195,15 +194,6 @@ struct GemmArgs {
     // the pipeline waits give up after 50 ms, so the launch returns with
     // MOE_ERR_TIMEOUT flagged and nothing in flight
     int test_starve;
-    // the shared expert inside the routed single-SM grouped GEMM (shared_grp = E;
-    // -1: none): its tiles read A2 [a2_rows, K] and B2 [b2_rows, K], end at
-    // rows_shared and write out_s (EPI_SWIGLU) or add into out with weight 1
-    // (EPI_COMBINE); the m-tile list holds their tiles as group E
-    int shared_grp;
-    const uint16_t *A2, *B2;
-    long long a2_rows, b2_rows, rows_shared;
-    void *out_s;
-    int hist_shared_rows;     // EPI_ROUTER_TOPK with the folded histogram: add these tiles
 };
 
 int launch_gemm_tc(const GemmArgs &g, cudaStream_t st);

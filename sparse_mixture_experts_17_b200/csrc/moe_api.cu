@@ -111,8 +111,7 @@ WsLayout ws_layout(const moe_shape_t &s)
     const size_t Kec = ec ? (size_t)std::min(std::max(s.capacity, 0), s.T) : 0;
     const size_t T = s.T, k = s.k, E = s.E, N = std::max(T * k, E * Kec);
     L.nchunks = (int)((T + kChunkTokens - 1) / kChunkTokens);
-    L.max_mt = (int)((N + kBlockM - 1) / kBlockM + E +
-                     (s.d_ff_shared > 0 ? (T + kBlockM - 1) / kBlockM : 0));
+    L.max_mt = (int)((N + kBlockM - 1) / kBlockM + E);
     L.max_mt2 = (int)((N + 2 * kBlockM - 1) / (2 * kBlockM) + E);
     L.logits = take(T * E * 4);
     L.topk_idx = take(N * 4);
@@ -267,27 +266,7 @@ static GemmArgs gemm_base()
 {
     GemmArgs g;
     std::memset(&g, 0, sizeof g);
-    g.shared_grp = -1;
     return g;
-}
-
-#ifndef MOE_MERGE_SHARED
-#define MOE_MERGE_SHARED 1
-#endif
-
-// Whether the shared expert runs inside the routed grouped GEMMs as one more
-// group (E): same width (d_ff_shared = d_ff), the single-SM kernel for both
-// GEMMs, the fused atomic combine. Its tensor-bound tiles then run among the
-// routed experts' tiles instead of in a stage of their own.
-static bool merge_shared(const moe_shape_t &s)
-{
-    if (!MOE_MERGE_SHARED || s.d_ff_shared <= 0 || s.d_ff_shared != s.d_ff)
-        return false;
-    if (s.flags & (MOE_FLAG_DETERMINISTIC | MOE_FLAG_SIMT_FFN | MOE_FLAG_GEMM_2SM |
-                   MOE_FLAG_MXFP8 | MOE_FLAG_NVFP4))
-        return false;
-    const long long avg = (long long)s.T * s.k / s.E;
-    return !use_pair(s, avg, 2 * s.d_ff, false) && !use_pair(s, avg, s.d, true);
 }
 
 // Routed grouped GEMMs: SwiGLU into H, then w2 with the chosen epilogue.
@@ -296,13 +275,10 @@ static int expert_ffn_core(const moe_shape_t &s, const WsLayout &L, void *ws,
                            const uint16_t *W2, const int32_t *perm_token, const int32_t *slot_pos,
                            const float *topk_w, float *y_perm, float *out, uint32_t *status,
                            cudaStream_t st, long long n_rows = -1, const float *perm_w = nullptr,
-                           bool allow_pair = true, bool test_starve = false,
-                           const uint16_t *x_sh = nullptr, const uint16_t *W13s = nullptr,
-                           const uint16_t *W2s = nullptr)
+                           bool allow_pair = true, bool test_starve = false)
 {
     const long long N = n_rows >= 0 ? n_rows : (long long)s.T * s.k;
     uint16_t *H = at<uint16_t>(ws, L.H);
-    uint16_t *Hs = at<uint16_t>(ws, L.H_shared);
     GemmArgs g = gemm_base();
     g.mode = EPI_SWIGLU;
     g.A = x_perm;
@@ -319,15 +295,6 @@ static int expert_ffn_core(const moe_shape_t &s, const WsLayout &L, void *ws,
     g.ldo = s.d_ff;
     g.status = status;
     g.test_starve = test_starve ? 1 : 0;
-    if (x_sh) {   // the shared expert as group E (merge_shared)
-        g.shared_grp = s.E;
-        g.A2 = x_sh;
-        g.a2_rows = s.T;
-        g.B2 = W13s;
-        g.b2_rows = 2LL * s.d_ff;
-        g.rows_shared = s.T;
-        g.out_s = Hs;
-    }
     int rc;
     {
         StageMark m(MOE_STAGE_W13, st);
@@ -336,11 +303,6 @@ static int expert_ffn_core(const moe_shape_t &s, const WsLayout &L, void *ws,
     if (rc)
         return rc;
     g.test_starve = 0;
-    if (x_sh) {
-        g.A2 = Hs;
-        g.B2 = W2s;
-        g.b2_rows = s.d;
-    }
     g.A = H;
     g.B = W2;
     g.b_rows_total = (long long)s.E * s.d;
@@ -484,8 +446,7 @@ struct HistOut {
 
 static int router_topk_hist(const moe_shape_t &s, const uint16_t *x, const uint16_t *Wg,
                             const float *bias, float *logits, int32_t *idx, float *w,
-                            int32_t *counter, const HistOut &h, uint32_t *status, cudaStream_t st,
-                            int shared_rows = 0)
+                            int32_t *counter, const HistOut &h, uint32_t *status, cudaStream_t st)
 {
     GemmArgs g = gemm_base();
     g.mode = EPI_ROUTER_TOPK;
@@ -519,7 +480,6 @@ static int router_topk_hist(const moe_shape_t &s, const uint16_t *x, const uint1
     g.hist_mt2_group = h.mt2_group;
     g.hist_num_mt2 = h.num_mt2;
     g.capacity = s.capacity;
-    g.hist_shared_rows = shared_rows;
     // the ticket starts at zero whatever an earlier, aborted call left in it
     if (cudaMemsetAsync(counter, 0, sizeof(int32_t), st) != cudaSuccess)
         return MOE_ERR_CUDA;
@@ -573,12 +533,10 @@ static int forward_impl(const moe_shape_t &s, const WsLayout &L, void *ws, const
                           at<int32_t>(ws, L.mt2_row0),     at<int32_t>(ws, L.mt2_group),
                           at<int32_t>(ws, L.num_mt2)};
     const bool hist_fused = !decode && router_hist_fusable(s);
-    const bool merged = !decode && merge_shared(s);
     int rc;
     if (hist_fused) {
         StageMark m(MOE_STAGE_ROUTER, st);
-        rc = router_topk_hist(s, x, Wg, bias, logits, idx, w, counter, hist, status, st,
-                              merged ? s.T : 0);
+        rc = router_topk_hist(s, x, Wg, bias, logits, idx, w, counter, hist, status, st);
     } else {
         rc = route_tokens(s, x, Wg, bias, logits, idx, w, counter, status, st);
     }
@@ -611,15 +569,14 @@ static int forward_impl(const moe_shape_t &s, const WsLayout &L, void *ws, const
                               at<int32_t>(ws, L.n_kept), at<int32_t>(ws, L.mt_row0),
                               at<int32_t>(ws, L.mt_group), at<int32_t>(ws, L.num_mt),
                               at<int32_t>(ws, L.mt2_row0), at<int32_t>(ws, L.mt2_group),
-                              at<int32_t>(ws, L.num_mt2), status, st, nullptr,
-                              merged ? s.T : 0);
+                              at<int32_t>(ws, L.num_mt2), status, st);
     }
     if (rc)
         return rc;
     {
         StageMark m(MOE_STAGE_PERMUTE, st);
         rc = launch_permute(s, idx, chunk, rank, offsets, x, slot_pos, perm_token, x_perm,
-                            ((!shared || merged) && !det) ? out : nullptr, st,
+                            (!shared && !det) ? out : nullptr, st,
                             hist_fused ? kBlockM : kChunkTokens);
     }
     if (rc)
@@ -629,7 +586,7 @@ static int forward_impl(const moe_shape_t &s, const WsLayout &L, void *ws, const
                                     at<int32_t>(ws, L.n_kept), at<int32_t>(ws, L.dbg_seen),
                                     status, st)))
         return rc;
-    if (shared && !merged) {
+    if (shared) {
         StageMark m(MOE_STAGE_SHARED, st);
         rc = shared_expert(s, L, ws, x, W13s, W2s, out, status, st);
         if (rc)
@@ -637,7 +594,7 @@ static int forward_impl(const moe_shape_t &s, const WsLayout &L, void *ws, const
     }
     float *Y = det ? at<float>(ws, L.Y) : nullptr;
     rc = expert_ffn_core(s, L, ws, x_perm, offsets, W13, W2, perm_token, slot_pos, w, Y, out,
-                         status, st, -1, nullptr, true, false, merged ? x : nullptr, W13s, W2s);
+                         status, st);
     if (rc)
         return rc;
     if (det) {

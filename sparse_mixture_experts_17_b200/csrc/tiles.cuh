@@ -81,27 +81,19 @@ __device__ __forceinline__ int spread_merge_pos(int j, int n, int m, bool first)
 // set (block-scaled operands, whose activation scales are keyed by tile
 // index) the list is in plain expert order and tile_start receives each
 // expert's first tile index.
-//
-// shared_rows > 0 (spread order only) adds the shared expert as group E: its
-// ceil(shared_rows / tile_m) tiles (rows 0.. of the token batch) join the
-// several-tile kind after the routed experts, so the one grouped GEMM runs
-// the shared expert's tensor-bound tiles among the routed experts' tiles.
 __device__ inline void build_tiles(const int *s_kept, const int32_t *offsets_smem_or_global, int E,
                                    int tile_m, int32_t *mt_row0, int32_t *mt_group,
-                                   int32_t *num_mt, int *s_warp, int32_t *tile_start = nullptr,
-                                   int shared_rows = 0)
+                                   int32_t *num_mt, int *s_warp, int32_t *tile_start = nullptr)
 {
     const int tid = threadIdx.x;
     const int e = tid;
     const int nt = (e < E) ? (s_kept[e] + tile_m - 1) / tile_m : 0;
     const bool spread = tile_start == nullptr;
     const bool multi = nt >= 2;
-    const int nt_sh = spread ? (shared_rows + tile_m - 1) / tile_m : 0;
     int total, n_multi, n_single;
     const int start = block_excl_scan(nt, s_warp, &total);
     const int start_m = block_excl_scan(spread && multi ? nt : 0, s_warp, &n_multi);
     const int start_s = block_excl_scan(spread && !multi ? nt : 0, s_warp, &n_single);
-    const int n_multi_all = n_multi + nt_sh;
     if (e < E && tile_start)
         tile_start[e] = start;
     if (e < E) {
@@ -111,22 +103,15 @@ __device__ inline void build_tiles(const int *s_kept, const int32_t *offsets_sme
         for (int i = 0; i < nt; ++i) {
             int pos = start + i;
             if (spread)
-                pos = multi ? spread_merge_pos(start_m + i, n_multi_all, n_single, true)
-                            : spread_merge_pos(start_s + i, n_single, n_multi_all, false);
+                pos = multi ? spread_merge_pos(start_m + i, n_multi, n_single, true)
+                            : spread_merge_pos(start_s + i, n_single, n_multi, false);
             mt_row0[pos] = base + i * tile_m;
             const bool half = (tile_m == kBlockM) && (i == nt - 1) && rem <= 64;
             mt_group[pos] = e | (half ? kHalfTileBit : 0);
         }
     }
-    const int rem_sh = shared_rows - (nt_sh - 1) * tile_m;
-    for (int i = tid; i < nt_sh; i += blockDim.x) {
-        const int pos = spread_merge_pos(n_multi + i, n_multi_all, n_single, true);
-        mt_row0[pos] = i * tile_m;
-        const bool half = (tile_m == kBlockM) && (i == nt_sh - 1) && rem_sh <= 64;
-        mt_group[pos] = E | (half ? kHalfTileBit : 0);
-    }
     if (tid == 0)
-        *num_mt = total + nt_sh;
+        *num_mt = total;
 }
 
 // Run by every thread of the last CTA (after a fence that makes the other
@@ -135,14 +120,13 @@ __device__ inline void build_tiles(const int *s_kept, const int32_t *offsets_sme
 // it is replaced by the exclusive prefix in rank order (slots, then chunks).
 // Then counts, capacity, offsets (E + 1), n_kept, the 128-row m-tile list
 // (and the 256-row one when mt2_row0 is set), and the ticket is re-armed.
-// shared_rows > 0 adds the shared expert's tiles to the 128-row list.
 // s_kept, s_off: MOE_MAX_E (+1) ints of shared memory; s_warp: 17 ints.
 __device__ inline void hist_finish(int32_t *chunk_counts, int nchunks, int nj, int E, int C,
                                    int32_t *counts, int32_t *offsets, int32_t *n_kept,
                                    int32_t *mt_row0, int32_t *mt_group, int32_t *num_mt,
                                    int32_t *mt2_row0, int32_t *mt2_group, int32_t *num_mt2,
                                    int32_t *tile_start, int32_t *counter, int *s_kept, int *s_off,
-                                   int *s_warp, int shared_rows = 0)
+                                   int *s_warp)
 {
     const int tid = threadIdx.x;
     const int R = nj * nchunks;   // count rows of one expert, in rank order r = j * nchunks + c
@@ -183,8 +167,7 @@ __device__ inline void hist_finish(int32_t *chunk_counts, int nchunks, int nj, i
         *n_kept = total;
     }
     __syncthreads();
-    build_tiles(s_kept, s_off, E, kBlockM, mt_row0, mt_group, num_mt, s_warp, tile_start,
-                shared_rows);
+    build_tiles(s_kept, s_off, E, kBlockM, mt_row0, mt_group, num_mt, s_warp, tile_start);
     if (mt2_row0)
         build_tiles(s_kept, s_off, E, 2 * kBlockM, mt2_row0, mt2_group, num_mt2, s_warp);
     if (tid == 0)
