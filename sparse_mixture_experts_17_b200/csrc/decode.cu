@@ -346,10 +346,19 @@ __global__ void __launch_bounds__(256, (MAXT <= 2) ? 4 : 2)
 }
 
 // ---------------------------------------------------------------- phase 2: W2 + combine
+// Work item = (output row r, source): one chosen expert's W2_e[r], or the
+// shared expert's row, streamed once by one warp. A CTA takes RG consecutive
+// rows at a time (RG * n_src items, n_src = chosen experts + shared; RG = 8 /
+// n_src, at least 1), its eight warps take the items, and each item leaves its
+// per-token contribution w * (W2_e[r] . h) in shared memory; the CTA then adds
+// the sources of each row in a fixed order (ascending expert, then the shared
+// expert): deterministic. Splitting a row's sources over warps doubles (at
+// top-2) the streams in flight against one warp per row.
 // At MAXT = 1 the weight stream is software-pipelined (two 16-byte loads per
 // lane in flight while two are consumed); at MAXT >= 2 a batch of eight (four
-// above MAXT = 2) loads is issued and then consumed. Both measured best for
-// their token counts on the Mixtral shape.
+// above MAXT = 2) loads is issued and then consumed.
+constexpr int kDecW2MaxItems = MOE_MAX_E + 8;
+
 template <int MAXT>
 __global__ void __launch_bounds__(256, (MAXT <= 2) ? 4 : 2)
     k_dec_w2(const int32_t *__restrict__ idx, const float *__restrict__ topk_w, int T, int d,
@@ -359,107 +368,129 @@ __global__ void __launch_bounds__(256, (MAXT <= 2) ? 4 : 2)
              const uint16_t *__restrict__ Hs, float *__restrict__ out, uint32_t *status)
 {
     __shared__ DecPlanSmem P;
+    __shared__ float contrib[kDecW2MaxItems][MAXT];
     pdl_wait();      // h comes from the w1/w3 kernel
     build_plan(P, idx, T, E, k, C, slot_major, status);
-    const int lane = threadIdx.x & 31;
-    const int nwarps = gridDim.x * (blockDim.x >> 5);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int n_src = P.U + (W2s ? 1 : 0);
-    for (int r = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; r < d; r += nwarps) {
-        float acc[MAXT];
+    if (n_src == 0) {   // every assignment dropped and no shared expert: out = 0
+        for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < (long long)T * d;
+             i += (long long)gridDim.x * blockDim.x)
+            out[i] = 0.f;
+        return;
+    }
+    const int RG = max(1, 8 / n_src);
+    const int items = RG * n_src;   // <= max(8, n_src) <= kDecW2MaxItems
+    for (int r0 = blockIdx.x * RG; r0 < d; r0 += gridDim.x * RG) {
+        for (int it = warp; it < items; it += 8) {
+            const int r = r0 + it / n_src, u = it % n_src;
+            float tok[MAXT];
 #pragma unroll
-        for (int t = 0; t < MAXT; ++t)
-            acc[t] = 0.f;
-        for (int u = 0; u < n_src; ++u) {
-            const bool shared = (u == P.U);
-            const int ff = shared ? d_ff_s : d_ff;
-            const uint4 *wrow = reinterpret_cast<const uint4 *>(
-                shared ? W2s + (size_t)r * d_ff_s : W2 + ((size_t)P.uniq[u] * d + r) * d_ff);
-            const int a0 = shared ? 0 : P.ustart[u];
-            const int na = shared ? T : P.ustart[u + 1] - a0;
-            const uint16_t *hb = shared ? Hs : Hdec;
-            const uint4 *hr[MAXT];
-            int tk[MAXT];
-            float wt[MAXT];
+            for (int t = 0; t < MAXT; ++t)
+                tok[t] = 0.f;
+            if (r < d) {
+                const bool shared = (u == P.U);
+                const int ff = shared ? d_ff_s : d_ff;
+                const uint4 *wrow = reinterpret_cast<const uint4 *>(
+                    shared ? W2s + (size_t)r * d_ff_s : W2 + ((size_t)P.uniq[u] * d + r) * d_ff);
+                const int a0 = shared ? 0 : P.ustart[u];
+                const int na = shared ? T : P.ustart[u + 1] - a0;
+                const uint16_t *hb = shared ? Hs : Hdec;
+                const uint4 *hr[MAXT];
+                int tk[MAXT];
+                float wt[MAXT];
 #pragma unroll
-            for (int s = 0; s < MAXT; ++s) {
-                const int a = (s < na) ? (shared ? s : P.list[a0 + s]) : 0;
-                hr[s] = reinterpret_cast<const uint4 *>(hb + (size_t)a * ff);
-                tk[s] = shared ? s : a / k;
-                wt[s] = (s < na) ? (shared ? 1.f : topk_w[a]) : 0.f;
-            }
-            const int nv = ff / 8;
-            float pa[MAXT];
-#pragma unroll
-            for (int s = 0; s < MAXT; ++s)
-                pa[s] = 0.f;
-            if constexpr (MAXT == 1) {
-                constexpr int UNR = 2;
-                uint4 cur[UNR], nxt[UNR];
-#pragma unroll
-                for (int i = 0; i < UNR; ++i) {
-                    const int ci = lane + 32 * i;
-                    if (ci < nv)
-                        cur[i] = ld_stream_v4(wrow + ci);
+                for (int s = 0; s < MAXT; ++s) {
+                    const int a = (s < na) ? (shared ? s : P.list[a0 + s]) : 0;
+                    hr[s] = reinterpret_cast<const uint4 *>(hb + (size_t)a * ff);
+                    tk[s] = shared ? s : a / k;
+                    wt[s] = (s < na) ? (shared ? 1.f : topk_w[a]) : 0.f;
                 }
-                for (int cb = 0; cb < nv; cb += 32 * UNR) {
-                    const int nb = cb + 32 * UNR;
+                const int nv = ff / 8;
+                float pa[MAXT];
+#pragma unroll
+                for (int s = 0; s < MAXT; ++s)
+                    pa[s] = 0.f;
+                if constexpr (MAXT == 1) {
+                    constexpr int UNR = 2;
+                    uint4 cur[UNR], nxt[UNR];
 #pragma unroll
                     for (int i = 0; i < UNR; ++i) {
-                        const int ci = nb + lane + 32 * i;
+                        const int ci = lane + 32 * i;
                         if (ci < nv)
-                            nxt[i] = ld_stream_v4(wrow + ci);
+                            cur[i] = ld_stream_v4(wrow + ci);
                     }
+                    for (int cb = 0; cb < nv; cb += 32 * UNR) {
+                        const int nb = cb + 32 * UNR;
 #pragma unroll
-                    for (int i = 0; i < UNR; ++i) {
-                        const int ci = cb + lane + 32 * i;
-                        if (ci < nv && na > 0)
-                            pa[0] = dot8(cur[i], __ldg(hr[0] + ci), pa[0]);
+                        for (int i = 0; i < UNR; ++i) {
+                            const int ci = nb + lane + 32 * i;
+                            if (ci < nv)
+                                nxt[i] = ld_stream_v4(wrow + ci);
+                        }
+#pragma unroll
+                        for (int i = 0; i < UNR; ++i) {
+                            const int ci = cb + lane + 32 * i;
+                            if (ci < nv && na > 0)
+                                pa[0] = dot8(cur[i], __ldg(hr[0] + ci), pa[0]);
+                        }
+#pragma unroll
+                        for (int i = 0; i < UNR; ++i)
+                            cur[i] = nxt[i];
                     }
+                } else {
+                    constexpr int UNR = (MAXT <= 2) ? 8 : kDecUnroll;
+                    for (int cb = 0; cb < nv; cb += 32 * UNR) {
+                        uint4 wv[UNR];
 #pragma unroll
-                    for (int i = 0; i < UNR; ++i)
-                        cur[i] = nxt[i];
+                        for (int i = 0; i < UNR; ++i) {
+                            const int ci = cb + lane + 32 * i;
+                            if (ci < nv)
+                                wv[i] = ld_stream_v4(wrow + ci);
+                        }
+#pragma unroll
+                        for (int i = 0; i < UNR; ++i) {
+                            const int ci = cb + lane + 32 * i;
+                            if (ci >= nv)
+                                continue;
+#pragma unroll
+                            for (int s = 0; s < MAXT; ++s)
+                                if (s < na)
+                                    pa[s] = dot8(wv[i], __ldg(hr[s] + ci), pa[s]);
+                        }
+                    }
                 }
-            } else {
-                constexpr int UNR = (MAXT <= 2) ? 8 : kDecUnroll;
-                for (int cb = 0; cb < nv; cb += 32 * UNR) {
-                    uint4 wv[UNR];
+                // this source's weighted contribution to each token of row r
 #pragma unroll
-                    for (int i = 0; i < UNR; ++i) {
-                        const int ci = cb + lane + 32 * i;
-                        if (ci < nv)
-                            wv[i] = ld_stream_v4(wrow + ci);
-                    }
+                for (int s = 0; s < MAXT; ++s) {
+                    if (s < na) {
+                        const float v = wt[s] * warp_sum(pa[s]);
 #pragma unroll
-                    for (int i = 0; i < UNR; ++i) {
-                        const int ci = cb + lane + 32 * i;
-                        if (ci >= nv)
-                            continue;
-#pragma unroll
-                        for (int s = 0; s < MAXT; ++s)
-                            if (s < na)
-                                pa[s] = dot8(wv[i], __ldg(hr[s] + ci), pa[s]);
+                        for (int tt = 0; tt < MAXT; ++tt)
+                            if (tt == tk[s])
+                                tok[tt] += v;
                     }
                 }
             }
-            // fold the lane partials into the tokens' accumulators, weighted
+            if (lane == 0) {
 #pragma unroll
-            for (int s = 0; s < MAXT; ++s) {
-                if (s < na) {
-#pragma unroll
-                    for (int tt = 0; tt < MAXT; ++tt)
-                        if (tt == tk[s])
-                            acc[tt] = fmaf(wt[s], pa[s], acc[tt]);
-                }
+                for (int t = 0; t < MAXT; ++t)
+                    contrib[it][t] = tok[t];
             }
         }
-#pragma unroll
-        for (int t = 0; t < MAXT; ++t) {
-            if (t < T) {
-                const float s = warp_sum(acc[t]);
-                if (lane == 0)
-                    out[(size_t)t * d + r] = s;
+        __syncthreads();
+        // fixed-order sum of each row's sources
+        for (int q = threadIdx.x; q < RG * T; q += blockDim.x) {
+            const int j = q / T, t = q - j * T;
+            const int r = r0 + j;
+            if (r < d) {
+                float v = 0.f;
+                for (int u = 0; u < n_src; ++u)
+                    v += contrib[j * n_src + u][t];
+                out[(size_t)t * d + r] = v;
             }
         }
+        __syncthreads();
     }
 }
 

@@ -120,6 +120,8 @@ __global__ void __launch_bounds__(256) k_topk(const float *__restrict__ logits, 
                                               float *__restrict__ w, int32_t *counter_to_zero,
                                               uint32_t *status)
 {
+    pdl_wait();      // the logits come from the router kernel
+    pdl_trigger();
     if (counter_to_zero && blockIdx.x == 0 && threadIdx.x == 0)
         *counter_to_zero = 0;
     const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -136,24 +138,9 @@ int launch_topk(const moe_shape_t &s, const float *logits, int32_t *idx, float *
         return MOE_OK;
     const int blocks = (s.T + 7) / 8;
     const int vpl = (s.E + 31) / 32;
-#define MOE_TOPK_CASE(V)                                                                         \
-    case V:                                                                                      \
-        k_topk<V><<<blocks, 256, 0, st>>>(logits, s.T, s.E, s.k, idx, w, counter_to_zero,       \
-                                          status);                                               \
-        break;
-    switch (vpl) {
-        MOE_TOPK_CASE(1)
-        MOE_TOPK_CASE(2)
-        MOE_TOPK_CASE(4)
-        MOE_TOPK_CASE(8)
-    case 3:
-        k_topk<4><<<blocks, 256, 0, st>>>(logits, s.T, s.E, s.k, idx, w, counter_to_zero, status);
-        break;
-    default:
-        k_topk<8><<<blocks, 256, 0, st>>>(logits, s.T, s.E, s.k, idx, w, counter_to_zero, status);
-        break;
-    }
-#undef MOE_TOPK_CASE
+    auto kern = vpl <= 1 ? k_topk<1> : vpl <= 2 ? k_topk<2> : vpl <= 4 ? k_topk<4> : k_topk<8>;
+    launch_pdl_ex(kern, dim3(blocks), dim3(256), 0, st, logits, s.T, s.E, s.k, idx, w,
+                  counter_to_zero, status);
     return launched();
 }
 
@@ -176,6 +163,8 @@ __global__ void __launch_bounds__(256) k_hist_scan(
     int32_t *mt_row0, int32_t *mt_group, int32_t *num_mt, int32_t *mt2_row0, int32_t *mt2_group,
     int32_t *num_mt2, int32_t *tile_start, uint32_t *status)
 {
+    pdl_wait();      // the expert ids come from the routing kernels
+    pdl_trigger();
     __shared__ uint32_t mask[8][MOE_MAX_E];
     __shared__ int32_t wpre[8][MOE_MAX_E];
     __shared__ int s_last;
@@ -186,21 +175,31 @@ __global__ void __launch_bounds__(256) k_hist_scan(
     const int t = blockIdx.x * kChunkTokens + tid;
     const bool live = t < T;
 
-    // expert of slot j of this thread's token, -1 if absent, out of range or a
-    // repeat of an earlier slot (those two are flagged)
+    // the token's expert ids, read once; an id out of range or repeating an
+    // earlier slot becomes -1 (and is flagged)
+    int ids[MOE_MAX_K];
     bool flagged = false;
-    auto slot_expert = [&](int j) {
-        int e = live ? idx[(size_t)t * k + j] : -1;
-        if (live && (e < 0 || e >= E)) {
+#pragma unroll
+    for (int j = 0; j < MOE_MAX_K; ++j) {
+        int e = (live && j < k) ? idx[(size_t)t * k + j] : -1;
+        if (live && j < k && (e < 0 || e >= E)) {
             flagged = true;
-            return -1;
+            e = -1;
         }
-        if (e >= 0)
-            for (int jj = 0; jj < j; ++jj)
-                if (idx[(size_t)t * k + jj] == e) {
-                    flagged = true;
-                    return -1;
-                }
+#pragma unroll
+        for (int jj = 0; jj < j; ++jj)
+            if (e >= 0 && ids[jj] == e) {
+                flagged = true;
+                e = -1;
+            }
+        ids[j] = e;
+    }
+    auto slot_expert = [&](int j) {
+        int e = -1;
+#pragma unroll
+        for (int jj = 0; jj < MOE_MAX_K; ++jj)
+            if (jj == j)
+                e = ids[jj];
         return e;
     };
     // one group of slots [j0, j1): per-warp lane masks, then per-expert warp
@@ -229,16 +228,9 @@ __global__ void __launch_bounds__(256) k_hist_scan(
         __syncthreads();
         if (live) {
             for (int j = j0; j < j1; ++j) {
-                const int e = idx[(size_t)t * k + j];
-                int r = -1;
-                if (e >= 0 && e < E) {
-                    bool dup = false;
-                    for (int jj = 0; jj < j; ++jj)
-                        dup |= (idx[(size_t)t * k + jj] == e);
-                    if (!dup)
-                        r = wpre[warp][e] + __popc(mask[warp][e] & lanemask_lt());
-                }
-                rank_local[(size_t)t * k + j] = r;
+                const int e = slot_expert(j);
+                rank_local[(size_t)t * k + j] =
+                    e >= 0 ? wpre[warp][e] + __popc(mask[warp][e] & lanemask_lt()) : -1;
             }
         }
         __syncthreads();
@@ -276,10 +268,9 @@ int launch_hist_scan(const moe_shape_t &s, const int32_t *idx, int32_t *chunk_co
     const int nchunks = (s.T + kChunkTokens - 1) / kChunkTokens;
     if (nchunks == 0)
         return MOE_OK;
-    k_hist_scan<<<nchunks, 256, 0, st>>>(idx, s.T, s.E, s.k, s.capacity, slot_major(s),
-                                         chunk_counts, rank_local, counter, counts, offsets,
-                                         n_kept, mt_row0, mt_group, num_mt, mt2_row0, mt2_group,
-                                         num_mt2, tile_start, status);
+    launch_pdl_ex(k_hist_scan, dim3(nchunks), dim3(256), 0, st, idx, s.T, s.E, s.k, s.capacity,
+                  slot_major(s), chunk_counts, rank_local, counter, counts, offsets, n_kept,
+                  mt_row0, mt_group, num_mt, mt2_row0, mt2_group, num_mt2, tile_start, status);
     return launched();
 }
 
@@ -296,6 +287,8 @@ __global__ void __launch_bounds__(256) k_permute(
     const int32_t *__restrict__ offsets, const uint4 *__restrict__ x, int32_t *__restrict__ slot_pos,
     int32_t *__restrict__ perm_token, uint4 *__restrict__ x_perm, float4 *__restrict__ out_zero)
 {
+    pdl_wait();      // offsets, chunk bases and ranks come from the histogram
+    pdl_trigger();
     const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
     if (t >= T)
@@ -359,11 +352,10 @@ int launch_permute(const moe_shape_t &s, const int32_t *idx, const int32_t *chun
 {
     if (s.T == 0)
         return MOE_OK;
-    k_permute<<<(s.T + 7) / 8, 256, 0, st>>>(
-        idx, s.T, s.E, s.k, s.capacity, slot_major(s), s.d, chunk_tokens, chunk_base, rank_local,
-        offsets,
-        reinterpret_cast<const uint4 *>(x), slot_pos, perm_token, reinterpret_cast<uint4 *>(x_perm),
-        reinterpret_cast<float4 *>(out_zero));
+    launch_pdl_ex(k_permute, dim3((s.T + 7) / 8), dim3(256), 0, st, idx, s.T, s.E, s.k, s.capacity,
+                  slot_major(s), s.d, chunk_tokens, chunk_base, rank_local, offsets,
+                  reinterpret_cast<const uint4 *>(x), slot_pos, perm_token,
+                  reinterpret_cast<uint4 *>(x_perm), reinterpret_cast<float4 *>(out_zero));
     return launched();
 }
 

@@ -396,7 +396,7 @@ __device__ __forceinline__ void epilogue_tile(const TcArgs &p, uint32_t tb, long
 template <int BN, int MODE>
 __global__ void __launch_bounds__(192, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-              const TcArgs p)
+              const __grid_constant__ CUtensorMap tmA64, const TcArgs p)
 {
     using C = TcCfg<BN>;
     extern __shared__ uint8_t smem_raw[];
@@ -427,10 +427,8 @@ __global__ void __launch_bounds__(192, 1)
     if (warp == 0 && lane == 0) {
         tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmB);
-        // the fused router also re-arms the histogram kernel's ticket (which
-        // runs after this kernel in stream order)
-        if (MODE == EPI_ROUTER_TOPK && blockIdx.x == 0 && p.counter_zero)
-            *p.counter_zero = 0;
+        tma_prefetch_desc(&tmA64);
+
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, C::TMEM_COLS);
@@ -440,6 +438,15 @@ __global__ void __launch_bounds__(192, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    // launched with programmatic stream serialization: the setup above overlaps
+    // the predecessor's tail; nothing the predecessor writes is read before this
+    pdl_wait();
+    pdl_trigger();
+
+    // the fused router also re-arms the histogram kernel's ticket (which runs
+    // after this kernel in stream order)
+    if (MODE == EPI_ROUTER_TOPK && blockIdx.x == 0 && threadIdx.x == 0 && p.counter_zero)
+        *p.counter_zero = 0;
 
     const int num_mt = p.num_mt_dev ? *p.num_mt_dev : p.num_mt_host;
     const long long total = (long long)num_mt * p.n_tiles;
@@ -453,6 +460,12 @@ __global__ void __launch_bounds__(192, 1)
                 const int row0 = p.mt_row0 ? p.mt_row0[m_idx] : m_idx * C::BM;
                 const int grp = p.mt_group ? (p.mt_group[m_idx] & ~kHalfTileBit) : 0;
                 const int brow = grp * p.b_rows_per_group + n_idx * BN;
+                // a tile of <= 64 rows runs M = 64 MMAs, which read A's first 64
+                // rows only: it loads those (a 64-row box), not 128
+                const bool half = p.mt_group && (p.mt_group[m_idx] & kHalfTileBit);
+                const void *ta = half ? static_cast<const void *>(&tmA64)
+                                      : static_cast<const void *>(&tmA);
+                const uint32_t stage_bytes = half ? C::STAGE_BYTES - C::A_BYTES / 2 : C::STAGE_BYTES;
                 // K-grouped GEMMs contract over their group's own k-block range
                 const int kb0 = p.grp_kb0 ? p.grp_kb0[grp] : 0;
                 const int nkb = p.grp_kb0 ? p.grp_nkb[grp] : p.kblocks;
@@ -464,8 +477,8 @@ __global__ void __launch_bounds__(192, 1)
                         ok = false;
                         break;
                     }
-                    mbar_arrive_expect_tx(&full[s], C::STAGE_BYTES);
-                    tma_load_2d(sA + s * C::A_BYTES, &tmA, (kb0 + kb) * C::BK, row0, &full[s]);
+                    mbar_arrive_expect_tx(&full[s], stage_bytes);
+                    tma_load_2d(sA + s * C::A_BYTES, ta, (kb0 + kb) * C::BK, row0, &full[s]);
                     tma_load_2d(sB + s * C::B_BYTES, &tmB, (kb0 + kb) * C::BK, brow, &full[s]);
                 }
                 if (!ok)
@@ -792,8 +805,11 @@ static int launch_tc_impl(const GemmArgs &g, cudaStream_t st)
 {
     using C = TcCfg<BN>;
     CUtensorMap tA, tB;
+    CUtensorMap tA64;
     int rc = make_tmap(&tA, g.A, g.K, g.a_rows, 128);
     if (rc)
+        return rc;
+    if ((rc = make_tmap(&tA64, g.A, g.K, g.a_rows, 64)))
         return rc;
     rc = make_tmap(&tB, g.B, g.K, g.b_rows_total, BN);
     if (rc)
@@ -864,7 +880,7 @@ static int launch_tc_impl(const GemmArgs &g, cudaStream_t st)
     if (tiles <= 0)
         return MOE_OK;
     const int grid = (int)std::min<long long>(tiles, num_sms());
-    k_gemm_tc<BN, MODE><<<grid, 192, SMEM, st>>>(tA, tB, p);
+    launch_pdl_ex(k_gemm_tc<BN, MODE>, dim3(grid), dim3(192), SMEM, st, tA, tB, tA64, p);
     return launched();
 }
 

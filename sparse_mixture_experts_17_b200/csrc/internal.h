@@ -19,6 +19,27 @@ inline int launched()
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
+// Launch with programmatic stream serialization: the kernel may start while
+// its predecessor in the stream is still running, so it must execute
+// griddepcontrol.wait (pdl_wait) before it reads anything a predecessor
+// writes. Returns the launch's error code.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl_ex(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                                 cudaStream_t st, Args... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 constexpr int kBlockM = 128;      // rows of one grouped-GEMM m-tile
 // Bit of an m-tile's group entry marking a tail tile of at most 64 rows: the
 // single-SM tensor-core GEMM runs it with M = 64 MMAs (half the tensor time).

@@ -130,30 +130,70 @@ __device__ inline void hist_finish(int32_t *chunk_counts, int nchunks, int nj, i
 {
     const int tid = threadIdx.x;
     const int R = nj * nchunks;   // count rows of one expert, in rank order r = j * nchunks + c
-    constexpr int U = 16;         // loads in flight per thread
-    for (int e = tid; e < MOE_MAX_E; e += blockDim.x) {
-        int kept = 0;
-        if (e < E) {
-            int run = 0;
-            for (int r0 = 0; r0 < R; r0 += U) {
-                int v[U];
+    auto row_at = [&](int r, int e) -> size_t {
+        const int j = r / nchunks, c = r - j * nchunks;
+        return ((size_t)c * nj + j) * E + e;
+    };
+    const int nwarps = blockDim.x >> 5;
+    if (E * 4 <= nwarps * 32 && R >= 64) {
+        // few experts, many rows: a warp per expert, each lane a contiguous
+        // range of rows (loads in flight together), then a warp scan of the
+        // lane totals
+        const int lane = tid & 31, warp = tid >> 5;
+        const int per = (R + 31) / 32;
+        for (int e = warp; e < MOE_MAX_E; e += nwarps) {
+            int kept = 0;
+            if (e < E) {
+                const int r0 = lane * per, r1 = min(R, r0 + per);
+                int sum = 0;
+                for (int r = r0; r < r1; ++r)
+                    sum += __ldcg(&chunk_counts[row_at(r, e)]);
+                int inc = sum;
 #pragma unroll
-                for (int u = 0; u < U; ++u) {
-                    const int r = r0 + u, j = r / nchunks, c = r - j * nchunks;
-                    v[u] = r < R ? __ldcg(&chunk_counts[((size_t)c * nj + j) * E + e]) : 0;
+                for (int off = 1; off < 32; off <<= 1) {
+                    const int o = __shfl_up_sync(kFullMask, inc, off);
+                    if (lane >= off)
+                        inc += o;
                 }
-#pragma unroll
-                for (int u = 0; u < U; ++u) {
-                    const int r = r0 + u, j = r / nchunks, c = r - j * nchunks;
-                    if (r < R)
-                        __stcg(&chunk_counts[((size_t)c * nj + j) * E + e], run);
-                    run += v[u];
+                int run = inc - sum;
+                for (int r = r0; r < r1; ++r) {
+                    const size_t i = row_at(r, e);
+                    const int v = __ldcg(&chunk_counts[i]);
+                    __stcg(&chunk_counts[i], run);
+                    run += v;
                 }
+                const int total = __shfl_sync(kFullMask, inc, 31);
+                if (lane == 0)
+                    counts[e] = total;
+                kept = (C > 0 && total > C) ? C : total;
             }
-            counts[e] = run;
-            kept = (C > 0 && run > C) ? C : run;
+            if (lane == 0)
+                s_kept[e] = kept;
         }
-        s_kept[e] = kept;
+    } else {
+        // many experts: a thread per expert, 16 loads in flight
+        constexpr int U = 16;
+        for (int e = tid; e < MOE_MAX_E; e += blockDim.x) {
+            int kept = 0;
+            if (e < E) {
+                int run = 0;
+                for (int r0 = 0; r0 < R; r0 += U) {
+                    int v[U];
+#pragma unroll
+                    for (int u = 0; u < U; ++u)
+                        v[u] = (r0 + u) < R ? __ldcg(&chunk_counts[row_at(r0 + u, e)]) : 0;
+#pragma unroll
+                    for (int u = 0; u < U; ++u) {
+                        if (r0 + u < R)
+                            __stcg(&chunk_counts[row_at(r0 + u, e)], run);
+                        run += v[u];
+                    }
+                }
+                counts[e] = run;
+                kept = (C > 0 && run > C) ? C : run;
+            }
+            s_kept[e] = kept;
+        }
     }
     __syncthreads();
     int total;
