@@ -171,9 +171,15 @@ __device__ __forceinline__ void tile_coords(long long tile, int num_mt, int n_ti
 // Epilogue of one accumulator tile for this thread's row (TMEM lane): `tb`
 // addresses the row's BN fp32 columns. tcgen05.ld is warp-collective, so all
 // lanes run it; only rows inside the expert's segment (`valid`) are written.
+// Per-warp staging of the combine epilogue: 32 rows x 32 floats, rows padded
+// to 36 floats (144 bytes: 16-byte aligned rows).
+constexpr int kXposeStride = 36;
+constexpr int kXposeBytes = 4 * 32 * kXposeStride * 4;   // the four epilogue warps
+
 template <int BN, int MODE>
 __device__ __forceinline__ void epilogue_tile(const TcArgs &p, uint32_t tb, long long row,
-                                              bool valid, int n_idx, int grp, bool empty_k)
+                                              bool valid, int n_idx, int grp, bool empty_k,
+                                              float *xpose = nullptr)
 {
     if (MODE == EPI_SWIGLU_SAVE) {
         // as EPI_SWIGLU, and the raw accumulators (gate | up of this 128-column
@@ -292,18 +298,50 @@ __device__ __forceinline__ void epilogue_tile(const TcArgs &p, uint32_t tb, long
                         wgt = p.topk_w[(long long)t * p.k + j];
             }
         }
-        float *o = static_cast<float *>(p.out) + (long long)t * p.ldo + n_idx * BN;
+        if (xpose) {
+            // lanes hold rows, so each thread's 16-byte atomics would go to 32
+            // different rows at once; staging 32 x 32 floats per warp in shared
+            // memory lets eight lanes cover one row's 128 contiguous bytes, a
+            // quarter of the L2 atomic requests per warp instruction
+            const int lane = threadIdx.x & 31;
+            float4 *mine = reinterpret_cast<float4 *>(xpose + lane * kXposeStride);
+            float *obase = static_cast<float *>(p.out) + n_idx * BN;
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
-            float v[32];
-            tmem_ld32(tb + c * 32, v);
-            tmem_ld_wait();
-            if (valid) {
-                float4 *dst = reinterpret_cast<float4 *>(o + c * 32);
+            for (int c = 0; c < BN / 32; ++c) {
+                float v[32];
+                tmem_ld32(tb + c * 32, v);
+                tmem_ld_wait();
 #pragma unroll
                 for (int i = 0; i < 8; ++i)
-                    atomicAdd(dst + i, make_float4(wgt * v[4 * i], wgt * v[4 * i + 1],
-                                                   wgt * v[4 * i + 2], wgt * v[4 * i + 3]));
+                    mine[i] = make_float4(wgt * v[4 * i], wgt * v[4 * i + 1], wgt * v[4 * i + 2],
+                                          wgt * v[4 * i + 3]);
+                __syncwarp();
+#pragma unroll
+                for (int pass = 0; pass < 8; ++pass) {
+                    const int r = 4 * pass + (lane >> 3), seg = lane & 7;
+                    const int tr = __shfl_sync(kFullMask, t, r);
+                    const int vr = __shfl_sync(kFullMask, valid ? 1 : 0, r);
+                    const float4 val = reinterpret_cast<const float4 *>(xpose + r * kXposeStride)[seg];
+                    if (vr)
+                        atomicAdd(reinterpret_cast<float4 *>(obase + (long long)tr * p.ldo + c * 32) + seg,
+                                  val);
+                }
+                __syncwarp();
+            }
+        } else {
+            float *o = static_cast<float *>(p.out) + (long long)t * p.ldo + n_idx * BN;
+#pragma unroll 1
+            for (int c = 0; c < BN / 32; ++c) {
+                float v[32];
+                tmem_ld32(tb + c * 32, v);
+                tmem_ld_wait();
+                if (valid) {
+                    float4 *dst = reinterpret_cast<float4 *>(o + c * 32);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        atomicAdd(dst + i, make_float4(wgt * v[4 * i], wgt * v[4 * i + 1],
+                                                       wgt * v[4 * i + 2], wgt * v[4 * i + 3]));
+                }
             }
         }
     } else if (MODE == EPI_STORE_F32) {
@@ -550,7 +588,12 @@ __global__ void __launch_bounds__(192, 1)
             const bool empty_k = p.grp_kb0 && p.grp_nkb[grp] == 0;
 
             if (got)
-                epilogue_tile<BN, MODE>(p, tb, row, valid, n_idx, grp, empty_k);
+                epilogue_tile<BN, MODE>(
+                    p, tb, row, valid, n_idx, grp, empty_k,
+                    MODE == EPI_COMBINE
+                        ? reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(full) + C::BAR_BYTES) +
+                              q * 32 * kXposeStride
+                        : nullptr);
             if constexpr (MODE == EPI_ROUTER_TOPK) {
                 if (p.hist_chunk)
                     router_hist_tile(p, *reinterpret_cast<RouterHistSmem *>(
@@ -865,7 +908,9 @@ static int launch_tc_impl(const GemmArgs &g, cudaStream_t st)
     p.wait_ns = g.test_starve ? kTestWaitLimitNs : kWaitLimitNs;
 
     // the router with the folded histogram also needs its tile-histogram area
-    constexpr int SMEM = C::SMEM_BYTES + (MODE == EPI_ROUTER_TOPK ? (int)sizeof(RouterHistSmem) : 0);
+    constexpr int SMEM = C::SMEM_BYTES + (MODE == EPI_ROUTER_TOPK ? (int)sizeof(RouterHistSmem) : 0) +
+                         (MODE == EPI_COMBINE ? kXposeBytes : 0);
+    static_assert(SMEM <= 232448, "shared memory per CTA");
     static int attr_done[64] = {0};
     int dev = 0;
     cudaGetDevice(&dev);
