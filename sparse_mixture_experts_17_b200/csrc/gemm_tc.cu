@@ -344,6 +344,36 @@ __device__ __forceinline__ void epilogue_tile(const TcArgs &p, uint32_t tb, long
                 }
             }
         }
+    } else if (MODE == EPI_STORE_F32 && xpose && (p.ldo & 3) == 0) {
+        // rows through shared memory: eight lanes store one row's 128 bytes
+        const int lane = threadIdx.x & 31;
+        float4 *mine = reinterpret_cast<float4 *>(xpose + lane * kXposeStride);
+        float *obase = static_cast<float *>(p.out) + (long long)grp * p.out_group_stride + n_idx * BN;
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+            float v[32];
+            tmem_ld32(tb + c * 32, v);
+            tmem_ld_wait();
+            if (empty_k) {   // a group with no k-blocks: its output block is zero
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    v[i] = 0.f;
+            }
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                mine[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+            __syncwarp();
+#pragma unroll
+            for (int pass = 0; pass < 8; ++pass) {
+                const int r = 4 * pass + (lane >> 3), seg = lane & 7;
+                const long long rr = __shfl_sync(kFullMask, row, r);
+                const int vr = __shfl_sync(kFullMask, valid ? 1 : 0, r);
+                if (vr)
+                    reinterpret_cast<float4 *>(obase + rr * p.ldo + c * 32)[seg] =
+                        reinterpret_cast<const float4 *>(xpose + r * kXposeStride)[seg];
+            }
+            __syncwarp();
+        }
     } else if (MODE == EPI_STORE_F32) {
         float *o = static_cast<float *>(p.out) + (long long)grp * p.out_group_stride +
                    row * p.ldo + n_idx * BN;
@@ -411,6 +441,40 @@ __device__ __forceinline__ void epilogue_tile(const TcArgs &p, uint32_t tb, long
                 p.route_idx[row * p.k + j] = sel[j];
                 p.route_w[row * p.k + j] = ex[j] / sum;
             }
+        }
+    } else if (xpose && (p.n_valid & 3) == 0 && (p.ldo & 3) == 0) {   // EPI_ROUTER, staged
+        // as the combine epilogue: rows through shared memory so that eight
+        // lanes write one row's 128 contiguous bytes
+        const int lane = threadIdx.x & 31;
+        float4 *mine = reinterpret_cast<float4 *>(xpose + lane * kXposeStride);
+        const long long row_base = row - lane;   // this warp's first row (M = 128 tiles)
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+            float v[32];
+            tmem_ld32(tb + c * 32, v);
+            tmem_ld_wait();
+            const int n0 = n_idx * BN + c * 32;
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                mine[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+            __syncwarp();
+#pragma unroll
+            for (int pass = 0; pass < 8; ++pass) {
+                const int r = 4 * pass + (lane >> 3), seg = lane & 7;
+                const int vr = __shfl_sync(kFullMask, valid ? 1 : 0, r);
+                const int n = n0 + seg * 4;
+                if (vr && n < p.n_valid) {
+                    float4 val = reinterpret_cast<const float4 *>(xpose + r * kXposeStride)[seg];
+                    if (p.bias) {
+                        val.x += p.bias[n];
+                        val.y += p.bias[n + 1];
+                        val.z += p.bias[n + 2];
+                        val.w += p.bias[n + 3];
+                    }
+                    *reinterpret_cast<float4 *>(static_cast<float *>(p.out) + (row_base + r) * p.ldo + n) = val;
+                }
+            }
+            __syncwarp();
         }
     } else {   // EPI_ROUTER
         float *o = static_cast<float *>(p.out) + row * p.ldo;
@@ -590,7 +654,7 @@ __global__ void __launch_bounds__(192, 1)
             if (got)
                 epilogue_tile<BN, MODE>(
                     p, tb, row, valid, n_idx, grp, empty_k,
-                    MODE == EPI_COMBINE
+                    (MODE == EPI_COMBINE || MODE == EPI_STORE_F32 || (MODE == EPI_ROUTER && !half))
                         ? reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(full) + C::BAR_BYTES) +
                               q * 32 * kXposeStride
                         : nullptr);
@@ -650,7 +714,8 @@ struct TcPairCfg {
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
     static constexpr int STAGES = 6;
     static constexpr int TMEM_COLS = 512;   // two 256-column accumulators
-    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 256;
+    static constexpr int BAR_BYTES = 256;
+    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES + kXposeBytes;
 };
 
 template <int MODE>
@@ -779,7 +844,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
             const long long row = row0 + q * 32 + lane;
             const bool valid = row < row_end;
             const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + b * BN;
-            epilogue_tile<BN, MODE>(p, tb, row, valid, n_idx, grp, false);
+            epilogue_tile<BN, MODE>(p, tb, row, valid, n_idx, grp, false,
+                                    reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(full) +
+                                                              C::BAR_BYTES) +
+                                        q * 32 * kXposeStride);
             tc_fence_before();
             __syncwarp();
             if (lane == 0)
@@ -909,7 +977,9 @@ static int launch_tc_impl(const GemmArgs &g, cudaStream_t st)
 
     // the router with the folded histogram also needs its tile-histogram area
     constexpr int SMEM = C::SMEM_BYTES + (MODE == EPI_ROUTER_TOPK ? (int)sizeof(RouterHistSmem) : 0) +
-                         (MODE == EPI_COMBINE ? kXposeBytes : 0);
+                         ((MODE == EPI_COMBINE || MODE == EPI_ROUTER || MODE == EPI_STORE_F32)
+                              ? kXposeBytes
+                              : 0);
     static_assert(SMEM <= 232448, "shared memory per CTA");
     static int attr_done[64] = {0};
     int dev = 0;

@@ -139,33 +139,43 @@ __device__ inline void hist_finish(int32_t *chunk_counts, int nchunks, int nj, i
         // few experts, many rows: a warp per expert, each lane a contiguous
         // range of rows (loads in flight together), then a warp scan of the
         // lane totals
+        // A lane holds up to 8 consecutive rows in registers (all loads in
+        // flight together); longer lists take rounds of 256 rows.
         const int lane = tid & 31, warp = tid >> 5;
-        const int per = (R + 31) / 32;
+        constexpr int V = 8;
         for (int e = warp; e < MOE_MAX_E; e += nwarps) {
             int kept = 0;
             if (e < E) {
-                const int r0 = lane * per, r1 = min(R, r0 + per);
-                int sum = 0;
-                for (int r = r0; r < r1; ++r)
-                    sum += __ldcg(&chunk_counts[row_at(r, e)]);
-                int inc = sum;
+                int carry = 0;
+                for (int base = 0; base < R; base += 32 * V) {
+                    const int r0 = base + lane * V;
+                    int v[V];
 #pragma unroll
-                for (int off = 1; off < 32; off <<= 1) {
-                    const int o = __shfl_up_sync(kFullMask, inc, off);
-                    if (lane >= off)
-                        inc += o;
+                    for (int u = 0; u < V; ++u)
+                        v[u] = (r0 + u < R) ? __ldcg(&chunk_counts[row_at(r0 + u, e)]) : 0;
+                    int sum = 0;
+#pragma unroll
+                    for (int u = 0; u < V; ++u)
+                        sum += v[u];
+                    int inc = sum;
+#pragma unroll
+                    for (int off = 1; off < 32; off <<= 1) {
+                        const int o = __shfl_up_sync(kFullMask, inc, off);
+                        if (lane >= off)
+                            inc += o;
+                    }
+                    int run = carry + inc - sum;
+#pragma unroll
+                    for (int u = 0; u < V; ++u) {
+                        if (r0 + u < R)
+                            __stcg(&chunk_counts[row_at(r0 + u, e)], run);
+                        run += v[u];
+                    }
+                    carry += __shfl_sync(kFullMask, inc, 31);
                 }
-                int run = inc - sum;
-                for (int r = r0; r < r1; ++r) {
-                    const size_t i = row_at(r, e);
-                    const int v = __ldcg(&chunk_counts[i]);
-                    __stcg(&chunk_counts[i], run);
-                    run += v;
-                }
-                const int total = __shfl_sync(kFullMask, inc, 31);
                 if (lane == 0)
-                    counts[e] = total;
-                kept = (C > 0 && total > C) ? C : total;
+                    counts[e] = carry;
+                kept = (C > 0 && carry > C) ? C : carry;
             }
             if (lane == 0)
                 s_kept[e] = kept;
