@@ -174,7 +174,10 @@ TRAFFIC_SOURCES = ["sparse_mixture_experts_17_b200/csrc/gemm_tc.cu",
                    "sparse_mixture_experts_17_b200/csrc/common.cuh",
                    "sparse_mixture_experts_17_b200/csrc/tiles.cuh",
                    "sparse_mixture_experts_17_b200/csrc/moe_api.cu"]
-TRAFFIC = {}
+TRAFFIC = {
+    "prefill": {"bytes": 2187448064 + 929578240, "sources_sha": "8b3a5bc27187645e",
+                "profile": "profiles/gemm_w13_traffic_mixtral_t16384.md"},
+}
 
 
 def sources_sha() -> str:
@@ -402,6 +405,9 @@ def run_ours(a, world, rank, local):
     value = tokens_all / (step_ms_max / 1e3)
 
     flops, w13_flops, w2_flops = prefill_flops(w, n_kept)
+    # bytes the w1/w3 launch must move: every expert's W13 (all hold rows at
+    # this size), the permuted activations read once, H written once
+    w13_alg_bytes = int(w.E * 2 * w.d_ff * w.d * 2 + n_kept * w.d * 2 + n_kept * w.d_ff * 2)
     # MXFP8: the fp8 dense peak, twice the measured sustained bf16 figure (the
     # nominal fp8:bf16 ratio; no fp8 peak is measured on this machine)
     ratio = 2.0 if a.mxfp8 else 4.0 if a.nvfp4 else 1.0   # NVFP4: the fp4:bf16 nominal ratio
@@ -431,6 +437,7 @@ def run_ours(a, world, rank, local):
                         "kernel": "k_gemm_tc<256,EPI_SWIGLU> (grouped w1/w3 GEMM + SwiGLU)",
                         "achieved": round(ach, 1), "peak": peak_t, "unit": "TFLOP/s",
                         "frac": round(ach / peak_t, 4), "traffic": headline_traffic(w),
+                        "algorithmic_bytes_per_launch": w13_alg_bytes,
                         "peak_source": f"{peak_src} bf16_tflops (burst)",
                         "frac_of_sustained": round(ach / peaks["bf16_tflops_sustained"], 4),
                         "frac_of_nominal_2250": round(ach / 2250.0, 4),

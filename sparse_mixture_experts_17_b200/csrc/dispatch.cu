@@ -161,7 +161,7 @@ __global__ void __launch_bounds__(256) k_hist_scan(
     int32_t *chunk_counts, int32_t *__restrict__ rank_local, int32_t *counter,
     int32_t *__restrict__ counts, int32_t *__restrict__ offsets, int32_t *__restrict__ n_kept,
     int32_t *mt_row0, int32_t *mt_group, int32_t *num_mt, int32_t *mt2_row0, int32_t *mt2_group,
-    int32_t *num_mt2, int32_t *tile_start, uint32_t *status)
+    int32_t *num_mt2, int32_t *tile_start, int32_t *mt_first, int32_t *mt2_first, uint32_t *status)
 {
     pdl_wait();      // the expert ids come from the routing kernels
     pdl_trigger();
@@ -256,21 +256,22 @@ __global__ void __launch_bounds__(256) k_hist_scan(
     __threadfence();
     hist_finish(chunk_counts, gridDim.x, slot_major ? k : 1, E, C, counts, offsets, n_kept,
                 mt_row0, mt_group, num_mt, mt2_row0, mt2_group, num_mt2, tile_start, counter,
-                s_kept, s_off, s_warp);
+                s_kept, s_off, s_warp, mt_first, mt2_first);
 }
 
 int launch_hist_scan(const moe_shape_t &s, const int32_t *idx, int32_t *chunk_counts,
                      int32_t *rank_local, int32_t *counter, int32_t *counts, int32_t *offsets,
                      int32_t *n_kept, int32_t *mt_row0, int32_t *mt_group, int32_t *num_mt,
                      int32_t *mt2_row0, int32_t *mt2_group, int32_t *num_mt2, uint32_t *status,
-                     cudaStream_t st, int32_t *tile_start)
+                     cudaStream_t st, int32_t *tile_start, int32_t *mt_first, int32_t *mt2_first)
 {
     const int nchunks = (s.T + kChunkTokens - 1) / kChunkTokens;
     if (nchunks == 0)
         return MOE_OK;
     launch_pdl_ex(k_hist_scan, dim3(nchunks), dim3(256), 0, st, idx, s.T, s.E, s.k, s.capacity,
                   slot_major(s), chunk_counts, rank_local, counter, counts, offsets, n_kept,
-                  mt_row0, mt_group, num_mt, mt2_row0, mt2_group, num_mt2, tile_start, status);
+                  mt_row0, mt_group, num_mt, mt2_row0, mt2_group, num_mt2, tile_start, mt_first,
+                  mt2_first, status);
     return launched();
 }
 
@@ -364,7 +365,8 @@ __global__ void __launch_bounds__(256) k_tiles_from_offsets(const int32_t *__res
                                                             int E, int32_t *mt_row0,
                                                             int32_t *mt_group, int32_t *num_mt,
                                                             int32_t *mt2_row0, int32_t *mt2_group,
-                                                            int32_t *num_mt2)
+                                                            int32_t *num_mt2, int32_t *mt_first,
+                                                            int32_t *mt2_first)
 {
     __shared__ int s_kept[MOE_MAX_E];
     __shared__ int s_off[MOE_MAX_E];
@@ -373,17 +375,19 @@ __global__ void __launch_bounds__(256) k_tiles_from_offsets(const int32_t *__res
     s_kept[e] = (e < E) ? max(0, offsets[e + 1] - offsets[e]) : 0;
     s_off[e] = (e < E) ? offsets[e] : 0;
     __syncthreads();
-    build_tiles(s_kept, s_off, E, kBlockM, mt_row0, mt_group, num_mt, s_warp);
+    build_tiles(s_kept, s_off, E, kBlockM, mt_row0, mt_group, num_mt, s_warp, nullptr, mt_first);
     if (mt2_row0)
-        build_tiles(s_kept, s_off, E, 2 * kBlockM, mt2_row0, mt2_group, num_mt2, s_warp);
+        build_tiles(s_kept, s_off, E, 2 * kBlockM, mt2_row0, mt2_group, num_mt2, s_warp, nullptr,
+                    mt2_first);
 }
 
 int launch_tiles_from_offsets(const moe_shape_t &s, const int32_t *offsets, int32_t *mt_row0,
                               int32_t *mt_group, int32_t *num_mt, int32_t *mt2_row0,
-                              int32_t *mt2_group, int32_t *num_mt2, cudaStream_t st)
+                              int32_t *mt2_group, int32_t *num_mt2, cudaStream_t st,
+                              int32_t *mt_first, int32_t *mt2_first)
 {
     k_tiles_from_offsets<<<1, 256, 0, st>>>(offsets, s.E, mt_row0, mt_group, num_mt, mt2_row0,
-                                            mt2_group, num_mt2);
+                                            mt2_group, num_mt2, mt_first, mt2_first);
     return launched();
 }
 

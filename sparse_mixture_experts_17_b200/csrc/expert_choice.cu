@@ -75,7 +75,8 @@ constexpr int kEcThreads = 1024;
 __global__ void __launch_bounds__(kEcThreads) k_ec_select(
     const float *__restrict__ scores, int T, int E, int K, int32_t *__restrict__ tokens,
     float *__restrict__ weights, int32_t *__restrict__ offsets, int32_t *__restrict__ mt_row0,
-    int32_t *__restrict__ mt_group, int32_t *__restrict__ num_mt, uint32_t *status)
+    int32_t *__restrict__ mt_group, int32_t *__restrict__ num_mt, int32_t *__restrict__ mt_first,
+    uint32_t *status)
 {
     __shared__ int hist[256];
     __shared__ uint32_t s_prefix;
@@ -168,9 +169,11 @@ __global__ void __launch_bounds__(kEcThreads) k_ec_select(
     const int nt = (K + kBlockM - 1) / kBlockM;
     if (tid == 0) {
         offsets[e] = e * K;
+        mt_first[e] = e * nt;   // plain expert order: one part, bands per expert
         if (e == E - 1) {
             offsets[E] = E * K;
             *num_mt = E * nt;
+            mt_first[E] = E * nt;
         }
     }
     const int rem = K - (nt - 1) * kBlockM;
@@ -222,12 +225,12 @@ int launch_softmax_rows(const moe_shape_t &s, const float *logits, float *scores
 
 int launch_ec_select(const moe_shape_t &s, int K, const float *scores, int32_t *tokens,
                      float *weights, int32_t *offsets, int32_t *mt_row0, int32_t *mt_group,
-                     int32_t *num_mt, uint32_t *status, cudaStream_t st)
+                     int32_t *num_mt, int32_t *mt_first, uint32_t *status, cudaStream_t st)
 {
     if (s.T == 0 || K == 0)
         return MOE_OK;
     k_ec_select<<<s.E, kEcThreads, 0, st>>>(scores, s.T, s.E, K, tokens, weights, offsets, mt_row0,
-                                            mt_group, num_mt, status);
+                                            mt_group, num_mt, mt_first, status);
     return launched();
 }
 

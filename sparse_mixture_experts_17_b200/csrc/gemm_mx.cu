@@ -52,6 +52,7 @@
 #include "internal.h"
 #include "mxfp8.cuh"
 #include "nvfp4.cuh"
+#include "tiles.cuh"
 
 namespace moe {
 
@@ -66,6 +67,10 @@ struct MxArgs {
     int kblocks;            // K stages (K / 128 E4M3 or K / 256 E2M1 elements)
     int n_tiles;
     int group_m;
+    // band order over the routed list (band_coords); NULL: plain bands
+    const int32_t *mt_first;
+    int n_groups;
+    int band_g;
     int b_rows_per_group;
     const int32_t *mt_row0;
     const int32_t *mt_group;
@@ -118,6 +123,16 @@ __device__ __forceinline__ void mx_tile_coords(long long tile, int num_mt, int n
     const int r = (int)(tile - (long long)band * band_size);
     m_idx = first_m + r % rows;
     n_idx = r / rows;
+}
+
+__device__ __forceinline__ void mx_coords(const MxArgs &p, long long tile, int num_mt, int &m_idx,
+                                          int &n_idx)
+{
+    if (p.mt_first)
+        band_coords(tile, num_mt, p.n_tiles, p.band_g, kBlockM, p.mt_first, p.n_groups, p.mt_group,
+                    p.seg_offsets, m_idx, n_idx);
+    else
+        mx_tile_coords(tile, num_mt, p.n_tiles, p.group_m, m_idx, n_idx);
 }
 
 // Shared-memory descriptor of one 32-row x 16-byte scale atom (no swizzle:
@@ -347,7 +362,7 @@ __global__ void __launch_bounds__(192, 1)
             bool ok = true;
             for (long long tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
                 int m_idx, n_idx;
-                mx_tile_coords(tile, num_mt, p.n_tiles, p.group_m, m_idx, n_idx);
+                mx_coords(p, tile, num_mt, m_idx, n_idx);
                 const long long row0 = p.mt_row0 ? p.mt_row0[m_idx] : (long long)m_idx * C::BM;
                 const int grp = p.mt_group ? (p.mt_group[m_idx] & ~kHalfTileBit) : 0;
                 const long long brow = (long long)grp * p.b_rows_per_group + (long long)n_idx * C::BN;
@@ -425,7 +440,7 @@ __global__ void __launch_bounds__(192, 1)
         uint32_t local = 0;
         for (long long tile = blockIdx.x; tile < total; tile += gridDim.x, ++local) {
             int m_idx, n_idx;
-            mx_tile_coords(tile, num_mt, p.n_tiles, p.group_m, m_idx, n_idx);
+            mx_coords(p, tile, num_mt, m_idx, n_idx);
             const long long row0 = p.mt_row0 ? p.mt_row0[m_idx] : (long long)m_idx * C::BM;
             const int grp = p.mt_group ? (p.mt_group[m_idx] & ~kHalfTileBit) : 0;
             const long long row_end = p.seg_offsets ? p.seg_offsets[grp + 1] : p.rows_valid;
@@ -509,6 +524,11 @@ static int launch_mx_impl(const GemmArgs &g, cudaStream_t st)
     p.kblocks = g.K / C::BK;
     p.n_tiles = g.N / C::BN;
     p.group_m = (MODE == EPI_SWIGLU_MX) ? MOE_GM_MX_W13 : MOE_GM_MX_W2;
+    // bands hold at most 48 MiB of activation codes
+    p.mt_first = g.mt_row0 ? g.mt_first : nullptr;
+    p.n_groups = g.n_groups;
+    p.band_g = (int)std::min<long long>(
+        std::max<long long>((48LL << 20) / std::max(128 * row_bytes, 1LL), 1), 1 << 20);
     p.b_rows_per_group = g.b_rows_per_group;
     p.mt_row0 = g.mt_row0;
     p.mt_group = g.mt_group;

@@ -52,6 +52,11 @@ struct TcArgs {
     int kblocks;
     int n_tiles;
     int group_m;
+    // band order over a routed list (band_coords); mt_first NULL: plain bands
+    // of group_m m-tiles
+    const int32_t *mt_first;
+    int n_groups;
+    int band_g;
     int b_rows_per_group;
     const int32_t *mt_row0;
     const int32_t *mt_group;
@@ -80,7 +85,7 @@ struct TcArgs {
     long long out_group_stride;
     int32_t *hist_chunk, *hist_rank, *hist_counter, *hist_counts, *hist_offsets, *hist_n_kept;
     int32_t *hist_mt_row0, *hist_mt_group, *hist_num_mt, *hist_mt2_row0, *hist_mt2_group,
-        *hist_num_mt2;
+        *hist_num_mt2, *hist_mt_first, *hist_mt2_first;
     int capacity;
     // bound of every pipeline wait; `starve` (test only): the producer issues
     // no loads, so the first wait on a full stage runs out and every role unwinds
@@ -166,6 +171,17 @@ __device__ __forceinline__ void tile_coords(long long tile, int num_mt, int n_ti
     const int r = (int)(tile - (long long)band * band_size);
     m_idx = first_m + r % rows;
     n_idx = r / rows;
+}
+
+// Tile -> (m-tile, n-tile): band order over a routed list, else plain bands.
+__device__ __forceinline__ void tc_coords(const TcArgs &p, long long tile, int num_mt, int tile_m,
+                                          int &m_idx, int &n_idx)
+{
+    if (p.mt_first)
+        band_coords(tile, num_mt, p.n_tiles, p.band_g, tile_m, p.mt_first, p.n_groups,
+                    p.mt_group, p.seg_offsets, m_idx, n_idx);
+    else
+        tile_coords(tile, num_mt, p.n_tiles, p.group_m, m_idx, n_idx);
 }
 
 // Epilogue of one accumulator tile for this thread's row (TMEM lane): `tb`
@@ -558,7 +574,7 @@ __global__ void __launch_bounds__(192, 1)
             uint32_t it = 0;
             for (long long tile = blockIdx.x; tile < total; tile += gridDim.x) {
                 int m_idx, n_idx;
-                tile_coords(tile, num_mt, p.n_tiles, p.group_m, m_idx, n_idx);
+                tc_coords(p, tile, num_mt, C::BM, m_idx, n_idx);
                 const int row0 = p.mt_row0 ? p.mt_row0[m_idx] : m_idx * C::BM;
                 const int grp = p.mt_group ? (p.mt_group[m_idx] & ~kHalfTileBit) : 0;
                 const int brow = grp * p.b_rows_per_group + n_idx * BN;
@@ -595,7 +611,7 @@ __global__ void __launch_bounds__(192, 1)
             for (long long tile = blockIdx.x; tile < total; tile += gridDim.x, ++local) {
                 const uint32_t b = local & 1u, aph = (local >> 1) & 1u;
                 int m_idx, n_idx;
-                tile_coords(tile, num_mt, p.n_tiles, p.group_m, m_idx, n_idx);
+                tc_coords(p, tile, num_mt, C::BM, m_idx, n_idx);
                 const bool half = p.mt_group && (p.mt_group[m_idx] & kHalfTileBit);
                 const uint32_t IDESC = half ? IDESC64 : IDESC128;
                 const int grp = p.mt_group ? (p.mt_group[m_idx] & ~kHalfTileBit) : 0;
@@ -631,7 +647,7 @@ __global__ void __launch_bounds__(192, 1)
         uint32_t local = 0;
         for (long long tile = blockIdx.x; tile < total; tile += gridDim.x, ++local) {
             int m_idx, n_idx;
-            tile_coords(tile, num_mt, p.n_tiles, p.group_m, m_idx, n_idx);
+            tc_coords(p, tile, num_mt, C::BM, m_idx, n_idx);
             const long long row0 = p.mt_row0 ? p.mt_row0[m_idx] : (long long)m_idx * C::BM;
             const int gword = p.mt_group ? p.mt_group[m_idx] : 0;
             const int grp = gword & ~kHalfTileBit;
@@ -691,7 +707,8 @@ __global__ void __launch_bounds__(192, 1)
                 hist_finish(p.hist_chunk, num_mt, 1, p.n_valid, p.capacity, p.hist_counts,
                             p.hist_offsets, p.hist_n_kept, p.hist_mt_row0, p.hist_mt_group,
                             p.hist_num_mt, p.hist_mt2_row0, p.hist_mt2_group, p.hist_num_mt2,
-                            nullptr, p.hist_counter, H.kept, H.off, H.warp);
+                            nullptr, p.hist_counter, H.kept, H.off, H.warp, p.hist_mt_first,
+                            p.hist_mt2_first);
             }
         }
     }
@@ -774,7 +791,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
             uint32_t it = 0;
             for (long long tile = pair; tile < total; tile += npairs) {
                 int m_idx, n_idx;
-                tile_coords(tile, num_mt, p.n_tiles, p.group_m, m_idx, n_idx);
+                tc_coords(p, tile, num_mt, 256, m_idx, n_idx);
                 const int row0 = (p.mt_row0 ? p.mt_row0[m_idx] : m_idx * 256) + 128 * (int)rank;
                 const int grp = p.mt_group ? (p.mt_group[m_idx] & ~kHalfTileBit) : 0;
                 const int brow = grp * p.b_rows_per_group + n_idx * BN + 128 * (int)rank;
@@ -833,7 +850,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
         uint32_t local = 0;
         for (long long tile = pair; tile < total; tile += npairs, ++local) {
             int m_idx, n_idx;
-            tile_coords(tile, num_mt, p.n_tiles, p.group_m, m_idx, n_idx);
+            tc_coords(p, tile, num_mt, 256, m_idx, n_idx);
             const long long row0 = (p.mt_row0 ? p.mt_row0[m_idx] : (long long)m_idx * 256) + 128 * rank;
             const int grp = p.mt_group ? (p.mt_group[m_idx] & ~kHalfTileBit) : 0;
             const long long row_end = p.seg_offsets ? p.seg_offsets[grp + 1] : p.rows_valid;
@@ -901,6 +918,19 @@ static int make_tmap(CUtensorMap *m, const void *base, long long cols, long long
     return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
 }
 
+// Band height of a routed GEMM (band_coords): a band's activation rows stay
+// in L2 while it sweeps the n-tiles, so its m-tiles are bounded by
+// MOE_BAND_MB MiB of bf16 rows of length K.
+#ifndef MOE_BAND_MB
+#define MOE_BAND_MB 48
+#endif
+static int band_tiles(long long tile_rows, int K)
+{
+    const long long per = std::max(tile_rows * K * 2, 1LL);
+    return (int)std::min<long long>(std::max<long long>(((long long)MOE_BAND_MB << 20) / per, 1),
+                                    1 << 20);
+}
+
 int num_sms()
 {
     int dev = 0, n = 0;
@@ -926,6 +956,7 @@ static int launch_tc_impl(const GemmArgs &g, cudaStream_t st)
     if (rc)
         return rc;
     TcArgs p;
+    std::memset(&p, 0, sizeof p);
     p.kblocks = g.K / 64;
     p.n_tiles = (MODE == EPI_SWIGLU || MODE == EPI_SWIGLU_SAVE) ? g.N / 256 : (g.N + BN - 1) / BN;
     // Rasterisation: consecutive tiles sweep a band of group_m m-tiles across
@@ -933,6 +964,9 @@ static int launch_tc_impl(const GemmArgs &g, cudaStream_t st)
     // its A rows stay in L2. Measured on the Mixtral-shape prefill: bands of 32
     // cut w1/w3 DRAM reads by ~15% and time by ~5% against 8; w2 is flat.
     p.group_m = (MODE == EPI_SWIGLU) ? MOE_GM_1SM_W13 : MOE_GM_1SM_W2;
+    p.mt_first = g.mt_row0 ? g.mt_first : nullptr;
+    p.n_groups = g.n_groups;
+    p.band_g = band_tiles(C::BM, g.K);
     p.b_rows_per_group = g.b_rows_per_group;
     p.mt_row0 = g.mt_row0;
     p.mt_group = g.mt_group;
@@ -971,6 +1005,8 @@ static int launch_tc_impl(const GemmArgs &g, cudaStream_t st)
     p.hist_mt2_row0 = g.hist_mt2_row0;
     p.hist_mt2_group = g.hist_mt2_group;
     p.hist_num_mt2 = g.hist_num_mt2;
+    p.hist_mt_first = g.hist_mt_first;
+    p.hist_mt2_first = g.hist_mt2_first;
     p.capacity = g.capacity;
     p.starve = g.test_starve;
     p.wait_ns = g.test_starve ? kTestWaitLimitNs : kWaitLimitNs;
@@ -1015,6 +1051,9 @@ static int launch_tc2_impl(const GemmArgs &g, cudaStream_t st)
     p.kblocks = g.K / 64;
     p.n_tiles = g.N / 256;
     p.group_m = (MODE == EPI_SWIGLU) ? MOE_GM_2SM_W13 : MOE_GM_2SM_W2;
+    p.mt_first = g.mt_row0 ? g.mt_first : nullptr;
+    p.n_groups = g.n_groups;
+    p.band_g = band_tiles(256, g.K);
     p.b_rows_per_group = g.b_rows_per_group;
     p.mt_row0 = g.mt_row0;
     p.mt_group = g.mt_group;

@@ -65,6 +65,7 @@ struct WsLayout {
     size_t slot_pos, perm_token;
     size_t mt_row0, mt_group;
     size_t mt2_row0, mt2_group, num_mt2;   // 256-row tiles of the 2-SM GEMM
+    size_t mt_first, mt2_first;            // E + 1 ints each (build_tiles)
     size_t x_perm, H, H_shared, Y;
     size_t dec_H;
     size_t x_stage, out_stage;
@@ -97,18 +98,22 @@ int launch_router_simt(const moe_shape_t &s, const uint16_t *x, const uint16_t *
 int launch_topk(const moe_shape_t &s, const float *logits, int32_t *idx, float *w,
                 int32_t *counter_to_zero, uint32_t *status, cudaStream_t st);
 // Also writes the 256-row m-tile list of the 2-SM GEMM when mt2_row0 is non-NULL.
+// mt_first / mt2_first (E + 1 ints each, may be NULL): the lists' expert
+// positions for the GEMMs' band order (build_tiles in tiles.cuh).
 int launch_hist_scan(const moe_shape_t &s, const int32_t *idx, int32_t *chunk_counts,
                      int32_t *rank_local, int32_t *counter, int32_t *counts, int32_t *offsets,
                      int32_t *n_kept, int32_t *mt_row0, int32_t *mt_group, int32_t *num_mt,
                      int32_t *mt2_row0, int32_t *mt2_group, int32_t *num_mt2, uint32_t *status,
-                     cudaStream_t st, int32_t *tile_start = nullptr);
+                     cudaStream_t st, int32_t *tile_start = nullptr, int32_t *mt_first = nullptr,
+                     int32_t *mt2_first = nullptr);
 int launch_permute(const moe_shape_t &s, const int32_t *idx, const int32_t *chunk_base,
                    const int32_t *rank_local, const int32_t *offsets, const uint16_t *x,
                    int32_t *slot_pos, int32_t *perm_token, uint16_t *x_perm, float *out_zero,
                    cudaStream_t st, int chunk_tokens = kChunkTokens);
 int launch_tiles_from_offsets(const moe_shape_t &s, const int32_t *offsets, int32_t *mt_row0,
                               int32_t *mt_group, int32_t *num_mt, int32_t *mt2_row0,
-                              int32_t *mt2_group, int32_t *num_mt2, cudaStream_t st);
+                              int32_t *mt2_group, int32_t *num_mt2, cudaStream_t st,
+                              int32_t *mt_first = nullptr, int32_t *mt2_first = nullptr);
 int launch_combine(const moe_shape_t &s, const float *y_perm, const int32_t *slot_pos,
                    const float *topk_w, const float *shared_out, float *out, cudaStream_t st);
 int launch_pack_w13(int E, int d_ff, int d, const uint16_t *W1, const uint16_t *W3,
@@ -165,6 +170,10 @@ struct GemmArgs {
     const int32_t *num_mt_dev; // NULL: use num_mt_host
     int num_mt_host;
     int max_mt;               // upper bound of the m-tile count (grid sizing)
+    // routed lists in build_tiles' order: each group's first position, and at
+    // [n_groups] the multi-tile part's length; NULL: plain bands of m-tiles
+    const int32_t *mt_first;
+    int n_groups;
     const int32_t *seg_offsets; // group g rows end at seg_offsets[g+1]; NULL: rows_valid
     long long rows_valid;
     // epilogue
@@ -209,7 +218,7 @@ struct GemmArgs {
     // 128-token m-tile expert counts and ranks, then the last CTA's scan
     int32_t *hist_chunk, *hist_rank, *hist_counter, *hist_counts, *hist_offsets, *hist_n_kept;
     int32_t *hist_mt_row0, *hist_mt_group, *hist_num_mt, *hist_mt2_row0, *hist_mt2_group,
-        *hist_num_mt2;
+        *hist_num_mt2, *hist_mt_first, *hist_mt2_first;
     int capacity;
     // test only (single-SM tensor-core kernel): the producer issues no loads and
     // the pipeline waits give up after 50 ms, so the launch returns with
@@ -312,7 +321,7 @@ int launch_softmax_rows(const moe_shape_t &s, const float *logits, float *scores
                         uint32_t *status, cudaStream_t st);
 int launch_ec_select(const moe_shape_t &s, int K, const float *scores, int32_t *tokens,
                      float *weights, int32_t *offsets, int32_t *mt_row0, int32_t *mt_group,
-                     int32_t *num_mt, uint32_t *status, cudaStream_t st);
+                     int32_t *num_mt, int32_t *mt_first, uint32_t *status, cudaStream_t st);
 int launch_ec_gather(const moe_shape_t &s, int rows, const uint16_t *x, const int32_t *tokens,
                      uint16_t *x_perm, float *out_zero, cudaStream_t st);
 

@@ -133,6 +133,8 @@ WsLayout ws_layout(const moe_shape_t &s)
     L.mt2_row0 = take((size_t)L.max_mt2 * 4);
     L.mt2_group = take((size_t)L.max_mt2 * 4);
     L.num_mt2 = take(4);
+    L.mt_first = take((E + 1) * 4);
+    L.mt2_first = take((E + 1) * 4);
     const bool mx = (s.flags & MOE_FLAG_MXFP8) != 0;
     const bool nv = (s.flags & MOE_FLAG_NVFP4) != 0;
     const bool lowp = mx || nv;   // block-scaled experts: codes instead of bf16 copies
@@ -253,9 +255,11 @@ static bool use_pair(const moe_shape_t &s, long long avg_rows, int n_out, bool i
 }
 
 // Point a routed GEMM at the m-tile list of its engine.
-static void set_tiles(GemmArgs &g, const WsLayout &L, void *ws, bool pair)
+static void set_tiles(GemmArgs &g, const moe_shape_t &s, const WsLayout &L, void *ws, bool pair)
 {
     g.pair = pair ? 1 : 0;
+    g.mt_first = reinterpret_cast<int32_t *>(static_cast<char *>(ws) + (pair ? L.mt2_first : L.mt_first));
+    g.n_groups = s.E;
     g.mt_row0 = reinterpret_cast<int32_t *>(static_cast<char *>(ws) + (pair ? L.mt2_row0 : L.mt_row0));
     g.mt_group = reinterpret_cast<int32_t *>(static_cast<char *>(ws) + (pair ? L.mt2_group : L.mt_group));
     g.num_mt_dev = reinterpret_cast<int32_t *>(static_cast<char *>(ws) + (pair ? L.num_mt2 : L.num_mt));
@@ -289,7 +293,7 @@ static int expert_ffn_core(const moe_shape_t &s, const WsLayout &L, void *ws,
     g.N = 2 * s.d_ff;
     g.b_rows_per_group = 2 * s.d_ff;
     const long long avg_rows = N / s.E;
-    set_tiles(g, L, ws, allow_pair && use_pair(s, avg_rows, g.N, false));
+    set_tiles(g, s, L, ws, allow_pair && use_pair(s, avg_rows, g.N, false));
     g.seg_offsets = offsets;
     g.out = H;
     g.ldo = s.d_ff;
@@ -310,7 +314,7 @@ static int expert_ffn_core(const moe_shape_t &s, const WsLayout &L, void *ws,
     g.N = s.d;
     g.b_rows_per_group = s.d;
     g.ldo = s.d;
-    set_tiles(g, L, ws, allow_pair && use_pair(s, avg_rows, g.N, true));
+    set_tiles(g, s, L, ws, allow_pair && use_pair(s, avg_rows, g.N, true));
     if (y_perm) {
         g.mode = EPI_STORE_F32;
         g.out = y_perm;
@@ -441,7 +445,7 @@ static bool router_hist_fusable(const moe_shape_t &s)
 
 struct HistOut {
     int32_t *chunk, *rank, *counts, *offsets, *n_kept, *mt_row0, *mt_group, *num_mt, *mt2_row0,
-        *mt2_group, *num_mt2;
+        *mt2_group, *num_mt2, *mt_first, *mt2_first;
 };
 
 static int router_topk_hist(const moe_shape_t &s, const uint16_t *x, const uint16_t *Wg,
@@ -479,6 +483,8 @@ static int router_topk_hist(const moe_shape_t &s, const uint16_t *x, const uint1
     g.hist_mt2_row0 = h.mt2_row0;
     g.hist_mt2_group = h.mt2_group;
     g.hist_num_mt2 = h.num_mt2;
+    g.hist_mt_first = h.mt_first;
+    g.hist_mt2_first = h.mt2_first;
     g.capacity = s.capacity;
     // the ticket starts at zero whatever an earlier, aborted call left in it
     if (cudaMemsetAsync(counter, 0, sizeof(int32_t), st) != cudaSuccess)
@@ -531,7 +537,8 @@ static int forward_impl(const moe_shape_t &s, const WsLayout &L, void *ws, const
                           at<int32_t>(ws, L.n_kept),       at<int32_t>(ws, L.mt_row0),
                           at<int32_t>(ws, L.mt_group),     at<int32_t>(ws, L.num_mt),
                           at<int32_t>(ws, L.mt2_row0),     at<int32_t>(ws, L.mt2_group),
-                          at<int32_t>(ws, L.num_mt2)};
+                          at<int32_t>(ws, L.num_mt2),      at<int32_t>(ws, L.mt_first),
+                          at<int32_t>(ws, L.mt2_first)};
     const bool hist_fused = !decode && router_hist_fusable(s);
     int rc;
     if (hist_fused) {
@@ -569,7 +576,8 @@ static int forward_impl(const moe_shape_t &s, const WsLayout &L, void *ws, const
                               at<int32_t>(ws, L.n_kept), at<int32_t>(ws, L.mt_row0),
                               at<int32_t>(ws, L.mt_group), at<int32_t>(ws, L.num_mt),
                               at<int32_t>(ws, L.mt2_row0), at<int32_t>(ws, L.mt2_group),
-                              at<int32_t>(ws, L.num_mt2), status, st);
+                              at<int32_t>(ws, L.num_mt2), status, st, nullptr,
+                              at<int32_t>(ws, L.mt_first), at<int32_t>(ws, L.mt2_first));
     }
     if (rc)
         return rc;
@@ -639,7 +647,7 @@ static int expert_ffn_mx(const moe_shape_t &s, const WsLayout &L, void *ws, cons
     g.K = s.d;
     g.N = 2 * s.d_ff;
     g.b_rows_per_group = 2 * s.d_ff;
-    set_tiles(g, L, ws, false);
+    set_tiles(g, s, L, ws, false);
     g.seg_offsets = offsets;
     g.out = at<uint8_t>(ws, L.Hq);
     g.ldo = s.d_ff;
@@ -813,7 +821,8 @@ static int forward_mx_impl(const moe_shape_t &s, const WsLayout &L, void *ws, co
         rc = launch_hist_scan(s, idx, chunk, rank, counter, at<int32_t>(ws, L.counts), offsets,
                               at<int32_t>(ws, L.n_kept), at<int32_t>(ws, L.mt_row0),
                               at<int32_t>(ws, L.mt_group), at<int32_t>(ws, L.num_mt), nullptr,
-                              nullptr, nullptr, status, st, at<int32_t>(ws, L.tile_start));
+                              nullptr, nullptr, status, st, at<int32_t>(ws, L.tile_start),
+                              at<int32_t>(ws, L.mt_first));
     }
     if (rc)
         return rc;
@@ -1000,7 +1009,7 @@ static int backward_impl(const moe_shape_t &s, const WsLayout &L, void *ws, cons
         rc = launch_hist_scan(s, idx, chunk, rank, counter, at<int32_t>(ws, L.counts), offsets,
                               at<int32_t>(ws, L.n_kept), at<int32_t>(ws, L.mt_row0),
                               at<int32_t>(ws, L.mt_group), at<int32_t>(ws, L.num_mt), nullptr,
-                              nullptr, nullptr, status, st);
+                              nullptr, nullptr, status, st, nullptr, at<int32_t>(ws, L.mt_first));
     }
     if (rc)
         return rc;
@@ -1022,7 +1031,7 @@ static int backward_impl(const moe_shape_t &s, const WsLayout &L, void *ws, cons
     g.K = s.d;
     g.N = 2 * s.d_ff;
     g.b_rows_per_group = 2 * s.d_ff;
-    set_tiles(g, L, ws, false);
+    set_tiles(g, s, L, ws, false);
     g.seg_offsets = offsets;
     g.out = H;
     g.ldo = s.d_ff;
@@ -1046,7 +1055,7 @@ static int backward_impl(const moe_shape_t &s, const WsLayout &L, void *ws, cons
     g.K = s.d;
     g.N = s.d_ff;
     g.b_rows_per_group = s.d_ff;
-    set_tiles(g, L, ws, false);
+    set_tiles(g, s, L, ws, false);
     g.seg_offsets = offsets;
     g.out = dGU;
     g.ldo = s.d_ff;
@@ -1068,7 +1077,7 @@ static int backward_impl(const moe_shape_t &s, const WsLayout &L, void *ws, cons
     g.K = 2 * s.d_ff;
     g.N = s.d;
     g.b_rows_per_group = s.d;
-    set_tiles(g, L, ws, false);
+    set_tiles(g, s, L, ws, false);
     g.seg_offsets = offsets;
     g.out = dx;
     g.ldo = s.d;
@@ -1179,7 +1188,7 @@ static int ec_route(const moe_shape_t &s, const WsLayout &L, void *ws, const uin
     StageMark m(MOE_STAGE_HIST, st);
     return launch_ec_select(s, K, scores, tokens, weights, at<int32_t>(ws, L.offsets),
                             at<int32_t>(ws, L.mt_row0), at<int32_t>(ws, L.mt_group),
-                            at<int32_t>(ws, L.num_mt), status, st);
+                            at<int32_t>(ws, L.num_mt), at<int32_t>(ws, L.mt_first), status, st);
 }
 
 // ---------------------------------------------------------------- host I/O pipeline
@@ -1420,7 +1429,8 @@ int moe_permute(const moe_shape_t *shape, const int32_t *topk_idx, const moe_bf1
     rc = launch_hist_scan(s, topk_idx, chunk, rank, counter, expert_counts, expert_offsets, nk,
                           at<int32_t>(ws, L.mt_row0), at<int32_t>(ws, L.mt_group),
                           at<int32_t>(ws, L.num_mt), at<int32_t>(ws, L.mt2_row0),
-                          at<int32_t>(ws, L.mt2_group), at<int32_t>(ws, L.num_mt2), status, st);
+                          at<int32_t>(ws, L.mt2_group), at<int32_t>(ws, L.num_mt2), status, st,
+                          nullptr, at<int32_t>(ws, L.mt_first), at<int32_t>(ws, L.mt2_first));
     if (rc)
         return rc;
     rc = launch_permute(s, topk_idx, chunk, rank, expert_offsets, x, slot_pos, perm_token,
@@ -1484,7 +1494,8 @@ int moe_expert_ffn(const moe_shape_t *shape, const moe_bf16_t *x_perm,
     rc = launch_tiles_from_offsets(s, expert_offsets, at<int32_t>(ws, L.mt_row0),
                                    at<int32_t>(ws, L.mt_group), at<int32_t>(ws, L.num_mt),
                                    at<int32_t>(ws, L.mt2_row0), at<int32_t>(ws, L.mt2_group),
-                                   at<int32_t>(ws, L.num_mt2), st);
+                                   at<int32_t>(ws, L.num_mt2), st, at<int32_t>(ws, L.mt_first),
+                                   at<int32_t>(ws, L.mt2_first));
     if (rc)
         return rc;
     return expert_ffn_core(s, L, ws, x_perm, expert_offsets, W13, W2, perm_token, slot_pos, topk_w,

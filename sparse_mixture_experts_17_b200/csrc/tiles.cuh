@@ -46,72 +46,98 @@ __device__ __forceinline__ int block_excl_scan(int v, int *s_warp, int *total)
     return r;
 }
 
-// Position of element j of one sorted list (length n) in the merge of two
-// lists of lengths n and m spread evenly over each other: element j carries
-// the key (j + 1/2) / n, the other list's element i the key (i + 1/2) / m,
-// and ties go to `first` (the list whose elements precede on equal keys).
-__device__ __forceinline__ int spread_merge_pos(int j, int n, int m, bool first)
-{
-    if (m == 0)
-        return j;
-    const long long a = (long long)(2 * j + 1) * m;   // key of j, scaled by 2 n m
-    long long before;                                 // elements of the other list before j
-    if (first) {   // other elements i with (2i + 1) n < a
-        const long long num = a - n;
-        before = num <= 0 ? 0 : (num + 2LL * n - 1) / (2LL * n);
-    } else {       // other elements i with (2i + 1) n <= a
-        const long long num = a - n;
-        before = num < 0 ? 0 : num / (2LL * n) + 1;
-    }
-    return j + (int)(before < m ? before : m);
-}
-
 // Writes the grouped-GEMM m-tile list for kept counts in s_kept[E]: expert e
 // contributes ceil(kept/tile_m) tiles starting at rows offsets[e] + tile_m i.
 // Thread e handles expert e (blockDim.x >= E).
 //
-// Order. With tile_start == NULL the list interleaves two kinds of expert:
-// experts of one tile (few rows: their GEMM tiles stream a whole weight
-// block for few rows, so they are bound by DRAM) and experts of several
-// tiles (their tiles share each weight block through L2, so they are bound
-// by the tensor cores). Each list keeps expert order, and the two are spread
-// evenly over each other, so every stretch of the list that the GEMM runs at
-// once holds both kinds and the weight stream of the first overlaps the
-// arithmetic of the second. An expert's tiles stay in order. With tile_start
-// set (block-scaled operands, whose activation scales are keyed by tile
-// index) the list is in plain expert order and tile_start receives each
-// expert's first tile index.
+// Order. With tile_start == NULL the list holds first the experts of several
+// tiles, then the experts of one tile, each part in expert order and each
+// expert's tiles together and in order. The grouped GEMMs interleave the two
+// parts tile by tile (band_coords): one-tile experts stream a whole weight
+// block for few rows and are bound by DRAM, multi-tile experts share each
+// weight block between their tiles through L2 and are bound by the tensor
+// cores, so the mix keeps both busy. With tile_start set (block-scaled
+// operands, whose activation scales are keyed by tile index) the list is in
+// plain expert order and tile_start receives each expert's first tile index.
+// `first` (E + 1 ints, may be NULL) receives each expert's first position in
+// the list and, at [E], the length of the first part (the whole list in
+// plain order).
 __device__ inline void build_tiles(const int *s_kept, const int32_t *offsets_smem_or_global, int E,
                                    int tile_m, int32_t *mt_row0, int32_t *mt_group,
-                                   int32_t *num_mt, int *s_warp, int32_t *tile_start = nullptr)
+                                   int32_t *num_mt, int *s_warp, int32_t *tile_start = nullptr,
+                                   int32_t *first = nullptr)
 {
-    const int tid = threadIdx.x;
-    const int e = tid;
+    const int e = threadIdx.x;
     const int nt = (e < E) ? (s_kept[e] + tile_m - 1) / tile_m : 0;
-    const bool spread = tile_start == nullptr;
-    const bool multi = nt >= 2;
-    int total, n_multi, n_single;
-    const int start = block_excl_scan(nt, s_warp, &total);
-    const int start_m = block_excl_scan(spread && multi ? nt : 0, s_warp, &n_multi);
-    const int start_s = block_excl_scan(spread && !multi ? nt : 0, s_warp, &n_single);
-    if (e < E && tile_start)
-        tile_start[e] = start;
+    const bool multi = tile_start != nullptr || nt >= 2;
+    int n_multi, n_single;
+    const int start_m = block_excl_scan(multi ? nt : 0, s_warp, &n_multi);
+    const int start_s = block_excl_scan(multi ? 0 : nt, s_warp, &n_single);
+    const int start = multi ? start_m : n_multi + start_s;
     if (e < E) {
+        if (tile_start)
+            tile_start[e] = start;
+        if (first)
+            first[e] = start;
         const int base = offsets_smem_or_global[e];
         // a last tile of <= 64 rows is marked for the M = 64 MMA (128-row lists only)
         const int rem = s_kept[e] - (nt - 1) * tile_m;
         for (int i = 0; i < nt; ++i) {
-            int pos = start + i;
-            if (spread)
-                pos = multi ? spread_merge_pos(start_m + i, n_multi, n_single, true)
-                            : spread_merge_pos(start_s + i, n_single, n_multi, false);
-            mt_row0[pos] = base + i * tile_m;
+            mt_row0[start + i] = base + i * tile_m;
             const bool half = (tile_m == kBlockM) && (i == nt - 1) && rem <= 64;
-            mt_group[pos] = e | (half ? kHalfTileBit : 0);
+            mt_group[start + i] = e | (half ? kHalfTileBit : 0);
         }
     }
-    if (tid == 0)
-        *num_mt = total;
+    if (e == 0) {
+        *num_mt = n_multi + n_single;
+        if (first)
+            first[E] = n_multi;
+    }
+}
+
+// Maps tile t (0 <= t < num_mt * n_tiles) of a grouped GEMM to its m-tile and
+// n-tile, over a list in build_tiles' order (first[e]: expert e's first
+// position; first[E] = nh, the multi-tile part). The tiles of the two parts
+// are interleaved evenly: position t belongs to the multi-tile part when
+// floor((t + 1) Th / Tt) > floor(t Th / Tt), Th and Tt being that part's and
+// the whole list's tile counts.
+//  - Multi-tile part: each expert's m-tiles form bands of at most gmax
+//    (split into near-equal bands when it has more), and a band's tiles run
+//    m-tile fastest, then n-tile, so every weight block of the expert is
+//    fetched from DRAM once per band and its other m-tiles read it from L2;
+//    bands never hold two experts. gmax bounds the activation rows a band
+//    keeps in L2 while it sweeps the n-tiles.
+//  - One-tile part: each expert's n-tiles in order (its activation tile stays
+//    in L2 across them).
+// tile_m is the list's tile height (counts come from the kept offsets seg).
+__host__ __device__ __forceinline__ void band_coords(long long t, int num_mt, int n_tiles, int gmax,
+                                            int tile_m, const int32_t *first, int E,
+                                            const int32_t *mt_group, const int32_t *seg,
+                                            int &m_idx, int &n_idx)
+{
+    const int nh = first[E];
+    const long long Tt = (long long)num_mt * n_tiles, Th = (long long)nh * n_tiles;
+    const long long a = (t + 1) * Th / Tt;   // multi-part tiles among positions 0..t
+    if (a > t * Th / Tt) {
+        const long long u = a - 1;
+        const int pm = (int)(u / n_tiles);
+        const int e = mt_group[pm] & ~kHalfTileBit;
+        const int f = first[e];
+        const int cnt = (seg[e + 1] - seg[e] + tile_m - 1) / tile_m;
+        const int nb = (cnt + gmax - 1) / gmax;
+        const int q = cnt / nb, r = cnt - q * nb;   // r bands of q + 1, then bands of q
+        const int j = pm - f, big = r * (q + 1);
+        const int bi = j < big ? j / (q + 1) : r + (j - big) / q;
+        const int b0 = f + (bi < r ? bi * (q + 1) : big + (bi - r) * q);
+        const int rows = q + (bi < r ? 1 : 0);
+        const long long rr = u - (long long)b0 * n_tiles;
+        m_idx = b0 + (int)(rr % rows);
+        n_idx = (int)(rr / rows);
+    } else {
+        const long long v = t - a;
+        m_idx = nh + (int)(v / n_tiles);
+        n_idx = (int)(v - (long long)(v / n_tiles) * n_tiles);
+    }
 }
 
 // Run by every thread of the last CTA (after a fence that makes the other
@@ -126,7 +152,7 @@ __device__ inline void hist_finish(int32_t *chunk_counts, int nchunks, int nj, i
                                    int32_t *mt_row0, int32_t *mt_group, int32_t *num_mt,
                                    int32_t *mt2_row0, int32_t *mt2_group, int32_t *num_mt2,
                                    int32_t *tile_start, int32_t *counter, int *s_kept, int *s_off,
-                                   int *s_warp)
+                                   int *s_warp, int32_t *mt_first, int32_t *mt2_first)
 {
     const int tid = threadIdx.x;
     const int R = nj * nchunks;   // count rows of one expert, in rank order r = j * nchunks + c
@@ -217,9 +243,10 @@ __device__ inline void hist_finish(int32_t *chunk_counts, int nchunks, int nj, i
         *n_kept = total;
     }
     __syncthreads();
-    build_tiles(s_kept, s_off, E, kBlockM, mt_row0, mt_group, num_mt, s_warp, tile_start);
+    build_tiles(s_kept, s_off, E, kBlockM, mt_row0, mt_group, num_mt, s_warp, tile_start, mt_first);
     if (mt2_row0)
-        build_tiles(s_kept, s_off, E, 2 * kBlockM, mt2_row0, mt2_group, num_mt2, s_warp);
+        build_tiles(s_kept, s_off, E, 2 * kBlockM, mt2_row0, mt2_group, num_mt2, s_warp, nullptr,
+                    mt2_first);
     if (tid == 0)
         *counter = 0;
 }
