@@ -42,7 +42,8 @@ inline cudaError_t launch_pdl_ex(void (*kernel)(KArgs...), dim3 grid, dim3 block
 
 constexpr int kBlockM = 128;      // rows of one grouped-GEMM m-tile
 // Bit of an m-tile's group entry marking a tail tile of at most 64 rows: the
-// single-SM tensor-core GEMM runs it with M = 64 MMAs (half the tensor time).
+// single-SM tensor-core GEMM runs it with M = 64 MMAs and loads 64 A rows
+// (an M = 64 MMA takes as many tensor-pipe cycles as an M = 128 one).
 constexpr int32_t kHalfTileBit = 1 << 30;
 constexpr int kChunkTokens = 256; // tokens per histogram chunk (one CTA)
 

@@ -241,17 +241,20 @@ static int run_gemm(const moe_shape_t &s, const GemmArgs &g, cudaStream_t st)
 }
 
 // Engine choice. The 2-SM pair kernel (256-row tiles) moves a third less
-// operand data per FLOP. In interleaved measurements on the power-capped B200
-// it is 3-5% faster on the long-K w2 GEMM when experts hold >= 1024 rows, and
-// no faster on w1/w3, so by default only w2 takes it. Short groups would pad
-// up to 255 rows per tile. Output widths must be multiples of 256.
+// operand data per FLOP from L2 into shared memory, the other limit of a
+// stage beside the tensor pipe. With experts of >= 1024 rows it is the faster
+// engine for both GEMMs in interleaved measurements on the power-capped B200
+// (the prefill layer about 6% faster with w1/w3 on it as well). Short groups
+// would pad up to 255 rows per tile, so they stay on the single-SM kernel.
+// Output widths must be multiples of 256.
 static bool use_pair(const moe_shape_t &s, long long avg_rows, int n_out, bool is_w2)
 {
+    (void)is_w2;
     if ((s.flags & (MOE_FLAG_SIMT_FFN | MOE_FLAG_GEMM_1SM)) || n_out % 256 != 0)
         return false;
     if (s.flags & MOE_FLAG_GEMM_2SM)
         return true;
-    return is_w2 && avg_rows >= 1024;
+    return avg_rows >= 1024;
 }
 
 // Point a routed GEMM at the m-tile list of its engine.
