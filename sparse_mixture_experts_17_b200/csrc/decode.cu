@@ -25,7 +25,9 @@
 // The kernels are instantiated for MAXT in {1, 2, 4, 8, 16} >= T, the most
 // assignments one expert can have (a token picks an expert at most once), so
 // the per-token accumulators stay in registers and the code stays small.
+#include <algorithm>
 #include <cstring>
+#include <mutex>
 
 #include "common.cuh"
 #include "internal.h"
@@ -750,120 +752,200 @@ __device__ __forceinline__ float nv_chunk_dot(const uint4 &w, float sw0, float s
     return fmaf(b1, sw1 * xs.y, b0 * (sw0 * xs.x));
 }
 
-// Phase 1: one work unit = h column c of one chosen expert (its packed gate
-// and up rows, each streamed once), or of the shared expert.
+// Phase 1, fed by the TMA. Work item = one 128-row tile of a source's packed
+// W13: 64 gate and 64 up rows, i.e. h columns 64 t .. 64 t + 63 of source u
+// (a chosen expert, or the shared expert after them). A producer thread
+// streams the tile through a ring of K stages: 128 rows x 128 bytes of codes
+// (256 elements, one TMA box) and the stage's four 512-byte scale atoms (one
+// bulk copy); the copy engine keeps kNdStages stages in flight whatever the
+// consumers' registers. Four consumer warps own 32 rows each: lane l takes
+// the 32-element chunk l % 8 of rows l / 8 + 4 j (j < 8), so one load of x's
+// chunk serves eight rows and each 16-byte code read is conflict-free. At
+// the end of a tile the eight lanes of a row reduce their sums, and the h
+// columns are formed from the gate and up row sums in shared memory.
+constexpr int kNdStages = 4;
+constexpr int kNdStageBytes = 128 * 128;   // codes of one K stage (256 elements x 128 rows)
+constexpr int kNdSfBytes = 4 * 512;        // its four scale atoms
+constexpr int kNdThreads = 160;            // four consumer warps, then the producer warp
+
 template <int MAXT>
-__global__ void __launch_bounds__(256, 2)
-    k_dec_w13_nv(const uint16_t *__restrict__ xh, const float *__restrict__ xs, float x_gs,
-                 const int32_t *__restrict__ idx, int T, int d, int d_ff, int E, int k, int C,
-                 int slot_major, const uint8_t *__restrict__ W13q,
-                 const uint8_t *__restrict__ W13sf, const float *__restrict__ gs13, int d_ff_s,
-                 const uint8_t *__restrict__ W13s_q, const uint8_t *__restrict__ W13s_sf,
-                 const float *__restrict__ gs13s, float *__restrict__ H32,
-                 float *__restrict__ Hs32, uint32_t *status)
+struct NdSmem {
+    uint8_t code[kNdStages][kNdStageBytes];
+    uint8_t sf[kNdStages][kNdSfBytes];
+    uint64_t full[kNdStages], empty[kNdStages];
+    float rowsum[128][MAXT];
+    int abort;
+};
+
+__device__ __forceinline__ void nd_bulk_load(void *smem_dst, const void *src, uint32_t bytes,
+                                             uint64_t *bar)
 {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        ::"r"(smem_u32(smem_dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// named barrier of the four consumer warps
+__device__ __forceinline__ void nd_consumer_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+template <int MAXT>
+__global__ void __launch_bounds__(kNdThreads, 2)
+    k_dec_w13_nv(const __grid_constant__ CUtensorMap tmR, const __grid_constant__ CUtensorMap tmS,
+                 const uint16_t *__restrict__ xh, const float *__restrict__ xs, float x_gs,
+                 const int32_t *__restrict__ idx, int T, int d, int d_ff, int E, int k, int C,
+                 int slot_major, const uint8_t *__restrict__ W13sf,
+                 const float *__restrict__ gs13, int d_ff_s, int has_shared,
+                 const uint8_t *__restrict__ W13s_sf, const float *__restrict__ gs13s,
+                 float *__restrict__ H32, float *__restrict__ Hs32, uint32_t *status)
+{
+    extern __shared__ uint8_t nd_raw[];
+    NdSmem<MAXT> &S = *reinterpret_cast<NdSmem<MAXT> *>(
+        (reinterpret_cast<uintptr_t>(nd_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     __shared__ DecPlanSmem P;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kNdStages; ++s) {
+            mbar_init(&S.full[s], 1);
+            mbar_init(&S.empty[s], 4);
+        }
+        S.abort = 0;
+        fence_mbar_init();
+    }
     pdl_wait();
     pdl_trigger();
-    build_plan(P, idx, T, E, k, C, slot_major, status);
-    const int lane = threadIdx.x & 31;
-    const int nwarps = gridDim.x * (blockDim.x >> 5);
-    const long long routed_units = (long long)P.U * d_ff;
-    const long long units = routed_units + (W13s_q ? d_ff_s : 0);
-    const int nv = d / 32;   // 16-byte chunks of a packed row
-    for (long long unit = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; unit < units;
-         unit += nwarps) {
-        const uint8_t *qb, *sb;
-        int a0, na, c, ldh;
-        float *hout;
-        float gsw;
-        const bool shared = unit >= routed_units;
-        size_t prow;
-        if (!shared) {
-            const int u = (int)(unit / d_ff);
-            c = (int)(unit - (long long)u * d_ff);
-            // packed gate row of h column c; the up row is 64 rows further
-            prow = (size_t)P.uniq[u] * 2 * d_ff + (size_t)(c / 64) * 128 + (c % 64);
-            qb = W13q;
-            sb = W13sf;
-            gsw = gs13[P.uniq[u]];
-            a0 = P.ustart[u];
-            na = P.ustart[u + 1] - a0;
-            hout = H32;
-            ldh = d_ff;
-        } else {
-            c = (int)(unit - routed_units);
-            prow = (size_t)(c / 64) * 128 + (c % 64);
-            qb = W13s_q;
-            sb = W13s_sf;
-            gsw = gs13s[0];
-            a0 = 0;
-            na = T;
-            hout = Hs32;
-            ldh = d_ff_s;
+    build_plan(P, idx, T, E, k, C, slot_major, status);   // ends with __syncthreads
+    volatile int *abort_flag = &S.abort;
+    const int tpr = 2 * d_ff / 128;                        // tiles of a routed expert
+    const int routed_items = P.U * tpr;
+    const int items = routed_items + (has_shared ? 2 * d_ff_s / 128 : 0);
+    const int nks = (d + 255) / 256;   // K stages of a tile; the last holds 128 or 256 elements
+
+    if (warp == 4) {
+        if (lane == 0) {   // ---------------- producer
+            uint32_t it = 0;
+            bool ok = true;
+            for (int item = blockIdx.x; ok && item < items; item += gridDim.x) {
+                const bool shared = item >= routed_items;
+                const int t = shared ? item - routed_items : item % tpr;
+                const long long row0 =
+                    shared ? (long long)t * 128 : (long long)P.uniq[item / tpr] * 2 * d_ff + t * 128;
+                const uint8_t *sfb = (shared ? W13s_sf : W13sf) + (size_t)(row0 / 128) * (d / 64) * 512;
+                for (int ks = 0; ks < nks; ++ks, ++it) {
+                    const int s = it % kNdStages;
+                    const uint32_t ph = (it / kNdStages) & 1u;
+                    if (!mbar_wait(&S.empty[s], ph ^ 1u, abort_flag, status)) {
+                        ok = false;
+                        break;
+                    }
+                    // a 128-element last stage: the TMA box still spans 128 bytes per
+                    // row (the half past the row reads as zeros), the scales two atoms
+                    const uint32_t sf_bytes = (uint32_t)min(256, d - ks * 256) / 64 * 512;
+                    mbar_arrive_expect_tx(&S.full[s], kNdStageBytes + sf_bytes);
+                    tma_load_2d(S.code[s], shared ? &tmS : &tmR, ks * 128, (int)row0, &S.full[s]);
+                    nd_bulk_load(S.sf[s], sfb + (size_t)ks * kNdSfBytes, sf_bytes, &S.full[s]);
+                }
+            }
+            if (!ok) {
+                // let the copies already issued land before the CTA can exit
+                int never = 0;
+                const uint32_t first = it >= kNdStages ? it - kNdStages : 0;
+                for (uint32_t i = first; i < it; ++i)
+                    mbar_wait(&S.full[i % kNdStages], (i / kNdStages) & 1u, &never, status);
+            }
         }
-        const uint4 *gate = reinterpret_cast<const uint4 *>(qb + prow * (d / 2));
-        const uint4 *up = reinterpret_cast<const uint4 *>(qb + (prow + 64) * (d / 2));
-        const long long gt = (long long)(prow >> 7), ut = (long long)((prow + 64) >> 7);
-        const int gm = (int)(prow & 127), um = (int)((prow + 64) & 127);
+        return;
+    }
+    // ---------------- consumers (warps 0..3)
+    const int c = lane & 7, rsub = lane >> 3;
+    uint32_t it = 0;
+    for (int item = blockIdx.x; item < items; item += gridDim.x) {
+        const bool shared = item >= routed_items;
+        const int u = shared ? 0 : item / tpr;
+        const int t = shared ? item - routed_items : item % tpr;
+        const int a0 = shared ? 0 : P.ustart[u];
+        const int na = shared ? T : P.ustart[u + 1] - a0;
+        const float gsw = shared ? gs13s[0] : gs13[P.uniq[u]];
         const uint4 *xr[MAXT];
         const float2 *sr[MAXT];
 #pragma unroll
-        for (int s = 0; s < MAXT; ++s) {
-            const int tok = (s < na) ? (shared ? s : P.list[a0 + s] / k) : 0;
-            xr[s] = reinterpret_cast<const uint4 *>(xh + (size_t)tok * d);
-            sr[s] = reinterpret_cast<const float2 *>(xs + (size_t)tok * (d / 16));
+        for (int q = 0; q < MAXT; ++q) {
+            const int tok = (q < na) ? (shared ? q : P.list[a0 + q] / k) : 0;
+            xr[q] = reinterpret_cast<const uint4 *>(xh + (size_t)tok * d);
+            sr[q] = reinterpret_cast<const float2 *>(xs + (size_t)tok * (d / 16));
         }
-        float ag[MAXT], au[MAXT];
+        float acc[8][MAXT];
 #pragma unroll
-        for (int s = 0; s < MAXT; ++s)
-            ag[s] = au[s] = 0.f;
-        for (int cb = 0; cb < nv; cb += 32 * kDecUnroll) {
-            uint4 wg[kDecUnroll], wu[kDecUnroll];
-            uint32_t sg[kDecUnroll], su[kDecUnroll];
+        for (int j = 0; j < 8; ++j)
 #pragma unroll
-            for (int i = 0; i < kDecUnroll; ++i) {
-                const int ci = cb + lane + 32 * i;
-                if (ci < nv) {
-                    wg[i] = ld_stream_v4(gate + ci);
-                    wu[i] = ld_stream_v4(up + ci);
-                    // blocks 2ci and 2ci + 1: adjacent bytes of one scale word
-                    sg[i] = __ldg(reinterpret_cast<const uint16_t *>(sb + nv_sf_offset(gt, gm, 2 * ci, d)));
-                    su[i] = __ldg(reinterpret_cast<const uint16_t *>(sb + nv_sf_offset(ut, um, 2 * ci, d)));
-                }
-            }
+            for (int q = 0; q < MAXT; ++q)
+                acc[j][q] = 0.f;
+        for (int ks = 0; ks < nks; ++ks, ++it) {
+            const int s = it % kNdStages;
+            const uint32_t ph = (it / kNdStages) & 1u;
+            const bool got = mbar_wait(&S.full[s], ph, abort_flag, status);
+            // chunk c (elements ks * 256 + 32 c ..) lies inside the row
+            if (got && ks * 256 + c * 32 < d) {
+                // x's chunk c of this stage (32 values) and its two block scales
+                uint4 xv[MAXT][4];
+                float2 xsc[MAXT];
 #pragma unroll
-            for (int i = 0; i < kDecUnroll; ++i) {
-                const int ci = cb + lane + 32 * i;
-                if (ci >= nv)
-                    continue;
-                const float g0 = nv_scale_value(sg[i]), g1 = nv_scale_value(sg[i] >> 8);
-                const float u0 = nv_scale_value(su[i]), u1 = nv_scale_value(su[i] >> 8);
+                for (int q = 0; q < MAXT; ++q) {
+                    if (q < na) {
+                        const int x4 = ks * 32 + c * 4;
 #pragma unroll
-                for (int s = 0; s < MAXT; ++s) {
-                    if (s < na) {
-                        // x's 32 values and two scales, loaded once for the gate and up rows
-                        const uint4 xv[4] = {__ldg(xr[s] + 4 * ci), __ldg(xr[s] + 4 * ci + 1),
-                                             __ldg(xr[s] + 4 * ci + 2), __ldg(xr[s] + 4 * ci + 3)};
-                        const float2 xsc = __ldg(sr[s] + ci);
-                        ag[s] += nv_chunk_dot(wg[i], g0, g1, xv, xsc);
-                        au[s] += nv_chunk_dot(wu[i], u0, u1, xv, xsc);
+                        for (int i = 0; i < 4; ++i)
+                            xv[q][i] = __ldg(xr[q] + x4 + i);
+                        xsc[q] = __ldg(sr[q] + ks * 8 + c);
                     }
                 }
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int r = warp * 32 + rsub + 4 * j;
+                    const uint4 w = *reinterpret_cast<const uint4 *>(S.code[s] + r * 128 + c * 16);
+                    // blocks 2c and 2c + 1 of this stage: K group c / 2, row r
+                    const uint32_t sw = *reinterpret_cast<const uint16_t *>(
+                        S.sf[s] + (c >> 1) * 512 + (r & 31) * 16 + (r >> 5) * 4 + 2 * (c & 1));
+                    const float s0 = nv_scale_value(sw), s1 = nv_scale_value(sw >> 8);
+#pragma unroll
+                    for (int q = 0; q < MAXT; ++q)
+                        if (q < na)
+                            acc[j][q] += nv_chunk_dot(w, s0, s1, xv[q], xsc[q]);
+                }
             }
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(&S.empty[s]);
         }
+        // row sums: the eight lanes of a row differ in bits 0..2 of the lane id
         const float inv = 1.0f / (x_gs * gsw);
 #pragma unroll
-        for (int s = 0; s < MAXT; ++s) {
-            if (s < na) {
-                const float g = warp_sum(ag[s]) * inv;
-                const float uu = warp_sum(au[s]) * inv;
-                if (lane == 0) {
-                    const int row = shared ? s : P.list[a0 + s];
-                    hout[(size_t)row * ldh + c] = silu_mul(g, uu);
+        for (int j = 0; j < 8; ++j)
+#pragma unroll
+            for (int q = 0; q < MAXT; ++q) {
+                float v = acc[j][q];
+                v += __shfl_xor_sync(kFullMask, v, 1);
+                v += __shfl_xor_sync(kFullMask, v, 2);
+                v += __shfl_xor_sync(kFullMask, v, 4);
+                if (c == 0)
+                    S.rowsum[warp * 32 + rsub + 4 * j][q] = v * inv;
+            }
+        nd_consumer_sync();
+        // h columns 64 t + i: gate row i, up row 64 + i of the tile
+        if (threadIdx.x < 64) {
+            const int i = threadIdx.x;
+#pragma unroll
+            for (int q = 0; q < MAXT; ++q) {
+                if (q < na) {
+                    const float h = silu_mul(S.rowsum[i][q], S.rowsum[64 + i][q]);
+                    if (shared)
+                        Hs32[(size_t)q * d_ff_s + 64 * t + i] = h;
+                    else
+                        H32[(size_t)P.list[a0 + q] * d_ff + 64 * t + i] = h;
                 }
             }
         }
+        nd_consumer_sync();
     }
 }
 
@@ -991,6 +1073,53 @@ static void launch_pdl(void (*kernel)(KArgs...), int grid, int block, cudaStream
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
+// Raises a kernel's dynamic shared memory limit once per (kernel, device).
+static int smem_attr_once(const void *kernel, size_t smem)
+{
+    constexpr int kMax = 64;
+    static std::mutex mu;
+    static const void *done_k[kMax];
+    static int done_d[kMax];
+    static int n_done = 0;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i = 0; i < n_done; ++i)
+        if (done_k[i] == kernel && done_d[i] == dev)
+            return MOE_OK;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess)
+        return MOE_ERR_CUDA;
+    if (n_done < kMax) {
+        done_k[n_done] = kernel;
+        done_d[n_done] = dev;
+        ++n_done;
+    }
+    return MOE_OK;
+}
+
+// The same, with dynamic shared memory.
+template <typename... KArgs, typename... Args>
+static int launch_pdl_smem(void (*kernel)(KArgs...), int grid, int block, size_t smem,
+                           cudaStream_t st, Args... args)
+{
+    if (const int rc = smem_attr_once(reinterpret_cast<const void *>(kernel), smem))
+        return rc;
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof cfg);
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(block);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaLaunchKernelEx(&cfg, kernel, args...);
+    return MOE_OK;
 }
 
 static int maxt_for(int T) { return T <= 1 ? 1 : T <= 2 ? 2 : T <= 4 ? 4 : T <= 8 ? 8 : 16; }
@@ -1157,17 +1286,34 @@ int launch_dec_w13_nv(const moe_shape_t &s, const uint16_t *xh, const float *xs,
         return MOE_OK;
     if (s.T > 2)
         return MOE_ERR_UNSUPPORTED;
-    const int blocks = num_sms() * 2;
+    // packed code rows of d / 2 bytes, read 128 rows x 128 bytes per K stage
+    CUtensorMap tmR, tmS;
+    int rc = make_tmap_u8_rows(&tmR, W13q, s.d / 2, (long long)s.E * 2 * s.d_ff, 128);
+    if (rc)
+        return rc;
+    const bool shared = s.d_ff_shared > 0 && W13s_q;
+    if (shared) {
+        if ((rc = make_tmap_u8_rows(&tmS, W13s_q, s.d / 2, 2LL * s.d_ff_shared, 128)))
+            return rc;
+    } else {
+        tmS = tmR;
+    }
+    // at most min(E, T k) chosen experts of 2 d_ff / 128 tiles, then the shared expert's
+    const long long items = (long long)std::min(s.E, s.T * s.k) * (2 * s.d_ff / 128) +
+                            (shared ? 2 * s.d_ff_shared / 128 : 0);
+    const int blocks = (int)std::max<long long>(1, std::min<long long>(items, 2LL * num_sms()));
     float *Hs = H32 + (size_t)s.T * s.k * s.d_ff;
-    const uint8_t *wq = s.d_ff_shared ? W13s_q : nullptr;
-    if (s.T == 1)
-        launch_pdl(k_dec_w13_nv<1>, blocks, 256, st, xh, xs, x_gs, topk_idx, s.T, s.d, s.d_ff,
-                   s.E, s.k, s.capacity, slot_major(s), W13q, W13sf, gs13, s.d_ff_shared, wq,
-                   W13s_sf, gs13s, H32, Hs, status);
-    else
-        launch_pdl(k_dec_w13_nv<2>, blocks, 256, st, xh, xs, x_gs, topk_idx, s.T, s.d, s.d_ff,
-                   s.E, s.k, s.capacity, slot_major(s), W13q, W13sf, gs13, s.d_ff_shared, wq,
-                   W13s_sf, gs13s, H32, Hs, status);
+    rc = s.T == 1
+             ? launch_pdl_smem(k_dec_w13_nv<1>, blocks, kNdThreads, sizeof(NdSmem<1>) + 1024, st,
+                               tmR, tmS, xh, xs, x_gs, topk_idx, s.T, s.d, s.d_ff, s.E, s.k,
+                               s.capacity, slot_major(s), W13sf, gs13, s.d_ff_shared,
+                               shared ? 1 : 0, W13s_sf, gs13s, H32, Hs, status)
+             : launch_pdl_smem(k_dec_w13_nv<2>, blocks, kNdThreads, sizeof(NdSmem<2>) + 1024, st,
+                               tmR, tmS, xh, xs, x_gs, topk_idx, s.T, s.d, s.d_ff, s.E, s.k,
+                               s.capacity, slot_major(s), W13sf, gs13, s.d_ff_shared,
+                               shared ? 1 : 0, W13s_sf, gs13s, H32, Hs, status);
+    if (rc)
+        return rc;
     return launched();
 }
 

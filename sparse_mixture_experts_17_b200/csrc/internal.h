@@ -1,6 +1,7 @@
 // internal.h -- host-side interface between the C-ABI layer and the kernels.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -229,6 +230,10 @@ struct GemmArgs {
 
 int launch_gemm_tc(const GemmArgs &g, cudaStream_t st);
 int launch_gemm_mx(const GemmArgs &g, cudaStream_t st);
+// 2-D TMA map of a byte matrix [rows, cols], unswizzled box of 128 bytes x
+// box_rows (gemm_mx.cu). Returns MOE_OK or MOE_ERR_CUDA.
+int make_tmap_u8_rows(CUtensorMap *m, const void *base, long long cols, long long rows,
+                      int box_rows);
 int launch_gemm_simt(const GemmArgs &g, cudaStream_t st);
 int num_sms();
 
