@@ -758,15 +758,17 @@ __device__ __forceinline__ float nv_chunk_dot(const uint4 &w, float sw0, float s
 // streams the tile through a ring of K stages: 128 rows x 128 bytes of codes
 // (256 elements, one TMA box) and the stage's four 512-byte scale atoms (one
 // bulk copy); the copy engine keeps kNdStages stages in flight whatever the
-// consumers' registers. Four consumer warps own 32 rows each: lane l takes
-// the 32-element chunk l % 8 of rows l / 8 + 4 j (j < 8), so one load of x's
+// consumers' registers. Eight consumer warps own 16 rows each: lane l takes
+// the 32-element chunk l % 8 of rows l / 8 + 4 j (j < 4), so one load of x's
 // chunk serves eight rows and each 16-byte code read is conflict-free. At
 // the end of a tile the eight lanes of a row reduce their sums, and the h
 // columns are formed from the gate and up row sums in shared memory.
 constexpr int kNdStages = 4;
 constexpr int kNdStageBytes = 128 * 128;   // codes of one K stage (256 elements x 128 rows)
 constexpr int kNdSfBytes = 4 * 512;        // its four scale atoms
-constexpr int kNdThreads = 160;            // four consumer warps, then the producer warp
+constexpr int kNdConsumers = 8;            // consumer warps (16 rows each)
+constexpr int kNdRowsPerLane = 128 / kNdConsumers / 4;
+constexpr int kNdThreads = 32 * kNdConsumers + 32;   // the consumers, then the producer warp
 
 template <int MAXT>
 struct NdSmem {
@@ -777,6 +779,13 @@ struct NdSmem {
     int abort;
 };
 
+// Bytes of NdSmem<MAXT> rounded up to 16 (x is staged after it).
+template <int MAXT>
+__host__ __device__ constexpr size_t nd_smem_bytes()
+{
+    return (sizeof(NdSmem<MAXT>) + 15) / 16 * 16;
+}
+
 __device__ __forceinline__ void nd_bulk_load(void *smem_dst, const void *src, uint32_t bytes,
                                              uint64_t *bar)
 {
@@ -786,8 +795,11 @@ __device__ __forceinline__ void nd_bulk_load(void *smem_dst, const void *src, ui
         : "memory");
 }
 
-// named barrier of the four consumer warps
-__device__ __forceinline__ void nd_consumer_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+// named barrier of the consumer warps
+__device__ __forceinline__ void nd_consumer_sync()
+{
+    asm volatile("bar.sync 1, %0;" ::"n"(32 * kNdConsumers) : "memory");
+}
 
 template <int MAXT>
 __global__ void __launch_bounds__(kNdThreads, 2)
@@ -807,7 +819,7 @@ __global__ void __launch_bounds__(kNdThreads, 2)
     if (threadIdx.x == 0) {
         for (int s = 0; s < kNdStages; ++s) {
             mbar_init(&S.full[s], 1);
-            mbar_init(&S.empty[s], 4);
+            mbar_init(&S.empty[s], kNdConsumers);
         }
         S.abort = 0;
         fence_mbar_init();
@@ -815,13 +827,23 @@ __global__ void __launch_bounds__(kNdThreads, 2)
     pdl_wait();
     pdl_trigger();
     build_plan(P, idx, T, E, k, C, slot_major, status);   // ends with __syncthreads
+    // x (T rows of f16 values) and its block scales, staged in shared memory
+    // once: every tile reads them again, and global loads there left the
+    // consumers waiting on L2 latency at each stage
+    uint4 *x_sm = reinterpret_cast<uint4 *>(reinterpret_cast<uint8_t *>(&S) + nd_smem_bytes<MAXT>());
+    float *xs_sm = reinterpret_cast<float *>(x_sm + (size_t)T * (d / 8));
+    for (int i = threadIdx.x; i < T * (d / 8); i += blockDim.x)
+        x_sm[i] = __ldg(reinterpret_cast<const uint4 *>(xh) + i);
+    for (int i = threadIdx.x; i < T * (d / 16); i += blockDim.x)
+        xs_sm[i] = __ldg(xs + i);
+    __syncthreads();
     volatile int *abort_flag = &S.abort;
     const int tpr = 2 * d_ff / 128;                        // tiles of a routed expert
     const int routed_items = P.U * tpr;
     const int items = routed_items + (has_shared ? 2 * d_ff_s / 128 : 0);
     const int nks = (d + 255) / 256;   // K stages of a tile; the last holds 128 or 256 elements
 
-    if (warp == 4) {
+    if (warp == kNdConsumers) {
         if (lane == 0) {   // ---------------- producer
             uint32_t it = 0;
             bool ok = true;
@@ -856,7 +878,7 @@ __global__ void __launch_bounds__(kNdThreads, 2)
         }
         return;
     }
-    // ---------------- consumers (warps 0..3)
+    // ---------------- consumers (warps 0 .. kNdConsumers - 1)
     const int c = lane & 7, rsub = lane >> 3;
     uint32_t it = 0;
     for (int item = blockIdx.x; item < items; item += gridDim.x) {
@@ -871,12 +893,12 @@ __global__ void __launch_bounds__(kNdThreads, 2)
 #pragma unroll
         for (int q = 0; q < MAXT; ++q) {
             const int tok = (q < na) ? (shared ? q : P.list[a0 + q] / k) : 0;
-            xr[q] = reinterpret_cast<const uint4 *>(xh + (size_t)tok * d);
-            sr[q] = reinterpret_cast<const float2 *>(xs + (size_t)tok * (d / 16));
+            xr[q] = x_sm + (size_t)tok * (d / 8);
+            sr[q] = reinterpret_cast<const float2 *>(xs_sm + (size_t)tok * (d / 16));
         }
-        float acc[8][MAXT];
+        float acc[kNdRowsPerLane][MAXT];
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
+        for (int j = 0; j < kNdRowsPerLane; ++j)
 #pragma unroll
             for (int q = 0; q < MAXT; ++q)
                 acc[j][q] = 0.f;
@@ -895,13 +917,13 @@ __global__ void __launch_bounds__(kNdThreads, 2)
                         const int x4 = ks * 32 + c * 4;
 #pragma unroll
                         for (int i = 0; i < 4; ++i)
-                            xv[q][i] = __ldg(xr[q] + x4 + i);
-                        xsc[q] = __ldg(sr[q] + ks * 8 + c);
+                            xv[q][i] = xr[q][x4 + i];
+                        xsc[q] = sr[q][ks * 8 + c];
                     }
                 }
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const int r = warp * 32 + rsub + 4 * j;
+                for (int j = 0; j < kNdRowsPerLane; ++j) {
+                    const int r = warp * (4 * kNdRowsPerLane) + rsub + 4 * j;
                     const uint4 w = *reinterpret_cast<const uint4 *>(S.code[s] + r * 128 + c * 16);
                     // blocks 2c and 2c + 1 of this stage: K group c / 2, row r
                     const uint32_t sw = *reinterpret_cast<const uint16_t *>(
@@ -920,7 +942,7 @@ __global__ void __launch_bounds__(kNdThreads, 2)
         // row sums: the eight lanes of a row differ in bits 0..2 of the lane id
         const float inv = 1.0f / (x_gs * gsw);
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
+        for (int j = 0; j < kNdRowsPerLane; ++j)
 #pragma unroll
             for (int q = 0; q < MAXT; ++q) {
                 float v = acc[j][q];
@@ -928,7 +950,7 @@ __global__ void __launch_bounds__(kNdThreads, 2)
                 v += __shfl_xor_sync(kFullMask, v, 2);
                 v += __shfl_xor_sync(kFullMask, v, 4);
                 if (c == 0)
-                    S.rowsum[warp * 32 + rsub + 4 * j][q] = v * inv;
+                    S.rowsum[warp * (4 * kNdRowsPerLane) + rsub + 4 * j][q] = v * inv;
             }
         nd_consumer_sync();
         // h columns 64 t + i: gate row i, up row 64 + i of the tile
@@ -1075,7 +1097,8 @@ static void launch_pdl(void (*kernel)(KArgs...), int grid, int block, cudaStream
     cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
-// Raises a kernel's dynamic shared memory limit once per (kernel, device).
+// Raises a kernel's dynamic shared memory limit to the device's opt-in
+// maximum once per (kernel, device); fails if `smem` exceeds it.
 static int smem_attr_once(const void *kernel, size_t smem)
 {
     constexpr int kMax = 64;
@@ -1089,8 +1112,16 @@ static int smem_attr_once(const void *kernel, size_t smem)
     for (int i = 0; i < n_done; ++i)
         if (done_k[i] == kernel && done_d[i] == dev)
             return MOE_OK;
-    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-        cudaSuccess)
+    // the device's opt-in maximum less the kernel's static shared memory, so
+    // that every later size fits as well
+    int optin = 0;
+    cudaFuncAttributes fa;
+    if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess ||
+        cudaFuncGetAttributes(&fa, kernel) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    const int dyn_max = optin - (int)fa.sharedSizeBytes;
+    if (dyn_max < (int)smem ||
+        cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn_max) != cudaSuccess)
         return MOE_ERR_CUDA;
     if (n_done < kMax) {
         done_k[n_done] = kernel;
@@ -1303,12 +1334,14 @@ int launch_dec_w13_nv(const moe_shape_t &s, const uint16_t *xh, const float *xs,
                             (shared ? 2 * s.d_ff_shared / 128 : 0);
     const int blocks = (int)std::max<long long>(1, std::min<long long>(items, 2LL * num_sms()));
     float *Hs = H32 + (size_t)s.T * s.k * s.d_ff;
+    // x staged in shared memory: T rows of d f16 values and d / 16 fp32 scales
+    const size_t xbytes = (size_t)s.T * s.d * 2 + (size_t)s.T * (s.d / 16) * 4;
     rc = s.T == 1
-             ? launch_pdl_smem(k_dec_w13_nv<1>, blocks, kNdThreads, sizeof(NdSmem<1>) + 1024, st,
+             ? launch_pdl_smem(k_dec_w13_nv<1>, blocks, kNdThreads, nd_smem_bytes<1>() + 1024 + xbytes, st,
                                tmR, tmS, xh, xs, x_gs, topk_idx, s.T, s.d, s.d_ff, s.E, s.k,
                                s.capacity, slot_major(s), W13sf, gs13, s.d_ff_shared,
                                shared ? 1 : 0, W13s_sf, gs13s, H32, Hs, status)
-             : launch_pdl_smem(k_dec_w13_nv<2>, blocks, kNdThreads, sizeof(NdSmem<2>) + 1024, st,
+             : launch_pdl_smem(k_dec_w13_nv<2>, blocks, kNdThreads, nd_smem_bytes<2>() + 1024 + xbytes, st,
                                tmR, tmS, xh, xs, x_gs, topk_idx, s.T, s.d, s.d_ff, s.E, s.k,
                                s.capacity, slot_major(s), W13sf, gs13, s.d_ff_shared,
                                shared ? 1 : 0, W13s_sf, gs13s, H32, Hs, status);
