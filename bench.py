@@ -459,13 +459,16 @@ def run_ours(a, world, rank, local):
         idx_now = torch.empty(w.T, w.k, dtype=torch.int32, device=dev)
         layer.forward(x, out=out, topk_idx_out=idx_now)
         U, nbytes, w13_bytes, expert_bytes = decode_bytes(w, w.T, idx_now)
-        if a.mxfp8:   # a code byte and 1/32 of a scale byte per weight instead of 2 bytes
-            mx = (1.0 + 1.0 / 32.0) / 2.0
+        if a.mxfp8 or a.nvfp4:
+            # bytes per weight instead of 2: a code byte and 1/32 of a scale
+            # byte (MXFP8), or half a code byte and 1/16 of a scale byte (NVFP4)
+            mx = ((1.0 + 1.0 / 32.0) if a.mxfp8 else (0.5 + 1.0 / 16.0)) / 2.0
             nbytes = int(nbytes - expert_bytes * (1.0 - mx))
             w13_bytes, expert_bytes = int(w13_bytes * mx), int(expert_bytes * mx)
         k13 = stages["dec_w13"][0] / stages["dec_w13"][1]
         ach = w13_bytes / (k13 / 1e3) / 1e9
-        roofline = {"bound": "hbm", "kernel": "k_dec_w13 (chosen experts' w1/w3 rows + SwiGLU)",
+        dec_kernel = "k_dec_w13_mx" if a.mxfp8 else "k_dec_w13_nv" if a.nvfp4 else "k_dec_w13"
+        roofline = {"bound": "hbm", "kernel": f"{dec_kernel} (chosen experts' w1/w3 rows + SwiGLU)",
                     "achieved": round(ach, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                     "frac": round(ach / peaks["hbm_gbs"], 4), "traffic": None,
                     "peak_source": f"{peak_src} hbm_gbs",
