@@ -100,14 +100,18 @@ struct MxCfg {
     static constexpr int BK = FMT == FMT_NV4 ? 256 : 128; // ... = 256 E2M1 or 128 E4M3 elements
     static constexpr int A_BYTES = BM * BK_BYTES;
     static constexpr int B_BYTES = BN * BK_BYTES;
-    static constexpr int SF_ATOMS = FMT == FMT_NV4 ? 4 : 1;   // 512-byte scale atoms per stage
-    static constexpr int SF_BYTES = 512 * SF_ATOMS;       // per operand per stage
-    static constexpr int STAGES = 6;
+    static constexpr int SF_ATOMS = FMT == FMT_NV4 ? 4 : 1;   // K groups (512-byte atoms) per stage
+    // per stage: B's scale atoms; A's scales in the activation layout for
+    // NVFP4 (two 4 KB tcgen05.cp 128x256b sources, nvfp4.cuh), else atoms
+    static constexpr int SFB_BYTES = 512 * SF_ATOMS;
+    static constexpr int SFA_BYTES = FMT == FMT_NV4 ? 8192 : 512;
+    static constexpr int SF_STAGE_BYTES = SFA_BYTES + SFB_BYTES;
+    static constexpr int STAGES = FMT == FMT_NV4 ? 5 : 6;
     static constexpr int TMEM_COLS = 512;
     static constexpr int SF_COL = 2 * BN;                 // scale columns after the accumulators
-    static constexpr int SF_COLS_PER_STAGE = 8 * SF_ATOMS; // 4 per atom, A's then B's
+    static constexpr int SF_COLS_PER_STAGE = 8 * SF_ATOMS; // 4 per K group, A's then B's
     static constexpr int SMEM_BYTES =
-        1024 + STAGES * (A_BYTES + B_BYTES) + STAGES * 2 * SF_BYTES + 256;
+        1024 + STAGES * (A_BYTES + B_BYTES) + STAGES * SF_STAGE_BYTES + 256;
     static_assert(SF_COL + STAGES * SF_COLS_PER_STAGE <= TMEM_COLS,
                   "accumulators and per-stage scale columns must fit the TMEM allocation");
     static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
@@ -168,6 +172,27 @@ __device__ __forceinline__ uint32_t idesc_nv4()
     return (1u << 7) | (1u << 10)            // A and B: E2M1
            | ((uint32_t)(128 >> 3) << 17)    // N = 128
            | ((uint32_t)(128 >> 4) << 24);   // M = 128
+}
+
+// Shared-memory descriptor of one 4 KB activation-scale copy source
+// (nvfp4.cuh nv_sfa_offset): 128 lane rows of two 16-byte chunks, the first
+// chunks of all rows (2 KB) before the second ones; no swizzle, 8-row core
+// matrices 128 bytes apart, the two chunk columns 2 KB apart.
+__device__ __forceinline__ uint64_t smem_desc_sfa(uint32_t smem_addr)
+{
+    uint64_t d = 0;
+    d |= (uint64_t)((smem_addr & 0x3FFFFu) >> 4);
+    d |= (uint64_t)(2048u >> 4) << 16;   // leading byte offset: the second 16-byte chunk
+    d |= (uint64_t)(128u >> 4) << 32;    // stride byte offset: next 8 rows
+    d |= (uint64_t)1 << 46;              // descriptor version
+    return d;                            // layout type 0: no swizzle
+}
+
+// 128 lanes x 256 bits (eight TMEM columns) from a shared-memory source, no
+// replication over the lane quarters.
+__device__ __forceinline__ void tc_cp_sf_128x256(uint32_t taddr, uint64_t desc)
+{
+    asm volatile("tcgen05.cp.cta_group::1.128x256b [%0], %1;" ::"r"(taddr), "l"(desc) : "memory");
 }
 
 __device__ __forceinline__ void tc_cp_sf(uint32_t taddr, uint64_t desc)
@@ -236,7 +261,7 @@ __device__ __forceinline__ void mx_epilogue(const MxArgs &p, uint32_t tb, long l
                 *reinterpret_cast<uint4 *>(hq + c * 16) = make_uint4(q0.x, q0.y, q1.x, q1.y);
                 // blocks 4 n_idx + 2c and + 1: adjacent bytes of one atom word
                 *reinterpret_cast<uint16_t *>(p.out_sf +
-                                              nv_sf_offset(m_idx, m, 4 * n_idx + 2 * c, (int)p.ldo)) =
+                                              nv_sfa_offset(m_idx, m, 4 * n_idx + 2 * c, (int)p.ldo)) =
                     (uint16_t)(s0 | (s1 << 8));
             }
         }
@@ -320,7 +345,7 @@ __global__ void __launch_bounds__(192, 1)
     uint8_t *sA = smem;
     uint8_t *sB = sA + C::STAGES * C::A_BYTES;
     uint8_t *sSF = sB + C::STAGES * C::B_BYTES;   // per stage: A's scale atoms, then B's
-    uint64_t *full = reinterpret_cast<uint64_t *>(sSF + C::STAGES * 2 * C::SF_BYTES);
+    uint64_t *full = reinterpret_cast<uint64_t *>(sSF + C::STAGES * C::SF_STAGE_BYTES);
     uint64_t *empty = full + C::STAGES;
     uint64_t *tfull = empty + C::STAGES;
     uint64_t *tempty = tfull + 2;
@@ -366,9 +391,9 @@ __global__ void __launch_bounds__(192, 1)
                 const long long row0 = p.mt_row0 ? p.mt_row0[m_idx] : (long long)m_idx * C::BM;
                 const int grp = p.mt_group ? (p.mt_group[m_idx] & ~kHalfTileBit) : 0;
                 const long long brow = (long long)grp * p.b_rows_per_group + (long long)n_idx * C::BN;
-                // a 128-row band's atoms: kblocks stages of SF_BYTES each
-                const uint8_t *sfa = p.A_sf + (long long)m_idx * p.kblocks * C::SF_BYTES;
-                const uint8_t *sfb = p.B_sf + (brow >> 7) * p.kblocks * C::SF_BYTES;
+                // a 128-row band's scales: kblocks stages of SFA / SFB bytes each
+                const uint8_t *sfa = p.A_sf + (long long)m_idx * p.kblocks * C::SFA_BYTES;
+                const uint8_t *sfb = p.B_sf + (brow >> 7) * p.kblocks * C::SFB_BYTES;
                 for (int kb = 0; kb < p.kblocks; ++kb, ++it) {
                     const int s = it % C::STAGES;
                     const uint32_t ph = (it / C::STAGES) & 1u;
@@ -376,12 +401,12 @@ __global__ void __launch_bounds__(192, 1)
                         ok = false;
                         break;
                     }
-                    uint8_t *sf = sSF + s * 2 * C::SF_BYTES;
-                    mbar_arrive_expect_tx(&full[s], C::A_BYTES + C::B_BYTES + 2 * C::SF_BYTES);
+                    uint8_t *sf = sSF + s * C::SF_STAGE_BYTES;
+                    mbar_arrive_expect_tx(&full[s], C::A_BYTES + C::B_BYTES + C::SF_STAGE_BYTES);
                     tma_load_2d(sA + s * C::A_BYTES, &tmA, kb * C::BK_BYTES, (int)row0, &full[s]);
                     tma_load_2d(sB + s * C::B_BYTES, &tmB, kb * C::BK_BYTES, (int)brow, &full[s]);
-                    bulk_load(sf, sfa + (long long)kb * C::SF_BYTES, C::SF_BYTES, &full[s]);
-                    bulk_load(sf + C::SF_BYTES, sfb + (long long)kb * C::SF_BYTES, C::SF_BYTES,
+                    bulk_load(sf, sfa + (long long)kb * C::SFA_BYTES, C::SFA_BYTES, &full[s]);
+                    bulk_load(sf + C::SFA_BYTES, sfb + (long long)kb * C::SFB_BYTES, C::SFB_BYTES,
                               &full[s]);
                 }
             }
@@ -404,16 +429,24 @@ __global__ void __launch_bounds__(192, 1)
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t sf0 = smem_u32(sSF + s * 2 * C::SF_BYTES);
+                    const uint32_t sf0 = smem_u32(sSF + s * C::SF_STAGE_BYTES);
                     // each stage has its own scale columns: the copy for this
                     // stage never overwrites columns that earlier MMAs still read
                     const uint32_t sf_a = tmem_base + C::SF_COL + s * C::SF_COLS_PER_STAGE;
                     const uint32_t sf_b = sf_a + 4 * C::SF_ATOMS;
+                    if constexpr (FMT == FMT_NV4) {
+                        // A: two 128x256b copies, K groups 2h and 2h + 1 in the
+                        // 4-column slots sf_a + 8h and sf_a + 8h + 4 (each lane
+                        // quarter reads its own column of a slot)
 #pragma unroll
-                    for (int i = 0; i < C::SF_ATOMS; ++i) {
-                        tc_cp_sf(sf_a + 4 * i, smem_desc_sf(sf0 + 512 * i));
-                        tc_cp_sf(sf_b + 4 * i, smem_desc_sf(sf0 + C::SF_BYTES + 512 * i));
+                        for (int h = 0; h < 2; ++h)
+                            tc_cp_sf_128x256(sf_a + 8 * h, smem_desc_sfa(sf0 + 4096 * h));
+                    } else {
+                        tc_cp_sf(sf_a, smem_desc_sf(sf0));
                     }
+#pragma unroll
+                    for (int i = 0; i < C::SF_ATOMS; ++i)
+                        tc_cp_sf(sf_b + 4 * i, smem_desc_sf(sf0 + C::SFA_BYTES + 512 * i));
                     const uint32_t a0 = smem_u32(sA + s * C::A_BYTES);
                     const uint32_t b0 = smem_u32(sB + s * C::B_BYTES);
                     // four MMAs of 32 bytes of K each (K = 32 E4M3 or 64 E2M1)

@@ -265,9 +265,11 @@ int launch_mx_gather(const moe_shape_t &s, const uint16_t *x, const int32_t *idx
 int launch_nv_weight_scales(const moe_shape_t &s, const uint16_t *W1, const uint16_t *W3,
                             const uint16_t *W2, float *gs13, float *gs2, cudaStream_t st);
 // rows of a bf16 matrix; global scale gs_arr[row / rows_per_gs], or gs_const
+// a_layout: scales in the activation layout (nv_sfa_offset, an A operand)
+// instead of the weights' atom layout.
 int launch_nv_quantize_rows(const uint16_t *src, long long rows, int K, const float *gs_arr,
                             long long rows_per_gs, float gs_const, uint8_t *codes,
-                            uint8_t *scales, cudaStream_t st);
+                            uint8_t *scales, cudaStream_t st, bool a_layout = false);
 int launch_nv_pack_w13(const moe_shape_t &s, const uint16_t *W1, const uint16_t *W3,
                        const float *gs13, uint8_t *codes, uint8_t *scales, cudaStream_t st);
 int launch_nv_gather(const moe_shape_t &s, const uint16_t *x, const int32_t *idx,

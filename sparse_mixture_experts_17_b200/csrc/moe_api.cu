@@ -149,12 +149,13 @@ WsLayout ws_layout(const moe_shape_t &s)
     L.dec_H32 = take(lowp ? (Td * k * s.d_ff + Td * dfs) * 4 : 0);
     L.dec_xs = take(nv ? Td * (s.d / 16) * 4 : 0);
     L.dec_hs = take(nv ? (Td * k * s.d_ff + Td * dfs) / 16 * 4 : 0);
-    // scales in the atom layout: routed operands keyed by m-tile (at most
-    // max_mt tiles of 128 rows), shared-expert operands by row / 128; NVFP4
-    // has twice the scales (16-element blocks) and half the code bytes
+    // activation scales: routed operands keyed by m-tile (at most max_mt
+    // tiles of 128 rows), shared-expert operands by row / 128; MXFP8 in the
+    // atom layout, NVFP4 (16-element blocks) in the activation layout of
+    // nvfp4.cuh (8 KB per tile and 256-element K stage)
     const size_t mt_rows = (size_t)L.max_mt * 128;
     auto sf_bytes = [&](size_t rows, size_t K) {
-        return (size_t)(nv ? nv_sf_bytes((long long)rows, (int)K) : sf_atom_bytes((long long)rows, (int)K));
+        return (size_t)(nv ? nv_sfa_bytes((long long)rows, (int)K) : sf_atom_bytes((long long)rows, (int)K));
     };
     L.xq = take(lowp ? N * s.d : 0);
     L.xsf = take(lowp ? sf_bytes(mt_rows, s.d) : 0);
@@ -697,7 +698,8 @@ static int shared_expert_mx(const moe_shape_t &s, const WsLayout &L, void *ws, c
 {
     const int dfs = s.d_ff_shared;
     int rc = lw.fmt == FMT_NV4 ? launch_nv_quantize_rows(x, s.T, s.d, nullptr, 0, lw.x_gs,
-                                                   at<uint8_t>(ws, L.xq_s), at<uint8_t>(ws, L.xsf_s), st)
+                                                   at<uint8_t>(ws, L.xq_s), at<uint8_t>(ws, L.xsf_s), st,
+                                                   true)
                          : launch_mx_quantize_rows(x, s.T, s.d, at<uint8_t>(ws, L.xq_s),
                                                    at<uint8_t>(ws, L.xsf_s), st);
     if (rc)

@@ -7,6 +7,7 @@
 //                       atomicMax; several tensors may share one maximum
 //   k_nv_gs_finalize    max -> global encode scale 448 * 6 / max (1 for 0)
 //   k_nv_quantize_rows  bf16 [rows, K] -> codes + scales in the atom layout
+//                       (weights) or the activation layout (nv_sfa_offset)
 //                       (tile = row / 128); the global scale per group of
 //                       rows, or one constant
 //   k_nv_pack_w13       W1, W3 [E, d_ff, d] -> the packed gate/up operand of
@@ -84,7 +85,8 @@ __global__ void __launch_bounds__(256) k_nv_quantize_rows(const uint16_t *__rest
                                                           const float *__restrict__ gs_arr,
                                                           long long rows_per_gs, float gs_const,
                                                           uint8_t *__restrict__ codes,
-                                                          uint8_t *__restrict__ scales)
+                                                          uint8_t *__restrict__ scales,
+                                                          int a_layout)
 {
     const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= nblocks)
@@ -96,7 +98,9 @@ __global__ void __launch_bounds__(256) k_nv_quantize_rows(const uint16_t *__rest
     load_bf16x16(src + i * kNvBlock, v);
     const float gs = gs_arr ? gs_arr[row / rows_per_gs] : gs_const;
     uint2 q;
-    scales[nv_sf_offset(row >> 7, (int)(row & 127), b, K)] = nv_quantize16(v, gs, q);
+    const long long off = a_layout ? nv_sfa_offset(row >> 7, (int)(row & 127), b, K)
+                                   : nv_sf_offset(row >> 7, (int)(row & 127), b, K);
+    scales[off] = nv_quantize16(v, gs, q);
     reinterpret_cast<uint2 *>(codes)[i] = q;
 }
 
@@ -211,7 +215,7 @@ __global__ void __launch_bounds__(256) k_nv_gather(const uint16_t *__restrict__ 
         for (int j = 0; j < MOE_MAX_K; ++j) {
             if (j < k && pos[j] >= 0) {
                 reinterpret_cast<uint2 *>(xq + (size_t)pos[j] * (d / 2))[b] = q;
-                xsf[nv_sf_offset(tl[j], rw[j], b, d)] = sc;
+                xsf[nv_sfa_offset(tl[j], rw[j], b, d)] = sc;
             }
         }
     }
@@ -251,13 +255,14 @@ int launch_nv_weight_scales(const moe_shape_t &s, const uint16_t *W1, const uint
 
 int launch_nv_quantize_rows(const uint16_t *src, long long rows, int K, const float *gs_arr,
                             long long rows_per_gs, float gs_const, uint8_t *codes,
-                            uint8_t *scales, cudaStream_t st)
+                            uint8_t *scales, cudaStream_t st, bool a_layout)
 {
     const long long nblocks = rows * (K / kNvBlock);
     if (nblocks <= 0)
         return MOE_OK;
     k_nv_quantize_rows<<<(unsigned)((nblocks + 255) / 256), 256, 0, st>>>(
-        src, nblocks, K, gs_arr, rows_per_gs > 0 ? rows_per_gs : 1, gs_const, codes, scales);
+        src, nblocks, K, gs_arr, rows_per_gs > 0 ? rows_per_gs : 1, gs_const, codes, scales,
+        a_layout ? 1 : 0);
     return launched();
 }
 

@@ -94,4 +94,26 @@ __host__ __device__ __forceinline__ long long nv_sf_bytes(long long rows, int K)
     return (rows + 127) / 128 * (K / 64) * 512;
 }
 
+// Activation (A operand) scales of the block-scaled GEMM in the layout one
+// tcgen05.cp 128x256b copy per two K groups serves: the MMA's lane quarter q
+// (rows 32 q .. 32 q + 31) reads column slot + q of a K group's 4-column
+// slot, so row m needs its four block scales only at bytes 4 q .. 4 q + 3 of
+// that slot's 16-byte lane chunk, and no replication over the quarters.
+// Per 128-row tile and 256-element K stage an 8 KB region: two 4 KB copy
+// sources (K groups 0-1 and 2-3 of the stage), each two 2 KB chunks (the
+// first and the second K group), each 128 lane rows of 16 bytes. The other
+// 12 bytes of a lane row are never read.
+__host__ __device__ __forceinline__ long long nv_sfa_offset(long long tile, int m, int b, int K)
+{
+    const int stage = b >> 4, g = (b >> 2) & 3;   // K stage (16 blocks), K group within it
+    return (tile * ((K + 255) / 256) + stage) * 8192 + (g >> 1) * 4096 + (g & 1) * 2048 + m * 16 +
+           (m >> 5) * 4 + (b & 3);
+}
+
+// Bytes of an activation scale buffer in that layout (rows padded to 128).
+__host__ __device__ __forceinline__ long long nv_sfa_bytes(long long rows, int K)
+{
+    return (rows + 127) / 128 * ((K + 255) / 256) * 8192;
+}
+
 } // namespace moe
