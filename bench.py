@@ -175,7 +175,7 @@ TRAFFIC_SOURCES = ["sparse_mixture_experts_17_b200/csrc/gemm_tc.cu",
                    "sparse_mixture_experts_17_b200/csrc/tiles.cuh",
                    "sparse_mixture_experts_17_b200/csrc/moe_api.cu"]
 TRAFFIC = {
-    "prefill": {"bytes": 2310400256 + 929892608, "sources_sha": "a1ab63d7980847a7",
+    "prefill": {"bytes": 3930873344 + 929801728, "sources_sha": "7efe44fd561229b7",
                 "profile": "profiles/gemm_w13_traffic_mixtral_t16384.md"},
 }
 
