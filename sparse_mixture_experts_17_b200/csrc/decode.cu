@@ -1075,6 +1075,269 @@ __global__ void __launch_bounds__(256, 2)
     }
 }
 
+// ---------------------------------------------------------------- NVFP4 decode w1/w3, tensor cores
+// NVFP4 decode w1/w3 on the tensor cores: the chosen experts'
+// weights are the M side of block-scaled MMAs (128 packed W13 rows per tile)
+// and the tokens the N side (16 columns, rows past T read as zeros), so the
+// 4-bit codes are multiplied where they land in shared memory and no CUDA
+// core converts them. Work item = one 128-row tile of a chosen expert's
+// packed W13 (64 gate and 64 up rows: h columns 64 t .. 64 t + 63), or of
+// the shared expert after them.
+//
+// Structure (one CTA per SM, 192 threads), as the block-scaled GEMM:
+//   warp 0     producer: per 256-element K stage, TMA of the 128 x 128-byte
+//              weight tile and the 16 x 128-byte token tile (128-byte
+//              swizzle) and bulk copies of both operands' four scale atoms
+//   warp 1     TMEM (two 16-column accumulators, then the stages' scale
+//              columns); one thread copies the scale atoms into TMEM
+//              (32x128b.warpx4) and issues four M=128 N=16 K=64
+//              kind::mxf4nvf4 MMAs per stage
+//   warps 2-5  epilogue: the tile's 128 x 16 sums to shared memory, then
+//              h[a, c] = silu(gate) * up for each assignment a of the tile's
+//              expert, scaled by 1 / (gs_x gs_w), in fp32 (as the CUDA-core
+//              decode kernel writes it for the w2 phase)
+// Every pipeline wait is bounded (mbar_wait); on expiry the roles unwind.
+namespace {
+
+constexpr int kDtStages = 6;
+constexpr int kDtN = 16;                  // token columns of an MMA
+constexpr int kDtABytes = 128 * 128;      // weight codes of one K stage (256 elements x 128 rows)
+constexpr int kDtBBytes = kDtN * 128;     // token codes of one K stage
+constexpr int kDtSfBytes = 2048;          // four scale atoms per operand and stage
+constexpr int kDtSfCols = 32;             // TMEM scale columns per stage (A's 16, then B's)
+constexpr int kDtTmemCols = 256;          // 2 x 16 accumulator columns, then 6 x 32 scale columns
+
+struct DtSmem {
+    uint8_t a[kDtStages][kDtABytes];      // 1024-aligned: 128-byte swizzle atoms
+    uint8_t b[kDtStages][kDtBBytes];
+    uint8_t sfa[kDtStages][kDtSfBytes];
+    uint8_t sfb[kDtStages][kDtSfBytes];
+    float d[128][kDtN + 1];               // one tile's sums (the gate / up pairing)
+    uint64_t full[kDtStages], empty[kDtStages], tfull[2], tempty[2];
+    uint32_t tmem_slot;
+    int abort;
+};
+
+__device__ __forceinline__ uint64_t dt_desc_atom(uint32_t smem_addr)
+{
+    uint64_t d = 0;   // one 32-row x 16-byte scale atom: no swizzle, 8-row core matrices
+    d |= (uint64_t)((smem_addr & 0x3FFFFu) >> 4);
+    d |= (uint64_t)(16u >> 4) << 16;
+    d |= (uint64_t)(128u >> 4) << 32;
+    d |= (uint64_t)1 << 46;
+    return d;
+}
+
+__device__ __forceinline__ void dt_cp_atom(uint32_t taddr, uint64_t desc)
+{
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(desc)
+                 : "memory");
+}
+
+// kind::mxf4nvf4 with 16-element E4M3 scales, E2M1 A and B, M = 128, N = 16
+constexpr uint32_t kDtIdesc =
+    (1u << 7) | (1u << 10) | ((uint32_t)(kDtN >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+
+__device__ __forceinline__ void dt_mma(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                       uint32_t sfa, uint32_t sfb, uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(kDtIdesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+        : "memory");
+}
+
+__device__ __forceinline__ void dt_bulk_load(void *smem_dst, const void *src, uint32_t bytes,
+                                             uint64_t *bar)
+{
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        ::"r"(smem_u32(smem_dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// 16 consecutive fp32 columns of this thread's TMEM lane (32x32b shape).
+__device__ __forceinline__ void dt_tmem_ld16(uint32_t taddr, float (&v)[16])
+{
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+        v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void dt_epi_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+} // namespace
+
+__global__ void __launch_bounds__(192, 1)
+    k_dec_w13_nvtc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmAs,
+                   const __grid_constant__ CUtensorMap tmB, float x_gs,
+                   const int32_t *__restrict__ idx, int T, int d, int d_ff, int E, int k, int C,
+                   int slot_major, const uint8_t *__restrict__ W13sf,
+                   const float *__restrict__ gs13, int d_ff_s, int has_shared,
+                   const uint8_t *__restrict__ W13s_sf, const float *__restrict__ gs13s,
+                   const uint8_t *__restrict__ xsf, float *__restrict__ H32,
+                   float *__restrict__ Hs32, uint32_t *status)
+{
+    extern __shared__ uint8_t dt_raw[];
+    DtSmem &S = *reinterpret_cast<DtSmem *>(
+        (reinterpret_cast<uintptr_t>(dt_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    __shared__ DecPlanSmem P;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kDtStages; ++s) {
+            mbar_init(&S.full[s], 1);
+            mbar_init(&S.empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&S.tfull[b], 1);
+            mbar_init(&S.tempty[b], 4);
+        }
+        S.abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB);
+    }
+    if (warp == 1) {
+        tmem_alloc(&S.tmem_slot, kDtTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = S.tmem_slot;
+    pdl_wait();
+    pdl_trigger();
+    build_plan(P, idx, T, E, k, C, slot_major, status);   // ends with __syncthreads
+    volatile int *abort_flag = &S.abort;
+    const int tpr = 2 * d_ff / 128;                        // tiles of a routed expert
+    const int routed_items = P.U * tpr;
+    const int items = routed_items + (has_shared ? 2 * d_ff_s / 128 : 0);
+    const int nks = d / 256;                               // K stages of a tile
+
+    if (warp == 0) {
+        if (lane == 0) {   // ---------------- producer
+            uint32_t it = 0;
+            bool ok = true;
+            for (int item = blockIdx.x; ok && item < items; item += gridDim.x) {
+                const bool shared = item >= routed_items;
+                const int t = shared ? item - routed_items : item % tpr;
+                const long long row0 =
+                    shared ? (long long)t * 128 : (long long)P.uniq[item / tpr] * 2 * d_ff + t * 128;
+                const uint8_t *sfa = (shared ? W13s_sf : W13sf) + (size_t)(row0 / 128) * (d / 64) * 512;
+                for (int kb = 0; kb < nks; ++kb, ++it) {
+                    const int s = it % kDtStages;
+                    const uint32_t ph = (it / kDtStages) & 1u;
+                    if (!mbar_wait(&S.empty[s], ph ^ 1u, abort_flag, status)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&S.full[s], kDtABytes + kDtBBytes + 2 * kDtSfBytes);
+                    tma_load_2d(S.a[s], shared ? &tmAs : &tmA, kb * 128, (int)row0, &S.full[s]);
+                    tma_load_2d(S.b[s], &tmB, kb * 128, 0, &S.full[s]);
+                    dt_bulk_load(S.sfa[s], sfa + (size_t)kb * kDtSfBytes, kDtSfBytes, &S.full[s]);
+                    dt_bulk_load(S.sfb[s], xsf + (size_t)kb * kDtSfBytes, kDtSfBytes, &S.full[s]);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {   // ---------------- MMA issuer
+            uint32_t it = 0, local = 0;
+            for (int item = blockIdx.x; item < items; item += gridDim.x, ++local) {
+                const uint32_t b = local & 1u, aph = (local >> 1) & 1u;
+                if (!mbar_wait(&S.tempty[b], aph ^ 1u, abort_flag, status))
+                    break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + b * kDtN;
+                bool ok = true;
+                for (int kb = 0; kb < nks; ++kb, ++it) {
+                    const int s = it % kDtStages;
+                    const uint32_t ph = (it / kDtStages) & 1u;
+                    if (!mbar_wait(&S.full[s], ph, abort_flag, status)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    // each stage has its own scale columns after the accumulators
+                    const uint32_t sf_a = tmem_base + 2 * kDtN + s * kDtSfCols;
+                    const uint32_t sf_b = sf_a + 16;
+#pragma unroll
+                    for (int g = 0; g < 4; ++g) {
+                        dt_cp_atom(sf_a + 4 * g, dt_desc_atom(smem_u32(S.sfa[s]) + 512 * g));
+                        dt_cp_atom(sf_b + 4 * g, dt_desc_atom(smem_u32(S.sfb[s]) + 512 * g));
+                    }
+                    const uint32_t a0 = smem_u32(S.a[s]), b0 = smem_u32(S.b[s]);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        dt_mma(d_tmem, smem_desc_k128(a0 + kk * 32), smem_desc_k128(b0 + kk * 32),
+                               sf_a + 4 * kk, sf_b + 4 * kk, (kb | kk) != 0);
+                    tc_commit(&S.empty[s]);
+                }
+                if (!ok)
+                    break;
+                tc_commit(&S.tfull[b]);
+            }
+        }
+    } else {   // ---------------- epilogue warps 2..5
+        const int q = warp & 3;   // TMEM lane quarter this warp may access
+        const int et = threadIdx.x - 64;   // 0..127
+        uint32_t local = 0;
+        for (int item = blockIdx.x; item < items; item += gridDim.x, ++local) {
+            const uint32_t b = local & 1u, aph = (local >> 1) & 1u;
+            const bool got = mbar_wait(&S.tfull[b], aph, abort_flag, status);
+            tc_fence_after();
+            if (got) {
+                float v[16];
+                dt_tmem_ld16(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + b * kDtN, v);
+                tmem_ld_wait();
+#pragma unroll
+                for (int i = 0; i < kDtN; ++i)
+                    S.d[q * 32 + lane][i] = v[i];
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(&S.tempty[b]);
+            dt_epi_sync();
+            if (got && et < 64) {
+                const bool shared = item >= routed_items;
+                const int u = shared ? 0 : item / tpr;
+                const int t = shared ? item - routed_items : item % tpr;
+                const int a0 = shared ? 0 : P.ustart[u];
+                const int na = shared ? T : P.ustart[u + 1] - a0;
+                const float inv = 1.0f / (x_gs * (shared ? gs13s[0] : gs13[P.uniq[u]]));
+                for (int qa = 0; qa < na; ++qa) {
+                    const int a = shared ? qa : P.list[a0 + qa];
+                    const int tok = shared ? qa : a / k;
+                    const float h = silu_mul(S.d[et][tok] * inv, S.d[64 + et][tok] * inv);
+                    if (shared)
+                        Hs32[(size_t)qa * d_ff_s + 64 * t + et] = h;
+                    else
+                        H32[(size_t)a * d_ff + 64 * t + et] = h;
+                }
+            }
+            dt_epi_sync();
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, kDtTmemCols);
+    }
+}
+
 // ---------------------------------------------------------------- host side
 
 // Launch with programmatic stream serialization (the kernel calls pdl_wait()
@@ -1345,6 +1608,41 @@ int launch_dec_w13_nv(const moe_shape_t &s, const uint16_t *xh, const float *xs,
                                tmR, tmS, xh, xs, x_gs, topk_idx, s.T, s.d, s.d_ff, s.E, s.k,
                                s.capacity, slot_major(s), W13sf, gs13, s.d_ff_shared,
                                shared ? 1 : 0, W13s_sf, gs13s, H32, Hs, status);
+    if (rc)
+        return rc;
+    return launched();
+}
+
+int launch_dec_w13_nvtc(const moe_shape_t &s, const uint8_t *xq, const uint8_t *xsf, float x_gs,
+                        const int32_t *topk_idx, const uint8_t *W13q, const uint8_t *W13sf,
+                        const float *gs13, const uint8_t *W13s_q, const uint8_t *W13s_sf,
+                        const float *gs13s, float *H32, uint32_t *status, cudaStream_t st)
+{
+    if (s.T == 0)
+        return MOE_OK;
+    if (s.T > kDtN || s.d % 256 != 0)
+        return MOE_ERR_UNSUPPORTED;
+    CUtensorMap tmA, tmAs, tmB;
+    int rc = make_tmap_u8_sw128(&tmA, W13q, s.d / 2, (long long)s.E * 2 * s.d_ff, 128);
+    if (rc)
+        return rc;
+    const bool shared = s.d_ff_shared > 0 && W13s_q;
+    if (shared) {
+        if ((rc = make_tmap_u8_sw128(&tmAs, W13s_q, s.d / 2, 2LL * s.d_ff_shared, 128)))
+            return rc;
+    } else {
+        tmAs = tmA;
+    }
+    // the tokens' codes: T rows, read as a 16-row box (rows past T are zeros)
+    if ((rc = make_tmap_u8_sw128(&tmB, xq, s.d / 2, s.T, kDtN)))
+        return rc;
+    const long long items = (long long)std::min(s.E, s.T * s.k) * (2 * s.d_ff / 128) +
+                            (shared ? 2 * s.d_ff_shared / 128 : 0);
+    const int blocks = (int)std::max<long long>(1, std::min<long long>(items, num_sms()));
+    float *Hs = H32 + (size_t)s.T * s.k * s.d_ff;
+    rc = launch_pdl_smem(k_dec_w13_nvtc, blocks, 192, sizeof(DtSmem) + 1024, st, tmA, tmAs, tmB, x_gs,
+                         topk_idx, s.T, s.d, s.d_ff, s.E, s.k, s.capacity, slot_major(s), W13sf, gs13,
+                         s.d_ff_shared, shared ? 1 : 0, W13s_sf, gs13s, xsf, H32, Hs, status);
     if (rc)
         return rc;
     return launched();

@@ -535,6 +535,24 @@ static int make_tmap_u8(CUtensorMap *m, const void *base, long long cols, long l
     return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
 }
 
+// Byte matrix [rows, cols] as a 2-D TMA tensor with a 128-byte-swizzled box
+// of 128 bytes x box_rows (the operand layout of the block-scaled MMAs).
+int make_tmap_u8_sw128(CUtensorMap *m, const void *base, long long cols, long long rows,
+                       int box_rows)
+{
+    auto fn = encode_fn_mx();
+    if (!fn)
+        return MOE_ERR_CUDA;
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)cols};
+    cuuint32_t box[2] = {128u, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1u, 1u};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
+}
+
 // Byte matrix [rows, cols] as a 2-D TMA tensor with an unswizzled box of
 // 128 bytes x box_rows (rows land 128 bytes apart in shared memory), for
 // kernels that read the tile with CUDA cores.

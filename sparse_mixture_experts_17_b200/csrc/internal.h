@@ -234,6 +234,16 @@ int launch_gemm_mx(const GemmArgs &g, cudaStream_t st);
 // box_rows (gemm_mx.cu). Returns MOE_OK or MOE_ERR_CUDA.
 int make_tmap_u8_rows(CUtensorMap *m, const void *base, long long cols, long long rows,
                       int box_rows);
+// The same with a 128-byte-swizzled box (the block-scaled MMAs' operand layout).
+int make_tmap_u8_sw128(CUtensorMap *m, const void *base, long long cols, long long rows,
+                       int box_rows);
+// NVFP4 decode w1/w3 on the tensor cores (T <= 16): x as NVFP4 codes (xq,
+// [T, d / 2]) with atom-layout scales (xsf, tile 0); writes H32 like
+// launch_dec_w13_nv.
+int launch_dec_w13_nvtc(const moe_shape_t &s, const uint8_t *xq, const uint8_t *xsf, float x_gs,
+                        const int32_t *topk_idx, const uint8_t *W13q, const uint8_t *W13sf,
+                        const float *gs13, const uint8_t *W13s_q, const uint8_t *W13s_sf,
+                        const float *gs13s, float *H32, uint32_t *status, cudaStream_t st);
 int launch_gemm_simt(const GemmArgs &g, cudaStream_t st);
 int num_sms();
 

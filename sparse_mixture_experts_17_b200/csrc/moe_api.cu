@@ -12,6 +12,11 @@
 #include "mxfp8.cuh"
 #include "nvfp4.cuh"
 
+// NVFP4 decode w1/w3 on the tensor cores (1) or on the CUDA cores (0)
+#ifndef MOE_NV_DEC_TC
+#define MOE_NV_DEC_TC 1
+#endif
+
 namespace moe {
 
 // ---------------------------------------------------------------- instrumentation
@@ -780,10 +785,21 @@ static int forward_mx_impl(const moe_shape_t &s, const WsLayout &L, void *ws, co
         const long long nh = (long long)s.T * s.k * s.d_ff + (long long)s.T * s.d_ff_shared;
         {
             StageMark m(MOE_STAGE_DEC_W13, st);
+#if MOE_NV_DEC_TC
+            // w1/w3 on the tensor cores: x as NVFP4 codes with atom-layout scales
+            (void)xh;
+            (void)xs;
+            uint8_t *xq = at<uint8_t>(ws, L.xq), *xsf = at<uint8_t>(ws, L.xsf);
+            rc = launch_nv_quantize_rows(x, s.T, s.d, nullptr, 0, lw.x_gs, xq, xsf, st);
+            if (!rc)
+                rc = launch_dec_w13_nvtc(s, xq, xsf, lw.x_gs, idx, W13q, W13sf, lw.W13gs, W13s_q,
+                                         W13s_sf, lw.W13s_gs, H32, status, st);
+#else
             rc = launch_nv_qrows_f16_bf16(x, (long long)s.T * s.d, lw.x_gs, xh, xs, st);
             if (!rc)
                 rc = launch_dec_w13_nv(s, xh, xs, lw.x_gs, idx, W13q, W13sf, lw.W13gs, W13s_q,
                                        W13s_sf, lw.W13s_gs, H32, status, st);
+#endif
         }
         if (rc)
             return rc;
