@@ -175,7 +175,7 @@ TRAFFIC_SOURCES = ["sparse_mixture_experts_17_b200/csrc/gemm_tc.cu",
                    "sparse_mixture_experts_17_b200/csrc/tiles.cuh",
                    "sparse_mixture_experts_17_b200/csrc/moe_api.cu"]
 TRAFFIC = {
-    "prefill": {"bytes": 3930873344 + 929801728, "sources_sha": "7efe44fd561229b7",
+    "prefill": {"bytes": 3373873920 + 931441664, "sources_sha": "71c2980b0c41d4c6",
                 "profile": "profiles/gemm_w13_traffic_mixtral_t16384.md"},
 }
 
@@ -467,7 +467,9 @@ def run_ours(a, world, rank, local):
             w13_bytes, expert_bytes = int(w13_bytes * mx), int(expert_bytes * mx)
         k13 = stages["dec_w13"][0] / stages["dec_w13"][1]
         ach = w13_bytes / (k13 / 1e3) / 1e9
-        dec_kernel = "k_dec_w13_mx" if a.mxfp8 else "k_dec_w13_nv" if a.nvfp4 else "k_dec_w13"
+        dec_kernel = ("k_dec_w13_mx" if a.mxfp8 else
+                      "k_nv_quantize_rows + k_dec_w13_nvtc (x to NVFP4, then tensor-core tiles)"
+                      if a.nvfp4 else "k_dec_w13")
         roofline = {"bound": "hbm", "kernel": f"{dec_kernel} (chosen experts' w1/w3 rows + SwiGLU)",
                     "achieved": round(ach, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                     "frac": round(ach / peaks["hbm_gbs"], 4), "traffic": None,
