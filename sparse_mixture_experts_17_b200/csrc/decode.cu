@@ -1076,47 +1076,109 @@ __global__ void __launch_bounds__(256, 2)
 }
 
 // ---------------------------------------------------------------- NVFP4 decode w1/w3, tensor cores
-// NVFP4 decode w1/w3 on the tensor cores: the chosen experts'
-// weights are the M side of block-scaled MMAs (128 packed W13 rows per tile)
-// and the tokens the N side (16 columns, rows past T read as zeros), so the
-// 4-bit codes are multiplied where they land in shared memory and no CUDA
-// core converts them. Work item = one 128-row tile of a chosen expert's
-// packed W13 (64 gate and 64 up rows: h columns 64 t .. 64 t + 63), or of
-// the shared expert after them.
+// NVFP4 decode w1/w3 on the tensor cores: the chosen experts' weights are
+// the M side of block-scaled MMAs (128 packed W13 rows per tile) and the
+// tokens the N side (16 columns; rows past T are zeros), so the 4-bit codes
+// are multiplied where they land in shared memory and no CUDA core converts
+// them. Work item = one 128-row tile of a chosen expert's packed W13 (64 gate
+// and 64 up rows: h columns 64 t .. 64 t + 63), or of the shared expert after
+// them.
 //
 // Structure (one CTA per SM, 192 threads), as the block-scaled GEMM:
+//   all        x quantized to NVFP4 (the prefill quantizer's arithmetic,
+//              global scale gs_x) straight into the MMA's operand layout:
+//              every K stage's 16 x 128-byte token tile (128-byte swizzle)
+//              and its four scale atoms stay resident for the whole launch
 //   warp 0     producer: per 256-element K stage, TMA of the 128 x 128-byte
-//              weight tile and the 16 x 128-byte token tile (128-byte
-//              swizzle) and bulk copies of both operands' four scale atoms
-//   warp 1     TMEM (two 16-column accumulators, then the stages' scale
-//              columns); one thread copies the scale atoms into TMEM
-//              (32x128b.warpx4) and issues four M=128 N=16 K=64
+//              weight tile (128-byte swizzle) and a bulk copy of its four
+//              scale atoms, through a ring of nst stages
+//   warp 1     TMEM (256 columns: two 16-column accumulators, then the
+//              stages' scale columns); one thread copies both operands' scale atoms into
+//              TMEM (32x128b.warpx4) and issues four M=128 N=16 K=64
 //              kind::mxf4nvf4 MMAs per stage
 //   warps 2-5  epilogue: the tile's 128 x 16 sums to shared memory, then
 //              h[a, c] = silu(gate) * up for each assignment a of the tile's
 //              expert, scaled by 1 / (gs_x gs_w), in fp32 (as the CUDA-core
 //              decode kernel writes it for the w2 phase)
+// Load balance: with G CTAs, the first items / G rounds are whole tiles; the
+// R = items mod G tiles left over are cut along K into pieces (dt_split) so
+// that the last round spreads over all CTAs. A piece writes its fp32 sums
+// to `part`, and k_dec_w13_nvtc_fix adds a tile's pieces in piece order
+// (deterministic) and forms its h columns.
 // Every pipeline wait is bounded (mbar_wait); on expiry the roles unwind.
 namespace {
 
-constexpr int kDtStages = 6;
+constexpr int kDtMaxStages = 6;
 constexpr int kDtN = 16;                  // token columns of an MMA
 constexpr int kDtABytes = 128 * 128;      // weight codes of one K stage (256 elements x 128 rows)
 constexpr int kDtBBytes = kDtN * 128;     // token codes of one K stage
 constexpr int kDtSfBytes = 2048;          // four scale atoms per operand and stage
 constexpr int kDtSfCols = 32;             // TMEM scale columns per stage (A's 16, then B's)
-constexpr int kDtTmemCols = 256;          // 2 x 16 accumulator columns, then 6 x 32 scale columns
+constexpr int kDtMaxRing = 6;             // ring stages: 2 x 16 accumulator + 6 x 32 scale columns <= 256
 
-struct DtSmem {
-    uint8_t a[kDtStages][kDtABytes];      // 1024-aligned: 128-byte swizzle atoms
-    uint8_t b[kDtStages][kDtBBytes];
-    uint8_t sfa[kDtStages][kDtSfBytes];
-    uint8_t sfb[kDtStages][kDtSfBytes];
-    float d[128][kDtN + 1];               // one tile's sums (the gate / up pairing)
-    uint64_t full[kDtStages], empty[kDtStages], tfull[2], tempty[2];
-    uint32_t tmem_slot;
-    int abort;
+// Dynamic shared memory of k_dec_w13_nvtc (byte offsets from a 1024-aligned
+// base; every operand region starts on a 1024-byte boundary):
+//   a    [nst][128 x 128 B]  weight codes of a K stage
+//   sfa  [nst][2 KB]         their scale atoms
+//   xb   [nks][16 x 128 B]   the tokens' codes, every K stage (resident)
+//   xsf  [nks][2 KB]         their scale atoms (resident)
+//   d    [128][17] fp32      one tile's sums
+struct DtCarve {
+    uint32_t a, sfa, xb, xsf, d, total;
 };
+
+__host__ __device__ __forceinline__ DtCarve dt_carve(int nst, int nks)
+{
+    DtCarve c;
+    c.a = 0;
+    c.sfa = c.a + (uint32_t)nst * kDtABytes;
+    c.xb = c.sfa + (uint32_t)nst * kDtSfBytes;
+    c.xsf = c.xb + (uint32_t)nks * kDtBBytes;
+    c.d = c.xsf + (uint32_t)nks * kDtSfBytes;
+    c.total = c.d + 128u * (kDtN + 1) * 4u;
+    return c;
+}
+
+// The work of one launch over G CTAs: `full` rounds of whole tiles (CTA c
+// takes tiles c + r G), then the R = items - full G tiles left over, each cut
+// into np pieces of ps K stages (the last piece may be shorter). Unit u =
+// piece u % np of leftover tile u / np goes to CTA u mod G.
+struct DtSplit {
+    int full, R, ps, np, units;
+};
+
+__host__ __device__ __forceinline__ DtSplit dt_split(int items, int G, int nks)
+{
+    DtSplit s;
+    s.full = items / G;
+    s.R = items - s.full * G;
+    s.ps = s.R ? (s.R * nks + G - 1) / G : nks;
+    s.np = (nks + s.ps - 1) / s.ps;
+    s.units = s.R * s.np;
+    return s;
+}
+
+// Work w of CTA c: the tile, its K-stage range, and the unit (-1: whole tile).
+__device__ __forceinline__ void dt_work(const DtSplit &sp, int G, int c, int w, int nks, int &item,
+                                        int &kb0, int &kb1, int &unit)
+{
+    if (w < sp.full) {
+        item = c + w * G;
+        kb0 = 0;
+        kb1 = nks;
+        unit = -1;
+    } else {
+        unit = c + (w - sp.full) * G;
+        item = sp.full * G + unit / sp.np;
+        kb0 = (unit % sp.np) * sp.ps;
+        kb1 = min(nks, kb0 + sp.ps);
+    }
+}
+
+__device__ __forceinline__ int dt_num_works(const DtSplit &sp, int G, int c)
+{
+    return sp.full + (c < sp.units ? (sp.units - 1 - c) / G + 1 : 0);
+}
 
 __device__ __forceinline__ uint64_t dt_desc_atom(uint32_t smem_addr)
 {
@@ -1176,95 +1238,170 @@ __device__ __forceinline__ void dt_tmem_ld16(uint32_t taddr, float (&v)[16])
 
 __device__ __forceinline__ void dt_epi_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
+// Orders this thread's generic-proxy shared-memory writes before later
+// async-proxy reads (tcgen05.cp, tcgen05.mma).
+__device__ __forceinline__ void dt_fence_proxy_async()
+{
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Tile `item` of a launch: whether it is the shared expert's, its index t
+// within its source (h columns 64 t ..), and its source's unique-expert slot.
+struct DtTile {
+    bool shared;
+    int u, t;
+};
+
+__device__ __forceinline__ DtTile dt_tile(int item, int routed_items, int tpr)
+{
+    DtTile r;
+    r.shared = item >= routed_items;
+    r.u = r.shared ? 0 : item / tpr;
+    r.t = r.shared ? item - routed_items : item % tpr;
+    return r;
+}
+
 } // namespace
 
 __global__ void __launch_bounds__(192, 1)
     k_dec_w13_nvtc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmAs,
-                   const __grid_constant__ CUtensorMap tmB, float x_gs,
-                   const int32_t *__restrict__ idx, int T, int d, int d_ff, int E, int k, int C,
-                   int slot_major, const uint8_t *__restrict__ W13sf,
-                   const float *__restrict__ gs13, int d_ff_s, int has_shared,
-                   const uint8_t *__restrict__ W13s_sf, const float *__restrict__ gs13s,
-                   const uint8_t *__restrict__ xsf, float *__restrict__ H32,
-                   float *__restrict__ Hs32, uint32_t *status)
+                   const uint16_t *__restrict__ x, float x_gs, const int32_t *__restrict__ idx,
+                   int T, int d, int d_ff, int E, int k, int C, int slot_major, int nst,
+                   const uint8_t *__restrict__ W13sf, const float *__restrict__ gs13, int d_ff_s,
+                   int has_shared, const uint8_t *__restrict__ W13s_sf,
+                   const float *__restrict__ gs13s, float *__restrict__ H32,
+                   float *__restrict__ Hs32, float *__restrict__ part, uint32_t *status)
 {
     extern __shared__ uint8_t dt_raw[];
-    DtSmem &S = *reinterpret_cast<DtSmem *>(
+    uint8_t *base = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(dt_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    const int nks = d / 256;   // K stages of a tile
+    const DtCarve cv = dt_carve(nst, nks);
+    uint8_t *const sa = base + cv.a, *const ssfa = base + cv.sfa;
+    uint8_t *const sxb = base + cv.xb, *const sxsf = base + cv.xsf;
+    float(*const sd)[kDtN + 1] = reinterpret_cast<float(*)[kDtN + 1]>(base + cv.d);
+    __shared__ uint64_t full[kDtMaxStages], empty[kDtMaxStages], tfull[2], tempty[2];
+    __shared__ uint32_t tmem_slot;
+    __shared__ int abort_s;
     __shared__ DecPlanSmem P;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kDtStages; ++s) {
-            mbar_init(&S.full[s], 1);
-            mbar_init(&S.empty[s], 1);
+        for (int s = 0; s < nst; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
-            mbar_init(&S.tfull[b], 1);
-            mbar_init(&S.tempty[b], 4);
+            mbar_init(&tfull[b], 1);
+            mbar_init(&tempty[b], 4);
         }
-        S.abort = 0;
+        abort_s = 0;
         fence_mbar_init();
     }
     if (warp == 0 && lane == 0) {
         tma_prefetch_desc(&tmA);
-        tma_prefetch_desc(&tmB);
+        if (has_shared)
+            tma_prefetch_desc(&tmAs);
     }
     if (warp == 1) {
-        tmem_alloc(&S.tmem_slot, kDtTmemCols);
+        tmem_alloc(&tmem_slot, 256);
         tmem_relinquish();
+    }
+    // x (an input of the layer, final before the routing kernel started):
+    // rows past T and their scales are zeros
+    {
+        uint4 *z = reinterpret_cast<uint4 *>(sxb);
+        const int n16 = nks * (kDtBBytes + kDtSfBytes) / 16;
+        for (int i = threadIdx.x; i < n16; i += blockDim.x)
+            z[i] = make_uint4(0u, 0u, 0u, 0u);
+        __syncthreads();
+        const int bpr = d / kNvBlock;   // 16-element blocks of a row
+        for (int i = threadIdx.x; i < T * bpr; i += blockDim.x) {
+            const int r = i / bpr, b = i - r * bpr;
+            const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)r * d + b * kNvBlock);
+            float v[16];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const uint4 w = __ldg(src + h);
+                const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    v[8 * h + 2 * j] = bf16lo(ww[j]);
+                    v[8 * h + 2 * j + 1] = bf16hi(ww[j]);
+                }
+            }
+            uint2 q;
+            const uint8_t sc = nv_quantize16(v, x_gs, q);
+            // block ib of K stage kb: bytes 8 ib .. 8 ib + 7 of the stage's
+            // 128-byte row r, whose 16-byte chunk c sits at chunk c ^ (r & 7)
+            const int kb = b >> 4, ib = b & 15;
+            *reinterpret_cast<uint2 *>(sxb + kb * kDtBBytes + r * 128 +
+                                       (((ib >> 1) ^ (r & 7)) << 4) + (ib & 1) * 8) = q;
+            sxsf[nv_sf_offset(0, r, b, d)] = sc;
+        }
+        dt_fence_proxy_async();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tmem_base = S.tmem_slot;
+    const uint32_t tmem_base = tmem_slot;
     pdl_wait();
     pdl_trigger();
     build_plan(P, idx, T, E, k, C, slot_major, status);   // ends with __syncthreads
-    volatile int *abort_flag = &S.abort;
+    volatile int *abort_flag = &abort_s;
     const int tpr = 2 * d_ff / 128;                        // tiles of a routed expert
     const int routed_items = P.U * tpr;
     const int items = routed_items + (has_shared ? 2 * d_ff_s / 128 : 0);
-    const int nks = d / 256;                               // K stages of a tile
+    const int G = gridDim.x, c = blockIdx.x;
+    const DtSplit sp = dt_split(items, G, nks);
+    const int nw = dt_num_works(sp, G, c);
 
     if (warp == 0) {
         if (lane == 0) {   // ---------------- producer
             uint32_t it = 0;
             bool ok = true;
-            for (int item = blockIdx.x; ok && item < items; item += gridDim.x) {
-                const bool shared = item >= routed_items;
-                const int t = shared ? item - routed_items : item % tpr;
-                const long long row0 =
-                    shared ? (long long)t * 128 : (long long)P.uniq[item / tpr] * 2 * d_ff + t * 128;
-                const uint8_t *sfa = (shared ? W13s_sf : W13sf) + (size_t)(row0 / 128) * (d / 64) * 512;
-                for (int kb = 0; kb < nks; ++kb, ++it) {
-                    const int s = it % kDtStages;
-                    const uint32_t ph = (it / kDtStages) & 1u;
-                    if (!mbar_wait(&S.empty[s], ph ^ 1u, abort_flag, status)) {
+            for (int w = 0; ok && w < nw; ++w) {
+                int item, kb0, kb1, unit;
+                dt_work(sp, G, c, w, nks, item, kb0, kb1, unit);
+                const DtTile tl = dt_tile(item, routed_items, tpr);
+                const long long row0 = tl.shared ? (long long)tl.t * 128
+                                                 : (long long)P.uniq[tl.u] * 2 * d_ff + tl.t * 128;
+                const uint8_t *sfa = (tl.shared ? W13s_sf : W13sf) + (size_t)(row0 / 128) * (d / 64) * 512;
+                for (int kb = kb0; kb < kb1; ++kb, ++it) {
+                    const int s = it % nst;
+                    const uint32_t ph = (it / nst) & 1u;
+                    if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag, status)) {
                         ok = false;
                         break;
                     }
-                    mbar_arrive_expect_tx(&S.full[s], kDtABytes + kDtBBytes + 2 * kDtSfBytes);
-                    tma_load_2d(S.a[s], shared ? &tmAs : &tmA, kb * 128, (int)row0, &S.full[s]);
-                    tma_load_2d(S.b[s], &tmB, kb * 128, 0, &S.full[s]);
-                    dt_bulk_load(S.sfa[s], sfa + (size_t)kb * kDtSfBytes, kDtSfBytes, &S.full[s]);
-                    dt_bulk_load(S.sfb[s], xsf + (size_t)kb * kDtSfBytes, kDtSfBytes, &S.full[s]);
+                    mbar_arrive_expect_tx(&full[s], kDtABytes + kDtSfBytes);
+                    tma_load_2d(sa + s * kDtABytes, tl.shared ? &tmAs : &tmA, kb * 128, (int)row0, &full[s]);
+                    dt_bulk_load(ssfa + s * kDtSfBytes, sfa + (size_t)kb * kDtSfBytes, kDtSfBytes, &full[s]);
                 }
+            }
+            if (!ok) {
+                // let the copies already issued land before the CTA can exit
+                int never = 0;
+                const uint32_t first = it >= (uint32_t)nst ? it - nst : 0;
+                for (uint32_t i = first; i < it; ++i)
+                    mbar_wait(&full[i % nst], (i / nst) & 1u, &never, status);
             }
         }
     } else if (warp == 1) {
         if (lane == 0) {   // ---------------- MMA issuer
-            uint32_t it = 0, local = 0;
-            for (int item = blockIdx.x; item < items; item += gridDim.x, ++local) {
-                const uint32_t b = local & 1u, aph = (local >> 1) & 1u;
-                if (!mbar_wait(&S.tempty[b], aph ^ 1u, abort_flag, status))
+            uint32_t it = 0;
+            for (int w = 0; w < nw; ++w) {
+                int item, kb0, kb1, unit;
+                dt_work(sp, G, c, w, nks, item, kb0, kb1, unit);
+                const uint32_t b = w & 1, aph = (w >> 1) & 1u;
+                if (!mbar_wait(&tempty[b], aph ^ 1u, abort_flag, status))
                     break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + b * kDtN;
                 bool ok = true;
-                for (int kb = 0; kb < nks; ++kb, ++it) {
-                    const int s = it % kDtStages;
-                    const uint32_t ph = (it / kDtStages) & 1u;
-                    if (!mbar_wait(&S.full[s], ph, abort_flag, status)) {
+                for (int kb = kb0; kb < kb1; ++kb, ++it) {
+                    const int s = it % nst;
+                    const uint32_t ph = (it / nst) & 1u;
+                    if (!mbar_wait(&full[s], ph, abort_flag, status)) {
                         ok = false;
                         break;
                     }
@@ -1272,30 +1409,33 @@ __global__ void __launch_bounds__(192, 1)
                     // each stage has its own scale columns after the accumulators
                     const uint32_t sf_a = tmem_base + 2 * kDtN + s * kDtSfCols;
                     const uint32_t sf_b = sf_a + 16;
+                    const uint32_t a_sf = smem_u32(ssfa + s * kDtSfBytes);
+                    const uint32_t b_sf = smem_u32(sxsf + kb * kDtSfBytes);
 #pragma unroll
                     for (int g = 0; g < 4; ++g) {
-                        dt_cp_atom(sf_a + 4 * g, dt_desc_atom(smem_u32(S.sfa[s]) + 512 * g));
-                        dt_cp_atom(sf_b + 4 * g, dt_desc_atom(smem_u32(S.sfb[s]) + 512 * g));
+                        dt_cp_atom(sf_a + 4 * g, dt_desc_atom(a_sf + 512 * g));
+                        dt_cp_atom(sf_b + 4 * g, dt_desc_atom(b_sf + 512 * g));
                     }
-                    const uint32_t a0 = smem_u32(S.a[s]), b0 = smem_u32(S.b[s]);
+                    const uint32_t a0 = smem_u32(sa + s * kDtABytes), b0 = smem_u32(sxb + kb * kDtBBytes);
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
                         dt_mma(d_tmem, smem_desc_k128(a0 + kk * 32), smem_desc_k128(b0 + kk * 32),
-                               sf_a + 4 * kk, sf_b + 4 * kk, (kb | kk) != 0);
-                    tc_commit(&S.empty[s]);
+                               sf_a + 4 * kk, sf_b + 4 * kk, (kb != kb0 || kk != 0) ? 1u : 0u);
+                    tc_commit(&empty[s]);
                 }
                 if (!ok)
                     break;
-                tc_commit(&S.tfull[b]);
+                tc_commit(&tfull[b]);
             }
         }
     } else {   // ---------------- epilogue warps 2..5
-        const int q = warp & 3;   // TMEM lane quarter this warp may access
+        const int q = warp & 3;            // TMEM lane quarter this warp may access
         const int et = threadIdx.x - 64;   // 0..127
-        uint32_t local = 0;
-        for (int item = blockIdx.x; item < items; item += gridDim.x, ++local) {
-            const uint32_t b = local & 1u, aph = (local >> 1) & 1u;
-            const bool got = mbar_wait(&S.tfull[b], aph, abort_flag, status);
+        for (int w = 0; w < nw; ++w) {
+            int item, kb0, kb1, unit;
+            dt_work(sp, G, c, w, nks, item, kb0, kb1, unit);
+            const uint32_t b = w & 1, aph = (w >> 1) & 1u;
+            const bool got = mbar_wait(&tfull[b], aph, abort_flag, status);
             tc_fence_after();
             if (got) {
                 float v[16];
@@ -1303,28 +1443,30 @@ __global__ void __launch_bounds__(192, 1)
                 tmem_ld_wait();
 #pragma unroll
                 for (int i = 0; i < kDtN; ++i)
-                    S.d[q * 32 + lane][i] = v[i];
+                    sd[q * 32 + lane][i] = v[i];
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0)
-                mbar_arrive(&S.tempty[b]);
+                mbar_arrive(&tempty[b]);
             dt_epi_sync();
-            if (got && et < 64) {
-                const bool shared = item >= routed_items;
-                const int u = shared ? 0 : item / tpr;
-                const int t = shared ? item - routed_items : item % tpr;
-                const int a0 = shared ? 0 : P.ustart[u];
-                const int na = shared ? T : P.ustart[u + 1] - a0;
-                const float inv = 1.0f / (x_gs * (shared ? gs13s[0] : gs13[P.uniq[u]]));
+            if (got && unit >= 0) {
+                // a piece: its sums, row et of token column tok
+                for (int tok = 0; tok < T; ++tok)
+                    part[((size_t)unit * T + tok) * 128 + et] = sd[et][tok];
+            } else if (got && et < 64) {
+                const DtTile tl = dt_tile(item, routed_items, tpr);
+                const int a0 = tl.shared ? 0 : P.ustart[tl.u];
+                const int na = tl.shared ? T : P.ustart[tl.u + 1] - a0;
+                const float inv = 1.0f / (x_gs * (tl.shared ? gs13s[0] : gs13[P.uniq[tl.u]]));
                 for (int qa = 0; qa < na; ++qa) {
-                    const int a = shared ? qa : P.list[a0 + qa];
-                    const int tok = shared ? qa : a / k;
-                    const float h = silu_mul(S.d[et][tok] * inv, S.d[64 + et][tok] * inv);
-                    if (shared)
-                        Hs32[(size_t)qa * d_ff_s + 64 * t + et] = h;
+                    const int a = tl.shared ? qa : P.list[a0 + qa];
+                    const int tok = tl.shared ? qa : a / k;
+                    const float h = silu_mul(sd[et][tok] * inv, sd[64 + et][tok] * inv);
+                    if (tl.shared)
+                        Hs32[(size_t)qa * d_ff_s + 64 * tl.t + et] = h;
                     else
-                        H32[(size_t)a * d_ff + 64 * t + et] = h;
+                        H32[(size_t)a * d_ff + 64 * tl.t + et] = h;
                 }
             }
             dt_epi_sync();
@@ -1334,7 +1476,62 @@ __global__ void __launch_bounds__(192, 1)
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, kDtTmemCols);
+        tmem_dealloc(tmem_base, 256);
+    }
+}
+
+// The leftover tiles of k_dec_w13_nvtc (same G): block j adds the np pieces
+// of leftover tile j in piece order and forms its 64 h columns.
+__global__ void __launch_bounds__(64)
+    k_dec_w13_nvtc_fix(const int32_t *__restrict__ idx, int T, int d, int d_ff, int E, int k, int C,
+                       int slot_major, int G, int d_ff_s, int has_shared, float x_gs,
+                       const float *__restrict__ gs13, const float *__restrict__ gs13s,
+                       const float *__restrict__ part, float *__restrict__ H32,
+                       float *__restrict__ Hs32, uint32_t *status)
+{
+    __shared__ DecPlanSmem P;
+    build_plan(P, idx, T, E, k, C, slot_major, status);   // idx is final: the w1/w3 kernel read it
+    pdl_wait();      // the pieces come from the w1/w3 kernel
+    pdl_trigger();
+    const int tpr = 2 * d_ff / 128;
+    const int routed_items = P.U * tpr;
+    const int items = routed_items + (has_shared ? 2 * d_ff_s / 128 : 0);
+    const DtSplit sp = dt_split(items, G, d / 256);
+    const int j = blockIdx.x;
+    if (j >= sp.R)
+        return;
+    const DtTile tl = dt_tile(sp.full * G + j, routed_items, tpr);
+    const int a0 = tl.shared ? 0 : P.ustart[tl.u];
+    const int na = tl.shared ? T : P.ustart[tl.u + 1] - a0;
+    const float inv = 1.0f / (x_gs * (tl.shared ? gs13s[0] : gs13[P.uniq[tl.u]]));
+    const int et = threadIdx.x;
+    for (int qa = 0; qa < na; ++qa) {
+        const int a = tl.shared ? qa : P.list[a0 + qa];
+        const int tok = tl.shared ? qa : a / k;
+        const float *pp = part + ((size_t)j * sp.np * T + tok) * 128 + et;
+        const size_t stride = (size_t)T * 128;   // from one piece to the next
+        float g = 0.f, u = 0.f;
+        // eight pieces' loads in flight at a time, added in piece order
+        for (int p0 = 0; p0 < sp.np; p0 += 8) {
+            float vg[8], vu[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const bool in = p0 + i < sp.np;
+                vg[i] = in ? __ldcg(pp + (p0 + i) * stride) : 0.f;
+                vu[i] = in ? __ldcg(pp + (p0 + i) * stride + 64) : 0.f;
+            }
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                if (p0 + i < sp.np) {
+                    g += vg[i];
+                    u += vu[i];
+                }
+        }
+        const float h = silu_mul(g * inv, u * inv);
+        if (tl.shared)
+            Hs32[(size_t)qa * d_ff_s + 64 * tl.t + et] = h;
+        else
+            H32[(size_t)a * d_ff + 64 * tl.t + et] = h;
     }
 }
 
@@ -1395,6 +1592,39 @@ static int smem_attr_once(const void *kernel, size_t smem)
 }
 
 // The same, with dynamic shared memory.
+// The dynamic shared memory a launch of `kernel` may take on this device:
+// the opt-in maximum less the kernel's static shared memory.
+static int smem_limit(const void *kernel, int &dyn_max)
+{
+    constexpr int kMax = 64;
+    static std::mutex mu;
+    static const void *seen_k[kMax];
+    static int seen_d[kMax], seen_v[kMax];
+    static int n_seen = 0;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i = 0; i < n_seen; ++i)
+        if (seen_k[i] == kernel && seen_d[i] == dev) {
+            dyn_max = seen_v[i];
+            return MOE_OK;
+        }
+    int optin = 0;
+    cudaFuncAttributes fa;
+    if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess ||
+        cudaFuncGetAttributes(&fa, kernel) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    dyn_max = optin - (int)fa.sharedSizeBytes;
+    if (n_seen < kMax) {
+        seen_k[n_seen] = kernel;
+        seen_d[n_seen] = dev;
+        seen_v[n_seen] = dyn_max;
+        ++n_seen;
+    }
+    return MOE_OK;
+}
+
 template <typename... KArgs, typename... Args>
 static int launch_pdl_smem(void (*kernel)(KArgs...), int grid, int block, size_t smem,
                            cudaStream_t st, Args... args)
@@ -1613,38 +1843,56 @@ int launch_dec_w13_nv(const moe_shape_t &s, const uint16_t *xh, const float *xs,
     return launched();
 }
 
-int launch_dec_w13_nvtc(const moe_shape_t &s, const uint8_t *xq, const uint8_t *xsf, float x_gs,
+int launch_dec_w13_nvtc(const moe_shape_t &s, const uint16_t *x, float x_gs,
                         const int32_t *topk_idx, const uint8_t *W13q, const uint8_t *W13sf,
                         const float *gs13, const uint8_t *W13s_q, const uint8_t *W13s_sf,
-                        const float *gs13s, float *H32, uint32_t *status, cudaStream_t st)
+                        const float *gs13s, float *H32, float *part, size_t part_floats,
+                        uint32_t *status, cudaStream_t st)
 {
     if (s.T == 0)
         return MOE_OK;
-    if (s.T > kDtN || s.d % 256 != 0)
+    const bool shared = s.d_ff_shared > 0 && W13s_q;
+    if (s.T > kDtN || s.d % 256 != 0 || (2 * s.d_ff) % 128 != 0 ||
+        (shared && (2 * s.d_ff_shared) % 128 != 0))
         return MOE_ERR_UNSUPPORTED;
-    CUtensorMap tmA, tmAs, tmB;
+    const int nks = s.d / 256;
+    const long long items = (long long)std::min(s.E, s.T * s.k) * (2 * s.d_ff / 128) +
+                            (shared ? 2 * s.d_ff_shared / 128 : 0);
+    const int blocks = (int)std::max<long long>(1, std::min<long long>(items, num_sms()));
+    // pieces: fewer than 2 G units of T x 128 sums
+    if ((size_t)2 * blocks * s.T * 128 > part_floats)
+        return MOE_ERR_UNSUPPORTED;
+    // the deepest ring (2..kDtMaxStages stages) that fits beside the resident x
+    int dyn_max = 0;
+    if (const int rc = smem_limit(reinterpret_cast<const void *>(k_dec_w13_nvtc), dyn_max))
+        return rc;
+    int nst = kDtMaxRing;
+    while (nst >= 2 && (int)dt_carve(nst, nks).total + 1024 > dyn_max)
+        --nst;
+    if (nst < 2)
+        return MOE_ERR_UNSUPPORTED;
+    CUtensorMap tmA, tmAs;
     int rc = make_tmap_u8_sw128(&tmA, W13q, s.d / 2, (long long)s.E * 2 * s.d_ff, 128);
     if (rc)
         return rc;
-    const bool shared = s.d_ff_shared > 0 && W13s_q;
     if (shared) {
         if ((rc = make_tmap_u8_sw128(&tmAs, W13s_q, s.d / 2, 2LL * s.d_ff_shared, 128)))
             return rc;
     } else {
         tmAs = tmA;
     }
-    // the tokens' codes: T rows, read as a 16-row box (rows past T are zeros)
-    if ((rc = make_tmap_u8_sw128(&tmB, xq, s.d / 2, s.T, kDtN)))
-        return rc;
-    const long long items = (long long)std::min(s.E, s.T * s.k) * (2 * s.d_ff / 128) +
-                            (shared ? 2 * s.d_ff_shared / 128 : 0);
-    const int blocks = (int)std::max<long long>(1, std::min<long long>(items, num_sms()));
     float *Hs = H32 + (size_t)s.T * s.k * s.d_ff;
-    rc = launch_pdl_smem(k_dec_w13_nvtc, blocks, 192, sizeof(DtSmem) + 1024, st, tmA, tmAs, tmB, x_gs,
-                         topk_idx, s.T, s.d, s.d_ff, s.E, s.k, s.capacity, slot_major(s), W13sf, gs13,
-                         s.d_ff_shared, shared ? 1 : 0, W13s_sf, gs13s, xsf, H32, Hs, status);
+    rc = launch_pdl_smem(k_dec_w13_nvtc, blocks, 192, dt_carve(nst, nks).total + 1024, st, tmA, tmAs,
+                         x, x_gs, topk_idx, s.T, s.d, s.d_ff, s.E, s.k, s.capacity, slot_major(s), nst,
+                         W13sf, gs13, s.d_ff_shared, shared ? 1 : 0, W13s_sf, gs13s, H32, Hs, part,
+                         status);
     if (rc)
         return rc;
+    if ((rc = launched()))
+        return rc;
+    launch_pdl(k_dec_w13_nvtc_fix, blocks, 64, st, topk_idx, s.T, s.d, s.d_ff, s.E, s.k, s.capacity,
+               slot_major(s), blocks, s.d_ff_shared, shared ? 1 : 0, x_gs, gs13, gs13s,
+               (const float *)part, H32, Hs, status);
     return launched();
 }
 

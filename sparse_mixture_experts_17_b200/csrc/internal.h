@@ -75,6 +75,7 @@ struct WsLayout {
     size_t xq, xsf, Hq, Hsf, xq_s, xsf_s, Hsq, Hssf;   // MXFP8 operands
     size_t dec_xdq, dec_H32;                             // MXFP8 / NVFP4 decode
     size_t dec_xs, dec_hs;                               // NVFP4 decode: scale values
+    size_t dec_part;                                     // NVFP4 decode: split-K sums
     size_t tile_start;                                   // first m-tile of each expert
     size_t dbg_seen;                                     // dispatch checks: count per row
     // backward pass
@@ -237,13 +238,17 @@ int make_tmap_u8_rows(CUtensorMap *m, const void *base, long long cols, long lon
 // The same with a 128-byte-swizzled box (the block-scaled MMAs' operand layout).
 int make_tmap_u8_sw128(CUtensorMap *m, const void *base, long long cols, long long rows,
                        int box_rows);
-// NVFP4 decode w1/w3 on the tensor cores (T <= 16): x as NVFP4 codes (xq,
-// [T, d / 2]) with atom-layout scales (xsf, tile 0); writes H32 like
-// launch_dec_w13_nv.
-int launch_dec_w13_nvtc(const moe_shape_t &s, const uint8_t *xq, const uint8_t *xsf, float x_gs,
+// NVFP4 decode w1/w3 on the tensor cores (T <= 16): quantizes x (bf16
+// [T, d]) with x_gs inside the kernel and writes H32 like launch_dec_w13_nv;
+// tiles left over after the whole rounds are split along K, their pieces'
+// sums go to `part` (part_floats floats, at least 2 x CTAs x T x 128) and a
+// second kernel adds them. Returns MOE_ERR_UNSUPPORTED (nothing launched)
+// for shapes it does not take.
+int launch_dec_w13_nvtc(const moe_shape_t &s, const uint16_t *x, float x_gs,
                         const int32_t *topk_idx, const uint8_t *W13q, const uint8_t *W13sf,
                         const float *gs13, const uint8_t *W13s_q, const uint8_t *W13s_sf,
-                        const float *gs13s, float *H32, uint32_t *status, cudaStream_t st);
+                        const float *gs13s, float *H32, float *part, size_t part_floats,
+                        uint32_t *status, cudaStream_t st);
 int launch_gemm_simt(const GemmArgs &g, cudaStream_t st);
 int num_sms();
 

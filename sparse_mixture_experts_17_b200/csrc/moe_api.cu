@@ -12,11 +12,6 @@
 #include "mxfp8.cuh"
 #include "nvfp4.cuh"
 
-// NVFP4 decode w1/w3 on the tensor cores (1) or on the CUDA cores (0)
-#ifndef MOE_NV_DEC_TC
-#define MOE_NV_DEC_TC 1
-#endif
-
 namespace moe {
 
 // ---------------------------------------------------------------- instrumentation
@@ -102,6 +97,13 @@ int check_shape(const moe_shape_t *s)
 
 static bool al16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// fp32 split-K sums of the NVFP4 decode w1/w3 kernel: 2 x 1024 CTAs x
+// (T <= 2) x 128 (non-decreasing in T)
+static size_t dec_part_floats(const moe_shape_t &s)
+{
+    return (size_t)2 * 1024 * (size_t)std::min(s.T, 2) * 128;
+}
+
 WsLayout ws_layout(const moe_shape_t &s)
 {
     WsLayout L;
@@ -154,6 +156,7 @@ WsLayout ws_layout(const moe_shape_t &s)
     L.dec_H32 = take(lowp ? (Td * k * s.d_ff + Td * dfs) * 4 : 0);
     L.dec_xs = take(nv ? Td * (s.d / 16) * 4 : 0);
     L.dec_hs = take(nv ? (Td * k * s.d_ff + Td * dfs) / 16 * 4 : 0);
+    L.dec_part = take(nv ? dec_part_floats(s) * 4 : 0);
     // activation scales: routed operands keyed by m-tile (at most max_mt
     // tiles of 128 rows), shared-expert operands by row / 128; MXFP8 in the
     // atom layout, NVFP4 (16-element blocks) in the activation layout of
@@ -785,21 +788,17 @@ static int forward_mx_impl(const moe_shape_t &s, const WsLayout &L, void *ws, co
         const long long nh = (long long)s.T * s.k * s.d_ff + (long long)s.T * s.d_ff_shared;
         {
             StageMark m(MOE_STAGE_DEC_W13, st);
-#if MOE_NV_DEC_TC
-            // w1/w3 on the tensor cores: x as NVFP4 codes with atom-layout scales
-            (void)xh;
-            (void)xs;
-            uint8_t *xq = at<uint8_t>(ws, L.xq), *xsf = at<uint8_t>(ws, L.xsf);
-            rc = launch_nv_quantize_rows(x, s.T, s.d, nullptr, 0, lw.x_gs, xq, xsf, st);
-            if (!rc)
-                rc = launch_dec_w13_nvtc(s, xq, xsf, lw.x_gs, idx, W13q, W13sf, lw.W13gs, W13s_q,
-                                         W13s_sf, lw.W13s_gs, H32, status, st);
-#else
-            rc = launch_nv_qrows_f16_bf16(x, (long long)s.T * s.d, lw.x_gs, xh, xs, st);
-            if (!rc)
-                rc = launch_dec_w13_nv(s, xh, xs, lw.x_gs, idx, W13q, W13sf, lw.W13gs, W13s_q,
-                                       W13s_sf, lw.W13s_gs, H32, status, st);
-#endif
+            // w1/w3 on the tensor cores; shapes that kernel does not take go
+            // through the CUDA-core kernel on f16 code values
+            rc = launch_dec_w13_nvtc(s, x, lw.x_gs, idx, W13q, W13sf, lw.W13gs, W13s_q, W13s_sf,
+                                     lw.W13s_gs, H32, at<float>(ws, L.dec_part), dec_part_floats(s),
+                                     status, st);
+            if (rc == MOE_ERR_UNSUPPORTED) {
+                rc = launch_nv_qrows_f16_bf16(x, (long long)s.T * s.d, lw.x_gs, xh, xs, st);
+                if (!rc)
+                    rc = launch_dec_w13_nv(s, xh, xs, lw.x_gs, idx, W13q, W13sf, lw.W13gs, W13s_q,
+                                           W13s_sf, lw.W13s_gs, H32, status, st);
+            }
         }
         if (rc)
             return rc;

@@ -194,9 +194,10 @@ def test_nvfp4_small_batches(T):
 
 @pytest.mark.parametrize("T", [1, 2])
 def test_nvfp4_decode_kernels_and_chain(T):
-    """The NVFP4 decode kernels (codes streamed through CUDA cores, exact
-    16-element block dot products) and the tensor-core chain on the same
-    inputs, both against the oracle, at d = 4096."""
+    """The NVFP4 decode kernels (w1/w3 as M = 128, N = 16 block-scaled MMAs;
+    w2 as exact 16-element block dot products on the CUDA cores) and the
+    tensor-core chain on the same inputs, both against the oracle, at
+    d = 4096."""
     w = small_workload("nvdk", T, 4096, 1536, 8, 2, zipf_s=0.5)
     inp = I.make_inputs(w, "cuda", seed=10 + T)
     x_gs = float(2688.0 / inp["x"].float().abs().max().item())
@@ -212,6 +213,24 @@ def test_nvfp4_decode_kernels_and_chain(T):
     assert_layer_close(out_p, ref, f"nvfp4 tensor-core chain T={T}")
     # the default path at T <= 2 is the decode kernels (deterministic: fixed order)
     assert torch.equal(out_0, out_d)
+
+
+@pytest.mark.parametrize("T", [1, 2])
+def test_nvfp4_decode_split_tail(T):
+    """More w1/w3 tiles than SMs with some left over (2 x 152 routed + 4
+    shared tiles): the decode kernel cuts the leftover tiles along K and a
+    second kernel adds their pieces in a fixed order."""
+    w = small_workload("nvsplit", T, 1024, 9728, 2, 2, d_ff_shared=256)
+    inp = I.make_inputs(w, "cuda", seed=20 + T)
+    layer = M.MoeLayerNv4(inp, h_gs=2.0)
+    logits = torch.empty(T, w.E, dtype=torch.float32, device="cuda")
+    out = layer.forward(inp["x"], logits_out=logits).clone()
+    out2 = layer.forward(inp["x"]).clone()
+    torch.cuda.synchronize()
+    assert int(layer.status.item()) == 0
+    _, _, ref = _oracle_out(inp, logits.cpu().numpy(), w.k, 0, np.float32(1.0), np.float32(2.0))
+    assert_layer_close(out, ref, f"nvfp4 decode split T={T}")
+    assert torch.equal(out, out2)
 
 
 @pytest.mark.parametrize("C", [0, 1])
