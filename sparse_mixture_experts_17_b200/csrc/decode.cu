@@ -1123,8 +1123,10 @@ constexpr int kDtMaxRing = 6;             // ring stages: 2 x 16 accumulator + 6
 //   xb   [nks][16 x 128 B]   the tokens' codes, every K stage (resident)
 //   xsf  [nks][2 KB]         their scale atoms (resident)
 //   d    [128][17] fp32      one tile's sums
+//   hb   [16][64] fp32       one tile's h columns, per assignment (quantized
+//                            to NVFP4 from here)
 struct DtCarve {
-    uint32_t a, sfa, xb, xsf, d, total;
+    uint32_t a, sfa, xb, xsf, d, hb, total;
 };
 
 __host__ __device__ __forceinline__ DtCarve dt_carve(int nst, int nks)
@@ -1135,7 +1137,8 @@ __host__ __device__ __forceinline__ DtCarve dt_carve(int nst, int nks)
     c.xb = c.sfa + (uint32_t)nst * kDtSfBytes;
     c.xsf = c.xb + (uint32_t)nks * kDtBBytes;
     c.d = c.xsf + (uint32_t)nks * kDtSfBytes;
-    c.total = c.d + 128u * (kDtN + 1) * 4u;
+    c.hb = c.d + 128u * (kDtN + 1) * 4u;
+    c.total = c.hb + kDtN * 64u * 4u;
     return c;
 }
 
@@ -1261,6 +1264,23 @@ __device__ __forceinline__ DtTile dt_tile(int item, int routed_items, int tpr)
     return r;
 }
 
+// h block bi (columns 64 t + 16 bi ..) of row `row` of an NVFP4 operand with
+// K columns: 8 bytes of codes and the E4M3 scale in the atom layout, the
+// arithmetic of every other NVFP4 quantizer here (nv_quantize16).
+__device__ __forceinline__ void dt_quantize_h(const float *hrow16, float h_gs, int row, int t, int bi,
+                                              int K, uint8_t *codes, uint8_t *sf)
+{
+    float v[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+        v[i] = hrow16[i];
+    uint2 q;
+    const uint8_t sc = nv_quantize16(v, h_gs, q);
+    const int col = 64 * t + 16 * bi;
+    *reinterpret_cast<uint2 *>(codes + (size_t)row * (K / 2) + col / 2) = q;
+    sf[nv_sf_offset(row >> 7, row & 127, col / kNvBlock, K)] = sc;
+}
+
 } // namespace
 
 __global__ void __launch_bounds__(192, 1)
@@ -1270,7 +1290,9 @@ __global__ void __launch_bounds__(192, 1)
                    const uint8_t *__restrict__ W13sf, const float *__restrict__ gs13, int d_ff_s,
                    int has_shared, const uint8_t *__restrict__ W13s_sf,
                    const float *__restrict__ gs13s, float *__restrict__ H32,
-                   float *__restrict__ Hs32, float *__restrict__ part, uint32_t *status)
+                   float *__restrict__ Hs32, float *__restrict__ part, float h_gs,
+                   uint8_t *__restrict__ hq, uint8_t *__restrict__ hsf, uint8_t *__restrict__ hqs,
+                   uint8_t *__restrict__ hsfs, uint32_t *status)
 {
     extern __shared__ uint8_t dt_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>(
@@ -1280,6 +1302,7 @@ __global__ void __launch_bounds__(192, 1)
     uint8_t *const sa = base + cv.a, *const ssfa = base + cv.sfa;
     uint8_t *const sxb = base + cv.xb, *const sxsf = base + cv.xsf;
     float(*const sd)[kDtN + 1] = reinterpret_cast<float(*)[kDtN + 1]>(base + cv.d);
+    float(*const shb)[64] = reinterpret_cast<float(*)[64]>(base + cv.hb);
     __shared__ uint64_t full[kDtMaxStages], empty[kDtMaxStages], tfull[2], tempty[2];
     __shared__ uint32_t tmem_slot;
     __shared__ int abort_s;
@@ -1463,10 +1486,24 @@ __global__ void __launch_bounds__(192, 1)
                     const int a = tl.shared ? qa : P.list[a0 + qa];
                     const int tok = tl.shared ? qa : a / k;
                     const float h = silu_mul(sd[et][tok] * inv, sd[64 + et][tok] * inv);
+                    shb[qa][et] = h;
                     if (tl.shared)
                         Hs32[(size_t)qa * d_ff_s + 64 * tl.t + et] = h;
                     else
                         H32[(size_t)a * d_ff + 64 * tl.t + et] = h;
+                }
+            }
+            dt_epi_sync();
+            if (got && unit < 0 && hq) {
+                // h as the w2 kernel's NVFP4 operand: block et & 3 of assignment et >> 2
+                const DtTile tl = dt_tile(item, routed_items, tpr);
+                const int a0 = tl.shared ? 0 : P.ustart[tl.u];
+                const int na = tl.shared ? T : P.ustart[tl.u + 1] - a0;
+                if (et < 4 * na) {
+                    const int qa = et >> 2, bi = et & 3;
+                    const int row = tl.shared ? qa : P.list[a0 + qa];
+                    dt_quantize_h(&shb[qa][16 * bi], h_gs, row, tl.t, bi, tl.shared ? d_ff_s : d_ff,
+                                  tl.shared ? hqs : hq, tl.shared ? hsfs : hsf);
                 }
             }
             dt_epi_sync();
@@ -1487,9 +1524,12 @@ __global__ void __launch_bounds__(64)
                        int slot_major, int G, int d_ff_s, int has_shared, float x_gs,
                        const float *__restrict__ gs13, const float *__restrict__ gs13s,
                        const float *__restrict__ part, float *__restrict__ H32,
-                       float *__restrict__ Hs32, uint32_t *status)
+                       float *__restrict__ Hs32, float h_gs, uint8_t *__restrict__ hq,
+                       uint8_t *__restrict__ hsf, uint8_t *__restrict__ hqs,
+                       uint8_t *__restrict__ hsfs, uint32_t *status)
 {
     __shared__ DecPlanSmem P;
+    __shared__ float shb[kDtN][64];
     build_plan(P, idx, T, E, k, C, slot_major, status);   // idx is final: the w1/w3 kernel read it
     pdl_wait();      // the pieces come from the w1/w3 kernel
     pdl_trigger();
@@ -1528,11 +1568,354 @@ __global__ void __launch_bounds__(64)
                 }
         }
         const float h = silu_mul(g * inv, u * inv);
+        shb[qa][et] = h;
         if (tl.shared)
             Hs32[(size_t)qa * d_ff_s + 64 * tl.t + et] = h;
         else
             H32[(size_t)a * d_ff + 64 * tl.t + et] = h;
     }
+    if (!hq)
+        return;
+    __syncthreads();
+    if (et < 4 * na) {
+        const int qa = et >> 2, bi = et & 3;
+        const int row = tl.shared ? qa : P.list[a0 + qa];
+        dt_quantize_h(&shb[qa][16 * bi], h_gs, row, tl.t, bi, tl.shared ? d_ff_s : d_ff,
+                      tl.shared ? hqs : hq, tl.shared ? hsfs : hsf);
+    }
+}
+
+// ---------------------------------------------------------------- NVFP4 decode w2, tensor cores
+// NVFP4 decode w2 on the tensor cores: a chosen expert's W2 rows are the M
+// side (128 output rows per tile, K = d_ff) and the assignments' h rows the N
+// side (16 columns: routed h rows a = t k + j, quantized by the w1/w3 kernel;
+// the shared expert's tiles take the T shared h rows). Tiles: source u (the
+// chosen experts ascending, then the shared expert) x row tile rt. There are
+// few of them (64 at one token), so the launch is split evenly over its G
+// CTAs along the flattened (tile, K stage) sequence ("stream-K"): CTA c runs
+// stages [c F / G, (c + 1) F / G), one piece per tile it touches. A piece's
+// epilogue weights column a by w_a / (gs_h gs_w2[e]) and writes, for every
+// token, its rows' sums to `part` (zero where the token did not choose the
+// expert); k_dec_w2_nvtc_reduce adds, per output, the pieces of every source
+// in (source, CTA) order: deterministic.
+// Roles as k_dec_w13_nvtc; the ring carries the weight tile (16 KB), the h
+// tile (2 KB) and both operands' scale atoms (2 KB each) per K stage.
+namespace {
+
+struct D2Space {
+    int U, src, RT, nks, nks_s, routed_items, items;
+    long long Fr, F;   // routed stages, all stages
+};
+
+__host__ __device__ __forceinline__ D2Space d2_space(int U, int has_shared, int d, int d_ff, int d_ff_s)
+{
+    D2Space z;
+    z.U = U;
+    z.src = U + (has_shared ? 1 : 0);
+    z.RT = d / 128;
+    z.nks = d_ff / 256;
+    z.nks_s = has_shared ? d_ff_s / 256 : 0;
+    z.routed_items = U * z.RT;
+    z.items = z.src * z.RT;
+    z.Fr = (long long)z.routed_items * z.nks;
+    z.F = z.Fr + (long long)(has_shared ? z.RT : 0) * z.nks_s;
+    return z;
+}
+
+__host__ __device__ __forceinline__ long long d2_f0(const D2Space &z, int G, int c)
+{
+    return (long long)c * z.F / G;
+}
+
+__host__ __device__ __forceinline__ int d2_item_of(const D2Space &z, long long f)
+{
+    return f < z.Fr ? (int)(f / z.nks) : z.routed_items + (int)((f - z.Fr) / z.nks_s);
+}
+
+__host__ __device__ __forceinline__ long long d2_item_start(const D2Space &z, int i)
+{
+    return i <= z.routed_items ? (long long)i * z.nks : z.Fr + (long long)(i - z.routed_items) * z.nks_s;
+}
+
+// Piece lp of CTA c: its tile and K-stage range; false past the CTA's range.
+__host__ __device__ __forceinline__ bool d2_piece(const D2Space &z, int G, int c, int lp, int &item, int &kb0,
+                                         int &kb1)
+{
+    const long long a = d2_f0(z, G, c), b = d2_f0(z, G, c + 1);
+    if (a >= b)
+        return false;
+    item = d2_item_of(z, a) + lp;
+    const long long s0 = d2_item_start(z, item), s1 = d2_item_start(z, item + 1);
+    const long long lo = a > s0 ? a : s0, hi = b < s1 ? b : s1;
+    if (lo >= hi)
+        return false;
+    kb0 = (int)(lo - s0);
+    kb1 = (int)(hi - s0);
+    return true;
+}
+
+constexpr uint32_t kD2StageBytes = kDtABytes + kDtBBytes + 2 * kDtSfBytes;
+constexpr int kD2MaxCtas = 1024;   // CTAs of one k_dec_w2_nvtc launch
+
+} // namespace
+
+__global__ void __launch_bounds__(192, 1)
+    k_dec_w2_nvtc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmAs,
+                  const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmBs,
+                  const int32_t *__restrict__ idx, const float *__restrict__ topk_w, int T, int d,
+                  int d_ff, int E, int k, int C, int slot_major, int nst,
+                  const uint8_t *__restrict__ W2sf, const float *__restrict__ gs2, int d_ff_s,
+                  int has_shared, const uint8_t *__restrict__ W2s_sf, const float *__restrict__ gs2s,
+                  const uint8_t *__restrict__ hsf, const uint8_t *__restrict__ hsfs, float h_gs,
+                  float *__restrict__ part, int pmax, uint32_t *status)
+{
+    extern __shared__ uint8_t dt_raw[];
+    uint8_t *base = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(dt_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    // ring: a [nst][16 KB], b [nst][2 KB], sfa [nst][2 KB], sfb [nst][2 KB]
+    uint8_t *const sa = base, *const sb = base + nst * kDtABytes;
+    uint8_t *const ssfa = sb + nst * kDtBBytes, *const ssfb = ssfa + nst * kDtSfBytes;
+    __shared__ uint64_t full[kDtMaxStages], empty[kDtMaxStages], tfull[2], tempty[2];
+    __shared__ uint32_t tmem_slot;
+    __shared__ int abort_s;
+    __shared__ DecPlanSmem P;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < nst; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&tfull[b], 1);
+            mbar_init(&tempty[b], 4);
+        }
+        abort_s = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB);
+        if (has_shared) {
+            tma_prefetch_desc(&tmAs);
+            tma_prefetch_desc(&tmBs);
+        }
+    }
+    if (warp == 1) {
+        tmem_alloc(&tmem_slot, 256);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = tmem_slot;
+    build_plan(P, idx, T, E, k, C, slot_major, status);   // idx: final before the w1/w3 kernel ran
+    pdl_wait();      // h comes from the w1/w3 kernels
+    pdl_trigger();
+    volatile int *abort_flag = &abort_s;
+    const D2Space z = d2_space(P.U, has_shared, d, d_ff, d_ff_s);
+    const int G = gridDim.x, c = blockIdx.x;
+
+    if (warp == 0) {
+        if (lane == 0) {   // ---------------- producer
+            uint32_t it = 0;
+            bool ok = true;
+            int item, kb0, kb1;
+            for (int lp = 0; ok && lp < pmax && d2_piece(z, G, c, lp, item, kb0, kb1); ++lp) {
+                const bool shared = item >= z.routed_items;
+                const int rt = item % z.RT;
+                const long long row0 = shared ? (long long)rt * 128
+                                              : ((long long)P.uniq[item / z.RT] * d + rt * 128);
+                const int K = shared ? d_ff_s : d_ff;
+                const uint8_t *sfa = (shared ? W2s_sf : W2sf) + (size_t)(row0 / 128) * (K / 64) * 512;
+                const uint8_t *sfb = shared ? hsfs : hsf;
+                for (int kb = kb0; kb < kb1; ++kb, ++it) {
+                    const int s = it % nst;
+                    const uint32_t ph = (it / nst) & 1u;
+                    if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag, status)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&full[s], kD2StageBytes);
+                    tma_load_2d(sa + s * kDtABytes, shared ? &tmAs : &tmA, kb * 128, (int)row0, &full[s]);
+                    tma_load_2d(sb + s * kDtBBytes, shared ? &tmBs : &tmB, kb * 128, 0, &full[s]);
+                    dt_bulk_load(ssfa + s * kDtSfBytes, sfa + (size_t)kb * kDtSfBytes, kDtSfBytes, &full[s]);
+                    dt_bulk_load(ssfb + s * kDtSfBytes, sfb + (size_t)kb * kDtSfBytes, kDtSfBytes, &full[s]);
+                }
+            }
+            if (!ok) {
+                // let the copies already issued land before the CTA can exit
+                int never = 0;
+                const uint32_t first = it >= (uint32_t)nst ? it - nst : 0;
+                for (uint32_t i = first; i < it; ++i)
+                    mbar_wait(&full[i % nst], (i / nst) & 1u, &never, status);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {   // ---------------- MMA issuer
+            uint32_t it = 0;
+            int item, kb0, kb1;
+            for (int lp = 0; lp < pmax && d2_piece(z, G, c, lp, item, kb0, kb1); ++lp) {
+                const uint32_t b = lp & 1, aph = (lp >> 1) & 1u;
+                if (!mbar_wait(&tempty[b], aph ^ 1u, abort_flag, status))
+                    break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + b * kDtN;
+                bool ok = true;
+                for (int kb = kb0; kb < kb1; ++kb, ++it) {
+                    const int s = it % nst;
+                    const uint32_t ph = (it / nst) & 1u;
+                    if (!mbar_wait(&full[s], ph, abort_flag, status)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t sf_a = tmem_base + 2 * kDtN + s * kDtSfCols;
+                    const uint32_t sf_b = sf_a + 16;
+                    const uint32_t a_sf = smem_u32(ssfa + s * kDtSfBytes);
+                    const uint32_t b_sf = smem_u32(ssfb + s * kDtSfBytes);
+#pragma unroll
+                    for (int g = 0; g < 4; ++g) {
+                        dt_cp_atom(sf_a + 4 * g, dt_desc_atom(a_sf + 512 * g));
+                        dt_cp_atom(sf_b + 4 * g, dt_desc_atom(b_sf + 512 * g));
+                    }
+                    const uint32_t a0 = smem_u32(sa + s * kDtABytes), b0 = smem_u32(sb + s * kDtBBytes);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        dt_mma(d_tmem, smem_desc_k128(a0 + kk * 32), smem_desc_k128(b0 + kk * 32),
+                               sf_a + 4 * kk, sf_b + 4 * kk, (kb != kb0 || kk != 0) ? 1u : 0u);
+                    tc_commit(&empty[s]);
+                }
+                if (!ok)
+                    break;
+                tc_commit(&tfull[b]);
+            }
+        }
+    } else {   // ---------------- epilogue warps 2..5: one output row per thread
+        const int q = warp & 3;
+        const int row = q * 32 + lane;
+        int item, kb0, kb1;
+        for (int lp = 0; lp < pmax && d2_piece(z, G, c, lp, item, kb0, kb1); ++lp) {
+            const uint32_t b = lp & 1, aph = (lp >> 1) & 1u;
+            const bool got = mbar_wait(&tfull[b], aph, abort_flag, status);
+            tc_fence_after();
+            float v[16];
+            if (got) {
+                dt_tmem_ld16(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + b * kDtN, v);
+                tmem_ld_wait();
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(&tempty[b]);
+            if (!got)
+                continue;
+            const bool shared = item >= z.routed_items;
+            const int u = shared ? 0 : item / z.RT;
+            const float inv = 1.0f / (h_gs * (shared ? gs2s[0] : gs2[P.uniq[u]]));
+            float *dst = part + (size_t)(c * pmax + lp) * T * 128 + row;
+            for (int tok = 0; tok < T; ++tok) {
+                float val = 0.f;
+                if (shared) {
+#pragma unroll
+                    for (int j = 0; j < kDtN; ++j)
+                        val = (j == tok) ? v[j] * inv : val;
+                } else {
+                    for (int qa = P.ustart[u]; qa < P.ustart[u + 1]; ++qa) {
+                        const int a = P.list[qa];
+                        if (a / k != tok)
+                            continue;
+                        float pick = 0.f;
+#pragma unroll
+                        for (int j = 0; j < kDtN; ++j)
+                            pick = (j == a) ? v[j] : pick;
+                        val = topk_w[a] * inv * pick;
+                    }
+                }
+                dst[(size_t)tok * 128] = val;
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, 256);
+    }
+}
+
+// out[t, r] = the sum, over the sources in order (chosen experts ascending,
+// then the shared expert) and over the CTAs that ran pieces of the source's
+// row tile (ascending), of the pieces' sums. One block per (row tile, token),
+// 128 threads (one output row each); G and pmax as for k_dec_w2_nvtc. One
+// thread lists the pieces' slots, up to 512 at a time, and every thread adds
+// its row of them in list order, eight loads in flight.
+__global__ void __launch_bounds__(128)
+    k_dec_w2_nvtc_reduce(const int32_t *__restrict__ idx, int T, int d, int d_ff, int E, int k, int C,
+                         int slot_major, int G, int pmax, int d_ff_s, int has_shared,
+                         const float *__restrict__ part, float *__restrict__ out, uint32_t *status)
+{
+    constexpr int kList = 512;
+    __shared__ DecPlanSmem P;
+    __shared__ int terms[kList];   // piece slots (units of T x 128 floats), in summation order
+    __shared__ long long f0s[kD2MaxCtas + 1];   // the CTAs' first stages
+    __shared__ int nterms, g_src, g_cc, g_done;
+    build_plan(P, idx, T, E, k, C, slot_major, status);
+    const D2Space z = d2_space(P.U, has_shared, d, d_ff, d_ff_s);
+    for (int cc = threadIdx.x; cc <= G; cc += blockDim.x)
+        f0s[cc] = d2_f0(z, G, cc);
+    pdl_wait();      // the pieces come from the w2 kernel
+    pdl_trigger();
+    const int rt = blockIdx.x, tok = blockIdx.y, r = threadIdx.x;
+    if (r == 0) {
+        g_src = 0;
+        g_cc = -1;
+    }
+    const float *pp = part + (size_t)tok * 128 + r;
+    const size_t stride = (size_t)T * 128;
+    float acc = 0.f;
+    for (;;) {
+        __syncthreads();   // the previous list is consumed
+        if (r == 0) {
+            int n = 0, src = g_src, cc = g_cc;
+            while (n < kList && src < z.src) {
+                const int item = src * z.RT + rt;
+                const long long s0 = d2_item_start(z, item), s1 = d2_item_start(z, item + 1);
+                if (cc < 0) {   // the last CTA whose range starts at or before s0
+                    cc = (int)(((s0 + 1) * G + z.F - 1) / z.F) - 1;
+                    cc = cc < 0 ? 0 : cc;
+                }
+                const long long a = cc < G ? f0s[cc] : s1;
+                if (a >= s1) {
+                    ++src;
+                    cc = -1;
+                    continue;
+                }
+                const long long b = f0s[cc + 1];
+                if (b > s0 && b > a)   // a non-empty range that meets the tile
+                    terms[n++] = cc * pmax + (item - d2_item_of(z, a));
+                ++cc;
+            }
+            nterms = n;
+            g_src = src;
+            g_cc = cc;
+            g_done = src >= z.src;
+        }
+        __syncthreads();
+        const int n = nterms;
+        for (int i0 = 0; i0 < n; i0 += 8) {
+            float v[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                v[i] = i0 + i < n ? __ldcg(pp + (size_t)terms[i0 + i] * stride) : 0.f;
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                if (i0 + i < n)
+                    acc += v[i];
+        }
+        if (g_done)
+            break;
+    }
+    out[(size_t)tok * d + rt * 128 + r] = acc;
 }
 
 // ---------------------------------------------------------------- host side
@@ -1847,6 +2230,7 @@ int launch_dec_w13_nvtc(const moe_shape_t &s, const uint16_t *x, float x_gs,
                         const int32_t *topk_idx, const uint8_t *W13q, const uint8_t *W13sf,
                         const float *gs13, const uint8_t *W13s_q, const uint8_t *W13s_sf,
                         const float *gs13s, float *H32, float *part, size_t part_floats,
+                        float h_gs, uint8_t *hq, uint8_t *hsf, uint8_t *hqs, uint8_t *hsfs,
                         uint32_t *status, cudaStream_t st)
 {
     if (s.T == 0)
@@ -1885,14 +2269,76 @@ int launch_dec_w13_nvtc(const moe_shape_t &s, const uint16_t *x, float x_gs,
     rc = launch_pdl_smem(k_dec_w13_nvtc, blocks, 192, dt_carve(nst, nks).total + 1024, st, tmA, tmAs,
                          x, x_gs, topk_idx, s.T, s.d, s.d_ff, s.E, s.k, s.capacity, slot_major(s), nst,
                          W13sf, gs13, s.d_ff_shared, shared ? 1 : 0, W13s_sf, gs13s, H32, Hs, part,
-                         status);
+                         h_gs, hq, hsf, hqs, hsfs, status);
     if (rc)
         return rc;
     if ((rc = launched()))
         return rc;
     launch_pdl(k_dec_w13_nvtc_fix, blocks, 64, st, topk_idx, s.T, s.d, s.d_ff, s.E, s.k, s.capacity,
                slot_major(s), blocks, s.d_ff_shared, shared ? 1 : 0, x_gs, gs13, gs13s,
-               (const float *)part, H32, Hs, status);
+               (const float *)part, H32, Hs, h_gs, hq, hsf, hqs, hsfs, status);
+    return launched();
+}
+
+int launch_dec_w2_nvtc(const moe_shape_t &s, const int32_t *topk_idx, const float *topk_w,
+                       const uint8_t *W2q, const uint8_t *W2sf, const float *gs2,
+                       const uint8_t *W2s_q, const uint8_t *W2s_sf, const float *gs2s,
+                       const uint8_t *hq, const uint8_t *hsf, const uint8_t *hqs, const uint8_t *hsfs,
+                       float h_gs, float *part, size_t part_floats, float *out, uint32_t *status,
+                       cudaStream_t st)
+{
+    if (s.T == 0)
+        return MOE_OK;
+    const bool shared = s.d_ff_shared > 0 && W2s_q;
+    // h rows are the N side: every routed row (and the T shared rows) in 16 columns
+    if (s.T * s.k > kDtN || s.d % 128 != 0 || s.d_ff % 256 != 0 ||
+        (shared && s.d_ff_shared % 256 != 0))
+        return MOE_ERR_UNSUPPORTED;
+    const int RT = s.d / 128, nks = s.d_ff / 256, nks_s = shared ? s.d_ff_shared / 256 : nks;
+    const long long Fmax = (long long)std::min(s.E, s.T * s.k) * RT * nks +
+                           (shared ? (long long)RT * nks_s : 0);
+    const int G = (int)std::max<long long>(1, std::min<long long>(Fmax, num_sms()));
+    if (G > kD2MaxCtas)
+        return MOE_ERR_UNSUPPORTED;
+    // pieces per CTA: a range of at most ceil(F / G) stages meets at most
+    // ceil(that / the shortest tile) + 1 tiles
+    const long long per = (Fmax + G - 1) / G;
+    const int pmax = (int)((per + std::min(nks, nks_s) - 1) / std::min(nks, nks_s)) + 1;
+    if ((size_t)G * pmax * s.T * 128 > part_floats)
+        return MOE_ERR_UNSUPPORTED;
+    int dyn_max = 0;
+    if (const int rc = smem_limit(reinterpret_cast<const void *>(k_dec_w2_nvtc), dyn_max))
+        return rc;
+    int nst = kDtMaxRing;
+    while (nst >= 2 && (int)(nst * kD2StageBytes) + 1024 > dyn_max)
+        --nst;
+    if (nst < 2)
+        return MOE_ERR_UNSUPPORTED;
+    CUtensorMap tmA, tmAs, tmB, tmBs;
+    int rc = make_tmap_u8_sw128(&tmA, W2q, s.d_ff / 2, (long long)s.E * s.d, 128);
+    if (!rc)
+        rc = make_tmap_u8_sw128(&tmB, hq, s.d_ff / 2, (long long)s.T * s.k, kDtN);
+    if (!rc && shared) {
+        rc = make_tmap_u8_sw128(&tmAs, W2s_q, s.d_ff_shared / 2, s.d, 128);
+        if (!rc)
+            rc = make_tmap_u8_sw128(&tmBs, hqs, s.d_ff_shared / 2, s.T, kDtN);
+    } else {
+        tmAs = tmA;
+        tmBs = tmB;
+    }
+    if (rc)
+        return rc;
+    rc = launch_pdl_smem(k_dec_w2_nvtc, G, 192, (size_t)nst * kD2StageBytes + 1024, st, tmA, tmAs, tmB,
+                         tmBs, topk_idx, topk_w, s.T, s.d, s.d_ff, s.E, s.k, s.capacity, slot_major(s),
+                         nst, W2sf, gs2, s.d_ff_shared, shared ? 1 : 0, W2s_sf, gs2s, hsf, hsfs, h_gs,
+                         part, pmax, status);
+    if (rc)
+        return rc;
+    if ((rc = launched()))
+        return rc;
+    launch_pdl_ex(k_dec_w2_nvtc_reduce, dim3(RT, s.T), dim3(128), 0, st, topk_idx, s.T, s.d, s.d_ff,
+                  s.E, s.k, s.capacity, slot_major(s), G, pmax, s.d_ff_shared, shared ? 1 : 0,
+                  (const float *)part, out, status);
     return launched();
 }
 

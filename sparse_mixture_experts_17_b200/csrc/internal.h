@@ -76,6 +76,7 @@ struct WsLayout {
     size_t dec_xdq, dec_H32;                             // MXFP8 / NVFP4 decode
     size_t dec_xs, dec_hs;                               // NVFP4 decode: scale values
     size_t dec_part;                                     // NVFP4 decode: split-K sums
+    size_t dec_hq, dec_hsf, dec_hqs, dec_hsfs;           // NVFP4 decode: h as the w2 operand
     size_t tile_start;                                   // first m-tile of each expert
     size_t dbg_seen;                                     // dispatch checks: count per row
     // backward pass
@@ -242,13 +243,28 @@ int make_tmap_u8_sw128(CUtensorMap *m, const void *base, long long cols, long lo
 // [T, d]) with x_gs inside the kernel and writes H32 like launch_dec_w13_nv;
 // tiles left over after the whole rounds are split along K, their pieces'
 // sums go to `part` (part_floats floats, at least 2 x CTAs x T x 128) and a
-// second kernel adds them. Returns MOE_ERR_UNSUPPORTED (nothing launched)
-// for shapes it does not take.
+// second kernel adds them. With hq != NULL it also writes h as the NVFP4
+// operand of launch_dec_w2_nvtc (h_gs; routed rows a = t k + j into hq/hsf,
+// the shared expert's rows into hqs/hsfs). Returns MOE_ERR_UNSUPPORTED
+// (nothing launched) for shapes it does not take.
 int launch_dec_w13_nvtc(const moe_shape_t &s, const uint16_t *x, float x_gs,
                         const int32_t *topk_idx, const uint8_t *W13q, const uint8_t *W13sf,
                         const float *gs13, const uint8_t *W13s_q, const uint8_t *W13s_sf,
                         const float *gs13s, float *H32, float *part, size_t part_floats,
+                        float h_gs, uint8_t *hq, uint8_t *hsf, uint8_t *hqs, uint8_t *hsfs,
                         uint32_t *status, cudaStream_t st);
+// NVFP4 decode w2 on the tensor cores (T k <= 16): h as the NVFP4 operand the
+// w1/w3 kernel wrote (hq [T k, d_ff / 2] with atom-layout scales hsf; the
+// shared expert's hqs [T, d_ff_shared / 2], hsfs), split evenly over the
+// CTAs along (tile, K stage); its pieces' sums go to `part` and a second
+// kernel adds them into out [T, d] in a fixed order. MOE_ERR_UNSUPPORTED
+// (nothing launched) for shapes it does not take.
+int launch_dec_w2_nvtc(const moe_shape_t &s, const int32_t *topk_idx, const float *topk_w,
+                       const uint8_t *W2q, const uint8_t *W2sf, const float *gs2,
+                       const uint8_t *W2s_q, const uint8_t *W2s_sf, const float *gs2s,
+                       const uint8_t *hq, const uint8_t *hsf, const uint8_t *hqs, const uint8_t *hsfs,
+                       float h_gs, float *part, size_t part_floats, float *out, uint32_t *status,
+                       cudaStream_t st);
 int launch_gemm_simt(const GemmArgs &g, cudaStream_t st);
 int num_sms();
 

@@ -157,6 +157,14 @@ WsLayout ws_layout(const moe_shape_t &s)
     L.dec_xs = take(nv ? Td * (s.d / 16) * 4 : 0);
     L.dec_hs = take(nv ? (Td * k * s.d_ff + Td * dfs) / 16 * 4 : 0);
     L.dec_part = take(nv ? dec_part_floats(s) * 4 : 0);
+    {
+        // h of at most two tokens as the NVFP4 w2 operand (codes, atom-layout scales)
+        const size_t Th = std::min<size_t>(T, 2);
+        L.dec_hq = take(nv ? Th * k * s.d_ff / 2 : 0);
+        L.dec_hsf = take(nv ? (size_t)nv_sf_bytes((long long)(Th * k), (int)s.d_ff) : 0);
+        L.dec_hqs = take(nv && dfs ? Th * dfs / 2 : 0);
+        L.dec_hsfs = take(nv && dfs ? (size_t)nv_sf_bytes((long long)Th, (int)dfs) : 0);
+    }
     // activation scales: routed operands keyed by m-tile (at most max_mt
     // tiles of 128 rows), shared-expert operands by row / 128; MXFP8 in the
     // atom layout, NVFP4 (16-element blocks) in the activation layout of
@@ -786,13 +794,20 @@ static int forward_mx_impl(const moe_shape_t &s, const WsLayout &L, void *ws, co
         uint16_t *hh = at<uint16_t>(ws, L.dec_H);
         float *hs = at<float>(ws, L.dec_hs);
         const long long nh = (long long)s.T * s.k * s.d_ff + (long long)s.T * s.d_ff_shared;
+        // h as the tensor-core w2 kernel's NVFP4 operand, written by the w1/w3 kernel
+        float *part = at<float>(ws, L.dec_part);
+        uint8_t *hq = at<uint8_t>(ws, L.dec_hq), *hsf = at<uint8_t>(ws, L.dec_hsf);
+        uint8_t *hqs = s.d_ff_shared ? at<uint8_t>(ws, L.dec_hqs) : nullptr;
+        uint8_t *hsfs = s.d_ff_shared ? at<uint8_t>(ws, L.dec_hsfs) : nullptr;
+        bool hq_written = false;
         {
             StageMark m(MOE_STAGE_DEC_W13, st);
             // w1/w3 on the tensor cores; shapes that kernel does not take go
             // through the CUDA-core kernel on f16 code values
             rc = launch_dec_w13_nvtc(s, x, lw.x_gs, idx, W13q, W13sf, lw.W13gs, W13s_q, W13s_sf,
-                                     lw.W13s_gs, H32, at<float>(ws, L.dec_part), dec_part_floats(s),
-                                     status, st);
+                                     lw.W13s_gs, H32, part, dec_part_floats(s), lw.h_gs, hq, hsf,
+                                     hqs, hsfs, status, st);
+            hq_written = rc == MOE_OK;
             if (rc == MOE_ERR_UNSUPPORTED) {
                 rc = launch_nv_qrows_f16_bf16(x, (long long)s.T * s.d, lw.x_gs, xh, xs, st);
                 if (!rc)
@@ -803,10 +818,17 @@ static int forward_mx_impl(const moe_shape_t &s, const WsLayout &L, void *ws, co
         if (rc)
             return rc;
         StageMark m(MOE_STAGE_DEC_W2, st);
-        rc = launch_nv_qrows_f16_f32(H32, nh, lw.h_gs, hh, hs, st);
-        if (!rc)
-            rc = launch_dec_w2_nv(s, idx, w, W2q, W2sf, lw.W2gs, W2s_q, W2s_sf, lw.W2s_gs, hh, hs,
-                                  lw.h_gs, out, status, st);
+        // w2 on the tensor cores; otherwise on the CUDA cores from f16 code values
+        rc = hq_written ? launch_dec_w2_nvtc(s, idx, w, W2q, W2sf, lw.W2gs, W2s_q, W2s_sf, lw.W2s_gs,
+                                             hq, hsf, hqs, hsfs, lw.h_gs, part, dec_part_floats(s),
+                                             out, status, st)
+                        : MOE_ERR_UNSUPPORTED;
+        if (rc == MOE_ERR_UNSUPPORTED) {
+            rc = launch_nv_qrows_f16_f32(H32, nh, lw.h_gs, hh, hs, st);
+            if (!rc)
+                rc = launch_dec_w2_nv(s, idx, w, W2q, W2sf, lw.W2gs, W2s_q, W2s_sf, lw.W2s_gs, hh,
+                                      hs, lw.h_gs, out, status, st);
+        }
         return rc;
     }
     if (decode) {
