@@ -468,7 +468,7 @@ def run_ours(a, world, rank, local):
         k13 = stages["dec_w13"][0] / stages["dec_w13"][1]
         ach = w13_bytes / (k13 / 1e3) / 1e9
         dec_kernel = ("k_dec_w13_mx" if a.mxfp8 else
-                      "k_nv_quantize_rows + k_dec_w13_nvtc (x to NVFP4, then tensor-core tiles)"
+                      "k_dec_w13_nvtc + k_dec_w13_nvtc_fix (x to NVFP4 in-kernel, tensor-core tiles)"
                       if a.nvfp4 else "k_dec_w13")
         roofline = {"bound": "hbm", "kernel": f"{dec_kernel} (chosen experts' w1/w3 rows + SwiGLU)",
                     "achieved": round(ach, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
