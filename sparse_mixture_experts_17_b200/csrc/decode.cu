@@ -177,7 +177,7 @@ __global__ void __launch_bounds__(256) k_dec_router(const uint16_t *__restrict__
 
 // Router and top-k in one CTA of 512 threads, for W_g up to kFusedRouteBytes.
 // Work item = (expert e, slice of d): with E < 16 each expert's row is split
-// into 16/E slices so all 16 warps stream W_g; each lane keeps four 16-byte
+// into 16/E slices so all 16 warps stream W_g; each lane keeps eight 16-byte
 // loads in flight. Partial dot products meet in shared memory, then warp t
 // selects token t's experts.
 constexpr size_t kFusedRouteBytes = 256 * 1024;
@@ -208,23 +208,47 @@ __global__ void __launch_bounds__(512) k_dec_route(const uint16_t *__restrict__ 
         for (int t = 0; t < MAXT; ++t)
             acc[t] = 0.f;
         const uint4 *wr = reinterpret_cast<const uint4 *>(Wg + (size_t)e * d);
-        for (int cb = c0; cb < c1; cb += 128) {
-            uint4 wv[4];
+        // eight 16-byte loads of W_g per lane in flight (a 2048-element slice
+        // in one round trip), and for T <= 2 the matching x loads with them
+        for (int cb = c0; cb < c1; cb += 256) {
+            uint4 wv[8];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
+            for (int i = 0; i < 8; ++i) {
                 const int c = cb + lane + 32 * i;
                 if (c < c1)
                     wv[i] = ld_stream_v4(wr + c);
             }
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int c = cb + lane + 32 * i;
-                if (c >= c1)
-                    continue;
+            if (MAXT <= 2) {
+                uint4 xv[MAXT][8];
 #pragma unroll
                 for (int t = 0; t < MAXT; ++t)
-                    if (t < T)
-                        acc[t] = dot8(wv[i], __ldg(reinterpret_cast<const uint4 *>(x + (size_t)t * d) + c), acc[t]);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const int c = cb + lane + 32 * i;
+                        if (t < T && c < c1)
+                            xv[t][i] = __ldg(reinterpret_cast<const uint4 *>(x + (size_t)t * d) + c);
+                    }
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int c = cb + lane + 32 * i;
+                    if (c >= c1)
+                        continue;
+#pragma unroll
+                    for (int t = 0; t < MAXT; ++t)
+                        if (t < T)
+                            acc[t] = dot8(wv[i], xv[t][i], acc[t]);
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int c = cb + lane + 32 * i;
+                    if (c >= c1)
+                        continue;
+#pragma unroll
+                    for (int t = 0; t < MAXT; ++t)
+                        if (t < T)
+                            acc[t] = dot8(wv[i], __ldg(reinterpret_cast<const uint4 *>(x + (size_t)t * d) + c), acc[t]);
+                }
             }
         }
 #pragma unroll
