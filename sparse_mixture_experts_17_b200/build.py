@@ -24,7 +24,7 @@ BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libmoe.so")
 SOURCES = ["dispatch.cu", "gemm_simt.cu", "gemm_tc.cu", "gemm_mx.cu", "mx_quant.cu", "nv_quant.cu", "decode.cu",
            "expert_choice.cu", "backward.cu", "moe_api.cu", "permute_static.cu"]
-HEADERS = ["common.cuh", "internal.h", "topk.cuh", "mxfp8.cuh", "nvfp4.cuh", "tiles.cuh"]
+HEADERS = ["common.cuh", "internal.h", "topk.cuh", "mxfp8.cuh", "nvfp4.cuh", "tiles.cuh", "decode_split.cuh"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC",

@@ -33,6 +33,7 @@
 #include "internal.h"
 #include "mxfp8.cuh"
 #include "nvfp4.cuh"
+#include "decode_split.cuh"
 #include "topk.cuh"
 
 namespace moe {
@@ -1166,47 +1167,6 @@ __host__ __device__ __forceinline__ DtCarve dt_carve(int nst, int nks)
     return c;
 }
 
-// The work of one launch over G CTAs: `full` rounds of whole tiles (CTA c
-// takes tiles c + r G), then the R = items - full G tiles left over, each cut
-// into np pieces of ps K stages (the last piece may be shorter). Unit u =
-// piece u % np of leftover tile u / np goes to CTA u mod G.
-struct DtSplit {
-    int full, R, ps, np, units;
-};
-
-__host__ __device__ __forceinline__ DtSplit dt_split(int items, int G, int nks)
-{
-    DtSplit s;
-    s.full = items / G;
-    s.R = items - s.full * G;
-    s.ps = s.R ? (s.R * nks + G - 1) / G : nks;
-    s.np = (nks + s.ps - 1) / s.ps;
-    s.units = s.R * s.np;
-    return s;
-}
-
-// Work w of CTA c: the tile, its K-stage range, and the unit (-1: whole tile).
-__device__ __forceinline__ void dt_work(const DtSplit &sp, int G, int c, int w, int nks, int &item,
-                                        int &kb0, int &kb1, int &unit)
-{
-    if (w < sp.full) {
-        item = c + w * G;
-        kb0 = 0;
-        kb1 = nks;
-        unit = -1;
-    } else {
-        unit = c + (w - sp.full) * G;
-        item = sp.full * G + unit / sp.np;
-        kb0 = (unit % sp.np) * sp.ps;
-        kb1 = min(nks, kb0 + sp.ps);
-    }
-}
-
-__device__ __forceinline__ int dt_num_works(const DtSplit &sp, int G, int c)
-{
-    return sp.full + (c < sp.units ? (sp.units - 1 - c) / G + 1 : 0);
-}
-
 __device__ __forceinline__ uint64_t dt_desc_atom(uint32_t smem_addr)
 {
     uint64_t d = 0;   // one 32-row x 16-byte scale atom: no swizzle, 8-row core matrices
@@ -1626,58 +1586,6 @@ __global__ void __launch_bounds__(64)
 // tile (2 KB) and both operands' scale atoms (2 KB each) per K stage.
 namespace {
 
-struct D2Space {
-    int U, src, RT, nks, nks_s, routed_items, items;
-    long long Fr, F;   // routed stages, all stages
-};
-
-__host__ __device__ __forceinline__ D2Space d2_space(int U, int has_shared, int d, int d_ff, int d_ff_s)
-{
-    D2Space z;
-    z.U = U;
-    z.src = U + (has_shared ? 1 : 0);
-    z.RT = d / 128;
-    z.nks = d_ff / 256;
-    z.nks_s = has_shared ? d_ff_s / 256 : 0;
-    z.routed_items = U * z.RT;
-    z.items = z.src * z.RT;
-    z.Fr = (long long)z.routed_items * z.nks;
-    z.F = z.Fr + (long long)(has_shared ? z.RT : 0) * z.nks_s;
-    return z;
-}
-
-__host__ __device__ __forceinline__ long long d2_f0(const D2Space &z, int G, int c)
-{
-    return (long long)c * z.F / G;
-}
-
-__host__ __device__ __forceinline__ int d2_item_of(const D2Space &z, long long f)
-{
-    return f < z.Fr ? (int)(f / z.nks) : z.routed_items + (int)((f - z.Fr) / z.nks_s);
-}
-
-__host__ __device__ __forceinline__ long long d2_item_start(const D2Space &z, int i)
-{
-    return i <= z.routed_items ? (long long)i * z.nks : z.Fr + (long long)(i - z.routed_items) * z.nks_s;
-}
-
-// Piece lp of CTA c: its tile and K-stage range; false past the CTA's range.
-__host__ __device__ __forceinline__ bool d2_piece(const D2Space &z, int G, int c, int lp, int &item, int &kb0,
-                                         int &kb1)
-{
-    const long long a = d2_f0(z, G, c), b = d2_f0(z, G, c + 1);
-    if (a >= b)
-        return false;
-    item = d2_item_of(z, a) + lp;
-    const long long s0 = d2_item_start(z, item), s1 = d2_item_start(z, item + 1);
-    const long long lo = a > s0 ? a : s0, hi = b < s1 ? b : s1;
-    if (lo >= hi)
-        return false;
-    kb0 = (int)(lo - s0);
-    kb1 = (int)(hi - s0);
-    return true;
-}
-
 constexpr uint32_t kD2StageBytes = kDtABytes + kDtBBytes + 2 * kDtSfBytes;
 constexpr int kD2MaxCtas = 1024;   // CTAs of one k_dec_w2_nvtc launch
 
@@ -1904,10 +1812,8 @@ __global__ void __launch_bounds__(128)
             while (n < kList && src < z.src) {
                 const int item = src * z.RT + rt;
                 const long long s0 = d2_item_start(z, item), s1 = d2_item_start(z, item + 1);
-                if (cc < 0) {   // the last CTA whose range starts at or before s0
-                    cc = (int)(((s0 + 1) * G + z.F - 1) / z.F) - 1;
-                    cc = cc < 0 ? 0 : cc;
-                }
+                if (cc < 0)
+                    cc = d2_first_cta(z, G, s0);
                 const long long a = cc < G ? f0s[cc] : s1;
                 if (a >= s1) {
                     ++src;
@@ -2326,8 +2232,7 @@ int launch_dec_w2_nvtc(const moe_shape_t &s, const int32_t *topk_idx, const floa
         return MOE_ERR_UNSUPPORTED;
     // pieces per CTA: a range of at most ceil(F / G) stages meets at most
     // ceil(that / the shortest tile) + 1 tiles
-    const long long per = (Fmax + G - 1) / G;
-    const int pmax = (int)((per + std::min(nks, nks_s) - 1) / std::min(nks, nks_s)) + 1;
+    const int pmax = d2_pmax(Fmax, G, std::min(nks, nks_s));
     if ((size_t)G * pmax * s.T * 128 > part_floats)
         return MOE_ERR_UNSUPPORTED;
     int dyn_max = 0;
