@@ -20,6 +20,7 @@ import hashlib
 import json
 import math
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -167,24 +168,42 @@ def decode_bytes(w, T, idx):
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of
 # the headline kernel, from one ncu capture of the full-size launch; the
 # summary, with the command that made it, is under profiles/. `sources_sha`
-# is the SHA-256 of TRAFFIC_SOURCES when the counters were taken: once any of
-# them changes the figure no longer describes the kernel, and the line
-# reports null instead.
+# is the SHA-256 of what decides that launch when the counters were taken:
+# the kernel's sources (TRAFFIC_SOURCES) and the host functions that pick its
+# engine and build its tile lists (TRAFFIC_FUNCS). Once any of them changes
+# the figure no longer describes the launch, and the line reports null.
 TRAFFIC_SOURCES = ["sparse_mixture_experts_17_b200/csrc/gemm_tc.cu",
                    "sparse_mixture_experts_17_b200/csrc/common.cuh",
-                   "sparse_mixture_experts_17_b200/csrc/tiles.cuh",
-                   "sparse_mixture_experts_17_b200/csrc/moe_api.cu"]
+                   "sparse_mixture_experts_17_b200/csrc/tiles.cuh"]
+TRAFFIC_FUNCS = [("sparse_mixture_experts_17_b200/csrc/moe_api.cu", ["use_pair", "set_tiles"])]
 TRAFFIC = {
-    "prefill": {"bytes": 3373873920 + 931441664, "sources_sha": "71c2980b0c41d4c6",
+    "prefill": {"bytes": 3373873920 + 931441664, "sources_sha": "e4adf1cb5b4a22bc",
+                "kernel": "k_gemm_tc2<EPI_SWIGLU>",
                 "profile": "profiles/gemm_w13_traffic_mixtral_t16384.md"},
 }
 
 
-def sources_sha() -> str:
+def function_text(src: str, name: str) -> str:
+    """The text of top-level function `name` in C++ source `src`: from its
+    definition line (starting in column 0) to the first closing brace in
+    column 0."""
+    m = re.search(r"^[A-Za-z].*\b" + re.escape(name) + r"\(.*$", src, re.M)
+    if not m:
+        raise KeyError(name)
+    end = src.index("\n}\n", m.start())
+    return src[m.start():end + 3]
+
+
+def sources_sha(root: str = ROOT) -> str:
     h = hashlib.sha256()
     for f in TRAFFIC_SOURCES:
-        with open(os.path.join(ROOT, f), "rb") as fh:
+        with open(os.path.join(root, f), "rb") as fh:
             h.update(fh.read())
+    for f, names in TRAFFIC_FUNCS:
+        with open(os.path.join(root, f)) as fh:
+            src = fh.read()
+        for n in names:
+            h.update(function_text(src, n).encode())
     return h.hexdigest()[:16]
 
 
@@ -199,7 +218,7 @@ def w13_kernel_name(w):
 
 def headline_traffic(w):
     t = TRAFFIC.get(w.name)
-    if not t or t["sources_sha"] != sources_sha():
+    if not t or t["sources_sha"] != sources_sha() or not w13_kernel_name(w).startswith(t["kernel"]):
         return None
     return t["bytes"]
 
