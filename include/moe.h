@@ -390,8 +390,11 @@ MOE_API int moe_quantize_experts_nvfp4(const moe_shape_t *shape, const moe_bf16_
  * granite-4.0-h single-token MoE through the fused kernel": a 4-bit
  * single-token path fed by the top-k indices and weights): x and h are
  * quantized as the tensor-core chain quantizes them, and each chosen expert's
- * codes and scales are streamed once through CUDA cores, every 16-element
- * block dot product exact in f16. Larger T runs the block-scaled tensor-core
+ * codes and scales are streamed once into block-scaled tensor-core MMAs whose
+ * N side is the tokens (d a multiple of 256, T k <= 16 for w2; other shapes
+ * stream them through CUDA cores, every 16-element block dot product exact
+ * in f16). The output is the same bit for bit on every call with the same
+ * inputs and launch shape (fixed-order sums). Larger T runs the block-scaled tensor-core
  * GEMMs, which also read each chosen expert's codes and scales once (4.5
  * bits a weight). MOE_FLAG_FORCE_DECODE takes the decode kernels for T <= 2
  * and is MOE_ERR_UNSUPPORTED above; MOE_FLAG_FORCE_PREFILL takes the chain.
